@@ -1,0 +1,18 @@
+"""fp64 CPU oracle for the DyRA approximated linear layer.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product (the CUDA library and its
+Python binding) imports, calls or links anything here. Only tests/, the
+smoke check in __graft_entry__.py and the CPU-baseline leg of bench.py use it.
+"""
+
+from .dyra_oracle import (  # noqa: F401
+    Factors,
+    dense,
+    error_report,
+    inference,
+    offline_prepare,
+    offline_prepare_from_svd,
+    rel_fro,
+    round_to,
+    weight_only,
+)
