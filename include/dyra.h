@@ -1,0 +1,149 @@
+/*
+ * dyra.h - C ABI of the DyRA approximated linear layer on NVIDIA B200 (sm_100a).
+ *
+ * Method: "DyRA: Dynamic Residual Approximation for Efficient Matrix
+ * Multiplication in DNNs" (Chae, Chung, Lee, Kim), cited as [DyRA].
+ *
+ * The layer approximates Y = X W^T (PyTorch layout, W is d_out x d_in) by
+ *   Y = (X V) U^T + L C,                      [DyRA] Sec. 2.3 Eq. 6
+ * where U (d_out x r) and V (d_in x r) are a static rank-r factorisation of W,
+ * and L C is a rank-k correction of the residual output X W_res^T fitted to
+ * the input with one ridge-regularised ALS step ([DyRA] Sec. 2.2 Eq. 4-5,
+ * footnote 2; Appendix A, Algorithm 1, procedure Inference):
+ *   L = X P                                    (P precomputed, Eq. 7)
+ *   C = (L^T L + lambda I)^-1 (L^T X) W_res^T
+ * The correction is fitted separately for each batch instance ([DyRA]
+ * Sec. 2.4): X holds B consecutive instances of T rows each.
+ *
+ * Letters follow this library (static rank r, correction rank k); the paper
+ * uses k for the static rank and r for the correction rank.
+ *
+ * Conventions for every call:
+ *  - Matrices are dense, row-major, in the plan's storage type (float for
+ *    DYRA_F32, bfloat16 bit patterns for DYRA_BF16). Accumulation is fp32.
+ *  - Pointers to matrices are CUDA device pointers on the plan's device,
+ *    aligned to 16 bytes. The caller owns them.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous; no call below synchronises the device
+ *    except dyra_last_status and dyra_plan_destroy.
+ *  - A plan must not be used from two host threads or two streams at once.
+ *  - No call throws; each returns DYRA_OK (0) or a negative DYRA_ERR_* code.
+ */
+#ifndef DYRA_H_
+#define DYRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+typedef struct CUstream_st *dyra_stream_t;
+
+typedef struct dyra_plan *dyra_plan_t;
+
+typedef enum {
+  DYRA_F32 = 0,  /* float storage; SIMT fp32 kernels (no TF32) */
+  DYRA_BF16 = 1  /* bfloat16 storage; tcgen05 tensor-core kernels */
+} dyra_dtype_t;
+
+enum {
+  DYRA_OK = 0,
+  DYRA_ERR_INVALID_ARG = -1,    /* null pointer, non-positive or inconsistent size */
+  DYRA_ERR_NOT_LOADED = -2,     /* forward before dyra_load_factors */
+  DYRA_ERR_ALIGNMENT = -3,      /* pointer not 16-byte aligned, or a bf16 size not a multiple of 8 */
+  DYRA_ERR_RANK_DEFICIENT = -4, /* lambda == 0 and T < k: L^T L is singular */
+  DYRA_ERR_ALLOC = -5,          /* device allocation failed */
+  DYRA_ERR_CUDA = -6,           /* a CUDA runtime/driver call failed */
+  DYRA_ERR_UNSUPPORTED = -7,    /* device is not compute capability 10.0 (B200) */
+  DYRA_ERR_DEVICE = -8          /* a kernel raised its status word (see dyra_last_status) */
+};
+
+/* Device status bits reported by dyra_last_status (OR-ed together). */
+enum {
+  DYRA_STATUS_NONPOSITIVE_PIVOT = 1, /* Cholesky of L^T L + lambda I met a pivot <= 0 or NaN;
+                                        that instance's correction was set to zero */
+  DYRA_STATUS_WAIT_TIMEOUT = 2       /* a kernel's pipeline wait exceeded its time limit and the
+                                        kernel returned early; outputs are undefined */
+};
+
+/*
+ * Create a plan for one layer shape.
+ *   d_in, d_out : layer sizes (>= 1)
+ *   r           : static rank, 1 <= r
+ *   k           : correction rank, 0 <= k <= 128 (k == 0 gives the weight-only
+ *                 layer (X V) U^T, [DyRA] Sec. 2.1)
+ *   r + k <= min(d_in, d_out)   (both come from one SVD of W, Alg. 1 offline)
+ *   DYRA_BF16 additionally needs d_in, d_out, r, k to be multiples of 8
+ *   (16-byte rows for the tensor-memory-access unit), else DYRA_ERR_ALIGNMENT.
+ * The plan binds to the current CUDA device. *out receives the handle; it is
+ * left unchanged on error.
+ */
+int dyra_plan_create(dyra_plan_t *out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype);
+
+/*
+ * Copy the offline factors into the plan ([DyRA] Alg. 1, Offline Preparation
+ * outputs: the structured approximation, W_res and P_L).
+ *   U      : d_out x r   (singular values folded in: W_hat = U V^T)
+ *   V      : d_in x r
+ *   P      : d_in x k    (ignored when k == 0; may be NULL then)
+ *   W_res  : d_out x d_in, W - U V^T (ignored when k == 0; may be NULL then)
+ *   lambda : ridge constant >= 0 added to L^T L (footnote 2 of Sec. 2.2)
+ * The arrays are device pointers in the plan dtype; they are repacked into
+ * plan-owned buffers on `stream`, so the caller may free them once the stream
+ * has passed this call. May be called again to replace the factors.
+ */
+int dyra_load_factors(dyra_plan_t p, const void *U, const void *V, const void *P,
+                      const void *W_res, float lambda, dyra_stream_t stream);
+
+/*
+ * Y = DyRA(X) for one instance of N rows (B = 1, T = N).
+ *   X : N x d_in input, Y : N x d_out output (overwritten), N >= 0.
+ * N == 0 is a no-op. Returns DYRA_ERR_RANK_DEFICIENT if lambda == 0 and N < k.
+ */
+int dyra_forward(dyra_plan_t p, const void *X, void *Y, int64_t N, dyra_stream_t stream);
+
+/*
+ * Y = DyRA(X) with the correction fitted per instance: X and Y hold B
+ * consecutive instances of T rows ([DyRA] Sec. 2.4). B*T == 0 is a no-op.
+ * Returns DYRA_ERR_RANK_DEFICIENT if lambda == 0 and T < k.
+ */
+int dyra_forward_batched(dyra_plan_t p, const void *X, void *Y, int64_t B, int64_t T,
+                         dyra_stream_t stream);
+
+/*
+ * Y = (X V) U^T, the weight-only approximation ([DyRA] Sec. 2.1, first term of
+ * Eq. 2) with the plan's static factors, whatever the plan's k.
+ */
+int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
+                             dyra_stream_t stream);
+
+/*
+ * Grow the plan's workspace for up to B instances of T rows, so that later
+ * forwards of that size allocate nothing (call it before capturing a CUDA
+ * graph or timing). Forward calls grow the workspace themselves otherwise.
+ */
+int dyra_reserve(dyra_plan_t p, int64_t B, int64_t T);
+
+/*
+ * Synchronise the plan's device, then return and clear the device status
+ * bits (DYRA_STATUS_*) raised since the last call, or a negative error code.
+ */
+int dyra_last_status(dyra_plan_t p);
+
+/* Free the plan and its device buffers (synchronises the device). NULL is a no-op. */
+int dyra_plan_destroy(dyra_plan_t p);
+
+/* Static text for a DYRA_OK / DYRA_ERR_* code. */
+const char *dyra_error_string(int code);
+
+/* Bytes of device memory the plan currently owns (factors + workspace). */
+size_t dyra_plan_device_bytes(dyra_plan_t p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYRA_H_ */

@@ -1,0 +1,50 @@
+/*
+ * dyra_debug.h - diagnostics for include/dyra.h: read access to a plan's
+ * intermediate buffers, so each stage of the forward can be checked on its own.
+ * Not needed to run the layer.
+ */
+#ifndef DYRA_DEBUG_H_
+#define DYRA_DEBUG_H_
+
+#include <stddef.h>
+
+#include "dyra.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Workspace buffers, valid after a forward on the same stream has completed.
+ * Layouts for a DYRA_BF16 plan and a forward of B instances x T rows (N = B*T):
+ *   DYRA_BUF_Z   N x r bf16     X V                      ([DyRA] Alg. 1 line 10, first factor)
+ *   DYRA_BUF_L   N x k bf16     X P                      (line 11)
+ *   DYRA_BUF_TG  S x B x k x (d_in + k) fp32: per row split s and instance b,
+ *                columns [0, d_in) hold L_b^T X_b, columns [d_in, d_in + k) L_b^T L_b
+ *   DYRA_BUF_TP  (B*k) x d_in bf16   (L^T L + lambda I)^-1 L^T X per instance
+ *   DYRA_BUF_CT  d_out x (B*k) bf16  C^T = W_res T'^T   (line 12's R^(1), transposed)
+ * For a DYRA_F32 plan: Z holds N x (r+k) fp32 ([Z | L]), TG has S = 1,
+ * TP is fp32, and CT holds C as (B*k) x d_out fp32. */
+enum {
+  DYRA_BUF_Z = 0,
+  DYRA_BUF_L = 1,
+  DYRA_BUF_TG = 2,
+  DYRA_BUF_TP = 3,
+  DYRA_BUF_CT = 4
+};
+
+/* *ptr receives the device address of buffer `which` and *bytes its capacity
+ * (0 and NULL if not allocated). Returns DYRA_OK or DYRA_ERR_INVALID_ARG. */
+int dyra_debug_buffer(dyra_plan_t p, int which, const void **ptr, size_t *bytes);
+
+/* Copy `bytes` bytes of buffer `which` to host memory `dst` (synchronous on
+ * the plan's device). Returns DYRA_ERR_INVALID_ARG if the buffer is smaller. */
+int dyra_debug_copy(dyra_plan_t p, int which, void *dst, size_t bytes);
+
+/* Row splits S and rows per split used by the Gram stage for B x T. */
+int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int *splits, int *split_rows);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DYRA_DEBUG_H_ */

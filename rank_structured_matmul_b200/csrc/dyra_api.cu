@@ -1,0 +1,468 @@
+// dyra_api.cu - the C ABI declared in include/dyra.h.
+//
+// Owns the plan (shape, device, packed factors, workspace, status word),
+// validates every argument before touching the device, and dispatches the
+// forward to the tcgen05 kernels (bf16) or the SIMT kernels (fp32).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "dyra.h"
+#include "dyra_debug.h"
+#include "internal.h"
+
+struct dyra_plan {
+  int d_in = 0, d_out = 0, r = 0, k = 0;
+  dyra_dtype_t dtype = DYRA_BF16;
+  dyra::DeviceInfo dev;
+  bool loaded = false;
+  bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
+  float lambda = 0.f;
+  // packed factors
+  void* VPt = nullptr;   // (r+k) x d_in
+  void* U = nullptr;     // d_out x r
+  void* W_res = nullptr; // d_out x d_in
+  // workspace
+  void* Z = nullptr;     // bf16: N x r; fp32: N x (r+k)
+  void* L = nullptr;     // bf16: N x k
+  float* TG = nullptr;   // splits x B x k x (d_in + k)
+  void* Tp = nullptr;    // (B*k) x d_in
+  void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
+  size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0;
+  int* status = nullptr;
+  size_t factor_bytes = 0;
+};
+
+namespace {
+
+size_t elem_size(dyra_dtype_t t) { return t == DYRA_F32 ? 4 : 2; }
+
+bool fail_alloc_for_test() {
+  const char* e = std::getenv("DYRA_TEST_FAIL_ALLOC");
+  return e != nullptr && e[0] == '1';
+}
+
+int dev_alloc(void** p, size_t bytes) {
+  if (fail_alloc_for_test()) return DYRA_ERR_ALLOC;
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return DYRA_ERR_ALLOC;
+  }
+  return DYRA_OK;
+}
+
+void dev_free(void*& p) {
+  if (p) cudaFree(p);
+  p = nullptr;
+}
+
+// Grow a workspace buffer to at least `bytes`.
+int grow(void*& p, size_t& cap, size_t bytes) {
+  if (bytes <= cap) return DYRA_OK;
+  dev_free(p);
+  cap = 0;
+  const size_t rounded = (bytes + 255) & ~static_cast<size_t>(255);
+  int rc = dev_alloc(&p, rounded);
+  if (rc) return rc;
+  cap = rounded;
+  return DYRA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Run on the plan's device, restoring the caller's device afterwards.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
+  const int64_t N = B * T;
+  const size_t es = elem_size(p->dtype);
+  const int k = p->k;
+  int rc;
+  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+    if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
+    if (k > 0) {
+      int splits = 1, rows = 64;
+      dyra::gram_split(T, B, p->dev.sm_count, &splits, &rows);
+      if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
+      void* tg = p->TG;
+      rc = grow(tg, p->cap_TG,
+                static_cast<size_t>(splits) * B * k * (p->d_in + k) * sizeof(float));
+      p->TG = static_cast<float*>(tg);
+      if (rc) return rc;
+      if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
+      if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
+    }
+  } else {
+    if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * (p->r + k) * es))) return rc;
+    if (k > 0) {
+      void* tg = p->TG;
+      rc = grow(tg, p->cap_TG, static_cast<size_t>(B) * k * (p->d_in + k) * sizeof(float));
+      p->TG = static_cast<float*>(tg);
+      if (rc) return rc;
+      if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
+      if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
+    }
+  }
+  return DYRA_OK;
+}
+
+int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool weight_only,
+                cudaStream_t s) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (B < 0 || T < 0) return DYRA_ERR_INVALID_ARG;
+  const int64_t N = B * T;
+  if (N == 0) return DYRA_OK;
+  if (X == nullptr || Y == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (N > (static_cast<int64_t>(1) << 31) - 1 || B * static_cast<int64_t>(p->k) > (1 << 30))
+    return DYRA_ERR_INVALID_ARG;
+  if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  if (!aligned16(X) || !aligned16(Y)) return DYRA_ERR_ALIGNMENT;
+  const bool correct = !weight_only && p->k > 0;
+  if (correct && p->lambda == 0.f && T < p->k) return DYRA_ERR_RANK_DEFICIENT;
+
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  int rc = ensure_workspace(p, B, T);
+  if (rc) return rc;
+
+  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+    dyra::Bf16Forward a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = p->k;
+    a.B = B;
+    a.T = T;
+    a.X = X;
+    a.Y = Y;
+    a.VPt = p->VPt;
+    a.U = p->U;
+    a.W_res = p->W_res;
+    a.lambda = p->lambda;
+    a.weight_only = !correct;
+    a.Z = p->Z;
+    a.L = p->L;
+    a.TG = p->TG;
+    a.Tp = p->Tp;
+    a.Ct = p->Ct;
+    a.splits = 1;
+    a.split_rows = 64;
+    if (correct) dyra::gram_split(T, B, p->dev.sm_count, &a.splits, &a.split_rows);
+    a.status = p->status;
+    rc = dyra::launch_bf16_forward(a, p->dev, s);
+  } else if (p->dtype == DYRA_BF16) {
+    dyra::SimtForward<__nv_bfloat16> a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = p->k;
+    a.B = B;
+    a.Trows = T;
+    a.X = static_cast<const __nv_bfloat16*>(X);
+    a.Y = static_cast<__nv_bfloat16*>(Y);
+    a.VPt = static_cast<const __nv_bfloat16*>(p->VPt);
+    a.U = static_cast<const __nv_bfloat16*>(p->U);
+    a.W_res = static_cast<const __nv_bfloat16*>(p->W_res);
+    a.lambda = p->lambda;
+    a.weight_only = !correct;
+    a.ZL = static_cast<__nv_bfloat16*>(p->Z);
+    a.TG = p->TG;
+    a.Tp = static_cast<__nv_bfloat16*>(p->Tp);
+    a.Cm = static_cast<__nv_bfloat16*>(p->Ct);
+    a.status = p->status;
+    rc = dyra::launch_simt_forward(a, p->dev, s);
+  } else {
+    dyra::SimtForward<float> a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = p->k;
+    a.B = B;
+    a.Trows = T;
+    a.X = static_cast<const float*>(X);
+    a.Y = static_cast<float*>(Y);
+    a.VPt = static_cast<const float*>(p->VPt);
+    a.U = static_cast<const float*>(p->U);
+    a.W_res = static_cast<const float*>(p->W_res);
+    a.lambda = p->lambda;
+    a.weight_only = !correct;
+    a.ZL = static_cast<float*>(p->Z);
+    a.TG = p->TG;
+    a.Tp = static_cast<float*>(p->Tp);
+    a.Cm = static_cast<float*>(p->Ct);
+    a.status = p->status;
+    rc = dyra::launch_simt_forward(a, p->dev, s);
+  }
+  if (rc != 0) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  return DYRA_OK;
+}
+
+}  // namespace
+
+namespace dyra {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (swizzle_bytes == 32) sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  if (swizzle_bytes == 64) sw = CU_TENSOR_MAP_SWIZZLE_64B;
+  if (swizzle_bytes == 128) sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  cuuint64_t d[5];
+  cuuint64_t st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides_bytes[i];
+  }
+  std::memset(map, 0, sizeof(*map));
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+            const_cast<void*>(base), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace dyra
+
+extern "C" {
+
+const char* dyra_error_string(int code) {
+  switch (code) {
+    case DYRA_OK: return "ok";
+    case DYRA_ERR_INVALID_ARG: return "invalid argument";
+    case DYRA_ERR_NOT_LOADED: return "factors not loaded";
+    case DYRA_ERR_ALIGNMENT: return "misaligned pointer or size";
+    case DYRA_ERR_RANK_DEFICIENT: return "lambda == 0 and fewer rows than the correction rank";
+    case DYRA_ERR_ALLOC: return "device allocation failed";
+    case DYRA_ERR_CUDA: return "CUDA call failed";
+    case DYRA_ERR_UNSUPPORTED: return "device is not compute capability 10.0";
+    case DYRA_ERR_DEVICE: return "device status raised";
+    default: return "unknown error";
+  }
+}
+
+int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype) {
+  if (out == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
+  if (d_in < 1 || d_out < 1 || r < 1 || k < 0 || k > 128) return DYRA_ERR_INVALID_ARG;
+  const int m = d_in < d_out ? d_in : d_out;
+  if (r + k > m) return DYRA_ERR_INVALID_ARG;
+  if (dtype == DYRA_BF16 && (d_in % 8 || d_out % 8 || r % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return DYRA_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return DYRA_ERR_UNSUPPORTED;
+
+  dyra_plan* p = new (std::nothrow) dyra_plan();
+  if (!p) return DYRA_ERR_ALLOC;
+  p->d_in = d_in;
+  p->d_out = d_out;
+  p->r = r;
+  p->k = k;
+  p->dtype = dtype;
+  p->dev.device = dev;
+  p->dev.sm_count = prop.multiProcessorCount;
+  p->dev.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+  p->dev.cc_major = prop.major;
+  p->dev.cc_minor = prop.minor;
+  const char* kv = std::getenv("DYRA_KERNELS");
+  p->force_simt = kv != nullptr && std::strcmp(kv, "simt") == 0;
+  void* st = nullptr;
+  if (dev_alloc(&st, 256) != DYRA_OK) {
+    delete p;
+    return DYRA_ERR_ALLOC;
+  }
+  p->status = static_cast<int*>(st);
+  if (cudaMemset(p->status, 0, sizeof(int)) != cudaSuccess) {
+    dev_free(st);
+    delete p;
+    return DYRA_ERR_CUDA;
+  }
+  *out = p;
+  return DYRA_OK;
+}
+
+int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P,
+                      const void* W_res, float lambda, dyra_stream_t stream) {
+  if (p == nullptr || U == nullptr || V == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (p->k > 0 && (P == nullptr || W_res == nullptr)) return DYRA_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f) || !std::isfinite(lambda)) return DYRA_ERR_INVALID_ARG;
+  if (!aligned16(U) || !aligned16(V) || (p->k > 0 && (!aligned16(P) || !aligned16(W_res))))
+    return DYRA_ERR_ALIGNMENT;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(p->dtype);
+  const size_t vpt = static_cast<size_t>(p->r + p->k) * p->d_in * es;
+  const size_t ub = static_cast<size_t>(p->d_out) * p->r * es;
+  const size_t wb = p->k > 0 ? static_cast<size_t>(p->d_out) * p->d_in * es : 0;
+  int rc;
+  if (!p->VPt && (rc = dev_alloc(&p->VPt, vpt))) return rc;
+  if (!p->U && (rc = dev_alloc(&p->U, ub))) return rc;
+  if (wb && !p->W_res && (rc = dev_alloc(&p->W_res, wb))) return rc;
+  p->factor_bytes = vpt + ub + wb;
+  if (cudaMemcpyAsync(p->U, U, ub, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return DYRA_ERR_CUDA;
+  if (wb && cudaMemcpyAsync(p->W_res, W_res, wb, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return DYRA_ERR_CUDA;
+  if (p->dtype == DYRA_BF16)
+    rc = dyra::launch_pack_vp(static_cast<const __nv_bfloat16*>(V),
+                              static_cast<const __nv_bfloat16*>(P),
+                              static_cast<__nv_bfloat16*>(p->VPt), p->d_in, p->r, p->k, s);
+  else
+    rc = dyra::launch_pack_vp(static_cast<const float*>(V), static_cast<const float*>(P),
+                              static_cast<float*>(p->VPt), p->d_in, p->r, p->k, s);
+  if (rc) return DYRA_ERR_CUDA;
+  p->lambda = lambda;
+  p->loaded = true;
+  return DYRA_OK;
+}
+
+int dyra_forward(dyra_plan_t p, const void* X, void* Y, int64_t N, dyra_stream_t stream) {
+  return run_forward(p, X, Y, 1, N, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dyra_forward_batched(dyra_plan_t p, const void* X, void* Y, int64_t B, int64_t T,
+                         dyra_stream_t stream) {
+  return run_forward(p, X, Y, B, T, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dyra_forward_weight_only(dyra_plan_t p, const void* X, void* Y, int64_t N,
+                             dyra_stream_t stream) {
+  return run_forward(p, X, Y, 1, N, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dyra_reserve(dyra_plan_t p, int64_t B, int64_t T) {
+  if (p == nullptr || B < 0 || T < 0) return DYRA_ERR_INVALID_ARG;
+  if (B * T == 0) return DYRA_OK;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  return ensure_workspace(p, B, T);
+}
+
+int dyra_last_status(dyra_plan_t p) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DYRA_ERR_CUDA;
+  int st = 0;
+  if (cudaMemcpy(&st, p->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DYRA_ERR_CUDA;
+  if (cudaMemset(p->status, 0, sizeof(int)) != cudaSuccess) return DYRA_ERR_CUDA;
+  return st;
+}
+
+int dyra_plan_destroy(dyra_plan_t p) {
+  if (p == nullptr) return DYRA_OK;
+  {
+    DeviceGuard g(p->dev.device);
+    cudaDeviceSynchronize();
+    dev_free(p->VPt);
+    dev_free(p->U);
+    dev_free(p->W_res);
+    dev_free(p->Z);
+    dev_free(p->L);
+    void* tg = p->TG;
+    dev_free(tg);
+    dev_free(p->Tp);
+    dev_free(p->Ct);
+    void* st = p->status;
+    dev_free(st);
+  }
+  delete p;
+  return DYRA_OK;
+}
+
+int dyra_debug_buffer(dyra_plan_t p, int which, const void** ptr, size_t* bytes) {
+  if (p == nullptr || ptr == nullptr || bytes == nullptr) return DYRA_ERR_INVALID_ARG;
+  switch (which) {
+    case DYRA_BUF_Z: *ptr = p->Z; *bytes = p->cap_Z; break;
+    case DYRA_BUF_L: *ptr = p->L; *bytes = p->cap_L; break;
+    case DYRA_BUF_TG: *ptr = p->TG; *bytes = p->cap_TG; break;
+    case DYRA_BUF_TP: *ptr = p->Tp; *bytes = p->cap_Tp; break;
+    case DYRA_BUF_CT: *ptr = p->Ct; *bytes = p->cap_Ct; break;
+    default: return DYRA_ERR_INVALID_ARG;
+  }
+  return DYRA_OK;
+}
+
+int dyra_debug_copy(dyra_plan_t p, int which, void* dst, size_t bytes) {
+  const void* src = nullptr;
+  size_t cap = 0;
+  int rc = dyra_debug_buffer(p, which, &src, &cap);
+  if (rc) return rc;
+  if (dst == nullptr || src == nullptr || bytes > cap) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DYRA_ERR_CUDA;
+  return cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? DYRA_OK
+                                                                            : DYRA_ERR_CUDA;
+}
+
+int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int* split_rows) {
+  if (p == nullptr || splits == nullptr || split_rows == nullptr || B < 0 || T < 0)
+    return DYRA_ERR_INVALID_ARG;
+  if (p->dtype == DYRA_F32 || p->force_simt) {
+    *splits = 1;
+    *split_rows = static_cast<int>(T);
+    return DYRA_OK;
+  }
+  dyra::gram_split(T, B, p->dev.sm_count, splits, split_rows);
+  return DYRA_OK;
+}
+
+size_t dyra_plan_device_bytes(dyra_plan_t p) {
+  if (p == nullptr) return 0;
+  return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + 256;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// internal.h - interfaces between the C ABI (dyra_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace dyra {
+
+struct DeviceInfo {
+  int device = 0;
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  int cc_major = 0, cc_minor = 0;
+};
+
+// ---------------------------------------------------------------- TMA ----
+
+// Encode a 2-D or 3-D bf16 tiled tensor map (dims and box innermost first,
+// strides in bytes for dims 1..rank-1). swizzle_bytes: 0, 32, 64 or 128.
+// Returns false if the driver rejects it.
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
+
+// --------------------------------------------------- bf16 forward (tcgen05) ----
+
+struct Bf16Forward {
+  int d_in, d_out, r, k;
+  int64_t B, T;          // instances x rows per instance
+  const void* X;         // N x d_in
+  void* Y;               // N x d_out
+  const void* VPt;       // (r+k) x d_in   ([V | P] transposed)
+  const void* U;         // d_out x r
+  const void* W_res;     // d_out x d_in
+  float lambda;
+  bool weight_only;      // skip the correction (k treated as 0)
+  // workspace
+  void* Z;               // N x r
+  void* L;               // N x k
+  float* TG;             // splits x B x k x (d_in + k)
+  void* Tp;              // (B*k) x d_in
+  void* Ct;              // d_out x (B*k)
+  int splits;            // row splits of the Gram reduction
+  int split_rows;        // rows per split (multiple of 64)
+  int* status;
+};
+
+// Rows per split and split count used for a given T (shared with the
+// workspace sizing).
+void gram_split(int64_t T, int64_t B, int sm_count, int* splits, int* split_rows);
+
+int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s);
+
+// ------------------------------------------------------- SIMT (fp32) ----
+
+template <typename T>
+struct SimtForward {
+  int d_in, d_out, r, k;
+  int64_t B, Trows;
+  const T* X;
+  T* Y;
+  const T* VPt;
+  const T* U;
+  const T* W_res;
+  float lambda;
+  bool weight_only;
+  T* ZL;        // N x (r+k)
+  float* TG;    // B x k x (d_in + k)
+  T* Tp;        // (B*k) x d_in
+  T* Cm;        // (B*k) x d_out
+  int* status;
+};
+
+template <typename T>
+int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStream_t s);
+
+// Solve (L^T L + lambda I) T' = T for every instance from the Gram partials.
+template <typename TOut>
+int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda,
+                 TOut* Tp, int* status, cudaStream_t s, bool pdl);
+
+// Pack [V | P]^T: VPt[c][j] = V[j][c] (c < r), P[j][c-r] (c >= r).
+template <typename T>
+int launch_pack_vp(const T* V, const T* P, T* VPt, int d_in, int r, int k, cudaStream_t s);
+
+}  // namespace dyra

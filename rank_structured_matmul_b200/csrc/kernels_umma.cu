@@ -1,0 +1,615 @@
+// kernels_umma.cu - the bf16 DyRA forward on tcgen05 tensor cores.
+//
+// Method: "DyRA: Dynamic Residual Approximation for Efficient Matrix
+// Multiplication in DNNs", Appendix A, Algorithm 1, procedure Inference, with
+// the correction fitted per batch instance (Sec. 2.4). Letters: static rank r,
+// correction rank k, Y = X W^T with W = d_out x d_in.
+//
+// Four tensor-core GEMMs and one small solve, stream-ordered:
+//   proj    [Z | L] = X [V | P]              Alg. 1 lines 10-11, Eq. 7
+//   gram    per instance b: [T_b | G_b] = L_b^T [X_b | L_b]      line 12
+//   solve   T'_b = (G_b + lambda I)^-1 T_b   (kernels_simt.cu)  line 12
+//   rfactor C^T = W_res T'^T, all instances at once              line 12
+//   out     Y = Z U^T + sum_b mask_b(L) C_b, one TMEM accumulation  line 13
+// C_b is the paper's R^(1) for instance b; computing (G^-1 L^T X) W_res^T
+// instead of G^-1 ((L^T X) W_res^T) is the same product reassociated.
+//
+// Storage bf16, accumulation fp32 in tensor memory. Every operand tile is
+// brought in by TMA with 128-byte swizzling (64 bf16 per row); tiles that run
+// past a tensor's edge are zero-filled by TMA, which also masks instance
+// boundaries: L and X are addressed as 3-D (k or d_in, T, B) tensors, so rows
+// outside the instance read as zero.
+#include <algorithm>
+#include <cstdio>
+
+#include "internal.h"
+#include "umma_gemm.cuh"
+
+namespace dyra {
+
+using namespace sm100;
+
+namespace {
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int ks) {
+  // K-major, 128-byte swizzle: rows of 64 bf16, 8-row atoms 1024 bytes apart;
+  // the k-th group of 16 elements starts 32 bytes further into each row.
+  return smem_desc(base + static_cast<uint32_t>(ks) * 32u, 16u, 1024u, kLayoutSw128);
+}
+
+__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+
+// Write eight fp32 accumulator values as one 16-byte bf16 vector.
+__device__ __forceinline__ void store8_bf16(void* dst, const uint32_t (&v)[32], int g) {
+  st_global_v4(dst, pack_bf16x2(f32(v[8 * g + 0]), f32(v[8 * g + 1])),
+               pack_bf16x2(f32(v[8 * g + 2]), f32(v[8 * g + 3])),
+               pack_bf16x2(f32(v[8 * g + 4]), f32(v[8 * g + 5])),
+               pack_bf16x2(f32(v[8 * g + 6]), f32(v[8 * g + 7])));
+}
+
+__device__ __forceinline__ int ceil_div_dev(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+// =================================================================== proj ====
+// [Z | L] = X . [V | P]: A = X (K-major), B = [V|P]^T (K-major). X is read
+// from HBM once; the n-tiles of one m-tile run on neighbouring CTAs and share
+// it through L2.
+struct ProjPolicy {
+  struct Params {
+    GemmCommon c;
+    CUtensorMap tmX;  // (d_in, N), box (64, 128)
+    CUtensorMap tmW;  // (d_in, r+k), box (64, bn)
+    int N, d_in, r, k, bn, n_tiles_n;
+    __nv_bfloat16* Z;
+    __nv_bfloat16* L;
+  };
+  struct Tile {
+    int m0, n0;
+  };
+  static constexpr uint32_t kEpiSmemBytes = 0;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmW);
+  }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 128;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile&) {
+    return ceil_div_dev(p.d_in, 64);
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    tma_load_2d(sa, &p.tmX, bar, it * 64, t.m0);
+    tma_load_2d(sb, &p.tmW, bar, it * 64, t.n0);
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
+    return min(4, ceil_div_dev(p.d_in - it * 64, 16));
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    const int grow = t.m0 + e.row;
+    const int rk = p.r + p.k;
+    for (int cc = 0; cc < p.bn; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + cc, v);
+      tmem_ld_wait();
+      if (grow < p.N) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = t.n0 + cc + 8 * g;
+          if (col < rk) {
+            void* dst = col < p.r
+                            ? static_cast<void*>(p.Z + static_cast<size_t>(grow) * p.r + col)
+                            : static_cast<void*>(p.L + static_cast<size_t>(grow) * p.k + (col - p.r));
+            store8_bf16(dst, v, g);
+          }
+        }
+      }
+    }
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
+};
+
+// =================================================================== gram ====
+// For every instance b and row split s: D = [X_b | L_b]^T L_b over the split's
+// rows, i.e. T_b^T (d_in x k) and G_b (k x k) partial sums, written to
+// TG[s][b][i][j] (j < d_in: T_b[i][j]; j = d_in + i': G_b[i][i']).
+// Both operands are MN-major (the reduction runs over rows of X and L).
+struct GramPolicy {
+  struct Params {
+    GemmCommon c;
+    CUtensorMap tmX;   // (d_in, T, B), box (64, 64, 1), 128B swizzle
+    CUtensorMap tmLa;  // (k, T, B),    box (64, 64, 1), 128B swizzle   (A role)
+    CUtensorMap tmLb;  // (k, T, B),    box (w, 64, 1),  w*2-byte swizzle (B role)
+    int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total, J;
+    uint32_t b_layout;
+    float* TG;
+  };
+  struct Tile {
+    int mt, b, s, t0, t1;
+  };
+  static constexpr uint32_t kEpiSmemBytes = 0;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmLa);
+    tma_prefetch_desc(&p.tmLb);
+  }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.mt = tile % p.mt_total;
+    const int rest = tile / p.mt_total;
+    t.b = rest % p.B;
+    t.s = rest / p.B;
+    t.t0 = t.s * p.Ts;
+    t.t1 = min(p.T, t.t0 + p.Ts);
+  }
+  static __device__ __forceinline__ int kiters(const Params&, const Tile& t) {
+    return ceil_div_dev(t.t1 - t.t0, 64);
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    const int row = t.t0 + it * 64;
+    if (t.mt < p.mtx) {
+      const int j0 = t.mt * 128;
+      tma_load_3d(sa, &p.tmX, bar, j0, row, t.b);
+      tma_load_3d(sa + 8192u, &p.tmX, bar, j0 + 64, row, t.b);
+    } else {
+      const int i0 = (t.mt - p.mtx) * 128;
+      tma_load_3d(sa, &p.tmLa, bar, i0, row, t.b);
+      tma_load_3d(sa + 8192u, &p.tmLa, bar, i0 + 64, row, t.b);
+    }
+    const uint32_t box_b = static_cast<uint32_t>(p.w) * 2u * 64u;
+    for (int q = 0; q < p.nbox_b; ++q) tma_load_3d(sb + q * box_b, &p.tmLb, bar, 64 * q, row, t.b);
+  }
+  static __device__ __forceinline__ int ksteps(const Params&, const Tile&, int) { return 4; }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    // MN-major, 128-byte swizzle: 64 elements of M per 128-byte row, 8 K-rows
+    // per 1024-byte atom (SBO), the second 64-wide M block 8 KB away (LBO).
+    return smem_desc(a + static_cast<uint32_t>(ks) * 2048u, 8192u, 1024u, kLayoutSw128);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params& p, uint32_t b, int ks) {
+    const uint32_t rb = static_cast<uint32_t>(p.w) * 2u;  // bytes per K-row of one block
+    return smem_desc(b + static_cast<uint32_t>(ks) * 16u * rb, 64u * rb, 8u * rb, p.b_layout);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    int jcol;
+    bool valid;
+    if (t.mt < p.mtx) {
+      jcol = t.mt * 128 + e.row;
+      valid = jcol < p.d_in;
+    } else {
+      const int i2 = (t.mt - p.mtx) * 128 + e.row;
+      jcol = p.d_in + i2;
+      valid = i2 < p.k;
+    }
+    float* out = p.TG + static_cast<size_t>(t.s * p.B + t.b) * p.k * p.J + jcol;
+    for (int cc = 0; cc < p.kpad; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + cc, v);
+      tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int i = cc + jj;
+          if (i < p.k) out[static_cast<size_t>(i) * p.J] = f32(v[jj]);
+        }
+      }
+    }
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
+};
+
+// ================================================================ rfactor ====
+// C^T = W_res . T'^T (d_out x B*k): A = W_res (K-major), B = T' (K-major).
+// W_res is streamed from HBM once per n-tile column of C^T.
+struct RFactorPolicy {
+  struct Params {
+    GemmCommon c;
+    CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
+    CUtensorMap tmT;  // (d_in, B*k),   box (64, bn)
+    int d_in, d_out, Bk, bn, n_tiles_n;
+    __nv_bfloat16* Ct;
+  };
+  struct Tile {
+    int m0, n0;
+  };
+  static constexpr uint32_t kEpiSmemBytes = 0;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmW);
+    tma_prefetch_desc(&p.tmT);
+  }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 128;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile&) {
+    return ceil_div_dev(p.d_in, 64);
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    tma_load_2d(sa, &p.tmW, bar, it * 64, t.m0);
+    tma_load_2d(sb, &p.tmT, bar, it * 64, t.n0);
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
+    return min(4, ceil_div_dev(p.d_in - it * 64, 16));
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    const int grow = t.m0 + e.row;
+    for (int cc = 0; cc < p.bn; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + cc, v);
+      tmem_ld_wait();
+      if (grow < p.d_out) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = t.n0 + cc + 8 * g;
+          if (col < p.Bk) store8_bf16(p.Ct + static_cast<size_t>(grow) * p.Bk + col, v, g);
+        }
+      }
+    }
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
+};
+
+// ==================================================================== out ====
+// Y = Z U^T + sum over the instances b the m-tile touches of mask_b(L) C_b,
+// accumulated in one TMEM tile: K-segments [Z | L_b_lo | ... | L_b_hi] against
+// [U ; C_b_lo ; ... ; C_b_hi]. mask_b(L) is L's rows of instance b and zero
+// elsewhere, produced by TMA's out-of-bounds fill on the 3-D view of L.
+// The bf16 result goes out through a swizzled shared-memory box and TMA
+// stores, double buffered so the next box is written while one drains.
+struct OutPolicy {
+  struct Params {
+    GemmCommon c;
+    CUtensorMap tmZ;  // (r, N),        box (64, 128)
+    CUtensorMap tmU;  // (r, d_out),    box (64, bn)
+    CUtensorMap tmL;  // (k, T, B),     box (64, 128, 1)
+    CUtensorMap tmC;  // (B*k, d_out),  box (64, bn)
+    CUtensorMap tmY;  // (d_out, N),    box (64, 128), store
+    int N, r, k, T, B, bn, n_tiles_n, nkz, nkl;
+  };
+  struct Tile {
+    int m0, n0, b_lo, nseg;
+  };
+  static constexpr uint32_t kBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
+  static constexpr uint32_t kEpiSmemBytes = 2u * kBoxBytes;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmZ);
+    tma_prefetch_desc(&p.tmU);
+    if (p.nkl > 0) {
+      tma_prefetch_desc(&p.tmL);
+      tma_prefetch_desc(&p.tmC);
+    }
+    tma_prefetch_desc(&p.tmY);
+  }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 128;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+    if (p.nkl > 0) {
+      t.b_lo = t.m0 / p.T;
+      const int b_hi = min(p.B - 1, (t.m0 + 127) / p.T);
+      t.nseg = b_hi - t.b_lo + 1;
+    } else {
+      t.b_lo = 0;
+      t.nseg = 0;
+    }
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    return p.nkz + t.nseg * p.nkl;
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    if (it < p.nkz) {
+      tma_load_2d(sa, &p.tmZ, bar, it * 64, t.m0);
+      tma_load_2d(sb, &p.tmU, bar, it * 64, t.n0);
+    } else {
+      const int j = it - p.nkz;
+      const int seg = j / p.nkl;
+      const int ch = j - seg * p.nkl;
+      const int b = t.b_lo + seg;
+      tma_load_3d(sa, &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
+      tma_load_2d(sb, &p.tmC, bar, b * p.k + ch * 64, t.n0);
+    }
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
+    if (it < p.nkz) return min(4, ceil_div_dev(p.r - it * 64, 16));
+    const int ch = (it - p.nkz) % p.nkl;
+    return min(4, ceil_div_dev(p.k - ch * 64, 16));
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    const int nbox = p.bn / 64;
+    for (int bx = 0; bx < nbox; ++bx) {
+      const uint32_t buf = e.counter & 1u;
+      ++e.counter;
+      // The buffer about to be overwritten was handed to TMA two boxes ago.
+      if (e.tid == 0) tma_store_wait_read<1>();
+      named_bar_sync(1, 128);
+      uint8_t* sbuf = e.smem + buf * kBoxBytes;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tacc + bx * 64 + half * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = half * 4 + ch;
+          const uint32_t off = static_cast<uint32_t>(e.row) * 128u +
+                               static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+          uint4 q;
+          q.x = pack_bf16x2(f32(v[8 * ch + 0]), f32(v[8 * ch + 1]));
+          q.y = pack_bf16x2(f32(v[8 * ch + 2]), f32(v[8 * ch + 3]));
+          q.z = pack_bf16x2(f32(v[8 * ch + 4]), f32(v[8 * ch + 5]));
+          q.w = pack_bf16x2(f32(v[8 * ch + 6]), f32(v[8 * ch + 7]));
+          *reinterpret_cast<uint4*>(sbuf + off) = q;
+        }
+      }
+      fence_async_shared();
+      named_bar_sync(1, 128);
+      if (e.tid == 0) {
+        tma_store_2d(&p.tmY, e.smem_u32 + buf * kBoxBytes, t.n0 + bx * 64, t.m0);
+        tma_store_commit();
+      }
+    }
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) {
+    if (e.tid == 0) tma_store_wait_all();
+  }
+};
+
+// ============================================================= host side ====
+
+namespace {
+
+inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+uint32_t pow2_at_least(uint32_t x) {
+  uint32_t v = 32;
+  while (v < x) v <<= 1;
+  return v;
+}
+
+// Fill the shared part of the launch parameters; returns dynamic smem bytes
+// or 0 if the tile shape does not fit.
+template <class Pol>
+uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b_bytes,
+                      int mma_n, bool a_mn, bool b_mn, int* status, const DeviceInfo& dev) {
+  c.num_tiles = num_tiles;
+  c.a_stage_bytes = a_bytes;
+  c.b_stage_bytes = b_bytes;
+  c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
+  c.tmem_cols = pow2_at_least(2 * c.acc_cols);
+  if (c.tmem_cols > 512) return 0;
+  c.idesc = idesc_bf16(128, mma_n, a_mn, b_mn);
+  c.status = status;
+  const uint32_t fixed = gemm_smem_bytes(0, a_bytes, b_bytes, Pol::kEpiSmemBytes);
+  const int budget = dev.max_smem_optin - static_cast<int>(fixed);
+  int stages = budget / static_cast<int>(a_bytes + b_bytes);
+  stages = std::min(stages, kMaxStages);
+  if (stages < 2) return 0;
+  c.stages = stages;
+  return gemm_smem_bytes(stages, a_bytes, b_bytes, Pol::kEpiSmemBytes);
+}
+
+template <class Pol>
+int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& dev,
+                cudaStream_t s, bool pdl) {
+  if (p.c.num_tiles <= 0) return 0;
+  auto kfn = umma_gemm_kernel<Pol>;
+  static uint32_t configured = 0;
+  if (smem > configured) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+    configured = smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min(p.c.num_tiles, dev.sm_count)));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kfn, p) == cudaSuccess ? 0 : -1;
+}
+
+// Column tile for a K-major B operand of n columns: at most 256 wide, a
+// multiple of 32, chosen so the tiles split n evenly.
+int pick_bn(int n) {
+  const int tiles = ceil_div(n, 256);
+  int bn = ceil_div(ceil_div(n, tiles), 32) * 32;
+  return std::min(bn, 256);
+}
+
+}  // namespace
+
+void gram_split(int64_t T, int64_t B, int sm_count, int* splits, int* split_rows) {
+  // Enough (instance, split) pairs to cover the SMs for long instances;
+  // splits are whole 64-row blocks so no block straddles two splits.
+  const int64_t blocks = (T + 63) / 64;
+  int64_t want = std::max<int64_t>(1, (2 * sm_count) / std::max<int64_t>(1, B * 8));
+  want = std::min<int64_t>(want, blocks);
+  const int64_t per = (blocks + want - 1) / want;
+  *split_rows = static_cast<int>(per * 64);
+  *splits = static_cast<int>((blocks + per - 1) / per);
+}
+
+int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s) {
+  const int64_t N = a.B * a.T;
+  if (N == 0) return 0;
+  const int k = a.weight_only ? 0 : a.k;
+  const int rk = a.r + a.k;  // VPt rows always hold [V | P]
+  const bool pdl = true;
+
+  // ---------------------------------------------------------------- proj
+  {
+    ProjPolicy::Params p;
+    const int n_cols = a.weight_only ? a.r : rk;
+    p.N = static_cast<int>(N);
+    p.d_in = a.d_in;
+    p.r = a.r;
+    p.k = a.weight_only ? 0 : a.k;
+    p.bn = pick_bn(n_cols);
+    p.n_tiles_n = ceil_div(n_cols, p.bn);
+    p.Z = static_cast<__nv_bfloat16*>(a.Z);
+    p.L = static_cast<__nv_bfloat16*>(a.L);
+    uint64_t dx[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(N)};
+    uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
+    uint32_t bx[2] = {64, 128};
+    if (!encode_tmap_bf16(&p.tmX, a.X, 2, dx, sx, bx, 128)) return -2;
+    uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(rk)};
+    uint32_t bw[2] = {64, static_cast<uint32_t>(p.bn)};
+    if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
+    const int tiles = ceil_div(N, 128) * p.n_tiles_n;
+    const uint32_t smem = setup_common<ProjPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
+                                                   false, a.status, dev);
+    if (!smem) return -3;
+    if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
+  }
+
+  if (k > 0) {
+    const int J = a.d_in + a.k;
+    // -------------------------------------------------------------- gram
+    {
+      GramPolicy::Params p;
+      p.d_in = a.d_in;
+      p.k = a.k;
+      p.kpad = a.k <= 32 ? 32 : ceil_div(a.k, 64) * 64;
+      p.w = std::min(p.kpad, 64);
+      p.nbox_b = p.kpad / p.w;
+      p.T = static_cast<int>(a.T);
+      p.B = static_cast<int>(a.B);
+      p.S = a.splits;
+      p.Ts = a.split_rows;
+      p.mtx = ceil_div(a.d_in, 128);
+      p.mt_total = p.mtx + ceil_div(a.k, 128);
+      p.J = J;
+      p.TG = a.TG;
+      p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
+      uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
+                        static_cast<uint64_t>(a.B)};
+      uint64_t sx[2] = {static_cast<uint64_t>(a.d_in) * 2,
+                        static_cast<uint64_t>(a.d_in) * 2 * static_cast<uint64_t>(a.T)};
+      uint32_t bx[3] = {64, 64, 1};
+      if (!encode_tmap_bf16(&p.tmX, a.X, 3, dx, sx, bx, 128)) return -2;
+      uint64_t dl[3] = {static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.T),
+                        static_cast<uint64_t>(a.B)};
+      uint64_t sl[2] = {static_cast<uint64_t>(a.k) * 2,
+                        static_cast<uint64_t>(a.k) * 2 * static_cast<uint64_t>(a.T)};
+      if (!encode_tmap_bf16(&p.tmLa, a.L, 3, dl, sl, bx, 128)) return -2;
+      uint32_t bl[3] = {static_cast<uint32_t>(p.w), 64, 1};
+      if (!encode_tmap_bf16(&p.tmLb, a.L, 3, dl, sl, bl, p.w * 2)) return -2;
+      const int tiles = p.mt_total * p.B * p.S;
+      const uint32_t smem =
+          setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
+                                   p.kpad, true, true, a.status, dev);
+      if (!smem) return -3;
+      if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl)) return -1;
+    }
+    // ------------------------------------------------------------- solve
+    if (launch_solve<__nv_bfloat16>(a.TG, a.splits, a.B, a.k, a.d_in, a.lambda,
+                                    static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl))
+      return -1;
+    // ----------------------------------------------------------- rfactor
+    {
+      RFactorPolicy::Params p;
+      const int Bk = static_cast<int>(a.B) * a.k;
+      p.d_in = a.d_in;
+      p.d_out = a.d_out;
+      p.Bk = Bk;
+      p.bn = pick_bn(Bk);
+      p.n_tiles_n = ceil_div(Bk, p.bn);
+      p.Ct = static_cast<__nv_bfloat16*>(a.Ct);
+      uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.d_out)};
+      uint64_t sw[1] = {static_cast<uint64_t>(a.d_in) * 2};
+      uint32_t bw[2] = {64, 128};
+      if (!encode_tmap_bf16(&p.tmW, a.W_res, 2, dw, sw, bw, 128)) return -2;
+      uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
+      uint32_t bt[2] = {64, static_cast<uint32_t>(p.bn)};
+      if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
+      const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
+      const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
+                                                        false, false, a.status, dev);
+      if (!smem) return -3;
+      if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
+    }
+  }
+
+  // ------------------------------------------------------------------ out
+  {
+    OutPolicy::Params p;
+    p.N = static_cast<int>(N);
+    p.r = a.r;
+    p.k = k;
+    p.T = static_cast<int>(a.T);
+    p.B = static_cast<int>(a.B);
+    p.bn = a.d_out % 256 == 0 ? 256 : (a.d_out % 128 == 0 ? 128 : 64);
+    if (a.d_out < p.bn) p.bn = 64;
+    p.n_tiles_n = ceil_div(a.d_out, p.bn);
+    p.nkz = ceil_div(a.r, 64);
+    p.nkl = k > 0 ? ceil_div(k, 64) : 0;
+    uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
+    uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+    uint32_t bz[2] = {64, 128};
+    if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bz, 128)) return -2;
+    uint64_t du[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(a.d_out)};
+    uint32_t bu[2] = {64, static_cast<uint32_t>(p.bn)};
+    if (!encode_tmap_bf16(&p.tmU, a.U, 2, du, sz, bu, 128)) return -2;
+    if (k > 0) {
+      uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
+                        static_cast<uint64_t>(a.B)};
+      uint64_t sl[2] = {static_cast<uint64_t>(k) * 2,
+                        static_cast<uint64_t>(k) * 2 * static_cast<uint64_t>(a.T)};
+      uint32_t bl[3] = {64, 128, 1};
+      if (!encode_tmap_bf16(&p.tmL, a.L, 3, dl, sl, bl, 128)) return -2;
+      const int64_t Bk = a.B * k;
+      uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
+      uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
+      uint32_t bc[2] = {64, static_cast<uint32_t>(p.bn)};
+      if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
+    } else {
+      p.tmL = p.tmZ;
+      p.tmC = p.tmU;
+    }
+    uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
+    uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
+    uint32_t by[2] = {64, 128};
+    if (!encode_tmap_bf16(&p.tmY, a.Y, 2, dy, sy, by, 128)) return -2;
+    const int tiles = ceil_div(N, 128) * p.n_tiles_n;
+    const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
+                                                  false, a.status, dev);
+    if (!smem) return -3;
+    if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
+  }
+  return 0;
+}
+
+}  // namespace dyra

@@ -1,0 +1,228 @@
+// umma_gemm.cuh - persistent, warp-specialised tcgen05 GEMM skeleton.
+//
+// One CTA per SM (grid = min(tiles, SMs)), 192 threads:
+//   warp 0      TMA producer: fills a ring of `stages` shared-memory slots
+//   warp 1      MMA issuer: one elected thread issues tcgen05.mma (M = 128)
+//               into one of two TMEM accumulators, and owns the TMEM allocation
+//   warps 2..5  epilogue: tcgen05.ld the finished accumulator (warp w reads
+//               TMEM lanes 32*(w%4) .. +31, i.e. those rows of the tile) and
+//               hand the values to the policy's epilogue
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile
+// i+1. Every barrier wait is bounded (sm100::mbar_wait); on a timeout the CTA
+// raises its status word, drains the copies and MMAs it issued, frees TMEM and
+// returns.
+//
+// A policy `Pol` supplies:
+//   struct Params { GemmCommon c; ... };
+//   struct Tile { ... };
+//   static void decode(const Params&, int tile, Tile&);
+//   static int  kiters(const Params&, const Tile&);
+//   static void load(const Params&, const Tile&, int it, uint32_t sa, uint32_t sb, uint32_t bar);
+//   static int  ksteps(const Params&, const Tile&, int it);        // K16 MMAs in slot
+//   static uint64_t adesc(const Params&, uint32_t sa, int ks);
+//   static uint64_t bdesc(const Params&, uint32_t sb, int ks);
+//   static void epilogue(const Params&, const Tile&, uint32_t tacc, EpiCtx&);
+//   static void epilogue_drain(const Params&, EpiCtx&);
+//   static void prefetch(const Params&);
+//   static constexpr uint32_t kEpiSmemBytes;
+#pragma once
+
+#include "sm100.cuh"
+
+namespace dyra {
+
+constexpr int kGemmThreads = 192;
+constexpr int kMaxStages = 8;
+
+struct GemmCommon {
+  int num_tiles;
+  int stages;
+  uint32_t a_stage_bytes;
+  uint32_t b_stage_bytes;
+  uint32_t acc_cols;   // TMEM columns of one accumulator (>= MMA N)
+  uint32_t tmem_cols;  // allocated columns: power of two >= 2 * acc_cols, >= 32
+  uint32_t idesc;      // instruction descriptor (M = 128, N, majors)
+  int* status;         // device status word
+};
+
+struct EpiCtx {
+  int row;            // tile row owned by this thread, 0..127
+  int lane;           // lane in warp
+  int quad;           // TMEM lane quadrant of this warp
+  int tid;            // 0..127 among the epilogue threads
+  uint8_t* smem;      // policy scratch (kEpiSmemBytes), 1024-byte aligned
+  uint32_t smem_u32;  // same, as a shared-window address
+  uint32_t counter;   // running counter the policy may use (e.g. store buffers)
+};
+
+__host__ __device__ inline uint32_t gemm_smem_bytes(int stages, uint32_t a_bytes,
+                                                    uint32_t b_bytes, uint32_t epi_bytes) {
+  // 1024 alignment slack + stages + epilogue scratch + barriers/slots
+  return 1024u + static_cast<uint32_t>(stages) * (a_bytes + b_bytes) + epi_bytes + 256u;
+}
+
+template <class Pol>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ typename Pol::Params p) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  const GemmCommon& c = p.c;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw + pad;
+  const int S = c.stages;
+  const uint32_t sA = sbase;
+  const uint32_t sB = sA + static_cast<uint32_t>(S) * c.a_stage_bytes;
+  const uint32_t sEpi = sB + static_cast<uint32_t>(S) * c.b_stage_bytes;
+  const uint32_t sBar = sEpi + Pol::kEpiSmemBytes;
+  // barriers: full[S], empty[S], tfull[2], tempty[2], fin
+  auto full_bar = [&](int s) { return sBar + 8u * s; };
+  auto empty_bar = [&](int s) { return sBar + 8u * (kMaxStages + s); };
+  auto tfull_bar = [&](int i) { return sBar + 8u * (2 * kMaxStages + i); };
+  auto tempty_bar = [&](int i) { return sBar + 8u * (2 * kMaxStages + 2 + i); };
+  const uint32_t fin_bar = sBar + 8u * (2 * kMaxStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (sBar - sbase) + 8 * (2 * kMaxStages + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 4);
+    }
+    mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) Pol::prefetch(p);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), c.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Inputs written by the previous kernel in the stream are visible from here.
+  pdl_wait();
+
+  WaitCtx w{abort_flag, c.status};
+
+  if (warp == 0) {
+    if (elect_one_sync()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t last_phase[kMaxStages];
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < c.num_tiles; tile += gridDim.x) {
+        typename Pol::Tile t;
+        Pol::decode(p, tile, t);
+        const int nk = Pol::kiters(p, t);
+        for (int it = 0; it < nk; ++it) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, w)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), c.a_stage_bytes + c.b_stage_bytes);
+          Pol::load(p, t, it, sA + stage * c.a_stage_bytes, sB + stage * c.b_stage_bytes,
+                    full_bar(stage));
+          issued |= 1u << stage;
+          last_phase[stage] = phase;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every copy this thread issued has landed before the CTA leaves
+      // (one shared deadline for all slots).
+      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) (void)mbar_wait_until(full_bar(s), last_phase[s], deadline);
+    }
+  } else if (warp == 1) {
+    if (elect_one_sync()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int tile = blockIdx.x; tile < c.num_tiles; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, w)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc) * c.acc_cols;
+        typename Pol::Tile t;
+        Pol::decode(p, tile, t);
+        const int nk = Pol::kiters(p, t);
+        bool ok = true;
+        for (int it = 0; it < nk; ++it) {
+          if (!mbar_wait(full_bar(stage), phase, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = sA + stage * c.a_stage_bytes;
+          const uint32_t b = sB + stage * c.b_stage_bytes;
+          const int ks = Pol::ksteps(p, t, it);
+          for (int k = 0; k < ks; ++k)
+            mma_bf16(d, Pol::adesc(p, a, k), Pol::bdesc(p, b, k), c.idesc,
+                     (it > 0 || k > 0) ? 1u : 0u);
+          mma_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(acc));
+      }
+      // All MMAs issued by this thread are complete before TMEM is freed.
+      mma_commit(fin_bar);
+      (void)mbar_wait_until(fin_bar, 0, globaltimer_ns() + kWaitLimitNs);
+    }
+  } else {
+    EpiCtx e;
+    e.quad = warp & 3;
+    e.lane = lane;
+    e.row = e.quad * 32 + lane;
+    e.tid = threadIdx.x - 64;
+    e.smem = smem + (sEpi - sbase);
+    e.smem_u32 = sEpi;
+    e.counter = 0;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < c.num_tiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, w)) break;
+      tc_fence_after();
+      typename Pol::Tile t;
+      Pol::decode(p, tile, t);
+      const uint32_t tacc = tmem + static_cast<uint32_t>(acc) * c.acc_cols +
+                            (static_cast<uint32_t>(e.quad * 32) << 16);
+      Pol::epilogue(p, t, tacc, e);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+    Pol::epilogue_drain(p, e);
+  }
+
+  __syncthreads();
+  pdl_launch_dependents();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, c.tmem_cols);
+  }
+}
+
+}  // namespace dyra

@@ -1,0 +1,56 @@
+"""Offline preparation of a DyRA layer on the host (not on the hot path).
+
+"DyRA: Dynamic Residual Approximation for Efficient Matrix Multiplication in
+DNNs", Appendix A, Algorithm 1, procedure Offline Preparation, low-rank case
+(App. B): truncated SVD W ~ U V^T with the singular values on U, the residual
+W_res = W - U V^T, the fixed ALS start R0 = the top-k output-side singular
+vectors of W_res (App. D), and the projector P = W_res^T R0^T (R0 R0^T +
+lambda I)^-1 (Eq. 7 with the ridge of footnote 2). Computed in float64 with
+torch on the CPU; the result is what dyra_load_factors takes.
+"""
+
+from __future__ import annotations
+
+from typing import NamedTuple
+
+import torch
+
+
+class LayerFactors(NamedTuple):
+    U: torch.Tensor      # d_out x r
+    V: torch.Tensor      # d_in x r
+    P: torch.Tensor      # d_in x k
+    W_res: torch.Tensor  # d_out x d_in
+
+
+def _p_from_r0(W_res: torch.Tensor, R0: torch.Tensor, lam: float) -> torch.Tensor:
+    k = R0.shape[0]
+    gram = R0 @ R0.T + lam * torch.eye(k, dtype=torch.float64)
+    return torch.linalg.solve(gram, R0 @ W_res).T.contiguous()
+
+
+def prepare_from_weight(W, r: int, k: int, lam: float) -> LayerFactors:
+    """From a dense d_out x d_in weight (one SVD of W and one of W_res)."""
+    W = torch.as_tensor(W, dtype=torch.float64).cpu()
+    A, s, Bt = torch.linalg.svd(W, full_matrices=False)
+    U = (A[:, :r] * s[:r]).contiguous()
+    V = Bt[:r].T.contiguous()
+    W_res = W - U @ V.T
+    if k == 0:
+        return LayerFactors(U, V, torch.zeros(W.shape[1], 0, dtype=torch.float64), W_res)
+    Ar, _, _ = torch.linalg.svd(W_res, full_matrices=False)
+    return LayerFactors(U, V, _p_from_r0(W_res, Ar[:, :k].T, lam), W_res)
+
+
+def prepare_from_svd(left, sigma, right, r: int, k: int, lam: float) -> LayerFactors:
+    """From a weight given by its SVD W = left diag(sigma) right^T."""
+    left = torch.as_tensor(left, dtype=torch.float64).cpu()
+    sigma = torch.as_tensor(sigma, dtype=torch.float64).cpu()
+    right = torch.as_tensor(right, dtype=torch.float64).cpu()
+    U = (left[:, :r] * sigma[:r]).contiguous()
+    V = right[:, :r].contiguous()
+    W_res = (left[:, r:] * sigma[r:]) @ right[:, r:].T
+    if k == 0:
+        return LayerFactors(U, V, torch.zeros(right.shape[0], 0, dtype=torch.float64), W_res)
+    R0 = left[:, r:r + k].T
+    return LayerFactors(U, V, _p_from_r0(W_res, R0, lam), W_res)

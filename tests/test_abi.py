@@ -1,0 +1,95 @@
+"""The C ABI without a GPU: the library loads, exports what include/*.h
+declares, and rejects invalid arguments with status codes (no device call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from rank_structured_matmul_b200 import dyra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(dyra_[a-z_]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dyra.lib()
+    names = declared_functions()
+    assert {"dyra_plan_create", "dyra_load_factors", "dyra_forward", "dyra_plan_destroy"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), "libdyra.so does not export %s" % n
+    assert set(dyra.SIGNATURES) <= names
+
+
+def test_error_strings():
+    for code in range(0, -9, -1):
+        s = dyra.error_string(code)
+        assert s and s != "unknown error"
+    assert dyra.error_string(-99) == "unknown error"
+
+
+def _create(*args):
+    lib = dyra.lib()
+    h = ctypes.c_void_p()
+    rc = lib.dyra_plan_create(ctypes.byref(h), *args)
+    return rc, h
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 256, 32, 8, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),      # d_in < 1
+    ((256, -1, 32, 8, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),     # d_out < 1
+    ((256, 256, 0, 8, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),     # r < 1
+    ((256, 256, 32, -1, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),   # k < 0
+    ((256, 256, 32, 129, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),  # k > 128
+    ((64, 256, 60, 8, dyra.DYRA_F32), dyra.DYRA_ERR_INVALID_ARG),     # r + k > min(d_in, d_out)
+    ((256, 256, 32, 8, 7), dyra.DYRA_ERR_INVALID_ARG),                # bad dtype
+    ((260, 256, 32, 8, dyra.DYRA_BF16), dyra.DYRA_ERR_ALIGNMENT),     # d_in % 8
+    ((256, 252, 32, 8, dyra.DYRA_BF16), dyra.DYRA_ERR_ALIGNMENT),     # d_out % 8
+    ((256, 256, 30, 8, dyra.DYRA_BF16), dyra.DYRA_ERR_ALIGNMENT),     # r % 8
+    ((256, 256, 32, 12, dyra.DYRA_BF16), dyra.DYRA_ERR_ALIGNMENT),    # k % 8
+])
+def test_plan_create_rejects(args, code):
+    rc, h = _create(*args)
+    assert rc == code
+    assert h.value is None
+
+
+def test_null_handles():
+    lib = dyra.lib()
+    assert lib.dyra_plan_create(None, 256, 256, 32, 8, dyra.DYRA_F32) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_forward(None, None, None, 10, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_forward_batched(None, None, None, 2, 3, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_forward_weight_only(None, None, None, 1, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_load_factors(None, None, None, None, None, 0.0, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_reserve(None, 1, 1) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_last_status(None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_plan_destroy(None) == dyra.DYRA_OK
+    assert lib.dyra_plan_device_bytes(None) == 0
+
+
+def test_python_wrapper_raises():
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_plan_create(256, 256, 32, 12, dyra.DYRA_BF16)
+    assert e.value.code == dyra.DYRA_ERR_ALIGNMENT
+
+
+def test_plan_create_without_gpu_fails_cleanly():
+    """A valid shape needs a B200; on a machine without one the call returns
+    an error code (CUDA or UNSUPPORTED), never crashes."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc, h = _create(256, 256, 32, 8, dyra.DYRA_BF16)
+    assert rc in (dyra.DYRA_ERR_CUDA, dyra.DYRA_ERR_UNSUPPORTED)
+    assert h.value is None
