@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the DyRA approximated linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dyra|reference]
+
+One step is one DyRA forward (projection, Gram, solve, residual factor,
+output: every stage of Algorithm 1's inference procedure) over the workload's
+B x T rows, inputs resident in HBM. The L2 cache is flushed (256 MiB write)
+before every step, outside the step's CUDA events. Prints one JSON line.
+
+Under torchrun (N > 1) every rank runs its own replica of the workload on its
+own GPU (instances are independent; no collective on the data path); the
+step time is the maximum over ranks and `value` counts all ranks' work.
+
+--impl reference times the fp64 CPU oracle on the same workload instead (rank
+0 only); that arm is a deliberately slow baseline, not the target.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DyRA linear µs & dense-equiv TFLOP/s vs cuBLAS dense; % of roofline"
+UNIT = "TFLOP/s (dense-equivalent)"
+HEADLINE = "vit_fc1"
+STAGE_KERNELS = {"proj": "ProjPolicy", "gram": "GramPolicy", "solve": "solve_kernel",
+                 "rfactor": "RFactorPolicy", "out": "OutPolicy"}
+FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+         "source": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        m = json.load(open(path))
+        p.update({k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")
+                  if k in m})
+        p["source"] = "measured"
+    return p
+
+
+def csrc_digest() -> str:
+    """Hash of the kernel sources, to tell whether stored ncu counters are current."""
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "rank_structured_matmul_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(stage: str, workload: str):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    t = json.load(open(path)).get("%s:%s" % (stage, workload))
+    if not t or t.get("csrc_digest") != csrc_digest():
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ workload ----
+
+def workload_arrays(name: str):
+    from synth import generate, spec
+    s = spec(name)
+    w = generate(s)
+    return s, w
+
+
+def algorithmic(s):
+    """FLOPs and compulsory bytes of one forward and of its output stage."""
+    es = 2 if s.dtype == "bf16" else 4
+    N, di, do, r, k, B = s.N, s.d_in, s.d_out, s.r, s.k, s.B
+    flops = {
+        "proj": 2.0 * N * di * (r + k),
+        "gram": 2.0 * N * k * (di + k),
+        "solve": B * (k ** 3 / 3.0 + 2.0 * k * k * di),
+        "rfactor": 2.0 * B * k * di * do,
+        "out": 2.0 * N * do * (r + k),
+    }
+    bytes_ = {
+        "proj": es * (N * di + (r + k) * di + N * (r + k)),
+        "gram": es * (N * di + N * k) + 4.0 * B * k * (di + k),
+        "solve": 4.0 * B * k * (di + k) + es * B * k * di,
+        "rfactor": es * (do * di + B * k * di + do * B * k),
+        "out": es * (N * do + N * r + N * k + do * r + do * B * k),
+    }
+    layer_flops = sum(flops.values())
+    layer_bytes = es * (N * di + N * do + do * r + di * r + di * k + do * di)
+    return flops, bytes_, layer_flops, layer_bytes
+
+
+# -------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl)
+                          if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ dyra arm ----
+
+def run_dyra(args):
+    import torch
+    import torch.distributed as dist
+    from rank_structured_matmul_b200 import dyra, prep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    s, w = workload_arrays(args.workload)
+    f = prep.prepare_from_svd(w.left, w.sigma, w.right, s.r, s.k, s.lam)
+    td = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+    layer = dyra.DyraLinear(s.d_in, s.d_out, s.r, s.k, s.dtype)
+    layer.load(f.U, f.V, f.P, f.W_res, s.lam)
+    X = torch.from_numpy(w.X).to(dev, td)
+    Y = torch.empty(s.N, s.d_out, device=dev, dtype=td)
+    layer.reserve(s.B, s.T)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step():
+        layer.forward(X, B=s.B, T=s.T, Y=Y)
+
+    def timed(fn, K, W):
+        for _ in range(W):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # ---- the timed region: K steps, barrier + sync on both sides
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ms = timed(step, args.steps, 0)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    status = layer.status()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    dense_flops = 2.0 * s.N * s.d_in * s.d_out
+    value = dense_flops * world / (ms * 1e-3) / 1e12
+
+    # ---- cuBLAS dense X W^T of the same shape
+    Wd = torch.from_numpy(w.weight()).to(dev, td)
+    Yd = torch.empty_like(Y)
+    dense_ms = timed(lambda: torch.matmul(X, Wd.t(), out=Yd), args.steps, 3)
+
+    # ---- per-stage device time (events between the stage launches)
+    dyra.dyra_debug_set_stage_timing(layer.plan, True)
+    acc = {k: [] for k in dyra.STAGES}
+    for _ in range(max(5, args.steps)):
+        flush.zero_()
+        step()
+        for k2, v in dyra.dyra_debug_stage_times(layer.plan).items():
+            acc[k2].append(v)
+    dyra.dyra_debug_set_stage_timing(layer.plan, False)
+    stage_ms = {k2: float(np.mean(v)) for k2, v in acc.items()}
+
+    pk = peaks()
+    flops, bytes_, layer_flops, layer_bytes = algorithmic(s)
+    dom = max(stage_ms, key=stage_ms.get)
+    t_dom = stage_ms[dom] * 1e-3
+    tensor_t = flops[dom] / (pk["bf16_tflops"] * 1e12)
+    hbm_t = bytes_[dom] / (pk["hbm_gbs"] * 1e9)
+    if tensor_t >= hbm_t:
+        roof = {"bound": "tensor", "achieved": flops[dom] / t_dom / 1e12,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": bytes_[dom] / t_dom / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = stored_traffic(dom, args.workload)
+    roof["kernel"] = STAGE_KERNELS[dom]
+    roof["peak_source"] = pk["source"] + " burst"
+    layer_roof_us = max(layer_flops / (pk["bf16_tflops"] * 1e12),
+                        layer_bytes / (pk["hbm_gbs"] * 1e9)) * 1e6
+
+    # ---- end to end through the C ABI: pinned host X -> device, forward, Y -> pinned host
+    Xh = X.cpu().pin_memory()
+    Yh = torch.empty(Y.shape, dtype=td).pin_memory()
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        layer.forward(X, B=s.B, T=s.T, Y=Y)
+        Yh.copy_(Y, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, args.steps, 2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = dense_flops * world / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": s.dtype, "data": "synthetic (seeded; shapes and statistics "
+        "of the workload, random-orthogonal weights with a power-law spectrum)",
+        "config": {"workload": s.name, "d_in": s.d_in, "d_out": s.d_out, "r": s.r, "k": s.k,
+                   "instances": s.B, "rows_per_instance": s.T, "rows": s.N, "lambda": s.lam,
+                   "l2": "flushed before every step (256 MiB write, outside the step events)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "us_per_layer": ms * 1e3,
+        "cublas_dense_us": dense_ms * 1e3,
+        "speedup_vs_cublas_dense": dense_ms / ms,
+        "dyra_tflops_algorithmic": layer_flops / (ms * 1e-3) / 1e12,
+        "layer_roofline": {"us": layer_roof_us, "frac": layer_roof_us / (ms * 1e3),
+                           "flops": layer_flops, "bytes": layer_bytes},
+        "stage_us": {k2: v * 1e3 for k2, v in stage_ms.items()},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": X.numel() * X.element_size(),
+                "d2h_bytes_per_step": Y.numel() * Y.element_size(), "us": e2e_ms * 1e3},
+        "gpu_launches": (5 if s.k > 0 else 2) * args.steps,
+        "device_status": status,
+        "clocks": clk,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"], line["parity"] = cpu_baseline(s, w, Y)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- oracle ----
+
+def oracle_inputs(s, w):
+    import oracle
+    f = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, s.r, s.k, s.lam)
+    return f, [oracle.round_to(a, s.dtype) for a in (w.X, f.U, f.V, f.P, f.W_res)]
+
+
+def cpu_baseline(s, w, Y_gpu):
+    import oracle
+    f, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, w)
+    cores = len(os.sched_getaffinity(0))
+    # time the oracle on whole instances until ~10 s of work (at least one)
+    t0 = time.perf_counter()
+    Y1 = oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
+    t1 = time.perf_counter() - t0
+    n_inst = int(max(1, min(s.B, 10.0 // max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    Yo = oracle.inference(Xr[: n_inst * s.T], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+    t = time.perf_counter() - t0
+    flops = 2.0 * n_inst * s.T * s.d_in * s.d_out
+    base = {"value": flops / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "%d of %d instances (%d rows), fp64 NumPy, %.2f s" % (
+                n_inst, s.B, n_inst * s.T, t)}
+    Yg = Y_gpu[: n_inst * s.T].double().cpu().numpy()
+    W = w.weight()
+    rep = oracle.error_report(Xr[: n_inst * s.T], W, oracle.Factors(Ur, Vr, Pr, Wr, f.R0), s.lam,
+                              n_inst, s.T, Y=Yo)
+    parity = {"rel_fro_vs_oracle": oracle.rel_fro(Yg, Yo), "tol": 1e-2 if s.dtype == "bf16"
+              else 1e-5, "rows": n_inst * s.T, "oracle_err_weight_only": rep["err_wo"],
+              "oracle_err_dyra": rep["err_dyra"]}
+    return base, parity
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    s, w = workload_arrays(args.workload)
+    f, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, w)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
+    t1 = time.perf_counter() - t0
+    # each step a bounded sample: whole instances worth about 5 s at most
+    n_inst = int(max(1, min(s.B, 5.0 // max(t1, 1e-3))))
+    rows = n_inst * s.T
+    for _ in range(args.warmup):
+        oracle.inference(Xr[:rows], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.inference(Xr[:rows], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+        times.append(time.perf_counter() - t0)
+    t = float(np.mean(times))
+    value = 2.0 * rows * s.d_in * s.d_out / t / 1e12
+    sample = "%d of %d instances (%d rows) per step, fp64 NumPy" % (n_inst, s.B, rows)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": s.name, "d_in": s.d_in, "d_out": s.d_out, "r": s.r, "k": s.k,
+                       "instances": s.B, "rows_per_instance": s.T, "lambda": s.lam},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--impl", choices=("dyra", "reference"), default="dyra")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_dyra(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -43,6 +43,17 @@ int dyra_debug_copy(dyra_plan_t p, int which, void *dst, size_t bytes);
 /* Row splits S and rows per split used by the Gram stage for B x T. */
 int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int *splits, int *split_rows);
 
+/* Stage timing. When enabled, every forward records a CUDA event on its stream
+ * before each stage and after the last, which serialises the stages (no
+ * programmatic overlap between them). Stages of the bf16 path, in order:
+ *   0 proj (X [V|P]), 1 gram (L^T [X|L]), 2 solve, 3 rfactor (W_res T'^T), 4 out.
+ * Stages that did not run (k == 0) report 0. */
+int dyra_debug_set_stage_timing(dyra_plan_t p, int enable);
+
+/* Milliseconds of each of the 5 stages of the last forward (synchronises on
+ * its final event). Returns DYRA_ERR_INVALID_ARG if timing was not enabled. */
+int dyra_debug_stage_times(dyra_plan_t p, float *ms5);
+
 #ifdef __cplusplus
 }
 #endif

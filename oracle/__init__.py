@@ -10,6 +10,7 @@ from .dyra_oracle import (  # noqa: F401
     dense,
     error_report,
     inference,
+    inference_rows,
     offline_prepare,
     offline_prepare_from_svd,
     rel_fro,

@@ -152,6 +152,32 @@ def inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
     return Y
 
 
+def inference_rows(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
+                   W_res: np.ndarray, lam: float, B: int, T: int, rows) -> np.ndarray:
+    """Rows `rows` of inference(...), for layers too large to evaluate whole.
+
+    Each instance that owns a requested row is fitted on all of its T rows
+    exactly as in inference (Alg. 1 lines 11-12); lines 10 and 13 are then
+    evaluated for the requested rows only.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.int64)
+    k = P.shape[1]
+    out = np.empty((rows.size, U.shape[0]))
+    for b in np.unique(rows // T):
+        Xb = X[b * T:(b + 1) * T]
+        sel = np.nonzero(rows // T == b)[0]
+        xr = X[rows[sel]]
+        Yr = (xr @ V) @ U.T
+        if k > 0:
+            L = Xb @ P
+            G = L.T @ L + lam * np.eye(k)
+            C = np.linalg.solve(G, (L.T @ Xb) @ W_res.T)
+            Yr = Yr + (xr @ P) @ C
+        out[sel] = Yr
+    return out
+
+
 def rel_fro(A: np.ndarray, ref: np.ndarray) -> float:
     """Relative Frobenius error ||A - ref||_F / ||ref||_F ([DyRA] App. E.4)."""
     den = np.linalg.norm(ref)

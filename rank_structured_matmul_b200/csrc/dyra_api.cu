@@ -36,6 +36,9 @@ struct dyra_plan {
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
+  cudaEvent_t stage_ev[6] = {};
+  bool stage_timing = false;
+  bool stage_recorded = false;
 };
 
 namespace {
@@ -169,7 +172,9 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.split_rows = 64;
     if (correct) dyra::gram_split(T, B, p->dev.sm_count, &a.splits, &a.split_rows);
     a.status = p->status;
+    a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
+    p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
     a.d_in = p->d_in;
@@ -417,6 +422,8 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->Ct);
     void* st = p->status;
     dev_free(st);
+    for (auto& e : p->stage_ev)
+      if (e) cudaEventDestroy(e);
   }
   delete p;
   return DYRA_OK;
@@ -446,6 +453,33 @@ int dyra_debug_copy(dyra_plan_t p, int which, void* dst, size_t bytes) {
   if (cudaDeviceSynchronize() != cudaSuccess) return DYRA_ERR_CUDA;
   return cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? DYRA_OK
                                                                             : DYRA_ERR_CUDA;
+}
+
+int dyra_debug_set_stage_timing(dyra_plan_t p, int enable) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (enable && !p->stage_ev[0]) {
+    for (auto& e : p->stage_ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return DYRA_ERR_CUDA;
+  }
+  p->stage_timing = enable != 0 && p->dtype == DYRA_BF16 && !p->force_simt;
+  p->stage_recorded = false;
+  return p->stage_timing || !enable ? DYRA_OK : DYRA_ERR_INVALID_ARG;
+}
+
+int dyra_debug_stage_times(dyra_plan_t p, float* ms5) {
+  if (p == nullptr || ms5 == nullptr || !p->stage_recorded) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (cudaEventSynchronize(p->stage_ev[5]) != cudaSuccess) return DYRA_ERR_CUDA;
+  for (int i = 0; i < 5; ++i) {
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p->stage_ev[i], p->stage_ev[i + 1]) != cudaSuccess)
+      return DYRA_ERR_CUDA;
+    ms5[i] = ms;
+  }
+  return DYRA_OK;
 }
 
 int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int* split_rows) {

@@ -43,6 +43,7 @@ struct Bf16Forward {
   int splits;            // row splits of the Gram reduction
   int split_rows;        // rows per split (multiple of 64)
   int* status;
+  cudaEvent_t* stage_events;  // optional: 6 events recorded around the 5 stages
 };
 
 // Rows per split and split count used for a given T (shared with the

@@ -468,6 +468,10 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   const int k = a.weight_only ? 0 : a.k;
   const int rk = a.r + a.k;  // VPt rows always hold [V | P]
   const bool pdl = true;
+  auto mark = [&](int i) {
+    if (a.stage_events) cudaEventRecord(a.stage_events[i], s);
+  };
+  mark(0);
 
   // ---------------------------------------------------------------- proj
   {
@@ -494,6 +498,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     if (!smem) return -3;
     if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
   }
+  mark(1);
 
   if (k > 0) {
     const int J = a.d_in + a.k;
@@ -534,10 +539,12 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       if (!smem) return -3;
       if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl)) return -1;
     }
+    mark(2);
     // ------------------------------------------------------------- solve
     if (launch_solve<__nv_bfloat16>(a.TG, a.splits, a.B, a.k, a.d_in, a.lambda,
                                     static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl))
       return -1;
+    mark(3);
     // ----------------------------------------------------------- rfactor
     {
       RFactorPolicy::Params p;
@@ -561,7 +568,11 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       if (!smem) return -3;
       if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
     }
+  } else {
+    mark(2);
+    mark(3);
   }
+  mark(4);
 
   // ------------------------------------------------------------------ out
   {
@@ -609,6 +620,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     if (!smem) return -3;
     if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
   }
+  mark(5);
   return 0;
 }
 

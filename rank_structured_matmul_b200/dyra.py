@@ -47,7 +47,11 @@ SIGNATURES = {
     "dyra_debug_buffer": (_i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_size_t)]),
     "dyra_debug_copy": (_i, [_vp, _i, _vp, ctypes.c_size_t]),
     "dyra_debug_gram_split": (_i, [_vp, _i64, _i64, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "dyra_debug_set_stage_timing": (_i, [_vp, _i]),
+    "dyra_debug_stage_times": (_i, [_vp, ctypes.POINTER(ctypes.c_float)]),
 }
+
+STAGES = ("proj", "gram", "solve", "rfactor", "out")
 
 DYRA_BUF_Z, DYRA_BUF_L, DYRA_BUF_TG, DYRA_BUF_TP, DYRA_BUF_CT = range(5)
 
@@ -159,6 +163,18 @@ def dyra_debug_gram_split(plan: int, B: int, T: int):
     _check(lib().dyra_debug_gram_split(plan, B, T, ctypes.byref(s), ctypes.byref(r)),
            "dyra_debug_gram_split")
     return s.value, r.value
+
+
+def dyra_debug_set_stage_timing(plan: int, enable: bool) -> None:
+    _check(lib().dyra_debug_set_stage_timing(plan, int(bool(enable))),
+           "dyra_debug_set_stage_timing")
+
+
+def dyra_debug_stage_times(plan: int):
+    """{stage: milliseconds} of the last forward with stage timing enabled."""
+    ms = (ctypes.c_float * 5)()
+    _check(lib().dyra_debug_stage_times(plan, ms), "dyra_debug_stage_times")
+    return dict(zip(STAGES, list(ms)))
 
 
 # ---- convenience object ----

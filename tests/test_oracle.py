@@ -233,6 +233,16 @@ def test_hand_worked_example():
     np.testing.assert_allclose(orc.dense(X, W), yd, atol=0)
 
 
+def test_inference_rows_matches_full():
+    """Row sampling evaluates the same per-instance fit as the whole-matrix path."""
+    w = small_layer(B=4, T=6)
+    f = factors(w, 4, 3, 1e-3)
+    full = orc.inference(w.X, f.U, f.V, f.P, f.W_res, 1e-3, 4, 6)
+    rows = np.array([23, 0, 5, 6, 17, 11])
+    got = orc.inference_rows(w.X, f.U, f.V, f.P, f.W_res, 1e-3, 4, 6, rows)
+    np.testing.assert_allclose(got, full[rows], rtol=0, atol=1e-13)
+
+
 def test_error_report_orders():
     w = small_layer(B=2, T=12)
     f = factors(w, 4, 3, 1e-3)

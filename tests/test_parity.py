@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA DyRA forward (through the C ABI) against the fp64 oracle.
+
+Both sides receive the same seeded inputs, rounded once to the plan's storage
+type. Tolerances are the layer's bar: relative Frobenius error <= 1e-5 for
+fp32 plans and <= 1e-2 for bf16 plans (fp32 accumulation). Full-size layers
+whose oracle output is too large are compared on sampled rows (the oracle
+still fits each sampled instance on all of its rows), always including the
+first and last row of every instance and the rows around tile boundaries.
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from rank_structured_matmul_b200 import dyra
+from synth import CONFIGS, LayerSpec, generate
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 1e-2, "f32": 1e-5}
+ROW_TOL = 5e-2  # any single row: ||dy|| / rms row norm
+_CACHE = {}
+
+
+def prepared(s: LayerSpec):
+    """Workload + oracle factors, rounded to the storage type (cached per layer)."""
+    key = (s.d_in, s.d_out, s.r, s.k, s.p, s.x_kind, s.n_outlier, s.outlier_scale, s.seed,
+           s.lam, s.dtype, s.n_draw if s.n_draw else s.N)
+    if key not in _CACHE:
+        n_draw = s.n_draw if s.n_draw else s.N
+        w = generate(s.with_rows(1, n_draw))  # the whole draw; prefixes are sliced below
+        f = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, s.r, s.k, s.lam)
+        r = {n: oracle.round_to(a, s.dtype) for n, a in
+             (("X", w.X), ("U", f.U), ("V", f.V), ("P", f.P), ("W_res", f.W_res))}
+        _CACHE.clear()
+        _CACHE[key] = r
+    r = _CACHE[key]
+    return dict(r, X=r["X"][: s.N])
+
+
+def to_dev(a, dtype):
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return torch.from_numpy(np.ascontiguousarray(a)).to("cuda", td)
+
+
+def make_layer(s: LayerSpec, f, kernels="umma"):
+    os.environ["DYRA_KERNELS"] = kernels
+    try:
+        layer = dyra.DyraLinear(s.d_in, s.d_out, s.r, s.k, s.dtype)
+    finally:
+        os.environ.pop("DYRA_KERNELS", None)
+    layer.load(to_dev(f["U"], s.dtype), to_dev(f["V"], s.dtype),
+               to_dev(f["P"], s.dtype) if s.k else None,
+               to_dev(f["W_res"], s.dtype) if s.k else None, s.lam)
+    return layer
+
+
+def sample_rows(s: LayerSpec, n=384, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(s.N, size=min(n, s.N), replace=False).tolist())
+    for b in range(s.B):
+        rows |= {b * s.T, b * s.T + s.T - 1}
+    for m in range(128, s.N, 128 * 7):
+        rows |= {m - 1, m}
+    return np.array(sorted(r for r in rows if r < s.N))
+
+
+def check(s: LayerSpec, Y: torch.Tensor, f, full=None):
+    Yg = Y.double().cpu().numpy()
+    if full is None:
+        full = s.N * s.d_out <= 60_000_000
+    if full:
+        rows = np.arange(s.N)
+        Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, s.B, s.T)
+    else:
+        rows = sample_rows(s)
+        Yo = oracle.inference_rows(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, s.B, s.T,
+                                   rows)
+    Yg = Yg[rows]
+    err = oracle.rel_fro(Yg, Yo)
+    rms = np.sqrt(np.mean(np.sum(Yo ** 2, axis=1))) + 1e-300
+    worst_row = float(np.max(np.linalg.norm(Yg - Yo, axis=1)) / rms)
+    assert np.all(np.isfinite(Yg))
+    assert err <= TOL[s.dtype], "%s: rel Frobenius %.3e > %.0e" % (s.name, err, TOL[s.dtype])
+    assert worst_row <= ROW_TOL * (1 if s.dtype == "bf16" else 1e-3), \
+        "%s: worst row %.3e" % (s.name, worst_row)
+    return err
+
+
+def run_spec(s: LayerSpec, kernels="umma"):
+    f = prepared(s)
+    layer = make_layer(s, f, kernels)
+    X = to_dev(f["X"], s.dtype)
+    Y = layer.forward(X, B=s.B, T=s.T)
+    assert layer.status() == 0
+    err = check(s, Y, f)
+    layer.close()
+    return err
+
+
+# ------------------------------------------------------- the workloads ----
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_config_parity(name):
+    """Every configuration at full size, in the launch configuration the
+    benchmark times (one dyra_forward_batched of B x T rows)."""
+    run_spec(CONFIGS[name])
+
+
+# ------------------------------------------------------------ edge cases ----
+
+EDGE = [
+    # name, d_in, d_out, r, k, B, T, lam
+    ("ragged_tiles", 256, 512, 64, 32, 3, 201, 1e-3),      # N = 603, instances straddle tiles
+    ("many_small_instances", 256, 256, 64, 16, 40, 5, 1e-3),  # 26 instances per 128-row tile
+    ("one_row_instances", 128, 192, 32, 8, 300, 1, 1e-3),   # T = 1, k > T
+    ("single_row", 256, 512, 64, 32, 1, 1, 1e-3),           # N = 1
+    ("odd_sizes", 200, 328, 40, 8, 5, 37, 1e-3),            # d_in, d_out, r off the 64 grid
+    ("k72_two_chunks", 256, 512, 64, 72, 2, 300, 1e-3),     # k > 64
+    ("k128_max", 512, 384, 128, 128, 2, 260, 1e-3),         # largest supported k
+    ("row_splits", 256, 256, 64, 32, 1, 3000, 1e-3),        # Gram reduced over row splits
+    ("lambda_zero", 256, 512, 64, 32, 2, 150, 0.0),         # plain ALS normal equations
+    ("k_below_rows_lam", 256, 512, 64, 64, 4, 20, 1e-3),    # T < k, ridge keeps G SPD
+    ("tall_out", 64, 2048, 16, 16, 2, 100, 1e-3),
+    ("wide_in", 2048, 64, 16, 16, 2, 100, 1e-3),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_shapes(case):
+    name, d_in, d_out, r, k, B, T, lam = case
+    run_spec(LayerSpec(name, d_in, d_out, r, k, B, T, "bf16", 0.7, "lognormal", seed=1, lam=lam))
+
+
+def test_fp32_batched():
+    run_spec(LayerSpec("f32_batched", 96, 80, 12, 8, 3, 50, "f32", 0.9, "outlier", n_outlier=3,
+                       outlier_scale=20.0, seed=2))
+
+
+def test_simt_variant_bf16():
+    """DYRA_KERNELS=simt runs the bf16 plan on the CUDA-core kernels (a
+    debugging variant); it meets the same bar."""
+    run_spec(LayerSpec("simt", 256, 512, 64, 32, 3, 201, "bf16", 0.7, "lognormal", seed=1),
+             kernels="simt")
+
+
+# ----------------------------------------------------------- properties ----
+
+def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
+    s = LayerSpec("p", 256, 512, 64, k, B, T, dtype, 0.7, "lognormal", seed=4, lam=lam)
+    return s, prepared(s)
+
+
+def test_weight_only_k0_plan_matches_oracle_and_weight_only_entry():
+    s0, f0 = _small(k=0)
+    layer0 = make_layer(s0, f0)
+    X = to_dev(f0["X"], "bf16")
+    Y0 = layer0.forward(X, B=s0.B, T=s0.T)
+    Ywo = oracle.weight_only(f0["X"], f0["U"], f0["V"])
+    assert oracle.rel_fro(Y0.double().cpu().numpy(), Ywo) <= 1e-2
+    s, f = _small(k=32)
+    layer = make_layer(s, f)
+    Y1 = layer.forward_weight_only(X)
+    assert torch.equal(Y0, Y1)
+    layer.close()
+    layer0.close()
+
+
+def test_forward_is_batched_with_one_instance_and_deterministic():
+    s, f = _small(B=1, T=603)
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    Y1 = torch.empty(603, 512, device="cuda", dtype=torch.bfloat16)
+    Y2 = torch.empty_like(Y1)
+    Y3 = torch.empty_like(Y1)
+    dyra.dyra_forward(layer.plan, X, Y1, 603)
+    dyra.dyra_forward_batched(layer.plan, X, Y2, 1, 603)
+    dyra.dyra_forward(layer.plan, X, Y3, 603)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(Y1, Y3)
+    layer.close()
+
+
+def test_side_stream():
+    s, f = _small()
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    Y1 = layer.forward(X, B=s.B, T=s.T)
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        Y2 = layer.forward(X, B=s.B, T=s.T, stream=st)
+    st.synchronize()
+    assert torch.equal(Y1, Y2)
+    layer.close()
+
+
+def test_rank_deficient_is_an_error():
+    s, f = _small(k=32, lam=0.0, B=2, T=20)
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    with pytest.raises(dyra.DyraError) as e:
+        layer.forward(X, B=2, T=20)
+    assert e.value.code == dyra.DYRA_ERR_RANK_DEFICIENT
+    layer.close()
+
+
+def test_zero_input_without_ridge_flags_pivot():
+    """X_b = 0 and lambda = 0 make L^T L = 0: the solve flags the pivot and
+    drops that instance's correction, leaving the weight-only output (0)."""
+    s, f = _small(k=32, lam=0.0, B=2, T=64)
+    layer = make_layer(s, f)
+    X = torch.zeros(128, 256, device="cuda", dtype=torch.bfloat16)
+    Y = layer.forward(X, B=2, T=64)
+    st = layer.status()
+    assert st & dyra.DYRA_STATUS_NONPOSITIVE_PIVOT
+    assert torch.count_nonzero(Y).item() == 0
+    assert layer.status() == 0  # cleared by the read
+    layer.close()
+
+
+def test_not_loaded_and_misaligned():
+    plan = dyra.dyra_plan_create(256, 512, 64, 32, dyra.DYRA_BF16)
+    X = torch.zeros(64, 256, device="cuda", dtype=torch.bfloat16)
+    Y = torch.zeros(64, 512, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_forward(plan, X, Y, 64)
+    assert e.value.code == dyra.DYRA_ERR_NOT_LOADED
+    s, f = _small()
+    U, V, P, W = (to_dev(f[n], "bf16") for n in ("U", "V", "P", "W_res"))
+    dyra.dyra_load_factors(plan, U, V, P, W, 1e-3)
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_forward(plan, X.data_ptr() + 2, Y, 63)
+    assert e.value.code == dyra.DYRA_ERR_ALIGNMENT
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_load_factors(plan, U, V, P, W, -1.0)
+    assert e.value.code == dyra.DYRA_ERR_INVALID_ARG
+    dyra.dyra_forward(plan, X, Y, 0)  # empty input is a no-op
+    dyra.dyra_plan_destroy(plan)
+
+
+def test_allocation_failure_is_reported():
+    os.environ["DYRA_TEST_FAIL_ALLOC"] = "1"
+    try:
+        with pytest.raises(dyra.DyraError) as e:
+            dyra.dyra_plan_create(256, 512, 64, 32, dyra.DYRA_BF16)
+        assert e.value.code == dyra.DYRA_ERR_ALLOC
+    finally:
+        os.environ.pop("DYRA_TEST_FAIL_ALLOC")
