@@ -121,6 +121,40 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
                              dyra_stream_t stream);
 
 /*
+ * dyra_forward_batched without any device allocation. (No counterpart in the
+ * paper: this is a deployment convenience of this library.)
+ *
+ * Who needs it: callers that must not call cudaMalloc while serving, e.g.
+ * code that runs under a memory manager owning every byte of the device,
+ * real-time loops where an allocation's implicit synchronisation or its
+ * failure mid-run is not acceptable, or embedders that forbid the library
+ * from allocating once set-up is over. Instead of the plan's workspace, this
+ * call keeps the intermediates (X V, X P, the Gram partial sums, the solved
+ * factor and C) in one fixed array of DYRA_STATIC_SCRATCH_BYTES (16 MiB)
+ * compiled into the library; every GPU that loads that part of the library
+ * holds the array until the process exits.
+ *   - Arguments, layouts and results are those of dyra_forward_batched; the
+ *     plan (created and loaded beforehand) supplies the factors.
+ *   - If the intermediates of B x T rows do not fit in the array the call
+ *     returns DYRA_ERR_INVALID_ARG and enqueues nothing. For a bf16 plan they
+ *     take about 2*B*T*(r+k) + 4*S*B*k*(d_in+k) + 2*B*k*(d_in+d_out) bytes,
+ *     each part rounded up to 256, where S is the number of row splits of the
+ *     Gram stage (dyra_debug_gram_split in dyra_debug.h reports it).
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress); make that first call before capturing a stream
+ *     into a CUDA graph.
+ *   - All calls share the one array and it keeps whatever the last call left
+ *     there. Nothing in it has to start at zero: every stage overwrites what
+ *     the next stage reads. Calls whose execution overlaps on the GPU (other
+ *     streams, other host threads, other plans) race on the array and give
+ *     wrong results; serialise them.
+ */
+int dyra_forward_batched_noalloc(dyra_plan_t p, const void *X, void *Y, int64_t B, int64_t T,
+                                 dyra_stream_t stream);
+
+#define DYRA_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
  * Grow the plan's workspace for up to B instances of T rows, so that later
  * forwards of that size allocate nothing (call it before capturing a CUDA
  * graph or timing). Forward calls grow the workspace themselves otherwise.

@@ -500,3 +500,180 @@ size_t dyra_plan_device_bytes(dyra_plan_t p) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free forward ----
+// The intermediates of dyra_forward_batched_noalloc live in this array
+// instead of the plan's workspace. It is allocated when this file's device
+// code is loaded on a device and stays there until the process exits.
+static __device__ __align__(256) unsigned char dyra_static_scratch[DYRA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of dyra_static_scratch on `device` (which is current),
+// looked up once per device. Host code cannot use the array's name as a
+// device pointer; only this address may be handed to kernels.
+int static_scratch_address(int device, unsigned char** out) {
+  if (device < 0 || device >= kMaxScratchDevices) return DYRA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[device] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, dyra_static_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return DYRA_ERR_CUDA;
+    }
+    g_scratch_addr[device] = ptr;
+  }
+  *out = static_cast<unsigned char*>(g_scratch_addr[device]);
+  return DYRA_OK;
+}
+
+// Carves consecutive 256-byte-aligned pieces out of the fixed array.
+struct ScratchCarver {
+  unsigned char* base;
+  size_t used = 0;
+  bool fits = true;
+  void* take(size_t bytes) {
+    const size_t at = used;
+    used += (bytes + 255) & ~static_cast<size_t>(255);
+    if (used > DYRA_STATIC_SCRATCH_BYTES) fits = false;
+    return base ? base + at : nullptr;
+  }
+};
+
+}  // namespace
+
+extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* Y, int64_t B,
+                                            int64_t T, dyra_stream_t stream) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (B < 0 || T < 0) return DYRA_ERR_INVALID_ARG;
+  const int64_t N = B * T;
+  if (N == 0) return DYRA_OK;
+  if (X == nullptr || Y == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (N > (static_cast<int64_t>(1) << 31) - 1 || B * static_cast<int64_t>(p->k) > (1 << 30))
+    return DYRA_ERR_INVALID_ARG;
+  if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  if (!aligned16(X) || !aligned16(Y)) return DYRA_ERR_ALIGNMENT;
+  const int k = p->k;
+  if (k > 0 && p->lambda == 0.f && T < k) return DYRA_ERR_RANK_DEFICIENT;
+
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
+  const size_t es = elem_size(p->dtype);
+  int splits = 1, split_rows = 64;
+  if (umma && k > 0) dyra::gram_split(T, B, p->dev.sm_count, &splits, &split_rows);
+
+  // Size check first, without touching the device.
+  ScratchCarver sizing{nullptr};
+  if (umma) {
+    sizing.take(static_cast<size_t>(N) * p->r * es);
+    if (k > 0) {
+      sizing.take(static_cast<size_t>(N) * k * es);
+      sizing.take(static_cast<size_t>(splits) * B * k * (p->d_in + k) * sizeof(float));
+      sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
+      sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+    }
+  } else {
+    sizing.take(static_cast<size_t>(N) * (p->r + k) * es);
+    if (k > 0) {
+      sizing.take(static_cast<size_t>(B) * k * (p->d_in + k) * sizeof(float));
+      sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
+      sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+    }
+  }
+  if (!sizing.fits) return DYRA_ERR_INVALID_ARG;
+
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  unsigned char* base = nullptr;
+  int rc = static_scratch_address(p->dev.device, &base);
+  if (rc) return rc;
+  ScratchCarver carve{base};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (umma) {
+    dyra::Bf16Forward a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = k;
+    a.B = B;
+    a.T = T;
+    a.X = X;
+    a.Y = Y;
+    a.VPt = p->VPt;
+    a.U = p->U;
+    a.W_res = p->W_res;
+    a.lambda = p->lambda;
+    a.weight_only = k == 0;
+    a.Z = carve.take(static_cast<size_t>(N) * p->r * es);
+    a.L = k > 0 ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
+    a.TG = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(splits) * B * k *
+                                                  (p->d_in + k) * sizeof(float)))
+                 : nullptr;
+    a.Tp = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_in * es) : nullptr;
+    a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
+    a.splits = splits;
+    a.split_rows = split_rows;
+    a.status = p->status;
+    a.stage_events = nullptr;
+    rc = dyra::launch_bf16_forward(a, p->dev, s);
+  } else if (p->dtype == DYRA_BF16) {
+    dyra::SimtForward<__nv_bfloat16> a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = k;
+    a.B = B;
+    a.Trows = T;
+    a.X = static_cast<const __nv_bfloat16*>(X);
+    a.Y = static_cast<__nv_bfloat16*>(Y);
+    a.VPt = static_cast<const __nv_bfloat16*>(p->VPt);
+    a.U = static_cast<const __nv_bfloat16*>(p->U);
+    a.W_res = static_cast<const __nv_bfloat16*>(p->W_res);
+    a.lambda = p->lambda;
+    a.weight_only = k == 0;
+    a.ZL = static_cast<__nv_bfloat16*>(carve.take(static_cast<size_t>(N) * (p->r + k) * es));
+    a.TG = k > 0 ? static_cast<float*>(
+                       carve.take(static_cast<size_t>(B) * k * (p->d_in + k) * sizeof(float)))
+                 : nullptr;
+    a.Tp = k > 0 ? static_cast<__nv_bfloat16*>(carve.take(static_cast<size_t>(B) * k * p->d_in * es))
+                 : nullptr;
+    a.Cm = k > 0 ? static_cast<__nv_bfloat16*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
+                 : nullptr;
+    a.status = p->status;
+    rc = dyra::launch_simt_forward(a, p->dev, s);
+  } else {
+    dyra::SimtForward<float> a;
+    a.d_in = p->d_in;
+    a.d_out = p->d_out;
+    a.r = p->r;
+    a.k = k;
+    a.B = B;
+    a.Trows = T;
+    a.X = static_cast<const float*>(X);
+    a.Y = static_cast<float*>(Y);
+    a.VPt = static_cast<const float*>(p->VPt);
+    a.U = static_cast<const float*>(p->U);
+    a.W_res = static_cast<const float*>(p->W_res);
+    a.lambda = p->lambda;
+    a.weight_only = k == 0;
+    a.ZL = static_cast<float*>(carve.take(static_cast<size_t>(N) * (p->r + k) * es));
+    a.TG = k > 0 ? static_cast<float*>(
+                       carve.take(static_cast<size_t>(B) * k * (p->d_in + k) * sizeof(float)))
+                 : nullptr;
+    a.Tp = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(B) * k * p->d_in * es))
+                 : nullptr;
+    a.Cm = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
+                 : nullptr;
+    a.status = p->status;
+    rc = dyra::launch_simt_forward(a, p->dev, s);
+  }
+  if (rc != 0) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  return DYRA_OK;
+}

@@ -39,6 +39,7 @@ SIGNATURES = {
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
+    "dyra_forward_batched_noalloc": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_reserve": (_i, [_vp, _i64, _i64]),
     "dyra_last_status": (_i, [_vp]),
     "dyra_plan_destroy": (_i, [_vp]),
@@ -133,6 +134,13 @@ def dyra_forward_batched(plan: int, X, Y, B: int, T: int, stream=None) -> None:
 def dyra_forward_weight_only(plan: int, X, Y, N: int, stream=None) -> None:
     _check(lib().dyra_forward_weight_only(plan, _ptr(X), _ptr(Y), int(N), _stream(stream)),
            "dyra_forward_weight_only")
+
+
+def dyra_forward_batched_noalloc(plan: int, X, Y, B: int, T: int, stream=None) -> None:
+    """dyra_forward_batched with the intermediates in the library's fixed
+    device array instead of plan workspace; no device allocation."""
+    _check(lib().dyra_forward_batched_noalloc(plan, _ptr(X), _ptr(Y), int(B), int(T),
+                                              _stream(stream)), "dyra_forward_batched_noalloc")
 
 
 def dyra_reserve(plan: int, B: int, T: int) -> None:
