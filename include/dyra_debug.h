@@ -54,6 +54,19 @@ int dyra_debug_set_stage_timing(dyra_plan_t p, int enable);
  * its final event). Returns DYRA_ERR_INVALID_ARG if timing was not enabled. */
 int dyra_debug_stage_times(dyra_plan_t p, float *ms5);
 
+/* Kernel timelines. When enabled, each CTA of the four tensor-core stages of
+ * a bf16 forward (proj, gram, rfactor, out) writes %globaltimer nanosecond
+ * stamps at fixed milestones into a plan-owned buffer laid out as
+ * [stage 0..4][CTA 0..255][slot 0..31] (uint64; stage 2, the solve, stays 0):
+ *   0 entry, 1 set-up done, 2 inputs of the previous stage visible,
+ *   3 first copy issued, 4 last copy issued, 5 first operands arrived,
+ *   6 last accumulator committed, 7 first accumulator reached the epilogue,
+ *   8 exit, 9 + i epilogue of the CTA's i-th tile done.
+ * A slot a CTA did not reach stays 0. Disabling frees the buffer. */
+int dyra_debug_set_trace(dyra_plan_t p, int enable);
+size_t dyra_debug_trace_bytes(void);
+int dyra_debug_trace_copy(dyra_plan_t p, void *dst, size_t bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,22 @@ struct dyra_plan {
   cudaEvent_t stage_ev[6] = {};
   bool stage_timing = false;
   bool stage_recorded = false;
+  unsigned long long* trace = nullptr;  // timeline buffer (diagnostics)
+  // Captured forwards (CUDA graphs) keyed by their arguments; replayed with
+  // one cudaGraphLaunch. Invalidated when workspace or factors change.
+  struct GraphEntry {
+    const void* X = nullptr;
+    void* Y = nullptr;
+    int64_t B = 0, T = 0;
+    bool weight_only = false;
+    cudaGraphExec_t exec = nullptr;
+    uint64_t used = 0;
+  };
+  static constexpr int kGraphSlots = 8;
+  GraphEntry graphs[kGraphSlots];
+  uint64_t graph_clock = 0;
+  cudaStream_t capture_stream = nullptr;
+  bool use_graphs = true;
 };
 
 namespace {
@@ -79,6 +95,13 @@ int grow(void*& p, size_t& cap, size_t bytes) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+void drop_graphs(dyra_plan* p) {
+  for (auto& g : p->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g = dyra_plan::GraphEntry();
+  }
+}
+
 // Run on the plan's device, restoring the caller's device afterwards.
 struct DeviceGuard {
   int prev = -1;
@@ -96,7 +119,22 @@ struct DeviceGuard {
   }
 };
 
+int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
+
+// Grows the workspace; captured graphs point at the old buffers, so any
+// growth drops them.
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
+  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct;
+  const void* ptrs[5] = {p->Z, p->L, p->TG, p->Tp, p->Ct};
+  const int rc = ensure_workspace_impl(p, B, T);
+  const void* now[5] = {p->Z, p->L, p->TG, p->Tp, p->Ct};
+  bool moved = before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct;
+  for (int i = 0; i < 5; ++i) moved = moved || ptrs[i] != now[i];
+  if (moved) drop_graphs(p);
+  return rc;
+}
+
+int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   const int64_t N = B * T;
   const size_t es = elem_size(p->dtype);
   const int k = p->k;
@@ -105,7 +143,7 @@ int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
     if (k > 0) {
       int splits = 1, rows = 64;
-      dyra::gram_split(T, B, p->dev.sm_count, &splits, &rows);
+      dyra::gram_split(T, B, p->d_in, k, p->dev.sm_count, &splits, &rows);
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
       void* tg = p->TG;
       rc = grow(tg, p->cap_TG,
@@ -127,6 +165,63 @@ int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
     }
   }
   return DYRA_OK;
+}
+
+// Launch the bf16 forward, through a cached CUDA graph when possible: one
+// cudaGraphLaunch replaces five kernel launches and twelve tensor-map
+// encodings. Graphs are not used while the caller's stream is being captured
+// (the launches then go into the caller's graph), with stage timing or
+// tracing on, or when DYRA_GRAPHS=0.
+int launch_bf16_maybe_graph(dyra_plan* p, const dyra::Bf16Forward& a, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (!p->use_graphs || a.stage_events || a.trace ||
+      cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return dyra::launch_bf16_forward(a, p->dev, s);
+  }
+  dyra_plan::GraphEntry* hit = nullptr;
+  for (auto& g : p->graphs)
+    if (g.exec && g.X == a.X && g.Y == a.Y && g.B == a.B && g.T == a.T &&
+        g.weight_only == a.weight_only)
+      hit = &g;
+  if (!hit) {
+    if (!p->capture_stream &&
+        cudaStreamCreateWithFlags(&p->capture_stream, cudaStreamNonBlocking) != cudaSuccess)
+      return dyra::launch_bf16_forward(a, p->dev, s);
+    cudaGraph_t graph = nullptr;
+    if (cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return dyra::launch_bf16_forward(a, p->dev, s);
+    }
+    const int lrc = dyra::launch_bf16_forward(a, p->dev, p->capture_stream);
+    const cudaError_t ec = cudaStreamEndCapture(p->capture_stream, &graph);
+    cudaGraphExec_t exec = nullptr;
+    if (lrc != 0 || ec != cudaSuccess || graph == nullptr ||
+        cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      cudaGetLastError();
+      return dyra::launch_bf16_forward(a, p->dev, s);
+    }
+    cudaGraphDestroy(graph);
+    hit = &p->graphs[0];
+    for (auto& g : p->graphs) {
+      if (!g.exec) {
+        hit = &g;
+        break;
+      }
+      if (g.used < hit->used) hit = &g;
+    }
+    if (hit->exec) cudaGraphExecDestroy(hit->exec);
+    hit->X = a.X;
+    hit->Y = a.Y;
+    hit->B = a.B;
+    hit->T = a.T;
+    hit->weight_only = a.weight_only;
+    hit->exec = exec;
+  }
+  hit->used = ++p->graph_clock;
+  return cudaGraphLaunch(hit->exec, s) == cudaSuccess ? 0 : -1;
 }
 
 int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool weight_only,
@@ -170,10 +265,11 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Ct = p->Ct;
     a.splits = 1;
     a.split_rows = 64;
-    if (correct) dyra::gram_split(T, B, p->dev.sm_count, &a.splits, &a.split_rows);
+    if (correct) dyra::gram_split(T, B, p->d_in, p->k, p->dev.sm_count, &a.splits, &a.split_rows);
     a.status = p->status;
     a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
-    rc = dyra::launch_bf16_forward(a, p->dev, s);
+    a.trace = p->trace;
+    rc = launch_bf16_maybe_graph(p, a, s);
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
@@ -321,6 +417,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   p->dev.cc_minor = prop.minor;
   const char* kv = std::getenv("DYRA_KERNELS");
   p->force_simt = kv != nullptr && std::strcmp(kv, "simt") == 0;
+  const char* gv = std::getenv("DYRA_GRAPHS");
+  p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
   if (dev_alloc(&st, 256) != DYRA_OK) {
     delete p;
@@ -369,6 +467,7 @@ int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P
   if (rc) return DYRA_ERR_CUDA;
   p->lambda = lambda;
   p->loaded = true;
+  drop_graphs(p);  // lambda is baked into captured launches
   return DYRA_OK;
 }
 
@@ -424,6 +523,9 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(st);
     for (auto& e : p->stage_ev)
       if (e) cudaEventDestroy(e);
+    if (p->trace) cudaFree(p->trace);
+    drop_graphs(p);
+    if (p->capture_stream) cudaStreamDestroy(p->capture_stream);
   }
   delete p;
   return DYRA_OK;
@@ -482,6 +584,39 @@ int dyra_debug_stage_times(dyra_plan_t p, float* ms5) {
   return DYRA_OK;
 }
 
+int dyra_debug_set_trace(dyra_plan_t p, int enable) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (!enable) {
+    if (p->trace) cudaFree(p->trace);
+    p->trace = nullptr;
+    return DYRA_OK;
+  }
+  const size_t bytes = dyra_debug_trace_bytes();
+  if (!p->trace) {
+    void* t = nullptr;
+    int rc = dev_alloc(&t, bytes);
+    if (rc) return rc;
+    p->trace = static_cast<unsigned long long*>(t);
+  }
+  return cudaMemset(p->trace, 0, bytes) == cudaSuccess ? DYRA_OK : DYRA_ERR_CUDA;
+}
+
+size_t dyra_debug_trace_bytes(void) {
+  return static_cast<size_t>(5) * dyra::kTraceCtas * dyra::kTraceSlots * sizeof(unsigned long long);
+}
+
+int dyra_debug_trace_copy(dyra_plan_t p, void* dst, size_t bytes) {
+  if (p == nullptr || dst == nullptr || p->trace == nullptr || bytes > dyra_debug_trace_bytes())
+    return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DYRA_ERR_CUDA;
+  return cudaMemcpy(dst, p->trace, bytes, cudaMemcpyDeviceToHost) == cudaSuccess ? DYRA_OK
+                                                                                  : DYRA_ERR_CUDA;
+}
+
 int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int* split_rows) {
   if (p == nullptr || splits == nullptr || split_rows == nullptr || B < 0 || T < 0)
     return DYRA_ERR_INVALID_ARG;
@@ -490,7 +625,7 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
     *split_rows = static_cast<int>(T);
     return DYRA_OK;
   }
-  dyra::gram_split(T, B, p->dev.sm_count, splits, split_rows);
+  dyra::gram_split(T, B, p->d_in, p->k, p->dev.sm_count, splits, split_rows);
   return DYRA_OK;
 }
 
@@ -563,7 +698,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
   const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
   const size_t es = elem_size(p->dtype);
   int splits = 1, split_rows = 64;
-  if (umma && k > 0) dyra::gram_split(T, B, p->dev.sm_count, &splits, &split_rows);
+  if (umma && k > 0) dyra::gram_split(T, B, p->d_in, k, p->dev.sm_count, &splits, &split_rows);
 
   // Size check first, without touching the device.
   ScratchCarver sizing{nullptr};
@@ -619,6 +754,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.split_rows = split_rows;
     a.status = p->status;
     a.stage_events = nullptr;
+    a.trace = nullptr;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;

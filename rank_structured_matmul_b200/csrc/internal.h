@@ -44,11 +44,16 @@ struct Bf16Forward {
   int split_rows;        // rows per split (multiple of 64)
   int* status;
   cudaEvent_t* stage_events;  // optional: 6 events recorded around the 5 stages
+  unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
 };
+
+constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
+constexpr int kTraceSlots = 32;  // timestamps per CTA
 
 // Rows per split and split count used for a given T (shared with the
 // workspace sizing).
-void gram_split(int64_t T, int64_t B, int sm_count, int* splits, int* split_rows);
+void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits,
+                int* split_rows);
 
 int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s);
 
@@ -78,7 +83,8 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStre
 // Solve (L^T L + lambda I) T' = T for every instance from the Gram partials.
 template <typename TOut>
 int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda,
-                 TOut* Tp, int* status, cudaStream_t s, bool pdl);
+                 TOut* Tp, int* status, cudaStream_t s, bool pdl,
+                 unsigned long long* trace = nullptr);
 
 // Pack [V | P]^T: VPt[c][j] = V[j][c] (c < r), P[j][c-r] (c >= r).
 template <typename T>

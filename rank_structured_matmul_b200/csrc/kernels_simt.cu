@@ -44,8 +44,9 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
 
 constexpr int kSolveThreads = 128;
 
-// grid (B, ceil(d_in / 128)); each CTA factors G_b itself (k <= 128, a few
-// thousand flops) and solves for 128 columns of T_b, one column per thread.
+// General variant (any k <= 128). grid (B, ceil(d_in / 128)); each CTA
+// factors G_b itself (Cholesky in shared memory) and solves for 128 columns
+// of T_b, one column per thread.
 template <typename TOut>
 __global__ void __launch_bounds__(kSolveThreads)
     solve_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
@@ -123,6 +124,268 @@ __global__ void __launch_bounds__(kSolveThreads)
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
+  sm100::pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
+// Fast path for k <= 64. grid (B, ceil(d_in / 128)), 256 threads; each CTA
+// handles a 128-column chunk of T_b:
+//  1. loads: G_b (padded to KMAX with the identity) and the T chunk, summed
+//     over the row splits, into shared memory in one round trip;
+//  2. Gaussian elimination below the diagonal on [G_b | I]: after k steps the
+//     left half's diagonal is D and the right half is M = Lt^-1, where
+//     G_b = Lt D Lt^T (Lt unit lower). Each thread keeps a fixed RB x CB block
+//     of [G | I] in registers. Pivots go in panels of four: the panel's
+//     columns and rows are broadcast through ping-pong shared buffers, every
+//     thread eliminates the 4 x 4 pivot block itself and applies a rank-4
+//     update, so there is one barrier per four pivots;
+//  3. T' = M^T D^-1 (M T): two small products over the chunk, no sequential
+//     dependency (same accuracy as the two triangular solves).
+// G_b is symmetric positive definite after the ridge, so no pivoting.
+constexpr int kSolveThreads2 = 256;
+constexpr int kSolveCols = 128;  // columns of T_b per CTA
+constexpr int kPanel = 4;        // pivots eliminated per barrier
+
+template <int KMAX>
+struct SolveSmem {
+  static constexpr int LDG = KMAX + 1;  // staging of G (odd stride)
+  static constexpr int LDM = KMAX + 4;  // M rows, 16-byte aligned
+  float Tc[KMAX * kSolveCols];          // T chunk
+  float Us[KMAX * kSolveCols];          // D^-1 M T
+  float Gs[KMAX * LDG];
+  float Mr[KMAX * LDM];                 // Mr[i][q] = M[i][q]
+  float Mc[KMAX * LDM];                 // Mc[q][i] = M[i][q]
+  float colbuf[2][4][KMAX];             // [ping-pong][panel column][row]
+  float rowbuf[2][4][2 * KMAX];         // [ping-pong][panel row][column]
+  float dinv[KMAX];
+  int bad;
+};
+
+template <typename TOut, int KMAX>
+__global__ void __launch_bounds__(kSolveThreads2)
+    solve_ldl_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
+                     TOut* __restrict__ Tp, int* status, unsigned long long* trace) {
+  using Sm = SolveSmem<KMAX>;
+  extern __shared__ __align__(16) unsigned char smem_bytes[];
+  Sm& sm = *reinterpret_cast<Sm*>(smem_bytes);
+  constexpr int RB = KMAX / 8;       // rows of [G | I] per thread (warp = row group)
+  constexpr int CB = 2 * KMAX / 32;  // columns per thread (lane = column group)
+  constexpr int GPT = KMAX * KMAX / kSolveThreads2;
+  constexpr int TPT = KMAX * kSolveCols / kSolveThreads2;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int rg = tid >> 5, cg = tid & 31;
+  const int J = d_in + k;
+  const int c0 = blockIdx.y * kSolveCols;
+  const size_t inst = static_cast<size_t>(k) * J;
+  unsigned long long* const tr =
+      trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
+  if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
+  sm100::pdl_wait();
+  if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
+
+  // ---- 1. loads: G_b and the T chunk straight to shared memory, one round
+  // trip (every load of the first split issued before any store)
+  {
+    const float* part = TG + static_cast<size_t>(b) * inst;
+    float g[GPT], t[TPT];
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / KMAX, q = idx % KMAX;
+      g[u] = (i < k && q < k) ? part[static_cast<size_t>(i) * J + d_in + q] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / kSolveCols, c = idx % kSolveCols;
+      t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
+    }
+    for (int sp = 1; sp < S; ++sp) {
+      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
+#pragma unroll
+      for (int u = 0; u < GPT; ++u) {
+        const int idx = tid + u * kSolveThreads2;
+        const int i = idx / KMAX, q = idx % KMAX;
+        if (i < k && q < k) g[u] += ps[static_cast<size_t>(i) * J + d_in + q];
+      }
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) {
+        const int idx = tid + u * kSolveThreads2;
+        const int i = idx / kSolveCols, c = idx % kSolveCols;
+        if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / KMAX, q = idx % KMAX;
+      sm.Gs[i * Sm::LDG + q] =
+          (i < k && q < k) ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
+  }
+  if (tid == 0) sm.bad = 0;
+  __syncthreads();
+  if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
+
+  // ---- 2. elimination on [G | I], PANEL pivots per barrier
+  float a[RB][CB];
+#pragma unroll
+  for (int u = 0; u < RB; ++u)
+#pragma unroll
+    for (int v = 0; v < CB; ++v) {
+      const int i = rg * RB + u, q = cg * CB + v;
+      a[u][v] = q < KMAX ? sm.Gs[i * Sm::LDG + q] : (q - KMAX == i ? 1.f : 0.f);
+    }
+  auto publish = [&](int buf, int j1) {
+    // columns j1..j1+PANEL-1 (every row) and rows j1..j1+PANEL-1 (every column)
+#pragma unroll
+    for (int v = 0; v < CB; ++v) {
+      const int q = cg * CB + v;
+      if (q >= j1 && q < j1 + kPanel)
+#pragma unroll
+        for (int u = 0; u < RB; ++u) sm.colbuf[buf][q - j1][rg * RB + u] = a[u][v];
+    }
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int i = rg * RB + u;
+      if (i >= j1 && i < j1 + kPanel)
+#pragma unroll
+        for (int v = 0; v < CB; ++v) sm.rowbuf[buf][i - j1][cg * CB + v] = a[u][v];
+    }
+  };
+  publish(0, 0);
+  __syncthreads();
+  bool ok = true;
+  const int npanel = (k + kPanel - 1) / kPanel;
+  for (int pn = 0; pn < npanel; ++pn) {
+    const int buf = pn & 1, j0 = pn * kPanel;
+    // the panel's pivot rows, at the panel's columns and at this thread's columns
+    float Rp[kPanel][kPanel], Ro[kPanel][CB], rinv[kPanel];
+#pragma unroll
+    for (int r = 0; r < kPanel; ++r) {
+#pragma unroll
+      for (int c = 0; c < kPanel; ++c) Rp[r][c] = sm.rowbuf[buf][r][j0 + c];
+#pragma unroll
+      for (int v = 0; v < CB; ++v) Ro[r][v] = sm.rowbuf[buf][r][cg * CB + v];
+    }
+    // eliminate inside the panel
+#pragma unroll
+    for (int s2 = 0; s2 < kPanel; ++s2) {
+      const float piv = Rp[s2][s2];
+      ok = ok && piv > 0.f && isfinite(piv);
+      rinv[s2] = __frcp_rn(piv);
+#pragma unroll
+      for (int r = s2 + 1; r < kPanel; ++r) {
+        const float m = Rp[r][s2] * rinv[s2];
+#pragma unroll
+        for (int c = s2 + 1; c < kPanel; ++c) Rp[r][c] = fmaf(-m, Rp[s2][c], Rp[r][c]);
+#pragma unroll
+        for (int v = 0; v < CB; ++v) Ro[r][v] = fmaf(-m, Ro[s2][v], Ro[r][v]);
+      }
+    }
+    // this thread's rows: multipliers, then the rank-PANEL update
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int i = rg * RB + u;
+      float cv[kPanel], f[kPanel];
+#pragma unroll
+      for (int c = 0; c < kPanel; ++c) cv[c] = sm.colbuf[buf][c][i];
+#pragma unroll
+      for (int s2 = 0; s2 < kPanel; ++s2) {
+        f[s2] = i > j0 + s2 ? cv[s2] * rinv[s2] : 0.f;
+#pragma unroll
+        for (int c = s2 + 1; c < kPanel; ++c) cv[c] = fmaf(-f[s2], Rp[s2][c], cv[c]);
+      }
+#pragma unroll
+      for (int v = 0; v < CB; ++v)
+#pragma unroll
+        for (int s2 = 0; s2 < kPanel; ++s2) a[u][v] = fmaf(-f[s2], Ro[s2][v], a[u][v]);
+    }
+    if (j0 + kPanel < k) publish(buf ^ 1, j0 + kPanel);
+    __syncthreads();
+  }
+  if (!ok && tid == 0) sm.bad = 1;
+#pragma unroll
+  for (int u = 0; u < RB; ++u)
+#pragma unroll
+    for (int v = 0; v < CB; ++v) {
+      const int i = rg * RB + u, q = cg * CB + v;
+      if (q == i) sm.dinv[i] = __frcp_rn(a[u][v]);
+      if (q >= KMAX) {
+        sm.Mr[i * Sm::LDM + (q - KMAX)] = a[u][v];
+        sm.Mc[(q - KMAX) * Sm::LDM + i] = a[u][v];
+      }
+    }
+  __syncthreads();
+  if (tr && tid == 0) tr[4] = sm100::globaltimer_ns();
+
+  // ---- 3. T' = M^T D^-1 (M T): RPT rows x 4 columns per thread
+  constexpr int RPT = KMAX / 8;
+  float acc[RPT][4];
+#pragma unroll
+  for (int u = 0; u < RPT; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+#pragma unroll 4
+  for (int q = 0; q < k; ++q) {  // U = M T, M[i][q] = Mc[q][i]
+    const float4 t4 = *reinterpret_cast<const float4*>(&sm.Tc[q * kSolveCols + 4 * cg]);
+#pragma unroll
+    for (int u = 0; u < RPT; u += 4) {
+      const float4 m4 = *reinterpret_cast<const float4*>(&sm.Mc[q * Sm::LDM + rg * RPT + u]);
+      const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        acc[u + w][0] = fmaf(m[w], t4.x, acc[u + w][0]);
+        acc[u + w][1] = fmaf(m[w], t4.y, acc[u + w][1]);
+        acc[u + w][2] = fmaf(m[w], t4.z, acc[u + w][2]);
+        acc[u + w][3] = fmaf(m[w], t4.w, acc[u + w][3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < RPT; ++u) {
+    const int i = rg * RPT + u;
+    const float di = sm.dinv[i];
+    *reinterpret_cast<float4*>(&sm.Us[i * kSolveCols + 4 * cg]) =
+        make_float4(acc[u][0] * di, acc[u][1] * di, acc[u][2] * di, acc[u][3] * di);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+  }
+  __syncthreads();
+#pragma unroll 4
+  for (int q = 0; q < k; ++q) {  // T' = M^T V, M[q][i] = Mr[q][i]
+    const float4 v4 = *reinterpret_cast<const float4*>(&sm.Us[q * kSolveCols + 4 * cg]);
+#pragma unroll
+    for (int u = 0; u < RPT; u += 4) {
+      const float4 m4 = *reinterpret_cast<const float4*>(&sm.Mr[q * Sm::LDM + rg * RPT + u]);
+      const float m[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        acc[u + w][0] = fmaf(m[w], v4.x, acc[u + w][0]);
+        acc[u + w][1] = fmaf(m[w], v4.y, acc[u + w][1]);
+        acc[u + w][2] = fmaf(m[w], v4.z, acc[u + w][2]);
+        acc[u + w][3] = fmaf(m[w], v4.w, acc[u + w][3]);
+      }
+    }
+  }
+  if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
+  const bool zero = sm.bad != 0;
+  const int col = c0 + 4 * cg;
+#pragma unroll
+  for (int u = 0; u < RPT; ++u) {
+    const int i = rg * RPT + u;
+    if (i >= k) continue;
+    TOut* dst = Tp + (static_cast<size_t>(b) * k + i) * d_in + col;
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : acc[u][v]);
+  }
+  if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
+  __syncthreads();
+  if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
   sm100::pdl_launch_dependents();
 }
 
@@ -209,8 +472,48 @@ __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P,
 
 template <typename TOut>
 int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
-                 int* status, cudaStream_t s, bool pdl) {
+                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace) {
   if (B == 0 || k == 0) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.stream = s;
+  if (k <= 64) {
+    cfg.gridDim = dim3(static_cast<unsigned>(B),
+                       static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
+    cfg.blockDim = dim3(kSolveThreads2);
+    if (k <= 32) {
+      auto kfn = solve_ldl_kernel<TOut, 32>;
+      static bool set32 = false;
+      if (!set32) {
+        if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(SolveSmem<32>))) != cudaSuccess)
+          return -1;
+        set32 = true;
+      }
+      cfg.dynamicSmemBytes = sizeof(SolveSmem<32>);
+      return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
+                                status, trace) == cudaSuccess
+                 ? 0
+                 : -1;
+    }
+    auto kfn = solve_ldl_kernel<TOut, 64>;
+    static bool set64 = false;
+    if (!set64) {
+      if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sizeof(SolveSmem<64>))) != cudaSuccess)
+        return -1;
+      set64 = true;
+    }
+    cfg.dynamicSmemBytes = sizeof(SolveSmem<64>);
+    return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
+                              status, trace) == cudaSuccess
+               ? 0
+               : -1;
+  }
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
@@ -221,16 +524,9 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
       return -1;
     configured = smem;
   }
-  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(B), static_cast<unsigned>((d_in + kSolveThreads - 1) / kSolveThreads));
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
                             status) == cudaSuccess
              ? 0
@@ -238,9 +534,10 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
 }
 
 template int launch_solve<float>(const float*, int, int64_t, int, int, float, float*, int*,
-                                 cudaStream_t, bool);
+                                 cudaStream_t, bool, unsigned long long*);
 template int launch_solve<__nv_bfloat16>(const float*, int, int64_t, int, int, float,
-                                         __nv_bfloat16*, int*, cudaStream_t, bool);
+                                         __nv_bfloat16*, int*, cudaStream_t, bool,
+                                         unsigned long long*);
 
 template <typename T>
 int launch_pack_vp(const T* V, const T* P, T* VPt, int d_in, int r, int k, cudaStream_t s) {
@@ -279,7 +576,8 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
              s))
       return -1;
-    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false)) return -1;
+    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+      return -1;
     // C = T' W_res^T  (B*k x d_out)
     if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,
              0, 1, 0, s))

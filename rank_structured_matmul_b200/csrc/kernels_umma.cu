@@ -274,8 +274,9 @@ struct RFactorPolicy {
 // accumulated in one TMEM tile: K-segments [Z | L_b_lo | ... | L_b_hi] against
 // [U ; C_b_lo ; ... ; C_b_hi]. mask_b(L) is L's rows of instance b and zero
 // elsewhere, produced by TMA's out-of-bounds fill on the 3-D view of L.
-// The bf16 result goes out through a swizzled shared-memory box and TMA
-// stores, double buffered so the next box is written while one drains.
+// The bf16 result goes out through swizzled shared-memory boxes and TMA
+// stores; two boxes rotate, so one store drains while the next box is
+// written (more boxes would cost a pipeline stage).
 struct OutPolicy {
   struct Params {
     GemmCommon c;
@@ -290,7 +291,8 @@ struct OutPolicy {
     int m0, n0, b_lo, nseg;
   };
   static constexpr uint32_t kBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
-  static constexpr uint32_t kEpiSmemBytes = 2u * kBoxBytes;
+  static constexpr uint32_t kStoreBufs = 2;            // boxes in flight
+  static constexpr uint32_t kEpiSmemBytes = kStoreBufs * kBoxBytes;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmZ);
@@ -345,10 +347,10 @@ struct OutPolicy {
                                                   EpiCtx& e) {
     const int nbox = p.bn / 64;
     for (int bx = 0; bx < nbox; ++bx) {
-      const uint32_t buf = e.counter & 1u;
+      const uint32_t buf = e.counter % kStoreBufs;
       ++e.counter;
-      // The buffer about to be overwritten was handed to TMA two boxes ago.
-      if (e.tid == 0) tma_store_wait_read<1>();
+      // The buffer about to be overwritten was handed to TMA kStoreBufs boxes ago.
+      if (e.tid == 0) tma_store_wait_read<kStoreBufs - 1>();
       named_bar_sync(1, 128);
       uint8_t* sbuf = e.smem + buf * kBoxBytes;
 #pragma unroll
@@ -407,6 +409,7 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   if (c.tmem_cols > 512) return 0;
   c.idesc = idesc_bf16(128, mma_n, a_mn, b_mn);
   c.status = status;
+  c.trace = nullptr;
   const uint32_t fixed = gemm_smem_bytes(0, a_bytes, b_bytes, Pol::kEpiSmemBytes);
   const int budget = dev.max_smem_optin - static_cast<int>(fixed);
   int stages = budget / static_cast<int>(a_bytes + b_bytes);
@@ -451,12 +454,15 @@ int pick_bn(int n) {
 
 }  // namespace
 
-void gram_split(int64_t T, int64_t B, int sm_count, int* splits, int* split_rows) {
-  // Enough (instance, split) pairs to cover the SMs for long instances;
-  // splits are whole 64-row blocks so no block straddles two splits.
+void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits,
+                int* split_rows) {
+  // Split each instance's rows only as far as needed to give every SM a
+  // tile; splits are whole 64-row blocks so no block straddles two splits.
   const int64_t blocks = (T + 63) / 64;
-  int64_t want = std::max<int64_t>(1, (2 * sm_count) / std::max<int64_t>(1, B * 8));
-  want = std::min<int64_t>(want, blocks);
+  const int64_t mtiles = (d_in + 127) / 128 + (k + 127) / 128;
+  const int64_t per_split_tiles = std::max<int64_t>(1, B * mtiles);
+  int64_t want = (sm_count + per_split_tiles - 1) / per_split_tiles;
+  want = std::max<int64_t>(1, std::min<int64_t>(want, blocks));
   const int64_t per = (blocks + want - 1) / want;
   *split_rows = static_cast<int>(per * 64);
   *splits = static_cast<int>((blocks + per - 1) / per);
@@ -496,6 +502,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     const uint32_t smem = setup_common<ProjPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
                                                    false, a.status, dev);
     if (!smem) return -3;
+    if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
     if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
   }
   mark(1);
@@ -537,12 +544,14 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
           setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
                                    p.kpad, true, true, a.status, dev);
       if (!smem) return -3;
-      if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (a.trace) p.c.trace = a.trace + 1 * kTraceCtas * kTraceSlots;
+    if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl)) return -1;
     }
     mark(2);
     // ------------------------------------------------------------- solve
     if (launch_solve<__nv_bfloat16>(a.TG, a.splits, a.B, a.k, a.d_in, a.lambda,
-                                    static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl))
+                                    static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
+                                    a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
     mark(3);
     // ----------------------------------------------------------- rfactor
@@ -566,7 +575,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
                                                         false, false, a.status, dev);
       if (!smem) return -3;
-      if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
+    if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
     }
   } else {
     mark(2);
@@ -618,6 +628,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
                                                   false, a.status, dev);
     if (!smem) return -3;
+    if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
     if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
   }
   mark(5);

@@ -27,12 +27,29 @@
 //   static constexpr uint32_t kEpiSmemBytes;
 #pragma once
 
+#include "internal.h"
 #include "sm100.cuh"
 
 namespace dyra {
 
 constexpr int kGemmThreads = 192;
 constexpr int kMaxStages = 8;
+
+// Optional timeline: when GemmCommon::trace is set, each CTA writes
+// %globaltimer (ns) into trace[blockIdx.x * kTraceSlots + slot]
+// (kTraceSlots is defined in internal.h).
+enum TraceSlot {
+  kTrEntry = 0,        // kernel entry
+  kTrSetup = 1,        // barriers initialised, TMEM allocated
+  kTrDepsReady = 2,    // the previous grid's results are visible
+  kTrFirstIssue = 3,   // producer issued its first copy
+  kTrLastIssue = 4,    // producer issued its last copy
+  kTrFirstData = 5,    // MMA thread saw its first full slot
+  kTrLastCommit = 6,   // MMA thread committed its last tile
+  kTrEpiFirst = 7,     // epilogue saw its first finished accumulator
+  kTrExit = 8,         // all roles done, before TMEM is freed
+  kTrTileDone = 9      // + i: epilogue finished its i-th tile (i < 23)
+};
 
 struct GemmCommon {
   int num_tiles;
@@ -43,6 +60,7 @@ struct GemmCommon {
   uint32_t tmem_cols;  // allocated columns: power of two >= 2 * acc_cols, >= 32
   uint32_t idesc;      // instruction descriptor (M = 128, N, majors)
   int* status;         // device status word
+  unsigned long long* trace;  // optional timeline, nullptr when off
 };
 
 struct EpiCtx {
@@ -88,6 +106,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  unsigned long long* const tr = c.trace ? c.trace + blockIdx.x * kTraceSlots : nullptr;
+  if (tr && threadIdx.x == 0) tr[kTrEntry] = globaltimer_ns();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -112,8 +132,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (tr && threadIdx.x == 0) tr[kTrSetup] = globaltimer_ns();
   // Inputs written by the previous kernel in the stream are visible from here.
   pdl_wait();
+  if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
 
@@ -136,6 +158,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(full_bar(stage), c.a_stage_bytes + c.b_stage_bytes);
           Pol::load(p, t, it, sA + stage * c.a_stage_bytes, sB + stage * c.b_stage_bytes,
                     full_bar(stage));
+          if (tr) {
+            if (!issued) tr[kTrFirstIssue] = globaltimer_ns();
+            tr[kTrLastIssue] = globaltimer_ns();
+          }
           issued |= 1u << stage;
           last_phase[stage] = phase;
           if (++stage == S) {
@@ -170,6 +196,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
           const uint32_t a = sA + stage * c.a_stage_bytes;
           const uint32_t b = sB + stage * c.b_stage_bytes;
@@ -185,6 +212,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         mma_commit(tfull_bar(acc));
+        if (tr) tr[kTrLastCommit] = globaltimer_ns();
       }
       // All MMAs issued by this thread are complete before TMEM is freed.
       mma_commit(fin_bar);
@@ -205,6 +233,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!mbar_wait(tfull_bar(acc), acc_phase, w)) break;
       tc_fence_after();
+      if (tr && e.tid == 0 && local == 0) tr[kTrEpiFirst] = globaltimer_ns();
       typename Pol::Tile t;
       Pol::decode(p, tile, t);
       const uint32_t tacc = tmem + static_cast<uint32_t>(acc) * c.acc_cols +
@@ -213,11 +242,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (tr && e.tid == 0 && local < kTraceSlots - kTrTileDone) tr[kTrTileDone + local] = globaltimer_ns();
     }
     Pol::epilogue_drain(p, e);
   }
 
   __syncthreads();
+  if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();
   pdl_launch_dependents();
   if (warp == 1) {
     tc_fence_after();

@@ -50,6 +50,9 @@ SIGNATURES = {
     "dyra_debug_gram_split": (_i, [_vp, _i64, _i64, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "dyra_debug_set_stage_timing": (_i, [_vp, _i]),
     "dyra_debug_stage_times": (_i, [_vp, ctypes.POINTER(ctypes.c_float)]),
+    "dyra_debug_set_trace": (_i, [_vp, _i]),
+    "dyra_debug_trace_bytes": (ctypes.c_size_t, []),
+    "dyra_debug_trace_copy": (_i, [_vp, _vp, ctypes.c_size_t]),
 }
 
 STAGES = ("proj", "gram", "solve", "rfactor", "out")
@@ -183,6 +186,19 @@ def dyra_debug_stage_times(plan: int):
     ms = (ctypes.c_float * 5)()
     _check(lib().dyra_debug_stage_times(plan, ms), "dyra_debug_stage_times")
     return dict(zip(STAGES, list(ms)))
+
+
+def dyra_debug_set_trace(plan: int, enable: bool) -> None:
+    _check(lib().dyra_debug_set_trace(plan, int(bool(enable))), "dyra_debug_set_trace")
+
+
+def dyra_debug_trace(plan: int):
+    """Timeline stamps as a uint64 array [5 stages][256 CTAs][32 slots]."""
+    import numpy as np
+    n = int(lib().dyra_debug_trace_bytes())
+    buf = (ctypes.c_char * n)()
+    _check(lib().dyra_debug_trace_copy(plan, buf, n), "dyra_debug_trace_copy")
+    return np.frombuffer(bytes(buf), dtype=np.uint64).reshape(5, 256, 32)
 
 
 # ---- convenience object ----

@@ -197,6 +197,46 @@ def test_side_stream():
     layer.close()
 
 
+def test_graph_replay_matches_direct_launches():
+    """The per-plan CUDA-graph cache replays exactly the launches a direct
+    forward makes (DYRA_GRAPHS=0 disables the cache)."""
+    s, f = _small()
+    X = to_dev(f["X"], "bf16")
+    os.environ["DYRA_GRAPHS"] = "0"
+    try:
+        direct = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_GRAPHS")
+    cached = make_layer(s, f)
+    Yd = direct.forward(X, B=s.B, T=s.T)
+    Yc = [cached.forward(X, B=s.B, T=s.T) for _ in range(3)]  # new Y each call: new graphs
+    Y = torch.empty_like(Yd)
+    for _ in range(3):
+        cached.forward(X, B=s.B, T=s.T, Y=Y)  # same arguments: replays one graph
+    torch.cuda.synchronize()
+    assert all(torch.equal(Yd, y) for y in Yc + [Y])
+    direct.close()
+    cached.close()
+
+
+def test_forward_inside_caller_graph_capture():
+    """A forward issued while the caller captures its stream is recorded into
+    the caller's graph (the workspace is reserved beforehand)."""
+    s, f = _small()
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    want = layer.forward(X, B=s.B, T=s.T)
+    Y = torch.zeros_like(want)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(X, B=s.B, T=s.T, Y=Y)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, want)
+    del g
+    layer.close()
+
+
 def test_rank_deficient_is_an_error():
     s, f = _small(k=32, lam=0.0, B=2, T=20)
     layer = make_layer(s, f)
