@@ -57,11 +57,14 @@ int dyra_debug_stage_times(dyra_plan_t p, float *ms5);
 /* Kernel timelines. When enabled, each CTA of the four tensor-core stages of
  * a bf16 forward (proj, gram, rfactor, out) writes %globaltimer nanosecond
  * stamps at fixed milestones into a plan-owned buffer laid out as
- * [stage 0..4][CTA 0..255][slot 0..31] (uint64; stage 2, the solve, stays 0):
+ * [stage 0..4][CTA 0..255][slot 0..63] (uint64):
  *   0 entry, 1 set-up done, 2 inputs of the previous stage visible,
  *   3 first copy issued, 4 last copy issued, 5 first operands arrived,
  *   6 last accumulator committed, 7 first accumulator reached the epilogue,
- *   8 exit, 9 + i epilogue of the CTA's i-th tile done.
+ *   8 exit, 9 + i epilogue of the CTA's i-th tile done (i < 27),
+ *   36 + i MMAs of the CTA's i-th tile committed (i < 28).
+ * The solve stage (2) uses 0 entry, 2 inputs visible, 3 loaded, 4 factored,
+ * 5 solved, 8 exit.
  * A slot a CTA did not reach stays 0. Disabling frees the buffer. */
 int dyra_debug_set_trace(dyra_plan_t p, int enable);
 size_t dyra_debug_trace_bytes(void);

@@ -22,6 +22,7 @@ struct dyra_plan {
   dyra::DeviceInfo dev;
   bool loaded = false;
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
+  bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
   float lambda = 0.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
@@ -269,6 +270,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.status = p->status;
     a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
     a.trace = p->trace;
+    a.use_pairs = p->use_pairs;
     rc = launch_bf16_maybe_graph(p, a, s);
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
@@ -417,6 +419,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   p->dev.cc_minor = prop.minor;
   const char* kv = std::getenv("DYRA_KERNELS");
   p->force_simt = kv != nullptr && std::strcmp(kv, "simt") == 0;
+  const char* pv = std::getenv("DYRA_PAIR");
+  p->use_pairs = !(pv != nullptr && pv[0] == '0');
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -755,6 +759,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.status = p->status;
     a.stage_events = nullptr;
     a.trace = nullptr;
+    a.use_pairs = p->use_pairs;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;

@@ -45,10 +45,11 @@ struct Bf16Forward {
   int* status;
   cudaEvent_t* stage_events;  // optional: 6 events recorded around the 5 stages
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
+  bool use_pairs;             // run the output stage on CTA pairs
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
-constexpr int kTraceSlots = 32;  // timestamps per CTA
+constexpr int kTraceSlots = 64;  // timestamps per CTA
 
 // Rows per split and split count used for a given T (shared with the
 // workspace sizing).

@@ -329,8 +329,10 @@ __global__ void __launch_bounds__(kSolveThreads2)
   for (int u = 0; u < RPT; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+  // M is unit lower triangular: rows rg*RPT.. need q <= their index only.
+  const int qmax = min(k, (rg + 1) * RPT);
 #pragma unroll 4
-  for (int q = 0; q < k; ++q) {  // U = M T, M[i][q] = Mc[q][i]
+  for (int q = 0; q < qmax; ++q) {  // U = M T, M[i][q] = Mc[q][i]
     const float4 t4 = *reinterpret_cast<const float4*>(&sm.Tc[q * kSolveCols + 4 * cg]);
 #pragma unroll
     for (int u = 0; u < RPT; u += 4) {
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
   }
   __syncthreads();
 #pragma unroll 4
-  for (int q = 0; q < k; ++q) {  // T' = M^T V, M[q][i] = Mr[q][i]
+  for (int q = rg * RPT; q < k; ++q) {  // T' = M^T V, M[q][i] = Mr[q][i], q >= i
     const float4 v4 = *reinterpret_cast<const float4*>(&sm.Us[q * kSolveCols + 4 * cg]);
 #pragma unroll
     for (int u = 0; u < RPT; u += 4) {
@@ -490,7 +492,9 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
       static bool set32 = false;
       if (!set32) {
         if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(SolveSmem<32>))) != cudaSuccess)
+                                 static_cast<int>(sizeof(SolveSmem<32>))) != cudaSuccess ||
+            cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+                cudaSuccess)
           return -1;
         set32 = true;
       }
@@ -504,7 +508,9 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
     static bool set64 = false;
     if (!set64) {
       if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sizeof(SolveSmem<64>))) != cudaSuccess)
+                               static_cast<int>(sizeof(SolveSmem<64>))) != cudaSuccess ||
+          cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+              cudaSuccess)
         return -1;
       set64 = true;
     }

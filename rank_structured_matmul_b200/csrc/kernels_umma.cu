@@ -24,6 +24,7 @@
 
 #include "internal.h"
 #include "umma_gemm.cuh"
+#include "umma_gemm_pair.cuh"
 
 namespace dyra {
 
@@ -49,6 +50,52 @@ __device__ __forceinline__ void store8_bf16(void* dst, const uint32_t (&v)[32], 
 
 __device__ __forceinline__ int ceil_div_dev(int a, int b) { return (a + b - 1) / b; }
 
+// Epilogue helper: writes one 128 x 64 box of the accumulator (TMEM columns
+// col0 .. col0+63 of this thread's row) as bf16 through a 128-byte-swizzled
+// shared-memory box and a TMA store at (x, y) of `tmap`. Two boxes rotate: a
+// box is rewritten only after the store issued two boxes earlier has read it.
+// All 128 epilogue threads call it; thread 0 issues the stores.
+constexpr uint32_t kStoreBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
+constexpr uint32_t kStoreBoxes = 2;
+
+__device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const void* tmap, int x,
+                                               int y, EpiCtx& e) {
+  const uint32_t buf = e.counter % kStoreBoxes;
+  ++e.counter;
+  if (e.tid == 0) tma_store_wait_read<kStoreBoxes - 1>();
+  named_bar_sync(1, 128);
+  uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
+  uint32_t vv[2][32];  // both TMEM loads in flight before one wait
+  tmem_ld_32x32b_x32(tacc + col0, vv[0]);
+  tmem_ld_32x32b_x32(tacc + col0 + 32, vv[1]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      const int chunk = half * 4 + ch;
+      const uint32_t off =
+          static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+      uint4 q;
+      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]), f32(vv[half][8 * ch + 1]));
+      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]), f32(vv[half][8 * ch + 3]));
+      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]), f32(vv[half][8 * ch + 5]));
+      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]), f32(vv[half][8 * ch + 7]));
+      *reinterpret_cast<uint4*>(sbuf + off) = q;
+    }
+  }
+  fence_async_shared();
+  named_bar_sync(1, 128);
+  if (e.tid == 0) {
+    tma_store_2d(tmap, e.smem_u32 + buf * kStoreBoxBytes, x, y);
+    tma_store_commit();
+  }
+}
+
+__device__ __forceinline__ void store_drain(EpiCtx& e) {
+  if (e.tid == 0) tma_store_wait_all();
+}
+
 }  // namespace
 
 // =================================================================== proj ====
@@ -60,18 +107,25 @@ struct ProjPolicy {
     GemmCommon c;
     CUtensorMap tmX;  // (d_in, N), box (64, 128)
     CUtensorMap tmW;  // (d_in, r+k), box (64, bn)
+    CUtensorMap tmZ;  // (r, N), box (64, 128), store
+    CUtensorMap tmL;  // (k, N), box (64, 128), store (a 64-column box covers k <= 64 columns)
     int N, d_in, r, k, bn, n_tiles_n;
+    int tma_store;    // r % 64 == 0 and k <= 64: every 64-column box is all Z or all L
     __nv_bfloat16* Z;
     __nv_bfloat16* L;
   };
   struct Tile {
     int m0, n0;
   };
-  static constexpr uint32_t kEpiSmemBytes = 0;
+  static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
     tma_prefetch_desc(&p.tmW);
+    if (p.tma_store) {
+      tma_prefetch_desc(&p.tmZ);
+      if (p.k > 0) tma_prefetch_desc(&p.tmL);
+    }
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 128;
@@ -96,8 +150,19 @@ struct ProjPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    const int grow = t.m0 + e.row;
     const int rk = p.r + p.k;
+    if (p.tma_store) {
+      for (int bx = 0; bx < p.bn / 64; ++bx) {
+        const int col = t.n0 + bx * 64;
+        if (col >= rk) break;
+        if (col < p.r)
+          store_box_bf16(tacc, bx * 64, &p.tmZ, col, t.m0, e);
+        else
+          store_box_bf16(tacc, bx * 64, &p.tmL, col - p.r, t.m0, e);
+      }
+      return;
+    }
+    const int grow = t.m0 + e.row;
     for (int cc = 0; cc < p.bn; cc += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tacc + cc, v);
@@ -116,7 +181,9 @@ struct ProjPolicy {
       }
     }
   }
-  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
+  static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
+    if (p.tma_store) store_drain(e);
+  }
 };
 
 // =================================================================== gram ====
@@ -217,17 +284,18 @@ struct RFactorPolicy {
     GemmCommon c;
     CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
     CUtensorMap tmT;  // (d_in, B*k),   box (64, bn)
+    CUtensorMap tmC;  // (B*k, d_out),  box (64, 128), store
     int d_in, d_out, Bk, bn, n_tiles_n;
-    __nv_bfloat16* Ct;
   };
   struct Tile {
     int m0, n0;
   };
-  static constexpr uint32_t kEpiSmemBytes = 0;
+  static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmW);
     tma_prefetch_desc(&p.tmT);
+    tma_prefetch_desc(&p.tmC);
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 128;
@@ -252,21 +320,10 @@ struct RFactorPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    const int grow = t.m0 + e.row;
-    for (int cc = 0; cc < p.bn; cc += 32) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tacc + cc, v);
-      tmem_ld_wait();
-      if (grow < p.d_out) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = t.n0 + cc + 8 * g;
-          if (col < p.Bk) store8_bf16(p.Ct + static_cast<size_t>(grow) * p.Bk + col, v, g);
-        }
-      }
-    }
+    for (int bx = 0; bx < p.bn / 64; ++bx)
+      store_box_bf16(tacc, bx * 64, &p.tmC, t.n0 + bx * 64, t.m0, e);
   }
-  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) { store_drain(e); }
 };
 
 // ==================================================================== out ====
@@ -290,9 +347,7 @@ struct OutPolicy {
   struct Tile {
     int m0, n0, b_lo, nseg;
   };
-  static constexpr uint32_t kBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
-  static constexpr uint32_t kStoreBufs = 2;            // boxes in flight
-  static constexpr uint32_t kEpiSmemBytes = kStoreBufs * kBoxBytes;
+  static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmZ);
@@ -345,42 +400,116 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    const int nbox = p.bn / 64;
-    for (int bx = 0; bx < nbox; ++bx) {
-      const uint32_t buf = e.counter % kStoreBufs;
-      ++e.counter;
-      // The buffer about to be overwritten was handed to TMA kStoreBufs boxes ago.
-      if (e.tid == 0) tma_store_wait_read<kStoreBufs - 1>();
-      named_bar_sync(1, 128);
-      uint8_t* sbuf = e.smem + buf * kBoxBytes;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tacc + bx * 64 + half * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = half * 4 + ch;
-          const uint32_t off = static_cast<uint32_t>(e.row) * 128u +
-                               static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
-          uint4 q;
-          q.x = pack_bf16x2(f32(v[8 * ch + 0]), f32(v[8 * ch + 1]));
-          q.y = pack_bf16x2(f32(v[8 * ch + 2]), f32(v[8 * ch + 3]));
-          q.z = pack_bf16x2(f32(v[8 * ch + 4]), f32(v[8 * ch + 5]));
-          q.w = pack_bf16x2(f32(v[8 * ch + 6]), f32(v[8 * ch + 7]));
-          *reinterpret_cast<uint4*>(sbuf + off) = q;
-        }
-      }
-      fence_async_shared();
-      named_bar_sync(1, 128);
-      if (e.tid == 0) {
-        tma_store_2d(&p.tmY, e.smem_u32 + buf * kBoxBytes, t.n0 + bx * 64, t.m0);
-        tma_store_commit();
-      }
+    for (int bx = 0; bx < p.bn / 64; ++bx)
+      store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e);
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) { store_drain(e); }
+};
+
+// ============================================================ proj, pairs ====
+// [Z | L] = X [V | P] on CTA pairs: tile 256 x bn, CTA r loads rows
+// m0 + 128 r of X and rows n0 + (bn/2) r of [V | P]^T and stores its 128 rows.
+struct ProjPairPolicy {
+  using Params = ProjPolicy::Params;  // tmW box is (64, bn/2) here
+  using Tile = ProjPolicy::Tile;
+  static constexpr uint32_t kEpiSmemBytes = ProjPolicy::kEpiSmemBytes;
+  static __device__ __forceinline__ void prefetch(const Params& p) { ProjPolicy::prefetch(p); }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 256;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    return ProjPolicy::kiters(p, t);
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar, uint32_t rank) {
+    tma_load_2d_pair(sa, &p.tmX, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
+    tma_load_2d_pair(sb, &p.tmW, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
+    return ProjPolicy::ksteps(p, t, it);
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    Tile h{t.m0 + 128 * e.rank, t.n0};
+    ProjPolicy::epilogue(p, h, tacc, e);
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
+    ProjPolicy::epilogue_drain(p, e);
+  }
+};
+
+// =============================================================== out, pairs ====
+// The output stage on CTA pairs: tile 256 x bn, CTA r of the pair owns rows
+// m0 + 128 r .. +127 of A and of Y, and rows n0 + (bn/2) r .. + bn/2 - 1 of
+// the B operand ([U ; C_b]); the epilogue is OutPolicy's for its 128 rows.
+struct OutPairPolicy {
+  using Params = OutPolicy::Params;  // tmU / tmC boxes are (64, bn/2) here
+  struct Tile {
+    int m0, n0, b_lo, nseg;
+  };
+  static constexpr uint32_t kEpiSmemBytes = OutPolicy::kEpiSmemBytes;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) { OutPolicy::prefetch(p); }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 256;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+    if (p.nkl > 0) {
+      t.b_lo = t.m0 / p.T;
+      const int b_hi = min(p.B - 1, (t.m0 + 255) / p.T);
+      t.nseg = b_hi - t.b_lo + 1;
+    } else {
+      t.b_lo = 0;
+      t.nseg = 0;
     }
   }
-  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) {
-    if (e.tid == 0) tma_store_wait_all();
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    return p.nkz + t.nseg * p.nkl;
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar, uint32_t rank) {
+    const int ma = t.m0 + 128 * static_cast<int>(rank);
+    const int nb = t.n0 + (p.bn / 2) * static_cast<int>(rank);
+    if (it < p.nkz) {
+      tma_load_2d_pair(sa, &p.tmZ, bar, it * 64, ma);
+      tma_load_2d_pair(sb, &p.tmU, bar, it * 64, nb);
+    } else {
+      const int j = it - p.nkz;
+      const int seg = j / p.nkl;
+      const int ch = j - seg * p.nkl;
+      const int b = t.b_lo + seg;
+      tma_load_3d_pair(sa, &p.tmL, bar, ch * 64, ma - b * p.T, b);
+      tma_load_2d_pair(sb, &p.tmC, bar, b * p.k + ch * 64, nb);
+    }
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
+    if (it < p.nkz) return min(4, ceil_div_dev(p.r - it * 64, 16));
+    const int ch = (it - p.nkz) % p.nkl;
+    return min(4, ceil_div_dev(p.k - ch * 64, 16));
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    OutPolicy::Tile h;
+    h.m0 = t.m0 + 128 * e.rank;
+    h.n0 = t.n0;
+    h.b_lo = t.b_lo;
+    h.nseg = t.nseg;
+    OutPolicy::epilogue(p, h, tacc, e);
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
+    OutPolicy::epilogue_drain(p, e);
   }
 };
 
@@ -427,7 +556,9 @@ int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& 
   static uint32_t configured = 0;
   if (smem > configured) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
       return -1;
     configured = smem;
   }
@@ -436,6 +567,41 @@ int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& 
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kfn, p) == cudaSuccess ? 0 : -1;
+}
+
+template <class Pol>
+int launch_gemm_pair(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& dev,
+                     cudaStream_t s, bool pdl) {
+  if (p.c.num_tiles <= 0) return 0;
+  auto kfn = umma_gemm_pair_kernel<Pol>;
+  static uint32_t configured = 0;
+  static int max_pairs = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  if (smem > configured) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
+      return -1;
+    configured = smem;
+    cfg.gridDim = dim3(2 * (dev.sm_count / 2));
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kfn, &cfg) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      clusters = dev.sm_count / 2;
+    }
+    max_pairs = clusters;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min(p.c.num_tiles, max_pairs)));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -487,7 +653,9 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     p.d_in = a.d_in;
     p.r = a.r;
     p.k = a.weight_only ? 0 : a.k;
+    p.tma_store = (a.r % 64 == 0 && p.k <= 64) ? 1 : 0;
     p.bn = pick_bn(n_cols);
+    if (p.tma_store) p.bn = std::min(256, (p.bn + 63) / 64 * 64);  // whole 64-column boxes
     p.n_tiles_n = ceil_div(n_cols, p.bn);
     p.Z = static_cast<__nv_bfloat16*>(a.Z);
     p.L = static_cast<__nv_bfloat16*>(a.L);
@@ -495,15 +663,39 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
     uint32_t bx[2] = {64, 128};
     if (!encode_tmap_bf16(&p.tmX, a.X, 2, dx, sx, bx, 128)) return -2;
+    // Pairs pay a longer set-up; they win once each pair streams several tiles.
+    const bool proj_pairs = a.use_pairs && p.bn % 32 == 0 && p.bn >= 64 &&
+                            ceil_div(N, 256) * p.n_tiles_n >= dev.sm_count;
     uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(rk)};
-    uint32_t bw[2] = {64, static_cast<uint32_t>(p.bn)};
+    uint32_t bw[2] = {64, static_cast<uint32_t>(proj_pairs ? p.bn / 2 : p.bn)};
     if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
-    const int tiles = ceil_div(N, 128) * p.n_tiles_n;
-    const uint32_t smem = setup_common<ProjPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
-                                                   false, a.status, dev);
-    if (!smem) return -3;
-    if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
-    if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
+    uint32_t bs[2] = {64, 128};
+    uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
+    uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+    if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bs, 128)) return -2;
+    if (p.k > 0) {
+      uint64_t dl[2] = {static_cast<uint64_t>(p.k), static_cast<uint64_t>(N)};
+      uint64_t sl[1] = {static_cast<uint64_t>(p.k) * 2};
+      if (!encode_tmap_bf16(&p.tmL, a.L, 2, dl, sl, bs, 128)) return -2;
+    } else {
+      p.tmL = p.tmZ;
+    }
+    if (proj_pairs) {
+      const int tiles = ceil_div(N, 256) * p.n_tiles_n;
+      const uint32_t smem = setup_common<ProjPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
+                                                         p.bn, false, false, a.status, dev);
+      if (!smem) return -3;
+      p.c.idesc = idesc_bf16(256, p.bn, false, false);
+      if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
+      if (launch_gemm_pair<ProjPairPolicy>(p, smem, dev, s, pdl)) return -1;
+    } else {
+      const int tiles = ceil_div(N, 128) * p.n_tiles_n;
+      const uint32_t smem = setup_common<ProjPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
+                                                     false, false, a.status, dev);
+      if (!smem) return -3;
+      if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
+      if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
+    }
   }
   mark(1);
 
@@ -561,9 +753,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.d_in = a.d_in;
       p.d_out = a.d_out;
       p.Bk = Bk;
-      p.bn = pick_bn(Bk);
+      p.bn = std::min(256, (pick_bn(Bk) + 63) / 64 * 64);  // whole 64-column store boxes
       p.n_tiles_n = ceil_div(Bk, p.bn);
-      p.Ct = static_cast<__nv_bfloat16*>(a.Ct);
       uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.d_out)};
       uint64_t sw[1] = {static_cast<uint64_t>(a.d_in) * 2};
       uint32_t bw[2] = {64, 128};
@@ -571,12 +762,16 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
       uint32_t bt[2] = {64, static_cast<uint32_t>(p.bn)};
       if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
+      uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
+      uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
+      uint32_t bc[2] = {64, 128};
+      if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
       const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
       const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
                                                         false, false, a.status, dev);
       if (!smem) return -3;
       if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
-    if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
     }
   } else {
     mark(2);
@@ -602,7 +797,9 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     uint32_t bz[2] = {64, 128};
     if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bz, 128)) return -2;
     uint64_t du[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(a.d_out)};
-    uint32_t bu[2] = {64, static_cast<uint32_t>(p.bn)};
+    const bool use_pairs = a.use_pairs && p.bn >= 128;
+    const uint32_t bbox = static_cast<uint32_t>(use_pairs ? p.bn / 2 : p.bn);
+    uint32_t bu[2] = {64, bbox};
     if (!encode_tmap_bf16(&p.tmU, a.U, 2, du, sz, bu, 128)) return -2;
     if (k > 0) {
       uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
@@ -614,7 +811,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       const int64_t Bk = a.B * k;
       uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
-      uint32_t bc[2] = {64, static_cast<uint32_t>(p.bn)};
+      uint32_t bc[2] = {64, bbox};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
     } else {
       p.tmL = p.tmZ;
@@ -624,12 +821,22 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
     uint32_t by[2] = {64, 128};
     if (!encode_tmap_bf16(&p.tmY, a.Y, 2, dy, sy, by, 128)) return -2;
-    const int tiles = ceil_div(N, 128) * p.n_tiles_n;
-    const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
-                                                  false, a.status, dev);
-    if (!smem) return -3;
-    if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
-    if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
+    if (use_pairs) {
+      const int tiles = ceil_div(N, 256) * p.n_tiles_n;
+      const uint32_t smem = setup_common<OutPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
+                                                        p.bn, false, false, a.status, dev);
+      if (!smem) return -3;
+      p.c.idesc = idesc_bf16(256, p.bn, false, false);
+      if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
+      if (launch_gemm_pair<OutPairPolicy>(p, smem, dev, s, pdl)) return -1;
+    } else {
+      const int tiles = ceil_div(N, 128) * p.n_tiles_n;
+      const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
+                                                    false, false, a.status, dev);
+      if (!smem) return -3;
+      if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
+      if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
+    }
   }
   mark(5);
   return 0;

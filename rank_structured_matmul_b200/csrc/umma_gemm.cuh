@@ -48,7 +48,8 @@ enum TraceSlot {
   kTrLastCommit = 6,   // MMA thread committed its last tile
   kTrEpiFirst = 7,     // epilogue saw its first finished accumulator
   kTrExit = 8,         // all roles done, before TMEM is freed
-  kTrTileDone = 9      // + i: epilogue finished its i-th tile (i < 23)
+  kTrTileDone = 9,     // + i: epilogue finished its i-th tile (i < 27)
+  kTrTileMma = 36      // + i: MMA thread committed its i-th tile (i < 28)
 };
 
 struct GemmCommon {
@@ -71,6 +72,7 @@ struct EpiCtx {
   uint8_t* smem;      // policy scratch (kEpiSmemBytes), 1024-byte aligned
   uint32_t smem_u32;  // same, as a shared-window address
   uint32_t counter;   // running counter the policy may use (e.g. store buffers)
+  int rank;           // CTA of the pair (0 for single-CTA kernels)
 };
 
 __host__ __device__ inline uint32_t gemm_smem_bytes(int stages, uint32_t a_bytes,
@@ -134,6 +136,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (tr && threadIdx.x == 0) tr[kTrSetup] = globaltimer_ns();
   // Inputs written by the previous kernel in the stream are visible from here.
+  // Every CTA of this grid is resident (grid <= SMs), so the next kernel in
+  // the stream may be launched now: its CTAs take SMs as ours leave and wait
+  // in pdl_wait() for our results. This hides launch and set-up latency.
+  pdl_launch_dependents();
   pdl_wait();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
@@ -212,7 +218,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         mma_commit(tfull_bar(acc));
-        if (tr) tr[kTrLastCommit] = globaltimer_ns();
+        if (tr) {
+          tr[kTrLastCommit] = globaltimer_ns();
+          if (local < kTraceSlots - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
+        }
       }
       // All MMAs issued by this thread are complete before TMEM is freed.
       mma_commit(fin_bar);
@@ -227,6 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     e.smem = smem + (sEpi - sbase);
     e.smem_u32 = sEpi;
     e.counter = 0;
+    e.rank = 0;
     int local = 0;
     for (int tile = blockIdx.x; tile < c.num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -242,14 +252,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
-      if (tr && e.tid == 0 && local < kTraceSlots - kTrTileDone) tr[kTrTileDone + local] = globaltimer_ns();
+      if (tr && e.tid == 0 && local < kTrTileMma - kTrTileDone)
+        tr[kTrTileDone + local] = globaltimer_ns();
     }
     Pol::epilogue_drain(p, e);
   }
 
   __syncthreads();
   if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();
-  pdl_launch_dependents();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, c.tmem_cols);

@@ -193,12 +193,12 @@ def dyra_debug_set_trace(plan: int, enable: bool) -> None:
 
 
 def dyra_debug_trace(plan: int):
-    """Timeline stamps as a uint64 array [5 stages][256 CTAs][32 slots]."""
+    """Timeline stamps as a uint64 array [5 stages][256 CTAs][64 slots]."""
     import numpy as np
     n = int(lib().dyra_debug_trace_bytes())
     buf = (ctypes.c_char * n)()
     _check(lib().dyra_debug_trace_copy(plan, buf, n), "dyra_debug_trace_copy")
-    return np.frombuffer(bytes(buf), dtype=np.uint64).reshape(5, 256, 32)
+    return np.frombuffer(bytes(buf), dtype=np.uint64).reshape(5, 256, 64)
 
 
 # ---- convenience object ----

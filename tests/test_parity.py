@@ -219,6 +219,26 @@ def test_graph_replay_matches_direct_launches():
     cached.close()
 
 
+def test_pair_output_stage_matches_single_cta():
+    """The output stage on CTA pairs (default) and on single CTAs
+    (DYRA_PAIR=0) agree and both meet the oracle bar."""
+    s, f = _small(B=3, T=201)
+    X = to_dev(f["X"], "bf16")
+    os.environ["DYRA_PAIR"] = "0"
+    try:
+        single = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_PAIR")
+    pair = make_layer(s, f)
+    Y1 = single.forward(X, B=s.B, T=s.T)
+    Y2 = pair.forward(X, B=s.B, T=s.T)
+    assert pair.status() == 0
+    assert oracle.rel_fro(Y2.double().cpu().numpy(), Y1.double().cpu().numpy()) <= 1e-3
+    check(s, Y2, f)
+    single.close()
+    pair.close()
+
+
 def test_forward_inside_caller_graph_capture():
     """A forward issued while the caller captures its stream is recorded into
     the caller's graph (the workspace is reserved beforehand)."""
