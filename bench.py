@@ -2,6 +2,7 @@
 """Benchmark of the DyRA approximated linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dyra|reference]
+                    [--layer-only] [--no-cpu-baseline]
 
 One step is one DyRA forward (projection, Gram, solve, residual factor,
 output: every stage of Algorithm 1's inference procedure) over the workload's
@@ -35,8 +36,9 @@ sys.path.insert(0, ROOT)
 METRIC = "DyRA linear µs & dense-equiv TFLOP/s vs cuBLAS dense; % of roofline"
 UNIT = "TFLOP/s (dense-equivalent)"
 HEADLINE = "vit_fc1"
-STAGE_KERNELS = {"proj": "ProjPolicy", "gram": "GramPolicy", "solve": "solve_kernel",
-                 "rfactor": "RFactorPolicy", "out": "OutPolicy"}
+STAGE_KERNELS = {"proj": "umma_gemm_kernel<ProjPolicy>", "gram": "umma_gemm_kernel<GramPolicy>",
+                 "solve": "solve_ldl_kernel", "rfactor": "umma_gemm_kernel<RFactorPolicy>",
+                 "out": "umma_gemm_pair_kernel<OutPairPolicy>"}
 FLUSH_BYTES = 256 << 20
 
 
@@ -107,51 +109,99 @@ def algorithmic(s):
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled every few ms while the timed
+    region runs (read-only NVML queries; nvidia-smi as a fallback)."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.cuda_index = cuda_index
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.stop_flag = False
+        self.handle = None
+        self.nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(pynvml)
+        except Exception:
+            self.nvml = None
+            self.handle = None
+
+    def _handle(self, pynvml):
+        import torch
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devid = getattr(props, "pci_device_id", 0)
+            bus_str = "%08x:%02x:%02x.0" % (dom, bus, devid)
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus_str)
+            except Exception:
+                pass
+        return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def _sample(self):
+        n, h = self.nvml, self.handle
+        sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+        try:
+            bits = n.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            bits = n.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.rows.append((float(sm), float(mx), int(bits)))
+
+    def _loop(self):
+        while not self.stop_flag:
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self.period)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+        self._sample()
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+        if self.handle is None:
+            return self._smi_once()
+        self.stop_flag = True
+        self.thread.join()
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append((float(f[1]), float(f[2]), f[5:9]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl)
-                          if v.lower() == "active"})
+            self._sample()
+        except Exception:
+            pass
+        rows = self.rows
+        reasons = sorted(name for name, bit in self.REASONS.items()
+                         if any(r[2] & bit for r in rows))
         return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvml, every 5 ms"}
+
+    def _smi_once(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(self.cuda_index),
+                                  "--query-gpu=" + fields, "--format=csv,noheader,nounits"],
+                                 capture_output=True, text=True, timeout=20).stdout
+            f = [x.strip() for x in out.strip().split(",")]
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            return {"sm_mhz": float(f[0]), "sm_max_mhz": float(f[1]),
+                    "reasons": [n for n, v in zip(names, f[2:6]) if v.lower() == "active"],
+                    "samples": 1, "source": "nvidia-smi after the timed region"}
+        except Exception:
+            return None
 
 
 # ------------------------------------------------------------ dyra arm ----
@@ -221,39 +271,59 @@ def run_dyra(args):
 
     dense_flops = 2.0 * s.N * s.d_in * s.d_out
     value = dense_flops * world / (ms * 1e-3) / 1e12
+    if args.layer_only:  # the timed steps only (for profiler launch lists)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                              "config": {"workload": s.name}, "device_status": status,
+                              "layer_only": True}), flush=True)
+        layer.close()
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     # ---- cuBLAS dense X W^T of the same shape
     Wd = torch.from_numpy(w.weight()).to(dev, td)
     Yd = torch.empty_like(Y)
     dense_ms = timed(lambda: torch.matmul(X, Wd.t(), out=Yd), args.steps, 3)
 
-    # ---- per-stage device time (events between the stage launches)
-    dyra.dyra_debug_set_stage_timing(layer.plan, True)
-    acc = {k: [] for k in dyra.STAGES}
-    for _ in range(max(5, args.steps)):
-        flush.zero_()
-        step()
-        for k2, v in dyra.dyra_debug_stage_times(layer.plan).items():
-            acc[k2].append(v)
-    dyra.dyra_debug_set_stage_timing(layer.plan, False)
-    stage_ms = {k2: float(np.mean(v)) for k2, v in acc.items()}
-
+    # ---- per-stage device time (events between the stage launches); the
+    # tensor-core path only (the fp32 path runs plain CUDA-core kernels)
     pk = peaks()
     flops, bytes_, layer_flops, layer_bytes = algorithmic(s)
-    dom = max(stage_ms, key=stage_ms.get)
-    t_dom = stage_ms[dom] * 1e-3
-    tensor_t = flops[dom] / (pk["bf16_tflops"] * 1e12)
-    hbm_t = bytes_[dom] / (pk["hbm_gbs"] * 1e9)
-    if tensor_t >= hbm_t:
-        roof = {"bound": "tensor", "achieved": flops[dom] / t_dom / 1e12,
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    umma = s.dtype == "bf16"
+    stage_ms = None
+    if umma:
+        dyra.dyra_debug_set_stage_timing(layer.plan, True)
+        acc = {k: [] for k in dyra.STAGES}
+        for _ in range(max(5, min(args.steps, 50))):
+            flush.zero_()
+            step()
+            for k2, v in dyra.dyra_debug_stage_times(layer.plan).items():
+                acc[k2].append(v)
+        dyra.dyra_debug_set_stage_timing(layer.plan, False)
+        stage_ms = {k2: float(np.mean(v)) for k2, v in acc.items()}
+        dom = max(stage_ms, key=stage_ms.get)
+        t_dom = stage_ms[dom] * 1e-3
+        tensor_t = flops[dom] / (pk["bf16_tflops"] * 1e12)
+        hbm_t = bytes_[dom] / (pk["hbm_gbs"] * 1e9)
+        if tensor_t >= hbm_t:
+            roof = {"bound": "tensor", "achieved": flops[dom] / t_dom / 1e12,
+                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": bytes_[dom] / t_dom / 1e9, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = stored_traffic(dom, args.workload)
+        roof["kernel"] = STAGE_KERNELS[dom]
+        roof["peak_source"] = pk["source"] + " burst"
     else:
-        roof = {"bound": "hbm", "achieved": bytes_[dom] / t_dom / 1e9, "peak": pk["hbm_gbs"],
-                "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = stored_traffic(dom, args.workload)
-    roof["kernel"] = STAGE_KERNELS[dom]
-    roof["peak_source"] = pk["source"] + " burst"
+        # fp32 FFMA: 148 SMs x 128 lanes x 2 FLOP at the maximum SM clock
+        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"bound": "alu", "achieved": layer_flops / (ms * 1e-3) / 1e12, "peak": fp32_peak,
+                "unit": "TFLOP/s", "traffic": None, "kernel": "whole layer (fp32 CUDA-core path)",
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
     layer_roof_us = max(layer_flops / (pk["bf16_tflops"] * 1e12),
                         layer_bytes / (pk["hbm_gbs"] * 1e9)) * 1e6
 
@@ -288,12 +358,12 @@ def run_dyra(args):
         "dyra_tflops_algorithmic": layer_flops / (ms * 1e-3) / 1e12,
         "layer_roofline": {"us": layer_roof_us, "frac": layer_roof_us / (ms * 1e3),
                            "flops": layer_flops, "bytes": layer_bytes},
-        "stage_us": {k2: v * 1e3 for k2, v in stage_ms.items()},
+        "stage_us": {k2: v * 1e3 for k2, v in stage_ms.items()} if stage_ms else None,
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": X.numel() * X.element_size(),
                 "d2h_bytes_per_step": Y.numel() * Y.element_size(), "us": e2e_ms * 1e3},
-        "gpu_launches": (5 if s.k > 0 else 2) * args.steps,
+        "gpu_launches": ((5 if s.k > 0 else 2) if umma else (7 if s.k > 0 else 2)) * args.steps,
         "device_status": status,
         "clocks": clk,
     }
@@ -353,8 +423,10 @@ def run_reference(args):
     t0 = time.perf_counter()
     oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
     t1 = time.perf_counter() - t0
-    # each step a bounded sample: whole instances worth about 5 s at most
-    n_inst = int(max(1, min(s.B, 5.0 // max(t1, 1e-3))))
+    # each step a bounded sample of whole instances, sized so that the whole
+    # run (warm-up included) takes about two minutes of host time
+    per_step = 120.0 / (args.steps + args.warmup)
+    n_inst = int(max(1, min(s.B, per_step // max(t1, 1e-4))))
     rows = n_inst * s.T
     for _ in range(args.warmup):
         oracle.inference(Xr[:rows], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
@@ -382,11 +454,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--impl", choices=("dyra", "reference"), default="dyra")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="time the DyRA steps only: no cuBLAS, stage timing, e2e or CPU legs")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed steps
     if args.impl == "reference":

@@ -23,6 +23,7 @@ struct dyra_plan {
   bool loaded = false;
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
   bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
+  bool factor_in_gram = false;  // DYRA_FACTOR=gram: factor G_b once, in the Gram stage
   float lambda = 0.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
@@ -34,7 +35,8 @@ struct dyra_plan {
   float* TG = nullptr;   // splits x B x k x (d_in + k)
   void* Tp = nullptr;    // (B*k) x d_in
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
-  size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0;
+  void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
+  size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -122,15 +124,30 @@ struct DeviceGuard {
 
 int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
+// Factor records plus arrival counters of the Gram stage (bf16, k <= 64).
+size_t factor_bytes(int64_t B, int k) {
+  const int rec = dyra::factor_record_floats(k);
+  if (rec == 0) return 0;
+  return static_cast<size_t>(B) * rec * sizeof(float) + static_cast<size_t>(B) * sizeof(int);
+}
+
+// Splits factor_bytes' buffer into its records and counters.
+void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters) {
+  const int rec = dyra::factor_record_floats(k);
+  *md = rec ? static_cast<float*>(buf) : nullptr;
+  *counters = rec && buf ? reinterpret_cast<int*>(static_cast<float*>(buf) + B * rec) : nullptr;
+}
+
 // Grows the workspace; captured graphs point at the old buffers, so any
 // growth drops them.
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
-  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct;
-  const void* ptrs[5] = {p->Z, p->L, p->TG, p->Tp, p->Ct};
+  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
+  const void* ptrs[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[5] = {p->Z, p->L, p->TG, p->Tp, p->Ct};
-  bool moved = before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct;
-  for (int i = 0; i < 5; ++i) moved = moved || ptrs[i] != now[i];
+  const void* now[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
+  bool moved =
+      before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
+  for (int i = 0; i < 6; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -153,6 +170,7 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if (rc) return rc;
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
+      if ((rc = grow(p->MD, p->cap_MD, factor_bytes(B, k)))) return rc;
     }
   } else {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * (p->r + k) * es))) return rc;
@@ -264,6 +282,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.TG = p->TG;
     a.Tp = p->Tp;
     a.Ct = p->Ct;
+    split_factor_buffer(correct && p->factor_in_gram ? p->MD : nullptr, B, p->k, &a.MD,
+                        &a.counters);
     a.splits = 1;
     a.split_rows = 64;
     if (correct) dyra::gram_split(T, B, p->d_in, p->k, p->dev.sm_count, &a.splits, &a.split_rows);
@@ -421,6 +441,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   p->force_simt = kv != nullptr && std::strcmp(kv, "simt") == 0;
   const char* pv = std::getenv("DYRA_PAIR");
   p->use_pairs = !(pv != nullptr && pv[0] == '0');
+  const char* fv = std::getenv("DYRA_FACTOR");
+  p->factor_in_gram = fv != nullptr && std::strcmp(fv, "gram") == 0;
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -523,6 +545,7 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(tg);
     dev_free(p->Tp);
     dev_free(p->Ct);
+    dev_free(p->MD);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -635,7 +658,8 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
-  return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + 256;
+  return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
+         256;
 }
 
 }  // extern "C"
@@ -713,6 +737,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
       sizing.take(static_cast<size_t>(splits) * B * k * (p->d_in + k) * sizeof(float));
       sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+      sizing.take(factor_bytes(B, k));
     }
   } else {
     sizing.take(static_cast<size_t>(N) * (p->r + k) * es);
@@ -754,6 +779,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
                  : nullptr;
     a.Tp = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_in * es) : nullptr;
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
+    split_factor_buffer(k > 0 && p->factor_in_gram ? carve.take(factor_bytes(B, k)) : nullptr, B,
+                        k, &a.MD, &a.counters);
     a.splits = splits;
     a.split_rows = split_rows;
     a.status = p->status;

@@ -40,6 +40,8 @@ struct Bf16Forward {
   float* TG;             // splits x B x k x (d_in + k)
   void* Tp;              // (B*k) x d_in
   void* Ct;              // d_out x (B*k)
+  float* MD;             // B factor records (factor_record_floats(k) floats each), or nullptr
+  int* counters;         // B arrival counters of the split Gram tiles (with MD)
   int splits;            // row splits of the Gram reduction
   int split_rows;        // rows per split (multiple of 64)
   int* status;
@@ -82,10 +84,16 @@ template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStream_t s);
 
 // Solve (L^T L + lambda I) T' = T for every instance from the Gram partials.
+// MD: per-instance factor records (ldl_panel.cuh) written by the Gram stage
+// (k <= 64 only), or nullptr to factor G_b inside the solve.
 template <typename TOut>
-int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda,
-                 TOut* Tp, int* status, cudaStream_t s, bool pdl,
+int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k, int d_in,
+                 float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
                  unsigned long long* trace = nullptr);
+
+// Floats per instance of the factor records for correction rank k (0 when
+// k > 64: the solve then factors G_b itself).
+int factor_record_floats(int k);
 
 // Pack [V | P]^T: VPt[c][j] = V[j][c] (c < r), P[j][c-r] (c >= r).
 template <typename T>

@@ -14,6 +14,7 @@
 #include <algorithm>
 
 #include "internal.h"
+#include "ldl_panel.cuh"
 #include "sm100.cuh"
 
 namespace dyra {
@@ -130,46 +131,39 @@ __global__ void __launch_bounds__(kSolveThreads)
 // ---------------------------------------------------------------------------
 // Fast path for k <= 64. grid (B, ceil(d_in / 128)), 256 threads; each CTA
 // handles a 128-column chunk of T_b:
-//  1. loads: G_b (padded to KMAX with the identity) and the T chunk, summed
-//     over the row splits, into shared memory in one round trip;
-//  2. Gaussian elimination below the diagonal on [G_b | I]: after k steps the
-//     left half's diagonal is D and the right half is M = Lt^-1, where
-//     G_b = Lt D Lt^T (Lt unit lower). Each thread keeps a fixed RB x CB block
-//     of [G | I] in registers. Pivots go in panels of four: the panel's
-//     columns and rows are broadcast through ping-pong shared buffers, every
-//     thread eliminates the 4 x 4 pivot block itself and applies a rank-4
-//     update, so there is one barrier per four pivots;
+//  1. loads: either the instance's factor record (M, D^-1 and the failure
+//     flag, written once per instance by the Gram stage) or, when there is
+//     none (kFactored false), G_b summed over the row splits; the T chunk's
+//     first split is requested at the same time and lands during step 2;
+//  2. (kFactored false) G_b + lambda I = Lt D Lt^T by the panel elimination
+//     of ldl_panel.cuh, giving M = Lt^-1 and D; then the T chunk, summed
+//     over the splits, goes to shared memory;
 //  3. T' = M^T D^-1 (M T): two small products over the chunk, no sequential
 //     dependency (same accuracy as the two triangular solves).
-// G_b is symmetric positive definite after the ridge, so no pivoting.
 constexpr int kSolveThreads2 = 256;
 constexpr int kSolveCols = 128;  // columns of T_b per CTA
-constexpr int kPanel = 4;        // pivots eliminated per barrier
 
 template <int KMAX>
 struct SolveSmem {
-  static constexpr int LDG = KMAX + 1;  // staging of G (odd stride)
   static constexpr int LDM = KMAX + 4;  // M rows, 16-byte aligned
   float Tc[KMAX * kSolveCols];          // T chunk
   float Us[KMAX * kSolveCols];          // D^-1 M T
-  float Gs[KMAX * LDG];
   float Mr[KMAX * LDM];                 // Mr[i][q] = M[i][q]
   float Mc[KMAX * LDM];                 // Mc[q][i] = M[i][q]
-  float colbuf[2][4][KMAX];             // [ping-pong][panel column][row]
-  float rowbuf[2][4][2 * KMAX];         // [ping-pong][panel row][column]
   float dinv[KMAX];
+  LdlScratch<KMAX> ldl;
   int bad;
 };
 
-template <typename TOut, int KMAX>
+template <typename TOut, int KMAX, bool kFactored>
 __global__ void __launch_bounds__(kSolveThreads2)
-    solve_ldl_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
-                     TOut* __restrict__ Tp, int* status, unsigned long long* trace) {
+    solve_ldl_kernel(const float* __restrict__ TG, const float* __restrict__ MD, int S, int B,
+                     int k, int d_in, float lambda, TOut* __restrict__ Tp, int* status,
+                     unsigned long long* trace) {
   using Sm = SolveSmem<KMAX>;
+  constexpr int LDG = LdlScratch<KMAX>::LDG;
   extern __shared__ __align__(16) unsigned char smem_bytes[];
   Sm& sm = *reinterpret_cast<Sm*>(smem_bytes);
-  constexpr int RB = KMAX / 8;       // rows of [G | I] per thread (warp = row group)
-  constexpr int CB = 2 * KMAX / 32;  // columns per thread (lane = column group)
   constexpr int GPT = KMAX * KMAX / kSolveThreads2;
   constexpr int TPT = KMAX * kSolveCols / kSolveThreads2;
   const int b = blockIdx.x;
@@ -184,141 +178,90 @@ __global__ void __launch_bounds__(kSolveThreads2)
   sm100::pdl_wait();
   if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
 
-  // ---- 1. loads: G_b and the T chunk straight to shared memory, one round
-  // trip (every load of the first split issued before any store)
+  // ---- 1. loads. G_b (or the factor record) goes to shared memory first;
+  // the first split's T chunk is requested at the same time but only stored
+  // after the elimination, which runs while those loads are in flight.
+  const float* part = TG + static_cast<size_t>(b) * inst;
+  float t[TPT];
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) {
+    const int idx = tid + u * kSolveThreads2;
+    const int i = idx / kSolveCols, c = idx % kSolveCols;
+    t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
+  }
   {
-    const float* part = TG + static_cast<size_t>(b) * inst;
-    float g[GPT], t[TPT];
+    const float* rec = MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
+    float g[GPT];
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {
       const int idx = tid + u * kSolveThreads2;
       const int i = idx / KMAX, q = idx % KMAX;
-      g[u] = (i < k && q < k) ? part[static_cast<size_t>(i) * J + d_in + q] : 0.f;
+      if constexpr (kFactored)
+        g[u] = rec[idx];
+      else
+        g[u] = (i < k && q < k) ? part[static_cast<size_t>(i) * J + d_in + q] : 0.f;
     }
+    float dv = 0.f;
+    int bad = 0;
+    if constexpr (kFactored) {
+      if (tid < KMAX) dv = rec[KMAX * KMAX + tid];
+      if (tid == 0) bad = rec[KMAX * KMAX + KMAX] != 0.f;
+    } else {
+      for (int sp = 1; sp < S; ++sp) {
+        const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
+#pragma unroll
+        for (int u = 0; u < GPT; ++u) {
+          const int idx = tid + u * kSolveThreads2;
+          const int i = idx / KMAX, q = idx % KMAX;
+          if (i < k && q < k) g[u] += ps[static_cast<size_t>(i) * J + d_in + q];
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / KMAX, q = idx % KMAX;
+      if constexpr (kFactored) {
+        sm.Mr[i * Sm::LDM + q] = g[u];
+        sm.Mc[q * Sm::LDM + i] = g[u];
+      } else {
+        sm.ldl.Gs[i * LDG + q] =
+            (i < k && q < k) ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
+      }
+    }
+    if constexpr (kFactored) {
+      if (tid < KMAX) sm.dinv[tid] = dv;
+      if (tid == 0) sm.bad = bad;
+    } else {
+      if (tid == 0) sm.bad = 0;
+    }
+  }
+  __syncthreads();
+  if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
+
+  // ---- 2. elimination on [G | I]
+  if constexpr (!kFactored) {
+    const bool ok = ldl_eliminate<KMAX, kSolveThreads2>(
+        sm.ldl, k, tid, [] { __syncthreads(); },
+        [&](int i, int q, float v) {
+          sm.Mr[i * Sm::LDM + q] = v;
+          sm.Mc[q * Sm::LDM + i] = v;
+        },
+        [&](int j, float v) { sm.dinv[j] = v; });
+    if (!ok && tid == 0) sm.bad = 1;
+  }
+  // the remaining splits of the T chunk
+  for (int sp = 1; sp < S; ++sp) {
+    const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
 #pragma unroll
     for (int u = 0; u < TPT; ++u) {
       const int idx = tid + u * kSolveThreads2;
       const int i = idx / kSolveCols, c = idx % kSolveCols;
-      t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
+      if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
     }
-    for (int sp = 1; sp < S; ++sp) {
-      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
-#pragma unroll
-      for (int u = 0; u < GPT; ++u) {
-        const int idx = tid + u * kSolveThreads2;
-        const int i = idx / KMAX, q = idx % KMAX;
-        if (i < k && q < k) g[u] += ps[static_cast<size_t>(i) * J + d_in + q];
-      }
-#pragma unroll
-      for (int u = 0; u < TPT; ++u) {
-        const int idx = tid + u * kSolveThreads2;
-        const int i = idx / kSolveCols, c = idx % kSolveCols;
-        if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < GPT; ++u) {
-      const int idx = tid + u * kSolveThreads2;
-      const int i = idx / KMAX, q = idx % KMAX;
-      sm.Gs[i * Sm::LDG + q] =
-          (i < k && q < k) ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
   }
-  if (tid == 0) sm.bad = 0;
-  __syncthreads();
-  if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
-
-  // ---- 2. elimination on [G | I], PANEL pivots per barrier
-  float a[RB][CB];
 #pragma unroll
-  for (int u = 0; u < RB; ++u)
-#pragma unroll
-    for (int v = 0; v < CB; ++v) {
-      const int i = rg * RB + u, q = cg * CB + v;
-      a[u][v] = q < KMAX ? sm.Gs[i * Sm::LDG + q] : (q - KMAX == i ? 1.f : 0.f);
-    }
-  auto publish = [&](int buf, int j1) {
-    // columns j1..j1+PANEL-1 (every row) and rows j1..j1+PANEL-1 (every column)
-#pragma unroll
-    for (int v = 0; v < CB; ++v) {
-      const int q = cg * CB + v;
-      if (q >= j1 && q < j1 + kPanel)
-#pragma unroll
-        for (int u = 0; u < RB; ++u) sm.colbuf[buf][q - j1][rg * RB + u] = a[u][v];
-    }
-#pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      const int i = rg * RB + u;
-      if (i >= j1 && i < j1 + kPanel)
-#pragma unroll
-        for (int v = 0; v < CB; ++v) sm.rowbuf[buf][i - j1][cg * CB + v] = a[u][v];
-    }
-  };
-  publish(0, 0);
-  __syncthreads();
-  bool ok = true;
-  const int npanel = (k + kPanel - 1) / kPanel;
-  for (int pn = 0; pn < npanel; ++pn) {
-    const int buf = pn & 1, j0 = pn * kPanel;
-    // the panel's pivot rows, at the panel's columns and at this thread's columns
-    float Rp[kPanel][kPanel], Ro[kPanel][CB], rinv[kPanel];
-#pragma unroll
-    for (int r = 0; r < kPanel; ++r) {
-#pragma unroll
-      for (int c = 0; c < kPanel; ++c) Rp[r][c] = sm.rowbuf[buf][r][j0 + c];
-#pragma unroll
-      for (int v = 0; v < CB; ++v) Ro[r][v] = sm.rowbuf[buf][r][cg * CB + v];
-    }
-    // eliminate inside the panel
-#pragma unroll
-    for (int s2 = 0; s2 < kPanel; ++s2) {
-      const float piv = Rp[s2][s2];
-      ok = ok && piv > 0.f && isfinite(piv);
-      rinv[s2] = __frcp_rn(piv);
-#pragma unroll
-      for (int r = s2 + 1; r < kPanel; ++r) {
-        const float m = Rp[r][s2] * rinv[s2];
-#pragma unroll
-        for (int c = s2 + 1; c < kPanel; ++c) Rp[r][c] = fmaf(-m, Rp[s2][c], Rp[r][c]);
-#pragma unroll
-        for (int v = 0; v < CB; ++v) Ro[r][v] = fmaf(-m, Ro[s2][v], Ro[r][v]);
-      }
-    }
-    // this thread's rows: multipliers, then the rank-PANEL update
-#pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      const int i = rg * RB + u;
-      float cv[kPanel], f[kPanel];
-#pragma unroll
-      for (int c = 0; c < kPanel; ++c) cv[c] = sm.colbuf[buf][c][i];
-#pragma unroll
-      for (int s2 = 0; s2 < kPanel; ++s2) {
-        f[s2] = i > j0 + s2 ? cv[s2] * rinv[s2] : 0.f;
-#pragma unroll
-        for (int c = s2 + 1; c < kPanel; ++c) cv[c] = fmaf(-f[s2], Rp[s2][c], cv[c]);
-      }
-#pragma unroll
-      for (int v = 0; v < CB; ++v)
-#pragma unroll
-        for (int s2 = 0; s2 < kPanel; ++s2) a[u][v] = fmaf(-f[s2], Ro[s2][v], a[u][v]);
-    }
-    if (j0 + kPanel < k) publish(buf ^ 1, j0 + kPanel);
-    __syncthreads();
-  }
-  if (!ok && tid == 0) sm.bad = 1;
-#pragma unroll
-  for (int u = 0; u < RB; ++u)
-#pragma unroll
-    for (int v = 0; v < CB; ++v) {
-      const int i = rg * RB + u, q = cg * CB + v;
-      if (q == i) sm.dinv[i] = __frcp_rn(a[u][v]);
-      if (q >= KMAX) {
-        sm.Mr[i * Sm::LDM + (q - KMAX)] = a[u][v];
-        sm.Mc[(q - KMAX) * Sm::LDM + i] = a[u][v];
-      }
-    }
+  for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
   __syncthreads();
   if (tr && tid == 0) tr[4] = sm100::globaltimer_ns();
 
@@ -385,7 +328,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
     for (int v = 0; v < 4; ++v)
       if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : acc[u][v]);
   }
-  if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
+  if (!kFactored && tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
   sm100::pdl_launch_dependents();
@@ -472,9 +415,34 @@ __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P,
 
 }  // namespace
 
+template <typename TOut, int KMAX, bool kFactored>
+int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, const float* MD, int splits,
+                     int64_t B, int k, int d_in, float lambda, TOut* Tp, int* status,
+                     unsigned long long* trace) {
+  auto kfn = solve_ldl_kernel<TOut, KMAX, kFactored>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(SolveSmem<KMAX>))) != cudaSuccess ||
+        cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
+      return -1;
+    configured = true;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(B),
+                     static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
+  cfg.blockDim = dim3(kSolveThreads2);
+  cfg.dynamicSmemBytes = sizeof(SolveSmem<KMAX>);
+  return cudaLaunchKernelEx(&cfg, kfn, TG, MD, splits, static_cast<int>(B), k, d_in, lambda, Tp,
+                            status, trace) == cudaSuccess
+             ? 0
+             : -1;
+}
+
 template <typename TOut>
-int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
-                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace) {
+int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k, int d_in,
+                 float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
+                 unsigned long long* trace) {
   if (B == 0 || k == 0) return 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -483,43 +451,16 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   cfg.stream = s;
-  if (k <= 64) {
-    cfg.gridDim = dim3(static_cast<unsigned>(B),
-                       static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
-    cfg.blockDim = dim3(kSolveThreads2);
-    if (k <= 32) {
-      auto kfn = solve_ldl_kernel<TOut, 32>;
-      static bool set32 = false;
-      if (!set32) {
-        if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(SolveSmem<32>))) != cudaSuccess ||
-            cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-                cudaSuccess)
-          return -1;
-        set32 = true;
-      }
-      cfg.dynamicSmemBytes = sizeof(SolveSmem<32>);
-      return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
-                                status, trace) == cudaSuccess
-                 ? 0
-                 : -1;
-    }
-    auto kfn = solve_ldl_kernel<TOut, 64>;
-    static bool set64 = false;
-    if (!set64) {
-      if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sizeof(SolveSmem<64>))) != cudaSuccess ||
-          cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
-              cudaSuccess)
-        return -1;
-      set64 = true;
-    }
-    cfg.dynamicSmemBytes = sizeof(SolveSmem<64>);
-    return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
-                              status, trace) == cudaSuccess
-               ? 0
-               : -1;
-  }
+  if (k <= 32)
+    return MD ? launch_solve_ldl<TOut, 32, true>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
+                                                 status, trace)
+              : launch_solve_ldl<TOut, 32, false>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
+                                                  status, trace);
+  if (k <= 64)
+    return MD ? launch_solve_ldl<TOut, 64, true>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
+                                                 status, trace)
+              : launch_solve_ldl<TOut, 64, false>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
+                                                  status, trace);
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
@@ -539,9 +480,9 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
              : -1;
 }
 
-template int launch_solve<float>(const float*, int, int64_t, int, int, float, float*, int*,
+template int launch_solve<float>(const float*, const float*, int, int64_t, int, int, float, float*, int*,
                                  cudaStream_t, bool, unsigned long long*);
-template int launch_solve<__nv_bfloat16>(const float*, int, int64_t, int, int, float,
+template int launch_solve<__nv_bfloat16>(const float*, const float*, int, int64_t, int, int, float,
                                          __nv_bfloat16*, int*, cudaStream_t, bool,
                                          unsigned long long*);
 
@@ -582,7 +523,7 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
              s))
       return -1;
-    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+    if (launch_solve<T>(a.TG, nullptr, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
       return -1;
     // C = T' W_res^T  (B*k x d_out)
     if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,

@@ -239,6 +239,31 @@ def test_pair_output_stage_matches_single_cta():
     pair.close()
 
 
+@pytest.mark.parametrize("k,B,T", [(32, 3, 201), (64, 2, 150), (24, 1, 3000), (64, 1, 3000)])
+def test_factor_in_gram_matches_factor_in_solve(k, B, T):
+    """Factoring G_b once in the Gram stage (DYRA_FACTOR=gram; one split, or
+    the last of several splits to arrive) gives the same layer as factoring it
+    in every solve block, also on a second call (the arrival counters start
+    from zero again)."""
+    s, f = _small(k=k, B=B, T=T)
+    X = to_dev(f["X"], "bf16")
+    os.environ["DYRA_FACTOR"] = "gram"
+    try:
+        in_gram = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_FACTOR")
+    in_solve = make_layer(s, f)
+    Ys = in_solve.forward(X, B=s.B, T=s.T)
+    Yg1 = in_gram.forward(X, B=s.B, T=s.T)
+    Yg2 = in_gram.forward(X, B=s.B, T=s.T)
+    assert in_gram.status() == 0 and in_solve.status() == 0
+    assert torch.equal(Yg1, Yg2)
+    assert oracle.rel_fro(Yg1.double().cpu().numpy(), Ys.double().cpu().numpy()) <= 1e-3
+    check(s, Yg1, f)
+    in_gram.close()
+    in_solve.close()
+
+
 def test_forward_inside_caller_graph_capture():
     """A forward issued while the caller captures its stream is recorded into
     the caller's graph (the workspace is reserved beforehand)."""
