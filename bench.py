@@ -204,6 +204,24 @@ class ClockSampler:
             return None
 
 
+# ------------------------------------------------------------ ranks ----
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's value: every rank takes part, rank order does not matter."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(flops_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_rank * world / seconds / 1e12
+
+
 # ------------------------------------------------------------ dyra arm ----
 
 def run_dyra(args):
@@ -264,13 +282,10 @@ def run_dyra(args):
     barrier()
     clk = clocks.stop()
     status = layer.status()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     dense_flops = 2.0 * s.N * s.d_in * s.d_out
-    value = dense_flops * world / (ms * 1e-3) / 1e12
+    value = job_value(dense_flops, world, ms * 1e-3)
     if args.layer_only:  # the timed steps only (for profiler launch lists)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -336,12 +351,8 @@ def run_dyra(args):
         layer.forward(X, B=s.B, T=s.T, Y=Y)
         Yh.copy_(Y, non_blocking=True)
 
-    e2e_ms = timed(e2e_step, args.steps, 2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = dense_flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(timed(e2e_step, args.steps, 2), world, dev)
+    e2e_value = job_value(dense_flops, world, e2e_ms * 1e-3)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

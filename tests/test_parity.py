@@ -292,11 +292,17 @@ def test_rank_deficient_is_an_error():
     layer.close()
 
 
-def test_zero_input_without_ridge_flags_pivot():
-    """X_b = 0 and lambda = 0 make L^T L = 0: the solve flags the pivot and
-    drops that instance's correction, leaving the weight-only output (0)."""
+@pytest.mark.parametrize("placement", ["solve", "gram"])
+def test_zero_input_without_ridge_flags_pivot(placement):
+    """X_b = 0 and lambda = 0 make L^T L = 0: the factorisation (in the solve,
+    or once per instance in the Gram stage) flags the pivot and drops that
+    instance's correction, leaving the weight-only output (0)."""
     s, f = _small(k=32, lam=0.0, B=2, T=64)
-    layer = make_layer(s, f)
+    os.environ["DYRA_FACTOR"] = placement
+    try:
+        layer = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_FACTOR")
     X = torch.zeros(128, 256, device="cuda", dtype=torch.bfloat16)
     Y = layer.forward(X, B=2, T=64)
     st = layer.status()
