@@ -41,7 +41,9 @@ struct Bf16Forward {
   void* Tp;              // (B*k) x d_in
   void* Ct;              // d_out x (B*k)
   float* MD;             // B factor records (factor_record_floats(k) floats each), or nullptr
-  int* counters;         // B arrival counters of the split Gram tiles (with MD)
+  int* counters;         // B ints: the solve's per-instance flags, or the Gram stage's
+                         // arrival counters (factor_in_gram); cleared by the projection
+  bool factor_in_gram;   // factor G_b in the Gram stage's epilogue instead of the solve
   int splits;            // row splits of the Gram reduction
   int split_rows;        // rows per split (multiple of 64)
   int* status;
@@ -84,11 +86,14 @@ template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStream_t s);
 
 // Solve (L^T L + lambda I) T' = T for every instance from the Gram partials.
-// MD: per-instance factor records (ldl_panel.cuh) written by the Gram stage
-// (k <= 64 only), or nullptr to factor G_b inside the solve.
+// mode 0: every solve block factors G_b itself (MD, flags unused);
+// mode 1: one block per instance factors G_b and publishes the factor record
+//         in MD (ldl_panel.cuh layout) behind flags[b], which must be zero at
+//         launch; mode 2: the Gram stage wrote the records (k <= 64 only for
+//         modes 1 and 2).
 template <typename TOut>
-int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k, int d_in,
-                 float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
+int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, int64_t B, int k,
+                 int d_in, float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
                  unsigned long long* trace = nullptr);
 
 // Floats per instance of the factor records for correction rank k (0 when

@@ -130,18 +130,22 @@ __global__ void __launch_bounds__(kSolveThreads)
 
 // ---------------------------------------------------------------------------
 // Fast path for k <= 64. grid (B, ceil(d_in / 128)), 256 threads; each CTA
-// handles a 128-column chunk of T_b:
-//  1. loads: either the instance's factor record (M, D^-1 and the failure
-//     flag, written once per instance by the Gram stage) or, when there is
-//     none (kFactored false), G_b summed over the row splits; the T chunk's
-//     first split is requested at the same time and lands during step 2;
-//  2. (kFactored false) G_b + lambda I = Lt D Lt^T by the panel elimination
-//     of ldl_panel.cuh, giving M = Lt^-1 and D; then the T chunk, summed
-//     over the splits, goes to shared memory;
-//  3. T' = M^T D^-1 (M T): two small products over the chunk, no sequential
-//     dependency (same accuracy as the two triangular solves).
+// handles a 128-column chunk of T_b. G_b + lambda I = Lt D Lt^T by the panel
+// elimination of ldl_panel.cuh gives M = Lt^-1 and D; the CTA then applies
+// T' = M^T D^-1 (M T) to its chunk: two small products, no sequential
+// dependency (same accuracy as the two triangular solves). Who factors:
+//  - kSolveSelf: every CTA factors G_b itself (the fp32 path);
+//  - kSolveShared: the instance's first CTA (chunk 0) factors G_b, writes the
+//    factor record (M, D^-1, failure flag) and raises the instance's flag;
+//    the other CTAs load their T chunk meanwhile, wait for the flag (bounded)
+//    and read the record. The first CTAs of the grid are the factoring ones,
+//    so a waiting CTA's producer has always been scheduled before it;
+//  - kSolvePrefactored: the Gram stage wrote the records; every CTA reads one.
+// The T chunk's first split is requested before the factorisation and lands
+// while it runs; the other splits are added afterwards.
 constexpr int kSolveThreads2 = 256;
 constexpr int kSolveCols = 128;  // columns of T_b per CTA
+enum SolveMode { kSolveSelf = 0, kSolveShared = 1, kSolvePrefactored = 2 };
 
 template <int KMAX>
 struct SolveSmem {
@@ -151,17 +155,17 @@ struct SolveSmem {
   float Mr[KMAX * LDM];                 // Mr[i][q] = M[i][q]
   float Mc[KMAX * LDM];                 // Mc[q][i] = M[i][q]
   float dinv[KMAX];
-  LdlScratch<KMAX> ldl;
+  LdlBlockScratch<KMAX> ldl;
   int bad;
 };
 
-template <typename TOut, int KMAX, bool kFactored>
+template <typename TOut, int KMAX, int MODE>
 __global__ void __launch_bounds__(kSolveThreads2)
-    solve_ldl_kernel(const float* __restrict__ TG, const float* __restrict__ MD, int S, int B,
-                     int k, int d_in, float lambda, TOut* __restrict__ Tp, int* status,
+    solve_ldl_kernel(const float* __restrict__ TG, float* MD, int* flags, int S, int B, int k,
+                     int d_in, float lambda, TOut* __restrict__ Tp, int* status,
                      unsigned long long* trace) {
   using Sm = SolveSmem<KMAX>;
-  constexpr int LDG = LdlScratch<KMAX>::LDG;
+  constexpr int LDG = LdlBlockScratch<KMAX>::LD;
   extern __shared__ __align__(16) unsigned char smem_bytes[];
   Sm& sm = *reinterpret_cast<Sm*>(smem_bytes);
   constexpr int GPT = KMAX * KMAX / kSolveThreads2;
@@ -172,15 +176,16 @@ __global__ void __launch_bounds__(kSolveThreads2)
   const int J = d_in + k;
   const int c0 = blockIdx.y * kSolveCols;
   const size_t inst = static_cast<size_t>(k) * J;
+  const bool factors = MODE == kSolveSelf || (MODE == kSolveShared && blockIdx.y == 0);
+  float* rec = MODE == kSolveSelf ? nullptr : MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
   unsigned long long* const tr =
       trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
   if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
   sm100::pdl_wait();
   if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
 
-  // ---- 1. loads. G_b (or the factor record) goes to shared memory first;
-  // the first split's T chunk is requested at the same time but only stored
-  // after the elimination, which runs while those loads are in flight.
+  // ---- 1. loads: the first split of the T chunk (kept in registers until
+  // after the factorisation), then G_b or, prefactored, the factor record
   const float* part = TG + static_cast<size_t>(b) * inst;
   float t[TPT];
 #pragma unroll
@@ -189,66 +194,57 @@ __global__ void __launch_bounds__(kSolveThreads2)
     const int i = idx / kSolveCols, c = idx % kSolveCols;
     t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
   }
-  {
-    const float* rec = MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
+  if (factors) {
     float g[GPT];
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {
       const int idx = tid + u * kSolveThreads2;
       const int i = idx / KMAX, q = idx % KMAX;
-      if constexpr (kFactored)
-        g[u] = rec[idx];
-      else
-        g[u] = (i < k && q < k) ? part[static_cast<size_t>(i) * J + d_in + q] : 0.f;
+      g[u] = (i < k && q < k) ? part[static_cast<size_t>(i) * J + d_in + q] : 0.f;
     }
-    float dv = 0.f;
-    int bad = 0;
-    if constexpr (kFactored) {
-      if (tid < KMAX) dv = rec[KMAX * KMAX + tid];
-      if (tid == 0) bad = rec[KMAX * KMAX + KMAX] != 0.f;
-    } else {
-      for (int sp = 1; sp < S; ++sp) {
-        const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
+    for (int sp = 1; sp < S; ++sp) {
+      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
 #pragma unroll
-        for (int u = 0; u < GPT; ++u) {
-          const int idx = tid + u * kSolveThreads2;
-          const int i = idx / KMAX, q = idx % KMAX;
-          if (i < k && q < k) g[u] += ps[static_cast<size_t>(i) * J + d_in + q];
-        }
+      for (int u = 0; u < GPT; ++u) {
+        const int idx = tid + u * kSolveThreads2;
+        const int i = idx / KMAX, q = idx % KMAX;
+        if (i < k && q < k) g[u] += ps[static_cast<size_t>(i) * J + d_in + q];
       }
     }
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {
       const int idx = tid + u * kSolveThreads2;
       const int i = idx / KMAX, q = idx % KMAX;
-      if constexpr (kFactored) {
-        sm.Mr[i * Sm::LDM + q] = g[u];
-        sm.Mc[q * Sm::LDM + i] = g[u];
-      } else {
-        sm.ldl.Gs[i * LDG + q] =
-            (i < k && q < k) ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
-      }
+      sm.ldl.Gs[i * LDG + q] =
+          (i < k && q < k) ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
     }
-    if constexpr (kFactored) {
-      if (tid < KMAX) sm.dinv[tid] = dv;
-      if (tid == 0) sm.bad = bad;
-    } else {
-      if (tid == 0) sm.bad = 0;
-    }
+    if (tid == 0) sm.bad = 0;
   }
   __syncthreads();
   if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
 
-  // ---- 2. elimination on [G | I]
-  if constexpr (!kFactored) {
-    const bool ok = ldl_eliminate<KMAX, kSolveThreads2>(
+  // ---- 2. the factorisation (factoring CTAs), published for the others
+  if (factors) {
+    const bool ok = ldl_blocked<KMAX, kSolveThreads2>(
         sm.ldl, k, tid, [] { __syncthreads(); },
         [&](int i, int q, float v) {
           sm.Mr[i * Sm::LDM + q] = v;
           sm.Mc[q * Sm::LDM + i] = v;
+          if (MODE == kSolveShared) rec[i * KMAX + q] = v;
         },
-        [&](int j, float v) { sm.dinv[j] = v; });
-    if (!ok && tid == 0) sm.bad = 1;
+        [&](int j, float v) {
+          sm.dinv[j] = v;
+          if (MODE == kSolveShared) rec[KMAX * KMAX + j] = v;
+        });
+    if (tid == 0) {
+      if (!ok) sm.bad = 1;
+      if (MODE == kSolveShared) rec[KMAX * KMAX + KMAX] = ok ? 0.f : 1.f;
+    }
+    if (MODE == kSolveShared) {
+      __threadfence();  // this thread's part of the record, before the flag
+      __syncthreads();
+      if (tid == 0) sm100::st_release_gpu(flags + b, 1);
+    }
   }
   // the remaining splits of the T chunk
   for (int sp = 1; sp < S; ++sp) {
@@ -262,6 +258,38 @@ __global__ void __launch_bounds__(kSolveThreads2)
   }
 #pragma unroll
   for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
+  if (!factors) {
+    // the record: ready at launch (prefactored) or once the flag is up
+    if (MODE == kSolveShared) {
+      if (tid == 0) {
+        int bad = 0;
+        const unsigned long long deadline = sm100::globaltimer_ns() + sm100::kWaitLimitNs;
+        while (sm100::ld_acquire_gpu(flags + b) == 0) {
+          if (sm100::globaltimer_ns() > deadline) {
+            atomicOr(status, sm100::kStatusTimeout);
+            bad = 1;
+            break;
+          }
+          __nanosleep(128);
+        }
+        sm.bad = bad;
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / KMAX, q = idx % KMAX;
+      const float m = __ldcg(rec + idx);
+      sm.Mr[i * Sm::LDM + q] = m;
+      sm.Mc[q * Sm::LDM + i] = m;
+    }
+    if (tid < KMAX) sm.dinv[tid] = __ldcg(rec + KMAX * KMAX + tid);
+    if (tid == 0) {
+      const bool failed = __ldcg(rec + KMAX * KMAX + KMAX) != 0.f;
+      sm.bad = (MODE == kSolveShared ? sm.bad : 0) | (failed ? 1 : 0);
+    }
+  }
   __syncthreads();
   if (tr && tid == 0) tr[4] = sm100::globaltimer_ns();
 
@@ -328,7 +356,8 @@ __global__ void __launch_bounds__(kSolveThreads2)
     for (int v = 0; v < 4; ++v)
       if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : acc[u][v]);
   }
-  if (!kFactored && tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
+  if (MODE != kSolvePrefactored && tid == 0 && blockIdx.y == 0 && zero)
+    atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
   sm100::pdl_launch_dependents();
@@ -415,11 +444,11 @@ __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P,
 
 }  // namespace
 
-template <typename TOut, int KMAX, bool kFactored>
-int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, const float* MD, int splits,
+template <typename TOut, int KMAX, int MODE>
+int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, float* MD, int* flags, int splits,
                      int64_t B, int k, int d_in, float lambda, TOut* Tp, int* status,
                      unsigned long long* trace) {
-  auto kfn = solve_ldl_kernel<TOut, KMAX, kFactored>;
+  auto kfn = solve_ldl_kernel<TOut, KMAX, MODE>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -429,21 +458,42 @@ int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, const float* MD, 
       return -1;
     configured = true;
   }
+  // blockIdx.x = instance, blockIdx.y = chunk: the chunk-0 CTAs (the ones
+  // that factor in the shared mode) are the grid's first B CTAs.
   cfg.gridDim = dim3(static_cast<unsigned>(B),
                      static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
   cfg.blockDim = dim3(kSolveThreads2);
   cfg.dynamicSmemBytes = sizeof(SolveSmem<KMAX>);
-  return cudaLaunchKernelEx(&cfg, kfn, TG, MD, splits, static_cast<int>(B), k, d_in, lambda, Tp,
-                            status, trace) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, kfn, TG, MD, flags, splits, static_cast<int>(B), k, d_in,
+                            lambda, Tp, status, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
+template <typename TOut, int KMAX>
+int launch_solve_mode(cudaLaunchConfig_t& cfg, int mode, const float* TG, float* MD, int* flags,
+                      int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
+                      int* status, unsigned long long* trace) {
+  switch (mode) {
+    case kSolveShared:
+      return launch_solve_ldl<TOut, KMAX, kSolveShared>(cfg, TG, MD, flags, splits, B, k, d_in,
+                                                         lambda, Tp, status, trace);
+    case kSolvePrefactored:
+      return launch_solve_ldl<TOut, KMAX, kSolvePrefactored>(cfg, TG, MD, flags, splits, B, k,
+                                                              d_in, lambda, Tp, status, trace);
+    default:
+      return launch_solve_ldl<TOut, KMAX, kSolveSelf>(cfg, TG, MD, flags, splits, B, k, d_in,
+                                                       lambda, Tp, status, trace);
+  }
+}
+
 template <typename TOut>
-int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k, int d_in,
-                 float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
+int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, int64_t B, int k,
+                 int d_in, float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
                  unsigned long long* trace) {
   if (B == 0 || k == 0) return 0;
+  if (mode != kSolveSelf && (MD == nullptr || (mode == kSolveShared && flags == nullptr)))
+    return -1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -452,15 +502,11 @@ int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k,
   cfg.numAttrs = pdl ? 1 : 0;
   cfg.stream = s;
   if (k <= 32)
-    return MD ? launch_solve_ldl<TOut, 32, true>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
-                                                 status, trace)
-              : launch_solve_ldl<TOut, 32, false>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
-                                                  status, trace);
+    return launch_solve_mode<TOut, 32>(cfg, mode, TG, MD, flags, splits, B, k, d_in, lambda, Tp,
+                                       status, trace);
   if (k <= 64)
-    return MD ? launch_solve_ldl<TOut, 64, true>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
-                                                 status, trace)
-              : launch_solve_ldl<TOut, 64, false>(cfg, TG, MD, splits, B, k, d_in, lambda, Tp,
-                                                  status, trace);
+    return launch_solve_mode<TOut, 64>(cfg, mode, TG, MD, flags, splits, B, k, d_in, lambda, Tp,
+                                       status, trace);
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
@@ -480,9 +526,9 @@ int launch_solve(const float* TG, const float* MD, int splits, int64_t B, int k,
              : -1;
 }
 
-template int launch_solve<float>(const float*, const float*, int, int64_t, int, int, float, float*, int*,
+template int launch_solve<float>(const float*, float*, int*, int, int, int64_t, int, int, float, float*, int*,
                                  cudaStream_t, bool, unsigned long long*);
-template int launch_solve<__nv_bfloat16>(const float*, const float*, int, int64_t, int, int, float,
+template int launch_solve<__nv_bfloat16>(const float*, float*, int*, int, int, int64_t, int, int, float,
                                          __nv_bfloat16*, int*, cudaStream_t, bool,
                                          unsigned long long*);
 
@@ -523,7 +569,7 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
              s))
       return -1;
-    if (launch_solve<T>(a.TG, nullptr, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+    if (launch_solve<T>(a.TG, nullptr, nullptr, 0, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
       return -1;
     // C = T' W_res^T  (B*k x d_out)
     if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,

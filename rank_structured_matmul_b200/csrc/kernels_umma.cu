@@ -114,7 +114,7 @@ struct ProjPolicy {
     int tma_store;    // r % 64 == 0 and k <= 64: every 64-column box is all Z or all L
     __nv_bfloat16* Z;
     __nv_bfloat16* L;
-    int* cnt;         // the Gram stage's arrival counters, cleared here (or nullptr)
+    int* cnt;         // the per-instance flags or counters of later stages, cleared here (or nullptr)
     int ncnt;
   };
   struct Tile {
@@ -217,7 +217,7 @@ struct GramPolicy {
     int mt, b, s, t0, t1;
   };
   // Elimination scratch, plus the "last arrival" flag.
-  static constexpr uint32_t kFlagOffset = sizeof(LdlScratch<64>);
+  static constexpr uint32_t kFlagOffset = sizeof(LdlBlockScratch<64>);
   static constexpr uint32_t kEpiSmemBytes = (kFlagOffset + 16 + 1023) / 1024 * 1024;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
@@ -288,7 +288,7 @@ struct GramPolicy {
     // factorisation straight from the accumulator.
     const bool factor = p.kmax > 0 && t.mt >= p.mtx;
     const bool stage = factor && p.S == 1 && valid;
-    const int ldg = p.kmax + 1;
+    const int ldg = p.kmax + 1;  // LdlBlockScratch<kmax>::LD
     float* gs = reinterpret_cast<float*>(e.smem) + (jcol - p.d_in) * ldg;
     for (int cc = 0; cc < p.kpad; cc += 32) {
       uint32_t v[32];
@@ -319,8 +319,8 @@ struct GramPolicy {
   // instance's factor record: M = Lt^-1, D^-1 and a failure flag.
   template <int KMAX>
   static __device__ __noinline__ void factor_instance(const Params& p, const Tile& t, EpiCtx& e) {
-    auto& sm = *reinterpret_cast<LdlScratch<KMAX>*>(e.smem);
-    constexpr int LDG = LdlScratch<KMAX>::LDG;
+    auto& sm = *reinterpret_cast<LdlBlockScratch<KMAX>*>(e.smem);
+    constexpr int LDG = LdlBlockScratch<KMAX>::LD;
     volatile int* last = reinterpret_cast<volatile int*>(e.smem + kFlagOffset);
     const int k = p.k;
     if (p.S > 1) {
@@ -350,7 +350,7 @@ struct GramPolicy {
     }
     named_bar_sync(2, 128);
     float* rec = p.MD + static_cast<size_t>(t.b) * ldl_record_floats<KMAX>();
-    const bool ok = ldl_eliminate<KMAX, 128>(
+    const bool ok = ldl_blocked<KMAX, 128>(
         sm, k, e.tid, [] { named_bar_sync(2, 128); },
         [&](int i, int q, float v) { rec[i * KMAX + q] = v; },
         [&](int j, float v) { rec[KMAX * KMAX + j] = v; });
@@ -750,8 +750,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     p.n_tiles_n = ceil_div(n_cols, p.bn);
     p.Z = static_cast<__nv_bfloat16*>(a.Z);
     p.L = static_cast<__nv_bfloat16*>(a.L);
-    const bool factor_in_gram = p.k > 0 && a.MD && factor_record_floats(p.k) > 0;
-    p.cnt = factor_in_gram ? a.counters : nullptr;
+    const bool records = p.k > 0 && a.MD && a.counters && factor_record_floats(p.k) > 0;
+    p.cnt = records ? a.counters : nullptr;
     p.ncnt = static_cast<int>(a.B);
     uint64_t dx[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(N)};
     uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
@@ -811,7 +811,9 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.mt_total = p.mtx + ceil_div(a.k, 128);
       p.J = J;
       p.TG = a.TG;
-      p.kmax = a.MD && factor_record_floats(a.k) > 0 ? (a.k <= 32 ? 32 : 64) : 0;
+      p.kmax = a.factor_in_gram && a.MD && a.counters && factor_record_floats(a.k) > 0
+                   ? (a.k <= 32 ? 32 : 64)
+                   : 0;
       p.lambda = a.lambda;
       p.MD = a.MD;
       p.cnt = a.counters;
@@ -839,9 +841,12 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     }
     mark(2);
     // ------------------------------------------------------------- solve
-    const float* md = a.MD && factor_record_floats(a.k) > 0 ? a.MD : nullptr;
-    if (launch_solve<__nv_bfloat16>(a.TG, md, a.splits, a.B, a.k, a.d_in, a.lambda,
-                                    static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
+    // once per instance: in the Gram stage (mode 2) or by the instance's
+    // first solve block (mode 1); without records every block factors (0)
+    const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
+    const int mode = !records ? 0 : (a.factor_in_gram ? 2 : 1);
+    if (launch_solve<__nv_bfloat16>(a.TG, a.MD, a.counters, mode, a.splits, a.B, a.k, a.d_in,
+                                    a.lambda, static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
                                     a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
     mark(3);

@@ -239,29 +239,40 @@ def test_pair_output_stage_matches_single_cta():
     pair.close()
 
 
-@pytest.mark.parametrize("k,B,T", [(32, 3, 201), (64, 2, 150), (24, 1, 3000), (64, 1, 3000)])
-def test_factor_in_gram_matches_factor_in_solve(k, B, T):
-    """Factoring G_b once in the Gram stage (DYRA_FACTOR=gram; one split, or
-    the last of several splits to arrive) gives the same layer as factoring it
-    in every solve block, also on a second call (the arrival counters start
-    from zero again)."""
+def _layer_with_factor(s, f, placement):
+    """placement: 'shared' (default: the first solve block of each instance
+    factors G_b), 'gram' (the Gram stage factors it) or 'self' (every solve
+    block factors it)."""
+    if placement != "shared":
+        os.environ["DYRA_FACTOR"] = placement
+    try:
+        return make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_FACTOR", None)
+
+
+@pytest.mark.parametrize("placement", ["gram", "self"])
+@pytest.mark.parametrize("k,B,T", [(32, 3, 201), (64, 2, 150), (24, 1, 3000), (64, 1, 3000),
+                                   (32, 40, 64)])
+def test_factor_placements_agree(placement, k, B, T):
+    """G_b factored once per instance by the first solve block (default), once
+    in the Gram stage (one split, or the last of several splits to arrive), or
+    by every solve block gives the same layer, also on a second call (the
+    per-instance flags and counters start from zero again)."""
     s, f = _small(k=k, B=B, T=T)
     X = to_dev(f["X"], "bf16")
-    os.environ["DYRA_FACTOR"] = "gram"
-    try:
-        in_gram = make_layer(s, f)
-    finally:
-        os.environ.pop("DYRA_FACTOR")
-    in_solve = make_layer(s, f)
-    Ys = in_solve.forward(X, B=s.B, T=s.T)
-    Yg1 = in_gram.forward(X, B=s.B, T=s.T)
-    Yg2 = in_gram.forward(X, B=s.B, T=s.T)
-    assert in_gram.status() == 0 and in_solve.status() == 0
-    assert torch.equal(Yg1, Yg2)
-    assert oracle.rel_fro(Yg1.double().cpu().numpy(), Ys.double().cpu().numpy()) <= 1e-3
-    check(s, Yg1, f)
-    in_gram.close()
-    in_solve.close()
+    other = _layer_with_factor(s, f, placement)
+    shared = _layer_with_factor(s, f, "shared")
+    Ys1 = shared.forward(X, B=s.B, T=s.T)
+    Ys2 = shared.forward(X, B=s.B, T=s.T)
+    Yo1 = other.forward(X, B=s.B, T=s.T)
+    Yo2 = other.forward(X, B=s.B, T=s.T)
+    assert other.status() == 0 and shared.status() == 0
+    assert torch.equal(Ys1, Ys2) and torch.equal(Yo1, Yo2)
+    assert oracle.rel_fro(Yo1.double().cpu().numpy(), Ys1.double().cpu().numpy()) <= 1e-3
+    check(s, Ys1, f)
+    other.close()
+    shared.close()
 
 
 def test_forward_inside_caller_graph_capture():
@@ -292,17 +303,13 @@ def test_rank_deficient_is_an_error():
     layer.close()
 
 
-@pytest.mark.parametrize("placement", ["solve", "gram"])
+@pytest.mark.parametrize("placement", ["shared", "gram", "self"])
 def test_zero_input_without_ridge_flags_pivot(placement):
-    """X_b = 0 and lambda = 0 make L^T L = 0: the factorisation (in the solve,
-    or once per instance in the Gram stage) flags the pivot and drops that
-    instance's correction, leaving the weight-only output (0)."""
+    """X_b = 0 and lambda = 0 make L^T L = 0: the factorisation (wherever it
+    runs) flags the pivot and drops that instance's correction, leaving the
+    weight-only output (0)."""
     s, f = _small(k=32, lam=0.0, B=2, T=64)
-    os.environ["DYRA_FACTOR"] = placement
-    try:
-        layer = make_layer(s, f)
-    finally:
-        os.environ.pop("DYRA_FACTOR")
+    layer = _layer_with_factor(s, f, placement)
     X = torch.zeros(128, 256, device="cuda", dtype=torch.bfloat16)
     Y = layer.forward(X, B=2, T=64)
     st = layer.status()
