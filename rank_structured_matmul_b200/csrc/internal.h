@@ -62,6 +62,15 @@ void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits
 
 int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s);
 
+// Tiling of the projection stage X [V | P] for N rows (k_eff = 0 for the
+// weight-only layer): column tile, tile count, CTA pairs or not, and the
+// split-K factor chosen when there are too few tiles for the SMs.
+struct ProjShape {
+  int bn, n_tiles_n, tiles, ksplit, kper, tma_store;
+  bool pairs;
+};
+ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count);
+
 // ------------------------------------------------------- SIMT (fp32) ----
 
 template <typename T>

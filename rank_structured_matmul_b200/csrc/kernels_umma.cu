@@ -116,9 +116,16 @@ struct ProjPolicy {
     __nv_bfloat16* L;
     int* cnt;         // the per-instance flags or counters of later stages, cleared here (or nullptr)
     int ncnt;
+    // Split-K for skinny N (ksplit > 1): the ksplit CTAs of output tile
+    // `base` form one cluster; CTA ks takes k-iterations [ks * kper,
+    // (ks + 1) * kper) and leaves its fp32 partial tile in its own shared
+    // memory; after a cluster barrier each CTA sums the partials of its slice
+    // of rows over distributed shared memory, in split order, and stores Z
+    // and L. One tile per CTA.
+    int ksplit, kper;
   };
   struct Tile {
-    int m0, n0;
+    int m0, n0, ks, base;
   };
   static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
@@ -131,19 +138,23 @@ struct ProjPolicy {
     }
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
-    t.m0 = (tile / p.n_tiles_n) * 128;
-    t.n0 = (tile % p.n_tiles_n) * p.bn;
+    t.base = tile / p.ksplit;
+    t.ks = tile - t.base * p.ksplit;
+    t.m0 = (t.base / p.n_tiles_n) * 128;
+    t.n0 = (t.base % p.n_tiles_n) * p.bn;
   }
-  static __device__ __forceinline__ int kiters(const Params& p, const Tile&) {
-    return ceil_div_dev(p.d_in, 64);
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    const int total = ceil_div_dev(p.d_in, 64);
+    return p.ksplit > 1 ? min(p.kper, total - t.ks * p.kper) : total;
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
-    tma_load_2d(sa, &p.tmX, bar, it * 64, t.m0);
-    tma_load_2d(sb, &p.tmW, bar, it * 64, t.n0);
+    const int kg = t.ks * p.kper + it;
+    tma_load_2d(sa, &p.tmX, bar, kg * 64, t.m0);
+    tma_load_2d(sb, &p.tmW, bar, kg * 64, t.n0);
   }
-  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
-    return min(4, ceil_div_dev(p.d_in - it * 64, 16));
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
+    return min(4, ceil_div_dev(p.d_in - (t.ks * p.kper + it) * 64, 16));
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
     return kmajor_desc(a, ks);
@@ -158,6 +169,10 @@ struct ProjPolicy {
     if (p.cnt && t.m0 == 0 && t.n0 == 0)
       for (int i = e.tid; i < p.ncnt; i += 128) p.cnt[i] = 0;
     const int rk = p.r + p.k;
+    if (p.ksplit > 1) {
+      split_epilogue(p, t, tacc, e);
+      return;
+    }
     if (p.tma_store) {
       for (int bx = 0; bx < p.bn / 64; ++bx) {
         const int col = t.n0 + bx * 64;
@@ -188,8 +203,88 @@ struct ProjPolicy {
       }
     }
   }
+  // Split-K, first half: the partial tile into this CTA's operand stages,
+  // column-major in float4 units ([c4][row]: a warp writes 512 contiguous
+  // bytes, and the reads below are conflict-free too).
+  static __device__ __forceinline__ void split_epilogue(const Params& p, const Tile&,
+                                                        uint32_t tacc, EpiCtx& e) {
+    float4* part = reinterpret_cast<float4*>(e.stage);
+    for (int cc = 0; cc < p.bn; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + cc, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        part[(cc / 4 + g) * 128 + e.row] =
+            make_float4(f32(v[4 * g]), f32(v[4 * g + 1]), f32(v[4 * g + 2]), f32(v[4 * g + 3]));
+    }
+    if (e.tr && e.tid == 0) e.tr[kTrSplitWritten] = globaltimer_ns();
+  }
+  static __device__ __forceinline__ bool cluster_finish(const Params& p) { return p.ksplit > 1; }
+  // Split-K, second half (after the cluster barrier): this CTA's slice of
+  // rows, summed over the cluster's partials in split order.
+  static __device__ __noinline__ void finish(const Params& p, int tid, uint32_t stage_u32,
+                                             unsigned long long* tr) {
+    if (tr && tid == 0) tr[kTrSplitArrived] = globaltimer_ns();
+    const int ks_me = static_cast<int>(cluster_ctarank());
+    Tile t;
+    decode(p, static_cast<int>(blockIdx.x), t);
+    const int rk = p.r + p.k, c4n = p.bn / 4;
+    const int rs = (128 + p.ksplit - 1) / p.ksplit;
+    const int row0 = ks_me * rs, nrows = min(128, row0 + rs) - row0;
+    const int nitems = nrows > 0 ? nrows * c4n : 0;
+    for (int i0 = tid; i0 < nitems; i0 += 2 * 128) {
+      uint32_t off[2];
+      bool valid[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = i0 + u * 128;
+        valid[u] = it < nitems;
+        const int c4 = valid[u] ? it / nrows : 0;
+        const int row = valid[u] ? row0 + (it - c4 * nrows) : row0;
+        off[u] = static_cast<uint32_t>(c4 * 128 + row);
+      }
+      float4 acc[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ks = 0; ks < p.ksplit; ks += 4) {
+        float4 v[4][2];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t peer = static_cast<uint32_t>(min(ks + j, p.ksplit - 1));
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            v[j][u] = ld_shared_cluster_v4(mapa_shared(stage_u32 + 16u * off[u], peer));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (ks + j < p.ksplit)
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              acc[u].x += v[j][u].x;
+              acc[u].y += v[j][u].y;
+              acc[u].z += v[j][u].z;
+              acc[u].w += v[j][u].w;
+            }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!valid[u]) continue;
+        const int c4 = static_cast<int>(off[u]) / 128, row = static_cast<int>(off[u]) - c4 * 128;
+        const int grow = t.m0 + row, col = t.n0 + 4 * c4;
+        if (grow >= p.N || col >= rk) continue;
+        __nv_bfloat16* dst = col < p.r ? p.Z + static_cast<size_t>(grow) * p.r + col
+                                       : p.L + static_cast<size_t>(grow) * p.k + (col - p.r);
+        uint2 w;
+        w.x = pack_bf16x2(acc[u].x, acc[u].y);
+        w.y = pack_bf16x2(acc[u].z, acc[u].w);
+        *reinterpret_cast<uint2*>(dst) = w;
+      }
+    }
+    if (tr && tid == 0) tr[kTrSplitReduced] = globaltimer_ns();
+  }
   static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
-    if (p.tma_store) store_drain(e);
+    if (p.tma_store && p.ksplit <= 1) store_drain(e);
   }
 };
 
@@ -359,6 +454,8 @@ struct GramPolicy {
       if (!ok) atomicOr(p.c.status, kStatusPivot);
     }
   }
+  static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
+  static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
 };
 
@@ -409,6 +506,8 @@ struct RFactorPolicy {
     for (int bx = 0; bx < p.bn / 64; ++bx)
       store_box_bf16(tacc, bx * 64, &p.tmC, t.n0 + bx * 64, t.m0, e);
   }
+  static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
+  static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) { store_drain(e); }
 };
 
@@ -489,6 +588,8 @@ struct OutPolicy {
     for (int bx = 0; bx < p.bn / 64; ++bx)
       store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e);
   }
+  static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
+  static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) { store_drain(e); }
 };
 
@@ -503,6 +604,8 @@ struct ProjPairPolicy {
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 256;
     t.n0 = (tile % p.n_tiles_n) * p.bn;
+    t.ks = 0;
+    t.base = tile;
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
     return ProjPolicy::kiters(p, t);
@@ -523,7 +626,7 @@ struct ProjPairPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    Tile h{t.m0 + 128 * e.rank, t.n0};
+    Tile h{t.m0 + 128 * e.rank, t.n0, 0, t.base};
     ProjPolicy::epilogue(p, h, tacc, e);
   }
   static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
@@ -636,7 +739,7 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
 
 template <class Pol>
 int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& dev,
-                cudaStream_t s, bool pdl) {
+                cudaStream_t s, bool pdl, int cluster = 1) {
   if (p.c.num_tiles <= 0) return 0;
   auto kfn = umma_gemm_kernel<Pol>;
   static uint32_t configured = 0;
@@ -649,15 +752,29 @@ int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& 
     configured = smem;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(std::min(p.c.num_tiles, dev.sm_count)));
+  // with clusters every CTA takes exactly one tile (the grid is the tile count)
+  cfg.gridDim = dim3(static_cast<unsigned>(
+      cluster > 1 ? p.c.num_tiles : std::min(p.c.num_tiles, dev.sm_count)));
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster > 1) {
+    if (p.c.num_tiles % cluster != 0) return -1;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = static_cast<unsigned>(na);
   return cudaLaunchKernelEx(&cfg, kfn, p) == cudaSuccess ? 0 : -1;
 }
 
@@ -706,6 +823,30 @@ int pick_bn(int n) {
 
 }  // namespace
 
+ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count) {
+  ProjShape ps;
+  const int n_cols = r + k_eff;
+  ps.tma_store = (r % 64 == 0 && k_eff <= 64) ? 1 : 0;
+  ps.bn = pick_bn(n_cols);
+  if (ps.tma_store) ps.bn = std::min(256, (ps.bn + 63) / 64 * 64);  // whole 64-column boxes
+  ps.n_tiles_n = ceil_div(n_cols, ps.bn);
+  // Pairs pay a longer set-up; they win once each pair streams several tiles.
+  ps.pairs = use_pairs && ps.bn % 32 == 0 && ps.bn >= 64 &&
+             ceil_div(N, 256) * ps.n_tiles_n >= sm_count;
+  ps.tiles = static_cast<int>(ps.pairs ? ceil_div(N, 256) : ceil_div(N, 128)) * ps.n_tiles_n;
+  ps.ksplit = 1;
+  const int kit = ceil_div(d_in, 64);
+  ps.kper = kit;
+  if (!ps.pairs && ps.tiles * 2 <= sm_count && kit >= 8) {
+    int want = std::min(sm_count / ps.tiles, std::min(kit / 4, 8));  // portable cluster size
+    if (want > 1) {
+      ps.kper = ceil_div(kit, want);
+      ps.ksplit = ceil_div(kit, ps.kper);
+    }
+  }
+  return ps;
+}
+
 int factor_record_floats(int k) {
   if (k <= 0 || k > 64) return 0;
   return k <= 32 ? ldl_record_floats<32>() : ldl_record_floats<64>();
@@ -739,29 +880,28 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   // ---------------------------------------------------------------- proj
   {
     ProjPolicy::Params p;
-    const int n_cols = a.weight_only ? a.r : rk;
+    const int k_eff = a.weight_only ? 0 : a.k;
+    const ProjShape ps = proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count);
     p.N = static_cast<int>(N);
     p.d_in = a.d_in;
     p.r = a.r;
-    p.k = a.weight_only ? 0 : a.k;
-    p.tma_store = (a.r % 64 == 0 && p.k <= 64) ? 1 : 0;
-    p.bn = pick_bn(n_cols);
-    if (p.tma_store) p.bn = std::min(256, (p.bn + 63) / 64 * 64);  // whole 64-column boxes
-    p.n_tiles_n = ceil_div(n_cols, p.bn);
+    p.k = k_eff;
+    p.tma_store = ps.tma_store;
+    p.bn = ps.bn;
+    p.n_tiles_n = ps.n_tiles_n;
     p.Z = static_cast<__nv_bfloat16*>(a.Z);
     p.L = static_cast<__nv_bfloat16*>(a.L);
     const bool records = p.k > 0 && a.MD && a.counters && factor_record_floats(p.k) > 0;
     p.cnt = records ? a.counters : nullptr;
     p.ncnt = static_cast<int>(a.B);
+    p.ksplit = ps.ksplit;
+    p.kper = ps.kper;
     uint64_t dx[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(N)};
     uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
     uint32_t bx[2] = {64, 128};
     if (!encode_tmap_bf16(&p.tmX, a.X, 2, dx, sx, bx, 128)) return -2;
-    // Pairs pay a longer set-up; they win once each pair streams several tiles.
-    const bool proj_pairs = a.use_pairs && p.bn % 32 == 0 && p.bn >= 64 &&
-                            ceil_div(N, 256) * p.n_tiles_n >= dev.sm_count;
     uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(rk)};
-    uint32_t bw[2] = {64, static_cast<uint32_t>(proj_pairs ? p.bn / 2 : p.bn)};
+    uint32_t bw[2] = {64, static_cast<uint32_t>(ps.pairs ? p.bn / 2 : p.bn)};
     if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
     uint32_t bs[2] = {64, 128};
     uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
@@ -774,21 +914,24 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     } else {
       p.tmL = p.tmZ;
     }
-    if (proj_pairs) {
-      const int tiles = ceil_div(N, 256) * p.n_tiles_n;
-      const uint32_t smem = setup_common<ProjPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
-                                                         p.bn, false, false, a.status, dev);
+    if (ps.pairs) {
+      const uint32_t smem = setup_common<ProjPairPolicy>(p.c, ps.tiles, 128 * 128,
+                                                         (p.bn / 2) * 128, p.bn, false, false,
+                                                         a.status, dev);
       if (!smem) return -3;
       p.c.idesc = idesc_bf16(256, p.bn, false, false);
       if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
       if (launch_gemm_pair<ProjPairPolicy>(p, smem, dev, s, pdl)) return -1;
     } else {
-      const int tiles = ceil_div(N, 128) * p.n_tiles_n;
-      const uint32_t smem = setup_common<ProjPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
-                                                     false, false, a.status, dev);
+      const uint32_t smem = setup_common<ProjPolicy>(p.c, ps.tiles * p.ksplit, 128 * 128,
+                                                     p.bn * 128, p.bn, false, false, a.status, dev);
       if (!smem) return -3;
+      // split-K keeps a 128 x bn fp32 partial in the operand stages
+      if (p.ksplit > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
+                              static_cast<size_t>(128) * p.bn * 4)
+        return -3;
       if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
-      if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl, p.ksplit)) return -1;
     }
   }
   mark(1);
@@ -896,6 +1039,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     p.n_tiles_n = ceil_div(a.d_out, p.bn);
     p.nkz = ceil_div(a.r, 64);
     p.nkl = k > 0 ? ceil_div(k, 64) : 0;
+
     uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
     uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
     uint32_t bz[2] = {64, 128};

@@ -49,7 +49,10 @@ enum TraceSlot {
   kTrEpiFirst = 7,     // epilogue saw its first finished accumulator
   kTrExit = 8,         // all roles done, before TMEM is freed
   kTrTileDone = 9,     // + i: epilogue finished its i-th tile (i < 27)
-  kTrTileMma = 36      // + i: MMA thread committed its i-th tile (i < 28)
+  kTrTileMma = 36,     // + i: MMA thread committed its i-th tile (i < 24)
+  kTrSplitWritten = 60,  // split-K: partial tile written and fenced
+  kTrSplitArrived = 61,  // split-K: every split of the tile has arrived
+  kTrSplitReduced = 62   // split-K: this split's slice is reduced and stored
 };
 
 struct GemmCommon {
@@ -73,6 +76,10 @@ struct EpiCtx {
   uint32_t smem_u32;  // same, as a shared-window address
   uint32_t counter;   // running counter the policy may use (e.g. store buffers)
   int rank;           // CTA of the pair (0 for single-CTA kernels)
+  unsigned long long* tr;  // this CTA's timeline row, or nullptr
+  uint8_t* stage;          // the operand stages (free once the CTA's last MMA is complete)
+  uint32_t stage_u32;
+  uint32_t stage_bytes;
 };
 
 __host__ __device__ inline uint32_t gemm_smem_bytes(int stages, uint32_t a_bytes,
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mma_commit(tfull_bar(acc));
         if (tr) {
           tr[kTrLastCommit] = globaltimer_ns();
-          if (local < kTraceSlots - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
+          if (local < kTrSplitWritten - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
         }
       }
       // All MMAs issued by this thread are complete before TMEM is freed.
@@ -237,6 +244,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     e.smem_u32 = sEpi;
     e.counter = 0;
     e.rank = 0;
+    e.tr = tr;
+    e.stage = smem;
+    e.stage_u32 = sA;
+    e.stage_bytes = static_cast<uint32_t>(S) * (c.a_stage_bytes + c.b_stage_bytes);
     int local = 0;
     for (int tile = blockIdx.x; tile < c.num_tiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -257,7 +268,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     Pol::epilogue_drain(p, e);
   }
-
+  // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
+  // that each warp arrives at the barrier once, with all its lanes (an
+  // aligned barrier reached by a diverged warp would count it twice and let
+  // the CTA past before the epilogue warps are done with TMEM).
+  __syncwarp();
+  // A policy whose tiles end in a cluster-wide step (split-K partials summed
+  // over distributed shared memory) runs it here: every CTA of the cluster has
+  // finished its tile when the first barrier opens, and none leaves before
+  // the others have read its shared memory.
+  if (Pol::cluster_finish(p)) {
+    cluster_sync_all();
+    if (warp >= 2) Pol::finish(p, threadIdx.x - 64, sA, tr);
+    cluster_sync_all();
+  }
   __syncthreads();
   if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();
   if (warp == 1) {

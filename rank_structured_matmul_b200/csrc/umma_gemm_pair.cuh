@@ -170,7 +170,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         mma_commit_pair(tfull_bar(acc));
         if (tr) {
           tr[kTrLastCommit] = globaltimer_ns();
-          if (local < kTraceSlots - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
+          if (local < kTrSplitWritten - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
         }
       }
       mma_commit_pair(fin_bar);
@@ -186,6 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     e.smem_u32 = sEpi;
     e.counter = 0;
     e.rank = static_cast<int>(rank);
+    e.tr = tr;
     int local = 0;
     for (int tile = pair; tile < c.num_tiles; tile += npairs, ++local) {
       const int acc = local & 1;
@@ -206,7 +207,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     Pol::epilogue_drain(p, e);
   }
-
+  // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
+  // that each warp arrives at the barrier once, with all its lanes (an
+  // aligned barrier reached by a diverged warp would count it twice and let
+  // the CTA past before the epilogue warps are done with TMEM).
+  __syncwarp();
   __syncthreads();
   cluster_sync_all();  // the leader's MMAs into both TMEMs are complete
   if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();

@@ -275,6 +275,28 @@ def test_factor_placements_agree(placement, k, B, T):
     shared.close()
 
 
+@pytest.mark.parametrize("d_in,B,T", [(1024, 1, 64), (2048, 2, 40), (4096, 1, 1)])
+def test_projection_split_k(d_in, B, T):
+    """Few row tiles and a long K: the projection splits K across the CTAs of
+    a cluster, which sum their fp32 partials over distributed shared memory
+    in split order. Repeated calls agree bit for bit, and the weight-only
+    layer (another tiling of the same stage) stays right."""
+    s = LayerSpec("sk", d_in, 512, 256, 32, B, T, "bf16", 0.7, "lognormal", seed=5, lam=1e-3)
+    f = prepared(s)
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    Y1 = layer.forward(X, B=s.B, T=s.T)
+    Y2 = layer.forward(X, B=s.B, T=s.T)
+    Ywo = layer.forward_weight_only(X)
+    Y3 = layer.forward(X, B=s.B, T=s.T)
+    assert layer.status() == 0
+    assert torch.equal(Y1, Y2) and torch.equal(Y1, Y3)
+    check(s, Y1, f)
+    wo = oracle.weight_only(f["X"], f["U"], f["V"])
+    assert oracle.rel_fro(Ywo.double().cpu().numpy(), wo) <= 1e-2
+    layer.close()
+
+
 def test_forward_inside_caller_graph_capture():
     """A forward issued while the caller captures its stream is recorded into
     the caller's graph (the workspace is reserved beforehand)."""

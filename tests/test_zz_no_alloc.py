@@ -61,6 +61,13 @@ def test_noalloc_matches_workspace_forward_bf16():
                        seed=7))
 
 
+def test_noalloc_matches_workspace_forward_split_k_projection():
+    """Few rows and a long K: the projection splits K across a cluster of
+    CTAs; the allocation-free forward agrees with the workspace forward."""
+    _compare(LayerSpec("noalloc_sk", 2048, 512, 256, 32, 1, 64, "bf16", 0.7, "lognormal",
+                       seed=7))
+
+
 def test_noalloc_matches_workspace_forward_fp32():
     _compare(LayerSpec("noalloc_f32", 256, 256, 32, 8, 2, 64, "f32", 1.0, "outlier",
                        n_outlier=4, outlier_scale=20.0, seed=7))
