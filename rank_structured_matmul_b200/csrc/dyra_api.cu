@@ -25,9 +25,7 @@ struct dyra_plan {
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
   bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
   // Where G_b is factored (bf16, k <= 64): once per instance by the first solve
-  // block (default), in the Gram stage (DYRA_FACTOR=gram), or by every solve
-  // block (DYRA_FACTOR=self, for comparison).
-  bool factor_in_gram = false;
+  // block (default), or by every solve block (DYRA_FACTOR=self, for comparison).
   bool factor_self = false;
   float lambda = 0.f;
   // packed factors
@@ -289,7 +287,6 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Ct = p->Ct;
     split_factor_buffer(correct && !p->factor_self ? p->MD : nullptr, B, p->k, &a.MD,
                         &a.counters);
-    a.factor_in_gram = p->factor_in_gram;
     a.splits = 1;
     a.split_rows = 64;
     if (correct) dyra::gram_split(T, B, p->d_in, p->k, p->dev.sm_count, &a.splits, &a.split_rows);
@@ -448,7 +445,6 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   const char* pv = std::getenv("DYRA_PAIR");
   p->use_pairs = !(pv != nullptr && pv[0] == '0');
   const char* fv = std::getenv("DYRA_FACTOR");
-  p->factor_in_gram = fv != nullptr && std::strcmp(fv, "gram") == 0;
   p->factor_self = fv != nullptr && std::strcmp(fv, "self") == 0;
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
@@ -788,7 +784,6 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     void* fac = k > 0 ? carve.take(factor_bytes(B, k)) : nullptr;
     split_factor_buffer(p->factor_self ? nullptr : fac, B, k, &a.MD, &a.counters);
-    a.factor_in_gram = p->factor_in_gram;
     a.splits = splits;
     a.split_rows = split_rows;
     a.status = p->status;

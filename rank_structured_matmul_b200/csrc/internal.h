@@ -41,9 +41,7 @@ struct Bf16Forward {
   void* Tp;              // (B*k) x d_in
   void* Ct;              // d_out x (B*k)
   float* MD;             // B factor records (factor_record_floats(k) floats each), or nullptr
-  int* counters;         // B ints: the solve's per-instance flags, or the Gram stage's
-                         // arrival counters (factor_in_gram); cleared by the projection
-  bool factor_in_gram;   // factor G_b in the Gram stage's epilogue instead of the solve
+  int* counters;         // B ints: the solve's per-instance flags; cleared by the projection
   int splits;            // row splits of the Gram reduction
   int split_rows;        // rows per split (multiple of 64)
   int* status;
@@ -98,8 +96,7 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStre
 // mode 0: every solve block factors G_b itself (MD, flags unused);
 // mode 1: one block per instance factors G_b and publishes the factor record
 //         in MD (ldl_panel.cuh layout) behind flags[b], which must be zero at
-//         launch; mode 2: the Gram stage wrote the records (k <= 64 only for
-//         modes 1 and 2).
+//         launch (k <= 64 only).
 template <typename TOut>
 int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, int64_t B, int k,
                  int d_in, float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,

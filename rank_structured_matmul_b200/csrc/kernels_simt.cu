@@ -139,13 +139,12 @@ __global__ void __launch_bounds__(kSolveThreads)
 //    factor record (M, D^-1, failure flag) and raises the instance's flag;
 //    the other CTAs load their T chunk meanwhile, wait for the flag (bounded)
 //    and read the record. The first CTAs of the grid are the factoring ones,
-//    so a waiting CTA's producer has always been scheduled before it;
-//  - kSolvePrefactored: the Gram stage wrote the records; every CTA reads one.
+//    so a waiting CTA's producer has always been scheduled before it.
 // The T chunk's first split is requested before the factorisation and lands
 // while it runs; the other splits are added afterwards.
 constexpr int kSolveThreads2 = 256;
 constexpr int kSolveCols = 128;  // columns of T_b per CTA
-enum SolveMode { kSolveSelf = 0, kSolveShared = 1, kSolvePrefactored = 2 };
+enum SolveMode { kSolveSelf = 0, kSolveShared = 1 };
 
 template <int KMAX>
 struct SolveSmem {
@@ -185,7 +184,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
   if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
 
   // ---- 1. loads: the first split of the T chunk (kept in registers until
-  // after the factorisation), then G_b or, prefactored, the factor record
+  // after the factorisation), then G_b (factoring CTAs)
   const float* part = TG + static_cast<size_t>(b) * inst;
   float t[TPT];
 #pragma unroll
@@ -259,8 +258,8 @@ __global__ void __launch_bounds__(kSolveThreads2)
 #pragma unroll
   for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
   if (!factors) {
-    // the record: ready at launch (prefactored) or once the flag is up
-    if (MODE == kSolveShared) {
+    // the record, once the flag is up
+    {
       if (tid == 0) {
         int bad = 0;
         const unsigned long long deadline = sm100::globaltimer_ns() + sm100::kWaitLimitNs;
@@ -287,7 +286,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
     if (tid < KMAX) sm.dinv[tid] = __ldcg(rec + KMAX * KMAX + tid);
     if (tid == 0) {
       const bool failed = __ldcg(rec + KMAX * KMAX + KMAX) != 0.f;
-      sm.bad = (MODE == kSolveShared ? sm.bad : 0) | (failed ? 1 : 0);
+      sm.bad = sm.bad | (failed ? 1 : 0);
     }
   }
   __syncthreads();
@@ -356,8 +355,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
     for (int v = 0; v < 4; ++v)
       if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : acc[u][v]);
   }
-  if (MODE != kSolvePrefactored && tid == 0 && blockIdx.y == 0 && zero)
-    atomicOr(status, sm100::kStatusPivot);
+  if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
   sm100::pdl_launch_dependents();
@@ -478,9 +476,6 @@ int launch_solve_mode(cudaLaunchConfig_t& cfg, int mode, const float* TG, float*
     case kSolveShared:
       return launch_solve_ldl<TOut, KMAX, kSolveShared>(cfg, TG, MD, flags, splits, B, k, d_in,
                                                          lambda, Tp, status, trace);
-    case kSolvePrefactored:
-      return launch_solve_ldl<TOut, KMAX, kSolvePrefactored>(cfg, TG, MD, flags, splits, B, k,
-                                                              d_in, lambda, Tp, status, trace);
     default:
       return launch_solve_ldl<TOut, KMAX, kSolveSelf>(cfg, TG, MD, flags, splits, B, k, d_in,
                                                        lambda, Tp, status, trace);

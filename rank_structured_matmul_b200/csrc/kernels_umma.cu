@@ -302,26 +302,19 @@ struct GramPolicy {
     int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total, J;
     uint32_t b_layout;
     float* TG;
-    // Factorisation of G_b + lambda I (k <= 64): kmax 32 or 64, else 0.
-    int kmax;
-    float lambda;
-    float* MD;  // B factor records (ldl_panel.cuh)
-    int* cnt;   // B arrival counters, zero at kernel start (the projection clears them)
   };
   struct Tile {
     int mt, b, s, t0, t1;
   };
-  // Elimination scratch, plus the "last arrival" flag.
-  static constexpr uint32_t kFlagOffset = sizeof(LdlBlockScratch<64>);
-  static constexpr uint32_t kEpiSmemBytes = (kFlagOffset + 16 + 1023) / 1024 * 1024;
+  static constexpr uint32_t kEpiSmemBytes = 0;
 
   static __device__ __forceinline__ void prefetch(const Params& p) {
     tma_prefetch_desc(&p.tmX);
     tma_prefetch_desc(&p.tmLa);
     tma_prefetch_desc(&p.tmLb);
   }
-  // Tiles of G (the m-tiles over L's columns) come first, so that their
-  // factorisation overlaps the T tiles of the other CTAs.
+  // Tiles of G (the m-tiles over L's columns) come first: the solve's
+  // factoring blocks read them first.
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     const int mtl = p.mt_total - p.mtx;
     const int ng = mtl * p.B * p.S;
@@ -379,12 +372,6 @@ struct GramPolicy {
       valid = i2 < p.k;
     }
     float* out = p.TG + static_cast<size_t>(t.s * p.B + t.b) * p.k * p.J + jcol;
-    // With a single split the tile holds all of G_b: stage it for the
-    // factorisation straight from the accumulator.
-    const bool factor = p.kmax > 0 && t.mt >= p.mtx;
-    const bool stage = factor && p.S == 1 && valid;
-    const int ldg = p.kmax + 1;  // LdlBlockScratch<kmax>::LD
-    float* gs = reinterpret_cast<float*>(e.smem) + (jcol - p.d_in) * ldg;
     for (int cc = 0; cc < p.kpad; cc += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tacc + cc, v);
@@ -393,65 +380,9 @@ struct GramPolicy {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int i = cc + jj;
-          if (i < p.k) {
-            out[static_cast<size_t>(i) * p.J] = f32(v[jj]);
-            if (stage) gs[i] = f32(v[jj]);
-          }
+          if (i < p.k) out[static_cast<size_t>(i) * p.J] = f32(v[jj]);
         }
       }
-    }
-    if (factor) {
-      if (p.kmax == 32)
-        factor_instance<32>(p, t, e);
-      else
-        factor_instance<64>(p, t, e);
-    }
-  }
-  // G_b + lambda I = Lt D Lt^T on the 128 epilogue threads, once per
-  // instance: by this tile if it holds all of G_b (one split), else by the
-  // tile whose partial arrives last, which sums the splits' partials in split
-  // order (so the result does not depend on the arrival order). Writes the
-  // instance's factor record: M = Lt^-1, D^-1 and a failure flag.
-  template <int KMAX>
-  static __device__ __noinline__ void factor_instance(const Params& p, const Tile& t, EpiCtx& e) {
-    auto& sm = *reinterpret_cast<LdlBlockScratch<KMAX>*>(e.smem);
-    constexpr int LDG = LdlBlockScratch<KMAX>::LD;
-    volatile int* last = reinterpret_cast<volatile int*>(e.smem + kFlagOffset);
-    const int k = p.k;
-    if (p.S > 1) {
-      __threadfence();  // this thread's partial is visible before the arrival
-      named_bar_sync(2, 128);
-      if (e.tid == 0) *last = atomicAdd(p.cnt + t.b, 1) == p.S - 1;
-      named_bar_sync(2, 128);
-      if (!*last) return;
-      __threadfence();
-      for (int idx = e.tid; idx < k * k; idx += 128) {
-        const int i = idx / k, q = idx - (idx / k) * k;
-        const float* src = p.TG + static_cast<size_t>(t.b) * k * p.J +
-                           static_cast<size_t>(i) * p.J + p.d_in + q;
-        float g = 0.f;
-        for (int sp = 0; sp < p.S; ++sp)
-          g += __ldcg(src + static_cast<size_t>(sp) * p.B * k * p.J);
-        sm.Gs[i * LDG + q] = g;
-      }
-    }
-    named_bar_sync(2, 128);
-    for (int idx = e.tid; idx < KMAX * KMAX; idx += 128) {
-      const int i = idx / KMAX, q = idx % KMAX;
-      if (i >= k || q >= k)
-        sm.Gs[i * LDG + q] = i == q ? 1.f : 0.f;
-      else if (i == q)
-        sm.Gs[i * LDG + q] += p.lambda;
-    }
-    named_bar_sync(2, 128);
-    float* rec = p.MD + static_cast<size_t>(t.b) * ldl_record_floats<KMAX>();
-    const bool ok = ldl_blocked<KMAX, 128>(
-        sm, k, e.tid, [] { named_bar_sync(2, 128); },
-        [&](int i, int q, float v) { rec[i * KMAX + q] = v; },
-        [&](int j, float v) { rec[KMAX * KMAX + j] = v; });
-    if (e.tid == 0) {
-      rec[KMAX * KMAX + KMAX] = ok ? 0.f : 1.f;
-      if (!ok) atomicOr(p.c.status, kStatusPivot);
     }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
@@ -954,12 +885,6 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.mt_total = p.mtx + ceil_div(a.k, 128);
       p.J = J;
       p.TG = a.TG;
-      p.kmax = a.factor_in_gram && a.MD && a.counters && factor_record_floats(a.k) > 0
-                   ? (a.k <= 32 ? 32 : 64)
-                   : 0;
-      p.lambda = a.lambda;
-      p.MD = a.MD;
-      p.cnt = a.counters;
       p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
       uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
                         static_cast<uint64_t>(a.B)};
@@ -984,10 +909,10 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     }
     mark(2);
     // ------------------------------------------------------------- solve
-    // once per instance: in the Gram stage (mode 2) or by the instance's
-    // first solve block (mode 1); without records every block factors (0)
+    // once per instance by the instance's first solve block (mode 1); without
+    // records every block factors G_b itself (mode 0)
     const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
-    const int mode = !records ? 0 : (a.factor_in_gram ? 2 : 1);
+    const int mode = records ? 1 : 0;
     if (launch_solve<__nv_bfloat16>(a.TG, a.MD, a.counters, mode, a.splits, a.B, a.k, a.d_in,
                                     a.lambda, static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
                                     a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))

@@ -241,8 +241,7 @@ def test_pair_output_stage_matches_single_cta():
 
 def _layer_with_factor(s, f, placement):
     """placement: 'shared' (default: the first solve block of each instance
-    factors G_b), 'gram' (the Gram stage factors it) or 'self' (every solve
-    block factors it)."""
+    factors G_b) or 'self' (every solve block factors it)."""
     if placement != "shared":
         os.environ["DYRA_FACTOR"] = placement
     try:
@@ -251,14 +250,13 @@ def _layer_with_factor(s, f, placement):
         os.environ.pop("DYRA_FACTOR", None)
 
 
-@pytest.mark.parametrize("placement", ["gram", "self"])
+@pytest.mark.parametrize("placement", ["self"])
 @pytest.mark.parametrize("k,B,T", [(32, 3, 201), (64, 2, 150), (24, 1, 3000), (64, 1, 3000),
                                    (32, 40, 64)])
 def test_factor_placements_agree(placement, k, B, T):
-    """G_b factored once per instance by the first solve block (default), once
-    in the Gram stage (one split, or the last of several splits to arrive), or
-    by every solve block gives the same layer, also on a second call (the
-    per-instance flags and counters start from zero again)."""
+    """G_b factored once per instance by the first solve block (default) or by
+    every solve block gives the same layer, also on a second call (the
+    per-instance flags start from zero again)."""
     s, f = _small(k=k, B=B, T=T)
     X = to_dev(f["X"], "bf16")
     other = _layer_with_factor(s, f, placement)
@@ -325,7 +323,7 @@ def test_rank_deficient_is_an_error():
     layer.close()
 
 
-@pytest.mark.parametrize("placement", ["shared", "gram", "self"])
+@pytest.mark.parametrize("placement", ["shared", "self"])
 def test_zero_input_without_ridge_flags_pivot(placement):
     """X_b = 0 and lambda = 0 make L^T L = 0: the factorisation (wherever it
     runs) flags the pivot and drops that instance's correction, leaving the
