@@ -24,6 +24,7 @@ struct dyra_plan {
   bool loaded = false;
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
   bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
+  int proj_pair_min_tiles = 0;  // DYRA_PROJ_PAIR_MIN=n: projection pairs from n pair tiles
   // Where G_b is factored (bf16, k <= 64): once per instance by the first solve
   // block (default), or by every solve block (DYRA_FACTOR=self, for comparison).
   bool factor_self = false;
@@ -294,6 +295,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
     a.trace = p->trace;
     a.use_pairs = p->use_pairs;
+    a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     rc = launch_bf16_maybe_graph(p, a, s);
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
@@ -444,6 +446,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   p->force_simt = kv != nullptr && std::strcmp(kv, "simt") == 0;
   const char* pv = std::getenv("DYRA_PAIR");
   p->use_pairs = !(pv != nullptr && pv[0] == '0');
+  const char* ppv = std::getenv("DYRA_PROJ_PAIR_MIN");
+  p->proj_pair_min_tiles = ppv ? std::atoi(ppv) : 0;
   const char* fv = std::getenv("DYRA_FACTOR");
   p->factor_self = fv != nullptr && std::strcmp(fv, "self") == 0;
   const char* gv = std::getenv("DYRA_GRAPHS");
@@ -790,6 +794,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.stage_events = nullptr;
     a.trace = nullptr;
     a.use_pairs = p->use_pairs;
+    a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;

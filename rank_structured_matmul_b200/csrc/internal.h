@@ -48,6 +48,7 @@ struct Bf16Forward {
   cudaEvent_t* stage_events;  // optional: 6 events recorded around the 5 stages
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
   bool use_pairs;             // run the output stage on CTA pairs
+  int proj_pair_min_tiles;    // see proj_shape (0: default)
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -67,7 +68,10 @@ struct ProjShape {
   int bn, n_tiles_n, tiles, ksplit, kper, tma_store;
   bool pairs;
 };
-ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count);
+// pair_min_tiles: pair tiles needed before the projection runs on CTA pairs
+// (0: a quarter of the SM count).
+ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count,
+                     int pair_min_tiles = 0);
 
 // ------------------------------------------------------- SIMT (fp32) ----
 

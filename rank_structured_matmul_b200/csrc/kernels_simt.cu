@@ -182,16 +182,38 @@ __global__ void __launch_bounds__(kSolveThreads2)
   if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
   sm100::pdl_wait();
   if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
+  // The next stage may be launched now: its blocks wait for this grid's
+  // results in their own pdl_wait and take SMs as these blocks leave.
+  sm100::pdl_launch_dependents();
 
   // ---- 1. loads: the first split of the T chunk (kept in registers until
   // after the factorisation), then G_b (factoring CTAs)
   const float* part = TG + static_cast<size_t>(b) * inst;
-  float t[TPT];
+  // bf16 plans (shared mode) have 16-byte TG rows: the first split goes
+  // straight to shared memory with asynchronous copies, holding no registers
+  // during the factorisation; otherwise it waits in registers.
+  constexpr bool kAsyncT = MODE == kSolveShared;
+  float t[kAsyncT ? 1 : TPT];
+  if constexpr (kAsyncT) {
+    constexpr int C4 = kSolveCols / 4;  // 16-byte chunks per row of the chunk
+    constexpr int CPT = KMAX * C4 / kSolveThreads2;
 #pragma unroll
-  for (int u = 0; u < TPT; ++u) {
-    const int idx = tid + u * kSolveThreads2;
-    const int i = idx / kSolveCols, c = idx % kSolveCols;
-    t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
+    for (int u = 0; u < CPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / C4, col = c0 + 4 * (idx % C4);
+      const int valid = i < k ? max(0, min(4, d_in - col)) : 0;
+      const float* src = valid ? part + static_cast<size_t>(i) * J + col : part;
+      sm100::cp_async_16(sm100::smem_u32(&sm.Tc[i * kSolveCols + (col - c0)]), src,
+                         static_cast<uint32_t>(valid) * 4u);
+    }
+    sm100::cp_async_commit();
+  } else {
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) {
+      const int idx = tid + u * kSolveThreads2;
+      const int i = idx / kSolveCols, c = idx % kSolveCols;
+      t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
+    }
   }
   if (factors) {
     float g[GPT];
@@ -246,17 +268,31 @@ __global__ void __launch_bounds__(kSolveThreads2)
     }
   }
   // the remaining splits of the T chunk
-  for (int sp = 1; sp < S; ++sp) {
-    const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
+  if constexpr (kAsyncT) {
+    sm100::cp_async_wait_all();
+    __syncthreads();  // every thread's copies have landed
+    for (int sp = 1; sp < S; ++sp) {
+      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
 #pragma unroll
-    for (int u = 0; u < TPT; ++u) {
-      const int idx = tid + u * kSolveThreads2;
-      const int i = idx / kSolveCols, c = idx % kSolveCols;
-      if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
+      for (int u = 0; u < TPT; ++u) {
+        const int idx = tid + u * kSolveThreads2;
+        const int i = idx / kSolveCols, c = idx % kSolveCols;
+        if (i < k && c0 + c < d_in) sm.Tc[idx] += ps[static_cast<size_t>(i) * J + c0 + c];
+      }
     }
-  }
+  } else {
+    for (int sp = 1; sp < S; ++sp) {
+      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
 #pragma unroll
-  for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
+      for (int u = 0; u < TPT; ++u) {
+        const int idx = tid + u * kSolveThreads2;
+        const int i = idx / kSolveCols, c = idx % kSolveCols;
+        if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
+  }
   if (!factors) {
     // the record, once the flag is up
     {
@@ -358,7 +394,6 @@ __global__ void __launch_bounds__(kSolveThreads2)
   if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
-  sm100::pdl_launch_dependents();
 }
 
 // C[b][m][n] (+)= sum_q A[b][m][q] * Bm[b][q][n] with arbitrary element strides.

@@ -754,16 +754,18 @@ int pick_bn(int n) {
 
 }  // namespace
 
-ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count) {
+ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count,
+                     int pair_min_tiles) {
   ProjShape ps;
   const int n_cols = r + k_eff;
   ps.tma_store = (r % 64 == 0 && k_eff <= 64) ? 1 : 0;
   ps.bn = pick_bn(n_cols);
   if (ps.tma_store) ps.bn = std::min(256, (ps.bn + 63) / 64 * 64);  // whole 64-column boxes
   ps.n_tiles_n = ceil_div(n_cols, ps.bn);
-  // Pairs pay a longer set-up; they win once each pair streams several tiles.
+  // Pairs halve each SM's B-operand traffic, which bounds this stage (bytes in
+  // flight per SM); they need enough pair tiles to keep the SMs busy.
   ps.pairs = use_pairs && ps.bn % 32 == 0 && ps.bn >= 64 &&
-             ceil_div(N, 256) * ps.n_tiles_n >= sm_count;
+             ceil_div(N, 256) * ps.n_tiles_n >= (pair_min_tiles > 0 ? pair_min_tiles : sm_count / 4);
   ps.tiles = static_cast<int>(ps.pairs ? ceil_div(N, 256) : ceil_div(N, 128)) * ps.n_tiles_n;
   ps.ksplit = 1;
   const int kit = ceil_div(d_in, 64);
@@ -812,7 +814,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   {
     ProjPolicy::Params p;
     const int k_eff = a.weight_only ? 0 : a.k;
-    const ProjShape ps = proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count);
+    const ProjShape ps =
+        proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count, a.proj_pair_min_tiles);
     p.N = static_cast<int>(N);
     p.d_in = a.d_in;
     p.r = a.r;

@@ -29,6 +29,20 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   return t;
 }
 
+// Asynchronous 16-byte global -> shared copy (L2 only); bytes beyond
+// src_bytes (0..16) are filled with zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Flag handshake between CTAs of one grid: the writer's earlier global stores
 // are visible to a reader that observes the flag (release / acquire, GPU scope).
 __device__ __forceinline__ void st_release_gpu(int* p, int v) {
