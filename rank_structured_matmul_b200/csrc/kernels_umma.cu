@@ -233,34 +233,33 @@ struct ProjPolicy {
     const int rs = (128 + p.ksplit - 1) / p.ksplit;
     const int row0 = ks_me * rs, nrows = min(128, row0 + rs) - row0;
     const int nitems = nrows > 0 ? nrows * c4n : 0;
-    for (int i0 = tid; i0 < nitems; i0 += 2 * 128) {
-      uint32_t off[2];
-      bool valid[2];
+    for (int i0 = tid; i0 < nitems; i0 += 4 * 128) {
+      uint32_t off[4];
+      bool valid[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < 4; ++u) {
         const int it = i0 + u * 128;
         valid[u] = it < nitems;
         const int c4 = valid[u] ? it / nrows : 0;
         const int row = valid[u] ? row0 + (it - c4 * nrows) : row0;
         off[u] = static_cast<uint32_t>(c4 * 128 + row);
       }
-      float4 acc[2];
+      float4 acc[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int ks = 0; ks < p.ksplit; ks += 4) {
-        float4 v[4][2];
+        float4 v[4][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint32_t peer = static_cast<uint32_t>(min(ks + j, p.ksplit - 1));
+          const uint32_t base = mapa_shared(stage_u32, static_cast<uint32_t>(min(ks + j, p.ksplit - 1)));
 #pragma unroll
-          for (int u = 0; u < 2; ++u)
-            v[j][u] = ld_shared_cluster_v4(mapa_shared(stage_u32 + 16u * off[u], peer));
+          for (int u = 0; u < 4; ++u) v[j][u] = ld_shared_cluster_v4(base + 16u * off[u]);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (ks + j < p.ksplit)
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < 4; ++u) {
               acc[u].x += v[j][u].x;
               acc[u].y += v[j][u].y;
               acc[u].z += v[j][u].z;
@@ -268,7 +267,7 @@ struct ProjPolicy {
             }
       }
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
+      for (int u = 0; u < 4; ++u) {
         if (!valid[u]) continue;
         const int c4 = static_cast<int>(off[u]) / 128, row = static_cast<int>(off[u]) - c4 * 128;
         const int grow = t.m0 + row, col = t.n0 + 4 * c4;
@@ -771,7 +770,15 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
   const int kit = ceil_div(d_in, 64);
   ps.kper = kit;
   if (!ps.pairs && ps.tiles * 2 <= sm_count && kit >= 8) {
-    int want = std::min(sm_count / ps.tiles, std::min(kit / 4, 8));  // portable cluster size
+    // Split-K: narrower column tiles first (more tiles, and half the fp32
+    // partial each CTA sums over the cluster), then up to 8 splits per tile
+    // (portable cluster size).
+    if (ps.bn > 128) {
+      ps.bn = 128;
+      ps.n_tiles_n = ceil_div(n_cols, ps.bn);
+      ps.tiles = static_cast<int>(ceil_div(N, 128)) * ps.n_tiles_n;
+    }
+    const int want = std::min(sm_count / ps.tiles, std::min(kit / 4, 8));
     if (want > 1) {
       ps.kper = ceil_div(kit, want);
       ps.ksplit = ceil_div(kit, ps.kper);
