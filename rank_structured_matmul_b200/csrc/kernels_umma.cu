@@ -524,6 +524,44 @@ struct OutPolicy {
 };
 
 // ============================================================ proj, pairs ====
+// C^T = W_res T'^T on CTA pairs: tile 256 x bn, CTA r loads rows m0 + 128 r
+// of W_res and rows n0 + (bn/2) r of T' and stores its 128 rows of C^T.
+struct RFactorPairPolicy {
+  using Params = RFactorPolicy::Params;  // tmT box is (64, bn/2) here
+  using Tile = RFactorPolicy::Tile;
+  static constexpr uint32_t kEpiSmemBytes = RFactorPolicy::kEpiSmemBytes;
+  static __device__ __forceinline__ void prefetch(const Params& p) { RFactorPolicy::prefetch(p); }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = (tile / p.n_tiles_n) * 256;
+    t.n0 = (tile % p.n_tiles_n) * p.bn;
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    return RFactorPolicy::kiters(p, t);
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar, uint32_t rank) {
+    tma_load_2d_pair(sa, &p.tmW, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
+    tma_load_2d_pair(sb, &p.tmT, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
+    return RFactorPolicy::ksteps(p, t, it);
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    Tile h{t.m0 + 128 * e.rank, t.n0};
+    RFactorPolicy::epilogue(p, h, tacc, e);
+  }
+  static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
+    RFactorPolicy::epilogue_drain(p, e);
+  }
+};
+
 // [Z | L] = X [V | P] on CTA pairs: tile 256 x bn, CTA r loads rows
 // m0 + 128 r of X and rows n0 + (bn/2) r of [V | P]^T and stores its 128 rows.
 struct ProjPairPolicy {
@@ -941,19 +979,33 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t sw[1] = {static_cast<uint64_t>(a.d_in) * 2};
       uint32_t bw[2] = {64, 128};
       if (!encode_tmap_bf16(&p.tmW, a.W_res, 2, dw, sw, bw, 128)) return -2;
+      // Pairs halve each SM's share of T' per k-step; they need enough pair
+      // tiles to keep the SMs busy and an even column tile.
+      const bool rf_pairs = a.use_pairs && p.bn % 32 == 0 && p.bn >= 64 &&
+                            ceil_div(a.d_out, 256) * p.n_tiles_n >= dev.sm_count / 4;
       uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
-      uint32_t bt[2] = {64, static_cast<uint32_t>(p.bn)};
+      uint32_t bt[2] = {64, static_cast<uint32_t>(rf_pairs ? p.bn / 2 : p.bn)};
       if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
       uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, 128};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
-      const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
-      const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
-                                                        false, false, a.status, dev);
-      if (!smem) return -3;
-      if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
-      if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (rf_pairs) {
+        const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
+        const uint32_t smem = setup_common<RFactorPairPolicy>(
+            p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false, false, a.status, dev);
+        if (!smem) return -3;
+        p.c.idesc = idesc_bf16(256, p.bn, false, false);
+        if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
+        if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
+      } else {
+        const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
+        const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128,
+                                                          p.bn, false, false, a.status, dev);
+        if (!smem) return -3;
+        if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
+        if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
+      }
     }
   } else {
     mark(2);
