@@ -256,15 +256,20 @@ __global__ void __launch_bounds__(kSolveThreads2)
         [&](int j, float v) {
           sm.dinv[j] = v;
           if (MODE == kSolveShared) rec[KMAX * KMAX + j] = v;
-        });
+        },
+        tr ? tr + 40 : nullptr);
     if (tid == 0) {
       if (!ok) sm.bad = 1;
       if (MODE == kSolveShared) rec[KMAX * KMAX + KMAX] = ok ? 0.f : 1.f;
     }
     if (MODE == kSolveShared) {
-      __threadfence();  // this thread's part of the record, before the flag
+      // the whole record before the flag: the barrier orders the block's
+      // writes before thread 0's fence, whose release covers them
       __syncthreads();
-      if (tid == 0) sm100::st_release_gpu(flags + b, 1);
+      if (tid == 0) {
+        __threadfence();
+        sm100::st_release_gpu(flags + b, 1);
+      }
     }
   }
   // the remaining splits of the T chunk
@@ -272,13 +277,17 @@ __global__ void __launch_bounds__(kSolveThreads2)
     sm100::cp_async_wait_all();
     __syncthreads();  // every thread's copies have landed
     for (int sp = 1; sp < S; ++sp) {
+      // all of a split's loads first, then the adds
       const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
+      float v[TPT];
 #pragma unroll
       for (int u = 0; u < TPT; ++u) {
         const int idx = tid + u * kSolveThreads2;
         const int i = idx / kSolveCols, c = idx % kSolveCols;
-        if (i < k && c0 + c < d_in) sm.Tc[idx] += ps[static_cast<size_t>(i) * J + c0 + c];
+        v[u] = (i < k && c0 + c < d_in) ? __ldg(ps + static_cast<size_t>(i) * J + c0 + c) : 0.f;
       }
+#pragma unroll
+      for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] += v[u];
     }
   } else {
     for (int sp = 1; sp < S; ++sp) {

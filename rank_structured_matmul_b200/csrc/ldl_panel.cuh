@@ -131,9 +131,20 @@ __device__ __forceinline__ void block16_mma(const float* A, const float* B, int 
 // emit_d(j, v) with v = 1 / D[j] for every j < KMAX. Returns false if a pivot
 // was <= 0 or not finite (the same answer in every thread). The block
 // products run one 16 x 16 block per warp.
+// ts (optional): a timeline row; thread 0 stamps %globaltimer into ts[2J] after
+// block column J's leaf and ts[2J + 1] after its trailing update, ts[8] after
+// the assembly of M and ts[9] after the emits.
 template <int KMAX, int NT, class Sync, class EmitM, class EmitD>
 __device__ __forceinline__ bool ldl_blocked(LdlBlockScratch<KMAX>& sm, int k, int tid, Sync sync,
-                                            EmitM emit_m, EmitD emit_d) {
+                                            EmitM emit_m, EmitD emit_d,
+                                            unsigned long long* ts = nullptr) {
+  auto stamp = [&](int slot) {
+    if (ts && tid == 0) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)::"memory");
+      ts[slot] = t;
+    }
+  };
   static_assert(KMAX == 32 || KMAX == 64, "blocked LDL needs KMAX 32 or 64");
   static_assert(NT % 32 == 0, "whole warps");
   constexpr int NB = KMAX / 16;
@@ -167,6 +178,7 @@ __device__ __forceinline__ bool ldl_blocked(LdlBlockScratch<KMAX>& sm, int k, in
       if (!ok && lane == 0) sm.bad = 1;
     }
     sync();
+    stamp(2 * J);
     if (J + 1 == NB) break;
     // panel: W_IJ = A_IJ M_JJ^T (into Wb) and L_IJ = W_IJ D_J^-1 (over A_IJ)
     for (int I = J + 1 + warp; I < NB; I += NW) {
@@ -204,6 +216,7 @@ __device__ __forceinline__ bool ldl_blocked(LdlBlockScratch<KMAX>& sm, int k, in
       }
     }
     sync();
+    stamp(2 * J + 1);
   }
   sync();  // identity-padded blocks above are written without a barrier of their own
   // M below the diagonal blocks: N_IP = -M_II L_IP (into Wb), then by distance
@@ -237,7 +250,9 @@ __device__ __forceinline__ bool ldl_blocked(LdlBlockScratch<KMAX>& sm, int k, in
     }
     sync();
   }
+  stamp(8);
   for (int e = tid; e < KMAX * KMAX; e += NT) emit_m(e / KMAX, e % KMAX, sm.Mb[(e / KMAX) * LD + e % KMAX]);
+  stamp(9);
   return sm.bad == 0;
 }
 
