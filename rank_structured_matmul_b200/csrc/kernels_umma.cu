@@ -832,14 +832,26 @@ int factor_record_floats(int k) {
 
 void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits,
                 int* split_rows) {
-  // Split each instance's rows only as far as needed to give every SM a
-  // tile; splits are whole 64-row blocks so no block straddles two splits.
+  // Split each instance's rows (whole 64-row blocks) to balance the tiles
+  // over the SMs: minimise (rounds of tiles per SM) x (blocks per tile),
+  // with a small charge per split for the fp32 partial sums it adds.
   const int64_t blocks = (T + 63) / 64;
   const int64_t mtiles = (d_in + 127) / 128 + (k + 127) / 128;
   const int64_t per_split_tiles = std::max<int64_t>(1, B * mtiles);
-  int64_t want = (sm_count + per_split_tiles - 1) / per_split_tiles;
-  want = std::max<int64_t>(1, std::min<int64_t>(want, blocks));
-  const int64_t per = (blocks + want - 1) / want;
+  int64_t best_s = 1;
+  double best = 0.0;
+  for (int64_t sp = 1; sp <= std::min<int64_t>(8, blocks); ++sp) {
+    const int64_t per = (blocks + sp - 1) / sp;
+    const int64_t used = (blocks + per - 1) / per;  // splits actually made
+    if (used != sp) continue;
+    const int64_t rounds = (per_split_tiles * sp + sm_count - 1) / sm_count;
+    const double cost = static_cast<double>(rounds * per) * (1.0 + 0.05 * static_cast<double>(sp));
+    if (sp == 1 || cost < best) {
+      best = cost;
+      best_s = sp;
+    }
+  }
+  const int64_t per = (blocks + best_s - 1) / best_s;
   *split_rows = static_cast<int>(per * 64);
   *splits = static_cast<int>((blocks + per - 1) / per);
 }
