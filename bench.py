@@ -36,8 +36,10 @@ sys.path.insert(0, ROOT)
 METRIC = "DyRA linear µs & dense-equiv TFLOP/s vs cuBLAS dense; % of roofline"
 UNIT = "TFLOP/s (dense-equivalent)"
 HEADLINE = "vit_fc1"
-STAGE_KERNELS = {"proj": "umma_gemm_kernel<ProjPolicy>", "gram": "umma_gemm_kernel<GramPolicy>",
-                 "solve": "solve_ldl_kernel", "rfactor": "umma_gemm_kernel<RFactorPolicy>",
+STAGE_KERNELS = {"proj": "ProjPolicy (CTA pairs, or split-K clusters at skinny N)",
+                 "gram": "umma_gemm_kernel<GramPolicy>",
+                 "solve": "solve_ldl_kernel",
+                 "rfactor": "RFactorPolicy (CTA pairs when there are enough tiles)",
                  "out": "umma_gemm_pair_kernel<OutPairPolicy>"}
 FLUSH_BYTES = 256 << 20
 
