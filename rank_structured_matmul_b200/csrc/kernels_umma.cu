@@ -796,14 +796,29 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
   ProjShape ps;
   const int n_cols = r + k_eff;
   ps.tma_store = (r % 64 == 0 && k_eff <= 64) ? 1 : 0;
-  ps.bn = pick_bn(n_cols);
-  if (ps.tma_store) ps.bn = std::min(256, (ps.bn + 63) / 64 * 64);  // whole 64-column boxes
-  ps.n_tiles_n = ceil_div(n_cols, ps.bn);
-  // Pairs halve each SM's B-operand traffic, which bounds this stage (bytes in
-  // flight per SM); they need enough pair tiles to keep the SMs busy.
-  ps.pairs = use_pairs && ps.bn % 32 == 0 && ps.bn >= 64 &&
-             ceil_div(N, 256) * ps.n_tiles_n >= (pair_min_tiles > 0 ? pair_min_tiles : sm_count / 4);
-  ps.tiles = static_cast<int>(ps.pairs ? ceil_div(N, 256) : ceil_div(N, 128)) * ps.n_tiles_n;
+  // Column tile and CTA pairs: the stage is bound by the bytes each CTA
+  // streams per k-step (128 rows of X, plus bn / 2 rows of [V | P]^T on a
+  // pair or bn rows alone) times the rounds of tiles per SM. Pick the
+  // cheapest of bn = 128, 192, 256 (whole 64-column store boxes).
+  const int pair_min = pair_min_tiles > 0 ? pair_min_tiles : sm_count / 4;
+  int64_t best = -1;
+  for (int bn : {192, 256, 128}) {
+    const int nt = ceil_div(n_cols, bn);
+    for (int pairs = 1; pairs >= 0; --pairs) {
+      if (pairs && !use_pairs) continue;
+      const int64_t tiles = (pairs ? ceil_div(N, 256) : ceil_div(N, 128)) * nt;
+      if (pairs && tiles < pair_min) continue;
+      const int64_t slots = pairs ? sm_count / 2 : sm_count;
+      const int64_t cost = (tiles + slots - 1) / slots * (128 + (pairs ? bn / 2 : bn));
+      if (best < 0 || cost < best) {
+        best = cost;
+        ps.bn = bn;
+        ps.n_tiles_n = nt;
+        ps.pairs = pairs != 0;
+        ps.tiles = static_cast<int>(tiles);
+      }
+    }
+  }
   ps.ksplit = 1;
   const int kit = ceil_div(d_in, 64);
   ps.kper = kit;
