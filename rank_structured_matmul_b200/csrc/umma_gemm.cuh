@@ -49,7 +49,10 @@ enum TraceSlot {
   kTrEpiFirst = 7,     // epilogue saw its first finished accumulator
   kTrExit = 8,         // all roles done, before TMEM is freed
   kTrTileDone = 9,     // + i: epilogue finished its i-th tile (i < 27)
-  kTrTileMma = 36,     // + i: MMA thread committed its i-th tile (i < 24)
+  kTrTileMma = 36,     // + i: MMA thread committed its i-th tile (i < 20)
+  kTrProducerDone = 56,  // producer's copies all landed
+  kTrMmaDone = 57,       // MMA thread's last MMA complete
+  kTrEpiDone = 58,       // epilogue warps done (before the closing barrier)
   kTrSplitWritten = 60,  // split-K: partial tile written and fenced
   kTrSplitArrived = 61,  // split-K: every split of the tile has arrived
   kTrSplitReduced = 62   // split-K: this split's slice is reduced and stored
@@ -151,13 +154,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
+  // producer state kept for the drain after the closing barrier
+  uint32_t last_phase[kMaxStages];
+  uint32_t issued = 0;
 
   if (warp == 0) {
     if (elect_one_sync()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t last_phase[kMaxStages];
-      uint32_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < c.num_tiles; tile += gridDim.x) {
         typename Pol::Tile t;
@@ -183,11 +187,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // Drain: every copy this thread issued has landed before the CTA leaves
-      // (one shared deadline for all slots).
-      const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
-      for (int s = 0; s < S; ++s)
-        if (issued & (1u << s)) (void)mbar_wait_until(full_bar(s), last_phase[s], deadline);
+      if (tr) tr[kTrProducerDone] = globaltimer_ns();
     }
   } else if (warp == 1) {
     if (elect_one_sync()) {
@@ -227,12 +227,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mma_commit(tfull_bar(acc));
         if (tr) {
           tr[kTrLastCommit] = globaltimer_ns();
-          if (local < kTrSplitWritten - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
+          if (local < kTrProducerDone - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
         }
       }
       // All MMAs issued by this thread are complete before TMEM is freed.
       mma_commit(fin_bar);
       (void)mbar_wait_until(fin_bar, 0, globaltimer_ns() + kWaitLimitNs);
+      if (tr) tr[kTrMmaDone] = globaltimer_ns();
     }
   } else {
     EpiCtx e;
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tr[kTrTileDone + local] = globaltimer_ns();
     }
     Pol::epilogue_drain(p, e);
+    if (tr && e.tid == 0) tr[kTrEpiDone] = globaltimer_ns();
   }
   // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
   // that each warp arrives at the barrier once, with all its lanes (an
@@ -283,6 +285,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     cluster_sync_all();
   }
   __syncthreads();
+  // Every copy the producer issued has landed before the CTA leaves: in a
+  // normal run the MMA thread waited for each of them, so only a run that
+  // gave up early drains here (one shared deadline for all slots).
+  if (warp == 0 && issued && *abort_flag) {
+    const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
+    for (int s = 0; s < S; ++s)
+      if (issued & (1u << s)) (void)mbar_wait_until(full_bar(s), last_phase[s], deadline);
+  }
   if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();
   if (warp == 1) {
     tc_fence_after();

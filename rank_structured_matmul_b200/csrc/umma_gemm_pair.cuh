@@ -92,13 +92,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
+  // producer state kept for the drain after the closing barrier
+  uint32_t last_phase[kMaxStages];
+  uint32_t issued = 0;
 
   if (warp == 0) {
     if (elect_one_sync()) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t last_phase[kMaxStages];
-      uint32_t issued = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < c.num_tiles; tile += npairs) {
         typename Pol::Tile t;
@@ -125,12 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      // The leader's full barriers also count the other CTA's copies.
-      if (leader) {
-        const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
-        for (int s = 0; s < S; ++s)
-          if (issued & (1u << s)) (void)mbar_wait_until(full_bar(s), last_phase[s], deadline);
-      }
+      if (tr) tr[kTrProducerDone] = globaltimer_ns();
     }
   } else if (warp == 1) {
     if (leader && elect_one_sync()) {
@@ -170,11 +166,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         mma_commit_pair(tfull_bar(acc));
         if (tr) {
           tr[kTrLastCommit] = globaltimer_ns();
-          if (local < kTrSplitWritten - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
+          if (local < kTrProducerDone - kTrTileMma) tr[kTrTileMma + local] = globaltimer_ns();
         }
       }
       mma_commit_pair(fin_bar);
       (void)mbar_wait_until(fin_bar, 0, globaltimer_ns() + kWaitLimitNs);
+      if (tr) tr[kTrMmaDone] = globaltimer_ns();
     }
   } else {
     EpiCtx e;
@@ -206,6 +203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tr[kTrTileDone + local] = globaltimer_ns();
     }
     Pol::epilogue_drain(p, e);
+    if (tr && e.tid == 0) tr[kTrEpiDone] = globaltimer_ns();
   }
   // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
   // that each warp arrives at the barrier once, with all its lanes (an
@@ -213,6 +211,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // the CTA past before the epilogue warps are done with TMEM).
   __syncwarp();
   __syncthreads();
+  // Every copy issued has landed before either CTA leaves. The leader's full
+  // barriers also count the other CTA's copies, and its MMA thread waited for
+  // each of them in a normal run, so only a leader that gave up early drains
+  // here, before the cluster barrier that holds the other CTA.
+  if (leader && warp == 0 && issued && *abort_flag) {
+    const unsigned long long deadline = globaltimer_ns() + kWaitLimitNs;
+    for (int s = 0; s < S; ++s)
+      if (issued & (1u << s)) (void)mbar_wait_until(full_bar(s), last_phase[s], deadline);
+  }
   cluster_sync_all();  // the leader's MMAs into both TMEMs are complete
   if (tr && threadIdx.x == 0) tr[kTrExit] = globaltimer_ns();
   if (warp == 1) {
