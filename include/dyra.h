@@ -129,18 +129,17 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
  * real-time loops where an allocation's implicit synchronisation or its
  * failure mid-run is not acceptable, or embedders that forbid the library
  * from allocating once set-up is over. Instead of the plan's workspace, this
- * call keeps the intermediates (X V, X P, the Gram partial sums, the solved
- * factor and C) in one fixed array of DYRA_STATIC_SCRATCH_BYTES (16 MiB)
+ * call keeps the intermediates (X V, X P, G_b, L_b^T X_b, the factor records
+ * and the rank-k factor) in one fixed array of DYRA_STATIC_SCRATCH_BYTES (16 MiB)
  * compiled into the library; every GPU that loads that part of the library
  * holds the array until the process exits.
  *   - Arguments, layouts and results are those of dyra_forward_batched; the
  *     plan (created and loaded beforehand) supplies the factors.
  *   - If the intermediates of B x T rows do not fit in the array the call
  *     returns DYRA_ERR_INVALID_ARG and enqueues nothing. For a bf16 plan they
- *     take about 2*B*T*(r+k) + 4*S*B*k*(d_in+k) + 2*B*k*(d_in+d_out) + 4*B*F
- *     bytes, each part rounded up to 256, where S is the number of row splits
- *     of the Gram stage (dyra_debug_gram_split in dyra_debug.h reports it) and
- *     F = K*K + K + 5 with K = 32 for k <= 32, 64 for k <= 64 (F = 0 above).
+ *     take about 2*B*T*(r+k) + 4*B*k*k + 2*B*k*(d_in+d_out) + 4*B*F bytes,
+ *     each part rounded up to 256, where F = K*K + K + 5 with K = 32 for
+ *     k <= 32, 64 for k <= 64 (F = 0 above).
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress); make that first call before capturing a stream
  *     into a CUDA graph.

@@ -25,9 +25,11 @@ struct dyra_plan {
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
   bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
   int proj_pair_min_tiles = 0;  // DYRA_PROJ_PAIR_MIN=n: projection pairs from n pair tiles
-  // Where G_b is factored (bf16, k <= 64): once per instance by the first solve
-  // block (default), or by every solve block (DYRA_FACTOR=self, for comparison).
-  bool factor_self = false;
+  // Where G_b is factored (bf16, k <= 64): by every solve block
+  // (DYRA_FACTOR=self), once per instance by the first solve block, which
+  // publishes it (DYRA_FACTOR=shared), or by size (unset: every block while
+  // the blocks fit the SMs).
+  int factor_mode = -1;
   float lambda = 0.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
@@ -36,7 +38,7 @@ struct dyra_plan {
   // workspace
   void* Z = nullptr;     // bf16: N x r; fp32: N x (r+k)
   void* L = nullptr;     // bf16: N x k
-  float* TG = nullptr;   // splits x B x k x (d_in + k)
+  float* TG = nullptr;   // bf16: B x k x k (G_b); fp32: B x k x (d_in + k) (T_b, G_b)
   void* Tp = nullptr;    // (B*k) x d_in
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
@@ -164,12 +166,9 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   if (p->dtype == DYRA_BF16 && !p->force_simt) {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
     if (k > 0) {
-      int splits = 1, rows = 64;
-      dyra::gram_split(T, B, p->d_in, k, p->dev.sm_count, &splits, &rows);
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
       void* tg = p->TG;
-      rc = grow(tg, p->cap_TG,
-                static_cast<size_t>(splits) * B * k * (p->d_in + k) * sizeof(float));
+      rc = grow(tg, p->cap_TG, static_cast<size_t>(B) * k * k * sizeof(float));
       p->TG = static_cast<float*>(tg);
       if (rc) return rc;
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
@@ -286,8 +285,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.TG = p->TG;
     a.Tp = p->Tp;
     a.Ct = p->Ct;
-    split_factor_buffer(correct && !p->factor_self ? p->MD : nullptr, B, p->k, &a.MD,
-                        &a.counters);
+    split_factor_buffer(correct ? p->MD : nullptr, B, p->k, &a.MD, &a.counters);
+    a.factor_mode = p->factor_mode;
     a.splits = 1;
     a.split_rows = 64;
     if (correct) dyra::gram_split(T, B, p->d_in, p->k, p->dev.sm_count, &a.splits, &a.split_rows);
@@ -440,6 +439,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   p->dev.device = dev;
   p->dev.sm_count = prop.multiProcessorCount;
   p->dev.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+  p->dev.smem_per_sm = static_cast<int>(prop.sharedMemPerMultiprocessor);
+  p->dev.smem_reserved = static_cast<int>(prop.reservedSharedMemPerBlock);
   p->dev.cc_major = prop.major;
   p->dev.cc_minor = prop.minor;
   const char* kv = std::getenv("DYRA_KERNELS");
@@ -449,7 +450,10 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   const char* ppv = std::getenv("DYRA_PROJ_PAIR_MIN");
   p->proj_pair_min_tiles = ppv ? std::atoi(ppv) : 0;
   const char* fv = std::getenv("DYRA_FACTOR");
-  p->factor_self = fv != nullptr && std::strcmp(fv, "self") == 0;
+  p->factor_mode = fv == nullptr                     ? -1
+                   : std::strcmp(fv, "self") == 0   ? 0
+                   : std::strcmp(fv, "shared") == 0 ? 1
+                                                    : -1;
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -741,7 +745,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     sizing.take(static_cast<size_t>(N) * p->r * es);
     if (k > 0) {
       sizing.take(static_cast<size_t>(N) * k * es);
-      sizing.take(static_cast<size_t>(splits) * B * k * (p->d_in + k) * sizeof(float));
+      sizing.take(static_cast<size_t>(B) * k * k * sizeof(float));
       sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
       sizing.take(factor_bytes(B, k));
@@ -781,13 +785,13 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.weight_only = k == 0;
     a.Z = carve.take(static_cast<size_t>(N) * p->r * es);
     a.L = k > 0 ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
-    a.TG = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(splits) * B * k *
-                                                  (p->d_in + k) * sizeof(float)))
+    a.TG = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(B) * k * k * sizeof(float)))
                  : nullptr;
     a.Tp = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_in * es) : nullptr;
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     void* fac = k > 0 ? carve.take(factor_bytes(B, k)) : nullptr;
-    split_factor_buffer(p->factor_self ? nullptr : fac, B, k, &a.MD, &a.counters);
+    split_factor_buffer(fac, B, k, &a.MD, &a.counters);
+    a.factor_mode = p->factor_mode;
     a.splits = splits;
     a.split_rows = split_rows;
     a.status = p->status;

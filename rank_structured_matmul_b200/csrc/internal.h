@@ -11,6 +11,8 @@ struct DeviceInfo {
   int device = 0;
   int sm_count = 0;
   int max_smem_optin = 0;
+  int smem_per_sm = 0;    // shared memory of one SM, shared by its resident blocks
+  int smem_reserved = 0;  // shared memory the system reserves per resident block
   int cc_major = 0, cc_minor = 0;
 };
 
@@ -37,11 +39,12 @@ struct Bf16Forward {
   // workspace
   void* Z;               // N x r
   void* L;               // N x k
-  float* TG;             // splits x B x k x (d_in + k)
-  void* Tp;              // (B*k) x d_in
+  float* TG;             // B x k x k: G_b (fp32, without the ridge)
+  void* Tp;              // (B*k) x d_in: T[b*k + i][j] = (L_b^T X_b)[i][j] (bf16)
   void* Ct;              // d_out x (B*k)
   float* MD;             // B factor records (factor_record_floats(k) floats each), or nullptr
   int* counters;         // B ints: the solve's per-instance flags; cleared by the projection
+  int factor_mode;       // who factors G_b: -1 chosen by size, 0 every solve block, 1 the first
   int splits;            // row splits of the Gram reduction
   int split_rows;        // rows per split (multiple of 64)
   int* status;
@@ -109,6 +112,16 @@ int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, i
 // Floats per instance of the factor records for correction rank k (0 when
 // k > 64: the solve then factors G_b itself).
 int factor_record_floats(int k);
+
+// L~ = L G^-1 per instance, over L (bf16 plans; kernels_simt.cu). mode 0: every
+// block factors G_b; 1: the instance's first block factors it and publishes a
+// record (MD, flags). G: B x k x k fp32 (G_b without the ridge).
+int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
+                  int k, float lambda, int* status, cudaStream_t s, bool pdl,
+                  unsigned long long* trace);
+// Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
+size_t ltilde_smem_bytes(int k);
+int ltilde_rows_per_block(int k);
 
 // Pack [V | P]^T: VPt[c][j] = V[j][c] (c < r), P[j][c-r] (c >= r).
 template <typename T>

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstddef>
 
 #include "internal.h"
 #include "ldl_panel.cuh"
@@ -405,6 +406,328 @@ __global__ void __launch_bounds__(kSolveThreads2)
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
 }
 
+// ---------------------------------------------------------------------------
+// Ridge solve on the side of L (bf16 plans): L~_b = L_b G_b^-1, written over
+// L_b. With it the correction of Algorithm 1 ("DyRA", App. A, procedure
+// Inference) is regrouped as
+//   L_b C_b = L_b G_b^-1 (T_b W_res^T) = L~_b Q_b,   Q_b = T_b W_res^T,
+// the same product up to rounding: the GEMM for Q_b needs T_b only, so it runs
+// while this kernel factors G_b, and the output stage multiplies L~ by Q.
+// grid (B, ceil(T / 256)), 256 threads, one row of L_b (one token) per thread:
+//   w = M^T D^-1 M l   for l = L_b[t, :]^T,   G_b = Lt D Lt^T,   M = Lt^-1,
+// (G_b symmetric, so L_b[t, :] G_b^-1 = (G_b^-1 l)^T). Who factors: every CTA
+// (kSolveSelf), or the instance's first CTA, which publishes the factor
+// record for the others (kSolveShared, as in solve_ldl_kernel).
+// The kernel lets the next grid start right after its own dependency wait:
+// that grid may then read what the grid before this one wrote.
+constexpr int kLtThreads = 256;
+
+// Rows of L_b per block: 256 for KMAX = 32, 128 for KMAX = 64 (the staged
+// rows then fit the factorisation's scratch, which is free by then).
+template <int KMAX>
+__host__ __device__ constexpr int lt_rows() {
+  return KMAX <= 32 ? 256 : 128;
+}
+
+template <int KMAX>
+struct LtSmem {
+  static constexpr int kVS = KMAX + 8;  // staged row stride (bf16): 16-byte rows, spread banks
+  LdlBlockScratch<KMAX> ldl;            // after the factorisation: Gs = M, Wb = G^-1 (stride KMAX)
+  // the block's rows of L_b (bf16, stride kVS); for KMAX = 64 they are staged
+  // over ldl.Gs and ldl.Mb instead, once G^-1 is formed
+  alignas(16) __nv_bfloat16 Vs[KMAX <= 32 ? lt_rows<KMAX>() * kVS : 8];
+};
+static_assert(2 * sizeof(float) * 64 * 65 >= sizeof(__nv_bfloat16) * 128 * 72,
+              "KMAX = 64: the staged rows fit over Gs and Mb");
+// 16-byte copies into the staged rows and float4 accesses to M and G^-1
+static_assert(offsetof(LtSmem<32>, Vs) % 16 == 0 && offsetof(LtSmem<64>, Vs) % 16 == 0,
+              "staged rows 16-byte aligned");
+static_assert(offsetof(LdlBlockScratch<32>, Wb) % 16 == 0 &&
+                  offsetof(LdlBlockScratch<64>, Wb) % 16 == 0 &&
+                  offsetof(LdlBlockScratch<64>, Mb) % 16 == 0,
+              "G^-1 and the KMAX = 64 staging 16-byte aligned");
+
+// 152 registers: a block fits on an SM beside a block of the rank-k factor
+// GEMM. Registers come from the SM's four sub-partitions, 16K each, and a
+// sub-partition may hold two warps of each block: 2 x 152 x 32 + 2 x 104 x 32
+// = 16384 (the GEMM's warps take up to 104 registers).
+template <int KMAX, int MODE>
+__global__ void __maxnreg__(152)
+    ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, float* MD, int* flags, int T,
+                  int k, float lambda, int* status, unsigned long long* trace) {
+  using Sm = LtSmem<KMAX>;
+  constexpr int LD = LdlBlockScratch<KMAX>::LD;
+  constexpr int ROWS = lt_rows<KMAX>();
+  constexpr int VS = Sm::kVS;
+  constexpr int NB = KMAX / 16;
+  extern __shared__ __align__(16) unsigned char smem_bytes[];
+  Sm& sm = *reinterpret_cast<Sm*>(smem_bytes);
+  float* const Ma = sm.ldl.Gs;  // M, row-major, stride KMAX (after the factorisation)
+  float* const Gi = sm.ldl.Wb;  // G^-1, row-major, stride KMAX
+  __nv_bfloat16* const Vs = KMAX <= 32 ? sm.Vs : reinterpret_cast<__nv_bfloat16*>(sm.ldl.Gs);
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const bool factors = MODE == kSolveSelf || blockIdx.y == 0;
+  float* rec = MODE == kSolveShared ? MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>()
+                                    : nullptr;
+  unsigned long long* const tr =
+      trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
+  if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
+  sm100::pdl_wait();
+  if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
+  sm100::pdl_launch_dependents();
+
+  const int t0 = blockIdx.y * ROWS;
+  const int nrows = min(ROWS, T - t0);
+  __nv_bfloat16* const rows = L + (static_cast<size_t>(b) * T + t0) * k;
+  // Stage the block's rows (zero beyond k and beyond nrows): 16-byte pieces
+  // when rows are 16-byte aligned (k % 8 == 0), elements otherwise.
+  auto stage_rows = [&](bool async) {
+    if ((k & 7) == 0) {
+      constexpr int C8 = KMAX / 8;
+      for (int e = tid; e < ROWS * C8; e += kLtThreads) {
+        const int rr = e / C8, c8 = e % C8;
+        const bool valid = rr < nrows && 8 * c8 < k;
+        const __nv_bfloat16* src = valid ? rows + static_cast<size_t>(rr) * k + 8 * c8 : rows;
+        __nv_bfloat16* dst = Vs + rr * VS + 8 * c8;
+        if (async)
+          sm100::cp_async_16(sm100::smem_u32(dst), src, valid ? 16u : 0u);
+        else
+          *reinterpret_cast<uint4*>(dst) =
+              valid ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
+      }
+      if (async) sm100::cp_async_commit();
+    } else {
+      for (int e = tid; e < ROWS * KMAX; e += kLtThreads) {
+        const int rr = e / KMAX, q = e % KMAX;
+        Vs[rr * VS + q] = rr < nrows && q < k ? rows[static_cast<size_t>(rr) * k + q]
+                                              : __float2bfloat16_rn(0.f);
+      }
+    }
+  };
+  if constexpr (KMAX <= 32) {
+    stage_rows((k & 7) == 0);  // lands while the factorisation runs
+  } else {
+    // read after the factorisation (the projection wrote them; bring them to L2)
+    for (int e = tid; e < nrows; e += kLtThreads)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(rows + static_cast<size_t>(e) * k));
+  }
+
+  if (factors) {
+    const float* Gb = G + static_cast<size_t>(b) * k * k;
+    constexpr int GPT = KMAX * KMAX / kLtThreads;
+    float g[GPT];
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {  // every load in flight at once
+      const int e = tid + u * kLtThreads, i = e / KMAX, q = e % KMAX;
+      g[u] = i < k && q < k ? __ldg(Gb + i * k + q) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < GPT; ++u) {
+      const int e = tid + u * kLtThreads, i = e / KMAX, q = e % KMAX;
+      sm.ldl.Gs[i * LD + q] =
+          i < k && q < k ? g[u] + (i == q ? lambda : 0.f) : (i == q ? 1.f : 0.f);
+    }
+    __syncthreads();
+    if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
+    // M is emitted over ldl.Gs, whose last read precedes the emits
+    const bool ok = ldl_blocked<KMAX, kLtThreads>(
+        sm.ldl, k, tid, [] { __syncthreads(); },
+        [&](int i, int q, float m) { Ma[i * KMAX + q] = m; }, [](int, float) {},
+        tr ? tr + 40 : nullptr);
+    __syncthreads();
+    // G^-1 = M^T D^-1 M, one 16 x 16 block (Q, J) per warp and step: lane
+    // (r, h) sums over rows i >= 16 max(Q, J) of M[i][16Q + r] D^-1[i] times
+    // M[i][16J + 8h .. +8] (M is zero above its diagonal).
+    {
+      const int r = lane & 15, h = lane >> 4;
+      for (int blk = warp; blk < NB * NB; blk += kLtThreads / 32) {
+        const int Q = blk / NB, J = blk % NB;
+        float acc[8] = {};
+        for (int i = 16 * max(Q, J); i < KMAX; ++i) {
+          const float a = Ma[i * KMAX + 16 * Q + r] * sm.ldl.dinv[i];
+          const float4 b0 = *reinterpret_cast<const float4*>(&Ma[i * KMAX + 16 * J + 8 * h]);
+          const float4 b1 = *reinterpret_cast<const float4*>(&Ma[i * KMAX + 16 * J + 8 * h + 4]);
+          acc[0] = fmaf(a, b0.x, acc[0]);
+          acc[1] = fmaf(a, b0.y, acc[1]);
+          acc[2] = fmaf(a, b0.z, acc[2]);
+          acc[3] = fmaf(a, b0.w, acc[3]);
+          acc[4] = fmaf(a, b1.x, acc[4]);
+          acc[5] = fmaf(a, b1.y, acc[5]);
+          acc[6] = fmaf(a, b1.z, acc[6]);
+          acc[7] = fmaf(a, b1.w, acc[7]);
+        }
+        float* dst = &Gi[(16 * Q + r) * KMAX + 16 * J + 8 * h];
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+    }
+    if (MODE == kSolveShared) {
+      __syncthreads();
+      for (int e = tid; e < KMAX * KMAX / 4; e += kLtThreads)
+        reinterpret_cast<float4*>(rec)[e] = reinterpret_cast<const float4*>(Gi)[e];
+      if (tid == 0) rec[KMAX * KMAX] = ok ? 0.f : 1.f;
+      // the whole record before the flag: the barrier orders the block's
+      // writes before thread 0's fence, whose release covers them
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        sm100::st_release_gpu(flags + b, 1);
+      }
+    }
+  } else {
+    if (tid == 0) {
+      int bad = 0;
+      const unsigned long long deadline = sm100::globaltimer_ns() + sm100::kWaitLimitNs;
+      while (sm100::ld_acquire_gpu(flags + b) == 0) {
+        if (sm100::globaltimer_ns() > deadline) {
+          atomicOr(status, sm100::kStatusTimeout);
+          bad = 1;
+          break;
+        }
+        __nanosleep(128);
+      }
+      sm.ldl.bad = bad;
+    }
+    __syncthreads();
+    // the record: G^-1 (row-major), the failure flag
+    for (int e = tid; e < KMAX * KMAX / 4; e += kLtThreads)
+      reinterpret_cast<float4*>(Gi)[e] = __ldcg(reinterpret_cast<const float4*>(rec) + e);
+    __syncthreads();
+    if (tid == 0 && __ldcg(rec + KMAX * KMAX) != 0.f) sm.ldl.bad = 1;
+  }
+  __syncthreads();  // G^-1 complete; Gs and Mb are free
+  if constexpr (KMAX <= 32) {
+    if ((k & 7) == 0) sm100::cp_async_wait_all();
+  } else {
+    stage_rows(false);
+  }
+  __syncthreads();
+  if (tr && tid == 0) tr[4] = sm100::globaltimer_ns();
+  const bool zero = sm.ldl.bad != 0;
+
+  // W = V G^-1 over the staged rows, 64 rows per pass: thread tile RT rows x
+  // 4 columns (cg: column group, rg: row group), K in steps of 4.
+  constexpr int CG = KMAX / 4;
+  constexpr int RT = 64 * KMAX / (4 * kLtThreads);
+  const int cg = tid % CG, rg = tid / CG;
+#pragma unroll 1
+  for (int p0 = 0; p0 < nrows; p0 += 64) {
+    float acc[RT][4];
+#pragma unroll
+    for (int rr = 0; rr < RT; ++rr)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[rr][c] = 0.f;
+#pragma unroll 4
+    for (int i4 = 0; i4 < KMAX / 4; ++i4) {
+      float4 gq[4];
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii)
+        gq[ii] = *reinterpret_cast<const float4*>(&Gi[(4 * i4 + ii) * KMAX + 4 * cg]);
+#pragma unroll
+      for (int rr = 0; rr < RT; ++rr) {
+        const uint2 vv = *reinterpret_cast<const uint2*>(&Vs[(p0 + RT * rg + rr) * VS + 4 * i4]);
+        const float v[4] = {__uint_as_float(vv.x << 16), __uint_as_float(vv.x & 0xffff0000u),
+                            __uint_as_float(vv.y << 16), __uint_as_float(vv.y & 0xffff0000u)};
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+          acc[rr][0] = fmaf(v[ii], gq[ii].x, acc[rr][0]);
+          acc[rr][1] = fmaf(v[ii], gq[ii].y, acc[rr][1]);
+          acc[rr][2] = fmaf(v[ii], gq[ii].z, acc[rr][2]);
+          acc[rr][3] = fmaf(v[ii], gq[ii].w, acc[rr][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < RT; ++rr) {
+      const int rl = p0 + RT * rg + rr;
+      if (rl >= nrows || 4 * cg >= k) continue;
+      __nv_bfloat16* dst = rows + static_cast<size_t>(rl) * k + 4 * cg;
+      if ((k & 3) == 0) {
+        const __nv_bfloat162 lo =
+            __floats2bfloat162_rn(zero ? 0.f : acc[rr][0], zero ? 0.f : acc[rr][1]);
+        const __nv_bfloat162 hi =
+            __floats2bfloat162_rn(zero ? 0.f : acc[rr][2], zero ? 0.f : acc[rr][3]);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(dst) = w;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (4 * cg + c < k) dst[c] = __float2bfloat16_rn(zero ? 0.f : acc[rr][c]);
+      }
+    }
+  }
+  if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
+  if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
+  if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
+}
+
+// General variant of the same (any k <= 128): every CTA factors G_b itself
+// (Cholesky G_b = R R^T in shared memory) and solves R R^T w = l for 128 rows
+// of L_b, one per thread.
+__global__ void __launch_bounds__(kSolveThreads)
+    ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, int T, int k,
+                          float lambda, int* status) {
+  extern __shared__ float sm[];
+  const int ldg = k + 1;
+  float* R = sm;                // k x (k+1): lower triangle becomes R
+  float* Ycol = sm + k * ldg;   // k x 128: one row of L_b per thread
+  __shared__ int bad;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  sm100::pdl_wait();
+  sm100::pdl_launch_dependents();
+  if (tid == 0) bad = 0;
+  const float* Gb = G + static_cast<size_t>(b) * k * k;
+  for (int idx = tid; idx < k * k; idx += kSolveThreads) {
+    const int i = idx / k, i2 = idx - (idx / k) * k;
+    R[i * ldg + i2] = Gb[idx] + (i == i2 ? lambda : 0.f);
+  }
+  __syncthreads();
+  for (int j = 0; j < k; ++j) {
+    if (tid == 0) {
+      const float d = R[j * ldg + j];
+      if (!(d > 0.f) || !isfinite(d)) {
+        bad = 1;
+        R[j * ldg + j] = 1.f;
+      } else {
+        R[j * ldg + j] = sqrtf(d);
+      }
+    }
+    __syncthreads();
+    const float inv = 1.f / R[j * ldg + j];
+    for (int i = j + 1 + tid; i < k; i += kSolveThreads) R[i * ldg + j] *= inv;
+    __syncthreads();
+    const int m = k - j - 1;
+    for (int idx = tid; idx < m * m; idx += kSolveThreads) {
+      const int i = j + 1 + idx / m, i2 = j + 1 + (idx - (idx / m) * m);
+      if (i2 <= i) R[i * ldg + i2] -= R[i * ldg + j] * R[i2 * ldg + j];
+    }
+    __syncthreads();
+  }
+  const int t = blockIdx.y * kSolveThreads + tid;
+  if (t < T) {
+    __nv_bfloat16* row = L + (static_cast<size_t>(b) * T + t) * k;
+    for (int i = 0; i < k; ++i) Ycol[i * kSolveThreads + tid] = __bfloat162float(row[i]);
+    for (int i = 0; i < k; ++i) {  // R y = l
+      float acc = Ycol[i * kSolveThreads + tid];
+      for (int q = 0; q < i; ++q) acc -= R[i * ldg + q] * Ycol[q * kSolveThreads + tid];
+      Ycol[i * kSolveThreads + tid] = acc / R[i * ldg + i];
+    }
+    for (int i = k - 1; i >= 0; --i) {  // R^T w = y
+      float acc = Ycol[i * kSolveThreads + tid];
+      for (int q = i + 1; q < k; ++q) acc -= R[q * ldg + i] * Ycol[q * kSolveThreads + tid];
+      Ycol[i * kSolveThreads + tid] = acc / R[i * ldg + i];
+    }
+    const bool zero = bad != 0;
+    for (int i = 0; i < k; ++i)
+      row[i] = __float2bfloat16_rn(zero ? 0.f : Ycol[i * kSolveThreads + tid]);
+  }
+  if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
+}
+
 // C[b][m][n] (+)= sum_q A[b][m][q] * Bm[b][q][n] with arbitrary element strides.
 constexpr int kGT = 64;   // tile
 constexpr int kGK = 16;   // k step
@@ -560,6 +883,89 @@ int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, i
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
   return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
+                            status) == cudaSuccess
+             ? 0
+             : -1;
+}
+
+int ltilde_rows_per_block(int k) {
+  return k <= 32 ? lt_rows<32>() : k <= 64 ? lt_rows<64>() : kSolveThreads;
+}
+
+size_t ltilde_smem_bytes(int k) {
+  if (k <= 0) return 0;
+  if (k <= 32) return sizeof(LtSmem<32>);
+  if (k <= 64) return sizeof(LtSmem<64>);
+  return (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) * sizeof(float);
+}
+
+template <int KMAX, int MODE>
+int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L, float* MD,
+                       int* flags, int64_t B, int64_t T, int k, float lambda, int* status,
+                       unsigned long long* trace) {
+  auto kfn = ltilde_kernel<KMAX, MODE>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(LtSmem<KMAX>))) != cudaSuccess ||
+        cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
+            cudaSuccess)
+      return -1;
+    configured = true;
+  }
+  // blockIdx.x = instance, blockIdx.y = chunk of rows: the chunk-0 CTAs (the
+  // factoring ones in the shared mode) are the grid's first B CTAs.
+  cfg.gridDim = dim3(static_cast<unsigned>(B),
+                     static_cast<unsigned>((T + lt_rows<KMAX>() - 1) / lt_rows<KMAX>()));
+  cfg.blockDim = dim3(kLtThreads);
+  cfg.dynamicSmemBytes = sizeof(LtSmem<KMAX>);
+  return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, status,
+                            trace) == cudaSuccess
+             ? 0
+             : -1;
+}
+
+int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
+                  int k, float lambda, int* status, cudaStream_t s, bool pdl,
+                  unsigned long long* trace) {
+  if (B == 0 || T == 0 || k == 0) return 0;
+  if (mode == kSolveShared && (MD == nullptr || flags == nullptr)) return -1;
+  if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
+    return -1;
+  auto* Lb = static_cast<__nv_bfloat16*>(L);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.stream = s;
+  if (k <= 32)
+    return mode == kSolveShared
+               ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+                                                      status, trace)
+               : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+                                                    status, trace);
+  if (k <= 64)
+    return mode == kSolveShared
+               ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+                                                      status, trace)
+               : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+                                                    status, trace);
+  const size_t smem = ltilde_smem_bytes(k);
+  static size_t configured = 48 * 1024;
+  if (smem > configured) {
+    if (cudaFuncSetAttribute(ltilde_general_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+    configured = smem;
+  }
+  if ((T + kSolveThreads - 1) / kSolveThreads > 65535) return -1;
+  cfg.gridDim = dim3(static_cast<unsigned>(B),
+                     static_cast<unsigned>((T + kSolveThreads - 1) / kSolveThreads));
+  cfg.blockDim = dim3(kSolveThreads);
+  cfg.dynamicSmemBytes = smem;
+  return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, static_cast<int>(T), k, lambda,
                             status) == cudaSuccess
              ? 0
              : -1;

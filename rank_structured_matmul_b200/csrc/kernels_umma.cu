@@ -288,19 +288,24 @@ struct ProjPolicy {
 };
 
 // =================================================================== gram ====
-// For every instance b and row split s: D = [X_b | L_b]^T L_b over the split's
-// rows, i.e. T_b^T (d_in x k) and G_b (k x k) partial sums, written to
-// TG[s][b][i][j] (j < d_in: T_b[i][j]; j = d_in + i': G_b[i][i']).
-// Both operands are MN-major (the reduction runs over rows of X and L).
+// For every instance b: D = [X_b | L_b]^T L_b, i.e. T_b^T (d_in x k) and G_b
+// (k x k), written as T[b*k + i][j] = T_b[i][j] (bf16, the next GEMM's
+// K-major operand) and G[b][i][i'] (fp32, for the factorisation). Both
+// operands are MN-major (the reduction runs over rows of X and L). With S > 1
+// row splits the S CTAs of one (m-tile, instance) form a cluster: each leaves
+// its fp32 partial tile in its own operand stages and, after a cluster
+// barrier, sums one slice of rows over all S partials through distributed
+// shared memory (split-K, as in the projection).
 struct GramPolicy {
   struct Params {
     GemmCommon c;
     CUtensorMap tmX;   // (d_in, T, B), box (64, 64, 1), 128B swizzle
     CUtensorMap tmLa;  // (k, T, B),    box (64, 64, 1), 128B swizzle   (A role)
     CUtensorMap tmLb;  // (k, T, B),    box (w, 64, 1),  w*2-byte swizzle (B role)
-    int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total, J;
+    int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total;
     uint32_t b_layout;
-    float* TG;
+    __nv_bfloat16* Tb;  // (B*k) x d_in
+    float* G;           // B x k x k
   };
   struct Tile {
     int mt, b, s, t0, t1;
@@ -312,21 +317,20 @@ struct GramPolicy {
     tma_prefetch_desc(&p.tmLa);
     tma_prefetch_desc(&p.tmLb);
   }
-  // Tiles of G (the m-tiles over L's columns) come first: the solve's
-  // factoring blocks read them first.
+  // The S splits of one output tile are neighbours (one cluster); tiles of G
+  // (the m-tiles over L's columns) come first.
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    const int g = tile / p.S;
+    t.s = tile - g * p.S;
     const int mtl = p.mt_total - p.mtx;
-    const int ng = mtl * p.B * p.S;
-    int rest;
-    if (tile < ng) {
-      t.mt = p.mtx + tile % mtl;
-      rest = tile / mtl;
+    const int ng = mtl * p.B;
+    if (g < ng) {
+      t.mt = p.mtx + g % mtl;
+      t.b = g / mtl;
     } else {
-      t.mt = (tile - ng) % p.mtx;
-      rest = (tile - ng) / p.mtx;
+      t.mt = (g - ng) % p.mtx;
+      t.b = (g - ng) / p.mtx;
     }
-    t.b = rest % p.B;
-    t.s = rest / p.B;
     t.t0 = t.s * p.Ts;
     t.t1 = min(p.T, t.t0 + p.Ts);
   }
@@ -358,34 +362,91 @@ struct GramPolicy {
     const uint32_t rb = static_cast<uint32_t>(p.w) * 2u;  // bytes per K-row of one block
     return smem_desc(b + static_cast<uint32_t>(ks) * 16u * rb, 64u * rb, 8u * rb, p.b_layout);
   }
+  // Stores v[0..n) = D[row][i0 .. i0+n) of tile t (tile row `row`): into T
+  // (bf16) for the m-tiles over X, into G (fp32) for the one over L.
+  template <int n>
+  static __device__ __forceinline__ void store_row(const Params& p, const Tile& t, int row, int i0,
+                                                   const float (&v)[n]) {
+    if (t.mt < p.mtx) {
+      const int j = t.mt * 128 + row;
+      if (j >= p.d_in) return;
+      __nv_bfloat16* dst = p.Tb + static_cast<size_t>(t.b) * p.k * p.d_in + j;
+#pragma unroll
+      for (int u = 0; u < n; ++u)
+        if (i0 + u < p.k) dst[static_cast<size_t>(i0 + u) * p.d_in] = __float2bfloat16_rn(v[u]);
+    } else {
+      const int i2 = (t.mt - p.mtx) * 128 + row;
+      if (i2 >= p.k) return;
+      float* dst = p.G + static_cast<size_t>(t.b) * p.k * p.k + i2;
+#pragma unroll
+      for (int u = 0; u < n; ++u)
+        if (i0 + u < p.k) dst[static_cast<size_t>(i0 + u) * p.k] = v[u];
+    }
+  }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    int jcol;
-    bool valid;
-    if (t.mt < p.mtx) {
-      jcol = t.mt * 128 + e.row;
-      valid = jcol < p.d_in;
-    } else {
-      const int i2 = (t.mt - p.mtx) * 128 + e.row;
-      jcol = p.d_in + i2;
-      valid = i2 < p.k;
+    if (p.S > 1) {
+      // the partial tile into this CTA's operand stages, [c4][row] float4s
+      float4* part = reinterpret_cast<float4*>(e.stage);
+      for (int cc = 0; cc < p.kpad; cc += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tacc + cc, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          part[(cc / 4 + g) * 128 + e.row] =
+              make_float4(f32(v[4 * g]), f32(v[4 * g + 1]), f32(v[4 * g + 2]), f32(v[4 * g + 3]));
+      }
+      if (e.tr && e.tid == 0) e.tr[kTrSplitWritten] = globaltimer_ns();
+      return;
     }
-    float* out = p.TG + static_cast<size_t>(t.s * p.B + t.b) * p.k * p.J + jcol;
     for (int cc = 0; cc < p.kpad; cc += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tacc + cc, v);
       tmem_ld_wait();
-      if (valid) {
+      float f[32];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int i = cc + jj;
-          if (i < p.k) out[static_cast<size_t>(i) * p.J] = f32(v[jj]);
-        }
-      }
+      for (int jj = 0; jj < 32; ++jj) f[jj] = f32(v[jj]);
+      store_row(p, t, e.row, cc, f);
     }
   }
-  static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
-  static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
+  static __device__ __forceinline__ bool cluster_finish(const Params& p) { return p.S > 1; }
+  // After the cluster barrier: this CTA's slice of rows, summed over the
+  // cluster's partials in split order.
+  static __device__ __noinline__ void finish(const Params& p, int tid, uint32_t stage_u32,
+                                             unsigned long long* tr) {
+    if (tr && tid == 0) tr[kTrSplitArrived] = globaltimer_ns();
+    const int ks_me = static_cast<int>(cluster_ctarank());
+    Tile t;
+    decode(p, static_cast<int>(blockIdx.x), t);
+    const int c4n = p.kpad / 4;
+    const int rs = (128 + p.S - 1) / p.S;
+    const int row0 = ks_me * rs, nrows = min(128, row0 + rs) - row0;
+    const int nitems = nrows > 0 ? nrows * c4n : 0;
+    for (int it = tid; it < nitems; it += 128) {
+      const int c4 = it / nrows, row = row0 + (it - c4 * nrows);
+      const uint32_t off = 16u * static_cast<uint32_t>(c4 * 128 + row);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ks = 0; ks < p.S; ks += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          v[j] = ld_shared_cluster_v4(
+              mapa_shared(stage_u32, static_cast<uint32_t>(min(ks + j, p.S - 1))) + off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (ks + j < p.S) {
+            acc.x += v[j].x;
+            acc.y += v[j].y;
+            acc.z += v[j].z;
+            acc.w += v[j].w;
+          }
+      }
+      const float f[4] = {acc.x, acc.y, acc.z, acc.w};
+      store_row(p, t, row, 4 * c4, f);
+    }
+    if (tr && tid == 0) tr[kTrSplitReduced] = globaltimer_ns();
+  }
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
 };
 
@@ -686,8 +747,10 @@ uint32_t pow2_at_least(uint32_t x) {
 // or 0 if the tile shape does not fit.
 template <class Pol>
 uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b_bytes,
-                      int mma_n, bool a_mn, bool b_mn, int* status, const DeviceInfo& dev) {
+                      int mma_n, bool a_mn, bool b_mn, int* status, const DeviceInfo& dev,
+                      int smem_cap = 0) {
   c.num_tiles = num_tiles;
+  c.defer_wait = 0;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -697,8 +760,14 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   c.status = status;
   c.trace = nullptr;
   const uint32_t fixed = gemm_smem_bytes(0, a_bytes, b_bytes, Pol::kEpiSmemBytes);
-  const int budget = dev.max_smem_optin - static_cast<int>(fixed);
-  int stages = budget / static_cast<int>(a_bytes + b_bytes);
+  const int full = (dev.max_smem_optin - static_cast<int>(fixed)) / static_cast<int>(a_bytes + b_bytes);
+  int stages = full;
+  if (smem_cap > 0) {
+    // a cap that would leave fewer than 3 stages is not worth its room
+    const int capped = (std::min(smem_cap, dev.max_smem_optin) - static_cast<int>(fixed)) /
+                       static_cast<int>(a_bytes + b_bytes);
+    if (capped >= 3) stages = capped;
+  }
   stages = std::min(stages, kMaxStages);
   if (stages < 2) return 0;
   c.stages = stages;
@@ -943,7 +1012,6 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   mark(1);
 
   if (k > 0) {
-    const int J = a.d_in + a.k;
     // -------------------------------------------------------------- gram
     {
       GramPolicy::Params p;
@@ -958,8 +1026,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.Ts = a.split_rows;
       p.mtx = ceil_div(a.d_in, 128);
       p.mt_total = p.mtx + ceil_div(a.k, 128);
-      p.J = J;
-      p.TG = a.TG;
+      p.Tb = static_cast<__nv_bfloat16*>(a.Tp);
+      p.G = a.TG;
       p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
       uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
                         static_cast<uint64_t>(a.B)};
@@ -979,21 +1047,37 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
           setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
                                    p.kpad, true, true, a.status, dev);
       if (!smem) return -3;
+      // split rows keep a 128 x kpad fp32 partial in the operand stages
+      if (p.S > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
+                         static_cast<size_t>(128) * p.kpad * 4)
+        return -3;
       if (a.trace) p.c.trace = a.trace + 1 * kTraceCtas * kTraceSlots;
-      if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl)) return -1;
+      if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S)) return -1;
     }
     mark(2);
     // ------------------------------------------------------------- solve
-    // once per instance by the instance's first solve block (mode 1); without
-    // records every block factors G_b itself (mode 0)
+    // L~ = L G^-1 over L. Every block factors its G_b while that fits the
+    // SMs; beyond, the instance's first block factors it for the others.
     const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
-    const int mode = records ? 1 : 0;
-    if (launch_solve<__nv_bfloat16>(a.TG, a.MD, a.counters, mode, a.splits, a.B, a.k, a.d_in,
-                                    a.lambda, static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
-                                    a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
+    int mode = a.factor_mode;
+    if (mode < 0)
+      mode = a.B * ceil_div(a.T, static_cast<int64_t>(ltilde_rows_per_block(a.k))) > dev.sm_count
+                 ? 1
+                 : 0;
+    if (!records) mode = 0;
+    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.status, s,
+                      pdl, a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
     mark(3);
     // ----------------------------------------------------------- rfactor
+    // Q = T W_res^T: needs the Gram stage's T only, so it starts while the
+    // solve blocks factor (its blocks wait for the solve before they exit,
+    // and the output stage waits for them). Its shared memory leaves room
+    // on every SM for one solve block beside it.
+    const int rf_smem_cap =
+        dev.smem_per_sm > 0 && a.k <= 64
+            ? dev.smem_per_sm - 2 * dev.smem_reserved - static_cast<int>(ltilde_smem_bytes(a.k))
+            : 0;
     {
       RFactorPolicy::Params p;
       const int Bk = static_cast<int>(a.B) * a.k;
@@ -1019,17 +1103,21 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
       if (rf_pairs) {
         const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
-        const uint32_t smem = setup_common<RFactorPairPolicy>(
-            p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false, false, a.status, dev);
+        const uint32_t smem =
+            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
+                                            false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.defer_wait = 1;
         p.c.idesc = idesc_bf16(256, p.bn, false, false);
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
       } else {
         const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
-        const uint32_t smem = setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128,
-                                                          p.bn, false, false, a.status, dev);
+        const uint32_t smem =
+            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false,
+                                        a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.defer_wait = 1;
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
       }

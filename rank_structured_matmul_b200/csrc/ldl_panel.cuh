@@ -53,8 +53,8 @@ template <int KMAX>
 struct LdlBlockScratch {
   static constexpr int LD = KMAX + 1;  // odd stride: conflict-free column access
   float Gs[KMAX * LD];                 // G + lambda I (identity padded); L below the diagonal blocks
-  float Wb[KMAX * LD];                 // W_IJ, then N_IP
   float Mb[KMAX * LD];                 // M = Lt^-1
+  float Wb[KMAX * LD];                 // W_IJ, then N_IP
   float dinv[KMAX];                    // 1 / D
   int bad;
 };

@@ -68,6 +68,11 @@ struct GemmCommon {
   uint32_t idesc;      // instruction descriptor (M = 128, N, majors)
   int* status;         // device status word
   unsigned long long* trace;  // optional timeline, nullptr when off
+  // 1: the operands do not depend on the grid launched just before this one
+  // (they depend on an earlier grid, complete once the previous grid's blocks
+  // have started); this grid then waits for the previous one only before it
+  // exits, so that the next grid can still rely on both.
+  int defer_wait;
 };
 
 struct EpiCtx {
@@ -118,7 +123,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  unsigned long long* const tr = c.trace ? c.trace + blockIdx.x * kTraceSlots : nullptr;
+  unsigned long long* const tr =
+      c.trace && blockIdx.x < kTraceCtas ? c.trace + blockIdx.x * kTraceSlots : nullptr;
   if (tr && threadIdx.x == 0) tr[kTrEntry] = globaltimer_ns();
 
   if (threadIdx.x == 0) {
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
   pdl_launch_dependents();
-  pdl_wait();
+  if (!c.defer_wait) pdl_wait();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
@@ -284,6 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp >= 2) Pol::finish(p, threadIdx.x - 64, sA, tr);
     cluster_sync_all();
   }
+  if (c.defer_wait) pdl_wait();
   __syncthreads();
   // Every copy the producer issued has landed before the CTA leaves: in a
   // normal run the MMA thread waited for each of them, so only a run that

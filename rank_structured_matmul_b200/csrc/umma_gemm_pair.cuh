@@ -56,7 +56,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
-  unsigned long long* const tr = c.trace ? c.trace + blockIdx.x * kTraceSlots : nullptr;
+  unsigned long long* const tr =
+      c.trace && blockIdx.x < kTraceCtas ? c.trace + blockIdx.x * kTraceSlots : nullptr;
   if (tr && threadIdx.x == 0) tr[kTrEntry] = globaltimer_ns();
 
   if (threadIdx.x == 0) {
@@ -88,7 +89,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
   pdl_launch_dependents();
-  pdl_wait();
+  if (!c.defer_wait) pdl_wait();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
@@ -210,6 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // aligned barrier reached by a diverged warp would count it twice and let
   // the CTA past before the epilogue warps are done with TMEM).
   __syncwarp();
+  if (c.defer_wait) pdl_wait();
   __syncthreads();
   // Every copy issued has landed before either CTA leaves. The leader's full
   // barriers also count the other CTA's copies, and its MMA thread waited for

@@ -240,10 +240,9 @@ def test_pair_output_stage_matches_single_cta():
 
 
 def _layer_with_factor(s, f, placement):
-    """placement: 'shared' (default: the first solve block of each instance
-    factors G_b) or 'self' (every solve block factors it)."""
-    if placement != "shared":
-        os.environ["DYRA_FACTOR"] = placement
+    """placement: 'shared' (the first solve block of each instance factors G_b
+    and publishes it) or 'self' (every solve block factors it)."""
+    os.environ["DYRA_FACTOR"] = placement
     try:
         return make_layer(s, f)
     finally:
@@ -254,9 +253,9 @@ def _layer_with_factor(s, f, placement):
 @pytest.mark.parametrize("k,B,T", [(32, 3, 201), (64, 2, 150), (24, 1, 3000), (64, 1, 3000),
                                    (32, 40, 64)])
 def test_factor_placements_agree(placement, k, B, T):
-    """G_b factored once per instance by the first solve block (default) or by
-    every solve block gives the same layer, also on a second call (the
-    per-instance flags start from zero again)."""
+    """G_b factored once per instance by the first solve block or by every
+    solve block gives the same layer, also on a second call (the per-instance
+    flags start from zero again)."""
     s, f = _small(k=k, B=B, T=T)
     X = to_dev(f["X"], "bf16")
     other = _layer_with_factor(s, f, placement)
