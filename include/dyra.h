@@ -138,7 +138,7 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
  *   - If the intermediates of B x T rows do not fit in the array the call
  *     returns DYRA_ERR_INVALID_ARG and enqueues nothing. For a bf16 plan they
  *     take about 2*B*T*(r+k) + 4*B*k*k + 2*B*k*(d_in+d_out) + 4*B*F bytes,
- *     each part rounded up to 256, where F = K*K + K + 5 with K = 32 for
+ *     each part rounded up to 256, where F = K*K + 5 with K = 32 for
  *     k <= 32, 64 for k <= 64 (F = 0 above).
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress); make that first call before capturing a stream

@@ -130,7 +130,7 @@ struct DeviceGuard {
 
 int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
-// Factor records plus arrival counters of the Gram stage (bf16, k <= 64).
+// Factor records of the solve plus its per-instance flags (bf16, k <= 64).
 size_t factor_bytes(int64_t B, int k) {
   const int rec = dyra::factor_record_floats(k);
   if (rec == 0) return 0;

@@ -99,15 +99,11 @@ struct SimtForward {
 template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStream_t s);
 
-// Solve (L^T L + lambda I) T' = T for every instance from the Gram partials.
-// mode 0: every solve block factors G_b itself (MD, flags unused);
-// mode 1: one block per instance factors G_b and publishes the factor record
-//         in MD (ldl_panel.cuh layout) behind flags[b], which must be zero at
-//         launch (k <= 64 only).
+// Solve (L^T L + lambda I) T' = T for every instance from the Gram partials
+// (the CUDA-core path): every solve block factors G_b itself.
 template <typename TOut>
-int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, int64_t B, int k,
-                 int d_in, float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
-                 unsigned long long* trace = nullptr);
+int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
+                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace = nullptr);
 
 // Floats per instance of the factor records for correction rank k (0 when
 // k > 64: the solve then factors G_b itself).

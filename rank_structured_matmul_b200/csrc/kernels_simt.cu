@@ -134,15 +134,10 @@ __global__ void __launch_bounds__(kSolveThreads)
 // handles a 128-column chunk of T_b. G_b + lambda I = Lt D Lt^T by the panel
 // elimination of ldl_panel.cuh gives M = Lt^-1 and D; the CTA then applies
 // T' = M^T D^-1 (M T) to its chunk: two small products, no sequential
-// dependency (same accuracy as the two triangular solves). Who factors:
-//  - kSolveSelf: every CTA factors G_b itself (the fp32 path);
-//  - kSolveShared: the instance's first CTA (chunk 0) factors G_b, writes the
-//    factor record (M, D^-1, failure flag) and raises the instance's flag;
-//    the other CTAs load their T chunk meanwhile, wait for the flag (bounded)
-//    and read the record. The first CTAs of the grid are the factoring ones,
-//    so a waiting CTA's producer has always been scheduled before it.
-// The T chunk's first split is requested before the factorisation and lands
-// while it runs; the other splits are added afterwards.
+// dependency (same accuracy as the two triangular solves). Every CTA factors
+// G_b itself (the CUDA-core path of fp32 plans). The T chunk's first split
+// is loaded before the factorisation and waits in registers while it runs;
+// the other splits are added afterwards.
 constexpr int kSolveThreads2 = 256;
 constexpr int kSolveCols = 128;  // columns of T_b per CTA
 enum SolveMode { kSolveSelf = 0, kSolveShared = 1 };
@@ -159,10 +154,10 @@ struct SolveSmem {
   int bad;
 };
 
-template <typename TOut, int KMAX, int MODE>
+template <typename TOut, int KMAX>
 __global__ void __launch_bounds__(kSolveThreads2)
-    solve_ldl_kernel(const float* __restrict__ TG, float* MD, int* flags, int S, int B, int k,
-                     int d_in, float lambda, TOut* __restrict__ Tp, int* status,
+    solve_ldl_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
+                     TOut* __restrict__ Tp, int* status,
                      unsigned long long* trace) {
   using Sm = SolveSmem<KMAX>;
   constexpr int LDG = LdlBlockScratch<KMAX>::LD;
@@ -176,8 +171,6 @@ __global__ void __launch_bounds__(kSolveThreads2)
   const int J = d_in + k;
   const int c0 = blockIdx.y * kSolveCols;
   const size_t inst = static_cast<size_t>(k) * J;
-  const bool factors = MODE == kSolveSelf || (MODE == kSolveShared && blockIdx.y == 0);
-  float* rec = MODE == kSolveSelf ? nullptr : MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
   unsigned long long* const tr =
       trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
   if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
@@ -188,35 +181,16 @@ __global__ void __launch_bounds__(kSolveThreads2)
   sm100::pdl_launch_dependents();
 
   // ---- 1. loads: the first split of the T chunk (kept in registers until
-  // after the factorisation), then G_b (factoring CTAs)
+  // after the factorisation), then G_b
   const float* part = TG + static_cast<size_t>(b) * inst;
-  // bf16 plans (shared mode) have 16-byte TG rows: the first split goes
-  // straight to shared memory with asynchronous copies, holding no registers
-  // during the factorisation; otherwise it waits in registers.
-  constexpr bool kAsyncT = MODE == kSolveShared;
-  float t[kAsyncT ? 1 : TPT];
-  if constexpr (kAsyncT) {
-    constexpr int C4 = kSolveCols / 4;  // 16-byte chunks per row of the chunk
-    constexpr int CPT = KMAX * C4 / kSolveThreads2;
+  float t[TPT];
 #pragma unroll
-    for (int u = 0; u < CPT; ++u) {
-      const int idx = tid + u * kSolveThreads2;
-      const int i = idx / C4, col = c0 + 4 * (idx % C4);
-      const int valid = i < k ? max(0, min(4, d_in - col)) : 0;
-      const float* src = valid ? part + static_cast<size_t>(i) * J + col : part;
-      sm100::cp_async_16(sm100::smem_u32(&sm.Tc[i * kSolveCols + (col - c0)]), src,
-                         static_cast<uint32_t>(valid) * 4u);
-    }
-    sm100::cp_async_commit();
-  } else {
-#pragma unroll
-    for (int u = 0; u < TPT; ++u) {
-      const int idx = tid + u * kSolveThreads2;
-      const int i = idx / kSolveCols, c = idx % kSolveCols;
-      t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
-    }
+  for (int u = 0; u < TPT; ++u) {
+    const int idx = tid + u * kSolveThreads2;
+    const int i = idx / kSolveCols, c = idx % kSolveCols;
+    t[u] = (i < k && c0 + c < d_in) ? part[static_cast<size_t>(i) * J + c0 + c] : 0.f;
   }
-  if (factors) {
+  {
     float g[GPT];
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {
@@ -245,96 +219,29 @@ __global__ void __launch_bounds__(kSolveThreads2)
   __syncthreads();
   if (tr && tid == 0) tr[3] = sm100::globaltimer_ns();
 
-  // ---- 2. the factorisation (factoring CTAs), published for the others
-  if (factors) {
+  // ---- 2. the factorisation
+  {
     const bool ok = ldl_blocked<KMAX, kSolveThreads2>(
         sm.ldl, k, tid, [] { __syncthreads(); },
         [&](int i, int q, float v) {
           sm.Mr[i * Sm::LDM + q] = v;
           sm.Mc[q * Sm::LDM + i] = v;
-          if (MODE == kSolveShared) rec[i * KMAX + q] = v;
         },
-        [&](int j, float v) {
-          sm.dinv[j] = v;
-          if (MODE == kSolveShared) rec[KMAX * KMAX + j] = v;
-        },
-        tr ? tr + 40 : nullptr);
-    if (tid == 0) {
-      if (!ok) sm.bad = 1;
-      if (MODE == kSolveShared) rec[KMAX * KMAX + KMAX] = ok ? 0.f : 1.f;
-    }
-    if (MODE == kSolveShared) {
-      // the whole record before the flag: the barrier orders the block's
-      // writes before thread 0's fence, whose release covers them
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        sm100::st_release_gpu(flags + b, 1);
-      }
-    }
+        [&](int j, float v) { sm.dinv[j] = v; }, tr ? tr + 40 : nullptr);
+    if (tid == 0 && !ok) sm.bad = 1;
   }
   // the remaining splits of the T chunk
-  if constexpr (kAsyncT) {
-    sm100::cp_async_wait_all();
-    __syncthreads();  // every thread's copies have landed
-    for (int sp = 1; sp < S; ++sp) {
-      // all of a split's loads first, then the adds
-      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
-      float v[TPT];
+  for (int sp = 1; sp < S; ++sp) {
+    const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
 #pragma unroll
-      for (int u = 0; u < TPT; ++u) {
-        const int idx = tid + u * kSolveThreads2;
-        const int i = idx / kSolveCols, c = idx % kSolveCols;
-        v[u] = (i < k && c0 + c < d_in) ? __ldg(ps + static_cast<size_t>(i) * J + c0 + c) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] += v[u];
-    }
-  } else {
-    for (int sp = 1; sp < S; ++sp) {
-      const float* ps = TG + (static_cast<size_t>(sp) * B + b) * inst;
-#pragma unroll
-      for (int u = 0; u < TPT; ++u) {
-        const int idx = tid + u * kSolveThreads2;
-        const int i = idx / kSolveCols, c = idx % kSolveCols;
-        if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
-  }
-  if (!factors) {
-    // the record, once the flag is up
-    {
-      if (tid == 0) {
-        int bad = 0;
-        const unsigned long long deadline = sm100::globaltimer_ns() + sm100::kWaitLimitNs;
-        while (sm100::ld_acquire_gpu(flags + b) == 0) {
-          if (sm100::globaltimer_ns() > deadline) {
-            atomicOr(status, sm100::kStatusTimeout);
-            bad = 1;
-            break;
-          }
-          __nanosleep(128);
-        }
-        sm.bad = bad;
-      }
-      __syncthreads();
-    }
-#pragma unroll
-    for (int u = 0; u < GPT; ++u) {
+    for (int u = 0; u < TPT; ++u) {
       const int idx = tid + u * kSolveThreads2;
-      const int i = idx / KMAX, q = idx % KMAX;
-      const float m = __ldcg(rec + idx);
-      sm.Mr[i * Sm::LDM + q] = m;
-      sm.Mc[q * Sm::LDM + i] = m;
-    }
-    if (tid < KMAX) sm.dinv[tid] = __ldcg(rec + KMAX * KMAX + tid);
-    if (tid == 0) {
-      const bool failed = __ldcg(rec + KMAX * KMAX + KMAX) != 0.f;
-      sm.bad = sm.bad | (failed ? 1 : 0);
+      const int i = idx / kSolveCols, c = idx % kSolveCols;
+      if (i < k && c0 + c < d_in) t[u] += ps[static_cast<size_t>(i) * J + c0 + c];
     }
   }
+#pragma unroll
+  for (int u = 0; u < TPT; ++u) sm.Tc[tid + u * kSolveThreads2] = t[u];
   __syncthreads();
   if (tr && tid == 0) tr[4] = sm100::globaltimer_ns();
 
@@ -809,11 +716,10 @@ __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P,
 
 }  // namespace
 
-template <typename TOut, int KMAX, int MODE>
-int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, float* MD, int* flags, int splits,
-                     int64_t B, int k, int d_in, float lambda, TOut* Tp, int* status,
-                     unsigned long long* trace) {
-  auto kfn = solve_ldl_kernel<TOut, KMAX, MODE>;
+template <typename TOut, int KMAX>
+int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, int splits, int64_t B, int k,
+                     int d_in, float lambda, TOut* Tp, int* status, unsigned long long* trace) {
+  auto kfn = solve_ldl_kernel<TOut, KMAX>;
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -823,39 +729,20 @@ int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, float* MD, int* f
       return -1;
     configured = true;
   }
-  // blockIdx.x = instance, blockIdx.y = chunk: the chunk-0 CTAs (the ones
-  // that factor in the shared mode) are the grid's first B CTAs.
   cfg.gridDim = dim3(static_cast<unsigned>(B),
                      static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
   cfg.blockDim = dim3(kSolveThreads2);
   cfg.dynamicSmemBytes = sizeof(SolveSmem<KMAX>);
-  return cudaLaunchKernelEx(&cfg, kfn, TG, MD, flags, splits, static_cast<int>(B), k, d_in,
-                            lambda, Tp, status, trace) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
+                            status, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
-template <typename TOut, int KMAX>
-int launch_solve_mode(cudaLaunchConfig_t& cfg, int mode, const float* TG, float* MD, int* flags,
-                      int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
-                      int* status, unsigned long long* trace) {
-  switch (mode) {
-    case kSolveShared:
-      return launch_solve_ldl<TOut, KMAX, kSolveShared>(cfg, TG, MD, flags, splits, B, k, d_in,
-                                                         lambda, Tp, status, trace);
-    default:
-      return launch_solve_ldl<TOut, KMAX, kSolveSelf>(cfg, TG, MD, flags, splits, B, k, d_in,
-                                                       lambda, Tp, status, trace);
-  }
-}
-
 template <typename TOut>
-int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, int64_t B, int k,
-                 int d_in, float lambda, TOut* Tp, int* status, cudaStream_t s, bool pdl,
-                 unsigned long long* trace) {
+int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
+                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace) {
   if (B == 0 || k == 0) return 0;
-  if (mode != kSolveSelf && (MD == nullptr || (mode == kSolveShared && flags == nullptr)))
-    return -1;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -864,11 +751,9 @@ int launch_solve(const float* TG, float* MD, int* flags, int mode, int splits, i
   cfg.numAttrs = pdl ? 1 : 0;
   cfg.stream = s;
   if (k <= 32)
-    return launch_solve_mode<TOut, 32>(cfg, mode, TG, MD, flags, splits, B, k, d_in, lambda, Tp,
-                                       status, trace);
+    return launch_solve_ldl<TOut, 32>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace);
   if (k <= 64)
-    return launch_solve_mode<TOut, 64>(cfg, mode, TG, MD, flags, splits, B, k, d_in, lambda, Tp,
-                                       status, trace);
+    return launch_solve_ldl<TOut, 64>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace);
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
@@ -971,9 +856,9 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
              : -1;
 }
 
-template int launch_solve<float>(const float*, float*, int*, int, int, int64_t, int, int, float, float*, int*,
+template int launch_solve<float>(const float*, int, int64_t, int, int, float, float*, int*,
                                  cudaStream_t, bool, unsigned long long*);
-template int launch_solve<__nv_bfloat16>(const float*, float*, int*, int, int, int64_t, int, int, float,
+template int launch_solve<__nv_bfloat16>(const float*, int, int64_t, int, int, float,
                                          __nv_bfloat16*, int*, cudaStream_t, bool,
                                          unsigned long long*);
 
@@ -1014,7 +899,7 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
              s))
       return -1;
-    if (launch_solve<T>(a.TG, nullptr, nullptr, 0, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
       return -1;
     // C = T' W_res^T  (B*k x d_out)
     if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,

@@ -21,12 +21,11 @@
 namespace dyra {
 
 // Per-instance factor record, written by the instance's factoring solve block
-// and read by the others:
-// M (KMAX x KMAX, row-major, unit lower), D^-1 (KMAX), a failure flag, padding
-// to a 16-byte multiple.
+// and read by the others: G^-1 (KMAX x KMAX, row-major), a failure flag,
+// padding to a 16-byte multiple.
 template <int KMAX>
 __host__ __device__ constexpr int ldl_record_floats() {
-  return KMAX * KMAX + KMAX + 4;
+  return KMAX * KMAX + 4;
 }
 
 // Reciprocal of a pivot (PTX rcp.approx: within one ulp; the factor's own

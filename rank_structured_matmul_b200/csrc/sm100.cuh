@@ -301,6 +301,9 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
 }
 
 // Arrive once on the leader CTA's copy of barrier `bar`.
+// Every thread of the block (barrier 0, non-aligned).
+__device__ __forceinline__ void block_sync_all() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_arrive_leader(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar & kLeaderMask) : "memory");
 }
@@ -374,8 +377,10 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
                : "memory");
 }
 
+// Non-aligned barriers: they count threads, so a warp may reach them with its
+// lanes diverged (for an aligned bar.sync that is undefined).
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Programmatic dependent launch: wait for the producing grid's memory, and

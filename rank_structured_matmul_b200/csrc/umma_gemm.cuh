@@ -276,10 +276,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     Pol::epilogue_drain(p, e);
     if (tr && e.tid == 0) tr[kTrEpiDone] = globaltimer_ns();
   }
-  // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
-  // that each warp arrives at the barrier once, with all its lanes (an
-  // aligned barrier reached by a diverged warp would count it twice and let
-  // the CTA past before the epilogue warps are done with TMEM).
+  // Warps 0 and 1 ran their roles on one elected lane: reconverge them
+  // before the closing barrier (which counts threads, so it holds the block
+  // until the epilogue warps are done with TMEM either way).
   __syncwarp();
   // A policy whose tiles end in a cluster-wide step (split-K partials summed
   // over distributed shared memory) runs it here: every CTA of the cluster has
@@ -291,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     cluster_sync_all();
   }
   if (c.defer_wait) pdl_wait();
-  __syncthreads();
+  block_sync_all();
   // Every copy the producer issued has landed before the CTA leaves: in a
   // normal run the MMA thread waited for each of them, so only a run that
   // gave up early drains here (one shared deadline for all slots).

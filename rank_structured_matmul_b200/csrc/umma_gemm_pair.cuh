@@ -206,13 +206,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     Pol::epilogue_drain(p, e);
     if (tr && e.tid == 0) tr[kTrEpiDone] = globaltimer_ns();
   }
-  // Warps 0 and 1 ran their roles on one elected lane: reconverge them, so
-  // that each warp arrives at the barrier once, with all its lanes (an
-  // aligned barrier reached by a diverged warp would count it twice and let
-  // the CTA past before the epilogue warps are done with TMEM).
+  // Warps 0 and 1 ran their roles on one elected lane: reconverge them
+  // before the closing barrier (which counts threads, so it holds the block
+  // until the epilogue warps are done with TMEM either way).
   __syncwarp();
   if (c.defer_wait) pdl_wait();
-  __syncthreads();
+  block_sync_all();
   // Every copy issued has landed before either CTA leaves. The leader's full
   // barriers also count the other CTA's copies, and its MMA thread waited for
   // each of them in a normal run, so only a leader that gave up early drains
