@@ -45,8 +45,10 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int *splits, int 
 
 /* Stage timing. When enabled, every forward records a CUDA event on its stream
  * before each stage and after the last, which serialises the stages (no
- * programmatic overlap between them). Stages of the bf16 path, in order:
- *   0 proj (X [V|P]), 1 gram (L^T [X|L]), 2 solve, 3 rfactor (W_res T'^T), 4 out.
+ * programmatic overlap between them). Stages of the bf16 path:
+ *   0 proj (X [V|P]), 1 gram (L^T [X|L]), 2 solve (L~ = L G^-1),
+ *   3 rfactor (Q = T W_res^T), 4 out (Z U^T + L~ Q);
+ * they are launched in the order 0 1 3 2 4 and reported in stage order.
  * Stages that did not run (k == 0) report 0. */
 int dyra_debug_set_stage_timing(dyra_plan_t p, int enable);
 
@@ -62,9 +64,13 @@ int dyra_debug_stage_times(dyra_plan_t p, float *ms5);
  *   3 first copy issued, 4 last copy issued, 5 first operands arrived,
  *   6 last accumulator committed, 7 first accumulator reached the epilogue,
  *   8 exit, 9 + i epilogue of the CTA's i-th tile done (i < 27),
- *   36 + i MMAs of the CTA's i-th tile committed (i < 28).
- * The solve stage (2) uses 0 entry, 2 inputs visible, 3 loaded, 4 factored,
- * 5 solved, 8 exit.
+ *   36 + i MMAs of the CTA's i-th tile committed (i < 20), 56 producer done,
+ *   57 last MMA complete, 58 epilogue done, 60..62 split-K partial written,
+ *   all partials arrived, slice reduced.
+ * The solve stage (2) uses 0 entry, 2 inputs visible, 3 loaded, 4 factored
+ * (G^-1 formed), 5 solved, 8 exit, and 40 + j the factorisation's phases.
+ * Stamps are read with the timer register, which the assembler may read a
+ * little before a preceding barrier.
  * A slot a CTA did not reach stays 0. Disabling frees the buffer. */
 int dyra_debug_set_trace(dyra_plan_t p, int enable);
 size_t dyra_debug_trace_bytes(void);

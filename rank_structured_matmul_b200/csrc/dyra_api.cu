@@ -613,11 +613,14 @@ int dyra_debug_stage_times(dyra_plan_t p, float* ms5) {
   DeviceGuard g(p->dev.device);
   if (!g.ok) return DYRA_ERR_CUDA;
   if (cudaEventSynchronize(p->stage_ev[5]) != cudaSuccess) return DYRA_ERR_CUDA;
+  // The events bracket the launches in stream order: proj, gram, rfactor,
+  // solve, out; the result is in stage order (proj, gram, solve, rfactor, out).
+  static const int kSlot[5] = {0, 1, 3, 2, 4};
   for (int i = 0; i < 5; ++i) {
     float ms = 0.f;
     if (cudaEventElapsedTime(&ms, p->stage_ev[i], p->stage_ev[i + 1]) != cudaSuccess)
       return DYRA_ERR_CUDA;
-    ms5[i] = ms;
+    ms5[kSlot[i]] = ms;
   }
   return DYRA_OK;
 }

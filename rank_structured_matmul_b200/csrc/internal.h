@@ -112,8 +112,11 @@ int factor_record_floats(int k);
 // L~ = L G^-1 per instance, over L (bf16 plans; kernels_simt.cu). mode 0: every
 // block factors G_b; 1: the instance's first block factors it and publishes a
 // record (MD, flags). G: B x k x k fp32 (G_b without the ridge).
+// defer_wait (with pdl): the grid launched just before waited for the one
+// that wrote G and L before letting this one start; this grid then waits
+// for it only before its blocks exit.
 int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl,
+                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
                   unsigned long long* trace);
 // Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
 size_t ltilde_smem_bytes(int k);

@@ -325,8 +325,10 @@ __global__ void __launch_bounds__(kSolveThreads2)
 // (G_b symmetric, so L_b[t, :] G_b^-1 = (G_b^-1 l)^T). Who factors: every CTA
 // (kSolveSelf), or the instance's first CTA, which publishes the factor
 // record for the others (kSolveShared, as in solve_ldl_kernel).
-// The kernel lets the next grid start right after its own dependency wait:
-// that grid may then read what the grid before this one wrote.
+// defer_wait: the grid launched just before this one (the GEMM for Q) has
+// already waited for the Gram stage before letting this grid start, so this
+// grid reads G and L at once and waits for that grid only before it exits
+// (the output stage then relies on both). The next grid may start at once.
 constexpr int kLtThreads = 256;
 
 // Rows of L_b per block: 256 for KMAX = 32, 128 for KMAX = 64 (the staged
@@ -361,7 +363,7 @@ static_assert(offsetof(LdlBlockScratch<32>, Wb) % 16 == 0 &&
 template <int KMAX, int MODE>
 __global__ void __maxnreg__(152)
     ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, float* MD, int* flags, int T,
-                  int k, float lambda, int* status, unsigned long long* trace) {
+                  int k, float lambda, int* status, int defer_wait, unsigned long long* trace) {
   using Sm = LtSmem<KMAX>;
   constexpr int LD = LdlBlockScratch<KMAX>::LD;
   constexpr int ROWS = lt_rows<KMAX>();
@@ -380,7 +382,7 @@ __global__ void __maxnreg__(152)
   unsigned long long* const tr =
       trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
   if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
-  sm100::pdl_wait();
+  if (!defer_wait) sm100::pdl_wait();
   if (tr && tid == 0) tr[2] = sm100::globaltimer_ns();
   sm100::pdl_launch_dependents();
 
@@ -568,6 +570,7 @@ __global__ void __maxnreg__(152)
   }
   if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
   if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
+  if (defer_wait) sm100::pdl_wait();
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
 }
 
@@ -576,7 +579,7 @@ __global__ void __maxnreg__(152)
 // of L_b, one per thread.
 __global__ void __launch_bounds__(kSolveThreads)
     ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, int T, int k,
-                          float lambda, int* status) {
+                          float lambda, int* status, int defer_wait) {
   extern __shared__ float sm[];
   const int ldg = k + 1;
   float* R = sm;                // k x (k+1): lower triangle becomes R
@@ -584,7 +587,7 @@ __global__ void __launch_bounds__(kSolveThreads)
   __shared__ int bad;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
-  sm100::pdl_wait();
+  if (!defer_wait) sm100::pdl_wait();
   sm100::pdl_launch_dependents();
   if (tid == 0) bad = 0;
   const float* Gb = G + static_cast<size_t>(b) * k * k;
@@ -633,6 +636,7 @@ __global__ void __launch_bounds__(kSolveThreads)
       row[i] = __float2bfloat16_rn(zero ? 0.f : Ycol[i * kSolveThreads + tid]);
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
+  if (defer_wait) sm100::pdl_wait();
 }
 
 // C[b][m][n] (+)= sum_q A[b][m][q] * Bm[b][q][n] with arbitrary element strides.
@@ -787,7 +791,7 @@ size_t ltilde_smem_bytes(int k) {
 template <int KMAX, int MODE>
 int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L, float* MD,
                        int* flags, int64_t B, int64_t T, int k, float lambda, int* status,
-                       unsigned long long* trace) {
+                       int defer_wait, unsigned long long* trace) {
   auto kfn = ltilde_kernel<KMAX, MODE>;
   static bool configured = false;
   if (!configured) {
@@ -805,14 +809,15 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
   cfg.blockDim = dim3(kLtThreads);
   cfg.dynamicSmemBytes = sizeof(LtSmem<KMAX>);
   return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, status,
-                            trace) == cudaSuccess
+                            defer_wait, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
 int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl,
+                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
                   unsigned long long* trace) {
+  const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
   if (mode == kSolveShared && (MD == nullptr || flags == nullptr)) return -1;
   if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
@@ -828,15 +833,15 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   if (k <= 32)
     return mode == kSolveShared
                ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, trace)
+                                                      status, dw, trace)
                : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, trace);
+                                                    status, dw, trace);
   if (k <= 64)
     return mode == kSolveShared
                ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, trace)
+                                                      status, dw, trace)
                : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, trace);
+                                                    status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
   static size_t configured = 48 * 1024;
   if (smem > configured) {
@@ -851,7 +856,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
   return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, static_cast<int>(T), k, lambda,
-                            status) == cudaSuccess
+                            status, dw) == cudaSuccess
              ? 0
              : -1;
 }

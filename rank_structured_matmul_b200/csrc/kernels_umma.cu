@@ -751,6 +751,7 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
                       int smem_cap = 0) {
   c.num_tiles = num_tiles;
   c.defer_wait = 0;
+  c.trigger_after_wait = 0;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -1055,25 +1056,11 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S)) return -1;
     }
     mark(2);
-    // ------------------------------------------------------------- solve
-    // L~ = L G^-1 over L. Every block factors its G_b while that fits the
-    // SMs; beyond, the instance's first block factors it for the others.
-    const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
-    int mode = a.factor_mode;
-    if (mode < 0)
-      mode = a.B * ceil_div(a.T, static_cast<int64_t>(ltilde_rows_per_block(a.k))) > dev.sm_count
-                 ? 1
-                 : 0;
-    if (!records) mode = 0;
-    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.status, s,
-                      pdl, a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
-      return -1;
-    mark(3);
     // ----------------------------------------------------------- rfactor
-    // Q = T W_res^T: needs the Gram stage's T only, so it starts while the
-    // solve blocks factor (its blocks wait for the solve before they exit,
-    // and the output stage waits for them). Its shared memory leaves room
-    // on every SM for one solve block beside it.
+    // Q = T W_res^T needs the Gram stage's T only. The solve is launched
+    // after it and runs beside it: this grid lets the solve start once its
+    // own wait for the Gram stage is over, and its shared memory leaves room
+    // on every SM for one solve block.
     const int rf_smem_cap =
         dev.smem_per_sm > 0 && a.k <= 64
             ? dev.smem_per_sm - 2 * dev.smem_reserved - static_cast<int>(ltilde_smem_bytes(a.k))
@@ -1107,7 +1094,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
             setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
                                             false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
-        p.c.defer_wait = 1;
+        p.c.trigger_after_wait = 1;
         p.c.idesc = idesc_bf16(256, p.bn, false, false);
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
@@ -1117,11 +1104,29 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
             setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false,
                                         a.status, dev, rf_smem_cap);
         if (!smem) return -3;
-        p.c.defer_wait = 1;
+        p.c.trigger_after_wait = 1;
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
       }
     }
+    mark(3);
+    // ------------------------------------------------------------- solve
+    // L~ = L G^-1 over L, beside the GEMM for Q: it reads what the Gram
+    // stage wrote and waits for the GEMM only before its blocks exit, so that
+    // the output stage can rely on both. Every block factors its G_b while
+    // that fits the SMs; beyond, the instance's first block factors it for
+    // the others.
+    const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
+    int mode = a.factor_mode;
+    if (mode < 0)
+      mode = a.B * ceil_div(a.T, static_cast<int64_t>(ltilde_rows_per_block(a.k))) > dev.sm_count
+                 ? 1
+                 : 0;
+    if (!records) mode = 0;
+    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.status, s,
+                      pdl, /*defer_wait=*/true,
+                      a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
+      return -1;
   } else {
     mark(2);
     mark(3);

@@ -73,6 +73,9 @@ struct GemmCommon {
   // have started); this grid then waits for the previous one only before it
   // exits, so that the next grid can still rely on both.
   int defer_wait;
+  // 1: the next grid may start only once this grid's own dependency wait is
+  // over (that grid then relies on what the grid before this one wrote).
+  int trigger_after_wait;
 };
 
 struct EpiCtx {
@@ -155,8 +158,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // Every CTA of this grid is resident (grid <= SMs), so the next kernel in
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
-  pdl_launch_dependents();
+  if (!c.trigger_after_wait) pdl_launch_dependents();
   if (!c.defer_wait) pdl_wait();
+  if (c.trigger_after_wait) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};

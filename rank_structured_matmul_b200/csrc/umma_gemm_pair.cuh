@@ -88,8 +88,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // Every CTA of this grid is resident (grid <= SMs), so the next kernel in
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
-  pdl_launch_dependents();
+  if (!c.trigger_after_wait) pdl_launch_dependents();
   if (!c.defer_wait) pdl_wait();
+  if (c.trigger_after_wait) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status};
