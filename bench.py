@@ -38,8 +38,8 @@ UNIT = "TFLOP/s (dense-equivalent)"
 HEADLINE = "vit_fc1"
 STAGE_KERNELS = {"proj": "ProjPolicy (CTA pairs, or split-K clusters at skinny N)",
                  "gram": "umma_gemm_kernel<GramPolicy>",
-                 "solve": "solve_ldl_kernel",
-                 "rfactor": "RFactorPolicy (CTA pairs when there are enough tiles)",
+                 "solve": "ltilde_kernel (L~ = L G^-1, beside the rank-k factor GEMM)",
+                 "rfactor": "RFactorPolicy (Q = T W_res^T; CTA pairs when there are enough tiles)",
                  "out": "umma_gemm_pair_kernel<OutPairPolicy>"}
 FLUSH_BYTES = 256 << 20
 
@@ -92,14 +92,14 @@ def algorithmic(s):
     flops = {
         "proj": 2.0 * N * di * (r + k),
         "gram": 2.0 * N * k * (di + k),
-        "solve": B * (k ** 3 / 3.0 + 2.0 * k * k * di),
+        "solve": B * (k ** 3 / 3.0 + k ** 3) + 2.0 * N * k * k,
         "rfactor": 2.0 * B * k * di * do,
         "out": 2.0 * N * do * (r + k),
     }
     bytes_ = {
         "proj": es * (N * di + (r + k) * di + N * (r + k)),
-        "gram": es * (N * di + N * k) + 4.0 * B * k * (di + k),
-        "solve": 4.0 * B * k * (di + k) + es * B * k * di,
+        "gram": es * (N * di + N * k + B * k * di) + 4.0 * B * k * k,
+        "solve": 4.0 * B * k * k + 2.0 * es * N * k,
         "rfactor": es * (do * di + B * k * di + do * B * k),
         "out": es * (N * do + N * r + N * k + do * r + do * B * k),
     }

@@ -389,33 +389,25 @@ __global__ void __maxnreg__(152)
   const int t0 = blockIdx.y * ROWS;
   const int nrows = min(ROWS, T - t0);
   __nv_bfloat16* const rows = L + (static_cast<size_t>(b) * T + t0) * k;
-  // Stage the block's rows (zero beyond k and beyond nrows): 16-byte pieces
-  // when rows are 16-byte aligned (k % 8 == 0), elements otherwise.
+  // Stage the block's rows (zero beyond k and beyond nrows) in 16-byte pieces
+  // (k is a multiple of 8, so every row starts on a 16-byte boundary).
   auto stage_rows = [&](bool async) {
-    if ((k & 7) == 0) {
-      constexpr int C8 = KMAX / 8;
-      for (int e = tid; e < ROWS * C8; e += kLtThreads) {
-        const int rr = e / C8, c8 = e % C8;
-        const bool valid = rr < nrows && 8 * c8 < k;
-        const __nv_bfloat16* src = valid ? rows + static_cast<size_t>(rr) * k + 8 * c8 : rows;
-        __nv_bfloat16* dst = Vs + rr * VS + 8 * c8;
-        if (async)
-          sm100::cp_async_16(sm100::smem_u32(dst), src, valid ? 16u : 0u);
-        else
-          *reinterpret_cast<uint4*>(dst) =
-              valid ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
-      }
-      if (async) sm100::cp_async_commit();
-    } else {
-      for (int e = tid; e < ROWS * KMAX; e += kLtThreads) {
-        const int rr = e / KMAX, q = e % KMAX;
-        Vs[rr * VS + q] = rr < nrows && q < k ? rows[static_cast<size_t>(rr) * k + q]
-                                              : __float2bfloat16_rn(0.f);
-      }
+    constexpr int C8 = KMAX / 8;
+    for (int e = tid; e < ROWS * C8; e += kLtThreads) {
+      const int rr = e / C8, c8 = e % C8;
+      const bool valid = rr < nrows && 8 * c8 < k;
+      const __nv_bfloat16* src = valid ? rows + static_cast<size_t>(rr) * k + 8 * c8 : rows;
+      __nv_bfloat16* dst = Vs + rr * VS + 8 * c8;
+      if (async)
+        sm100::cp_async_16(sm100::smem_u32(dst), src, valid ? 16u : 0u);
+      else
+        *reinterpret_cast<uint4*>(dst) =
+            valid ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
     }
+    if (async) sm100::cp_async_commit();
   };
   if constexpr (KMAX <= 32) {
-    stage_rows((k & 7) == 0);  // lands while the factorisation runs
+    stage_rows(true);  // lands while the factorisation runs
   } else {
     // read after the factorisation (the projection wrote them; bring them to L2)
     for (int e = tid; e < nrows; e += kLtThreads)
@@ -507,7 +499,7 @@ __global__ void __maxnreg__(152)
   }
   __syncthreads();  // G^-1 complete; Gs and Mb are free
   if constexpr (KMAX <= 32) {
-    if ((k & 7) == 0) sm100::cp_async_wait_all();
+    sm100::cp_async_wait_all();
   } else {
     stage_rows(false);
   }
@@ -552,20 +544,14 @@ __global__ void __maxnreg__(152)
       const int rl = p0 + RT * rg + rr;
       if (rl >= nrows || 4 * cg >= k) continue;
       __nv_bfloat16* dst = rows + static_cast<size_t>(rl) * k + 4 * cg;
-      if ((k & 3) == 0) {
-        const __nv_bfloat162 lo =
-            __floats2bfloat162_rn(zero ? 0.f : acc[rr][0], zero ? 0.f : acc[rr][1]);
-        const __nv_bfloat162 hi =
-            __floats2bfloat162_rn(zero ? 0.f : acc[rr][2], zero ? 0.f : acc[rr][3]);
-        uint2 w;
-        w.x = *reinterpret_cast<const uint32_t*>(&lo);
-        w.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(dst) = w;
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (4 * cg + c < k) dst[c] = __float2bfloat16_rn(zero ? 0.f : acc[rr][c]);
-      }
+      const __nv_bfloat162 lo =
+          __floats2bfloat162_rn(zero ? 0.f : acc[rr][0], zero ? 0.f : acc[rr][1]);
+      const __nv_bfloat162 hi =
+          __floats2bfloat162_rn(zero ? 0.f : acc[rr][2], zero ? 0.f : acc[rr][3]);
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(dst) = w;
     }
   }
   if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
@@ -819,6 +805,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
                   unsigned long long* trace) {
   const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
+  if (k % 8 != 0) return -1;  // bf16 plans: 16-byte rows of L
   if (mode == kSolveShared && (MD == nullptr || flags == nullptr)) return -1;
   if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
     return -1;
