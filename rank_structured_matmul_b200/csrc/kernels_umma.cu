@@ -63,12 +63,14 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
                                                int y, EpiCtx& e) {
   const uint32_t buf = e.counter % kStoreBoxes;
   ++e.counter;
+  // both TMEM loads in flight before one wait, and during the wait for the
+  // store buffer
+  uint32_t vv[2][32];
+  tmem_ld_32x32b_x32(tacc + col0, vv[0]);
+  tmem_ld_32x32b_x32(tacc + col0 + 32, vv[1]);
   if (e.tid == 0) tma_store_wait_read<kStoreBoxes - 1>();
   named_bar_sync(1, 128);
   uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
-  uint32_t vv[2][32];  // both TMEM loads in flight before one wait
-  tmem_ld_32x32b_x32(tacc + col0, vv[0]);
-  tmem_ld_32x32b_x32(tacc + col0 + 32, vv[1]);
   tmem_ld_wait();
 #pragma unroll
   for (int half = 0; half < 2; ++half) {

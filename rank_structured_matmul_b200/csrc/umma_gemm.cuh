@@ -78,6 +78,34 @@ struct GemmCommon {
   int trigger_after_wait;
 };
 
+// Issues one stage's ks MMAs (K = 16 each) back to back. The tensor pipe idles
+// whenever an MMA is issued late, even by a few dozen cycles of address
+// arithmetic (a runtime k-step loop measured 168 cycles per M=256, N=256 MMA
+// instead of 128), so the descriptors advance by a fixed step (their address
+// field is linear in the k-step) and the usual counts are unrolled.
+template <bool PAIR>
+__device__ __forceinline__ void issue_stage(uint32_t d, uint64_t a0, uint64_t da, uint64_t b0,
+                                            uint64_t db, uint32_t idesc, int ks, bool first) {
+  auto mma = [&](uint64_t ad, uint64_t bd, uint32_t accum) {
+    if constexpr (PAIR)
+      sm100::mma_bf16_pair(d, ad, bd, idesc, accum);
+    else
+      sm100::mma_bf16(d, ad, bd, idesc, accum);
+  };
+  const uint32_t acc0 = first ? 0u : 1u;
+  if (ks == 4) {
+    mma(a0, b0, acc0);
+    mma(a0 + da, b0 + db, 1u);
+    mma(a0 + 2 * da, b0 + 2 * db, 1u);
+    mma(a0 + 3 * da, b0 + 3 * db, 1u);
+  } else if (ks == 2) {
+    mma(a0, b0, acc0);
+    mma(a0 + da, b0 + db, 1u);
+  } else {
+    for (int k = 0; k < ks; ++k) mma(a0 + k * da, b0 + k * db, k == 0 ? acc0 : 1u);
+  }
+}
+
 struct EpiCtx {
   int row;            // tile row owned by this thread, 0..127
   int lane;           // lane in warp
@@ -204,6 +232,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      const uint32_t idesc = c.idesc;
+      const uint64_t da = Pol::adesc(p, sA, 1) - Pol::adesc(p, sA, 0);
+      const uint64_t db = Pol::bdesc(p, sB, 1) - Pol::bdesc(p, sB, 0);
+      uint32_t a = sA, b = sB;  // this stage's operands
       for (int tile = blockIdx.x; tile < c.num_tiles; tile += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -215,22 +247,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int nk = Pol::kiters(p, t);
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
+          // what the stage's MMAs need besides its data, before the wait
+          const int ks = Pol::ksteps(p, t, it);
+          const uint64_t a0 = Pol::adesc(p, a, 0), b0 = Pol::bdesc(p, b, 0);
           if (!mbar_wait(full_bar(stage), phase, w)) {
             ok = false;
             break;
           }
           if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
-          const uint32_t a = sA + stage * c.a_stage_bytes;
-          const uint32_t b = sB + stage * c.b_stage_bytes;
-          const int ks = Pol::ksteps(p, t, it);
-          for (int k = 0; k < ks; ++k)
-            mma_bf16(d, Pol::adesc(p, a, k), Pol::bdesc(p, b, k), c.idesc,
-                     (it > 0 || k > 0) ? 1u : 0u);
+          issue_stage<false>(d, a0, da, b0, db, idesc, ks, it == 0);
           mma_commit(empty_bar(stage));
+          a += c.a_stage_bytes;
+          b += c.b_stage_bytes;
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
+            a = sA;
+            b = sB;
           }
         }
         if (!ok) break;

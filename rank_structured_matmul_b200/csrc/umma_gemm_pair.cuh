@@ -135,6 +135,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      const uint32_t idesc = c.idesc;
+      const uint64_t da = Pol::adesc(p, sA, 1) - Pol::adesc(p, sA, 0);
+      const uint64_t db = Pol::bdesc(p, sB, 1) - Pol::bdesc(p, sB, 0);
+      uint32_t a = sA, b = sB;  // this stage's operands
       for (int tile = pair; tile < c.num_tiles; tile += npairs, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -146,22 +150,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int nk = Pol::kiters(p, t);
         bool ok = true;
         for (int it = 0; it < nk; ++it) {
+          // what the stage's MMAs need besides its data, before the wait
+          const int ks = Pol::ksteps(p, t, it);
+          const uint64_t a0 = Pol::adesc(p, a, 0), b0 = Pol::bdesc(p, b, 0);
           if (!mbar_wait(full_bar(stage), phase, w)) {
             ok = false;
             break;
           }
           if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
-          const uint32_t a = sA + stage * c.a_stage_bytes;
-          const uint32_t b = sB + stage * c.b_stage_bytes;
-          const int ks = Pol::ksteps(p, t, it);
-          for (int k = 0; k < ks; ++k)
-            mma_bf16_pair(d, Pol::adesc(p, a, k), Pol::bdesc(p, b, k), c.idesc,
-                          (it > 0 || k > 0) ? 1u : 0u);
+          issue_stage<true>(d, a0, da, b0, db, idesc, ks, it == 0);
           mma_commit_pair(empty_bar(stage));
+          a += c.a_stage_bytes;
+          b += c.b_stage_bytes;
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
+            a = sA;
+            b = sB;
           }
         }
         if (!ok) break;
