@@ -16,14 +16,16 @@ extern "C" {
 
 /* Workspace buffers, valid after a forward on the same stream has completed.
  * Layouts for a DYRA_BF16 plan and a forward of B instances x T rows (N = B*T):
- *   DYRA_BUF_Z   N x r bf16     X V                      ([DyRA] Alg. 1 line 10, first factor)
- *   DYRA_BUF_L   N x k bf16     X P                      (line 11)
- *   DYRA_BUF_TG  S x B x k x (d_in + k) fp32: per row split s and instance b,
- *                columns [0, d_in) hold L_b^T X_b, columns [d_in, d_in + k) L_b^T L_b
- *   DYRA_BUF_TP  (B*k) x d_in bf16   (L^T L + lambda I)^-1 L^T X per instance
- *   DYRA_BUF_CT  d_out x (B*k) bf16  C^T = W_res T'^T   (line 12's R^(1), transposed)
- * For a DYRA_F32 plan: Z holds N x (r+k) fp32 ([Z | L]), TG has S = 1,
- * TP is fp32, and CT holds C as (B*k) x d_out fp32. */
+ *   DYRA_BUF_Z   N x r bf16     X V   ([DyRA] Alg. 1, Inference: first factor of the static part)
+ *   DYRA_BUF_L   N x k bf16     X P (the correction's left factor), overwritten per instance by the
+ *                solve with L_b (L_b^T L_b + lambda I)^-1
+ *   DYRA_BUF_TG  B x k x k fp32 L_b^T L_b per instance (no ridge)
+ *   DYRA_BUF_TP  (B*k) x d_in bf16   L_b^T X_b per instance
+ *   DYRA_BUF_CT  d_out x (B*k) bf16  Q^T = W_res (L^T X)^T, so that the layer's
+ *                correction L R^(1) is the solved L times Q
+ * For a DYRA_F32 plan: Z holds N x (r+k) fp32 ([Z | L]), TG holds B x k x
+ * (d_in + k) fp32 (columns [0, d_in) L_b^T X_b, then L_b^T L_b), TP the solved
+ * (L^T L + lambda I)^-1 L^T X (fp32), and CT holds C = R^(1) as (B*k) x d_out fp32. */
 enum {
   DYRA_BUF_Z = 0,
   DYRA_BUF_L = 1,

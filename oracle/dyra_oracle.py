@@ -128,11 +128,11 @@ def inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
 
     The rows of X are B consecutive instances of T rows; the correction is
     fitted per instance (Sec. 2.4: one SPD system "for each batch instance").
-    For instance b with rows X_b:
-      line 10  Y_base = X_b W_hat^T              = (X_b V) U^T
-      line 11  L      = X_b P                    (T x k)
-      line 12  C      = (L^T L + lam I)^-1 (L^T X_b) W_res^T   (k x d_out)
-      line 13  Y_b    = Y_base + L C
+    For instance b with rows X_b, the procedure's steps in order:
+      static part   Y_base = X_b W_hat^T              = (X_b V) U^T
+      left factor   L      = X_b P                    (T x k)
+      right factor  C      = (L^T L + lam I)^-1 (L^T X_b) W_res^T   (k x d_out)
+      output        Y_b    = Y_base + L C
     """
     X = np.asarray(X, dtype=np.float64)
     N = X.shape[0]
@@ -157,8 +157,8 @@ def inference_rows(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
     """Rows `rows` of inference(...), for layers too large to evaluate whole.
 
     Each instance that owns a requested row is fitted on all of its T rows
-    exactly as in inference (Alg. 1 lines 11-12); lines 10 and 13 are then
-    evaluated for the requested rows only.
+    exactly as in inference (its left and right factors); the static part and
+    the output are then evaluated for the requested rows only.
     """
     X = np.asarray(X, dtype=np.float64)
     rows = np.asarray(rows, dtype=np.int64)

@@ -1,11 +1,15 @@
 // kernels_simt.cu - CUDA-core kernels of the DyRA forward.
 //
-//  * solve_kernel: per-instance ridge solve of Algorithm 1 line 12 ("DyRA:
-//    Dynamic Residual Approximation for Efficient Matrix Multiplication in
-//    DNNs", App. A; Sec. 2.4 uses a Cholesky solver for small k):
+//  * solve_kernel / solve_ldl_kernel (fp32 plans): per-instance ridge solve of
+//    the right factor in Algorithm 1, procedure Inference ("DyRA: Dynamic
+//    Residual Approximation for Efficient Matrix Multiplication in DNNs",
+//    App. A; Sec. 2.4 uses a Cholesky solver for small k):
 //      G_b = sum over row splits of L_b^T L_b  (+ lambda I, footnote 2 of Sec. 2.2)
 //      T_b = sum over row splits of L_b^T X_b
-//      T'_b = G_b^-1 T_b via Cholesky G_b = R R^T and two triangular solves.
+//      T'_b = G_b^-1 T_b (Cholesky with two triangular solves, or the blocked
+//      LDL^T of ldl_panel.cuh for k <= 64).
+//  * ltilde_kernel / ltilde_general_kernel (bf16 plans): L~_b = L_b G_b^-1
+//    over L, the same solve applied on the side of L.
 //  * simt_gemm_kernel: strided, batched fp32 GEMM used by the fp32 plans
 //    (fp32 accuracy needs plain FFMA; TF32 tensor cores would lose ~1e-3).
 //  * pack_vp_kernel: builds [V | P]^T once at factor-load time.
@@ -320,11 +324,13 @@ __global__ void __launch_bounds__(kSolveThreads2)
 //   L_b C_b = L_b G_b^-1 (T_b W_res^T) = L~_b Q_b,   Q_b = T_b W_res^T,
 // the same product up to rounding: the GEMM for Q_b needs T_b only, so it runs
 // while this kernel factors G_b, and the output stage multiplies L~ by Q.
-// grid (B, ceil(T / 256)), 256 threads, one row of L_b (one token) per thread:
-//   w = M^T D^-1 M l   for l = L_b[t, :]^T,   G_b = Lt D Lt^T,   M = Lt^-1,
-// (G_b symmetric, so L_b[t, :] G_b^-1 = (G_b^-1 l)^T). Who factors: every CTA
-// (kSolveSelf), or the instance's first CTA, which publishes the factor
-// record for the others (kSolveShared, as in solve_ldl_kernel).
+// grid (B, ceil(T / rows)), 256 threads, 256 (KMAX = 32) or 128 (KMAX = 64)
+// rows of L_b per block: G_b + lambda I = Lt D Lt^T by the blocked elimination
+// of ldl_panel.cuh gives M = Lt^-1 and D, then G_b^-1 = M^T D^-1 M is formed
+// once (fp32) and the block's rows are multiplied by it in a register-tiled
+// product (G_b is symmetric, so a row times G_b^-1 is G_b^-1 times the row).
+// Who factors: every CTA (kSolveSelf), or the instance's first CTA, which
+// publishes G_b^-1 and a failure flag for the others (kSolveShared).
 // defer_wait: the grid launched just before this one (the GEMM for Q) has
 // already waited for the Gram stage before letting this grid start, so this
 // grid reads G and L at once and waits for that grid only before it exits
@@ -402,7 +408,7 @@ __global__ void __maxnreg__(152)
         sm100::cp_async_16(sm100::smem_u32(dst), src, valid ? 16u : 0u);
       else
         *reinterpret_cast<uint4*>(dst) =
-            valid ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
+            valid ? __ldcg(reinterpret_cast<const uint4*>(src)) : make_uint4(0, 0, 0, 0);
     }
     if (async) sm100::cp_async_commit();
   };
@@ -421,7 +427,7 @@ __global__ void __maxnreg__(152)
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {  // every load in flight at once
       const int e = tid + u * kLtThreads, i = e / KMAX, q = e % KMAX;
-      g[u] = i < k && q < k ? __ldg(Gb + i * k + q) : 0.f;
+      g[u] = i < k && q < k ? __ldcg(Gb + i * k + q) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < GPT; ++u) {

@@ -6,13 +6,14 @@
 // correction rank k, Y = X W^T with W = d_out x d_in.
 //
 // Four tensor-core GEMMs and one small solve, stream-ordered:
-//   proj    [Z | L] = X [V | P]              Alg. 1 lines 10-11, Eq. 7
-//   gram    per instance b: [T_b | G_b] = L_b^T [X_b | L_b]      line 12
-//   solve   T'_b = (G_b + lambda I)^-1 T_b   (kernels_simt.cu)  line 12
-//   rfactor C^T = W_res T'^T, all instances at once              line 12
-//   out     Y = Z U^T + sum_b mask_b(L) C_b, one TMEM accumulation  line 13
-// C_b is the paper's R^(1) for instance b; computing (G^-1 L^T X) W_res^T
-// instead of G^-1 ((L^T X) W_res^T) is the same product reassociated.
+//   proj    [Z | L] = X [V | P]                     static part and left factor, Eq. 7
+//   gram    per instance b: T_b = L_b^T X_b (bf16), G_b = L_b^T L_b (fp32)
+//   rfactor Q^T = W_res T^T, all instances at once
+//   solve   L~_b = L_b (G_b + lambda I)^-1, beside rfactor (kernels_simt.cu)
+//   out     Y = Z U^T + sum_b mask_b(L~) Q_b, one TMEM accumulation (the output step)
+// L~_b Q_b = L_b C_b with C_b the paper's R^(1) for instance b, the right factor
+// (G_b + lambda I)^-1 (L_b^T X_b) W_res^T: the same product, grouped so that
+// the large GEMM needs no factorisation.
 //
 // Storage bf16, accumulation fp32 in tensor memory. Every operand tile is
 // brought in by TMA with 128-byte swizzling (64 bf16 per row); tiles that run
