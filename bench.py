@@ -108,6 +108,17 @@ def algorithmic(s):
     return flops, bytes_, layer_flops, layer_bytes
 
 
+def static_matched_rank(s) -> int:
+    """Rank r_s of a static-only layer (X V_s) U_s^T whose FLOPs 2 N r_s
+    (d_in + d_out) match the DyRA layer's ([DyRA] App. E.4: the static
+    baseline of rank r + k + k' with the same FLOPs), rounded down to a
+    multiple of 8 (16-byte rows of bf16 factors) and capped at min(d_in, d_out)."""
+    _, _, layer_flops, _ = algorithmic(s)
+    rs = int(layer_flops // (2.0 * s.N * (s.d_in + s.d_out)))
+    rs = min(rs - rs % 8, min(s.d_in, s.d_out) // 8 * 8)
+    return max(rs, 8)
+
+
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
@@ -356,6 +367,17 @@ def run_dyra(args):
     e2e_ms = max_over_ranks(timed(e2e_step, args.steps, 2), world, dev)
     e2e_value = job_value(dense_flops, world, e2e_ms * 1e-3)
 
+    # ---- the static-only layer with the same FLOPs (rank r_s, no correction),
+    # timed the same way, outside the timed region above
+    rs = static_matched_rank(s)
+    static = dyra.DyraLinear(s.d_in, s.d_out, rs, 0, s.dtype)
+    static.load(torch.as_tensor(np.ascontiguousarray(w.left[:, :rs] * w.sigma[:rs])),
+                torch.as_tensor(np.ascontiguousarray(w.right[:, :rs])), None, None, s.lam)
+    Ys = torch.empty_like(Y)
+    static_ms = max_over_ranks(timed(lambda: static.forward(X, B=s.B, T=s.T, Y=Ys), args.steps, 3),
+                               world, dev)
+    static_status = static.status()
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -379,10 +401,15 @@ def run_dyra(args):
         "gpu_launches": ((5 if s.k > 0 else 2) if umma else (7 if s.k > 0 else 2)) * args.steps,
         "device_status": status,
         "clocks": clk,
+        "static_matched": {"rank": rs, "flops": 2.0 * s.N * rs * (s.d_in + s.d_out),
+                           "dyra_flops": layer_flops, "us_per_layer": static_ms * 1e3,
+                           "dyra_us_per_layer": ms * 1e3, "device_status": static_status},
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"], line["parity"] = cpu_baseline(s, w, Y)
+        line["static_matched"].update(static_errors(s, w, Ys, rs, line["parity"]["rows"]))
+    static.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     layer.close()
@@ -391,6 +418,21 @@ def run_dyra(args):
 
 
 # ------------------------------------------------------------- oracle ----
+
+def static_errors(s, w, Ys_gpu, rs, rows):
+    """The FLOPs-matched static layer on the oracle's sample rows: its
+    approximation error relative to the dense product, and the GPU result
+    against the oracle's weight-only product of the same rounded factors."""
+    import oracle
+    Xr = oracle.round_to(w.X[:rows], s.dtype)
+    Us = oracle.round_to(w.left[:, :rs] * w.sigma[:rs], s.dtype)
+    Vs = oracle.round_to(w.right[:, :rs], s.dtype)
+    Yo = oracle.weight_only(Xr, Us, Vs)
+    Yd = oracle.dense(Xr, w.weight())
+    Yg = Ys_gpu[:rows].double().cpu().numpy()
+    return {"oracle_err_vs_dense": oracle.rel_fro(Yo, Yd),
+            "rel_fro_vs_oracle": oracle.rel_fro(Yg, Yo), "rows": rows}
+
 
 def oracle_inputs(s, w):
     import oracle
