@@ -7,6 +7,8 @@ smoke check in __graft_entry__.py and the CPU-baseline leg of bench.py use it.
 
 from .dyra_oracle import (  # noqa: F401
     Factors,
+    als_half_steps,
+    als_inference,
     dense,
     error_report,
     inference,

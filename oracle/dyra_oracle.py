@@ -14,6 +14,8 @@ Multiplication in DNNs" (Chae, Chung, Lee, Kim), cited below as [DyRA].
   - Appendix A, Algorithm 1: the offline and inference procedures written out.
   - Appendix D: R^(0) is the top singular vectors of the residual weight.
   - Sec. 2.4: one small SPD system per batch instance.
+  - Sec. 3.3, Fig. 9 (right): more ALS iterations (als_inference), and
+    Sec. 2.2: a Gaussian R^(0) (any R0 may be passed to the offline step).
 
 Letters. The paper writes the product as X W with W of shape c1 x c2, static
 rank k and correction rank r. This repository uses the PyTorch layout
@@ -71,14 +73,24 @@ def _projector(W_res: np.ndarray, R0: np.ndarray, lam: float) -> np.ndarray:
     return np.linalg.solve(gram, (W_res.T @ R0.T).T).T
 
 
-def offline_prepare(W: np.ndarray, r: int, k: int, lam: float) -> Factors:
+def _given_start(R0: np.ndarray, k: int, d_out: int) -> np.ndarray:
+    R0 = np.array(R0, dtype=np.float64)
+    if R0.shape != (k, d_out):
+        raise ValueError("R0 must be k x d_out = %d x %d, got %s" % (k, d_out, R0.shape))
+    return R0
+
+
+def offline_prepare(W: np.ndarray, r: int, k: int, lam: float,
+                    R0: Optional[np.ndarray] = None) -> Factors:
     """[DyRA] Alg. 1, procedure Offline Preparation, for the low-rank case.
 
     Step 2: the structured approximation is the rank-r truncated SVD
             (App. B, "Low-Rank Approximation"), with Sigma on the left factor.
     Step 3: W_res = W - W_hat.
     Step 4: R0 = top-k singular vectors of W_res on its output side (App. D;
-            the paper's "right" singular vectors of its transposed W_res).
+            the paper's "right" singular vectors of its transposed W_res),
+            unless a start R0 (k x d_out) is given, e.g. the Gaussian start
+            of Sec. 2.2.
     Step 5: P from _projector.
     """
     W = np.asarray(W, dtype=np.float64)
@@ -86,7 +98,9 @@ def offline_prepare(W: np.ndarray, r: int, k: int, lam: float) -> Factors:
     U = A[:, :r] * s[:r]
     V = Bt[:r].T.copy()
     W_res = W - U @ V.T
-    if k > 0:
+    if R0 is not None:
+        R0 = _given_start(R0, k, W.shape[0])
+    elif k > 0:
         Ares, _, _ = np.linalg.svd(W_res, full_matrices=False)
         R0 = Ares[:, :k].T.copy()
     else:
@@ -96,7 +110,8 @@ def offline_prepare(W: np.ndarray, r: int, k: int, lam: float) -> Factors:
 
 
 def offline_prepare_from_svd(left: np.ndarray, sigma: np.ndarray, right: np.ndarray,
-                             r: int, k: int, lam: float) -> Factors:
+                             r: int, k: int, lam: float,
+                             R0: Optional[np.ndarray] = None) -> Factors:
     """Alg. 1 offline preparation when W = left . diag(sigma) . right^T is given.
 
     Same steps as offline_prepare, reading the SVD instead of computing it
@@ -107,7 +122,10 @@ def offline_prepare_from_svd(left: np.ndarray, sigma: np.ndarray, right: np.ndar
     U = left[:, :r] * sigma[:r]
     V = right[:, :r].copy()
     W_res = (left[:, r:] * sigma[r:]) @ right[:, r:].T
-    R0 = left[:, r:r + k].T.copy()
+    if R0 is not None:
+        R0 = _given_start(R0, k, left.shape[0])
+    else:
+        R0 = left[:, r:r + k].T.copy()
     P = _projector(W_res, R0, lam) if k > 0 else np.zeros((right.shape[0], 0))
     return Factors(U, V, P, W_res, R0)
 
@@ -176,6 +194,64 @@ def inference_rows(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
             Yr = Yr + (xr @ P) @ C
         out[sel] = Yr
     return out
+
+
+def als_half_steps(Xb: np.ndarray, W_res: np.ndarray, R0: np.ndarray, lam: float,
+                   steps: int) -> list:
+    """Alternating ridge least squares on one instance's residual output.
+
+    [DyRA] Sec. 2.2: the residual product E = X_b W_res^T (T x d_out here) is
+    fitted by a rank-k product L R, alternating the two exact minimisers of
+    Eq. 4-5 with the ridge of footnote 2 on each Gram matrix:
+      left update   L = (X_b W_res^T R^T)(R R^T + lam I)^-1
+                      = argmin_L ||E - L R||^2 + lam ||L||^2
+      right update  R = (L^T L + lam I)^-1 (L^T X_b) W_res^T
+                      = argmin_R ||E - L R||^2 + lam ||R||^2
+    starting from the fixed R = R0 with a left update. Alg. 1 is the first two
+    half-steps (its P_L folds R0 into the left update). E is never formed: as
+    in Alg. 1, X_b multiplies W_res^T R^T and L^T X_b multiplies W_res^T.
+    Returns the pair (L, R) after each of `steps` half-steps.
+    """
+    Xb = np.asarray(Xb, dtype=np.float64)
+    k = R0.shape[0]
+    eye = np.eye(k)
+    R = np.asarray(R0, dtype=np.float64)
+    L = None
+    pairs = []
+    for h in range(steps):
+        if h % 2 == 0:
+            rhs = Xb @ (W_res.T @ R.T)                       # T x k
+            L = np.linalg.solve(R @ R.T + lam * eye, rhs.T).T
+        else:
+            R = np.linalg.solve(L.T @ L + lam * eye, (L.T @ Xb) @ W_res.T)
+        pairs.append((L, R))
+    return pairs
+
+
+def als_inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, W_res: np.ndarray,
+                  R0: np.ndarray, lam: float, B: int, T: int, t: float) -> np.ndarray:
+    """DyRA with t ALS iterations per instance ([DyRA] Sec. 3.3, Fig. 9 right).
+
+    One iteration is a left and a right update (Alg. 1 is t = 1); a half
+    iteration ends on a left update, so t = 1.5 runs L, R, L and t = 2 runs
+    L, R, L, R. The output of instance b is (X_b V) U^T + L R with the last
+    pair. t = 0 is the weight-only layer.
+    """
+    steps = int(round(2 * t))
+    if steps != 2 * t or steps < 0:
+        raise ValueError("t must be a non-negative multiple of 0.5")
+    X = np.asarray(X, dtype=np.float64)
+    if X.shape[0] != B * T:
+        raise ValueError("X has %d rows, expected B*T = %d" % (X.shape[0], B * T))
+    Y = np.empty((X.shape[0], U.shape[0]))
+    for b in range(B):
+        Xb = X[b * T:(b + 1) * T]
+        Yb = (Xb @ V) @ U.T
+        if steps > 0 and R0.shape[0] > 0:
+            L, R = als_half_steps(Xb, W_res, R0, lam, steps)[-1]
+            Yb = Yb + L @ R
+        Y[b * T:(b + 1) * T] = Yb
+    return Y
 
 
 def rel_fro(A: np.ndarray, ref: np.ndarray) -> float:

@@ -4,7 +4,8 @@
 DNNs", Appendix A, Algorithm 1, procedure Offline Preparation, low-rank case
 (App. B): truncated SVD W ~ U V^T with the singular values on U, the residual
 W_res = W - U V^T, the fixed ALS start R0 = the top-k output-side singular
-vectors of W_res (App. D), and the projector P = W_res^T R0^T (R0 R0^T +
+vectors of W_res (App. D) or a given k x d_out start (the Gaussian start of
+Sec. 2.2), and the projector P = W_res^T R0^T (R0 R0^T +
 lambda I)^-1 (Eq. 7 with the ridge of footnote 2). Computed in float64 with
 torch on the CPU; the result is what dyra_load_factors takes.
 """
@@ -25,12 +26,22 @@ class LayerFactors(NamedTuple):
 
 def _p_from_r0(W_res: torch.Tensor, R0: torch.Tensor, lam: float) -> torch.Tensor:
     k = R0.shape[0]
+    if R0.shape[1] != W_res.shape[0]:
+        raise ValueError("R0 must be k x d_out, got %s for d_out = %d" % (tuple(R0.shape), W_res.shape[0]))
     gram = R0 @ R0.T + lam * torch.eye(k, dtype=torch.float64)
     return torch.linalg.solve(gram, R0 @ W_res).T.contiguous()
 
 
-def prepare_from_weight(W, r: int, k: int, lam: float) -> LayerFactors:
-    """From a dense d_out x d_in weight (one SVD of W and one of W_res)."""
+def _start(R0, k: int):
+    R0 = torch.as_tensor(R0, dtype=torch.float64).cpu()
+    if R0.dim() != 2 or R0.shape[0] != k:
+        raise ValueError("R0 must have k = %d rows, got shape %s" % (k, tuple(R0.shape)))
+    return R0
+
+
+def prepare_from_weight(W, r: int, k: int, lam: float, R0=None) -> LayerFactors:
+    """From a dense d_out x d_in weight (one SVD of W and, without a given
+    start R0, one of W_res)."""
     W = torch.as_tensor(W, dtype=torch.float64).cpu()
     A, s, Bt = torch.linalg.svd(W, full_matrices=False)
     U = (A[:, :r] * s[:r]).contiguous()
@@ -38,11 +49,12 @@ def prepare_from_weight(W, r: int, k: int, lam: float) -> LayerFactors:
     W_res = W - U @ V.T
     if k == 0:
         return LayerFactors(U, V, torch.zeros(W.shape[1], 0, dtype=torch.float64), W_res)
-    Ar, _, _ = torch.linalg.svd(W_res, full_matrices=False)
-    return LayerFactors(U, V, _p_from_r0(W_res, Ar[:, :k].T, lam), W_res)
+    if R0 is None:
+        R0 = torch.linalg.svd(W_res, full_matrices=False)[0][:, :k].T
+    return LayerFactors(U, V, _p_from_r0(W_res, _start(R0, k), lam), W_res)
 
 
-def prepare_from_svd(left, sigma, right, r: int, k: int, lam: float) -> LayerFactors:
+def prepare_from_svd(left, sigma, right, r: int, k: int, lam: float, R0=None) -> LayerFactors:
     """From a weight given by its SVD W = left diag(sigma) right^T."""
     left = torch.as_tensor(left, dtype=torch.float64).cpu()
     sigma = torch.as_tensor(sigma, dtype=torch.float64).cpu()
@@ -52,5 +64,5 @@ def prepare_from_svd(left, sigma, right, r: int, k: int, lam: float) -> LayerFac
     W_res = (left[:, r:] * sigma[r:]) @ right[:, r:].T
     if k == 0:
         return LayerFactors(U, V, torch.zeros(right.shape[0], 0, dtype=torch.float64), W_res)
-    R0 = left[:, r:r + k].T
+    R0 = left[:, r:r + k].T if R0 is None else _start(R0, k)
     return LayerFactors(U, V, _p_from_r0(W_res, R0, lam), W_res)

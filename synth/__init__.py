@@ -1,7 +1,8 @@
 """Seeded synthetic workloads shared by the oracle, the tests and the benchmark.
 
 This package draws random numbers and nothing else: a weight matrix given by its
-singular factors W = left . diag(sigma) . right^T and an activation matrix X.
+singular factors W = left . diag(sigma) . right^T, an activation matrix X and,
+for the ALS start, a Gaussian matrix R0.
 It contains none of the DyRA arithmetic (no truncation, no residual, no
 projector, no solve); every consumer derives those on its own side.
 """
@@ -11,6 +12,7 @@ from .workloads import (  # noqa: F401
     LLAMA_SWEEP,
     LayerSpec,
     Workload,
+    gaussian_r0,
     generate,
     haar_orthonormal,
     make_activations,

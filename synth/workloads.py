@@ -177,3 +177,17 @@ def generate(s: LayerSpec, spectrum: Optional[np.ndarray] = None) -> Workload:
         if sigma.shape != (m,):
             raise ValueError("spectrum must have min(d_in, d_out) entries")
     return Workload(s, np.ascontiguousarray(X), left, sigma, right)
+
+
+def gaussian_r0(k: int, d_out: int, seed: int) -> np.ndarray:
+    """A Gaussian start R0 (k x d_out) for the alternating least squares.
+
+    The DyRA paper initialises R^(0) from a Gaussian distribution in its ALS
+    convergence study (Sec. 2.2, Fig. 2; App. E.3) without giving the variance.
+    Entries here are i.i.d. N(0, 1/d_out), so each row has squared norm about
+    1, like the orthonormal rows of the singular-vector start, and the ridge
+    term weighs the same against either. The draws come from their own stream,
+    numpy.random.default_rng([seed, 1]), so the layer draws above are unchanged.
+    """
+    rng = np.random.default_rng([seed, 1])
+    return rng.standard_normal((k, d_out)) / np.sqrt(d_out)

@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from rank_structured_matmul_b200 import dyra
-from synth import CONFIGS, LayerSpec, generate
+from synth import CONFIGS, LayerSpec, gaussian_r0, generate
 
 pytestmark = pytest.mark.gpu
 
@@ -145,6 +145,39 @@ def test_simt_variant_bf16():
     debugging variant); it meets the same bar."""
     run_spec(LayerSpec("simt", 256, 512, 64, 32, 3, 201, "bf16", 0.7, "lognormal", seed=1),
              kernels="simt")
+
+
+GAUSS = [
+    # name, d_in, d_out, r, k, B, T, dtype, x_kind (outliers: 8 channels x 20)
+    ("gauss_start_ragged", 256, 512, 64, 32, 3, 201, "bf16", "lognormal"),
+    ("gauss_start_outliers", 1024, 2048, 128, 64, 1, 128, "bf16", "outlier"),
+    ("gauss_start_f32", 96, 80, 12, 8, 3, 50, "f32", "outlier"),
+]
+
+
+@pytest.mark.parametrize("case", GAUSS, ids=[c[0] for c in GAUSS])
+def test_gaussian_start(case):
+    """A Gaussian ALS start R0 (DyRA Sec. 2.2) changes only the offline
+    projector P; the forward is the same one-step layer, checked here against
+    the oracle's t = 1 alternating least squares from that start."""
+    name, d_in, d_out, r, k, B, T, dtype, x_kind = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, x_kind, n_outlier=8,
+                  outlier_scale=20.0, seed=6)
+    w = generate(s)
+    R0 = gaussian_r0(k, d_out, s.seed)
+    fo = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, r, k, s.lam, R0=R0)
+    f = {n: oracle.round_to(a, dtype) for n, a in
+         (("X", w.X), ("U", fo.U), ("V", fo.V), ("P", fo.P), ("W_res", fo.W_res))}
+    layer = make_layer(s, f)
+    Y = layer.forward(to_dev(f["X"], dtype), B=B, T=T)
+    assert layer.status() == 0
+    check(s, Y, f, full=True)
+    layer.close()
+    # the oracle's one-step ALS from R0 is the layer the projector defines: it
+    # differs from the reference above only by P's rounding to the storage type
+    Ya = oracle.als_inference(f["X"], f["U"], f["V"], f["W_res"], fo.R0, s.lam, B, T, 1)
+    Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, B, T)
+    assert oracle.rel_fro(Ya, Yo) < TOL[dtype] / 10
 
 
 # ----------------------------------------------------------- properties ----
