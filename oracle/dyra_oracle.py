@@ -141,16 +141,20 @@ def dense(X: np.ndarray, W: np.ndarray) -> np.ndarray:
 
 
 def inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
-              W_res: np.ndarray, lam: float, B: int, T: int) -> np.ndarray:
+              W_res: np.ndarray, lam: float, B: int, T: int, *,
+              bias: Optional[np.ndarray] = None, alpha: float = 1.0) -> np.ndarray:
     """[DyRA] Alg. 1, procedure Inference, applied to each of B instances.
 
     The rows of X are B consecutive instances of T rows; the correction is
-    fitted per instance (Sec. 2.4: one SPD system "for each batch instance").
+    fitted per instance (Sec. 2.4: one small SPD system per batch instance).
     For instance b with rows X_b, the procedure's steps in order:
       static part   Y_base = X_b W_hat^T              = (X_b V) U^T
       left factor   L      = X_b P                    (T x k)
       right factor  C      = (L^T L + lam I)^-1 (L^T X_b) W_res^T   (k x d_out)
       output        Y_b    = Y_base + L C
+    Sec. 2.4 also writes the fused linear layer with a bias b (d_out) and a
+    weight alpha on the correction, Y_b = Y_base + b + alpha L C; Alg. 1 is
+    bias None and alpha 1 (the defaults).
     """
     X = np.asarray(X, dtype=np.float64)
     N = X.shape[0]
@@ -165,7 +169,9 @@ def inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, P: np.ndarray,
             L = Xb @ P
             G = L.T @ L + lam * np.eye(k)
             C = np.linalg.solve(G, (L.T @ Xb) @ W_res.T)
-            Yb = Yb + L @ C
+            Yb = Yb + alpha * (L @ C)
+        if bias is not None:
+            Yb = Yb + bias
         Y[b * T:(b + 1) * T] = Yb
     return Y
 
