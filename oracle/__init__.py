@@ -3,6 +3,8 @@
 TEST INFRASTRUCTURE ONLY. Nothing in the product (the CUDA library and its
 Python binding) imports, calls or links anything here. Only tests/, the
 smoke check in __graft_entry__.py and the CPU-baseline leg of bench.py use it.
+
+oracle.monarch holds the Monarch static part (DyRA App. B) and DyRA on top of it.
 """
 
 from .dyra_oracle import (  # noqa: F401

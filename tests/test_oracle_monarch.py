@@ -1,0 +1,215 @@
+"""Pins of the oracle's Monarch static part (DyRA App. B) and of DyRA on top of it.
+
+Paper: "DyRA: Dynamic Residual Approximation for Efficient Matrix
+Multiplication in DNNs", Appendix B ("Monarch Matrix") and Sec. 2.3 (DyRA
+corrects any structured static part).
+
+The pins check the oracle against facts that do not depend on how it is
+written:
+- the entry formula a hand derivation gives for P L P^T R, element by element;
+- exact recovery of a Monarch matrix;
+- degenerate block counts (b1 = 1 or b2 = 1), where every matrix is Monarch;
+- the block-wise Eckart-Young error, with the top singular value computed by
+  power iteration rather than by an SVD;
+- local optimality under perturbation of the factors;
+- the DyRA invariants on the Monarch base: k = 0, a fully covered residual,
+  and never worse than weight-only.
+test_planted_monarch_mistakes_are_caught swaps mistaken copies into the
+module and checks that some pin fails for each.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import dyra_oracle as orc
+from oracle import monarch as mon
+from synth import LayerSpec, generate
+
+
+def random_blocks(b1, b2, seed):
+    rng = np.random.default_rng(seed)
+    return ([rng.standard_normal((b1, b1)) for _ in range(b2)],
+            [rng.standard_normal((b2, b2)) for _ in range(b1)])
+
+
+def square_layer(N, k, B=2, T=9, seed=0, lam=1e-3):
+    s = LayerSpec("mon", N, N, 1, k, B, T, "f32", 0.5, "lognormal", seed=seed, lam=lam)
+    return s, generate(s)
+
+
+def top_singular_value(S, iters=500):
+    """Power iteration on S^T S (no SVD routine)."""
+    v = np.ones(S.shape[1]) / np.sqrt(S.shape[1])
+    for _ in range(iters):
+        w = S.T @ (S @ v)
+        v = w / np.linalg.norm(w)
+    return np.linalg.norm(S @ v)
+
+
+# ---------------------------------------------------------------- pins ----
+
+def check_entry_formula():
+    """Entry (m1*b2 + j2, j1*b2 + i2) of P L P^T R is L_j2[m1, j1] R_j1[j2, i2]."""
+    for b1, b2 in ((3, 4), (2, 5), (4, 4)):
+        Lb, Rb = random_blocks(b1, b2, seed=b1 * 10 + b2)
+        W = mon.monarch_matrix(Lb, Rb)
+        for m1 in range(b1):
+            for j2 in range(b2):
+                for j1 in range(b1):
+                    for i2 in range(b2):
+                        want = Lb[j2][m1, j1] * Rb[j1][j2, i2]
+                        assert abs(W[m1 * b2 + j2, j1 * b2 + i2] - want) <= 1e-12
+
+
+def check_shuffle_is_a_permutation():
+    for b1, b2 in ((3, 4), (1, 5), (5, 1)):
+        P = mon.shuffle(b1, b2)
+        np.testing.assert_array_equal(P @ P.T, np.eye(b1 * b2))
+        assert set(np.unique(P)) <= {0.0, 1.0}
+
+
+def check_recovers_monarch_matrices():
+    for b1, b2 in ((3, 4), (2, 5), (4, 4)):
+        W = mon.monarch_matrix(*random_blocks(b1, b2, seed=7 + b1))
+        Lb, Rb = mon.monarch_project(W, b1, b2)
+        np.testing.assert_allclose(mon.monarch_matrix(Lb, Rb), W, rtol=0, atol=1e-11)
+
+
+def check_degenerate_block_counts_are_exact():
+    """b1 = 1: L is diagonal and R one N x N block; b2 = 1: L one block and R
+    diagonal. Either way every N x N matrix is Monarch."""
+    rng = np.random.default_rng(3)
+    for b1, b2 in ((1, 6), (6, 1)):
+        W = rng.standard_normal((6, 6))
+        Lb, Rb = mon.monarch_project(W, b1, b2)
+        np.testing.assert_allclose(mon.monarch_matrix(Lb, Rb), W, rtol=0, atol=1e-12)
+
+
+def check_blockwise_eckart_young():
+    """||W - W_hat||^2 = sum over the (j1, j2) blocks S of ||S||^2 - s1(S)^2."""
+    b1, b2 = 3, 4
+    W = np.random.default_rng(5).standard_normal((12, 12))
+    Lb, Rb = mon.monarch_project(W, b1, b2)
+    err = np.sum((W - mon.monarch_matrix(Lb, Rb)) ** 2)
+    want = 0.0
+    for j1 in range(b1):
+        for j2 in range(b2):
+            S = np.array([[W[m1 * b2 + j2, j1 * b2 + i2] for i2 in range(b2)] for m1 in range(b1)])
+            want += np.sum(S ** 2) - top_singular_value(S) ** 2
+    assert err == pytest.approx(want, rel=1e-9)
+
+
+def check_locally_optimal():
+    """No small perturbation of the projected factors lowers the error."""
+    b1, b2 = 3, 4
+    rng = np.random.default_rng(6)
+    W = rng.standard_normal((12, 12))
+    Lb, Rb = mon.monarch_project(W, b1, b2)
+    best = np.sum((W - mon.monarch_matrix(Lb, Rb)) ** 2)
+    for _ in range(50):
+        Lp = [L + 1e-3 * rng.standard_normal(L.shape) for L in Lb]
+        Rp = [R + 1e-3 * rng.standard_normal(R.shape) for R in Rb]
+        assert np.sum((W - mon.monarch_matrix(Lp, Rp)) ** 2) >= best * (1 - 1e-12)
+
+
+def check_dyra_k0_is_the_monarch_product():
+    s, w = square_layer(12, 0)
+    f = mon.offline_prepare_monarch(w.weight(), 3, 4, 0, s.lam)
+    Y = mon.monarch_inference(w.X, f, s.lam, s.B, s.T)
+    np.testing.assert_allclose(Y, w.X @ mon.monarch_matrix(f.Lb, f.Rb), rtol=0, atol=1e-12)
+
+
+def check_dyra_full_residual_is_exact():
+    """k = N and lam = 0 with T >= N: col(X P) = col(X_b) holds the residual
+    output X_b W_res^T, so the correction restores X W^T."""
+    s, w = square_layer(12, 12, T=20, lam=0.0, seed=1)
+    f = mon.offline_prepare_monarch(w.weight(), 3, 4, 12, 0.0)
+    Y = mon.monarch_inference(w.X, f, 0.0, s.B, s.T)
+    Yd = w.X @ w.weight().T
+    np.testing.assert_allclose(Y, Yd, rtol=0, atol=1e-9 * np.abs(Yd).max())
+
+
+def check_dyra_never_worse_than_weight_only():
+    s, w = square_layer(12, 3, seed=2)
+    f = mon.offline_prepare_monarch(w.weight(), 3, 4, 3, s.lam)
+    Y = mon.monarch_inference(w.X, f, s.lam, s.B, s.T)
+    Yd = w.X @ w.weight().T
+    Ywo = w.X @ f.What.T
+    for b in range(s.B):
+        rows = slice(b * s.T, (b + 1) * s.T)
+        assert np.linalg.norm(Yd[rows] - Y[rows]) <= np.linalg.norm(Yd[rows] - Ywo[rows]) * (1 + 1e-12)
+    # and the static part is the Monarch product of the weight's projection
+    np.testing.assert_allclose(f.What, mon.monarch_matrix(*mon.monarch_project(w.weight().T, 3, 4)).T,
+                               rtol=0, atol=1e-12)
+
+
+PINS = [check_entry_formula, check_shuffle_is_a_permutation, check_recovers_monarch_matrices,
+        check_degenerate_block_counts_are_exact, check_blockwise_eckart_young, check_locally_optimal,
+        check_dyra_k0_is_the_monarch_product, check_dyra_full_residual_is_exact,
+        check_dyra_never_worse_than_weight_only]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
+def test_monarch_pin(pin):
+    pin()
+
+
+def test_rejects_non_square():
+    with pytest.raises(ValueError):
+        mon.monarch_project(np.zeros((12, 8)), 3, 4)
+
+
+def test_parameter_count():
+    """N (b1 + b2) parameters: b2 blocks of b1 x b1 and b1 blocks of b2 x b2."""
+    Lb, Rb = mon.monarch_project(np.random.default_rng(0).standard_normal((12, 12)), 3, 4)
+    assert len(Lb) == 4 and all(L.shape == (3, 3) for L in Lb)
+    assert len(Rb) == 3 and all(R.shape == (4, 4) for R in Rb)
+    assert sum(L.size for L in Lb) + sum(R.size for R in Rb) == 12 * (3 + 4)
+
+
+# ------------------------------------------------------ planted bugs ----
+
+_SHUFFLE, _PROJECT, _MATRIX = mon.shuffle, mon.monarch_project, mon.monarch_matrix
+
+
+def _identity_shuffle(b1, b2):
+    return np.eye(b1 * b2)
+
+
+def _contiguous_rows(Wp, b1, b2):
+    """Takes rows j2*b1 .. j2*b1 + b1 - 1 instead of the strided ones."""
+    Lb = [np.zeros((b1, b1)) for _ in range(b2)]
+    Rb = [np.zeros((b2, b2)) for _ in range(b1)]
+    for j1 in range(b1):
+        for j2 in range(b2):
+            u, s, vt = np.linalg.svd(Wp[j2 * b1:(j2 + 1) * b1, j1 * b2:(j1 + 1) * b2])
+            Lb[j2][:, j1] = np.sqrt(s[0]) * u[:, 0]
+            Rb[j1][j2, :] = np.sqrt(s[0]) * vt[0]
+    return Lb, Rb
+
+
+def _sigma_twice(Wp, b1, b2):
+    Lb, Rb = _PROJECT(Wp, b1, b2)
+    return [L * 1.0 for L in Lb], [R * 2.0 for R in Rb]
+
+
+def _swapped_factors(Lb, Rb):
+    b2, b1 = len(Lb), len(Rb)
+    P = _SHUFFLE(b1, b2)
+    return P @ mon.block_diag(Rb) @ P.T @ mon.block_diag(Lb) if b1 == b2 else _MATRIX(Lb, Rb).T
+
+
+MUTANTS = [("shuffle", _identity_shuffle), ("monarch_project", _contiguous_rows),
+           ("monarch_project", _sigma_twice), ("monarch_matrix", _swapped_factors)]
+
+
+@pytest.mark.parametrize("target,mutant", MUTANTS, ids=lambda m: getattr(m, "__name__", m))
+def test_planted_monarch_mistakes_are_caught(monkeypatch, target, mutant):
+    monkeypatch.setattr(mon, target, mutant)
+    failures = 0
+    for pin in PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError, np.linalg.LinAlgError):
+            failures += 1
+    assert failures > 0, "no pin catches the planted mistake %s" % mutant.__name__
