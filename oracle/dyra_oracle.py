@@ -1,4 +1,4 @@
-"""Plain fp64 reference of DyRA with one-step ALS residual approximation.
+"""Plain fp64 reference of the DyRA layer: a static part plus a one-step ALS correction.
 
 TEST INFRASTRUCTURE ONLY: used by tests/, by the smoke check and by the
 CPU-baseline leg of the benchmark. The CUDA library never calls into it and it
@@ -12,7 +12,7 @@ Multiplication in DNNs" (Chae, Chung, Lee, Kim), cited below as [DyRA].
   - Sec. 2.3, Eq. 6-7: one ALS iteration; the left factor's projector P_L is
     precomputed offline.
   - Appendix A, Algorithm 1: the offline and inference procedures written out.
-  - Appendix D: R^(0) is the top singular vectors of the residual weight.
+  - Appendix D: R^(0) is taken from the leading singular directions of W_res.
   - Sec. 2.4: one small SPD system per batch instance.
   - Sec. 3.3, Fig. 9 (right): more ALS iterations (als_inference), and
     Sec. 2.2: a Gaussian R^(0) (any R0 may be passed to the offline step).
