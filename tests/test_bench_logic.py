@@ -37,3 +37,35 @@ def test_algorithmic_counts_the_correction():
     flops, _, total, _ = bench.algorithmic(s)
     assert flops["gram"] == 0 and flops["solve"] == 0 and flops["rfactor"] == 0
     assert total == pytest.approx(2.0 * s.N * s.r * (s.d_in + s.d_out))
+
+
+def _run_reference(env_extra, workload="tiny_f32"):
+    import json
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", workload, "--steps", "3", "--warmup", "3"],
+                         cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_the_contract_line():
+    """The reference arm (the fp64 oracle on the host cores) prints one JSON
+    line with the keys the benchmark contract names, on the workload asked."""
+    (line,) = _run_reference({"RANK": "0", "WORLD_SIZE": "1"})
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 3 and line["warmup"] == 3
+    assert line["config"]["workload"] == "tiny_f32" and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
