@@ -8,7 +8,8 @@ from a Gaussian R^(0)) and Sec. 3.3, Fig. 9 right (t = 1, 1.5, 2 iterations).
 As in test_oracle.py, no pin re-types the oracle's update formulas: each
 checks them against an optimality condition, a monotonicity property of
 alternating minimisation, the Eckart-Young optimum they converge to, a closed
-form, or a least-squares solve of the augmented system by another routine.
+form, exact rational arithmetic of the rank-1 case worked by hand, or a
+least-squares solve of the augmented system by another routine.
 test_planted_als_mistakes_are_caught swaps a mistaken copy into the oracle
 module and checks that some pin fails.
 """
@@ -194,7 +195,34 @@ def check_iteration_count():
         np.testing.assert_allclose(Y, want, rtol=0, atol=1e-11 * np.abs(want).max())
 
 
-PINS = [check_t1_is_algorithm_1, check_t0_is_weight_only, check_half_step_closed_form,
+def check_rank1_exact_rationals():
+    """k = 1 by hand: each update is a scalar ridge regression,
+    L_i = sum_j E_ij R_j / (sum_j R_j^2 + lam) and
+    R_j = sum_i L_i E_ij / (sum_i L_i^2 + lam),
+    run here in exact rational arithmetic on a 3 x 2 residual output."""
+    from fractions import Fraction as F
+    Wres = [[3, 1, 0], [0, 2, 1]]                    # d_out x d_in
+    E = [[F(Wres[j][i]) for j in range(2)] for i in range(3)]   # X_b = I: E = W_res^T
+    for lam in (F(0), F(1, 2)):
+        R = [F(1), F(-2)]
+        L = None
+        want = []
+        for h in range(5):
+            if h % 2 == 0:
+                den = sum(r * r for r in R) + lam
+                L = [sum(E[i][j] * R[j] for j in range(2)) / den for i in range(3)]
+            else:
+                den = sum(l * l for l in L) + lam
+                R = [sum(L[i] * E[i][j] for i in range(3)) / den for j in range(2)]
+            want.append((list(L), list(R)))
+        got = orc.als_half_steps(np.eye(3), np.array(Wres, dtype=np.float64),
+                                 np.array([[1.0, -2.0]]), float(lam), 5)
+        for (wl, wr), (gl, gr) in zip(want, got):
+            np.testing.assert_allclose(gl[:, 0], [float(x) for x in wl], rtol=1e-13, atol=0)
+            np.testing.assert_allclose(gr[0], [float(x) for x in wr], rtol=1e-13, atol=0)
+
+
+PINS = [check_rank1_exact_rationals, check_t1_is_algorithm_1, check_t0_is_weight_only, check_half_step_closed_form,
         check_half_steps_are_ridge_minimisers, check_objective_never_increases,
         check_converges_to_eckart_young, check_matches_augmented_lstsq,
         check_never_worse_than_weight_only, check_iteration_count]
