@@ -222,7 +222,29 @@ def check_rank1_exact_rationals():
             np.testing.assert_allclose(gr[0], [float(x) for x in wr], rtol=1e-13, atol=0)
 
 
-PINS = [check_rank1_exact_rationals, check_t1_is_algorithm_1, check_t0_is_weight_only, check_half_step_closed_form,
+def check_t15_closed_form():
+    """t = 1.5 by hand from Alg. 1's quantities. With G = L^T L + lam I,
+    Q = (L^T X_b) W_res^T and S = Q Q^T, the second L update simplifies to
+    L(2) = X_b (Q W_res)^T (S + lam G^2)^-1 G, and the output adds L(2) R(1)
+    = X_b (Q W_res)^T (S + lam G^2)^-1 Q."""
+    s, w = layer(seed=12, x_kind="outlier")
+    for lam in (0.0, 1e-3, 0.05):
+        f = factors(w, s, lam, "gauss")
+        Y = orc.als_inference(w.X, f.U, f.V, f.W_res, f.R0, lam, s.B, s.T, 1.5)
+        for b in range(s.B):
+            Xb = w.X[b * s.T:(b + 1) * s.T]
+            L = Xb @ f.P
+            G = L.T @ L + lam * np.eye(s.k)
+            Q = (L.T @ Xb) @ f.W_res.T
+            M = (Xb @ (Q @ f.W_res).T) @ np.linalg.inv(Q @ Q.T + lam * G @ G)
+            want = Xb @ f.V @ f.U.T + M @ Q
+            got = Y[b * s.T:(b + 1) * s.T]
+            np.testing.assert_allclose(got, want, rtol=0, atol=1e-10 * np.abs(want).max())
+            L2 = orc.als_half_steps(Xb, f.W_res, f.R0, lam, 3)[-1][0]
+            np.testing.assert_allclose(L2, M @ G, rtol=0, atol=1e-10 * np.abs(L2).max())
+
+
+PINS = [check_rank1_exact_rationals, check_t15_closed_form, check_t1_is_algorithm_1, check_t0_is_weight_only, check_half_step_closed_form,
         check_half_steps_are_ridge_minimisers, check_objective_never_increases,
         check_converges_to_eckart_young, check_matches_augmented_lstsq,
         check_never_worse_than_weight_only, check_iteration_count]
