@@ -3,9 +3,30 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace dyra {
+
+// Launch set-up of one kernel, per device: cudaFuncSetAttribute acts on the
+// current device only, so each device of a process is configured on its own
+// (plans on several devices may share the process and run from several host
+// threads; setting an attribute twice is harmless).
+constexpr int kMaxDevices = 64;
+struct KernelSetup {
+  std::atomic<uint32_t> smem[kMaxDevices];  // dynamic shared memory configured so far
+  std::atomic<int> occupancy[kMaxDevices];  // cached occupancy figure (e.g. resident pairs)
+};
+
+// The current device, or -1 if it cannot be read or is beyond kMaxDevices.
+inline int setup_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return d < kMaxDevices ? d : -1;
+}
 
 struct DeviceInfo {
   int device = 0;

@@ -716,14 +716,16 @@ template <typename TOut, int KMAX>
 int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, int splits, int64_t B, int k,
                      int d_in, float lambda, TOut* Tp, int* status, unsigned long long* trace) {
   auto kfn = solve_ldl_kernel<TOut, KMAX>;
-  static bool configured = false;
-  if (!configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (setup.smem[d].load() == 0) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(SolveSmem<KMAX>))) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = true;
+    setup.smem[d].store(static_cast<uint32_t>(sizeof(SolveSmem<KMAX>)));
   }
   cfg.gridDim = dim3(static_cast<unsigned>(B),
                      static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
@@ -753,12 +755,14 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
-  static size_t configured = 48 * 1024;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (smem > 48 * 1024 && smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(static_cast<uint32_t>(smem));
   }
   cfg.gridDim = dim3(static_cast<unsigned>(B), static_cast<unsigned>((d_in + kSolveThreads - 1) / kSolveThreads));
   cfg.blockDim = dim3(kSolveThreads);
@@ -785,14 +789,16 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
                        int* flags, int64_t B, int64_t T, int k, float lambda, int* status,
                        int defer_wait, unsigned long long* trace) {
   auto kfn = ltilde_kernel<KMAX, MODE>;
-  static bool configured = false;
-  if (!configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (setup.smem[d].load() == 0) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(LtSmem<KMAX>))) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = true;
+    setup.smem[d].store(static_cast<uint32_t>(sizeof(LtSmem<KMAX>)));
   }
   // blockIdx.x = instance, blockIdx.y = chunk of rows: the chunk-0 CTAs (the
   // factoring ones in the shared mode) are the grid's first B CTAs.
@@ -836,12 +842,14 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
                : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
                                                     status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
-  static size_t configured = 48 * 1024;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (smem > 48 * 1024 && smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(ltilde_general_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(static_cast<uint32_t>(smem));
   }
   if ((T + kSolveThreads - 1) / kSolveThreads > 65535) return -1;
   cfg.gridDim = dim3(static_cast<unsigned>(B),

@@ -783,14 +783,16 @@ int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& 
                 cudaStream_t s, bool pdl, int cluster = 1) {
   if (p.c.num_tiles <= 0) return 0;
   auto kfn = umma_gemm_kernel<Pol>;
-  static uint32_t configured = 0;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = dev.device;
+  if (d < 0 || d >= kMaxDevices) return -1;
+  if (smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(smem);
   }
   cudaLaunchConfig_t cfg = {};
   // with clusters every CTA takes exactly one tile (the grid is the tile count)
@@ -824,27 +826,29 @@ int launch_gemm_pair(const typename Pol::Params& p, uint32_t smem, const DeviceI
                      cudaStream_t s, bool pdl) {
   if (p.c.num_tiles <= 0) return 0;
   auto kfn = umma_gemm_pair_kernel<Pol>;
-  static uint32_t configured = 0;
-  static int max_pairs = 0;
+  static KernelSetup setup;  // occupancy: resident pairs at the configured size
+  const int d = dev.device;
+  if (d < 0 || d >= kMaxDevices) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  if (smem > configured) {
+  if (smem > setup.smem[d].load() || setup.occupancy[d].load() < 1) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = smem;
     cfg.gridDim = dim3(2 * (dev.sm_count / 2));
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kfn, &cfg) != cudaSuccess || clusters < 1) {
       cudaGetLastError();
       clusters = dev.sm_count / 2;
     }
-    max_pairs = clusters;
+    setup.occupancy[d].store(clusters);
+    if (smem > setup.smem[d].load()) setup.smem[d].store(smem);
   }
+  const int max_pairs = setup.occupancy[d].load();
   cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min(p.c.num_tiles, max_pairs)));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
