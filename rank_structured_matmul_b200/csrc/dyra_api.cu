@@ -189,41 +189,44 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   return DYRA_OK;
 }
 
-// Launch the bf16 forward, through a cached CUDA graph when possible: one
-// cudaGraphLaunch replaces five kernel launches and twelve tensor-map
-// encodings. Graphs are not used while the caller's stream is being captured
-// (the launches then go into the caller's graph), with stage timing or
-// tracing on, or when DYRA_GRAPHS=0.
-int launch_bf16_maybe_graph(dyra_plan* p, const dyra::Bf16Forward& a, cudaStream_t s) {
+// Launch a forward through a cached CUDA graph when possible: one
+// cudaGraphLaunch replaces its kernel launches (five for the tensor-core
+// path, seven for the CUDA-core path) and, for the tensor-core path, twelve
+// tensor-map encodings. Graphs are not used while the caller's stream is being
+// captured (the launches then go into the caller's graph), when `direct` is
+// set (stage timing or tracing), or when DYRA_GRAPHS=0. `launch(stream)`
+// enqueues the forward's kernels on `stream` and returns 0 on success.
+template <class Launch>
+int launch_maybe_graph(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T,
+                       bool weight_only, bool direct, cudaStream_t s, const Launch& launch) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (!p->use_graphs || a.stage_events || a.trace ||
-      cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+  if (!p->use_graphs || direct || cudaStreamIsCapturing(s, &cs) != cudaSuccess ||
+      cs != cudaStreamCaptureStatusNone) {
     cudaGetLastError();
-    return dyra::launch_bf16_forward(a, p->dev, s);
+    return launch(s);
   }
   dyra_plan::GraphEntry* hit = nullptr;
   for (auto& g : p->graphs)
-    if (g.exec && g.X == a.X && g.Y == a.Y && g.B == a.B && g.T == a.T &&
-        g.weight_only == a.weight_only)
+    if (g.exec && g.X == X && g.Y == Y && g.B == B && g.T == T && g.weight_only == weight_only)
       hit = &g;
   if (!hit) {
     if (!p->capture_stream &&
         cudaStreamCreateWithFlags(&p->capture_stream, cudaStreamNonBlocking) != cudaSuccess)
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     cudaGraph_t graph = nullptr;
     if (cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal) !=
         cudaSuccess) {
       cudaGetLastError();
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     }
-    const int lrc = dyra::launch_bf16_forward(a, p->dev, p->capture_stream);
+    const int lrc = launch(p->capture_stream);
     const cudaError_t ec = cudaStreamEndCapture(p->capture_stream, &graph);
     cudaGraphExec_t exec = nullptr;
     if (lrc != 0 || ec != cudaSuccess || graph == nullptr ||
         cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
       if (graph) cudaGraphDestroy(graph);
       cudaGetLastError();
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     }
     cudaGraphDestroy(graph);
     hit = &p->graphs[0];
@@ -235,11 +238,11 @@ int launch_bf16_maybe_graph(dyra_plan* p, const dyra::Bf16Forward& a, cudaStream
       if (g.used < hit->used) hit = &g;
     }
     if (hit->exec) cudaGraphExecDestroy(hit->exec);
-    hit->X = a.X;
-    hit->Y = a.Y;
-    hit->B = a.B;
-    hit->T = a.T;
-    hit->weight_only = a.weight_only;
+    hit->X = X;
+    hit->Y = Y;
+    hit->B = B;
+    hit->T = T;
+    hit->weight_only = weight_only;
     hit->exec = exec;
   }
   hit->used = ++p->graph_clock;
@@ -295,7 +298,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.trace = p->trace;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
-    rc = launch_bf16_maybe_graph(p, a, s);
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
+                            [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
@@ -317,7 +321,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<__nv_bfloat16*>(p->Tp);
     a.Cm = static_cast<__nv_bfloat16*>(p->Ct);
     a.status = p->status;
-    rc = dyra::launch_simt_forward(a, p->dev, s);
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
+                            [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   } else {
     dyra::SimtForward<float> a;
     a.d_in = p->d_in;
@@ -338,7 +343,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<float*>(p->Tp);
     a.Cm = static_cast<float*>(p->Ct);
     a.status = p->status;
-    rc = dyra::launch_simt_forward(a, p->dev, s);
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
+                            [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   }
   if (rc != 0) {
     cudaGetLastError();
