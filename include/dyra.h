@@ -99,6 +99,20 @@ int dyra_load_factors(dyra_plan_t p, const void *U, const void *V, const void *P
                       const void *W_res, float lambda, dyra_stream_t stream);
 
 /*
+ * The full linear layer of [DyRA] Sec. 2.4: every later forward computes
+ * Y = (X V) U^T + b + alpha * (correction), the correction being the rank-k
+ * term of Alg. 1. Before any call there is no bias and alpha = 1 (Alg. 1).
+ *   bias  : device pointer to d_out values in the plan dtype, 16-byte aligned,
+ *           copied into a plan-owned buffer on `stream` (the caller may free it
+ *           once the stream has passed this call); NULL removes the bias.
+ *   alpha : finite weight of the correction (0 leaves the static part and b).
+ * dyra_forward_weight_only adds the bias too. Errors: DYRA_ERR_INVALID_ARG (NULL
+ * plan, non-finite alpha), DYRA_ERR_ALIGNMENT, DYRA_ERR_ALLOC, DYRA_ERR_CUDA;
+ * the plan is unchanged on error.
+ */
+int dyra_set_linear(dyra_plan_t p, const void *bias, float alpha, dyra_stream_t stream);
+
+/*
  * Y = DyRA(X) for one instance of N rows (B = 1, T = N).
  *   X : N x d_in input, Y : N x d_out output (overwritten), N >= 0.
  * N == 0 is a no-op. Returns DYRA_ERR_RANK_DEFICIENT if lambda == 0 and N < k.

@@ -31,6 +31,10 @@ struct dyra_plan {
   // the blocks fit the SMs).
   int factor_mode = -1;
   float lambda = 0.f;
+  // full linear layer (dyra_set_linear): Y = static + bias + alpha * correction
+  void* bias = nullptr;  // d_out values in the plan dtype (allocated on first use)
+  bool has_bias = false;
+  float alpha = 1.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
   void* U = nullptr;     // d_out x r
@@ -298,6 +302,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.trace = p->trace;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.bias = p->has_bias ? p->bias : nullptr;
+    a.alpha = p->alpha;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
                             [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
@@ -321,6 +327,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<__nv_bfloat16*>(p->Tp);
     a.Cm = static_cast<__nv_bfloat16*>(p->Ct);
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const __nv_bfloat16*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   } else {
@@ -343,6 +351,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<float*>(p->Tp);
     a.Cm = static_cast<float*>(p->Ct);
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const float*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   }
@@ -514,6 +524,27 @@ int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P
   return DYRA_OK;
 }
 
+int dyra_set_linear(dyra_plan_t p, const void* bias, float alpha, dyra_stream_t stream) {
+  if (p == nullptr || !std::isfinite(alpha)) return DYRA_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return DYRA_ERR_ALIGNMENT;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  const size_t bytes = static_cast<size_t>(p->d_out) * elem_size(p->dtype);
+  int rc;
+  if (bias != nullptr) {
+    if (!p->bias && (rc = dev_alloc(&p->bias, bytes))) return rc;
+    if (cudaMemcpyAsync(p->bias, bias, bytes, cudaMemcpyDeviceToDevice,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+      cudaGetLastError();
+      return DYRA_ERR_CUDA;
+    }
+  }
+  p->has_bias = bias != nullptr;
+  p->alpha = alpha;
+  drop_graphs(p);  // the bias pointer and alpha are baked into captured launches
+  return DYRA_OK;
+}
+
 int dyra_forward(dyra_plan_t p, const void* X, void* Y, int64_t N, dyra_stream_t stream) {
   return run_forward(p, X, Y, 1, N, false, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -556,6 +587,7 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->VPt);
     dev_free(p->U);
     dev_free(p->W_res);
+    dev_free(p->bias);
     dev_free(p->Z);
     dev_free(p->L);
     void* tg = p->TG;
@@ -679,7 +711,7 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         256;
+         256 + (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
 }  // extern "C"
@@ -808,6 +840,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.trace = nullptr;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.bias = p->has_bias ? p->bias : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
@@ -833,6 +867,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Cm = k > 0 ? static_cast<__nv_bfloat16*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
                  : nullptr;
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const __nv_bfloat16*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_simt_forward(a, p->dev, s);
   } else {
     dyra::SimtForward<float> a;
@@ -858,6 +894,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Cm = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
                  : nullptr;
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const float*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_simt_forward(a, p->dev, s);
   }
   if (rc != 0) {

@@ -73,6 +73,8 @@ struct Bf16Forward {
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
   bool use_pairs;             // run the output stage on CTA pairs
   int proj_pair_min_tiles;    // see proj_shape (0: default)
+  const void* bias = nullptr;  // d_out bf16 values added to Y, or nullptr
+  float alpha = 1.f;           // weight of the correction (the solve scales L~ by it)
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -115,6 +117,8 @@ struct SimtForward {
   T* Tp;        // (B*k) x d_in
   T* Cm;        // (B*k) x d_out
   int* status;
+  const T* bias = nullptr;  // d_out values added to Y, or nullptr
+  float alpha = 1.f;        // weight of the correction
 };
 
 template <typename T>
@@ -136,9 +140,10 @@ int factor_record_floats(int k);
 // defer_wait (with pdl): the grid launched just before waited for the one
 // that wrote G and L before letting this one start; this grid then waits
 // for it only before its blocks exit.
+// alpha scales the result (the correction weight of the full linear layer).
 int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
-                  unsigned long long* trace);
+                  int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+                  bool defer_wait, unsigned long long* trace);
 // Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
 size_t ltilde_smem_bytes(int k);
 int ltilde_rows_per_block(int k);

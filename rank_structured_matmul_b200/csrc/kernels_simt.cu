@@ -369,7 +369,8 @@ static_assert(offsetof(LdlBlockScratch<32>, Wb) % 16 == 0 &&
 template <int KMAX, int MODE>
 __global__ void __maxnreg__(152)
     ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, float* MD, int* flags, int T,
-                  int k, float lambda, int* status, int defer_wait, unsigned long long* trace) {
+                  int k, float lambda, float alpha, int* status, int defer_wait,
+                  unsigned long long* trace) {
   using Sm = LtSmem<KMAX>;
   constexpr int LD = LdlBlockScratch<KMAX>::LD;
   constexpr int ROWS = lt_rows<KMAX>();
@@ -550,10 +551,11 @@ __global__ void __maxnreg__(152)
       const int rl = p0 + RT * rg + rr;
       if (rl >= nrows || 4 * cg >= k) continue;
       __nv_bfloat16* dst = rows + static_cast<size_t>(rl) * k + 4 * cg;
-      const __nv_bfloat162 lo =
-          __floats2bfloat162_rn(zero ? 0.f : acc[rr][0], zero ? 0.f : acc[rr][1]);
-      const __nv_bfloat162 hi =
-          __floats2bfloat162_rn(zero ? 0.f : acc[rr][2], zero ? 0.f : acc[rr][3]);
+      // a failed factorisation writes zeros (not alpha times a non-finite value)
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][0],
+                                                      zero ? 0.f : alpha * acc[rr][1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][2],
+                                                      zero ? 0.f : alpha * acc[rr][3]);
       uint2 w;
       w.x = *reinterpret_cast<const uint32_t*>(&lo);
       w.y = *reinterpret_cast<const uint32_t*>(&hi);
@@ -571,7 +573,7 @@ __global__ void __maxnreg__(152)
 // of L_b, one per thread.
 __global__ void __launch_bounds__(kSolveThreads)
     ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, int T, int k,
-                          float lambda, int* status, int defer_wait) {
+                          float lambda, float alpha, int* status, int defer_wait) {
   extern __shared__ float sm[];
   const int ldg = k + 1;
   float* R = sm;                // k x (k+1): lower triangle becomes R
@@ -625,20 +627,22 @@ __global__ void __launch_bounds__(kSolveThreads)
     }
     const bool zero = bad != 0;
     for (int i = 0; i < k; ++i)
-      row[i] = __float2bfloat16_rn(zero ? 0.f : Ycol[i * kSolveThreads + tid]);
+      row[i] = __float2bfloat16_rn(zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid]);
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   if (defer_wait) sm100::pdl_wait();
 }
 
-// C[b][m][n] (+)= sum_q A[b][m][q] * Bm[b][q][n] with arbitrary element strides.
+// C[b][m][n] (+)= alpha sum_q A[b][m][q] * Bm[b][q][n] (+ bias[n]) with
+// arbitrary element strides.
 constexpr int kGT = 64;   // tile
 constexpr int kGK = 16;   // k step
 template <typename TA, typename TB, typename TC>
 __global__ void __launch_bounds__(256)
     simt_gemm_kernel(int M, int N, int K, const TA* __restrict__ A, int64_t am, int64_t ak,
                      int64_t ab, const TB* __restrict__ Bm, int64_t bk, int64_t bn, int64_t bb,
-                     TC* __restrict__ C, int64_t cm, int64_t cn, int64_t cb, int accumulate) {
+                     TC* __restrict__ C, int64_t cm, int64_t cn, int64_t cb, int accumulate,
+                     float alpha, const TC* __restrict__ bias) {
   __shared__ float As[kGK][kGT + 1];
   __shared__ float Bs[kGK][kGT + 1];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -680,7 +684,8 @@ __global__ void __launch_bounds__(256)
       const int gn = n0 + tx + 16 * j;
       if (gn >= N) continue;
       TC* dst = C + gm * cm + gn * cn;
-      float v = acc[i][j];
+      float v = alpha * acc[i][j];
+      if (bias) v += to_f<TC>(bias[gn]);
       if (accumulate) v += to_f<TC>(*dst);
       *dst = from_f<TC>(v);
     }
@@ -690,11 +695,12 @@ __global__ void __launch_bounds__(256)
 template <typename TA, typename TB, typename TC>
 int gemm(int M, int N, int K, const TA* A, int64_t am, int64_t ak, int64_t ab, const TB* Bm,
          int64_t bk, int64_t bn, int64_t bb, TC* C, int64_t cm, int64_t cn, int64_t cb,
-         int batches, int accumulate, cudaStream_t s) {
+         int batches, int accumulate, cudaStream_t s, float alpha = 1.f,
+         const TC* bias = nullptr) {
   if (M <= 0 || N <= 0 || batches <= 0) return 0;
   dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, batches);
   simt_gemm_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb, C,
-                                                    cm, cn, cb, accumulate);
+                                                    cm, cn, cb, accumulate, alpha, bias);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -786,8 +792,8 @@ size_t ltilde_smem_bytes(int k) {
 
 template <int KMAX, int MODE>
 int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L, float* MD,
-                       int* flags, int64_t B, int64_t T, int k, float lambda, int* status,
-                       int defer_wait, unsigned long long* trace) {
+                       int* flags, int64_t B, int64_t T, int k, float lambda, float alpha,
+                       int* status, int defer_wait, unsigned long long* trace) {
   auto kfn = ltilde_kernel<KMAX, MODE>;
   static KernelSetup setup;
   const int d = setup_device();
@@ -806,15 +812,15 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
                      static_cast<unsigned>((T + lt_rows<KMAX>() - 1) / lt_rows<KMAX>()));
   cfg.blockDim = dim3(kLtThreads);
   cfg.dynamicSmemBytes = sizeof(LtSmem<KMAX>);
-  return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, status,
-                            defer_wait, trace) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, alpha,
+                            status, defer_wait, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
 int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
-                  unsigned long long* trace) {
+                  int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+                  bool defer_wait, unsigned long long* trace) {
   const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
   if (k % 8 != 0) return -1;  // bf16 plans: 16-byte rows of L
@@ -832,15 +838,15 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   if (k <= 32)
     return mode == kSolveShared
                ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, dw, trace)
+                                                      alpha, status, dw, trace)
                : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, dw, trace);
+                                                    alpha, status, dw, trace);
   if (k <= 64)
     return mode == kSolveShared
                ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, dw, trace)
+                                                      alpha, status, dw, trace)
                : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, dw, trace);
+                                                    alpha, status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
   static KernelSetup setup;
   const int d = setup_device();
@@ -857,7 +863,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
   return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, static_cast<int>(T), k, lambda,
-                            status, dw) == cudaSuccess
+                            alpha, status, dw) == cudaSuccess
              ? 0
              : -1;
 }
@@ -912,15 +918,15 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              0, 1, 0, s))
       return -1;
   }
-  // Y = Z U^T
+  // Y = Z U^T (+ b)
   if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out, 1, 0,
-           1, 0, s))
+           1, 0, s, 1.f, a.bias))
     return -1;
   if (k > 0) {
-    // Y_b += L_b C_b
+    // Y_b += alpha L_b C_b
     if (gemm(Tr, a.d_out, k, a.ZL + a.r, rk, 1, static_cast<int64_t>(Tr) * rk, a.Cm, a.d_out, 1,
              static_cast<int64_t>(k) * a.d_out, a.Y, a.d_out, 1, static_cast<int64_t>(Tr) * a.d_out,
-             Bn, 1, s))
+             Bn, 1, s, a.alpha))
       return -1;
   }
   return 0;

@@ -56,12 +56,16 @@ __device__ __forceinline__ int ceil_div_dev(int a, int b) { return (a + b - 1) /
 // col0 .. col0+63 of this thread's row) as bf16 through a 128-byte-swizzled
 // shared-memory box and a TMA store at (x, y) of `tmap`. Two boxes rotate: a
 // box is rewritten only after the store issued two boxes earlier has read it.
-// All 128 epilogue threads call it; thread 0 issues the stores.
+// All 128 epilogue threads call it; thread 0 issues the stores. With `bias`
+// (ncols entries, ncols a multiple of 8) bias[x + j] is added to column j of
+// the box in fp32 before the rounding; columns at or beyond ncols read none.
 constexpr uint32_t kStoreBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kStoreBoxes = 2;
 
 __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const void* tmap, int x,
-                                               int y, EpiCtx& e) {
+                                               int y, EpiCtx& e,
+                                               const __nv_bfloat16* bias = nullptr,
+                                               int ncols = 0) {
   const uint32_t buf = e.counter % kStoreBoxes;
   ++e.counter;
   // both TMEM loads in flight before one wait, and during the wait for the
@@ -73,6 +77,25 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
   named_bar_sync(1, 128);
   uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
   tmem_ld_wait();
+  if (bias != nullptr) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
+        const uint4 bq = c < ncols ? __ldg(reinterpret_cast<const uint4*>(bias + c))
+                                   : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t& v0 = vv[half][8 * ch + 2 * j];
+          uint32_t& v1 = vv[half][8 * ch + 2 * j + 1];
+          v0 = __float_as_uint(f32(v0) + __uint_as_float(w[j] << 16));
+          v1 = __float_as_uint(f32(v1) + __uint_as_float(w[j] & 0xffff0000u));
+        }
+      }
+    }
+  }
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -522,6 +545,8 @@ struct OutPolicy {
     CUtensorMap tmC;  // (B*k, d_out),  box (64, bn)
     CUtensorMap tmY;  // (d_out, N),    box (64, 128), store
     int N, r, k, T, B, bn, n_tiles_n, nkz, nkl;
+    const __nv_bfloat16* bias;  // d_out, added in the epilogue, or nullptr
+    int d_out;
   };
   struct Tile {
     int m0, n0, b_lo, nseg;
@@ -580,7 +605,7 @@ struct OutPolicy {
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
     for (int bx = 0; bx < p.bn / 64; ++bx)
-      store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e);
+      store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias, p.d_out);
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
@@ -1130,8 +1155,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
                  ? 1
                  : 0;
     if (!records) mode = 0;
-    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.status, s,
-                      pdl, /*defer_wait=*/true,
+    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.alpha,
+                      a.status, s, pdl, /*defer_wait=*/true,
                       a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
   } else {
@@ -1153,6 +1178,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     p.n_tiles_n = ceil_div(a.d_out, p.bn);
     p.nkz = ceil_div(a.r, 64);
     p.nkl = k > 0 ? ceil_div(k, 64) : 0;
+    p.bias = static_cast<const __nv_bfloat16*>(a.bias);
+    p.d_out = a.d_out;
 
     uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
     uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};

@@ -36,6 +36,7 @@ _vp, _i, _i64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_floa
 SIGNATURES = {
     "dyra_plan_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
+    "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -123,6 +124,11 @@ def dyra_plan_create(d_in: int, d_out: int, r: int, k: int, dtype: int) -> int:
 def dyra_load_factors(plan: int, U, V, P, W_res, lam: float, stream=None) -> None:
     _check(lib().dyra_load_factors(plan, _ptr(U), _ptr(V), _ptr(P), _ptr(W_res), float(lam),
                                    _stream(stream)), "dyra_load_factors")
+
+
+def dyra_set_linear(plan: int, bias, alpha: float = 1.0, stream=None) -> None:
+    _check(lib().dyra_set_linear(plan, _ptr(bias), float(alpha), _stream(stream)),
+           "dyra_set_linear")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -226,6 +232,14 @@ class DyraLinear:
         U, V, P, W_res = (self._dev(t) for t in (U, V, P, W_res))
         dyra_load_factors(self.plan, U, V, P if self.k else None, W_res if self.k else None,
                           lam, stream)
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+
+    def set_linear(self, bias=None, alpha: float = 1.0, stream=None) -> None:
+        """Bias (d_out values, or None) and correction weight of the full
+        linear layer, Y = static + bias + alpha * correction."""
+        import torch
+        b = self._dev(bias)
+        dyra_set_linear(self.plan, b, alpha, stream)
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
 
     def _check_x(self, X):

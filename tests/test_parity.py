@@ -180,6 +180,54 @@ def test_gaussian_start(case):
     assert oracle.rel_fro(Ya, Yo) < TOL[dtype] / 10
 
 
+LINEAR = [
+    # name, d_in, d_out, r, k, B, T, dtype, alpha, pairs
+    ("linear_pairs", 256, 512, 64, 32, 3, 201, "bf16", 0.5, True),
+    ("linear_alpha1", 256, 512, 64, 32, 3, 201, "bf16", 1.0, True),
+    ("linear_alpha0", 256, 512, 64, 32, 3, 201, "bf16", 0.0, True),
+    ("linear_single_cta", 256, 512, 64, 32, 3, 201, "bf16", 0.5, False),
+    ("linear_odd_d_out", 200, 328, 40, 8, 5, 37, "bf16", 1.5, True),   # last box past d_out
+    ("linear_k72", 256, 512, 64, 72, 2, 300, "bf16", 0.5, True),        # the general solve
+    ("linear_weight_only", 256, 512, 64, 0, 3, 201, "bf16", 1.0, True),
+    ("linear_f32", 96, 80, 12, 8, 3, 50, "f32", 0.5, True),
+]
+
+
+@pytest.mark.parametrize("case", LINEAR, ids=[c[0] for c in LINEAR])
+def test_bias_and_alpha(case):
+    """The full linear layer (DyRA Sec. 2.4): Y = static + b + alpha * correction,
+    against the oracle with the same bias (rounded to the storage type) and alpha."""
+    name, d_in, d_out, r, k, B, T, dtype, alpha, pairs = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, "lognormal", seed=3)
+    f = prepared(s)
+    bias = oracle.round_to(np.random.default_rng(5).standard_normal(d_out) * 0.3, dtype)
+    if not pairs:
+        os.environ["DYRA_PAIR"] = "0"
+    try:
+        layer = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_PAIR", None)
+    X = to_dev(f["X"], dtype)
+    Y0 = layer.forward(X, B=B, T=T).double().cpu().numpy()  # captures a graph first
+    layer.set_linear(to_dev(bias, dtype), alpha)
+    Y = layer.forward(X, B=B, T=T)
+    assert layer.status() == 0
+    Yg = Y.double().cpu().numpy()
+    Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, B, T, bias=bias,
+                          alpha=alpha)
+    err = oracle.rel_fro(Yg, Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    # the weight-only entry adds the bias too
+    Yw = layer.forward_weight_only(X).double().cpu().numpy()
+    Ywo = (f["X"] @ f["V"]) @ f["U"].T + bias
+    assert oracle.rel_fro(Yw, Ywo) <= TOL[dtype]
+    # removing the bias and restoring alpha gives the plain layer back
+    layer.set_linear(None, 1.0)
+    Y1 = layer.forward(X, B=B, T=T).double().cpu().numpy()
+    np.testing.assert_array_equal(Y1, Y0)
+    layer.close()
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
