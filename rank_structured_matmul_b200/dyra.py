@@ -36,6 +36,7 @@ _vp, _i, _i64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_floa
 SIGNATURES = {
     "dyra_plan_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
+    "dyra_set_als_steps": (_i, [_vp, _i]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -123,6 +124,10 @@ def dyra_plan_create(d_in: int, d_out: int, r: int, k: int, dtype: int) -> int:
 def dyra_load_factors(plan: int, U, V, P, W_res, lam: float, stream=None) -> None:
     _check(lib().dyra_load_factors(plan, _ptr(U), _ptr(V), _ptr(P), _ptr(W_res), float(lam),
                                    _stream(stream)), "dyra_load_factors")
+
+
+def dyra_set_als_steps(plan: int, half_steps: int) -> None:
+    _check(lib().dyra_set_als_steps(plan, int(half_steps)), "dyra_set_als_steps")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -227,6 +232,13 @@ class DyraLinear:
         dyra_load_factors(self.plan, U, V, P if self.k else None, W_res if self.k else None,
                           lam, stream)
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+
+    def set_als_iterations(self, t: float) -> None:
+        """t ALS iterations per forward (t = 1, 1.5, 2, ...; DyRA Sec. 3.3)."""
+        steps = int(round(2 * t))
+        if steps != 2 * t:
+            raise ValueError("t must be a multiple of 0.5")
+        dyra_set_als_steps(self.plan, steps)
 
     def _check_x(self, X):
         import torch
