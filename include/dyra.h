@@ -113,6 +113,22 @@ int dyra_load_factors(dyra_plan_t p, const void *U, const void *V, const void *P
 int dyra_set_linear(dyra_plan_t p, const void *bias, float alpha, dyra_stream_t stream);
 
 /*
+ * Number of alternating least-squares updates per forward ([DyRA] Sec. 2.2,
+ * Eq. 4-5; Sec. 3.3 compares 1, 1.5 and 2 iterations). Updates alternate L and
+ * R from Alg. 1's first pair: half_steps = 2 is Alg. 1 (t = 1), 3 adds an L
+ * update (t = 1.5: the output uses the newest L with the previous R), 4 an R
+ * update (t = 2), and so on. Each L update after the first computes
+ * L_b = X_b (R_b W_res)^T (R_b R_b^T + lambda I)^-1, so it costs one more pass
+ * over X. Default 2.
+ *   half_steps : 2 .. 64, else DYRA_ERR_INVALID_ARG.
+ * Only the CUDA-core kernels (fp32 plans, or bf16 plans under
+ * DYRA_KERNELS=simt) run more than two; the tensor-core kernels return
+ * DYRA_ERR_UNSUPPORTED, as does dyra_forward_batched_noalloc, for any other
+ * count. Takes effect at the next forward.
+ */
+int dyra_set_als_steps(dyra_plan_t p, int half_steps);
+
+/*
  * Y = DyRA(X) for one instance of N rows (B = 1, T = N).
  *   X : N x d_in input, Y : N x d_out output (overwritten), N >= 0.
  * N == 0 is a no-op. Returns DYRA_ERR_RANK_DEFICIENT if lambda == 0 and N < k.

@@ -47,6 +47,13 @@ struct dyra_plan {
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
+  // ALS updates per forward (dyra_set_als_steps; CUDA-core plans beyond 2) and
+  // the buffers the further L updates use
+  int als_half_steps = 2;
+  void* Lt = nullptr;    // (B*k) x T
+  void* P2 = nullptr;    // (B*k) x d_in
+  float* TG2 = nullptr;  // B x k x (T + k)
+  size_t cap_Lt = 0, cap_P2 = 0, cap_TG2 = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -151,13 +158,16 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 // Grows the workspace; captured graphs point at the old buffers, so any
 // growth drops them.
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
-  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  const void* ptrs[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
+  auto caps = [p] {
+    return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Lt +
+           p->cap_P2 + p->cap_TG2;
+  };
+  const size_t before = caps();
+  const void* ptrs[9] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Lt, p->P2, p->TG2};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
-  bool moved =
-      before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  for (int i = 0; i < 6; ++i) moved = moved || ptrs[i] != now[i];
+  const void* now[9] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Lt, p->P2, p->TG2};
+  bool moved = before != caps();
+  for (int i = 0; i < 9; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -188,6 +198,14 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if (rc) return rc;
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
+      if (p->als_half_steps > 2) {
+        if ((rc = grow(p->Lt, p->cap_Lt, static_cast<size_t>(B) * k * T * es))) return rc;
+        if ((rc = grow(p->P2, p->cap_P2, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
+        void* tg2 = p->TG2;
+        rc = grow(tg2, p->cap_TG2, static_cast<size_t>(B) * k * (T + k) * sizeof(float));
+        p->TG2 = static_cast<float*>(tg2);
+        if (rc) return rc;
+      }
     }
   }
   return DYRA_OK;
@@ -329,6 +347,10 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.status = p->status;
     a.bias = p->has_bias ? static_cast<const __nv_bfloat16*>(p->bias) : nullptr;
     a.alpha = p->alpha;
+    a.half_steps = p->als_half_steps;
+    a.Lt = static_cast<__nv_bfloat16*>(p->Lt);
+    a.P2 = static_cast<__nv_bfloat16*>(p->P2);
+    a.TG2 = p->TG2;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   } else {
@@ -353,6 +375,10 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.status = p->status;
     a.bias = p->has_bias ? static_cast<const float*>(p->bias) : nullptr;
     a.alpha = p->alpha;
+    a.half_steps = p->als_half_steps;
+    a.Lt = static_cast<float*>(p->Lt);
+    a.P2 = static_cast<float*>(p->P2);
+    a.TG2 = p->TG2;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   }
@@ -545,6 +571,15 @@ int dyra_set_linear(dyra_plan_t p, const void* bias, float alpha, dyra_stream_t 
   return DYRA_OK;
 }
 
+int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
+  if (p == nullptr || half_steps < 2 || half_steps > 64) return DYRA_ERR_INVALID_ARG;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
+  if (umma && half_steps != 2) return DYRA_ERR_UNSUPPORTED;
+  p->als_half_steps = half_steps;
+  drop_graphs(p);  // captured forwards hold the old count
+  return DYRA_OK;
+}
+
 int dyra_forward(dyra_plan_t p, const void* X, void* Y, int64_t N, dyra_stream_t stream) {
   return run_forward(p, X, Y, 1, N, false, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -595,6 +630,10 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->Tp);
     dev_free(p->Ct);
     dev_free(p->MD);
+    dev_free(p->Lt);
+    dev_free(p->P2);
+    void* tg2 = p->TG2;
+    dev_free(tg2);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -711,7 +750,8 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         256 + (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
+         p->cap_Lt + p->cap_P2 + p->cap_TG2 + 256 +
+         (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
 }  // extern "C"
@@ -774,6 +814,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
   if (!aligned16(X) || !aligned16(Y)) return DYRA_ERR_ALIGNMENT;
   const int k = p->k;
   if (k > 0 && p->lambda == 0.f && T < k) return DYRA_ERR_RANK_DEFICIENT;
+  if (k > 0 && p->als_half_steps != 2) return DYRA_ERR_UNSUPPORTED;
 
   const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
   const size_t es = elem_size(p->dtype);

@@ -119,6 +119,13 @@ struct SimtForward {
   int* status;
   const T* bias = nullptr;  // d_out values added to Y, or nullptr
   float alpha = 1.f;        // weight of the correction
+  // More alternating least-squares updates ([DyRA] Sec. 3.3): half_steps
+  // updates in all, L and R alternating, Alg. 1 being the first two. Beyond
+  // two, each L update needs the buffers below.
+  int half_steps = 2;
+  T* Lt = nullptr;       // (B*k) x Trows: the latest L_b, transposed
+  T* P2 = nullptr;       // (B*k) x d_in: R_b W_res, the L update's projector before its solve
+  float* TG2 = nullptr;  // B x k x (Trows + k): [ (X_b P2_b^T)^T | R_b R_b^T ]
 };
 
 template <typename T>

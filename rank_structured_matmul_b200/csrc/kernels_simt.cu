@@ -887,7 +887,14 @@ template int launch_pack_vp<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bflo
                                            __nv_bfloat16*, int, int, int, cudaStream_t);
 
 // The fp32 forward: the same steps as the tensor-core path, each as a
-// strided batched SIMT GEMM, with fp32 storage of every intermediate.
+// strided batched SIMT GEMM, with fp32 storage of every intermediate. With
+// more than two half-steps, further L and R updates follow Alg. 1's pair
+// ([DyRA] Sec. 2.2, Eq. 4-5 with the ridge of footnote 2; Sec. 3.3):
+//   L update  L_b = X_b (R_b W_res)^T (R_b R_b^T + lambda I)^-1
+//   R update  R_b = (L_b^T L_b + lambda I)^-1 (L_b^T X_b) W_res^T
+// and the output takes the last pair. Both updates go through the same ridge
+// solve: the R update solves for R_b from [L_b^T X_b | L_b^T L_b], the L
+// update for L_b^T from [(X_b (R_b W_res)^T)^T | R_b R_b^T].
 template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t s) {
   const int64_t N = a.B * a.Trows;
@@ -896,37 +903,65 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
   const int k = a.weight_only ? 0 : a.k;
   const int Bn = static_cast<int>(a.B);
   const int Tr = static_cast<int>(a.Trows);
+  const int steps = k > 0 ? a.half_steps : 0;
+  if (k > 0 && (steps < 2 || (steps > 2 && (!a.Lt || !a.P2 || !a.TG2)))) return -1;
   // [Z | L] = X [V | P]
   if (gemm(static_cast<int>(N), rk, a.d_in, a.X, a.d_in, 1, 0, a.VPt, 1, a.d_in, 0, a.ZL, rk, 1,
            0, 1, 0, s))
     return -1;
-  if (k > 0) {
-    const int J = a.d_in + k;
-    // T_b = L_b^T X_b  -> TG[b][i][j], j < d_in
-    if (gemm(k, a.d_in, Tr, a.ZL + a.r, 1, rk, static_cast<int64_t>(Tr) * rk, a.X, a.d_in, 1,
-             static_cast<int64_t>(Tr) * a.d_in, a.TG, J, 1, static_cast<int64_t>(k) * J, Bn, 0, s))
-      return -1;
-    // G_b = L_b^T L_b -> TG[b][i][d_in + i']
-    if (gemm(k, k, Tr, a.ZL + a.r, 1, rk, static_cast<int64_t>(Tr) * rk, a.ZL + a.r, rk, 1,
-             static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
-             s))
-      return -1;
-    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
-      return -1;
-    // C = T' W_res^T  (B*k x d_out)
-    if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,
-             0, 1, 0, s))
-      return -1;
+  // the current L_b: element (t, i) at Lp[b * lb + t * lm + i * lq]
+  const T* Lp = a.ZL + a.r;
+  int64_t lm = rk, lq = 1, lb = static_cast<int64_t>(Tr) * rk;
+  for (int h = 1; h < steps; ++h) {
+    if (h % 2 == 1) {  // R update from the current L
+      const int J = a.d_in + k;
+      // T_b = L_b^T X_b  -> TG[b][i][j], j < d_in
+      if (gemm(k, a.d_in, Tr, Lp, lq, lm, lb, a.X, a.d_in, 1, static_cast<int64_t>(Tr) * a.d_in,
+               a.TG, J, 1, static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      // G_b = L_b^T L_b -> TG[b][i][d_in + i']
+      if (gemm(k, k, Tr, Lp, lq, lm, lb, Lp, lm, lq, lb, a.TG + a.d_in, J, 1,
+               static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+        return -1;
+      // R = T' W_res^T  (B*k x d_out)
+      if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out,
+               1, 0, 1, 0, s))
+        return -1;
+    } else {  // L update from the current R (in Cm)
+      const int J = Tr + k;
+      // P2 = R W_res  (B*k x d_in)
+      if (gemm(Bn * k, a.d_in, a.d_out, a.Cm, a.d_out, 1, 0, a.W_res, a.d_in, 1, 0, a.P2, a.d_in,
+               1, 0, 1, 0, s))
+        return -1;
+      // (X_b P2_b^T)^T -> TG2[b][i][t], t < Tr
+      if (gemm(k, Tr, a.d_in, a.P2, a.d_in, 1, static_cast<int64_t>(k) * a.d_in, a.X, 1, a.d_in,
+               static_cast<int64_t>(Tr) * a.d_in, a.TG2, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
+               s))
+        return -1;
+      // R_b R_b^T -> TG2[b][i][Tr + i']
+      if (gemm(k, k, a.d_out, a.Cm, a.d_out, 1, static_cast<int64_t>(k) * a.d_out, a.Cm, 1,
+               a.d_out, static_cast<int64_t>(k) * a.d_out, a.TG2 + Tr, J, 1,
+               static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      // L_b^T = (R_b R_b^T + lambda I)^-1 (X_b P2_b^T)^T  -> Lt[b*k + i][t]
+      if (launch_solve<T>(a.TG2, 1, a.B, k, Tr, a.lambda, a.Lt, a.status, s, false, nullptr))
+        return -1;
+      Lp = a.Lt;
+      lm = 1;
+      lq = Tr;
+      lb = static_cast<int64_t>(k) * Tr;
+    }
   }
   // Y = Z U^T (+ b)
   if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out, 1, 0,
            1, 0, s, 1.f, a.bias))
     return -1;
   if (k > 0) {
-    // Y_b += alpha L_b C_b
-    if (gemm(Tr, a.d_out, k, a.ZL + a.r, rk, 1, static_cast<int64_t>(Tr) * rk, a.Cm, a.d_out, 1,
-             static_cast<int64_t>(k) * a.d_out, a.Y, a.d_out, 1, static_cast<int64_t>(Tr) * a.d_out,
-             Bn, 1, s, a.alpha))
+    // Y_b += alpha L_b R_b (the last pair)
+    if (gemm(Tr, a.d_out, k, Lp, lm, lq, lb, a.Cm, a.d_out, 1, static_cast<int64_t>(k) * a.d_out,
+             a.Y, a.d_out, 1, static_cast<int64_t>(Tr) * a.d_out, Bn, 1, s, a.alpha))
       return -1;
   }
   return 0;

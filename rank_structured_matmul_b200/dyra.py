@@ -37,6 +37,7 @@ SIGNATURES = {
     "dyra_plan_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
+    "dyra_set_als_steps": (_i, [_vp, _i]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -129,6 +130,10 @@ def dyra_load_factors(plan: int, U, V, P, W_res, lam: float, stream=None) -> Non
 def dyra_set_linear(plan: int, bias, alpha: float = 1.0, stream=None) -> None:
     _check(lib().dyra_set_linear(plan, _ptr(bias), float(alpha), _stream(stream)),
            "dyra_set_linear")
+
+
+def dyra_set_als_steps(plan: int, half_steps: int) -> None:
+    _check(lib().dyra_set_als_steps(plan, int(half_steps)), "dyra_set_als_steps")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -241,6 +246,13 @@ class DyraLinear:
         b = self._dev(bias)
         dyra_set_linear(self.plan, b, alpha, stream)
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+
+    def set_als_iterations(self, t: float) -> None:
+        """t ALS iterations per forward (t = 1, 1.5, 2, ...; DyRA Sec. 3.3)."""
+        steps = int(round(2 * t))
+        if steps != 2 * t:
+            raise ValueError("t must be a multiple of 0.5")
+        dyra_set_als_steps(self.plan, steps)
 
     def _check_x(self, X):
         import torch

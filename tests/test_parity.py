@@ -228,6 +228,49 @@ def test_bias_and_alpha(case):
     layer.close()
 
 
+ALS = [
+    # name, d_in, d_out, r, k, B, T, dtype, t
+    ("als_f32_t1.5", 96, 80, 12, 8, 3, 50, "f32", 1.5),
+    ("als_f32_t2", 96, 80, 12, 8, 3, 50, "f32", 2.0),
+    ("als_f32_t3_k40", 128, 96, 16, 40, 2, 60, "f32", 3.0),
+    ("als_bf16_simt_t2", 256, 512, 64, 32, 3, 201, "bf16", 2.0),
+]
+
+
+@pytest.mark.parametrize("case", ALS, ids=[c[0] for c in ALS])
+def test_als_iterations(case):
+    """t alternating least-squares iterations (DyRA Sec. 2.2, Sec. 3.3) on the
+    CUDA-core kernels, against the oracle's ALS from the same start; t = 1
+    again afterwards gives the one-step layer."""
+    name, d_in, d_out, r, k, B, T, dtype, t = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, "outlier", n_outlier=4,
+                  outlier_scale=10.0, seed=2)
+    w = generate(s)
+    fo = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, r, k, s.lam)
+    f = {n: oracle.round_to(a, dtype) for n, a in
+         (("X", w.X), ("U", fo.U), ("V", fo.V), ("P", fo.P), ("W_res", fo.W_res))}
+    layer = make_layer(s, f, kernels="simt")
+    X = to_dev(f["X"], dtype)
+    layer.set_als_iterations(t)
+    Y = layer.forward(X, B=B, T=T)
+    assert layer.status() == 0
+    Yo = oracle.als_inference(f["X"], f["U"], f["V"], f["W_res"], fo.R0, s.lam, B, T, t)
+    err = oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    layer.set_als_iterations(1)
+    check(s, layer.forward(X, B=B, T=T), f, full=True)
+    layer.close()
+
+
+def test_als_iterations_need_the_cuda_core_kernels():
+    s, f = _small()
+    layer = make_layer(s, f)
+    layer.set_als_iterations(1)
+    with pytest.raises(dyra.DyraError):
+        layer.set_als_iterations(2)
+    layer.close()
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
