@@ -129,6 +129,21 @@ int dyra_set_linear(dyra_plan_t p, const void *bias, float alpha, dyra_stream_t 
 int dyra_set_als_steps(dyra_plan_t p, int half_steps);
 
 /*
+ * dyra_forward_batched on HOST buffers: X (B*T x d_in) and Y (B*T x d_out) in
+ * host memory, ideally page-locked (cudaHostAlloc), since pageable memory
+ * makes the copies synchronous. Whole instances move in chunks of at least
+ * about 1 MiB of X, at most 16 chunks. On three streams the copy of chunk
+ * c + 1 to the device, the forward of chunk c (on `stream`) and the copy of
+ * chunk c - 1 back overlap; an instance's result does not depend on the
+ * chunking. The call is asynchronous like cudaMemcpyAsync: work enqueued on
+ * `stream` afterwards, and a synchronisation of `stream`, see Y complete. The
+ * plan owns the device chunk buffers (grown on demand) and the copy streams.
+ * Errors as dyra_forward_batched; X and Y must not overlap.
+ */
+int dyra_forward_batched_host(dyra_plan_t p, const void *X, void *Y, int64_t B, int64_t T,
+                              dyra_stream_t stream);
+
+/*
  * Y = DyRA(X) for one instance of N rows (B = 1, T = N).
  *   X : N x d_in input, Y : N x d_out output (overwritten), N >= 0.
  * N == 0 is a no-op. Returns DYRA_ERR_RANK_DEFICIENT if lambda == 0 and N < k.

@@ -75,6 +75,15 @@ struct dyra_plan {
   uint64_t graph_clock = 0;
   cudaStream_t capture_stream = nullptr;
   bool use_graphs = true;
+  // dyra_forward_batched_host: two device buffers each for the input and the
+  // output chunks, the copy streams and the per-chunk events
+  static constexpr int kHostEvents = 16;
+  void* hx[2] = {nullptr, nullptr};
+  void* hy[2] = {nullptr, nullptr};
+  size_t cap_hx[2] = {0, 0}, cap_hy[2] = {0, 0};
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_start = nullptr;
+  cudaEvent_t ev_in[kHostEvents] = {}, ev_comp[kHostEvents] = {}, ev_out[kHostEvents] = {};
 };
 
 namespace {
@@ -580,6 +589,76 @@ int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
   return DYRA_OK;
 }
 
+int dyra_forward_batched_host(dyra_plan_t p, const void* X, void* Y, int64_t B, int64_t T,
+                              dyra_stream_t stream) {
+  if (p == nullptr || B < 0 || T < 0) return DYRA_ERR_INVALID_ARG;
+  if (B * T == 0) return DYRA_OK;
+  if (X == nullptr || Y == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(p->dtype);
+  // Chunks of whole instances (each instance's correction needs all of its
+  // rows): up to kHostEvents of them, at least about 1 MiB of input each.
+  const size_t inst_in = static_cast<size_t>(T) * p->d_in * es;
+  const size_t inst_out = static_cast<size_t>(T) * p->d_out * es;
+  int64_t per = std::max<int64_t>(1, (B + dyra_plan::kHostEvents - 1) / dyra_plan::kHostEvents);
+  per = std::max<int64_t>(per, std::min<int64_t>(B, static_cast<int64_t>((1u << 20) / inst_in) + 1));
+  const int64_t chunks = (B + per - 1) / per;
+  int rc;
+  for (int i = 0; i < 2; ++i) {
+    if ((rc = grow(p->hx[i], p->cap_hx[i], per * inst_in))) return rc;
+    if ((rc = grow(p->hy[i], p->cap_hy[i], per * inst_out))) return rc;
+  }
+  auto make_stream = [](cudaStream_t* st) {
+    return *st || cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) == cudaSuccess;
+  };
+  auto make_event = [](cudaEvent_t* e) {
+    return *e || cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  };
+  bool ok = make_stream(&p->h2d) && make_stream(&p->d2h) && make_event(&p->ev_start);
+  for (int i = 0; ok && i < dyra_plan::kHostEvents; ++i)
+    ok = make_event(&p->ev_in[i]) && make_event(&p->ev_comp[i]) && make_event(&p->ev_out[i]);
+  if (!ok) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  // chunk c: X -> hx[c % 2] on h2d, the forward on `stream`, hy[c % 2] -> Y on d2h.
+  // hx[c % 2] is rewritten once the forward of chunk c - 2 has read it, hy[c % 2]
+  // once the copy of chunk c - 2 has read it; `stream` then waits for the last copy.
+  const char* xs = static_cast<const char*>(X);
+  char* ys = static_cast<char*>(Y);
+  bool err = cudaEventRecord(p->ev_start, s) != cudaSuccess ||
+             cudaStreamWaitEvent(p->h2d, p->ev_start, 0) != cudaSuccess;
+  for (int64_t c = 0; !err && c < chunks; ++c) {
+    const int64_t b0 = c * per, bc = std::min<int64_t>(per, B - b0);
+    const int buf = static_cast<int>(c % 2);
+    const int e = static_cast<int>(c % dyra_plan::kHostEvents);
+    const int e2 = static_cast<int>((c + dyra_plan::kHostEvents - 2) % dyra_plan::kHostEvents);
+    if (c >= 2) err = cudaStreamWaitEvent(p->h2d, p->ev_comp[e2], 0) != cudaSuccess;
+    err = err || cudaMemcpyAsync(p->hx[buf], xs + b0 * inst_in, bc * inst_in,
+                                 cudaMemcpyHostToDevice, p->h2d) != cudaSuccess;
+    err = err || cudaEventRecord(p->ev_in[e], p->h2d) != cudaSuccess;
+    err = err || cudaStreamWaitEvent(s, p->ev_in[e], 0) != cudaSuccess;
+    if (c >= 2) err = err || cudaStreamWaitEvent(s, p->ev_out[e2], 0) != cudaSuccess;
+    if (err) break;
+    rc = run_forward(p, p->hx[buf], p->hy[buf], bc, T, false, s);
+    if (rc) return rc;
+    err = cudaEventRecord(p->ev_comp[e], s) != cudaSuccess ||
+          cudaStreamWaitEvent(p->d2h, p->ev_comp[e], 0) != cudaSuccess ||
+          cudaMemcpyAsync(ys + b0 * inst_out, p->hy[buf], bc * inst_out, cudaMemcpyDeviceToHost,
+                          p->d2h) != cudaSuccess ||
+          cudaEventRecord(p->ev_out[e], p->d2h) != cudaSuccess;
+    if (!err && c == chunks - 1) err = cudaStreamWaitEvent(s, p->ev_out[e], 0) != cudaSuccess;
+  }
+  if (err) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  return DYRA_OK;
+}
+
 int dyra_forward(dyra_plan_t p, const void* X, void* Y, int64_t N, dyra_stream_t stream) {
   return run_forward(p, X, Y, 1, N, false, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -641,6 +720,18 @@ int dyra_plan_destroy(dyra_plan_t p) {
     if (p->trace) cudaFree(p->trace);
     drop_graphs(p);
     if (p->capture_stream) cudaStreamDestroy(p->capture_stream);
+    for (int i = 0; i < 2; ++i) {
+      dev_free(p->hx[i]);
+      dev_free(p->hy[i]);
+    }
+    if (p->h2d) cudaStreamDestroy(p->h2d);
+    if (p->d2h) cudaStreamDestroy(p->d2h);
+    if (p->ev_start) cudaEventDestroy(p->ev_start);
+    for (int i = 0; i < dyra_plan::kHostEvents; ++i) {
+      if (p->ev_in[i]) cudaEventDestroy(p->ev_in[i]);
+      if (p->ev_comp[i]) cudaEventDestroy(p->ev_comp[i]);
+      if (p->ev_out[i]) cudaEventDestroy(p->ev_out[i]);
+    }
   }
   delete p;
   return DYRA_OK;

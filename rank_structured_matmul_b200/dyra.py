@@ -38,6 +38,7 @@ SIGNATURES = {
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
     "dyra_set_als_steps": (_i, [_vp, _i]),
+    "dyra_forward_batched_host": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -134,6 +135,12 @@ def dyra_set_linear(plan: int, bias, alpha: float = 1.0, stream=None) -> None:
 
 def dyra_set_als_steps(plan: int, half_steps: int) -> None:
     _check(lib().dyra_set_als_steps(plan, int(half_steps)), "dyra_set_als_steps")
+
+
+def dyra_forward_batched_host(plan: int, X, Y, B: int, T: int, stream=None) -> None:
+    """dyra_forward_batched on host buffers (X, Y page-locked CPU tensors or addresses)."""
+    _check(lib().dyra_forward_batched_host(plan, _ptr(X), _ptr(Y), int(B), int(T),
+                                           _stream(stream)), "dyra_forward_batched_host")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -272,6 +279,25 @@ class DyraLinear:
         if Y is None:
             Y = torch.empty((N, self.d_out), device=X.device, dtype=self.torch_dtype)
         dyra_forward_batched(self.plan, X, Y, B, T, stream)
+        return Y
+
+    def forward_host(self, X, B: int = 1, T: Optional[int] = None, Y=None, stream=None):
+        """forward() on host tensors: copies in, the layer and copies out overlap
+        by chunks of instances. X and Y should be pinned CPU tensors; the call is
+        asynchronous on the stream (synchronise it before reading Y)."""
+        import torch
+        if X.is_cuda or X.dtype != self.torch_dtype or not X.is_contiguous() or X.dim() != 2 \
+                or X.shape[1] != self.d_in:
+            raise ValueError("X must be a contiguous CPU %s tensor of shape (N, %d)"
+                             % (self.torch_dtype, self.d_in))
+        N = X.shape[0]
+        if T is None:
+            T = N // B
+        if B * T != N:
+            raise ValueError("B*T must equal the row count of X")
+        if Y is None:
+            Y = torch.empty((N, self.d_out), dtype=self.torch_dtype).pin_memory()
+        dyra_forward_batched_host(self.plan, X, Y, B, T, stream)
         return Y
 
     def forward_weight_only(self, X, Y=None, stream=None):

@@ -271,6 +271,26 @@ def test_als_iterations_need_the_cuda_core_kernels():
     layer.close()
 
 
+@pytest.mark.parametrize("B,T", [(32, 201), (3, 201), (1, 600)])
+def test_host_forward_matches_device_forward(B, T):
+    """dyra_forward_batched_host (host buffers, copies overlapped by chunks of
+    instances) meets the oracle like the device-buffer forward. The chunks are
+    forwards of fewer instances, whose Gram reduction may split rows
+    differently, so the two agree to rounding, not bit for bit."""
+    s = LayerSpec("host", 256, 512, 64, 32, B, T, "bf16", 0.7, "lognormal", seed=4)
+    f = prepared(s)
+    layer = make_layer(s, f)
+    Xd = to_dev(f["X"], "bf16")
+    Yd = layer.forward(Xd, B=B, T=T).cpu()
+    Xh = Xd.cpu().pin_memory()
+    Yh = layer.forward_host(Xh, B=B, T=T)
+    torch.cuda.current_stream().synchronize()
+    assert layer.status() == 0
+    check(s, Yh, f, full=True)
+    assert oracle.rel_fro(Yh.double().numpy(), Yd.double().numpy()) <= TOL["bf16"] / 2
+    layer.close()
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
