@@ -119,6 +119,52 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
   }
 }
 
+// The second half of store_box_bf16 for a box whose accumulator values the
+// caller already holds (loaded and waited for): lets the caller load the next
+// box from TMEM while this one is converted and stored.
+__device__ __forceinline__ void store_loaded_box_bf16(const uint32_t (&vv)[2][32], const void* tmap,
+                                                      int x, int y, EpiCtx& e,
+                                                      const __nv_bfloat16* bias = nullptr,
+                                                      int ncols = 0) {
+  const uint32_t buf = e.counter % kStoreBoxes;
+  ++e.counter;
+  if (e.tid == 0) tma_store_wait_read<kStoreBoxes - 1>();
+  named_bar_sync(1, 128);
+  uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      const int chunk = half * 4 + ch;
+      const uint32_t off =
+          static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+      float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
+      if (bias != nullptr && c < ncols) {
+        const uint4 bq = __ldg(reinterpret_cast<const uint4*>(bias + c));
+        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          b[2 * jj] = __uint_as_float(w[jj] << 16);
+          b[2 * jj + 1] = __uint_as_float(w[jj] & 0xffff0000u);
+        }
+      }
+      uint4 q;
+      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]) + b[0], f32(vv[half][8 * ch + 1]) + b[1]);
+      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]) + b[2], f32(vv[half][8 * ch + 3]) + b[3]);
+      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]) + b[4], f32(vv[half][8 * ch + 5]) + b[5]);
+      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]) + b[6], f32(vv[half][8 * ch + 7]) + b[7]);
+      *reinterpret_cast<uint4*>(sbuf + off) = q;
+    }
+  }
+  fence_async_shared();
+  named_bar_sync(1, 128);
+  if (e.tid == 0) {
+    tma_store_2d(tmap, e.smem_u32 + buf * kStoreBoxBytes, x, y);
+    tma_store_commit();
+  }
+}
+
 __device__ __forceinline__ void store_drain(EpiCtx& e) {
   if (e.tid == 0) tma_store_wait_all();
 }
@@ -604,8 +650,29 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    for (int bx = 0; bx < p.bn / 64; ++bx)
-      store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias, p.d_out);
+    // The next box's TMEM loads are in flight while this box is converted and
+    // stored (tcgen05.wait::ld waits for every earlier load of the thread, so
+    // each wait comes after the previous box is written out).
+    const int nb = p.bn / 64;
+    uint32_t va[2][32], vb[2][32];
+    tmem_ld_32x32b_x32(tacc, va[0]);
+    tmem_ld_32x32b_x32(tacc + 32, va[1]);
+    tmem_ld_wait();
+    for (int bx = 0; bx < nb; bx += 2) {
+      if (bx + 1 < nb) {
+        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64, vb[0]);
+        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64 + 32, vb[1]);
+      }
+      store_loaded_box_bf16(va, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias, p.d_out);
+      if (bx + 1 >= nb) break;
+      tmem_ld_wait();
+      if (bx + 2 < nb) {
+        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64, va[0]);
+        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64 + 32, va[1]);
+      }
+      store_loaded_box_bf16(vb, &p.tmY, t.n0 + (bx + 1) * 64, t.m0, e, p.bias, p.d_out);
+      tmem_ld_wait();
+    }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
