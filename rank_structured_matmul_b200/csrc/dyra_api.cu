@@ -30,6 +30,10 @@ struct dyra_plan {
   // publishes it (DYRA_FACTOR=shared), or by size (unset: every block while
   // the blocks fit the SMs).
   int factor_mode = -1;
+  // Compensated correction (low parts of L~ and Q^T, DYRA_HILO=1|0; unset:
+  // for single instances of up to 2048 rows, where the output stage is bound
+  // by reading U and the extra correction products cost nothing)
+  int hilo_mode = -1;
   float lambda = 0.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
@@ -42,7 +46,10 @@ struct dyra_plan {
   void* Tp = nullptr;    // (B*k) x d_in
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
+  void* Llo = nullptr;   // bf16, compensated correction: N x k
+  void* Ctlo = nullptr;  // bf16, compensated correction: d_out x (B*k)
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
+  size_t cap_Llo = 0, cap_Ctlo = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -130,6 +137,12 @@ struct DeviceGuard {
 
 int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
+// Whether a tensor-core forward of B x T rows uses the compensated correction.
+bool use_hilo(const dyra_plan* p, int64_t B, int64_t T) {
+  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->hilo_mode == 0) return false;
+  return p->hilo_mode == 1 || (B == 1 && T <= 2048);
+}
+
 // Factor records of the solve plus its per-instance flags (bf16, k <= 64).
 size_t factor_bytes(int64_t B, int k) {
   const int rec = dyra::factor_record_floats(k);
@@ -147,13 +160,16 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 // Grows the workspace; captured graphs point at the old buffers, so any
 // growth drops them.
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
-  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  const void* ptrs[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
+  auto caps = [p] {
+    return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Llo +
+           p->cap_Ctlo;
+  };
+  const size_t before = caps();
+  const void* ptrs[8] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Llo, p->Ctlo};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
-  bool moved =
-      before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  for (int i = 0; i < 6; ++i) moved = moved || ptrs[i] != now[i];
+  const void* now[8] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Llo, p->Ctlo};
+  bool moved = before != caps();
+  for (int i = 0; i < 8; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -174,6 +190,11 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
       if ((rc = grow(p->MD, p->cap_MD, factor_bytes(B, k)))) return rc;
+      if (use_hilo(p, B, T)) {
+        if ((rc = grow(p->Llo, p->cap_Llo, static_cast<size_t>(N) * k * es))) return rc;
+        if ((rc = grow(p->Ctlo, p->cap_Ctlo, static_cast<size_t>(B) * k * p->d_out * es)))
+          return rc;
+      }
     }
   } else {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * (p->r + k) * es))) return rc;
@@ -295,6 +316,9 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.trace = p->trace;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.hilo = correct && use_hilo(p, B, T);
+    a.Llo = a.hilo ? p->Llo : nullptr;
+    a.Ctlo = a.hilo ? p->Ctlo : nullptr;
     rc = launch_bf16_maybe_graph(p, a, s);
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
@@ -454,6 +478,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
                    : std::strcmp(fv, "self") == 0   ? 0
                    : std::strcmp(fv, "shared") == 0 ? 1
                                                     : -1;
+  const char* hv = std::getenv("DYRA_HILO");
+  p->hilo_mode = hv == nullptr ? -1 : (hv[0] == '1' ? 1 : (hv[0] == '0' ? 0 : -1));
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -557,6 +583,8 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->Tp);
     dev_free(p->Ct);
     dev_free(p->MD);
+    dev_free(p->Llo);
+    dev_free(p->Ctlo);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -673,7 +701,7 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         256;
+         p->cap_Llo + p->cap_Ctlo + 256;
 }
 
 }  // extern "C"
@@ -752,6 +780,10 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
       sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
       sizing.take(factor_bytes(B, k));
+      if (use_hilo(p, B, T)) {
+        sizing.take(static_cast<size_t>(N) * k * es);
+        sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+      }
     }
   } else {
     sizing.take(static_cast<size_t>(N) * (p->r + k) * es);
@@ -794,6 +826,9 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     void* fac = k > 0 ? carve.take(factor_bytes(B, k)) : nullptr;
     split_factor_buffer(fac, B, k, &a.MD, &a.counters);
+    a.hilo = k > 0 && use_hilo(p, B, T);
+    a.Llo = a.hilo ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
+    a.Ctlo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     a.factor_mode = p->factor_mode;
     a.splits = splits;
     a.split_rows = split_rows;

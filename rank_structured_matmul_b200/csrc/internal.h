@@ -52,6 +52,12 @@ struct Bf16Forward {
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
   bool use_pairs;             // run the output stage on CTA pairs
   int proj_pair_min_tiles;    // see proj_shape (0: default)
+  // Compensated correction: L~ and Q^T are also stored as their bf16 rounding
+  // errors (Llo, Ctlo) and the output stage adds hi.hi + hi.lo + lo.hi, which
+  // removes most of the cancellation error the grouping L~ . Q amplifies.
+  bool hilo = false;
+  void* Llo = nullptr;   // N x k
+  void* Ctlo = nullptr;  // d_out x (B*k)
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -115,9 +121,10 @@ int factor_record_floats(int k);
 // defer_wait (with pdl): the grid launched just before waited for the one
 // that wrote G and L before letting this one start; this grid then waits
 // for it only before its blocks exit.
-int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
-                  unsigned long long* trace);
+// Llo (optional, N x k like L): receives the bf16 rounding error of each L~ value.
+int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
+                  int64_t T, int k, float lambda, int* status, cudaStream_t s, bool pdl,
+                  bool defer_wait, unsigned long long* trace);
 // Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
 size_t ltilde_smem_bytes(int k);
 int ltilde_rows_per_block(int k);
