@@ -30,6 +30,10 @@ struct dyra_plan {
   // publishes it (DYRA_FACTOR=shared), or by size (unset: every block while
   // the blocks fit the SMs).
   int factor_mode = -1;
+  // Compensated correction (low parts of L~ and Q^T, DYRA_HILO=1|0; unset:
+  // for single instances of up to 2048 rows, where the output stage is bound
+  // by reading U and the extra correction products cost nothing)
+  int hilo_mode = -1;
   float lambda = 0.f;
   // full linear layer (dyra_set_linear): Y = static + bias + alpha * correction
   void* bias = nullptr;  // d_out values in the plan dtype (allocated on first use)
@@ -46,6 +50,8 @@ struct dyra_plan {
   void* Tp = nullptr;    // (B*k) x d_in
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
+  void* Llo = nullptr;   // bf16, compensated correction: N x k
+  void* Ctlo = nullptr;  // bf16, compensated correction: d_out x (B*k)
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
   // ALS updates per forward (dyra_set_als_steps; CUDA-core plans beyond 2) and
   // the buffers the further L updates use
@@ -54,6 +60,7 @@ struct dyra_plan {
   void* P2 = nullptr;    // (B*k) x d_in
   float* TG2 = nullptr;  // B x k x (T + k)
   size_t cap_Lt = 0, cap_P2 = 0, cap_TG2 = 0;
+  size_t cap_Llo = 0, cap_Ctlo = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -150,6 +157,12 @@ struct DeviceGuard {
 
 int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
+// Whether a tensor-core forward of B x T rows uses the compensated correction.
+bool use_hilo(const dyra_plan* p, int64_t B, int64_t T) {
+  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->hilo_mode == 0) return false;
+  return p->hilo_mode == 1 || (B == 1 && T <= 2048);
+}
+
 // Factor records of the solve plus its per-instance flags (bf16, k <= 64).
 size_t factor_bytes(int64_t B, int k) {
   const int rec = dyra::factor_record_floats(k);
@@ -169,14 +182,16 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
   auto caps = [p] {
     return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Lt +
-           p->cap_P2 + p->cap_TG2;
+           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo;
   };
   const size_t before = caps();
-  const void* ptrs[9] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Lt, p->P2, p->TG2};
+  const void* ptrs[11] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,  p->MD,
+                          p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[9] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD, p->Lt, p->P2, p->TG2};
+  const void* now[11] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,  p->MD,
+                         p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo};
   bool moved = before != caps();
-  for (int i = 0; i < 9; ++i) moved = moved || ptrs[i] != now[i];
+  for (int i = 0; i < 11; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -197,6 +212,11 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
       if ((rc = grow(p->MD, p->cap_MD, factor_bytes(B, k)))) return rc;
+      if (use_hilo(p, B, T)) {
+        if ((rc = grow(p->Llo, p->cap_Llo, static_cast<size_t>(N) * k * es))) return rc;
+        if ((rc = grow(p->Ctlo, p->cap_Ctlo, static_cast<size_t>(B) * k * p->d_out * es)))
+          return rc;
+      }
     }
   } else {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * (p->r + k) * es))) return rc;
@@ -331,6 +351,9 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     a.bias = p->has_bias ? p->bias : nullptr;
     a.alpha = p->alpha;
+    a.hilo = correct && use_hilo(p, B, T);
+    a.Llo = a.hilo ? p->Llo : nullptr;
+    a.Ctlo = a.hilo ? p->Ctlo : nullptr;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
                             [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
@@ -505,6 +528,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
                    : std::strcmp(fv, "self") == 0   ? 0
                    : std::strcmp(fv, "shared") == 0 ? 1
                                                     : -1;
+  const char* hv = std::getenv("DYRA_HILO");
+  p->hilo_mode = hv == nullptr ? -1 : (hv[0] == '1' ? 1 : (hv[0] == '0' ? 0 : -1));
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -713,6 +738,8 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->P2);
     void* tg2 = p->TG2;
     dev_free(tg2);
+    dev_free(p->Llo);
+    dev_free(p->Ctlo);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -841,7 +868,7 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         p->cap_Lt + p->cap_P2 + p->cap_TG2 + 256 +
+         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + 256 +
          (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
@@ -922,6 +949,10 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
       sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
       sizing.take(factor_bytes(B, k));
+      if (use_hilo(p, B, T)) {
+        sizing.take(static_cast<size_t>(N) * k * es);
+        sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+      }
     }
   } else {
     sizing.take(static_cast<size_t>(N) * (p->r + k) * es);
@@ -964,6 +995,9 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     void* fac = k > 0 ? carve.take(factor_bytes(B, k)) : nullptr;
     split_factor_buffer(fac, B, k, &a.MD, &a.counters);
+    a.hilo = k > 0 && use_hilo(p, B, T);
+    a.Llo = a.hilo ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
+    a.Ctlo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     a.factor_mode = p->factor_mode;
     a.splits = splits;
     a.split_rows = split_rows;

@@ -75,6 +75,12 @@ struct Bf16Forward {
   int proj_pair_min_tiles;    // see proj_shape (0: default)
   const void* bias = nullptr;  // d_out bf16 values added to Y, or nullptr
   float alpha = 1.f;           // weight of the correction (the solve scales L~ by it)
+  // Compensated correction: L~ and Q^T are also stored as their bf16 rounding
+  // errors (Llo, Ctlo) and the output stage adds hi.hi + hi.lo + lo.hi, which
+  // removes most of the cancellation error the grouping L~ . Q amplifies.
+  bool hilo = false;
+  void* Llo = nullptr;   // N x k
+  void* Ctlo = nullptr;  // d_out x (B*k)
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -147,9 +153,10 @@ int factor_record_floats(int k);
 // defer_wait (with pdl): the grid launched just before waited for the one
 // that wrote G and L before letting this one start; this grid then waits
 // for it only before its blocks exit.
-// alpha scales the result (the correction weight of the full linear layer).
-int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+// alpha scales the result (the correction weight of the full linear layer);
+// Llo (optional, N x k like L) receives the bf16 rounding error of each value.
+int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
+                  int64_t T, int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
                   bool defer_wait, unsigned long long* trace);
 // Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
 size_t ltilde_smem_bytes(int k);

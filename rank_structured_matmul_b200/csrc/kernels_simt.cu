@@ -368,8 +368,8 @@ static_assert(offsetof(LdlBlockScratch<32>, Wb) % 16 == 0 &&
 // = 16384 (the GEMM's warps take up to 104 registers).
 template <int KMAX, int MODE>
 __global__ void __maxnreg__(152)
-    ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, float* MD, int* flags, int T,
-                  int k, float lambda, float alpha, int* status, int defer_wait,
+    ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, __nv_bfloat16* Llo, float* MD,
+                  int* flags, int T, int k, float lambda, float alpha, int* status, int defer_wait,
                   unsigned long long* trace) {
   using Sm = LtSmem<KMAX>;
   constexpr int LD = LdlBlockScratch<KMAX>::LD;
@@ -560,6 +560,17 @@ __global__ void __maxnreg__(152)
       w.x = *reinterpret_cast<const uint32_t*>(&lo);
       w.y = *reinterpret_cast<const uint32_t*>(&hi);
       *reinterpret_cast<uint2*>(dst) = w;
+      if (Llo != nullptr) {  // the rounding errors of the four values just stored
+        const float2 l2 = __bfloat1622float2(lo), h2 = __bfloat1622float2(hi);
+        const __nv_bfloat162 elo = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][0] - l2.x,
+                                                         zero ? 0.f : alpha * acc[rr][1] - l2.y);
+        const __nv_bfloat162 ehi = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][2] - h2.x,
+                                                         zero ? 0.f : alpha * acc[rr][3] - h2.y);
+        uint2 we;
+        we.x = *reinterpret_cast<const uint32_t*>(&elo);
+        we.y = *reinterpret_cast<const uint32_t*>(&ehi);
+        *reinterpret_cast<uint2*>(Llo + (dst - L)) = we;
+      }
     }
   }
   if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
@@ -572,8 +583,8 @@ __global__ void __maxnreg__(152)
 // (Cholesky G_b = R R^T in shared memory) and solves R R^T w = l for 128 rows
 // of L_b, one per thread.
 __global__ void __launch_bounds__(kSolveThreads)
-    ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, int T, int k,
-                          float lambda, float alpha, int* status, int defer_wait) {
+    ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, __nv_bfloat16* Llo, int T,
+                          int k, float lambda, float alpha, int* status, int defer_wait) {
   extern __shared__ float sm[];
   const int ldg = k + 1;
   float* R = sm;                // k x (k+1): lower triangle becomes R
@@ -626,8 +637,12 @@ __global__ void __launch_bounds__(kSolveThreads)
       Ycol[i * kSolveThreads + tid] = acc / R[i * ldg + i];
     }
     const bool zero = bad != 0;
-    for (int i = 0; i < k; ++i)
-      row[i] = __float2bfloat16_rn(zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid]);
+    for (int i = 0; i < k; ++i) {
+      const float v = zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid];
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      row[i] = h;
+      if (Llo != nullptr) Llo[(row - L) + i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   if (defer_wait) sm100::pdl_wait();
@@ -791,9 +806,10 @@ size_t ltilde_smem_bytes(int k) {
 }
 
 template <int KMAX, int MODE>
-int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L, float* MD,
-                       int* flags, int64_t B, int64_t T, int k, float lambda, float alpha,
-                       int* status, int defer_wait, unsigned long long* trace) {
+int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L,
+                       __nv_bfloat16* Llo, float* MD, int* flags, int64_t B, int64_t T, int k,
+                       float lambda, float alpha, int* status, int defer_wait,
+                       unsigned long long* trace) {
   auto kfn = ltilde_kernel<KMAX, MODE>;
   static KernelSetup setup;
   const int d = setup_device();
@@ -812,14 +828,14 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
                      static_cast<unsigned>((T + lt_rows<KMAX>() - 1) / lt_rows<KMAX>()));
   cfg.blockDim = dim3(kLtThreads);
   cfg.dynamicSmemBytes = sizeof(LtSmem<KMAX>);
-  return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, alpha,
+  return cudaLaunchKernelEx(&cfg, kfn, G, L, Llo, MD, flags, static_cast<int>(T), k, lambda, alpha,
                             status, defer_wait, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
-int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
+                  int64_t T, int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
                   bool defer_wait, unsigned long long* trace) {
   const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
@@ -828,6 +844,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
     return -1;
   auto* Lb = static_cast<__nv_bfloat16*>(L);
+  auto* Lo = static_cast<__nv_bfloat16*>(Llo);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -837,15 +854,15 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   cfg.stream = s;
   if (k <= 32)
     return mode == kSolveShared
-               ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+               ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                       alpha, status, dw, trace)
-               : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+               : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                     alpha, status, dw, trace);
   if (k <= 64)
     return mode == kSolveShared
-               ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+               ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                       alpha, status, dw, trace)
-               : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
+               : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                     alpha, status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
   static KernelSetup setup;
@@ -862,7 +879,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
                      static_cast<unsigned>((T + kSolveThreads - 1) / kSolveThreads));
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
-  return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, static_cast<int>(T), k, lambda,
+  return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, Lo, static_cast<int>(T), k, lambda,
                             alpha, status, dw) == cudaSuccess
              ? 0
              : -1;

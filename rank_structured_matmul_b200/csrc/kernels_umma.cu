@@ -62,6 +62,9 @@ __device__ __forceinline__ int ceil_div_dev(int a, int b) { return (a + b - 1) /
 constexpr uint32_t kStoreBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kStoreBoxes = 2;
 
+// With LO set, the box receives the low part of each value instead,
+// bf16(v - bf16(v)): the two boxes together carry v to about 16 bits.
+template <bool LO = false>
 __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const void* tmap, int x,
                                                int y, EpiCtx& e,
                                                const __nv_bfloat16* bias = nullptr,
@@ -103,11 +106,15 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
       const int chunk = half * 4 + ch;
       const uint32_t off =
           static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+      auto val = [&](int c) {
+        const float v = f32(vv[half][8 * ch + c]);
+        return LO ? v - __bfloat162float(__float2bfloat16_rn(v)) : v;
+      };
       uint4 q;
-      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]), f32(vv[half][8 * ch + 1]));
-      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]), f32(vv[half][8 * ch + 3]));
-      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]), f32(vv[half][8 * ch + 5]));
-      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]), f32(vv[half][8 * ch + 7]));
+      q.x = pack_bf16x2(val(0), val(1));
+      q.y = pack_bf16x2(val(2), val(3));
+      q.z = pack_bf16x2(val(4), val(5));
+      q.w = pack_bf16x2(val(6), val(7));
       *reinterpret_cast<uint4*>(sbuf + off) = q;
     }
   }
@@ -531,7 +538,9 @@ struct RFactorPolicy {
     CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
     CUtensorMap tmT;  // (d_in, B*k),   box (64, bn)
     CUtensorMap tmC;  // (B*k, d_out),  box (64, 128), store
+    CUtensorMap tmClo;  // same over the low parts (hilo)
     int d_in, d_out, Bk, bn, n_tiles_n;
+    int hilo;  // also store the low parts of Q^T
   };
   struct Tile {
     int m0, n0;
@@ -542,6 +551,7 @@ struct RFactorPolicy {
     tma_prefetch_desc(&p.tmW);
     tma_prefetch_desc(&p.tmT);
     tma_prefetch_desc(&p.tmC);
+    if (p.hilo) tma_prefetch_desc(&p.tmClo);
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 128;
@@ -566,8 +576,10 @@ struct RFactorPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    for (int bx = 0; bx < p.bn / 64; ++bx)
+    for (int bx = 0; bx < p.bn / 64; ++bx) {
       store_box_bf16(tacc, bx * 64, &p.tmC, t.n0 + bx * 64, t.m0, e);
+      if (p.hilo) store_box_bf16<true>(tacc, bx * 64, &p.tmClo, t.n0 + bx * 64, t.m0, e);
+    }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
@@ -590,10 +602,22 @@ struct OutPolicy {
     CUtensorMap tmL;  // (k, T, B),     box (64, 128, 1)
     CUtensorMap tmC;  // (B*k, d_out),  box (64, bn)
     CUtensorMap tmY;  // (d_out, N),    box (64, 128), store
+    CUtensorMap tmLlo, tmClo;  // the low parts of L~ and Q^T (hilo)
     int N, r, k, T, B, bn, n_tiles_n, nkz, nkl;
     const __nv_bfloat16* bias;  // d_out, added in the epilogue, or nullptr
     int d_out;
+    int hilo;  // correction as hi L~ . hi Q + hi L~ . lo Q + lo L~ . hi Q
   };
+  // K-step j of the correction: instance segment, sub-product (0 hi.hi,
+  // 1 hi.lo, 2 lo.hi) and 64-wide chunk of k.
+  static __device__ __forceinline__ void correction_step(const Params& p, int j, int& seg,
+                                                         int& sub, int& ch) {
+    const int per = p.nkl * (p.hilo ? 3 : 1);
+    seg = j / per;
+    const int jj = j - seg * per;
+    sub = jj / p.nkl;
+    ch = jj - sub * p.nkl;
+  }
   struct Tile {
     int m0, n0, b_lo, nseg;
   };
@@ -605,6 +629,10 @@ struct OutPolicy {
     if (p.nkl > 0) {
       tma_prefetch_desc(&p.tmL);
       tma_prefetch_desc(&p.tmC);
+      if (p.hilo) {
+        tma_prefetch_desc(&p.tmLlo);
+        tma_prefetch_desc(&p.tmClo);
+      }
     }
     tma_prefetch_desc(&p.tmY);
   }
@@ -621,7 +649,7 @@ struct OutPolicy {
     }
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl;
+    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
@@ -629,12 +657,11 @@ struct OutPolicy {
       tma_load_2d(sa, &p.tmZ, bar, it * 64, t.m0);
       tma_load_2d(sb, &p.tmU, bar, it * 64, t.n0);
     } else {
-      const int j = it - p.nkz;
-      const int seg = j / p.nkl;
-      const int ch = j - seg * p.nkl;
+      int seg, sub, ch;
+      correction_step(p, it - p.nkz, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d(sa, &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
-      tma_load_2d(sb, &p.tmC, bar, b * p.k + ch * 64, t.n0);
+      tma_load_3d(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
+      tma_load_2d(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, t.n0);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
@@ -783,7 +810,7 @@ struct OutPairPolicy {
     }
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl;
+    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
@@ -793,12 +820,11 @@ struct OutPairPolicy {
       tma_load_2d_pair(sa, &p.tmZ, bar, it * 64, ma);
       tma_load_2d_pair(sb, &p.tmU, bar, it * 64, nb);
     } else {
-      const int j = it - p.nkz;
-      const int seg = j / p.nkl;
-      const int ch = j - seg * p.nkl;
+      int seg, sub, ch;
+      OutPolicy::correction_step(p, it - p.nkz, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d_pair(sa, &p.tmL, bar, ch * 64, ma - b * p.T, b);
-      tma_load_2d_pair(sb, &p.tmC, bar, b * p.k + ch * 64, nb);
+      tma_load_3d_pair(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, ma - b * p.T, b);
+      tma_load_2d_pair(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, nb);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
@@ -1187,6 +1213,12 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, 128};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
+      p.hilo = a.hilo ? 1 : 0;
+      if (a.hilo) {
+        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
+      } else {
+        p.tmClo = p.tmC;
+      }
       if (rf_pairs) {
         const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
         const uint32_t smem =
@@ -1222,8 +1254,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
                  ? 1
                  : 0;
     if (!records) mode = 0;
-    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.alpha,
-                      a.status, s, pdl, /*defer_wait=*/true,
+    if (launch_ltilde(a.TG, a.L, a.hilo ? a.Llo : nullptr, a.MD, a.counters, mode, a.B, a.T, a.k,
+                      a.lambda, a.alpha, a.status, s, pdl, /*defer_wait=*/true,
                       a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
   } else {
@@ -1269,10 +1301,20 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, bbox};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
+      if (a.hilo) {
+        if (!encode_tmap_bf16(&p.tmLlo, a.Llo, 3, dl, sl, bl, 128)) return -2;
+        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
+      } else {
+        p.tmLlo = p.tmL;
+        p.tmClo = p.tmC;
+      }
     } else {
       p.tmL = p.tmZ;
       p.tmC = p.tmU;
+      p.tmLlo = p.tmZ;
+      p.tmClo = p.tmU;
     }
+    p.hilo = k > 0 && a.hilo ? 1 : 0;
     uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
     uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
     uint32_t by[2] = {64, 128};

@@ -291,6 +291,43 @@ def test_host_forward_matches_device_forward(B, T):
     layer.close()
 
 
+HILO = [
+    # name, d_in, d_out, r, k, B, T, outlier channels (x20)
+    ("hilo_single", 1024, 2048, 128, 64, 1, 128, 8),
+    ("hilo_batched", 256, 512, 64, 32, 3, 201, 8),
+    ("hilo_needed", 512, 1024, 64, 64, 1, 128, 6),   # modelled 1.1e-2 without it, 6.8e-3 with
+]
+
+
+def _run_hilo(s, f, mode):
+    os.environ["DYRA_HILO"] = mode
+    try:
+        layer = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_HILO", None)
+    Y = layer.forward(to_dev(f["X"], s.dtype), B=s.B, T=s.T)
+    assert layer.status() == 0
+    layer.close()
+    Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, s.B, s.T)
+    return oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+
+
+@pytest.mark.parametrize("case", HILO, ids=[c[0] for c in HILO])
+def test_compensated_correction(case):
+    """L~ and Q^T with their bf16 rounding errors (hi.hi + hi.lo + lo.hi in
+    the output stage) cut the error the grouping L~ . Q amplifies on
+    ill-conditioned instances (outlier channels)."""
+    name, d_in, d_out, r, k, B, T, nout = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, "bf16", 0.6, "outlier", n_outlier=nout,
+                  outlier_scale=20.0, seed=5)
+    f = prepared(s)
+    err_on = _run_hilo(s, f, "1")
+    assert err_on <= TOL["bf16"], "%s: %.3e" % (name, err_on)
+    if name != "hilo_needed":
+        err_off = _run_hilo(s, f, "0")
+        assert err_on < 0.8 * err_off, (err_on, err_off)
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
