@@ -184,7 +184,7 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
  *     returns DYRA_ERR_INVALID_ARG and enqueues nothing. For a bf16 plan they
  *     take about 2*B*T*(r+k) + 4*B*k*k + 2*B*k*(d_in+d_out) + 4*B*F bytes,
  *     each part rounded up to 256, where F = K*K + 5 with K = 32 for
- *     k <= 32, 64 for k <= 64 (F = 0 above), plus 2*B*T*k + 2*B*k*d_out
+ *     k <= 32, 64 for k <= 64 (F = 0 above), plus 2*B*T*k + 2*B*k*(d_in + d_out)
  *     when the compensated correction is on (a single instance of at most
  *     2048 rows, or DYRA_HILO=1).
  *   - The first call on a device looks the array's device address up

@@ -52,6 +52,7 @@ struct dyra_plan {
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
   void* Llo = nullptr;   // bf16, compensated correction: N x k
   void* Ctlo = nullptr;  // bf16, compensated correction: d_out x (B*k)
+  void* Tplo = nullptr;  // bf16, compensated correction: (B*k) x d_in
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
   // ALS updates per forward (dyra_set_als_steps; CUDA-core plans beyond 2) and
   // the buffers the further L updates use
@@ -60,7 +61,7 @@ struct dyra_plan {
   void* P2 = nullptr;    // (B*k) x d_in
   float* TG2 = nullptr;  // B x k x (T + k)
   size_t cap_Lt = 0, cap_P2 = 0, cap_TG2 = 0;
-  size_t cap_Llo = 0, cap_Ctlo = 0;
+  size_t cap_Llo = 0, cap_Ctlo = 0, cap_Tplo = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -182,16 +183,16 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
   auto caps = [p] {
     return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Lt +
-           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo;
+           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo;
   };
   const size_t before = caps();
-  const void* ptrs[11] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,  p->MD,
-                          p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo};
+  const void* ptrs[12] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,
+                          p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[11] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,  p->MD,
-                         p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo};
+  const void* now[12] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,
+                         p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo};
   bool moved = before != caps();
-  for (int i = 0; i < 11; ++i) moved = moved || ptrs[i] != now[i];
+  for (int i = 0; i < 12; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -215,6 +216,8 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if (use_hilo(p, B, T)) {
         if ((rc = grow(p->Llo, p->cap_Llo, static_cast<size_t>(N) * k * es))) return rc;
         if ((rc = grow(p->Ctlo, p->cap_Ctlo, static_cast<size_t>(B) * k * p->d_out * es)))
+          return rc;
+        if ((rc = grow(p->Tplo, p->cap_Tplo, static_cast<size_t>(B) * k * p->d_in * es)))
           return rc;
       }
     }
@@ -354,6 +357,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.hilo = correct && use_hilo(p, B, T);
     a.Llo = a.hilo ? p->Llo : nullptr;
     a.Ctlo = a.hilo ? p->Ctlo : nullptr;
+    a.split_t = a.hilo;
+    a.Tplo = a.hilo ? p->Tplo : nullptr;
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
                             [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
@@ -740,6 +745,7 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(tg2);
     dev_free(p->Llo);
     dev_free(p->Ctlo);
+    dev_free(p->Tplo);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -868,7 +874,7 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + 256 +
+         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo + 256 +
          (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
@@ -952,6 +958,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
       if (use_hilo(p, B, T)) {
         sizing.take(static_cast<size_t>(N) * k * es);
         sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+        sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       }
     }
   } else {
@@ -998,6 +1005,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.hilo = k > 0 && use_hilo(p, B, T);
     a.Llo = a.hilo ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
     a.Ctlo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
+    a.split_t = a.hilo;
+    a.Tplo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_in * es) : nullptr;
     a.factor_mode = p->factor_mode;
     a.splits = splits;
     a.split_rows = split_rows;

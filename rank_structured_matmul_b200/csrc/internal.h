@@ -81,6 +81,11 @@ struct Bf16Forward {
   bool hilo = false;
   void* Llo = nullptr;   // N x k
   void* Ctlo = nullptr;  // d_out x (B*k)
+  // Split T: T = L^T X also as its bf16 rounding errors (Tplo), which the
+  // rank-k factor GEMM accumulates as a second B operand, so Q is formed from
+  // T to about 16 bits
+  bool split_t = false;
+  void* Tplo = nullptr;  // (B*k) x d_in
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)

@@ -384,6 +384,7 @@ struct GramPolicy {
     int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total;
     uint32_t b_layout;
     __nv_bfloat16* Tb;  // (B*k) x d_in
+    __nv_bfloat16* Tlo;  // (B*k) x d_in: the bf16 rounding errors of Tb, or nullptr
     float* G;           // B x k x k
   };
   struct Tile {
@@ -449,10 +450,17 @@ struct GramPolicy {
     if (t.mt < p.mtx) {
       const int j = t.mt * 128 + row;
       if (j >= p.d_in) return;
-      __nv_bfloat16* dst = p.Tb + static_cast<size_t>(t.b) * p.k * p.d_in + j;
+      const size_t off = static_cast<size_t>(t.b) * p.k * p.d_in + j;
+      __nv_bfloat16* dst = p.Tb + off;
 #pragma unroll
       for (int u = 0; u < n; ++u)
-        if (i0 + u < p.k) dst[static_cast<size_t>(i0 + u) * p.d_in] = __float2bfloat16_rn(v[u]);
+        if (i0 + u < p.k) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(v[u]);
+          dst[static_cast<size_t>(i0 + u) * p.d_in] = h;
+          if (p.Tlo != nullptr)
+            p.Tlo[off + static_cast<size_t>(i0 + u) * p.d_in] =
+                __float2bfloat16_rn(v[u] - __bfloat162float(h));
+        }
     } else {
       const int i2 = (t.mt - p.mtx) * 128 + row;
       if (i2 >= p.k) return;
@@ -539,8 +547,10 @@ struct RFactorPolicy {
     CUtensorMap tmT;  // (d_in, B*k),   box (64, bn)
     CUtensorMap tmC;  // (B*k, d_out),  box (64, 128), store
     CUtensorMap tmClo;  // same over the low parts (hilo)
+    CUtensorMap tmTlo;  // the low parts of T (split T), like tmT
     int d_in, d_out, Bk, bn, n_tiles_n;
-    int hilo;  // also store the low parts of Q^T
+    int hilo;    // also store the low parts of Q^T
+    int split_t;  // T arrives as hi and lo parts: a second B operand per stage
   };
   struct Tile {
     int m0, n0;
@@ -552,6 +562,7 @@ struct RFactorPolicy {
     tma_prefetch_desc(&p.tmT);
     tma_prefetch_desc(&p.tmC);
     if (p.hilo) tma_prefetch_desc(&p.tmClo);
+    if (p.split_t) tma_prefetch_desc(&p.tmTlo);
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 128;
@@ -564,6 +575,7 @@ struct RFactorPolicy {
                                               uint32_t sb, uint32_t bar) {
     tma_load_2d(sa, &p.tmW, bar, it * 64, t.m0);
     tma_load_2d(sb, &p.tmT, bar, it * 64, t.n0);
+    if (p.split_t) tma_load_2d(sb + static_cast<uint32_t>(p.bn) * 128u, &p.tmTlo, bar, it * 64, t.n0);
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
     return min(4, ceil_div_dev(p.d_in - it * 64, 16));
@@ -725,6 +737,9 @@ struct RFactorPairPolicy {
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
     tma_load_2d_pair(sa, &p.tmW, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
     tma_load_2d_pair(sb, &p.tmT, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
+    if (p.split_t)
+      tma_load_2d_pair(sb + static_cast<uint32_t>(p.bn / 2) * 128u, &p.tmTlo, bar, it * 64,
+                       t.n0 + (p.bn / 2) * static_cast<int>(rank));
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
     return RFactorPolicy::ksteps(p, t, it);
@@ -873,6 +888,8 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   c.num_tiles = num_tiles;
   c.defer_wait = 0;
   c.trigger_after_wait = 0;
+  c.b_parts = 1;
+  c.b_part_desc = 0;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -1153,6 +1170,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.mtx = ceil_div(a.d_in, 128);
       p.mt_total = p.mtx + ceil_div(a.k, 128);
       p.Tb = static_cast<__nv_bfloat16*>(a.Tp);
+      p.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
       p.G = a.TG;
       p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
       uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
@@ -1209,6 +1227,13 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
       uint32_t bt[2] = {64, static_cast<uint32_t>(rf_pairs ? p.bn / 2 : p.bn)};
       if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
+      p.split_t = a.split_t ? 1 : 0;
+      if (a.split_t) {
+        if (!encode_tmap_bf16(&p.tmTlo, a.Tplo, 2, dt, sw, bt, 128)) return -2;
+      } else {
+        p.tmTlo = p.tmT;
+      }
+      const uint32_t parts = a.split_t ? 2u : 1u;  // B operands per stage
       uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, 128};
@@ -1221,20 +1246,26 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       }
       if (rf_pairs) {
         const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
+        const uint32_t part_bytes = static_cast<uint32_t>(p.bn / 2) * 128u;
         const uint32_t smem =
-            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
+            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
                                             false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.b_parts = parts;
+        p.c.b_part_desc = part_bytes >> 4;
         p.c.trigger_after_wait = 1;
         p.c.idesc = idesc_bf16(256, p.bn, false, false);
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
       } else {
         const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
+        const uint32_t part_bytes = static_cast<uint32_t>(p.bn) * 128u;
         const uint32_t smem =
-            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false,
-                                        a.status, dev, rf_smem_cap);
+            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
+                                        false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.b_parts = parts;
+        p.c.b_part_desc = part_bytes >> 4;
         p.c.trigger_after_wait = 1;
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
