@@ -213,3 +213,31 @@ def test_planted_monarch_mistakes_are_caught(monkeypatch, target, mutant):
         except (AssertionError, ValueError, np.linalg.LinAlgError):
             failures += 1
     assert failures > 0, "no pin catches the planted mistake %s" % mutant.__name__
+
+
+# ------------------------------------------------ over random block counts ----
+
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(st.integers(1, 5), st.integers(1, 5), st.integers(0, 10_000))
+def test_projection_properties_over_block_counts(b1, b2, seed):
+    """For any b1, b2: a Monarch matrix is its own projection, and the
+    projection error is the block-wise Eckart-Young sum."""
+    rng = np.random.default_rng(seed)
+    N = b1 * b2
+    Lb = [rng.standard_normal((b1, b1)) for _ in range(b2)]
+    Rb = [rng.standard_normal((b2, b2)) for _ in range(b1)]
+    M = mon.monarch_matrix(Lb, Rb)
+    np.testing.assert_allclose(mon.monarch_matrix(*mon.monarch_project(M, b1, b2)), M, rtol=0,
+                               atol=1e-10 * max(1.0, np.abs(M).max()))
+    W = rng.standard_normal((N, N))
+    err = np.sum((W - mon.monarch_matrix(*mon.monarch_project(W, b1, b2))) ** 2)
+    want = 0.0
+    for j1 in range(b1):
+        for j2 in range(b2):
+            S = np.array([[W[m1 * b2 + j2, j1 * b2 + i2] for i2 in range(b2)] for m1 in range(b1)])
+            want += np.sum(S ** 2) - top_singular_value(S, iters=2000) ** 2
+    assert err == pytest.approx(want, rel=1e-7, abs=1e-9)
