@@ -94,6 +94,13 @@ struct SimtForward {
   T* Tp;        // (B*k) x d_in
   T* Cm;        // (B*k) x d_out
   int* status;
+  // Monarch static part ([DyRA] App. B), r = 0: y = x W_hat in the paper's
+  // layout, W_hat = P L P^T R with Lblk b2 blocks of mb1 x mb1 and Rblk mb1
+  // blocks of mb2 x mb2 (row-major, contiguous); Mtmp is N x n
+  const T* Lblk = nullptr;
+  const T* Rblk = nullptr;
+  int mb1 = 0, mb2 = 0;
+  T* Mtmp = nullptr;
 };
 
 template <typename T>

@@ -904,10 +904,20 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
              0, 1, 0, s))
       return -1;
   }
-  // Y = Z U^T
-  if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out, 1, 0,
-           1, 0, s))
+  if (a.Lblk != nullptr) {
+    // Monarch static part: y[j1*b2 + i2] = sum_{m1, j2} x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2],
+    // as two strided batched products through Mtmp[row][j2*b1 + j1]
+    const int n = a.d_in, b1 = a.mb1, b2 = a.mb2;
+    if (gemm(static_cast<int>(N), b1, b1, a.X, n, b2, 1, a.Lblk, b1, 1,
+             static_cast<int64_t>(b1) * b1, a.Mtmp, n, 1, b1, b2, 0, s))
+      return -1;
+    if (gemm(static_cast<int>(N), b2, b2, a.Mtmp, n, b1, 1, a.Rblk, b2, 1,
+             static_cast<int64_t>(b2) * b2, a.Y, n, 1, b2, b1, 0, s))
+      return -1;
+  } else if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out,
+                  1, 0, 1, 0, s)) {  // Y = Z U^T
     return -1;
+  }
   if (k > 0) {
     // Y_b += L_b C_b
     if (gemm(Tr, a.d_out, k, a.ZL + a.r, rk, 1, static_cast<int64_t>(Tr) * rk, a.Cm, a.d_out, 1,
