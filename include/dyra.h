@@ -84,6 +84,32 @@ enum {
 int dyra_plan_create(dyra_plan_t *out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype);
 
 /*
+ * A plan whose static part is a Monarch matrix ([DyRA] App. B) instead of the
+ * rank-r factorisation, for a square layer of n = b1 * b2 features (the pages
+ * define Monarch for square weights). The correction (rank k, 0 <= k <= n,
+ * k <= 128) is unchanged. In the paper's layout (Y = X W) the static product
+ * is X W_hat with W_hat = P L P^T R: y[j1*b2 + i2] = sum over m1, j2 of
+ * x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2], with P the perfect shuffle. These
+ * plans run on the CUDA-core kernels (fp32, or bf16 with bf16 intermediates);
+ * dyra_forward_batched_noalloc returns DYRA_ERR_UNSUPPORTED for them.
+ * Errors as dyra_plan_create; DYRA_ERR_INVALID_ARG also when n != b1 * b2.
+ */
+int dyra_plan_create_monarch(dyra_plan_t *out, int n, int b1, int b2, int k, dyra_dtype_t dtype);
+
+/*
+ * Load a Monarch plan's factors (the counterpart of dyra_load_factors):
+ *   Lblocks : b2 blocks of b1 x b1, row-major, one after the other (L_j2[m1][j1])
+ *   Rblocks : b1 blocks of b2 x b2, row-major, one after the other (R_j1[j2][i2])
+ *   P, W_res, lambda : as in dyra_load_factors, with W_res = W - W_hat^T in this
+ *                      library's n x n (d_out x d_in) layout
+ * Device pointers in the plan dtype, copied on `stream`. DYRA_ERR_INVALID_ARG
+ * for a plan not made by dyra_plan_create_monarch (and dyra_load_factors
+ * rejects Monarch plans).
+ */
+int dyra_load_monarch(dyra_plan_t p, const void *Lblocks, const void *Rblocks, const void *P,
+                      const void *W_res, float lambda, dyra_stream_t stream);
+
+/*
  * Copy the offline factors into the plan ([DyRA] Alg. 1, Offline Preparation
  * outputs: the structured approximation, W_res and P_L).
  *   U      : d_out x r   (singular values folded in: W_hat = U V^T)

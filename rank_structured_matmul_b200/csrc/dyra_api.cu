@@ -19,6 +19,14 @@
 
 struct dyra_plan {
   int d_in = 0, d_out = 0, r = 0, k = 0;
+  // Monarch static part ([DyRA] App. B) in place of U V^T: n = d_in = d_out =
+  // b1 * b2, b2 blocks of b1 x b1 (Lblk) and b1 blocks of b2 x b2 (Rblk); r = 0
+  bool monarch = false;
+  int mb1 = 0, mb2 = 0;
+  void* Lblk = nullptr;
+  void* Rblk = nullptr;
+  void* Mtmp = nullptr;  // workspace: N x n, the product's intermediate
+  size_t cap_Mtmp = 0;
   dyra_dtype_t dtype = DYRA_BF16;
   dyra::DeviceInfo dev;
   bool loaded = false;
@@ -160,7 +168,8 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
 // Whether a tensor-core forward of B x T rows uses the compensated correction.
 bool use_hilo(const dyra_plan* p, int64_t B, int64_t T) {
-  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->hilo_mode == 0) return false;
+  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->monarch || p->hilo_mode == 0)
+    return false;
   return p->hilo_mode == 1 || (B == 1 && T <= 2048);
 }
 
@@ -183,16 +192,16 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
   auto caps = [p] {
     return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Lt +
-           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo;
+           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo + p->cap_Mtmp;
   };
   const size_t before = caps();
-  const void* ptrs[12] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,
-                          p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo};
+  const void* ptrs[13] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,  p->Lt,
+                          p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo, p->Mtmp};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[12] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,
-                         p->Lt, p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo};
+  const void* now[13] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,  p->Lt,
+                         p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo, p->Mtmp};
   bool moved = before != caps();
-  for (int i = 0; i < 12; ++i) moved = moved || ptrs[i] != now[i];
+  for (int i = 0; i < 13; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -202,7 +211,12 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   const size_t es = elem_size(p->dtype);
   const int k = p->k;
   int rc;
-  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+  if (p->monarch) {
+    void* mt = p->Mtmp;
+    if ((rc = grow(mt, p->cap_Mtmp, static_cast<size_t>(N) * p->d_in * es))) return rc;
+    p->Mtmp = mt;
+  }
+  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
     if (k > 0) {
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
@@ -322,7 +336,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
   int rc = ensure_workspace(p, B, T);
   if (rc) return rc;
 
-  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
     dyra::Bf16Forward a;
     a.d_in = p->d_in;
     a.d_out = p->d_out;
@@ -388,6 +402,13 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Lt = static_cast<__nv_bfloat16*>(p->Lt);
     a.P2 = static_cast<__nv_bfloat16*>(p->P2);
     a.TG2 = p->TG2;
+    if (p->monarch) {
+      a.Lblk = static_cast<const __nv_bfloat16*>(p->Lblk);
+      a.Rblk = static_cast<const __nv_bfloat16*>(p->Rblk);
+      a.mb1 = p->mb1;
+      a.mb2 = p->mb2;
+      a.Mtmp = static_cast<__nv_bfloat16*>(p->Mtmp);
+    }
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   } else {
@@ -416,6 +437,13 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Lt = static_cast<float*>(p->Lt);
     a.P2 = static_cast<float*>(p->P2);
     a.TG2 = p->TG2;
+    if (p->monarch) {
+      a.Lblk = static_cast<const float*>(p->Lblk);
+      a.Rblk = static_cast<const float*>(p->Rblk);
+      a.mb1 = p->mb1;
+      a.mb2 = p->mb2;
+      a.Mtmp = static_cast<float*>(p->Mtmp);
+    }
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
                             [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   }
@@ -491,6 +519,9 @@ const char* dyra_error_string(int code) {
   }
 }
 
+static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
+                            dyra_dtype_t dtype);
+
 int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype) {
   if (out == nullptr) return DYRA_ERR_INVALID_ARG;
   if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
@@ -498,6 +529,25 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   const int m = d_in < d_out ? d_in : d_out;
   if (r + k > m) return DYRA_ERR_INVALID_ARG;
   if (dtype == DYRA_BF16 && (d_in % 8 || d_out % 8 || r % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
+  return plan_create_impl(out, d_in, d_out, r, k, dtype);
+}
+
+int dyra_plan_create_monarch(dyra_plan_t* out, int n, int b1, int b2, int k, dyra_dtype_t dtype) {
+  if (out == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
+  if (b1 < 1 || b2 < 1 || n != b1 * b2 || k < 0 || k > 128 || k > n) return DYRA_ERR_INVALID_ARG;
+  if (dtype == DYRA_BF16 && (n % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
+  const int rc = plan_create_impl(out, n, n, 0, k, dtype);
+  if (rc == DYRA_OK) {
+    (*out)->monarch = true;
+    (*out)->mb1 = b1;
+    (*out)->mb2 = b2;
+  }
+  return rc;
+}
+
+static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
+                            dyra_dtype_t dtype) {
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -554,7 +604,7 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
 
 int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P,
                       const void* W_res, float lambda, dyra_stream_t stream) {
-  if (p == nullptr || U == nullptr || V == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (p == nullptr || U == nullptr || V == nullptr || p->monarch) return DYRA_ERR_INVALID_ARG;
   if (p->k > 0 && (P == nullptr || W_res == nullptr)) return DYRA_ERR_INVALID_ARG;
   if (!(lambda >= 0.f) || !std::isfinite(lambda)) return DYRA_ERR_INVALID_ARG;
   if (!aligned16(U) || !aligned16(V) || (p->k > 0 && (!aligned16(P) || !aligned16(W_res))))
@@ -612,7 +662,7 @@ int dyra_set_linear(dyra_plan_t p, const void* bias, float alpha, dyra_stream_t 
 
 int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
   if (p == nullptr || half_steps < 2 || half_steps > 64) return DYRA_ERR_INVALID_ARG;
-  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
   if (umma && half_steps != 2) return DYRA_ERR_UNSUPPORTED;
   p->als_half_steps = half_steps;
   drop_graphs(p);  // captured forwards hold the old count
@@ -689,6 +739,47 @@ int dyra_forward_batched_host(dyra_plan_t p, const void* X, void* Y, int64_t B, 
   return DYRA_OK;
 }
 
+int dyra_load_monarch(dyra_plan_t p, const void* Lblocks, const void* Rblocks, const void* P,
+                      const void* W_res, float lambda, dyra_stream_t stream) {
+  if (p == nullptr || !p->monarch || Lblocks == nullptr || Rblocks == nullptr)
+    return DYRA_ERR_INVALID_ARG;
+  if (p->k > 0 && (P == nullptr || W_res == nullptr)) return DYRA_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f) || !std::isfinite(lambda)) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(p->dtype);
+  const size_t n = static_cast<size_t>(p->d_in);
+  const size_t lb = static_cast<size_t>(p->mb2) * p->mb1 * p->mb1 * es;
+  const size_t rb = static_cast<size_t>(p->mb1) * p->mb2 * p->mb2 * es;
+  const size_t vpt = static_cast<size_t>(p->k) * n * es;
+  const size_t wb = p->k > 0 ? n * n * es : 0;
+  int rc;
+  if (!p->Lblk && (rc = dev_alloc(&p->Lblk, lb))) return rc;
+  if (!p->Rblk && (rc = dev_alloc(&p->Rblk, rb))) return rc;
+  if (vpt && !p->VPt && (rc = dev_alloc(&p->VPt, vpt))) return rc;
+  if (wb && !p->W_res && (rc = dev_alloc(&p->W_res, wb))) return rc;
+  p->factor_bytes = lb + rb + vpt + wb;
+  if (cudaMemcpyAsync(p->Lblk, Lblocks, lb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(p->Rblk, Rblocks, rb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      (wb && cudaMemcpyAsync(p->W_res, W_res, wb, cudaMemcpyDeviceToDevice, s) != cudaSuccess))
+    return DYRA_ERR_CUDA;
+  if (vpt) {  // P^T (k x n): the projection's B operand, as [V | P]^T with r = 0
+    if (p->dtype == DYRA_BF16)
+      rc = dyra::launch_pack_vp(static_cast<const __nv_bfloat16*>(P),
+                                static_cast<const __nv_bfloat16*>(P),
+                                static_cast<__nv_bfloat16*>(p->VPt), p->d_in, 0, p->k, s);
+    else
+      rc = dyra::launch_pack_vp(static_cast<const float*>(P), static_cast<const float*>(P),
+                                static_cast<float*>(p->VPt), p->d_in, 0, p->k, s);
+    if (rc) return DYRA_ERR_CUDA;
+  }
+  p->lambda = lambda;
+  p->loaded = true;
+  drop_graphs(p);
+  return DYRA_OK;
+}
+
 int dyra_forward(dyra_plan_t p, const void* X, void* Y, int64_t N, dyra_stream_t stream) {
   return run_forward(p, X, Y, 1, N, false, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -732,6 +823,9 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->U);
     dev_free(p->W_res);
     dev_free(p->bias);
+    dev_free(p->Lblk);
+    dev_free(p->Rblk);
+    dev_free(p->Mtmp);
     dev_free(p->Z);
     dev_free(p->L);
     void* tg = p->TG;
@@ -804,7 +898,7 @@ int dyra_debug_set_stage_timing(dyra_plan_t p, int enable) {
     for (auto& e : p->stage_ev)
       if (cudaEventCreate(&e) != cudaSuccess) return DYRA_ERR_CUDA;
   }
-  p->stage_timing = enable != 0 && p->dtype == DYRA_BF16 && !p->force_simt;
+  p->stage_timing = enable != 0 && p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
   p->stage_recorded = false;
   return p->stage_timing || !enable ? DYRA_OK : DYRA_ERR_INVALID_ARG;
 }
@@ -874,7 +968,8 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo + 256 +
+         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo +
+         p->cap_Mtmp + 256 +
          (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
@@ -935,6 +1030,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
   if (N > (static_cast<int64_t>(1) << 31) - 1 || B * static_cast<int64_t>(p->k) > (1 << 30))
     return DYRA_ERR_INVALID_ARG;
   if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  if (p->monarch) return DYRA_ERR_UNSUPPORTED;
   if (!aligned16(X) || !aligned16(Y)) return DYRA_ERR_ALIGNMENT;
   const int k = p->k;
   if (k > 0 && p->lambda == 0.f && T < k) return DYRA_ERR_RANK_DEFICIENT;

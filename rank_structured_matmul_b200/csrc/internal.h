@@ -137,6 +137,13 @@ struct SimtForward {
   T* Lt = nullptr;       // (B*k) x Trows: the latest L_b, transposed
   T* P2 = nullptr;       // (B*k) x d_in: R_b W_res, the L update's projector before its solve
   float* TG2 = nullptr;  // B x k x (Trows + k): [ (X_b P2_b^T)^T | R_b R_b^T ]
+  // Monarch static part ([DyRA] App. B), r = 0: y = x W_hat in the paper's
+  // layout, W_hat = P L P^T R with Lblk b2 blocks of mb1 x mb1 and Rblk mb1
+  // blocks of mb2 x mb2 (row-major, contiguous); Mtmp is N x n
+  const T* Lblk = nullptr;
+  const T* Rblk = nullptr;
+  int mb1 = 0, mb2 = 0;
+  T* Mtmp = nullptr;
 };
 
 template <typename T>

@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(256)
     simt_gemm_kernel(int M, int N, int K, const TA* __restrict__ A, int64_t am, int64_t ak,
                      int64_t ab, const TB* __restrict__ Bm, int64_t bk, int64_t bn, int64_t bb,
                      TC* __restrict__ C, int64_t cm, int64_t cn, int64_t cb, int accumulate,
-                     float alpha, const TC* __restrict__ bias) {
+                     float alpha, const TC* __restrict__ bias, int64_t bias_b) {
   __shared__ float As[kGK][kGT + 1];
   __shared__ float Bs[kGK][kGT + 1];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -700,7 +700,7 @@ __global__ void __launch_bounds__(256)
       if (gn >= N) continue;
       TC* dst = C + gm * cm + gn * cn;
       float v = alpha * acc[i][j];
-      if (bias) v += to_f<TC>(bias[gn]);
+      if (bias) v += to_f<TC>(bias[batch * bias_b + gn]);
       if (accumulate) v += to_f<TC>(*dst);
       *dst = from_f<TC>(v);
     }
@@ -711,11 +711,11 @@ template <typename TA, typename TB, typename TC>
 int gemm(int M, int N, int K, const TA* A, int64_t am, int64_t ak, int64_t ab, const TB* Bm,
          int64_t bk, int64_t bn, int64_t bb, TC* C, int64_t cm, int64_t cn, int64_t cb,
          int batches, int accumulate, cudaStream_t s, float alpha = 1.f,
-         const TC* bias = nullptr) {
+         const TC* bias = nullptr, int64_t bias_b = 0) {
   if (M <= 0 || N <= 0 || batches <= 0) return 0;
   dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, batches);
   simt_gemm_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb, C,
-                                                    cm, cn, cb, accumulate, alpha, bias);
+                                                    cm, cn, cb, accumulate, alpha, bias, bias_b);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -971,10 +971,20 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
       lb = static_cast<int64_t>(k) * Tr;
     }
   }
-  // Y = Z U^T (+ b)
-  if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out, 1, 0,
-           1, 0, s, 1.f, a.bias))
+  if (a.Lblk != nullptr) {
+    // Monarch static part: y[j1*b2 + i2] = sum_{m1, j2} x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2],
+    // as two strided batched products through Mtmp[row][j2*b1 + j1]
+    const int n = a.d_in, b1 = a.mb1, b2 = a.mb2;
+    if (gemm(static_cast<int>(N), b1, b1, a.X, n, b2, 1, a.Lblk, b1, 1,
+             static_cast<int64_t>(b1) * b1, a.Mtmp, n, 1, b1, b2, 0, s))
+      return -1;
+    if (gemm(static_cast<int>(N), b2, b2, a.Mtmp, n, b1, 1, a.Rblk, b2, 1,
+             static_cast<int64_t>(b2) * b2, a.Y, n, 1, b2, b1, 0, s, 1.f, a.bias, b2))
+      return -1;
+  } else if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out,
+                  1, 0, 1, 0, s, 1.f, a.bias)) {  // Y = Z U^T (+ b)
     return -1;
+  }
   if (k > 0) {
     // Y_b += alpha L_b R_b (the last pair)
     if (gemm(Tr, a.d_out, k, Lp, lm, lq, lb, a.Cm, a.d_out, 1, static_cast<int64_t>(k) * a.d_out,

@@ -39,6 +39,8 @@ SIGNATURES = {
     "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
     "dyra_set_als_steps": (_i, [_vp, _i]),
     "dyra_forward_batched_host": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
+    "dyra_plan_create_monarch": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "dyra_load_monarch": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -141,6 +143,18 @@ def dyra_forward_batched_host(plan: int, X, Y, B: int, T: int, stream=None) -> N
     """dyra_forward_batched on host buffers (X, Y page-locked CPU tensors or addresses)."""
     _check(lib().dyra_forward_batched_host(plan, _ptr(X), _ptr(Y), int(B), int(T),
                                            _stream(stream)), "dyra_forward_batched_host")
+
+
+def dyra_plan_create_monarch(n: int, b1: int, b2: int, k: int, dtype: int) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().dyra_plan_create_monarch(ctypes.byref(h), n, b1, b2, k, dtype),
+           "dyra_plan_create_monarch")
+    return h.value
+
+
+def dyra_load_monarch(plan: int, Lblocks, Rblocks, P, W_res, lam: float, stream=None) -> None:
+    _check(lib().dyra_load_monarch(plan, _ptr(Lblocks), _ptr(Rblocks), _ptr(P), _ptr(W_res),
+                                   float(lam), _stream(stream)), "dyra_load_monarch")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -324,3 +338,25 @@ class DyraLinear:
             self.close()
         except Exception:
             pass
+
+
+class DyraMonarchLinear(DyraLinear):
+    """A DyRA layer whose static part is a Monarch matrix (DyRA App. B) of
+    n = b1 * b2 features; load() takes the blocks instead of U and V."""
+
+    def __init__(self, n: int, b1: int, b2: int, k: int, dtype: str = "bf16"):
+        import torch
+        self.d_in = self.d_out = n
+        self.r, self.k, self.b1, self.b2 = 0, k, b1, b2
+        self.dtype = dtype
+        self.torch_dtype = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
+        self.plan = dyra_plan_create_monarch(n, b1, b2, k,
+                                             DYRA_BF16 if dtype == "bf16" else DYRA_F32)
+
+    def load(self, Lblocks, Rblocks, P, W_res, lam: float, stream=None) -> None:
+        """Lblocks: (b2, b1, b1), Rblocks: (b1, b2, b2), P: (n, k), W_res: (n, n)."""
+        import torch
+        Lb, Rb, P, W_res = (self._dev(t) for t in (Lblocks, Rblocks, P, W_res))
+        dyra_load_monarch(self.plan, Lb, Rb, P if self.k else None, W_res if self.k else None,
+                          lam, stream)
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()

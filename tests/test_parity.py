@@ -328,6 +328,41 @@ def test_compensated_correction(case):
         assert err_on < 0.8 * err_off, (err_on, err_off)
 
 
+MONARCH = [
+    # name, b1, b2, k, B, T, dtype
+    ("monarch_f32", 8, 12, 8, 3, 50, "f32"),
+    ("monarch_f32_k0", 6, 6, 0, 2, 40, "f32"),
+    ("monarch_bf16", 16, 16, 32, 3, 201, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", MONARCH, ids=[c[0] for c in MONARCH])
+def test_monarch_static_part(case):
+    """A Monarch static part (DyRA App. B) under the same correction, on the
+    CUDA-core kernels, against the oracle's Monarch layer."""
+    from oracle import monarch as mon
+    name, b1, b2, k, B, T, dtype = case
+    n = b1 * b2
+    s = LayerSpec(name, n, n, 1, k, B, T, dtype, 0.7, "lognormal", seed=8)
+    w = generate(s)
+    fo = mon.offline_prepare_monarch(w.weight(), b1, b2, k, s.lam)
+    rd = lambda a: oracle.round_to(a, dtype)
+    Lb = rd(np.stack(fo.Lb))
+    Rb = rd(np.stack(fo.Rb))
+    P, W_res, X = rd(fo.P), rd(fo.W_res), rd(w.X)
+    layer = dyra.DyraMonarchLinear(n, b1, b2, k, dtype)
+    layer.load(to_dev(Lb, dtype), to_dev(Rb, dtype), to_dev(P, dtype) if k else None,
+               to_dev(W_res, dtype) if k else None, s.lam)
+    Y = layer.forward(to_dev(X, dtype), B=B, T=T)
+    assert layer.status() == 0
+    fr = mon.MonarchFactors(list(Lb), list(Rb), mon.monarch_matrix(list(Lb), list(Rb)).T, P, W_res,
+                            fo.R0)
+    Yo = mon.monarch_inference(X, fr, s.lam, B, T)
+    err = oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    layer.close()
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
