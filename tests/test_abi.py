@@ -98,3 +98,41 @@ def test_plan_create_without_gpu_fails_cleanly():
     rc, h = _create(256, 256, 32, 8, dyra.DYRA_BF16)
     assert rc in (dyra.DYRA_ERR_CUDA, dyra.DYRA_ERR_UNSUPPORTED)
     assert h.value is None
+
+
+def _declared_signatures():
+    """name -> list of parameter type strings, from include/*.h."""
+    sigs = {}
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if not f.endswith(".h"):
+            continue
+        text = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+        for m in re.finditer(r"\b(dyra_[a-z_]+)\s*\(([^;{)]*)\)\s*;", text):
+            params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+            sigs[m.group(1)] = params
+    return sigs
+
+
+def _kind(c_param):
+    """The ctypes class a C parameter declaration needs."""
+    t = re.sub(r"\b[A-Za-z_][A-Za-z_0-9]*$", "", c_param).strip()  # drop the parameter name
+    if "*" in t or t.endswith("_t") and t not in ("int64_t", "size_t", "dyra_dtype_t"):
+        return "ptr"
+    return {"int": "int", "dyra_dtype_t": "int", "int64_t": "int64", "float": "float",
+            "size_t": "size"}[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every call the binding declares has the header's parameter count and
+    kinds (pointer, int, int64, float, size), so a changed header cannot
+    silently misalign the ctypes arguments."""
+    kinds = {ctypes.c_void_p: "ptr", ctypes.c_int: "int", ctypes.c_int64: "int64",
+             ctypes.c_float: "float", ctypes.c_size_t: "size"}
+    declared = _declared_signatures()
+    for name, (_, args) in dyra.SIGNATURES.items():
+        assert name in declared, name
+        want = [_kind(p) for p in declared[name]]
+        got = ["ptr" if getattr(a, "_type_", None) is not None and a is not ctypes.c_void_p
+               and issubclass(a, ctypes._Pointer) else kinds[a] for a in args]
+        assert got == want, "%s: binding %s, header %s" % (name, got, want)
