@@ -84,6 +84,32 @@ enum {
 int dyra_plan_create(dyra_plan_t *out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype);
 
 /*
+ * A plan whose static part is a Monarch matrix ([DyRA] App. B) instead of the
+ * rank-r factorisation, for a square layer of n = b1 * b2 features (the pages
+ * define Monarch for square weights). The correction (rank k, 0 <= k <= n,
+ * k <= 128) is unchanged. In the paper's layout (Y = X W) the static product
+ * is X W_hat with W_hat = P L P^T R: y[j1*b2 + i2] = sum over m1, j2 of
+ * x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2], with P the perfect shuffle. These
+ * plans run on the CUDA-core kernels (fp32, or bf16 with bf16 intermediates);
+ * dyra_forward_batched_noalloc returns DYRA_ERR_UNSUPPORTED for them.
+ * Errors as dyra_plan_create; DYRA_ERR_INVALID_ARG also when n != b1 * b2.
+ */
+int dyra_plan_create_monarch(dyra_plan_t *out, int n, int b1, int b2, int k, dyra_dtype_t dtype);
+
+/*
+ * Load a Monarch plan's factors (the counterpart of dyra_load_factors):
+ *   Lblocks : b2 blocks of b1 x b1, row-major, one after the other (L_j2[m1][j1])
+ *   Rblocks : b1 blocks of b2 x b2, row-major, one after the other (R_j1[j2][i2])
+ *   P, W_res, lambda : as in dyra_load_factors, with W_res = W - W_hat^T in this
+ *                      library's n x n (d_out x d_in) layout
+ * Device pointers in the plan dtype, copied on `stream`. DYRA_ERR_INVALID_ARG
+ * for a plan not made by dyra_plan_create_monarch (and dyra_load_factors
+ * rejects Monarch plans).
+ */
+int dyra_load_monarch(dyra_plan_t p, const void *Lblocks, const void *Rblocks, const void *P,
+                      const void *W_res, float lambda, dyra_stream_t stream);
+
+/*
  * Copy the offline factors into the plan ([DyRA] Alg. 1, Offline Preparation
  * outputs: the structured approximation, W_res and P_L).
  *   U      : d_out x r   (singular values folded in: W_hat = U V^T)
@@ -97,6 +123,51 @@ int dyra_plan_create(dyra_plan_t *out, int d_in, int d_out, int r, int k, dyra_d
  */
 int dyra_load_factors(dyra_plan_t p, const void *U, const void *V, const void *P,
                       const void *W_res, float lambda, dyra_stream_t stream);
+
+/*
+ * The full linear layer of [DyRA] Sec. 2.4: every later forward computes
+ * Y = (X V) U^T + b + alpha * (correction), the correction being the rank-k
+ * term of Alg. 1. Before any call there is no bias and alpha = 1 (Alg. 1).
+ *   bias  : device pointer to d_out values in the plan dtype, 16-byte aligned,
+ *           copied into a plan-owned buffer on `stream` (the caller may free it
+ *           once the stream has passed this call); NULL removes the bias.
+ *   alpha : finite weight of the correction (0 leaves the static part and b).
+ * dyra_forward_weight_only adds the bias too. Errors: DYRA_ERR_INVALID_ARG (NULL
+ * plan, non-finite alpha), DYRA_ERR_ALIGNMENT, DYRA_ERR_ALLOC, DYRA_ERR_CUDA;
+ * the plan is unchanged on error.
+ */
+int dyra_set_linear(dyra_plan_t p, const void *bias, float alpha, dyra_stream_t stream);
+
+/*
+ * Number of alternating least-squares updates per forward ([DyRA] Sec. 2.2,
+ * Eq. 4-5; Sec. 3.3 compares 1, 1.5 and 2 iterations). Updates alternate L and
+ * R from Alg. 1's first pair: half_steps = 2 is Alg. 1 (t = 1), 3 adds an L
+ * update (t = 1.5: the output uses the newest L with the previous R), 4 an R
+ * update (t = 2), and so on. Each L update after the first computes
+ * L_b = X_b (R_b W_res)^T (R_b R_b^T + lambda I)^-1, so it costs one more pass
+ * over X. Default 2.
+ *   half_steps : 2 .. 64, else DYRA_ERR_INVALID_ARG.
+ * Only the CUDA-core kernels (fp32 plans, or bf16 plans under
+ * DYRA_KERNELS=simt) run more than two; the tensor-core kernels return
+ * DYRA_ERR_UNSUPPORTED, as does dyra_forward_batched_noalloc, for any other
+ * count. Takes effect at the next forward.
+ */
+int dyra_set_als_steps(dyra_plan_t p, int half_steps);
+
+/*
+ * dyra_forward_batched on HOST buffers: X (B*T x d_in) and Y (B*T x d_out) in
+ * host memory, ideally page-locked (cudaHostAlloc), since pageable memory
+ * makes the copies synchronous. Whole instances move in chunks of at least
+ * about 1 MiB of X, at most 16 chunks. On three streams the copy of chunk
+ * c + 1 to the device, the forward of chunk c (on `stream`) and the copy of
+ * chunk c - 1 back overlap; an instance's result does not depend on the
+ * chunking. The call is asynchronous like cudaMemcpyAsync: work enqueued on
+ * `stream` afterwards, and a synchronisation of `stream`, see Y complete. The
+ * plan owns the device chunk buffers (grown on demand) and the copy streams.
+ * Errors as dyra_forward_batched; X and Y must not overlap.
+ */
+int dyra_forward_batched_host(dyra_plan_t p, const void *X, void *Y, int64_t B, int64_t T,
+                              dyra_stream_t stream);
 
 /*
  * Y = DyRA(X) for one instance of N rows (B = 1, T = N).
@@ -139,7 +210,9 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
  *     returns DYRA_ERR_INVALID_ARG and enqueues nothing. For a bf16 plan they
  *     take about 2*B*T*(r+k) + 4*B*k*k + 2*B*k*(d_in+d_out) + 4*B*F bytes,
  *     each part rounded up to 256, where F = K*K + 5 with K = 32 for
- *     k <= 32, 64 for k <= 64 (F = 0 above).
+ *     k <= 32, 64 for k <= 64 (F = 0 above), plus 2*B*T*k + 2*B*k*(d_in + d_out)
+ *     when the compensated correction is on (a single instance of at most
+ *     2048 rows, or DYRA_HILO=1).
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress); make that first call before capturing a stream
  *     into a CUDA graph.

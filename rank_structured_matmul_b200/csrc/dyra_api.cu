@@ -19,6 +19,14 @@
 
 struct dyra_plan {
   int d_in = 0, d_out = 0, r = 0, k = 0;
+  // Monarch static part ([DyRA] App. B) in place of U V^T: n = d_in = d_out =
+  // b1 * b2, b2 blocks of b1 x b1 (Lblk) and b1 blocks of b2 x b2 (Rblk); r = 0
+  bool monarch = false;
+  int mb1 = 0, mb2 = 0;
+  void* Lblk = nullptr;
+  void* Rblk = nullptr;
+  void* Mtmp = nullptr;  // workspace: N x n, the product's intermediate
+  size_t cap_Mtmp = 0;
   dyra_dtype_t dtype = DYRA_BF16;
   dyra::DeviceInfo dev;
   bool loaded = false;
@@ -30,7 +38,15 @@ struct dyra_plan {
   // publishes it (DYRA_FACTOR=shared), or by size (unset: every block while
   // the blocks fit the SMs).
   int factor_mode = -1;
+  // Compensated correction (low parts of L~ and Q^T, DYRA_HILO=1|0; unset:
+  // for single instances of up to 2048 rows, where the output stage is bound
+  // by reading U and the extra correction products cost nothing)
+  int hilo_mode = -1;
   float lambda = 0.f;
+  // full linear layer (dyra_set_linear): Y = static + bias + alpha * correction
+  void* bias = nullptr;  // d_out values in the plan dtype (allocated on first use)
+  bool has_bias = false;
+  float alpha = 1.f;
   // packed factors
   void* VPt = nullptr;   // (r+k) x d_in
   void* U = nullptr;     // d_out x r
@@ -42,7 +58,18 @@ struct dyra_plan {
   void* Tp = nullptr;    // (B*k) x d_in
   void* Ct = nullptr;    // bf16: d_out x (B*k); fp32: (B*k) x d_out
   void* MD = nullptr;    // bf16, k <= 64: B factor records, then B arrival counters
+  void* Llo = nullptr;   // bf16, compensated correction: N x k
+  void* Ctlo = nullptr;  // bf16, compensated correction: d_out x (B*k)
+  void* Tplo = nullptr;  // bf16, compensated correction: (B*k) x d_in
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
+  // ALS updates per forward (dyra_set_als_steps; CUDA-core plans beyond 2) and
+  // the buffers the further L updates use
+  int als_half_steps = 2;
+  void* Lt = nullptr;    // (B*k) x T
+  void* P2 = nullptr;    // (B*k) x d_in
+  float* TG2 = nullptr;  // B x k x (T + k)
+  size_t cap_Lt = 0, cap_P2 = 0, cap_TG2 = 0;
+  size_t cap_Llo = 0, cap_Ctlo = 0, cap_Tplo = 0;
   int* status = nullptr;
   size_t factor_bytes = 0;
   cudaEvent_t stage_ev[6] = {};
@@ -64,6 +91,15 @@ struct dyra_plan {
   uint64_t graph_clock = 0;
   cudaStream_t capture_stream = nullptr;
   bool use_graphs = true;
+  // dyra_forward_batched_host: two device buffers each for the input and the
+  // output chunks, the copy streams and the per-chunk events
+  static constexpr int kHostEvents = 16;
+  void* hx[2] = {nullptr, nullptr};
+  void* hy[2] = {nullptr, nullptr};
+  size_t cap_hx[2] = {0, 0}, cap_hy[2] = {0, 0};
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev_start = nullptr;
+  cudaEvent_t ev_in[kHostEvents] = {}, ev_comp[kHostEvents] = {}, ev_out[kHostEvents] = {};
 };
 
 namespace {
@@ -130,6 +166,13 @@ struct DeviceGuard {
 
 int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
+// Whether a tensor-core forward of B x T rows uses the compensated correction.
+bool use_hilo(const dyra_plan* p, int64_t B, int64_t T) {
+  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->monarch || p->hilo_mode == 0)
+    return false;
+  return p->hilo_mode == 1 || (B == 1 && T <= 2048);
+}
+
 // Factor records of the solve plus its per-instance flags (bf16, k <= 64).
 size_t factor_bytes(int64_t B, int k) {
   const int rec = dyra::factor_record_floats(k);
@@ -147,13 +190,18 @@ void split_factor_buffer(void* buf, int64_t B, int k, float** md, int** counters
 // Grows the workspace; captured graphs point at the old buffers, so any
 // growth drops them.
 int ensure_workspace(dyra_plan* p, int64_t B, int64_t T) {
-  const size_t before = p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  const void* ptrs[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
+  auto caps = [p] {
+    return p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD + p->cap_Lt +
+           p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo + p->cap_Mtmp;
+  };
+  const size_t before = caps();
+  const void* ptrs[13] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,  p->Lt,
+                          p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo, p->Mtmp};
   const int rc = ensure_workspace_impl(p, B, T);
-  const void* now[6] = {p->Z, p->L, p->TG, p->Tp, p->Ct, p->MD};
-  bool moved =
-      before != p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD;
-  for (int i = 0; i < 6; ++i) moved = moved || ptrs[i] != now[i];
+  const void* now[13] = {p->Z,  p->L,  p->TG,  p->Tp,  p->Ct,   p->MD,  p->Lt,
+                         p->P2, p->TG2, p->Llo, p->Ctlo, p->Tplo, p->Mtmp};
+  bool moved = before != caps();
+  for (int i = 0; i < 13; ++i) moved = moved || ptrs[i] != now[i];
   if (moved) drop_graphs(p);
   return rc;
 }
@@ -163,7 +211,12 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   const size_t es = elem_size(p->dtype);
   const int k = p->k;
   int rc;
-  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+  if (p->monarch) {
+    void* mt = p->Mtmp;
+    if ((rc = grow(mt, p->cap_Mtmp, static_cast<size_t>(N) * p->d_in * es))) return rc;
+    p->Mtmp = mt;
+  }
+  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
     if (k > 0) {
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
@@ -174,6 +227,13 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
       if ((rc = grow(p->MD, p->cap_MD, factor_bytes(B, k)))) return rc;
+      if (use_hilo(p, B, T)) {
+        if ((rc = grow(p->Llo, p->cap_Llo, static_cast<size_t>(N) * k * es))) return rc;
+        if ((rc = grow(p->Ctlo, p->cap_Ctlo, static_cast<size_t>(B) * k * p->d_out * es)))
+          return rc;
+        if ((rc = grow(p->Tplo, p->cap_Tplo, static_cast<size_t>(B) * k * p->d_in * es)))
+          return rc;
+      }
     }
   } else {
     if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * (p->r + k) * es))) return rc;
@@ -184,46 +244,57 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
       if (rc) return rc;
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
       if ((rc = grow(p->Ct, p->cap_Ct, static_cast<size_t>(B) * k * p->d_out * es))) return rc;
+      if (p->als_half_steps > 2) {
+        if ((rc = grow(p->Lt, p->cap_Lt, static_cast<size_t>(B) * k * T * es))) return rc;
+        if ((rc = grow(p->P2, p->cap_P2, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
+        void* tg2 = p->TG2;
+        rc = grow(tg2, p->cap_TG2, static_cast<size_t>(B) * k * (T + k) * sizeof(float));
+        p->TG2 = static_cast<float*>(tg2);
+        if (rc) return rc;
+      }
     }
   }
   return DYRA_OK;
 }
 
-// Launch the bf16 forward, through a cached CUDA graph when possible: one
-// cudaGraphLaunch replaces five kernel launches and twelve tensor-map
-// encodings. Graphs are not used while the caller's stream is being captured
-// (the launches then go into the caller's graph), with stage timing or
-// tracing on, or when DYRA_GRAPHS=0.
-int launch_bf16_maybe_graph(dyra_plan* p, const dyra::Bf16Forward& a, cudaStream_t s) {
+// Launch a forward through a cached CUDA graph when possible: one
+// cudaGraphLaunch replaces its kernel launches (five for the tensor-core
+// path, seven for the CUDA-core path) and, for the tensor-core path, twelve
+// tensor-map encodings. Graphs are not used while the caller's stream is being
+// captured (the launches then go into the caller's graph), when `direct` is
+// set (stage timing or tracing), or when DYRA_GRAPHS=0. `launch(stream)`
+// enqueues the forward's kernels on `stream` and returns 0 on success.
+template <class Launch>
+int launch_maybe_graph(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T,
+                       bool weight_only, bool direct, cudaStream_t s, const Launch& launch) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (!p->use_graphs || a.stage_events || a.trace ||
-      cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+  if (!p->use_graphs || direct || cudaStreamIsCapturing(s, &cs) != cudaSuccess ||
+      cs != cudaStreamCaptureStatusNone) {
     cudaGetLastError();
-    return dyra::launch_bf16_forward(a, p->dev, s);
+    return launch(s);
   }
   dyra_plan::GraphEntry* hit = nullptr;
   for (auto& g : p->graphs)
-    if (g.exec && g.X == a.X && g.Y == a.Y && g.B == a.B && g.T == a.T &&
-        g.weight_only == a.weight_only)
+    if (g.exec && g.X == X && g.Y == Y && g.B == B && g.T == T && g.weight_only == weight_only)
       hit = &g;
   if (!hit) {
     if (!p->capture_stream &&
         cudaStreamCreateWithFlags(&p->capture_stream, cudaStreamNonBlocking) != cudaSuccess)
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     cudaGraph_t graph = nullptr;
     if (cudaStreamBeginCapture(p->capture_stream, cudaStreamCaptureModeThreadLocal) !=
         cudaSuccess) {
       cudaGetLastError();
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     }
-    const int lrc = dyra::launch_bf16_forward(a, p->dev, p->capture_stream);
+    const int lrc = launch(p->capture_stream);
     const cudaError_t ec = cudaStreamEndCapture(p->capture_stream, &graph);
     cudaGraphExec_t exec = nullptr;
     if (lrc != 0 || ec != cudaSuccess || graph == nullptr ||
         cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
       if (graph) cudaGraphDestroy(graph);
       cudaGetLastError();
-      return dyra::launch_bf16_forward(a, p->dev, s);
+      return launch(s);
     }
     cudaGraphDestroy(graph);
     hit = &p->graphs[0];
@@ -235,11 +306,11 @@ int launch_bf16_maybe_graph(dyra_plan* p, const dyra::Bf16Forward& a, cudaStream
       if (g.used < hit->used) hit = &g;
     }
     if (hit->exec) cudaGraphExecDestroy(hit->exec);
-    hit->X = a.X;
-    hit->Y = a.Y;
-    hit->B = a.B;
-    hit->T = a.T;
-    hit->weight_only = a.weight_only;
+    hit->X = X;
+    hit->Y = Y;
+    hit->B = B;
+    hit->T = T;
+    hit->weight_only = weight_only;
     hit->exec = exec;
   }
   hit->used = ++p->graph_clock;
@@ -265,7 +336,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
   int rc = ensure_workspace(p, B, T);
   if (rc) return rc;
 
-  if (p->dtype == DYRA_BF16 && !p->force_simt) {
+  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
     dyra::Bf16Forward a;
     a.d_in = p->d_in;
     a.d_out = p->d_out;
@@ -295,7 +366,15 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.trace = p->trace;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
-    rc = launch_bf16_maybe_graph(p, a, s);
+    a.bias = p->has_bias ? p->bias : nullptr;
+    a.alpha = p->alpha;
+    a.hilo = correct && use_hilo(p, B, T);
+    a.Llo = a.hilo ? p->Llo : nullptr;
+    a.Ctlo = a.hilo ? p->Ctlo : nullptr;
+    a.split_t = a.hilo;
+    a.Tplo = a.hilo ? p->Tplo : nullptr;
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
+                            [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
@@ -317,7 +396,21 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<__nv_bfloat16*>(p->Tp);
     a.Cm = static_cast<__nv_bfloat16*>(p->Ct);
     a.status = p->status;
-    rc = dyra::launch_simt_forward(a, p->dev, s);
+    a.bias = p->has_bias ? static_cast<const __nv_bfloat16*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
+    a.half_steps = p->als_half_steps;
+    a.Lt = static_cast<__nv_bfloat16*>(p->Lt);
+    a.P2 = static_cast<__nv_bfloat16*>(p->P2);
+    a.TG2 = p->TG2;
+    if (p->monarch) {
+      a.Lblk = static_cast<const __nv_bfloat16*>(p->Lblk);
+      a.Rblk = static_cast<const __nv_bfloat16*>(p->Rblk);
+      a.mb1 = p->mb1;
+      a.mb2 = p->mb2;
+      a.Mtmp = static_cast<__nv_bfloat16*>(p->Mtmp);
+    }
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
+                            [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   } else {
     dyra::SimtForward<float> a;
     a.d_in = p->d_in;
@@ -338,7 +431,21 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Tp = static_cast<float*>(p->Tp);
     a.Cm = static_cast<float*>(p->Ct);
     a.status = p->status;
-    rc = dyra::launch_simt_forward(a, p->dev, s);
+    a.bias = p->has_bias ? static_cast<const float*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
+    a.half_steps = p->als_half_steps;
+    a.Lt = static_cast<float*>(p->Lt);
+    a.P2 = static_cast<float*>(p->P2);
+    a.TG2 = p->TG2;
+    if (p->monarch) {
+      a.Lblk = static_cast<const float*>(p->Lblk);
+      a.Rblk = static_cast<const float*>(p->Rblk);
+      a.mb1 = p->mb1;
+      a.mb2 = p->mb2;
+      a.Mtmp = static_cast<float*>(p->Mtmp);
+    }
+    rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
+                            [&](cudaStream_t st) { return dyra::launch_simt_forward(a, p->dev, st); });
   }
   if (rc != 0) {
     cudaGetLastError();
@@ -412,6 +519,9 @@ const char* dyra_error_string(int code) {
   }
 }
 
+static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
+                            dyra_dtype_t dtype);
+
 int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_dtype_t dtype) {
   if (out == nullptr) return DYRA_ERR_INVALID_ARG;
   if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
@@ -419,6 +529,25 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   const int m = d_in < d_out ? d_in : d_out;
   if (r + k > m) return DYRA_ERR_INVALID_ARG;
   if (dtype == DYRA_BF16 && (d_in % 8 || d_out % 8 || r % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
+  return plan_create_impl(out, d_in, d_out, r, k, dtype);
+}
+
+int dyra_plan_create_monarch(dyra_plan_t* out, int n, int b1, int b2, int k, dyra_dtype_t dtype) {
+  if (out == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
+  if (b1 < 1 || b2 < 1 || n != b1 * b2 || k < 0 || k > 128 || k > n) return DYRA_ERR_INVALID_ARG;
+  if (dtype == DYRA_BF16 && (n % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
+  const int rc = plan_create_impl(out, n, n, 0, k, dtype);
+  if (rc == DYRA_OK) {
+    (*out)->monarch = true;
+    (*out)->mb1 = b1;
+    (*out)->mb2 = b2;
+  }
+  return rc;
+}
+
+static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
+                            dyra_dtype_t dtype) {
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -454,6 +583,8 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
                    : std::strcmp(fv, "self") == 0   ? 0
                    : std::strcmp(fv, "shared") == 0 ? 1
                                                     : -1;
+  const char* hv = std::getenv("DYRA_HILO");
+  p->hilo_mode = hv == nullptr ? -1 : (hv[0] == '1' ? 1 : (hv[0] == '0' ? 0 : -1));
   const char* gv = std::getenv("DYRA_GRAPHS");
   p->use_graphs = !(gv != nullptr && gv[0] == '0');
   void* st = nullptr;
@@ -473,7 +604,7 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
 
 int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P,
                       const void* W_res, float lambda, dyra_stream_t stream) {
-  if (p == nullptr || U == nullptr || V == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (p == nullptr || U == nullptr || V == nullptr || p->monarch) return DYRA_ERR_INVALID_ARG;
   if (p->k > 0 && (P == nullptr || W_res == nullptr)) return DYRA_ERR_INVALID_ARG;
   if (!(lambda >= 0.f) || !std::isfinite(lambda)) return DYRA_ERR_INVALID_ARG;
   if (!aligned16(U) || !aligned16(V) || (p->k > 0 && (!aligned16(P) || !aligned16(W_res))))
@@ -505,6 +636,147 @@ int dyra_load_factors(dyra_plan_t p, const void* U, const void* V, const void* P
   p->lambda = lambda;
   p->loaded = true;
   drop_graphs(p);  // lambda is baked into captured launches
+  return DYRA_OK;
+}
+
+int dyra_set_linear(dyra_plan_t p, const void* bias, float alpha, dyra_stream_t stream) {
+  if (p == nullptr || !std::isfinite(alpha)) return DYRA_ERR_INVALID_ARG;
+  if (bias != nullptr && !aligned16(bias)) return DYRA_ERR_ALIGNMENT;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  const size_t bytes = static_cast<size_t>(p->d_out) * elem_size(p->dtype);
+  int rc;
+  if (bias != nullptr) {
+    if (!p->bias && (rc = dev_alloc(&p->bias, bytes))) return rc;
+    if (cudaMemcpyAsync(p->bias, bias, bytes, cudaMemcpyDeviceToDevice,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+      cudaGetLastError();
+      return DYRA_ERR_CUDA;
+    }
+  }
+  p->has_bias = bias != nullptr;
+  p->alpha = alpha;
+  drop_graphs(p);  // the bias pointer and alpha are baked into captured launches
+  return DYRA_OK;
+}
+
+int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
+  if (p == nullptr || half_steps < 2 || half_steps > 64) return DYRA_ERR_INVALID_ARG;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
+  if (umma && half_steps != 2) return DYRA_ERR_UNSUPPORTED;
+  p->als_half_steps = half_steps;
+  drop_graphs(p);  // captured forwards hold the old count
+  return DYRA_OK;
+}
+
+int dyra_forward_batched_host(dyra_plan_t p, const void* X, void* Y, int64_t B, int64_t T,
+                              dyra_stream_t stream) {
+  if (p == nullptr || B < 0 || T < 0) return DYRA_ERR_INVALID_ARG;
+  if (B * T == 0) return DYRA_OK;
+  if (X == nullptr || Y == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(p->dtype);
+  // Chunks of whole instances (each instance's correction needs all of its
+  // rows): up to kHostEvents of them, at least about 1 MiB of input each.
+  const size_t inst_in = static_cast<size_t>(T) * p->d_in * es;
+  const size_t inst_out = static_cast<size_t>(T) * p->d_out * es;
+  int64_t per = std::max<int64_t>(1, (B + dyra_plan::kHostEvents - 1) / dyra_plan::kHostEvents);
+  per = std::max<int64_t>(per, std::min<int64_t>(B, static_cast<int64_t>((1u << 20) / inst_in) + 1));
+  const int64_t chunks = (B + per - 1) / per;
+  int rc;
+  for (int i = 0; i < 2; ++i) {
+    if ((rc = grow(p->hx[i], p->cap_hx[i], per * inst_in))) return rc;
+    if ((rc = grow(p->hy[i], p->cap_hy[i], per * inst_out))) return rc;
+  }
+  auto make_stream = [](cudaStream_t* st) {
+    return *st || cudaStreamCreateWithFlags(st, cudaStreamNonBlocking) == cudaSuccess;
+  };
+  auto make_event = [](cudaEvent_t* e) {
+    return *e || cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  };
+  bool ok = make_stream(&p->h2d) && make_stream(&p->d2h) && make_event(&p->ev_start);
+  for (int i = 0; ok && i < dyra_plan::kHostEvents; ++i)
+    ok = make_event(&p->ev_in[i]) && make_event(&p->ev_comp[i]) && make_event(&p->ev_out[i]);
+  if (!ok) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  // chunk c: X -> hx[c % 2] on h2d, the forward on `stream`, hy[c % 2] -> Y on d2h.
+  // hx[c % 2] is rewritten once the forward of chunk c - 2 has read it, hy[c % 2]
+  // once the copy of chunk c - 2 has read it; `stream` then waits for the last copy.
+  const char* xs = static_cast<const char*>(X);
+  char* ys = static_cast<char*>(Y);
+  bool err = cudaEventRecord(p->ev_start, s) != cudaSuccess ||
+             cudaStreamWaitEvent(p->h2d, p->ev_start, 0) != cudaSuccess;
+  for (int64_t c = 0; !err && c < chunks; ++c) {
+    const int64_t b0 = c * per, bc = std::min<int64_t>(per, B - b0);
+    const int buf = static_cast<int>(c % 2);
+    const int e = static_cast<int>(c % dyra_plan::kHostEvents);
+    const int e2 = static_cast<int>((c + dyra_plan::kHostEvents - 2) % dyra_plan::kHostEvents);
+    if (c >= 2) err = cudaStreamWaitEvent(p->h2d, p->ev_comp[e2], 0) != cudaSuccess;
+    err = err || cudaMemcpyAsync(p->hx[buf], xs + b0 * inst_in, bc * inst_in,
+                                 cudaMemcpyHostToDevice, p->h2d) != cudaSuccess;
+    err = err || cudaEventRecord(p->ev_in[e], p->h2d) != cudaSuccess;
+    err = err || cudaStreamWaitEvent(s, p->ev_in[e], 0) != cudaSuccess;
+    if (c >= 2) err = err || cudaStreamWaitEvent(s, p->ev_out[e2], 0) != cudaSuccess;
+    if (err) break;
+    rc = run_forward(p, p->hx[buf], p->hy[buf], bc, T, false, s);
+    if (rc) return rc;
+    err = cudaEventRecord(p->ev_comp[e], s) != cudaSuccess ||
+          cudaStreamWaitEvent(p->d2h, p->ev_comp[e], 0) != cudaSuccess ||
+          cudaMemcpyAsync(ys + b0 * inst_out, p->hy[buf], bc * inst_out, cudaMemcpyDeviceToHost,
+                          p->d2h) != cudaSuccess ||
+          cudaEventRecord(p->ev_out[e], p->d2h) != cudaSuccess;
+    if (!err && c == chunks - 1) err = cudaStreamWaitEvent(s, p->ev_out[e], 0) != cudaSuccess;
+  }
+  if (err) {
+    cudaGetLastError();
+    return DYRA_ERR_CUDA;
+  }
+  return DYRA_OK;
+}
+
+int dyra_load_monarch(dyra_plan_t p, const void* Lblocks, const void* Rblocks, const void* P,
+                      const void* W_res, float lambda, dyra_stream_t stream) {
+  if (p == nullptr || !p->monarch || Lblocks == nullptr || Rblocks == nullptr)
+    return DYRA_ERR_INVALID_ARG;
+  if (p->k > 0 && (P == nullptr || W_res == nullptr)) return DYRA_ERR_INVALID_ARG;
+  if (!(lambda >= 0.f) || !std::isfinite(lambda)) return DYRA_ERR_INVALID_ARG;
+  DeviceGuard g(p->dev.device);
+  if (!g.ok) return DYRA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(p->dtype);
+  const size_t n = static_cast<size_t>(p->d_in);
+  const size_t lb = static_cast<size_t>(p->mb2) * p->mb1 * p->mb1 * es;
+  const size_t rb = static_cast<size_t>(p->mb1) * p->mb2 * p->mb2 * es;
+  const size_t vpt = static_cast<size_t>(p->k) * n * es;
+  const size_t wb = p->k > 0 ? n * n * es : 0;
+  int rc;
+  if (!p->Lblk && (rc = dev_alloc(&p->Lblk, lb))) return rc;
+  if (!p->Rblk && (rc = dev_alloc(&p->Rblk, rb))) return rc;
+  if (vpt && !p->VPt && (rc = dev_alloc(&p->VPt, vpt))) return rc;
+  if (wb && !p->W_res && (rc = dev_alloc(&p->W_res, wb))) return rc;
+  p->factor_bytes = lb + rb + vpt + wb;
+  if (cudaMemcpyAsync(p->Lblk, Lblocks, lb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(p->Rblk, Rblocks, rb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      (wb && cudaMemcpyAsync(p->W_res, W_res, wb, cudaMemcpyDeviceToDevice, s) != cudaSuccess))
+    return DYRA_ERR_CUDA;
+  if (vpt) {  // P^T (k x n): the projection's B operand, as [V | P]^T with r = 0
+    if (p->dtype == DYRA_BF16)
+      rc = dyra::launch_pack_vp(static_cast<const __nv_bfloat16*>(P),
+                                static_cast<const __nv_bfloat16*>(P),
+                                static_cast<__nv_bfloat16*>(p->VPt), p->d_in, 0, p->k, s);
+    else
+      rc = dyra::launch_pack_vp(static_cast<const float*>(P), static_cast<const float*>(P),
+                                static_cast<float*>(p->VPt), p->d_in, 0, p->k, s);
+    if (rc) return DYRA_ERR_CUDA;
+  }
+  p->lambda = lambda;
+  p->loaded = true;
+  drop_graphs(p);
   return DYRA_OK;
 }
 
@@ -550,6 +822,10 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->VPt);
     dev_free(p->U);
     dev_free(p->W_res);
+    dev_free(p->bias);
+    dev_free(p->Lblk);
+    dev_free(p->Rblk);
+    dev_free(p->Mtmp);
     dev_free(p->Z);
     dev_free(p->L);
     void* tg = p->TG;
@@ -557,6 +833,13 @@ int dyra_plan_destroy(dyra_plan_t p) {
     dev_free(p->Tp);
     dev_free(p->Ct);
     dev_free(p->MD);
+    dev_free(p->Lt);
+    dev_free(p->P2);
+    void* tg2 = p->TG2;
+    dev_free(tg2);
+    dev_free(p->Llo);
+    dev_free(p->Ctlo);
+    dev_free(p->Tplo);
     void* st = p->status;
     dev_free(st);
     for (auto& e : p->stage_ev)
@@ -564,6 +847,18 @@ int dyra_plan_destroy(dyra_plan_t p) {
     if (p->trace) cudaFree(p->trace);
     drop_graphs(p);
     if (p->capture_stream) cudaStreamDestroy(p->capture_stream);
+    for (int i = 0; i < 2; ++i) {
+      dev_free(p->hx[i]);
+      dev_free(p->hy[i]);
+    }
+    if (p->h2d) cudaStreamDestroy(p->h2d);
+    if (p->d2h) cudaStreamDestroy(p->d2h);
+    if (p->ev_start) cudaEventDestroy(p->ev_start);
+    for (int i = 0; i < dyra_plan::kHostEvents; ++i) {
+      if (p->ev_in[i]) cudaEventDestroy(p->ev_in[i]);
+      if (p->ev_comp[i]) cudaEventDestroy(p->ev_comp[i]);
+      if (p->ev_out[i]) cudaEventDestroy(p->ev_out[i]);
+    }
   }
   delete p;
   return DYRA_OK;
@@ -603,7 +898,7 @@ int dyra_debug_set_stage_timing(dyra_plan_t p, int enable) {
     for (auto& e : p->stage_ev)
       if (cudaEventCreate(&e) != cudaSuccess) return DYRA_ERR_CUDA;
   }
-  p->stage_timing = enable != 0 && p->dtype == DYRA_BF16 && !p->force_simt;
+  p->stage_timing = enable != 0 && p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
   p->stage_recorded = false;
   return p->stage_timing || !enable ? DYRA_OK : DYRA_ERR_INVALID_ARG;
 }
@@ -673,7 +968,9 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int* splits, int*
 size_t dyra_plan_device_bytes(dyra_plan_t p) {
   if (p == nullptr) return 0;
   return p->factor_bytes + p->cap_Z + p->cap_L + p->cap_TG + p->cap_Tp + p->cap_Ct + p->cap_MD +
-         256;
+         p->cap_Lt + p->cap_P2 + p->cap_TG2 + p->cap_Llo + p->cap_Ctlo + p->cap_Tplo +
+         p->cap_Mtmp + 256 +
+         (p->bias ? static_cast<size_t>(p->d_out) * elem_size(p->dtype) : 0);
 }
 
 }  // extern "C"
@@ -733,9 +1030,11 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
   if (N > (static_cast<int64_t>(1) << 31) - 1 || B * static_cast<int64_t>(p->k) > (1 << 30))
     return DYRA_ERR_INVALID_ARG;
   if (!p->loaded) return DYRA_ERR_NOT_LOADED;
+  if (p->monarch) return DYRA_ERR_UNSUPPORTED;
   if (!aligned16(X) || !aligned16(Y)) return DYRA_ERR_ALIGNMENT;
   const int k = p->k;
   if (k > 0 && p->lambda == 0.f && T < k) return DYRA_ERR_RANK_DEFICIENT;
+  if (k > 0 && p->als_half_steps != 2) return DYRA_ERR_UNSUPPORTED;
 
   const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
   const size_t es = elem_size(p->dtype);
@@ -752,6 +1051,11 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
       sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
       sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
       sizing.take(factor_bytes(B, k));
+      if (use_hilo(p, B, T)) {
+        sizing.take(static_cast<size_t>(N) * k * es);
+        sizing.take(static_cast<size_t>(B) * k * p->d_out * es);
+        sizing.take(static_cast<size_t>(B) * k * p->d_in * es);
+      }
     }
   } else {
     sizing.take(static_cast<size_t>(N) * (p->r + k) * es);
@@ -794,6 +1098,11 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Ct = k > 0 ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
     void* fac = k > 0 ? carve.take(factor_bytes(B, k)) : nullptr;
     split_factor_buffer(fac, B, k, &a.MD, &a.counters);
+    a.hilo = k > 0 && use_hilo(p, B, T);
+    a.Llo = a.hilo ? carve.take(static_cast<size_t>(N) * k * es) : nullptr;
+    a.Ctlo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_out * es) : nullptr;
+    a.split_t = a.hilo;
+    a.Tplo = a.hilo ? carve.take(static_cast<size_t>(B) * k * p->d_in * es) : nullptr;
     a.factor_mode = p->factor_mode;
     a.splits = splits;
     a.split_rows = split_rows;
@@ -802,6 +1111,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.trace = nullptr;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.bias = p->has_bias ? p->bias : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;
@@ -827,6 +1138,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Cm = k > 0 ? static_cast<__nv_bfloat16*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
                  : nullptr;
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const __nv_bfloat16*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_simt_forward(a, p->dev, s);
   } else {
     dyra::SimtForward<float> a;
@@ -852,6 +1165,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.Cm = k > 0 ? static_cast<float*>(carve.take(static_cast<size_t>(B) * k * p->d_out * es))
                  : nullptr;
     a.status = p->status;
+    a.bias = p->has_bias ? static_cast<const float*>(p->bias) : nullptr;
+    a.alpha = p->alpha;
     rc = dyra::launch_simt_forward(a, p->dev, s);
   }
   if (rc != 0) {

@@ -3,9 +3,30 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 namespace dyra {
+
+// Launch set-up of one kernel, per device: cudaFuncSetAttribute acts on the
+// current device only, so each device of a process is configured on its own
+// (plans on several devices may share the process and run from several host
+// threads; setting an attribute twice is harmless).
+constexpr int kMaxDevices = 64;
+struct KernelSetup {
+  std::atomic<uint32_t> smem[kMaxDevices];  // dynamic shared memory configured so far
+  std::atomic<int> occupancy[kMaxDevices];  // cached occupancy figure (e.g. resident pairs)
+};
+
+// The current device, or -1 if it cannot be read or is beyond kMaxDevices.
+inline int setup_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return d < kMaxDevices ? d : -1;
+}
 
 struct DeviceInfo {
   int device = 0;
@@ -52,6 +73,19 @@ struct Bf16Forward {
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
   bool use_pairs;             // run the output stage on CTA pairs
   int proj_pair_min_tiles;    // see proj_shape (0: default)
+  const void* bias = nullptr;  // d_out bf16 values added to Y, or nullptr
+  float alpha = 1.f;           // weight of the correction (the solve scales L~ by it)
+  // Compensated correction: L~ and Q^T are also stored as their bf16 rounding
+  // errors (Llo, Ctlo) and the output stage adds hi.hi + hi.lo + lo.hi, which
+  // removes most of the cancellation error the grouping L~ . Q amplifies.
+  bool hilo = false;
+  void* Llo = nullptr;   // N x k
+  void* Ctlo = nullptr;  // d_out x (B*k)
+  // Split T: T = L^T X also as its bf16 rounding errors (Tplo), which the
+  // rank-k factor GEMM accumulates as a second B operand, so Q is formed from
+  // T to about 16 bits
+  bool split_t = false;
+  void* Tplo = nullptr;  // (B*k) x d_in
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -94,6 +128,22 @@ struct SimtForward {
   T* Tp;        // (B*k) x d_in
   T* Cm;        // (B*k) x d_out
   int* status;
+  const T* bias = nullptr;  // d_out values added to Y, or nullptr
+  float alpha = 1.f;        // weight of the correction
+  // More alternating least-squares updates ([DyRA] Sec. 3.3): half_steps
+  // updates in all, L and R alternating, Alg. 1 being the first two. Beyond
+  // two, each L update needs the buffers below.
+  int half_steps = 2;
+  T* Lt = nullptr;       // (B*k) x Trows: the latest L_b, transposed
+  T* P2 = nullptr;       // (B*k) x d_in: R_b W_res, the L update's projector before its solve
+  float* TG2 = nullptr;  // B x k x (Trows + k): [ (X_b P2_b^T)^T | R_b R_b^T ]
+  // Monarch static part ([DyRA] App. B), r = 0: y = x W_hat in the paper's
+  // layout, W_hat = P L P^T R with Lblk b2 blocks of mb1 x mb1 and Rblk mb1
+  // blocks of mb2 x mb2 (row-major, contiguous); Mtmp is N x n
+  const T* Lblk = nullptr;
+  const T* Rblk = nullptr;
+  int mb1 = 0, mb2 = 0;
+  T* Mtmp = nullptr;
 };
 
 template <typename T>
@@ -115,9 +165,11 @@ int factor_record_floats(int k);
 // defer_wait (with pdl): the grid launched just before waited for the one
 // that wrote G and L before letting this one start; this grid then waits
 // for it only before its blocks exit.
-int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
-                  unsigned long long* trace);
+// alpha scales the result (the correction weight of the full linear layer);
+// Llo (optional, N x k like L) receives the bf16 rounding error of each value.
+int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
+                  int64_t T, int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+                  bool defer_wait, unsigned long long* trace);
 // Dynamic shared memory of one launch_ltilde block, and its rows of L, for this k.
 size_t ltilde_smem_bytes(int k);
 int ltilde_rows_per_block(int k);

@@ -368,8 +368,9 @@ static_assert(offsetof(LdlBlockScratch<32>, Wb) % 16 == 0 &&
 // = 16384 (the GEMM's warps take up to 104 registers).
 template <int KMAX, int MODE>
 __global__ void __maxnreg__(152)
-    ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, float* MD, int* flags, int T,
-                  int k, float lambda, int* status, int defer_wait, unsigned long long* trace) {
+    ltilde_kernel(const float* __restrict__ G, __nv_bfloat16* L, __nv_bfloat16* Llo, float* MD,
+                  int* flags, int T, int k, float lambda, float alpha, int* status, int defer_wait,
+                  unsigned long long* trace) {
   using Sm = LtSmem<KMAX>;
   constexpr int LD = LdlBlockScratch<KMAX>::LD;
   constexpr int ROWS = lt_rows<KMAX>();
@@ -550,14 +551,26 @@ __global__ void __maxnreg__(152)
       const int rl = p0 + RT * rg + rr;
       if (rl >= nrows || 4 * cg >= k) continue;
       __nv_bfloat16* dst = rows + static_cast<size_t>(rl) * k + 4 * cg;
-      const __nv_bfloat162 lo =
-          __floats2bfloat162_rn(zero ? 0.f : acc[rr][0], zero ? 0.f : acc[rr][1]);
-      const __nv_bfloat162 hi =
-          __floats2bfloat162_rn(zero ? 0.f : acc[rr][2], zero ? 0.f : acc[rr][3]);
+      // a failed factorisation writes zeros (not alpha times a non-finite value)
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][0],
+                                                      zero ? 0.f : alpha * acc[rr][1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][2],
+                                                      zero ? 0.f : alpha * acc[rr][3]);
       uint2 w;
       w.x = *reinterpret_cast<const uint32_t*>(&lo);
       w.y = *reinterpret_cast<const uint32_t*>(&hi);
       *reinterpret_cast<uint2*>(dst) = w;
+      if (Llo != nullptr) {  // the rounding errors of the four values just stored
+        const float2 l2 = __bfloat1622float2(lo), h2 = __bfloat1622float2(hi);
+        const __nv_bfloat162 elo = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][0] - l2.x,
+                                                         zero ? 0.f : alpha * acc[rr][1] - l2.y);
+        const __nv_bfloat162 ehi = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][2] - h2.x,
+                                                         zero ? 0.f : alpha * acc[rr][3] - h2.y);
+        uint2 we;
+        we.x = *reinterpret_cast<const uint32_t*>(&elo);
+        we.y = *reinterpret_cast<const uint32_t*>(&ehi);
+        *reinterpret_cast<uint2*>(Llo + (dst - L)) = we;
+      }
     }
   }
   if (tr && tid == 0) tr[5] = sm100::globaltimer_ns();
@@ -570,8 +583,8 @@ __global__ void __maxnreg__(152)
 // (Cholesky G_b = R R^T in shared memory) and solves R R^T w = l for 128 rows
 // of L_b, one per thread.
 __global__ void __launch_bounds__(kSolveThreads)
-    ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, int T, int k,
-                          float lambda, int* status, int defer_wait) {
+    ltilde_general_kernel(const float* __restrict__ G, __nv_bfloat16* L, __nv_bfloat16* Llo, int T,
+                          int k, float lambda, float alpha, int* status, int defer_wait) {
   extern __shared__ float sm[];
   const int ldg = k + 1;
   float* R = sm;                // k x (k+1): lower triangle becomes R
@@ -624,21 +637,27 @@ __global__ void __launch_bounds__(kSolveThreads)
       Ycol[i * kSolveThreads + tid] = acc / R[i * ldg + i];
     }
     const bool zero = bad != 0;
-    for (int i = 0; i < k; ++i)
-      row[i] = __float2bfloat16_rn(zero ? 0.f : Ycol[i * kSolveThreads + tid]);
+    for (int i = 0; i < k; ++i) {
+      const float v = zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid];
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      row[i] = h;
+      if (Llo != nullptr) Llo[(row - L) + i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   if (defer_wait) sm100::pdl_wait();
 }
 
-// C[b][m][n] (+)= sum_q A[b][m][q] * Bm[b][q][n] with arbitrary element strides.
+// C[b][m][n] (+)= alpha sum_q A[b][m][q] * Bm[b][q][n] (+ bias[n]) with
+// arbitrary element strides.
 constexpr int kGT = 64;   // tile
 constexpr int kGK = 16;   // k step
 template <typename TA, typename TB, typename TC>
 __global__ void __launch_bounds__(256)
     simt_gemm_kernel(int M, int N, int K, const TA* __restrict__ A, int64_t am, int64_t ak,
                      int64_t ab, const TB* __restrict__ Bm, int64_t bk, int64_t bn, int64_t bb,
-                     TC* __restrict__ C, int64_t cm, int64_t cn, int64_t cb, int accumulate) {
+                     TC* __restrict__ C, int64_t cm, int64_t cn, int64_t cb, int accumulate,
+                     float alpha, const TC* __restrict__ bias, int64_t bias_b) {
   __shared__ float As[kGK][kGT + 1];
   __shared__ float Bs[kGK][kGT + 1];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -680,7 +699,8 @@ __global__ void __launch_bounds__(256)
       const int gn = n0 + tx + 16 * j;
       if (gn >= N) continue;
       TC* dst = C + gm * cm + gn * cn;
-      float v = acc[i][j];
+      float v = alpha * acc[i][j];
+      if (bias) v += to_f<TC>(bias[batch * bias_b + gn]);
       if (accumulate) v += to_f<TC>(*dst);
       *dst = from_f<TC>(v);
     }
@@ -690,11 +710,12 @@ __global__ void __launch_bounds__(256)
 template <typename TA, typename TB, typename TC>
 int gemm(int M, int N, int K, const TA* A, int64_t am, int64_t ak, int64_t ab, const TB* Bm,
          int64_t bk, int64_t bn, int64_t bb, TC* C, int64_t cm, int64_t cn, int64_t cb,
-         int batches, int accumulate, cudaStream_t s) {
+         int batches, int accumulate, cudaStream_t s, float alpha = 1.f,
+         const TC* bias = nullptr, int64_t bias_b = 0) {
   if (M <= 0 || N <= 0 || batches <= 0) return 0;
   dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, batches);
   simt_gemm_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb, C,
-                                                    cm, cn, cb, accumulate);
+                                                    cm, cn, cb, accumulate, alpha, bias, bias_b);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -716,14 +737,16 @@ template <typename TOut, int KMAX>
 int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, int splits, int64_t B, int k,
                      int d_in, float lambda, TOut* Tp, int* status, unsigned long long* trace) {
   auto kfn = solve_ldl_kernel<TOut, KMAX>;
-  static bool configured = false;
-  if (!configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (setup.smem[d].load() == 0) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(SolveSmem<KMAX>))) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = true;
+    setup.smem[d].store(static_cast<uint32_t>(sizeof(SolveSmem<KMAX>)));
   }
   cfg.gridDim = dim3(static_cast<unsigned>(B),
                      static_cast<unsigned>((d_in + kSolveCols - 1) / kSolveCols));
@@ -753,12 +776,14 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
-  static size_t configured = 48 * 1024;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (smem > 48 * 1024 && smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(static_cast<uint32_t>(smem));
   }
   cfg.gridDim = dim3(static_cast<unsigned>(B), static_cast<unsigned>((d_in + kSolveThreads - 1) / kSolveThreads));
   cfg.blockDim = dim3(kSolveThreads);
@@ -781,18 +806,21 @@ size_t ltilde_smem_bytes(int k) {
 }
 
 template <int KMAX, int MODE>
-int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L, float* MD,
-                       int* flags, int64_t B, int64_t T, int k, float lambda, int* status,
-                       int defer_wait, unsigned long long* trace) {
+int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L,
+                       __nv_bfloat16* Llo, float* MD, int* flags, int64_t B, int64_t T, int k,
+                       float lambda, float alpha, int* status, int defer_wait,
+                       unsigned long long* trace) {
   auto kfn = ltilde_kernel<KMAX, MODE>;
-  static bool configured = false;
-  if (!configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (setup.smem[d].load() == 0) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(sizeof(LtSmem<KMAX>))) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = true;
+    setup.smem[d].store(static_cast<uint32_t>(sizeof(LtSmem<KMAX>)));
   }
   // blockIdx.x = instance, blockIdx.y = chunk of rows: the chunk-0 CTAs (the
   // factoring ones in the shared mode) are the grid's first B CTAs.
@@ -800,15 +828,15 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
                      static_cast<unsigned>((T + lt_rows<KMAX>() - 1) / lt_rows<KMAX>()));
   cfg.blockDim = dim3(kLtThreads);
   cfg.dynamicSmemBytes = sizeof(LtSmem<KMAX>);
-  return cudaLaunchKernelEx(&cfg, kfn, G, L, MD, flags, static_cast<int>(T), k, lambda, status,
-                            defer_wait, trace) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, kfn, G, L, Llo, MD, flags, static_cast<int>(T), k, lambda, alpha,
+                            status, defer_wait, trace) == cudaSuccess
              ? 0
              : -1;
 }
 
-int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int64_t B, int64_t T,
-                  int k, float lambda, int* status, cudaStream_t s, bool pdl, bool defer_wait,
-                  unsigned long long* trace) {
+int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
+                  int64_t T, int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
+                  bool defer_wait, unsigned long long* trace) {
   const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
   if (k % 8 != 0) return -1;  // bf16 plans: 16-byte rows of L
@@ -816,6 +844,7 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
     return -1;
   auto* Lb = static_cast<__nv_bfloat16*>(L);
+  auto* Lo = static_cast<__nv_bfloat16*>(Llo);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -825,31 +854,33 @@ int launch_ltilde(const float* G, void* L, float* MD, int* flags, int mode, int6
   cfg.stream = s;
   if (k <= 32)
     return mode == kSolveShared
-               ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, dw, trace)
-               : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, dw, trace);
+               ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                      alpha, status, dw, trace)
+               : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                    alpha, status, dw, trace);
   if (k <= 64)
     return mode == kSolveShared
-               ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                      status, dw, trace)
-               : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, MD, flags, B, T, k, lambda,
-                                                    status, dw, trace);
+               ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                      alpha, status, dw, trace)
+               : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                    alpha, status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
-  static size_t configured = 48 * 1024;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (smem > 48 * 1024 && smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(ltilde_general_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(static_cast<uint32_t>(smem));
   }
   if ((T + kSolveThreads - 1) / kSolveThreads > 65535) return -1;
   cfg.gridDim = dim3(static_cast<unsigned>(B),
                      static_cast<unsigned>((T + kSolveThreads - 1) / kSolveThreads));
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
-  return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, static_cast<int>(T), k, lambda,
-                            status, dw) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, ltilde_general_kernel, G, Lb, Lo, static_cast<int>(T), k, lambda,
+                            alpha, status, dw) == cudaSuccess
              ? 0
              : -1;
 }
@@ -873,7 +904,14 @@ template int launch_pack_vp<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bflo
                                            __nv_bfloat16*, int, int, int, cudaStream_t);
 
 // The fp32 forward: the same steps as the tensor-core path, each as a
-// strided batched SIMT GEMM, with fp32 storage of every intermediate.
+// strided batched SIMT GEMM, with fp32 storage of every intermediate. With
+// more than two half-steps, further L and R updates follow Alg. 1's pair
+// ([DyRA] Sec. 2.2, Eq. 4-5 with the ridge of footnote 2; Sec. 3.3):
+//   L update  L_b = X_b (R_b W_res)^T (R_b R_b^T + lambda I)^-1
+//   R update  R_b = (L_b^T L_b + lambda I)^-1 (L_b^T X_b) W_res^T
+// and the output takes the last pair. Both updates go through the same ridge
+// solve: the R update solves for R_b from [L_b^T X_b | L_b^T L_b], the L
+// update for L_b^T from [(X_b (R_b W_res)^T)^T | R_b R_b^T].
 template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t s) {
   const int64_t N = a.B * a.Trows;
@@ -882,37 +920,75 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
   const int k = a.weight_only ? 0 : a.k;
   const int Bn = static_cast<int>(a.B);
   const int Tr = static_cast<int>(a.Trows);
+  const int steps = k > 0 ? a.half_steps : 0;
+  if (k > 0 && (steps < 2 || (steps > 2 && (!a.Lt || !a.P2 || !a.TG2)))) return -1;
   // [Z | L] = X [V | P]
   if (gemm(static_cast<int>(N), rk, a.d_in, a.X, a.d_in, 1, 0, a.VPt, 1, a.d_in, 0, a.ZL, rk, 1,
            0, 1, 0, s))
     return -1;
-  if (k > 0) {
-    const int J = a.d_in + k;
-    // T_b = L_b^T X_b  -> TG[b][i][j], j < d_in
-    if (gemm(k, a.d_in, Tr, a.ZL + a.r, 1, rk, static_cast<int64_t>(Tr) * rk, a.X, a.d_in, 1,
-             static_cast<int64_t>(Tr) * a.d_in, a.TG, J, 1, static_cast<int64_t>(k) * J, Bn, 0, s))
-      return -1;
-    // G_b = L_b^T L_b -> TG[b][i][d_in + i']
-    if (gemm(k, k, Tr, a.ZL + a.r, 1, rk, static_cast<int64_t>(Tr) * rk, a.ZL + a.r, rk, 1,
-             static_cast<int64_t>(Tr) * rk, a.TG + a.d_in, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
-             s))
-      return -1;
-    if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
-      return -1;
-    // C = T' W_res^T  (B*k x d_out)
-    if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out, 1,
-             0, 1, 0, s))
-      return -1;
+  // the current L_b: element (t, i) at Lp[b * lb + t * lm + i * lq]
+  const T* Lp = a.ZL + a.r;
+  int64_t lm = rk, lq = 1, lb = static_cast<int64_t>(Tr) * rk;
+  for (int h = 1; h < steps; ++h) {
+    if (h % 2 == 1) {  // R update from the current L
+      const int J = a.d_in + k;
+      // T_b = L_b^T X_b  -> TG[b][i][j], j < d_in
+      if (gemm(k, a.d_in, Tr, Lp, lq, lm, lb, a.X, a.d_in, 1, static_cast<int64_t>(Tr) * a.d_in,
+               a.TG, J, 1, static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      // G_b = L_b^T L_b -> TG[b][i][d_in + i']
+      if (gemm(k, k, Tr, Lp, lq, lm, lb, Lp, lm, lq, lb, a.TG + a.d_in, J, 1,
+               static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+        return -1;
+      // R = T' W_res^T  (B*k x d_out)
+      if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out,
+               1, 0, 1, 0, s))
+        return -1;
+    } else {  // L update from the current R (in Cm)
+      const int J = Tr + k;
+      // P2 = R W_res  (B*k x d_in)
+      if (gemm(Bn * k, a.d_in, a.d_out, a.Cm, a.d_out, 1, 0, a.W_res, a.d_in, 1, 0, a.P2, a.d_in,
+               1, 0, 1, 0, s))
+        return -1;
+      // (X_b P2_b^T)^T -> TG2[b][i][t], t < Tr
+      if (gemm(k, Tr, a.d_in, a.P2, a.d_in, 1, static_cast<int64_t>(k) * a.d_in, a.X, 1, a.d_in,
+               static_cast<int64_t>(Tr) * a.d_in, a.TG2, J, 1, static_cast<int64_t>(k) * J, Bn, 0,
+               s))
+        return -1;
+      // R_b R_b^T -> TG2[b][i][Tr + i']
+      if (gemm(k, k, a.d_out, a.Cm, a.d_out, 1, static_cast<int64_t>(k) * a.d_out, a.Cm, 1,
+               a.d_out, static_cast<int64_t>(k) * a.d_out, a.TG2 + Tr, J, 1,
+               static_cast<int64_t>(k) * J, Bn, 0, s))
+        return -1;
+      // L_b^T = (R_b R_b^T + lambda I)^-1 (X_b P2_b^T)^T  -> Lt[b*k + i][t]
+      if (launch_solve<T>(a.TG2, 1, a.B, k, Tr, a.lambda, a.Lt, a.status, s, false, nullptr))
+        return -1;
+      Lp = a.Lt;
+      lm = 1;
+      lq = Tr;
+      lb = static_cast<int64_t>(k) * Tr;
+    }
   }
-  // Y = Z U^T
-  if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out, 1, 0,
-           1, 0, s))
+  if (a.Lblk != nullptr) {
+    // Monarch static part: y[j1*b2 + i2] = sum_{m1, j2} x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2],
+    // as two strided batched products through Mtmp[row][j2*b1 + j1]
+    const int n = a.d_in, b1 = a.mb1, b2 = a.mb2;
+    if (gemm(static_cast<int>(N), b1, b1, a.X, n, b2, 1, a.Lblk, b1, 1,
+             static_cast<int64_t>(b1) * b1, a.Mtmp, n, 1, b1, b2, 0, s))
+      return -1;
+    if (gemm(static_cast<int>(N), b2, b2, a.Mtmp, n, b1, 1, a.Rblk, b2, 1,
+             static_cast<int64_t>(b2) * b2, a.Y, n, 1, b2, b1, 0, s, 1.f, a.bias, b2))
+      return -1;
+  } else if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out,
+                  1, 0, 1, 0, s, 1.f, a.bias)) {  // Y = Z U^T (+ b)
     return -1;
+  }
   if (k > 0) {
-    // Y_b += L_b C_b
-    if (gemm(Tr, a.d_out, k, a.ZL + a.r, rk, 1, static_cast<int64_t>(Tr) * rk, a.Cm, a.d_out, 1,
-             static_cast<int64_t>(k) * a.d_out, a.Y, a.d_out, 1, static_cast<int64_t>(Tr) * a.d_out,
-             Bn, 1, s))
+    // Y_b += alpha L_b R_b (the last pair)
+    if (gemm(Tr, a.d_out, k, Lp, lm, lq, lb, a.Cm, a.d_out, 1, static_cast<int64_t>(k) * a.d_out,
+             a.Y, a.d_out, 1, static_cast<int64_t>(Tr) * a.d_out, Bn, 1, s, a.alpha))
       return -1;
   }
   return 0;

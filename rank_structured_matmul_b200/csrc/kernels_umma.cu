@@ -56,12 +56,19 @@ __device__ __forceinline__ int ceil_div_dev(int a, int b) { return (a + b - 1) /
 // col0 .. col0+63 of this thread's row) as bf16 through a 128-byte-swizzled
 // shared-memory box and a TMA store at (x, y) of `tmap`. Two boxes rotate: a
 // box is rewritten only after the store issued two boxes earlier has read it.
-// All 128 epilogue threads call it; thread 0 issues the stores.
+// All 128 epilogue threads call it; thread 0 issues the stores. With `bias`
+// (ncols entries, ncols a multiple of 8) bias[x + j] is added to column j of
+// the box in fp32 before the rounding; columns at or beyond ncols read none.
 constexpr uint32_t kStoreBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kStoreBoxes = 2;
 
+// With LO set, the box receives the low part of each value instead,
+// bf16(v - bf16(v)): the two boxes together carry v to about 16 bits.
+template <bool LO = false>
 __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const void* tmap, int x,
-                                               int y, EpiCtx& e) {
+                                               int y, EpiCtx& e,
+                                               const __nv_bfloat16* bias = nullptr,
+                                               int ncols = 0) {
   const uint32_t buf = e.counter % kStoreBoxes;
   ++e.counter;
   // both TMEM loads in flight before one wait, and during the wait for the
@@ -73,6 +80,25 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
   named_bar_sync(1, 128);
   uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
   tmem_ld_wait();
+  if (bias != nullptr) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
+        const uint4 bq = c < ncols ? __ldg(reinterpret_cast<const uint4*>(bias + c))
+                                   : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t& v0 = vv[half][8 * ch + 2 * j];
+          uint32_t& v1 = vv[half][8 * ch + 2 * j + 1];
+          v0 = __float_as_uint(f32(v0) + __uint_as_float(w[j] << 16));
+          v1 = __float_as_uint(f32(v1) + __uint_as_float(w[j] & 0xffff0000u));
+        }
+      }
+    }
+  }
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -80,11 +106,61 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
       const int chunk = half * 4 + ch;
       const uint32_t off =
           static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+      auto val = [&](int c) {
+        const float v = f32(vv[half][8 * ch + c]);
+        return LO ? v - __bfloat162float(__float2bfloat16_rn(v)) : v;
+      };
       uint4 q;
-      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]), f32(vv[half][8 * ch + 1]));
-      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]), f32(vv[half][8 * ch + 3]));
-      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]), f32(vv[half][8 * ch + 5]));
-      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]), f32(vv[half][8 * ch + 7]));
+      q.x = pack_bf16x2(val(0), val(1));
+      q.y = pack_bf16x2(val(2), val(3));
+      q.z = pack_bf16x2(val(4), val(5));
+      q.w = pack_bf16x2(val(6), val(7));
+      *reinterpret_cast<uint4*>(sbuf + off) = q;
+    }
+  }
+  fence_async_shared();
+  named_bar_sync(1, 128);
+  if (e.tid == 0) {
+    tma_store_2d(tmap, e.smem_u32 + buf * kStoreBoxBytes, x, y);
+    tma_store_commit();
+  }
+}
+
+// The second half of store_box_bf16 for a box whose accumulator values the
+// caller already holds (loaded and waited for): lets the caller load the next
+// box from TMEM while this one is converted and stored.
+__device__ __forceinline__ void store_loaded_box_bf16(const uint32_t (&vv)[2][32], const void* tmap,
+                                                      int x, int y, EpiCtx& e,
+                                                      const __nv_bfloat16* bias = nullptr,
+                                                      int ncols = 0) {
+  const uint32_t buf = e.counter % kStoreBoxes;
+  ++e.counter;
+  if (e.tid == 0) tma_store_wait_read<kStoreBoxes - 1>();
+  named_bar_sync(1, 128);
+  uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      const int chunk = half * 4 + ch;
+      const uint32_t off =
+          static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
+      float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
+      if (bias != nullptr && c < ncols) {
+        const uint4 bq = __ldg(reinterpret_cast<const uint4*>(bias + c));
+        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          b[2 * jj] = __uint_as_float(w[jj] << 16);
+          b[2 * jj + 1] = __uint_as_float(w[jj] & 0xffff0000u);
+        }
+      }
+      uint4 q;
+      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]) + b[0], f32(vv[half][8 * ch + 1]) + b[1]);
+      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]) + b[2], f32(vv[half][8 * ch + 3]) + b[3]);
+      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]) + b[4], f32(vv[half][8 * ch + 5]) + b[5]);
+      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]) + b[6], f32(vv[half][8 * ch + 7]) + b[7]);
       *reinterpret_cast<uint4*>(sbuf + off) = q;
     }
   }
@@ -308,6 +384,7 @@ struct GramPolicy {
     int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total;
     uint32_t b_layout;
     __nv_bfloat16* Tb;  // (B*k) x d_in
+    __nv_bfloat16* Tlo;  // (B*k) x d_in: the bf16 rounding errors of Tb, or nullptr
     float* G;           // B x k x k
   };
   struct Tile {
@@ -373,10 +450,17 @@ struct GramPolicy {
     if (t.mt < p.mtx) {
       const int j = t.mt * 128 + row;
       if (j >= p.d_in) return;
-      __nv_bfloat16* dst = p.Tb + static_cast<size_t>(t.b) * p.k * p.d_in + j;
+      const size_t off = static_cast<size_t>(t.b) * p.k * p.d_in + j;
+      __nv_bfloat16* dst = p.Tb + off;
 #pragma unroll
       for (int u = 0; u < n; ++u)
-        if (i0 + u < p.k) dst[static_cast<size_t>(i0 + u) * p.d_in] = __float2bfloat16_rn(v[u]);
+        if (i0 + u < p.k) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(v[u]);
+          dst[static_cast<size_t>(i0 + u) * p.d_in] = h;
+          if (p.Tlo != nullptr)
+            p.Tlo[off + static_cast<size_t>(i0 + u) * p.d_in] =
+                __float2bfloat16_rn(v[u] - __bfloat162float(h));
+        }
     } else {
       const int i2 = (t.mt - p.mtx) * 128 + row;
       if (i2 >= p.k) return;
@@ -462,7 +546,11 @@ struct RFactorPolicy {
     CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
     CUtensorMap tmT;  // (d_in, B*k),   box (64, bn)
     CUtensorMap tmC;  // (B*k, d_out),  box (64, 128), store
+    CUtensorMap tmClo;  // same over the low parts (hilo)
+    CUtensorMap tmTlo;  // the low parts of T (split T), like tmT
     int d_in, d_out, Bk, bn, n_tiles_n;
+    int hilo;    // also store the low parts of Q^T
+    int split_t;  // T arrives as hi and lo parts: a second B operand per stage
   };
   struct Tile {
     int m0, n0;
@@ -473,6 +561,8 @@ struct RFactorPolicy {
     tma_prefetch_desc(&p.tmW);
     tma_prefetch_desc(&p.tmT);
     tma_prefetch_desc(&p.tmC);
+    if (p.hilo) tma_prefetch_desc(&p.tmClo);
+    if (p.split_t) tma_prefetch_desc(&p.tmTlo);
   }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 128;
@@ -485,6 +575,7 @@ struct RFactorPolicy {
                                               uint32_t sb, uint32_t bar) {
     tma_load_2d(sa, &p.tmW, bar, it * 64, t.m0);
     tma_load_2d(sb, &p.tmT, bar, it * 64, t.n0);
+    if (p.split_t) tma_load_2d(sb + static_cast<uint32_t>(p.bn) * 128u, &p.tmTlo, bar, it * 64, t.n0);
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
     return min(4, ceil_div_dev(p.d_in - it * 64, 16));
@@ -497,8 +588,10 @@ struct RFactorPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    for (int bx = 0; bx < p.bn / 64; ++bx)
+    for (int bx = 0; bx < p.bn / 64; ++bx) {
       store_box_bf16(tacc, bx * 64, &p.tmC, t.n0 + bx * 64, t.m0, e);
+      if (p.hilo) store_box_bf16<true>(tacc, bx * 64, &p.tmClo, t.n0 + bx * 64, t.m0, e);
+    }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
@@ -521,8 +614,22 @@ struct OutPolicy {
     CUtensorMap tmL;  // (k, T, B),     box (64, 128, 1)
     CUtensorMap tmC;  // (B*k, d_out),  box (64, bn)
     CUtensorMap tmY;  // (d_out, N),    box (64, 128), store
+    CUtensorMap tmLlo, tmClo;  // the low parts of L~ and Q^T (hilo)
     int N, r, k, T, B, bn, n_tiles_n, nkz, nkl;
+    const __nv_bfloat16* bias;  // d_out, added in the epilogue, or nullptr
+    int d_out;
+    int hilo;  // correction as hi L~ . hi Q + hi L~ . lo Q + lo L~ . hi Q
   };
+  // K-step j of the correction: instance segment, sub-product (0 hi.hi,
+  // 1 hi.lo, 2 lo.hi) and 64-wide chunk of k.
+  static __device__ __forceinline__ void correction_step(const Params& p, int j, int& seg,
+                                                         int& sub, int& ch) {
+    const int per = p.nkl * (p.hilo ? 3 : 1);
+    seg = j / per;
+    const int jj = j - seg * per;
+    sub = jj / p.nkl;
+    ch = jj - sub * p.nkl;
+  }
   struct Tile {
     int m0, n0, b_lo, nseg;
   };
@@ -534,6 +641,10 @@ struct OutPolicy {
     if (p.nkl > 0) {
       tma_prefetch_desc(&p.tmL);
       tma_prefetch_desc(&p.tmC);
+      if (p.hilo) {
+        tma_prefetch_desc(&p.tmLlo);
+        tma_prefetch_desc(&p.tmClo);
+      }
     }
     tma_prefetch_desc(&p.tmY);
   }
@@ -550,7 +661,7 @@ struct OutPolicy {
     }
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl;
+    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
@@ -558,12 +669,11 @@ struct OutPolicy {
       tma_load_2d(sa, &p.tmZ, bar, it * 64, t.m0);
       tma_load_2d(sb, &p.tmU, bar, it * 64, t.n0);
     } else {
-      const int j = it - p.nkz;
-      const int seg = j / p.nkl;
-      const int ch = j - seg * p.nkl;
+      int seg, sub, ch;
+      correction_step(p, it - p.nkz, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d(sa, &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
-      tma_load_2d(sb, &p.tmC, bar, b * p.k + ch * 64, t.n0);
+      tma_load_3d(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
+      tma_load_2d(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, t.n0);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
@@ -579,8 +689,29 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    for (int bx = 0; bx < p.bn / 64; ++bx)
-      store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e);
+    // The next box's TMEM loads are in flight while this box is converted and
+    // stored (tcgen05.wait::ld waits for every earlier load of the thread, so
+    // each wait comes after the previous box is written out).
+    const int nb = p.bn / 64;
+    uint32_t va[2][32], vb[2][32];
+    tmem_ld_32x32b_x32(tacc, va[0]);
+    tmem_ld_32x32b_x32(tacc + 32, va[1]);
+    tmem_ld_wait();
+    for (int bx = 0; bx < nb; bx += 2) {
+      if (bx + 1 < nb) {
+        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64, vb[0]);
+        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64 + 32, vb[1]);
+      }
+      store_loaded_box_bf16(va, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias, p.d_out);
+      if (bx + 1 >= nb) break;
+      tmem_ld_wait();
+      if (bx + 2 < nb) {
+        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64, va[0]);
+        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64 + 32, va[1]);
+      }
+      store_loaded_box_bf16(vb, &p.tmY, t.n0 + (bx + 1) * 64, t.m0, e, p.bias, p.d_out);
+      tmem_ld_wait();
+    }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
@@ -606,6 +737,9 @@ struct RFactorPairPolicy {
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
     tma_load_2d_pair(sa, &p.tmW, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
     tma_load_2d_pair(sb, &p.tmT, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
+    if (p.split_t)
+      tma_load_2d_pair(sb + static_cast<uint32_t>(p.bn / 2) * 128u, &p.tmTlo, bar, it * 64,
+                       t.n0 + (p.bn / 2) * static_cast<int>(rank));
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
     return RFactorPolicy::ksteps(p, t, it);
@@ -691,7 +825,7 @@ struct OutPairPolicy {
     }
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl;
+    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
@@ -701,12 +835,11 @@ struct OutPairPolicy {
       tma_load_2d_pair(sa, &p.tmZ, bar, it * 64, ma);
       tma_load_2d_pair(sb, &p.tmU, bar, it * 64, nb);
     } else {
-      const int j = it - p.nkz;
-      const int seg = j / p.nkl;
-      const int ch = j - seg * p.nkl;
+      int seg, sub, ch;
+      OutPolicy::correction_step(p, it - p.nkz, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d_pair(sa, &p.tmL, bar, ch * 64, ma - b * p.T, b);
-      tma_load_2d_pair(sb, &p.tmC, bar, b * p.k + ch * 64, nb);
+      tma_load_3d_pair(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, ma - b * p.T, b);
+      tma_load_2d_pair(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, nb);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
@@ -755,6 +888,8 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   c.num_tiles = num_tiles;
   c.defer_wait = 0;
   c.trigger_after_wait = 0;
+  c.b_parts = 1;
+  c.b_part_desc = 0;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -783,14 +918,16 @@ int launch_gemm(const typename Pol::Params& p, uint32_t smem, const DeviceInfo& 
                 cudaStream_t s, bool pdl, int cluster = 1) {
   if (p.c.num_tiles <= 0) return 0;
   auto kfn = umma_gemm_kernel<Pol>;
-  static uint32_t configured = 0;
-  if (smem > configured) {
+  static KernelSetup setup;
+  const int d = dev.device;
+  if (d < 0 || d >= kMaxDevices) return -1;
+  if (smem > setup.smem[d].load()) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = smem;
+    setup.smem[d].store(smem);
   }
   cudaLaunchConfig_t cfg = {};
   // with clusters every CTA takes exactly one tile (the grid is the tile count)
@@ -824,27 +961,29 @@ int launch_gemm_pair(const typename Pol::Params& p, uint32_t smem, const DeviceI
                      cudaStream_t s, bool pdl) {
   if (p.c.num_tiles <= 0) return 0;
   auto kfn = umma_gemm_pair_kernel<Pol>;
-  static uint32_t configured = 0;
-  static int max_pairs = 0;
+  static KernelSetup setup;  // occupancy: resident pairs at the configured size
+  const int d = dev.device;
+  if (d < 0 || d >= kMaxDevices) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  if (smem > configured) {
+  if (smem > setup.smem[d].load() || setup.occupancy[d].load() < 1) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess ||
         cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, 100) !=
             cudaSuccess)
       return -1;
-    configured = smem;
     cfg.gridDim = dim3(2 * (dev.sm_count / 2));
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, kfn, &cfg) != cudaSuccess || clusters < 1) {
       cudaGetLastError();
       clusters = dev.sm_count / 2;
     }
-    max_pairs = clusters;
+    setup.occupancy[d].store(clusters);
+    if (smem > setup.smem[d].load()) setup.smem[d].store(smem);
   }
+  const int max_pairs = setup.occupancy[d].load();
   cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min(p.c.num_tiles, max_pairs)));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1031,6 +1170,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       p.mtx = ceil_div(a.d_in, 128);
       p.mt_total = p.mtx + ceil_div(a.k, 128);
       p.Tb = static_cast<__nv_bfloat16*>(a.Tp);
+      p.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
       p.G = a.TG;
       p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
       uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
@@ -1087,26 +1227,45 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
       uint32_t bt[2] = {64, static_cast<uint32_t>(rf_pairs ? p.bn / 2 : p.bn)};
       if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
+      p.split_t = a.split_t ? 1 : 0;
+      if (a.split_t) {
+        if (!encode_tmap_bf16(&p.tmTlo, a.Tplo, 2, dt, sw, bt, 128)) return -2;
+      } else {
+        p.tmTlo = p.tmT;
+      }
+      const uint32_t parts = a.split_t ? 2u : 1u;  // B operands per stage
       uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, 128};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
+      p.hilo = a.hilo ? 1 : 0;
+      if (a.hilo) {
+        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
+      } else {
+        p.tmClo = p.tmC;
+      }
       if (rf_pairs) {
         const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
+        const uint32_t part_bytes = static_cast<uint32_t>(p.bn / 2) * 128u;
         const uint32_t smem =
-            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
+            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
                                             false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.b_parts = parts;
+        p.c.b_part_desc = part_bytes >> 4;
         p.c.trigger_after_wait = 1;
         p.c.idesc = idesc_bf16(256, p.bn, false, false);
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
       } else {
         const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
+        const uint32_t part_bytes = static_cast<uint32_t>(p.bn) * 128u;
         const uint32_t smem =
-            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false,
-                                        a.status, dev, rf_smem_cap);
+            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
+                                        false, a.status, dev, rf_smem_cap);
         if (!smem) return -3;
+        p.c.b_parts = parts;
+        p.c.b_part_desc = part_bytes >> 4;
         p.c.trigger_after_wait = 1;
         if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
         if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
@@ -1126,8 +1285,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
                  ? 1
                  : 0;
     if (!records) mode = 0;
-    if (launch_ltilde(a.TG, a.L, a.MD, a.counters, mode, a.B, a.T, a.k, a.lambda, a.status, s,
-                      pdl, /*defer_wait=*/true,
+    if (launch_ltilde(a.TG, a.L, a.hilo ? a.Llo : nullptr, a.MD, a.counters, mode, a.B, a.T, a.k,
+                      a.lambda, a.alpha, a.status, s, pdl, /*defer_wait=*/true,
                       a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
       return -1;
   } else {
@@ -1149,6 +1308,8 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     p.n_tiles_n = ceil_div(a.d_out, p.bn);
     p.nkz = ceil_div(a.r, 64);
     p.nkl = k > 0 ? ceil_div(k, 64) : 0;
+    p.bias = static_cast<const __nv_bfloat16*>(a.bias);
+    p.d_out = a.d_out;
 
     uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
     uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
@@ -1171,10 +1332,20 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
       uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
       uint32_t bc[2] = {64, bbox};
       if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
+      if (a.hilo) {
+        if (!encode_tmap_bf16(&p.tmLlo, a.Llo, 3, dl, sl, bl, 128)) return -2;
+        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
+      } else {
+        p.tmLlo = p.tmL;
+        p.tmClo = p.tmC;
+      }
     } else {
       p.tmL = p.tmZ;
       p.tmC = p.tmU;
+      p.tmLlo = p.tmZ;
+      p.tmClo = p.tmU;
     }
+    p.hilo = k > 0 && a.hilo ? 1 : 0;
     uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
     uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
     uint32_t by[2] = {64, 128};

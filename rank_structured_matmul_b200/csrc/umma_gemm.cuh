@@ -76,6 +76,11 @@ struct GemmCommon {
   // 1: the next grid may start only once this grid's own dependency wait is
   // over (that grid then relies on what the grid before this one wrote).
   int trigger_after_wait;
+  // B operands per stage (1, or 2 when a second operand, e.g. the low part of
+  // a split bf16 value, accumulates into the same tile with the same A), and
+  // the smem descriptor step from one part to the next
+  uint32_t b_parts;
+  uint64_t b_part_desc;
 };
 
 // Issues one stage's ks MMAs (K = 16 each) back to back. The tensor pipe idles
@@ -257,6 +262,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
           issue_stage<false>(d, a0, da, b0, db, idesc, ks, it == 0);
+          for (uint32_t part = 1; part < c.b_parts; ++part)
+            issue_stage<false>(d, a0, da, b0 + part * c.b_part_desc, db, idesc, ks, false);
           mma_commit(empty_bar(stage));
           a += c.a_stage_bytes;
           b += c.b_stage_bytes;

@@ -36,6 +36,11 @@ _vp, _i, _i64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_floa
 SIGNATURES = {
     "dyra_plan_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
+    "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
+    "dyra_set_als_steps": (_i, [_vp, _i]),
+    "dyra_forward_batched_host": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
+    "dyra_plan_create_monarch": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "dyra_load_monarch": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_forward_weight_only": (_i, [_vp, _vp, _vp, _i64, _vp]),
@@ -123,6 +128,33 @@ def dyra_plan_create(d_in: int, d_out: int, r: int, k: int, dtype: int) -> int:
 def dyra_load_factors(plan: int, U, V, P, W_res, lam: float, stream=None) -> None:
     _check(lib().dyra_load_factors(plan, _ptr(U), _ptr(V), _ptr(P), _ptr(W_res), float(lam),
                                    _stream(stream)), "dyra_load_factors")
+
+
+def dyra_set_linear(plan: int, bias, alpha: float = 1.0, stream=None) -> None:
+    _check(lib().dyra_set_linear(plan, _ptr(bias), float(alpha), _stream(stream)),
+           "dyra_set_linear")
+
+
+def dyra_set_als_steps(plan: int, half_steps: int) -> None:
+    _check(lib().dyra_set_als_steps(plan, int(half_steps)), "dyra_set_als_steps")
+
+
+def dyra_forward_batched_host(plan: int, X, Y, B: int, T: int, stream=None) -> None:
+    """dyra_forward_batched on host buffers (X, Y page-locked CPU tensors or addresses)."""
+    _check(lib().dyra_forward_batched_host(plan, _ptr(X), _ptr(Y), int(B), int(T),
+                                           _stream(stream)), "dyra_forward_batched_host")
+
+
+def dyra_plan_create_monarch(n: int, b1: int, b2: int, k: int, dtype: int) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().dyra_plan_create_monarch(ctypes.byref(h), n, b1, b2, k, dtype),
+           "dyra_plan_create_monarch")
+    return h.value
+
+
+def dyra_load_monarch(plan: int, Lblocks, Rblocks, P, W_res, lam: float, stream=None) -> None:
+    _check(lib().dyra_load_monarch(plan, _ptr(Lblocks), _ptr(Rblocks), _ptr(P), _ptr(W_res),
+                                   float(lam), _stream(stream)), "dyra_load_monarch")
 
 
 def dyra_forward(plan: int, X, Y, N: int, stream=None) -> None:
@@ -228,6 +260,21 @@ class DyraLinear:
                           lam, stream)
         torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
 
+    def set_linear(self, bias=None, alpha: float = 1.0, stream=None) -> None:
+        """Bias (d_out values, or None) and correction weight of the full
+        linear layer, Y = static + bias + alpha * correction."""
+        import torch
+        b = self._dev(bias)
+        dyra_set_linear(self.plan, b, alpha, stream)
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+
+    def set_als_iterations(self, t: float) -> None:
+        """t ALS iterations per forward (t = 1, 1.5, 2, ...; DyRA Sec. 3.3)."""
+        steps = int(round(2 * t))
+        if steps != 2 * t:
+            raise ValueError("t must be a multiple of 0.5")
+        dyra_set_als_steps(self.plan, steps)
+
     def _check_x(self, X):
         import torch
         if not (X.is_cuda and X.dtype == self.torch_dtype and X.is_contiguous()
@@ -246,6 +293,25 @@ class DyraLinear:
         if Y is None:
             Y = torch.empty((N, self.d_out), device=X.device, dtype=self.torch_dtype)
         dyra_forward_batched(self.plan, X, Y, B, T, stream)
+        return Y
+
+    def forward_host(self, X, B: int = 1, T: Optional[int] = None, Y=None, stream=None):
+        """forward() on host tensors: copies in, the layer and copies out overlap
+        by chunks of instances. X and Y should be pinned CPU tensors; the call is
+        asynchronous on the stream (synchronise it before reading Y)."""
+        import torch
+        if X.is_cuda or X.dtype != self.torch_dtype or not X.is_contiguous() or X.dim() != 2 \
+                or X.shape[1] != self.d_in:
+            raise ValueError("X must be a contiguous CPU %s tensor of shape (N, %d)"
+                             % (self.torch_dtype, self.d_in))
+        N = X.shape[0]
+        if T is None:
+            T = N // B
+        if B * T != N:
+            raise ValueError("B*T must equal the row count of X")
+        if Y is None:
+            Y = torch.empty((N, self.d_out), dtype=self.torch_dtype).pin_memory()
+        dyra_forward_batched_host(self.plan, X, Y, B, T, stream)
         return Y
 
     def forward_weight_only(self, X, Y=None, stream=None):
@@ -272,3 +338,25 @@ class DyraLinear:
             self.close()
         except Exception:
             pass
+
+
+class DyraMonarchLinear(DyraLinear):
+    """A DyRA layer whose static part is a Monarch matrix (DyRA App. B) of
+    n = b1 * b2 features; load() takes the blocks instead of U and V."""
+
+    def __init__(self, n: int, b1: int, b2: int, k: int, dtype: str = "bf16"):
+        import torch
+        self.d_in = self.d_out = n
+        self.r, self.k, self.b1, self.b2 = 0, k, b1, b2
+        self.dtype = dtype
+        self.torch_dtype = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
+        self.plan = dyra_plan_create_monarch(n, b1, b2, k,
+                                             DYRA_BF16 if dtype == "bf16" else DYRA_F32)
+
+    def load(self, Lblocks, Rblocks, P, W_res, lam: float, stream=None) -> None:
+        """Lblocks: (b2, b1, b1), Rblocks: (b1, b2, b2), P: (n, k), W_res: (n, n)."""
+        import torch
+        Lb, Rb, P, W_res = (self._dev(t) for t in (Lblocks, Rblocks, P, W_res))
+        dyra_load_monarch(self.plan, Lb, Rb, P if self.k else None, W_res if self.k else None,
+                          lam, stream)
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()

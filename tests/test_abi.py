@@ -73,6 +73,11 @@ def test_null_handles():
     assert lib.dyra_forward_weight_only(None, None, None, 1, None) == dyra.DYRA_ERR_INVALID_ARG
     assert lib.dyra_load_factors(None, None, None, None, None, 0.0, None) == dyra.DYRA_ERR_INVALID_ARG
     assert lib.dyra_reserve(None, 1, 1) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_set_linear(None, None, 1.0, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_set_als_steps(None, 2) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_forward_batched_host(None, None, None, 2, 3, None) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_plan_create_monarch(None, 12, 3, 4, 2, dyra.DYRA_F32) == dyra.DYRA_ERR_INVALID_ARG
+    assert lib.dyra_load_monarch(None, None, None, None, None, 0.0, None) == dyra.DYRA_ERR_INVALID_ARG
     assert lib.dyra_last_status(None) == dyra.DYRA_ERR_INVALID_ARG
     assert lib.dyra_plan_destroy(None) == dyra.DYRA_OK
     assert lib.dyra_plan_device_bytes(None) == 0

@@ -180,6 +180,189 @@ def test_gaussian_start(case):
     assert oracle.rel_fro(Ya, Yo) < TOL[dtype] / 10
 
 
+LINEAR = [
+    # name, d_in, d_out, r, k, B, T, dtype, alpha, pairs
+    ("linear_pairs", 256, 512, 64, 32, 3, 201, "bf16", 0.5, True),
+    ("linear_alpha1", 256, 512, 64, 32, 3, 201, "bf16", 1.0, True),
+    ("linear_alpha0", 256, 512, 64, 32, 3, 201, "bf16", 0.0, True),
+    ("linear_single_cta", 256, 512, 64, 32, 3, 201, "bf16", 0.5, False),
+    ("linear_odd_d_out", 200, 328, 40, 8, 5, 37, "bf16", 1.5, True),   # last box past d_out
+    ("linear_k72", 256, 512, 64, 72, 2, 300, "bf16", 0.5, True),        # the general solve
+    ("linear_weight_only", 256, 512, 64, 0, 3, 201, "bf16", 1.0, True),
+    ("linear_f32", 96, 80, 12, 8, 3, 50, "f32", 0.5, True),
+]
+
+
+@pytest.mark.parametrize("case", LINEAR, ids=[c[0] for c in LINEAR])
+def test_bias_and_alpha(case):
+    """The full linear layer (DyRA Sec. 2.4): Y = static + b + alpha * correction,
+    against the oracle with the same bias (rounded to the storage type) and alpha."""
+    name, d_in, d_out, r, k, B, T, dtype, alpha, pairs = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, "lognormal", seed=3)
+    f = prepared(s)
+    bias = oracle.round_to(np.random.default_rng(5).standard_normal(d_out) * 0.3, dtype)
+    if not pairs:
+        os.environ["DYRA_PAIR"] = "0"
+    try:
+        layer = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_PAIR", None)
+    X = to_dev(f["X"], dtype)
+    Y0 = layer.forward(X, B=B, T=T).double().cpu().numpy()  # captures a graph first
+    layer.set_linear(to_dev(bias, dtype), alpha)
+    Y = layer.forward(X, B=B, T=T)
+    assert layer.status() == 0
+    Yg = Y.double().cpu().numpy()
+    Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, B, T, bias=bias,
+                          alpha=alpha)
+    err = oracle.rel_fro(Yg, Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    # the weight-only entry adds the bias too
+    Yw = layer.forward_weight_only(X).double().cpu().numpy()
+    Ywo = (f["X"] @ f["V"]) @ f["U"].T + bias
+    assert oracle.rel_fro(Yw, Ywo) <= TOL[dtype]
+    # removing the bias and restoring alpha gives the plain layer back
+    layer.set_linear(None, 1.0)
+    Y1 = layer.forward(X, B=B, T=T).double().cpu().numpy()
+    np.testing.assert_array_equal(Y1, Y0)
+    layer.close()
+
+
+ALS = [
+    # name, d_in, d_out, r, k, B, T, dtype, t
+    ("als_f32_t1.5", 96, 80, 12, 8, 3, 50, "f32", 1.5),
+    ("als_f32_t2", 96, 80, 12, 8, 3, 50, "f32", 2.0),
+    ("als_f32_t3_k40", 128, 96, 16, 40, 2, 60, "f32", 3.0),
+    ("als_bf16_simt_t2", 256, 512, 64, 32, 3, 201, "bf16", 2.0),
+]
+
+
+@pytest.mark.parametrize("case", ALS, ids=[c[0] for c in ALS])
+def test_als_iterations(case):
+    """t alternating least-squares iterations (DyRA Sec. 2.2, Sec. 3.3) on the
+    CUDA-core kernels, against the oracle's ALS from the same start; t = 1
+    again afterwards gives the one-step layer."""
+    name, d_in, d_out, r, k, B, T, dtype, t = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, "outlier", n_outlier=4,
+                  outlier_scale=10.0, seed=2)
+    w = generate(s)
+    fo = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, r, k, s.lam)
+    f = {n: oracle.round_to(a, dtype) for n, a in
+         (("X", w.X), ("U", fo.U), ("V", fo.V), ("P", fo.P), ("W_res", fo.W_res))}
+    layer = make_layer(s, f, kernels="simt")
+    X = to_dev(f["X"], dtype)
+    layer.set_als_iterations(t)
+    Y = layer.forward(X, B=B, T=T)
+    assert layer.status() == 0
+    Yo = oracle.als_inference(f["X"], f["U"], f["V"], f["W_res"], fo.R0, s.lam, B, T, t)
+    err = oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    layer.set_als_iterations(1)
+    check(s, layer.forward(X, B=B, T=T), f, full=True)
+    layer.close()
+
+
+def test_als_iterations_need_the_cuda_core_kernels():
+    s, f = _small()
+    layer = make_layer(s, f)
+    layer.set_als_iterations(1)
+    with pytest.raises(dyra.DyraError):
+        layer.set_als_iterations(2)
+    layer.close()
+
+
+@pytest.mark.parametrize("B,T", [(32, 201), (3, 201), (1, 600)])
+def test_host_forward_matches_device_forward(B, T):
+    """dyra_forward_batched_host (host buffers, copies overlapped by chunks of
+    instances) meets the oracle like the device-buffer forward. The chunks are
+    forwards of fewer instances, whose Gram reduction may split rows
+    differently, so the two agree to rounding, not bit for bit."""
+    s = LayerSpec("host", 256, 512, 64, 32, B, T, "bf16", 0.7, "lognormal", seed=4)
+    f = prepared(s)
+    layer = make_layer(s, f)
+    Xd = to_dev(f["X"], "bf16")
+    Yd = layer.forward(Xd, B=B, T=T).cpu()
+    Xh = Xd.cpu().pin_memory()
+    Yh = layer.forward_host(Xh, B=B, T=T)
+    torch.cuda.current_stream().synchronize()
+    assert layer.status() == 0
+    check(s, Yh, f, full=True)
+    assert oracle.rel_fro(Yh.double().numpy(), Yd.double().numpy()) <= TOL["bf16"] / 2
+    layer.close()
+
+
+HILO = [
+    # name, d_in, d_out, r, k, B, T, outlier channels (x20)
+    ("hilo_single", 1024, 2048, 128, 64, 1, 128, 8),
+    ("hilo_batched", 256, 512, 64, 32, 3, 201, 8),
+    ("hilo_needed", 512, 1024, 64, 64, 1, 128, 6),   # modelled 1.1e-2 without it, 6.8e-3 with
+]
+
+
+def _run_hilo(s, f, mode):
+    os.environ["DYRA_HILO"] = mode
+    try:
+        layer = make_layer(s, f)
+    finally:
+        os.environ.pop("DYRA_HILO", None)
+    Y = layer.forward(to_dev(f["X"], s.dtype), B=s.B, T=s.T)
+    assert layer.status() == 0
+    layer.close()
+    Yo = oracle.inference(f["X"], f["U"], f["V"], f["P"], f["W_res"], s.lam, s.B, s.T)
+    return oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+
+
+@pytest.mark.parametrize("case", HILO, ids=[c[0] for c in HILO])
+def test_compensated_correction(case):
+    """L~ and Q^T with their bf16 rounding errors (hi.hi + hi.lo + lo.hi in
+    the output stage) cut the error the grouping L~ . Q amplifies on
+    ill-conditioned instances (outlier channels)."""
+    name, d_in, d_out, r, k, B, T, nout = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, "bf16", 0.6, "outlier", n_outlier=nout,
+                  outlier_scale=20.0, seed=5)
+    f = prepared(s)
+    err_on = _run_hilo(s, f, "1")
+    assert err_on <= TOL["bf16"], "%s: %.3e" % (name, err_on)
+    if name != "hilo_needed":
+        err_off = _run_hilo(s, f, "0")
+        assert err_on < 0.8 * err_off, (err_on, err_off)
+
+
+MONARCH = [
+    # name, b1, b2, k, B, T, dtype
+    ("monarch_f32", 8, 12, 8, 3, 50, "f32"),
+    ("monarch_f32_k0", 6, 6, 0, 2, 40, "f32"),
+    ("monarch_bf16", 16, 16, 32, 3, 201, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", MONARCH, ids=[c[0] for c in MONARCH])
+def test_monarch_static_part(case):
+    """A Monarch static part (DyRA App. B) under the same correction, on the
+    CUDA-core kernels, against the oracle's Monarch layer."""
+    from oracle import monarch as mon
+    name, b1, b2, k, B, T, dtype = case
+    n = b1 * b2
+    s = LayerSpec(name, n, n, 1, k, B, T, dtype, 0.7, "lognormal", seed=8)
+    w = generate(s)
+    fo = mon.offline_prepare_monarch(w.weight(), b1, b2, k, s.lam)
+    rd = lambda a: oracle.round_to(a, dtype)
+    Lb = rd(np.stack(fo.Lb))
+    Rb = rd(np.stack(fo.Rb))
+    P, W_res, X = rd(fo.P), rd(fo.W_res), rd(w.X)
+    layer = dyra.DyraMonarchLinear(n, b1, b2, k, dtype)
+    layer.load(to_dev(Lb, dtype), to_dev(Rb, dtype), to_dev(P, dtype) if k else None,
+               to_dev(W_res, dtype) if k else None, s.lam)
+    Y = layer.forward(to_dev(X, dtype), B=B, T=T)
+    assert layer.status() == 0
+    fr = mon.MonarchFactors(list(Lb), list(Rb), mon.monarch_matrix(list(Lb), list(Rb)).T, P, W_res,
+                            fo.R0)
+    Yo = mon.monarch_inference(X, fr, s.lam, B, T)
+    err = oracle.rel_fro(Y.double().cpu().numpy(), Yo)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    layer.close()
+
+
 # ----------------------------------------------------------- properties ----
 
 def _small(k=32, lam=1e-3, B=3, T=201, dtype="bf16"):
