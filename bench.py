@@ -2,12 +2,20 @@
 """Benchmark of the DyRA approximated linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl dyra|reference]
-                    [--layer-only] [--no-cpu-baseline]
+                    [--layer-only] [--no-cpu-baseline] [--no-per-config]
 
 One step is one DyRA forward (projection, Gram, solve, residual factor,
 output: every stage of Algorithm 1's inference procedure) over the workload's
-B x T rows, inputs resident in HBM. The L2 cache is flushed (256 MiB write)
-before every step, outside the step's CUDA events. Prints one JSON line.
+B x T rows, inputs resident in HBM. The default workload is the largest
+single-GPU configuration, the Llama-shaped up-projection at 8192 tokens
+(4096 -> 14336, r = 1024, k = 64). `--workload vit_block` runs the four
+ViT-L/16 block linears (qkv, proj, fc1, fc2; 64 x 201 tokens) back to back on
+one stream as one step. The L2 cache is flushed (256 MiB write) before every
+step, outside the step's CUDA events. Prints one JSON line.
+
+Beside the headline, `per_config` times every workload (each layer of the
+synthetic set and the ViT block sequence) against cuBLAS dense X W^T of the
+same shape and checks it against the fp64 oracle on sampled rows.
 
 Under torchrun (N > 1) every rank runs its own replica of the workload on its
 own GPU (instances are independent; no collective on the data path); the
@@ -25,7 +33,6 @@ import json
 import os
 import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -35,13 +42,45 @@ sys.path.insert(0, ROOT)
 
 METRIC = "DyRA linear µs & dense-equiv TFLOP/s vs cuBLAS dense; % of roofline"
 UNIT = "TFLOP/s (dense-equivalent)"
-HEADLINE = "vit_fc1"
+HEADLINE = "llama_up_8192"
+BLOCK = ("vit_block_qkv", "vit_block_proj", "vit_block_fc1", "vit_block_fc2")
 STAGE_KERNELS = {"proj": "ProjPolicy (CTA pairs, or split-K clusters at skinny N)",
                  "gram": "umma_gemm_kernel<GramPolicy>",
                  "solve": "ltilde_kernel (L~ = L G^-1, beside the rank-k factor GEMM)",
                  "rfactor": "RFactorPolicy (Q = T W_res^T; CTA pairs when there are enough tiles)",
                  "out": "umma_gemm_pair_kernel<OutPairPolicy>"}
 FLUSH_BYTES = 256 << 20
+L2_NOTE = "GPU arm: 256 MiB written before every step, outside the step events"
+DATA = ("synthetic (seeded; shapes and statistics of the workload, random-orthogonal weights "
+        "with a power-law spectrum)")
+
+
+def workload_names():
+    from synth import CONFIGS
+    return list(CONFIGS) + ["vit_block"]
+
+
+def specs_of(workload: str):
+    """The layers one step of `workload` runs, in order."""
+    from synth import spec
+    if workload == "vit_block":
+        return [spec(n) for n in BLOCK]
+    return [spec(workload)]
+
+
+def config_of(workload: str, world: int) -> dict:
+    """The `config` object of both arms' JSON lines (identical by construction)."""
+    ss = specs_of(workload)
+    layers = [{"name": s.name, "d_in": s.d_in, "d_out": s.d_out, "r": s.r, "k": s.k,
+               "instances": s.B, "rows_per_instance": s.T} for s in ss]
+    c = {"workload": workload}
+    if len(ss) == 1:
+        c.update({k: v for k, v in layers[0].items() if k != "name"})
+    else:
+        c["layers"] = layers
+    c.update({"rows": ss[0].N, "lambda": ss[0].lam, "l2": L2_NOTE,
+              "parallelism": "replicas" if world > 1 else "single GPU"})
+    return c
 
 
 def peaks():
@@ -78,15 +117,8 @@ def stored_traffic(stage: str, workload: str):
 
 # ------------------------------------------------------------ workload ----
 
-def workload_arrays(name: str):
-    from synth import generate, spec
-    s = spec(name)
-    w = generate(s)
-    return s, w
-
-
 def algorithmic(s):
-    """FLOPs and compulsory bytes of one forward and of its output stage."""
+    """FLOPs and compulsory bytes of one forward, per stage and for the layer."""
     es = 2 if s.dtype == "bf16" else 4
     N, di, do, r, k, B = s.N, s.d_in, s.d_out, s.r, s.k, s.B
     flops = {
@@ -108,6 +140,21 @@ def algorithmic(s):
     return flops, bytes_, layer_flops, layer_bytes
 
 
+def layer_roofline_us(s, pk) -> float:
+    """The slower of the layer's FLOPs at the bf16 peak and its compulsory
+    bytes at the HBM peak, in µs."""
+    _, _, f, b = algorithmic(s)
+    return max(f / (pk["bf16_tflops"] * 1e12), b / (pk["hbm_gbs"] * 1e9)) * 1e6
+
+
+def launches_per_forward(s) -> int:
+    """Library kernels one forward launches: five tensor-core stages (two
+    without the correction); the fp32 path's CUDA-core chain is seven."""
+    if s.dtype == "bf16":
+        return 5 if s.k > 0 else 2
+    return 7 if s.k > 0 else 2
+
+
 def static_matched_rank(s) -> int:
     """Rank r_s of a static-only layer (X V_s) U_s^T whose FLOPs 2 N r_s
     (d_in + d_out) match the DyRA layer's ([DyRA] App. E.4: the static
@@ -119,16 +166,29 @@ def static_matched_rank(s) -> int:
     return max(rs, 8)
 
 
+def parity_rows(s, max_rows: int = 1024):
+    """Rows of a workload that the oracle checks: every row of small layers;
+    otherwise whole leading instances (multi-instance layers) or evenly
+    spaced rows plus the last rows of a single long instance."""
+    if s.N <= max_rows:
+        return np.arange(s.N)
+    if s.B > 1:
+        n_inst = max(1, max_rows // s.T)
+        return np.arange(n_inst * s.T)
+    body = np.linspace(0, s.N - 1, max_rows - 64).astype(np.int64)
+    return np.unique(np.concatenate([body, np.arange(s.N - 64, s.N)]))
+
+
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every few ms while the timed
-    region runs (read-only NVML queries; nvidia-smi as a fallback)."""
+    """SM clock and clock-event reasons sampled every millisecond while the
+    timed region runs (read-only NVML queries; nvidia-smi as a fallback)."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4}
 
-    def __init__(self, cuda_index: int, period_s: float = 0.005):
+    def __init__(self, cuda_index: int, period_s: float = 0.001):
         self.cuda_index = cuda_index
         self.period = period_s
         self.rows = []
@@ -181,6 +241,7 @@ class ClockSampler:
         if self.handle is None:
             return
         import threading
+        self.rows, self.stop_flag = [], False
         self._sample()
         self.thread = threading.Thread(target=self._loop, daemon=True)
         self.thread.start()
@@ -198,7 +259,8 @@ class ClockSampler:
         reasons = sorted(name for name, bit in self.REASONS.items()
                          if any(r[2] & bit for r in rows))
         return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows), "source": "nvml, every 5 ms"}
+                "sm_mhz_min": float(min(r[0] for r in rows)), "reasons": reasons,
+                "samples": len(rows), "source": "nvml, every %g ms" % (self.period * 1e3)}
 
     def _smi_once(self):
         fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
@@ -237,10 +299,201 @@ def job_value(flops_per_rank: float, world: int, seconds: float) -> float:
 
 # ------------------------------------------------------------ dyra arm ----
 
+class LayerRun:
+    """One layer of a workload on the device: its plan with the factors loaded,
+    the seeded input X resident in HBM and the output Y."""
+
+    def __init__(self, s, dev, w=None):
+        import torch
+        from rank_structured_matmul_b200 import dyra, prep
+        from synth import generate
+        self.s = s
+        self.w = w if w is not None else generate(s)
+        f = prep.prepare_from_svd(self.w.left, self.w.sigma, self.w.right, s.r, s.k, s.lam)
+        self.td = torch.bfloat16 if s.dtype == "bf16" else torch.float32
+        self.layer = dyra.DyraLinear(s.d_in, s.d_out, s.r, s.k, s.dtype)
+        self.layer.load(f.U, f.V, f.P, f.W_res, s.lam)
+        self.X = torch.from_numpy(self.w.X).to(dev, self.td)
+        self.Y = torch.empty(s.N, s.d_out, device=dev, dtype=self.td)
+        self.layer.reserve(s.B, s.T)
+        self.dev = dev
+        self.Wd = self.Yd = None
+        self.Xh = self.Yh = None
+
+    def step(self):
+        self.layer.forward(self.X, B=self.s.B, T=self.s.T, Y=self.Y)
+
+    def dense_step(self):
+        import torch
+        if self.Wd is None:
+            self.Wd = torch.from_numpy(self.w.weight()).to(self.dev, self.td)
+            self.Yd = torch.empty_like(self.Y)
+        torch.matmul(self.X, self.Wd.t(), out=self.Yd)
+
+    def host_step(self):
+        """The forward through the C ABI on pinned host buffers."""
+        if self.Xh is None:
+            self.Xh = self.X.cpu().pin_memory()
+            import torch
+            self.Yh = torch.empty(self.Y.shape, dtype=self.td).pin_memory()
+        self.layer.forward_host(self.Xh, B=self.s.B, T=self.s.T, Y=self.Yh)
+
+    def free_dense(self):
+        self.Wd = self.Yd = None
+
+    def close(self):
+        self.layer.close()
+
+
+class Timer:
+    """Mean device time of a step over K launches, each after an L2 flush
+    outside its CUDA events (recorded on the current stream)."""
+
+    def __init__(self, dev):
+        import torch
+        self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self, fn, K, W):
+        import torch
+        for _ in range(W):
+            self.flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        for a, b in ev:
+            self.flush.zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+def stage_times(runs, timer, n_steps):
+    """Mean per-stage device time of each layer (events between the stage
+    launches, a separate loop with stage timing switched on), in ms."""
+    from rank_structured_matmul_b200 import dyra
+    out = []
+    for run in runs:
+        dyra.dyra_debug_set_stage_timing(run.layer.plan, True)
+        acc = {k: [] for k in dyra.STAGES}
+        for _ in range(n_steps):
+            timer.flush.zero_()
+            run.step()
+            for k2, v in dyra.dyra_debug_stage_times(run.layer.plan).items():
+                acc[k2].append(v)
+        dyra.dyra_debug_set_stage_timing(run.layer.plan, False)
+        out.append({k2: float(np.mean(v)) for k2, v in acc.items()})
+    return out
+
+
+def dominant_roofline(runs, st, pk, workload):
+    """Roofline of the stage with the most device time over the step's
+    layers: its algorithmic bytes or FLOPs over its live time."""
+    tot = {k: sum(t[k] for t in st) for k in st[0]}
+    dom = max(tot, key=tot.get)
+    t_dom = tot[dom] * 1e-3
+    fl = sum(algorithmic(r.s)[0][dom] for r in runs)
+    by = sum(algorithmic(r.s)[1][dom] for r in runs)
+    if fl / (pk["bf16_tflops"] * 1e12) >= by / (pk["hbm_gbs"] * 1e9):
+        roof = {"bound": "tensor", "achieved": fl / t_dom / 1e12, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": by / t_dom / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = stored_traffic(dom, workload)
+    roof["kernel"] = STAGE_KERNELS[dom]
+    roof["stage"] = dom
+    roof["peak_source"] = pk["source"] + " burst"
+    return roof
+
+
+def oracle_check(s, w, Y_gpu, rows=None):
+    """The GPU output on sampled rows against the fp64 oracle on the same
+    rounded inputs, with the oracle's own errors against the dense product."""
+    import oracle
+    f, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, w)
+    rows = parity_rows(s) if rows is None else rows
+    Yo = oracle.inference_rows(Xr, Ur, Vr, Pr, Wr, s.lam, s.B, s.T, rows)
+    Yg = Y_gpu[torch_index(rows, Y_gpu.device)].double().cpu().numpy()
+    Yd = oracle.dense(Xr[rows], w.weight())
+    Ywo = oracle.weight_only(Xr[rows], Ur, Vr)
+    return {"rel_fro_vs_oracle": oracle.rel_fro(Yg, Yo),
+            "tol": 1e-2 if s.dtype == "bf16" else 1e-5, "rows": int(len(rows)),
+            "oracle_err_weight_only": oracle.rel_fro(Ywo, Yd),
+            "oracle_err_dyra": oracle.rel_fro(Yo, Yd)}
+
+
+def torch_index(rows, device):
+    import torch
+    return torch.as_tensor(np.asarray(rows, dtype=np.int64), device=device)
+
+
+def per_config(names, dev, pk, steps, warmup, headline_entry=None):
+    """Every workload in `names`, timed against cuBLAS dense and checked
+    against the oracle. Returns the entries and the clocks sampled while
+    they ran."""
+    from synth import generate, spec
+    timer = Timer(dev)
+    entries = {}
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    llama_w = None
+    for name in names:
+        if headline_entry is not None and name == headline_entry[0]:
+            entries[name] = headline_entry[1]
+            continue
+        ss = specs_of(name)
+        runs = []
+        for s in ss:
+            w = None
+            if s.name.startswith("llama_up_"):
+                # one 8192-row draw; each sweep point is its N-row prefix
+                if llama_w is None:
+                    llama_w = generate(spec("llama_up_8192"))
+                w = dataclass_prefix(llama_w, s)
+            runs.append(LayerRun(s, dev, w))
+        seq = lambda: [r.step() for r in runs]
+        dense = lambda: [r.dense_step() for r in runs]
+        t = timer(seq, steps, warmup)
+        td = timer(dense, steps, 3)
+        flops = sum(2.0 * r.s.N * r.s.d_in * r.s.d_out for r in runs)
+        roof_us = sum(layer_roofline_us(r.s, pk) for r in runs)
+        e = {"us": t * 1e3, "cublas_dense_us": td * 1e3, "speedup_vs_cublas_dense": td / t,
+             "dense_equiv_tflops": flops / (t * 1e-3) / 1e12,
+             "layer_roofline_us": roof_us, "layer_roofline_frac": roof_us / (t * 1e3),
+             "device_status": max(r.layer.status() for r in runs)}
+        checks = [oracle_check(r.s, r.w, r.Y) for r in runs]
+        e["rel_fro_vs_oracle"] = max(c["rel_fro_vs_oracle"] for c in checks)
+        e["tol"] = checks[0]["tol"]
+        e["oracle_err_weight_only"] = [c["oracle_err_weight_only"] for c in checks]
+        e["oracle_err_dyra"] = [c["oracle_err_dyra"] for c in checks]
+        e["parity_rows"] = [c["rows"] for c in checks]
+        if len(runs) > 1:
+            e["layers"] = {}
+            for r in runs:
+                tl = timer(r.step, steps, 3)
+                tdl = timer(r.dense_step, steps, 3)
+                e["layers"][r.s.name] = {"us": tl * 1e3, "cublas_dense_us": tdl * 1e3}
+        for r in runs:
+            r.free_dense()
+            r.close()
+        entries[name] = e
+    clk = clocks.stop()
+    return entries, clk
+
+
+def dataclass_prefix(w, s):
+    """The N-row prefix of a larger draw of the same layer."""
+    import dataclasses
+    return dataclasses.replace(w, spec=s, X=np.ascontiguousarray(w.X[: s.N]))
+
+
 def run_dyra(args):
     import torch
     import torch.distributed as dist
-    from rank_structured_matmul_b200 import dyra, prep
+    from rank_structured_matmul_b200 import dyra
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -251,32 +504,13 @@ def run_dyra(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    s, w = workload_arrays(args.workload)
-    f = prep.prepare_from_svd(w.left, w.sigma, w.right, s.r, s.k, s.lam)
-    td = torch.bfloat16 if s.dtype == "bf16" else torch.float32
-    layer = dyra.DyraLinear(s.d_in, s.d_out, s.r, s.k, s.dtype)
-    layer.load(f.U, f.V, f.P, f.W_res, s.lam)
-    X = torch.from_numpy(w.X).to(dev, td)
-    Y = torch.empty(s.N, s.d_out, device=dev, dtype=td)
-    layer.reserve(s.B, s.T)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    ss = specs_of(args.workload)
+    runs = [LayerRun(s, dev) for s in ss]
+    timer = Timer(dev)
 
     def step():
-        layer.forward(X, B=s.B, T=s.T, Y=Y)
-
-    def timed(fn, K, W):
-        for _ in range(W):
-            flush.zero_()
-            fn()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
-        for a, b in ev:
-            flush.zero_()
-            a.record()
-            fn()
-            b.record()
-        torch.cuda.synchronize()
-        return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        for r in runs:
+            r.step()
 
     def barrier():
         if world > 1:
@@ -284,67 +518,50 @@ def run_dyra(args):
 
     # ---- the timed region: K steps, barrier + sync on both sides
     for _ in range(args.warmup):
-        flush.zero_()
+        timer.flush.zero_()
         step()
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    ms = timed(step, args.steps, 0)
+    ms = timer(step, args.steps, 0)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    status = layer.status()
+    status = max(r.layer.status() for r in runs)
     ms = max_over_ranks(ms, world, dev)
 
-    dense_flops = 2.0 * s.N * s.d_in * s.d_out
+    dense_flops = sum(2.0 * r.s.N * r.s.d_in * r.s.d_out for r in runs)
     value = job_value(dense_flops, world, ms * 1e-3)
     if args.layer_only:  # the timed steps only (for profiler launch lists)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                               "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-                              "config": {"workload": s.name}, "device_status": status,
+                              "config": {"workload": args.workload}, "device_status": status,
                               "layer_only": True}), flush=True)
-        layer.close()
+        for r in runs:
+            r.close()
         if world > 1:
             dist.destroy_process_group()
         return
 
-    # ---- cuBLAS dense X W^T of the same shape
-    Wd = torch.from_numpy(w.weight()).to(dev, td)
-    Yd = torch.empty_like(Y)
-    dense_ms = timed(lambda: torch.matmul(X, Wd.t(), out=Yd), args.steps, 3)
+    # ---- cuBLAS dense X W^T of the same shapes, timed the same way
+    dense_ms = max_over_ranks(timer(lambda: [r.dense_step() for r in runs], args.steps, 3),
+                              world, dev)
+    for r in runs:
+        r.free_dense()
 
-    # ---- per-stage device time (events between the stage launches); the
-    # tensor-core path only (the fp32 path runs plain CUDA-core kernels)
     pk = peaks()
-    flops, bytes_, layer_flops, layer_bytes = algorithmic(s)
-    umma = s.dtype == "bf16"
-    stage_ms = None
+    layer_flops = sum(algorithmic(r.s)[2] for r in runs)
+    layer_bytes = sum(algorithmic(r.s)[3] for r in runs)
+    layer_roof_us = sum(layer_roofline_us(r.s, pk) for r in runs)
+    umma = ss[0].dtype == "bf16"
+    stage_us = None
     if umma:
-        dyra.dyra_debug_set_stage_timing(layer.plan, True)
-        acc = {k: [] for k in dyra.STAGES}
-        for _ in range(max(5, min(args.steps, 50))):
-            flush.zero_()
-            step()
-            for k2, v in dyra.dyra_debug_stage_times(layer.plan).items():
-                acc[k2].append(v)
-        dyra.dyra_debug_set_stage_timing(layer.plan, False)
-        stage_ms = {k2: float(np.mean(v)) for k2, v in acc.items()}
-        dom = max(stage_ms, key=stage_ms.get)
-        t_dom = stage_ms[dom] * 1e-3
-        tensor_t = flops[dom] / (pk["bf16_tflops"] * 1e12)
-        hbm_t = bytes_[dom] / (pk["hbm_gbs"] * 1e9)
-        if tensor_t >= hbm_t:
-            roof = {"bound": "tensor", "achieved": flops[dom] / t_dom / 1e12,
-                    "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": bytes_[dom] / t_dom / 1e9, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["traffic"] = stored_traffic(dom, args.workload)
-        roof["kernel"] = STAGE_KERNELS[dom]
-        roof["peak_source"] = pk["source"] + " burst"
+        st = stage_times(runs, timer, max(5, min(args.steps, 50)))
+        roof = dominant_roofline(runs, st, pk, args.workload)
+        stage_us = ({k: v * 1e3 for k, v in st[0].items()} if len(runs) == 1 else
+                    {r.s.name: {k: v * 1e3 for k, v in t.items()} for r, t in zip(runs, st)})
     else:
         # fp32 FFMA: 148 SMs x 128 lanes x 2 FLOP at the maximum SM clock
         fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -352,85 +569,114 @@ def run_dyra(args):
                 "unit": "TFLOP/s", "traffic": None, "kernel": "whole layer (fp32 CUDA-core path)",
                 "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-    layer_roof_us = max(layer_flops / (pk["bf16_tflops"] * 1e12),
-                        layer_bytes / (pk["hbm_gbs"] * 1e9)) * 1e6
 
     # ---- end to end through the C ABI on host buffers (dyra_forward_batched_host):
     # pinned host X -> device, forward, Y -> pinned host, overlapped by chunks of instances
-    Xh = X.cpu().pin_memory()
-    Yh = torch.empty(Y.shape, dtype=td).pin_memory()
-
-    def e2e_step():
-        layer.forward_host(Xh, B=s.B, T=s.T, Y=Yh)
-
-    e2e_ms = max_over_ranks(timed(e2e_step, args.steps, 2), world, dev)
+    e2e_ms = max_over_ranks(timer(lambda: [r.host_step() for r in runs], args.steps, 2),
+                            world, dev)
     e2e_value = job_value(dense_flops, world, e2e_ms * 1e-3)
 
     # ---- the static-only layer with the same FLOPs (rank r_s, no correction),
     # timed the same way, outside the timed region above
-    rs = static_matched_rank(s)
-    static = dyra.DyraLinear(s.d_in, s.d_out, rs, 0, s.dtype)
-    static.load(torch.as_tensor(np.ascontiguousarray(w.left[:, :rs] * w.sigma[:rs])),
-                torch.as_tensor(np.ascontiguousarray(w.right[:, :rs])), None, None, s.lam)
-    Ys = torch.empty_like(Y)
-    static_ms = max_over_ranks(timed(lambda: static.forward(X, B=s.B, T=s.T, Y=Ys), args.steps, 3),
-                               world, dev)
-    static_status = static.status()
+    statics = []
+    for r in runs:
+        rs = static_matched_rank(r.s)
+        st_layer = dyra.DyraLinear(r.s.d_in, r.s.d_out, rs, 0, r.s.dtype)
+        st_layer.load(torch.as_tensor(np.ascontiguousarray(r.w.left[:, :rs] * r.w.sigma[:rs])),
+                      torch.as_tensor(np.ascontiguousarray(r.w.right[:, :rs])), None, None,
+                      r.s.lam)
+        statics.append((r, rs, st_layer, torch.empty_like(r.Y)))
+    static_ms = max_over_ranks(
+        timer(lambda: [sl.forward(r.X, B=r.s.B, T=r.s.T, Y=Ys) for r, _, sl, Ys in statics],
+              args.steps, 3), world, dev)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": s.dtype, "data": "synthetic (seeded; shapes and statistics "
-        "of the workload, random-orthogonal weights with a power-law spectrum)",
-        "config": {"workload": s.name, "d_in": s.d_in, "d_out": s.d_out, "r": s.r, "k": s.k,
-                   "instances": s.B, "rows_per_instance": s.T, "rows": s.N, "lambda": s.lam,
-                   "l2": "flushed before every step (256 MiB write, outside the step events)",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "vs_baseline": None, "dtype": ss[0].dtype, "data": DATA,
+        "config": config_of(args.workload, world),
         "us_per_layer": ms * 1e3,
+        "us_x_sm_mhz": ms * 1e3 * clk["sm_mhz"] if clk else None,
         "cublas_dense_us": dense_ms * 1e3,
         "speedup_vs_cublas_dense": dense_ms / ms,
         "dyra_tflops_algorithmic": layer_flops / (ms * 1e-3) / 1e12,
         "layer_roofline": {"us": layer_roof_us, "frac": layer_roof_us / (ms * 1e3),
                            "flops": layer_flops, "bytes": layer_bytes},
-        "stage_us": {k2: v * 1e3 for k2, v in stage_ms.items()} if stage_ms else None,
+        "stage_us": stage_us,
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": X.numel() * X.element_size(),
-                "d2h_bytes_per_step": Y.numel() * Y.element_size(), "us": e2e_ms * 1e3},
-        "gpu_launches": ((5 if s.k > 0 else 2) if umma else (7 if s.k > 0 else 2)) * args.steps,
+                "h2d_bytes_per_step": sum(r.X.numel() * r.X.element_size() for r in runs),
+                "d2h_bytes_per_step": sum(r.Y.numel() * r.Y.element_size() for r in runs),
+                "us": e2e_ms * 1e3, "path": "dyra_forward_batched_host (C ABI, pinned host "
+                "buffers, copies inside the timed region)"},
+        "gpu_launches": sum(launches_per_forward(r.s) for r in runs) * args.steps,
         "device_status": status,
         "clocks": clk,
-        "static_matched": {"rank": rs, "flops": 2.0 * s.N * rs * (s.d_in + s.d_out),
+        "static_matched": {"rank": [rs for _, rs, _, _ in statics],
+                           "flops": sum(2.0 * r.s.N * rs * (r.s.d_in + r.s.d_out)
+                                        for r, rs, _, _ in statics),
                            "dyra_flops": layer_flops, "us_per_layer": static_ms * 1e3,
-                           "dyra_us_per_layer": ms * 1e3, "device_status": static_status},
+                           "dyra_us_per_layer": ms * 1e3,
+                           "device_status": max(sl.status() for _, _, sl, _ in statics)},
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"], line["parity"] = cpu_baseline(s, w, Y)
-        line["static_matched"].update(static_errors(s, w, Ys, rs, line["parity"]["rows"]))
-    static.close()
+        line["cpu_baseline"] = cpu_baseline(runs)
+        checks = [oracle_check(r.s, r.w, r.Y) for r in runs]
+        line["parity"] = {"rel_fro_vs_oracle": max(c["rel_fro_vs_oracle"] for c in checks),
+                          "tol": checks[0]["tol"], "rows": [c["rows"] for c in checks],
+                          "oracle_err_weight_only": [c["oracle_err_weight_only"] for c in checks],
+                          "oracle_err_dyra": [c["oracle_err_dyra"] for c in checks]}
+        line["static_matched"].update(static_errors(statics))
+    for _, _, sl, _ in statics:
+        sl.close()
+
+    if rank == 0 and world == 1 and not args.no_per_config:
+        head = (args.workload, {
+            "us": ms * 1e3, "cublas_dense_us": dense_ms * 1e3,
+            "speedup_vs_cublas_dense": dense_ms / ms,
+            "dense_equiv_tflops": dense_flops / (ms * 1e-3) / 1e12,
+            "layer_roofline_us": layer_roof_us, "layer_roofline_frac": layer_roof_us / (ms * 1e3),
+            "device_status": status,
+            "rel_fro_vs_oracle": line.get("parity", {}).get("rel_fro_vs_oracle"),
+            "tol": line.get("parity", {}).get("tol"), "note": "the headline's own timed region"})
+        if "parity" not in line:
+            head = None
+        for r in runs:
+            r.close()
+        runs = []
+        entries, clk_pc = per_config(workload_names(), dev, pk, args.per_config_steps, 5, head)
+        line["per_config"] = entries
+        line["per_config_clocks"] = clk_pc
+        line["per_config_steps"] = args.per_config_steps
+    for r in runs:
+        r.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    layer.close()
     if world > 1:
         dist.destroy_process_group()
 
 
 # ------------------------------------------------------------- oracle ----
 
-def static_errors(s, w, Ys_gpu, rs, rows):
-    """The FLOPs-matched static layer on the oracle's sample rows: its
+def static_errors(statics):
+    """The FLOPs-matched static layers on the oracle's sample rows: their
     approximation error relative to the dense product, and the GPU result
     against the oracle's weight-only product of the same rounded factors."""
     import oracle
-    Xr = oracle.round_to(w.X[:rows], s.dtype)
-    Us = oracle.round_to(w.left[:, :rs] * w.sigma[:rs], s.dtype)
-    Vs = oracle.round_to(w.right[:, :rs], s.dtype)
-    Yo = oracle.weight_only(Xr, Us, Vs)
-    Yd = oracle.dense(Xr, w.weight())
-    Yg = Ys_gpu[:rows].double().cpu().numpy()
-    return {"oracle_err_vs_dense": oracle.rel_fro(Yo, Yd),
-            "rel_fro_vs_oracle": oracle.rel_fro(Yg, Yo), "rows": rows}
+    errs, pars = [], []
+    for r, rs, _, Ys in statics:
+        s, w = r.s, r.w
+        rows = parity_rows(s)
+        Xr = oracle.round_to(w.X[rows], s.dtype)
+        Us = oracle.round_to(w.left[:, :rs] * w.sigma[:rs], s.dtype)
+        Vs = oracle.round_to(w.right[:, :rs], s.dtype)
+        Yo = oracle.weight_only(Xr, Us, Vs)
+        Yd = oracle.dense(Xr, w.weight())
+        Yg = Ys[torch_index(rows, Ys.device)].double().cpu().numpy()
+        errs.append(oracle.rel_fro(Yo, Yd))
+        pars.append(oracle.rel_fro(Yg, Yo))
+    return {"oracle_err_vs_dense": errs, "rel_fro_vs_oracle": max(pars)}
 
 
 def oracle_inputs(s, w):
@@ -439,30 +685,26 @@ def oracle_inputs(s, w):
     return f, [oracle.round_to(a, s.dtype) for a in (w.X, f.U, f.V, f.P, f.W_res)]
 
 
-def cpu_baseline(s, w, Y_gpu):
+def cpu_baseline(runs, budget_s: float = 10.0):
+    """The oracle on the host cores over a bounded sample of whole instances
+    of each layer of the step (about `budget_s` of work in all)."""
     import oracle
-    f, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, w)
     cores = len(os.sched_getaffinity(0))
-    # time the oracle on whole instances until ~10 s of work (at least one)
-    t0 = time.perf_counter()
-    Y1 = oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
-    t1 = time.perf_counter() - t0
-    n_inst = int(max(1, min(s.B, 10.0 // max(t1, 1e-3))))
-    t0 = time.perf_counter()
-    Yo = oracle.inference(Xr[: n_inst * s.T], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
-    t = time.perf_counter() - t0
-    flops = 2.0 * n_inst * s.T * s.d_in * s.d_out
-    base = {"value": flops / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": "%d of %d instances (%d rows), fp64 NumPy, %.2f s" % (
-                n_inst, s.B, n_inst * s.T, t)}
-    Yg = Y_gpu[: n_inst * s.T].double().cpu().numpy()
-    W = w.weight()
-    rep = oracle.error_report(Xr[: n_inst * s.T], W, oracle.Factors(Ur, Vr, Pr, Wr, f.R0), s.lam,
-                              n_inst, s.T, Y=Yo)
-    parity = {"rel_fro_vs_oracle": oracle.rel_fro(Yg, Yo), "tol": 1e-2 if s.dtype == "bf16"
-              else 1e-5, "rows": n_inst * s.T, "oracle_err_weight_only": rep["err_wo"],
-              "oracle_err_dyra": rep["err_dyra"]}
-    return base, parity
+    flops, secs, parts = 0.0, 0.0, []
+    for r in runs:
+        s = r.s
+        _, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, r.w)
+        t0 = time.perf_counter()
+        oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
+        t1 = time.perf_counter() - t0
+        n_inst = int(max(1, min(s.B, (budget_s / len(runs)) // max(t1, 1e-3))))
+        t0 = time.perf_counter()
+        oracle.inference(Xr[: n_inst * s.T], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+        secs += time.perf_counter() - t0
+        flops += 2.0 * n_inst * s.T * s.d_in * s.d_out
+        parts.append("%s: %d of %d instances (%d rows)" % (s.name, n_inst, s.B, n_inst * s.T))
+    return {"value": flops / secs / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "; ".join(parts) + "; fp64 NumPy, %.2f s" % secs}
 
 
 def run_reference(args):
@@ -471,32 +713,44 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    s, w = workload_arrays(args.workload)
-    f, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, w)
+    from synth import generate
+    ss = specs_of(args.workload)
+    prepared = []
+    for s in ss:
+        _, arrs = oracle_inputs(s, generate(s))
+        prepared.append((s, arrs))
     cores = len(os.sched_getaffinity(0))
-    t0 = time.perf_counter()
-    oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
-    t1 = time.perf_counter() - t0
-    # each step a bounded sample of whole instances, sized so that the whole
-    # run (warm-up included) takes about two minutes of host time
-    per_step = 120.0 / (args.steps + args.warmup)
-    n_inst = int(max(1, min(s.B, per_step // max(t1, 1e-4))))
-    rows = n_inst * s.T
+    # each step a bounded sample of whole instances of every layer, sized so
+    # that the whole run (warm-up included) takes about two minutes of host time
+    per_step = 120.0 / (args.steps + args.warmup) / len(prepared)
+    plan = []
+    for s, (Xr, Ur, Vr, Pr, Wr) in prepared:
+        t0 = time.perf_counter()
+        oracle.inference(Xr[: s.T], Ur, Vr, Pr, Wr, s.lam, 1, s.T)
+        t1 = time.perf_counter() - t0
+        n_inst = int(max(1, min(s.B, per_step // max(t1, 1e-4))))
+        plan.append((s, n_inst, (Xr, Ur, Vr, Pr, Wr)))
+
+    def one_step():
+        for s, n, (Xr, Ur, Vr, Pr, Wr) in plan:
+            oracle.inference(Xr[: n * s.T], Ur, Vr, Pr, Wr, s.lam, n, s.T)
+
     for _ in range(args.warmup):
-        oracle.inference(Xr[:rows], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+        one_step()
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.inference(Xr[:rows], Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)
+        one_step()
         times.append(time.perf_counter() - t0)
     t = float(np.mean(times))
-    value = 2.0 * rows * s.d_in * s.d_out / t / 1e12
-    sample = "%d of %d instances (%d rows) per step, fp64 NumPy" % (n_inst, s.B, rows)
+    flops = sum(2.0 * n * s.T * s.d_in * s.d_out for s, n, _ in plan)
+    value = flops / t / 1e12
+    sample = "; ".join("%s: %d of %d instances (%d rows)" % (s.name, n, s.B, n * s.T)
+                       for s, n, _ in plan) + " per step, fp64 NumPy"
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": s.name, "d_in": s.d_in, "d_out": s.d_out, "r": s.r, "k": s.k,
-                       "instances": s.B, "rows_per_instance": s.T, "lambda": s.lam},
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": config_of(args.workload, world),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -508,11 +762,14 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--workload", default=HEADLINE, choices=workload_names())
     ap.add_argument("--impl", choices=("dyra", "reference"), default="dyra")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the sweep over every workload after the headline")
+    ap.add_argument("--per-config-steps", type=int, default=100)
     ap.add_argument("--layer-only", action="store_true",
                     help="time the DyRA steps only: no cuBLAS, stage timing, e2e or CPU legs")
     args = ap.parse_args()

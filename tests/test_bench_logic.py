@@ -6,6 +6,7 @@ import dataclasses
 import os
 import sys
 
+import numpy as np
 import pytest
 
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
@@ -69,3 +70,47 @@ def test_reference_arm_prints_the_contract_line():
 
 def test_reference_arm_other_ranks_do_no_work():
     assert _run_reference({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_reference_arm_config_matches_the_gpu_arm():
+    """Both arms build `config` from the same function, so the driver compares
+    lines on identical configurations."""
+    (line,) = _run_reference({"RANK": "0", "WORLD_SIZE": "1"})
+    assert line["config"] == bench.config_of("tiny_f32", 1)
+
+
+def test_vit_block_runs_the_four_block_linears_in_order():
+    names = [s.name for s in bench.specs_of("vit_block")]
+    assert names == ["vit_block_qkv", "vit_block_proj", "vit_block_fc1", "vit_block_fc2"]
+    c = bench.config_of("vit_block", 1)
+    assert [l["name"] for l in c["layers"]] == names and c["rows"] == 64 * 201
+    assert "vit_block" in bench.workload_names()
+    assert set(CONFIGS) < set(bench.workload_names())
+
+
+def test_headline_is_the_largest_single_gpu_configuration():
+    """The default workload is the configuration with the most dense FLOPs."""
+    big = max(CONFIGS.values(), key=lambda s: s.N * s.d_in * s.d_out)
+    assert bench.HEADLINE == big.name
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_parity_rows_are_valid_and_cover_whole_instances(name):
+    s = CONFIGS[name]
+    rows = bench.parity_rows(s)
+    assert rows.ndim == 1 and len(rows) > 0
+    assert rows.min() >= 0 and rows.max() < s.N and len(np.unique(rows)) == len(rows)
+    if s.N <= 1024:
+        assert len(rows) == s.N
+    elif s.B > 1:
+        # whole leading instances
+        assert len(rows) % s.T == 0 and rows[-1] == len(rows) - 1
+    else:
+        # a single long instance: its first and last rows (the ragged tail) are checked
+        assert rows[0] == 0 and rows[-1] == s.N - 1
+
+
+def test_launch_count_per_forward():
+    assert bench.launches_per_forward(CONFIGS["vit_fc1"]) == 5
+    assert bench.launches_per_forward(dataclasses.replace(CONFIGS["vit_fc1"], k=0)) == 2
+    assert bench.launches_per_forward(CONFIGS["tiny_f32"]) == 7
