@@ -214,8 +214,9 @@ int dyra_forward_weight_only(dyra_plan_t p, const void *X, void *Y, int64_t N,
  *     when the compensated correction is on (a single instance of at most
  *     2048 rows, or DYRA_HILO=1).
  *   - The first call on a device looks the array's device address up
- *     (cudaGetSymbolAddress); make that first call before capturing a stream
- *     into a CUDA graph.
+ *     (cudaGetSymbolAddress), and so does the first call after that device's
+ *     context was destroyed and created again (the array then has a new
+ *     address); make such a call before capturing a stream into a CUDA graph.
  *   - All calls share the one array and it keeps whatever the last call left
  *     there. Nothing in it has to start at zero: every stage overwrites what
  *     the next stage reads. Calls whose execution overlaps on the GPU (other

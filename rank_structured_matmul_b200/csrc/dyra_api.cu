@@ -76,6 +76,7 @@ struct dyra_plan {
   bool stage_timing = false;
   bool stage_recorded = false;
   unsigned long long* trace = nullptr;  // timeline buffer (diagnostics)
+  unsigned long long gram_wait_ns = 0;  // diagnostic wait limit of the Gram stage (0: default)
   // Captured forwards (CUDA graphs) keyed by their arguments; replayed with
   // one cudaGraphLaunch. Invalidated when workspace or factors change.
   struct GraphEntry {
@@ -364,6 +365,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.status = p->status;
     a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
     a.trace = p->trace;
+    a.gram_wait_ns = p->gram_wait_ns;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     a.bias = p->has_bias ? p->bias : nullptr;
@@ -903,6 +905,14 @@ int dyra_debug_set_stage_timing(dyra_plan_t p, int enable) {
   return p->stage_timing || !enable ? DYRA_OK : DYRA_ERR_INVALID_ARG;
 }
 
+int dyra_debug_set_wait_limit(dyra_plan_t p, int stage, uint64_t ns) {
+  if (p == nullptr) return DYRA_ERR_INVALID_ARG;
+  if (stage != 1) return DYRA_ERR_UNSUPPORTED;
+  p->gram_wait_ns = ns;
+  drop_graphs(p);  // the limit is a launch parameter of captured forwards
+  return DYRA_OK;
+}
+
 int dyra_debug_stage_times(dyra_plan_t p, float* ms5) {
   if (p == nullptr || ms5 == nullptr || !p->stage_recorded) return DYRA_ERR_INVALID_ARG;
   DeviceGuard g(p->dev.device);
@@ -986,20 +996,55 @@ namespace {
 constexpr int kMaxScratchDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_addr[kMaxScratchDevices] = {};
+unsigned long long g_scratch_ctx[kMaxScratchDevices] = {};
 
-// Device address of dyra_static_scratch on `device` (which is current),
-// looked up once per device. Host code cannot use the array's name as a
-// device pointer; only this address may be handed to kernels.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be
+// read). A context torn down and created again gets a new id, and the
+// library's device code, the array included, is loaded into it afresh.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of dyra_static_scratch on `device` (which is current).
+// Looked up once per device and context: the first call on a device does the
+// lookup, and so does the first call after that device's context was
+// destroyed and created again (the array then lives at a new address). Host
+// code cannot use the array's name as a device pointer; only this address
+// may be handed to kernels.
 int static_scratch_address(int device, unsigned char** out) {
   if (device < 0 || device >= kMaxScratchDevices) return DYRA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[device] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_addr[device] == nullptr || ctx == 0 || ctx != g_scratch_ctx[device]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, dyra_static_scratch) != cudaSuccess || ptr == nullptr) {
       cudaGetLastError();
       return DYRA_ERR_CUDA;
     }
     g_scratch_addr[device] = ptr;
+    g_scratch_ctx[device] = ctx;
   }
   *out = static_cast<unsigned char*>(g_scratch_addr[device]);
   return DYRA_OK;
