@@ -54,6 +54,17 @@ int dyra_debug_gram_split(dyra_plan_t p, int64_t B, int64_t T, int *splits, int 
  * Stages that did not run (k == 0) report 0. */
 int dyra_debug_set_stage_timing(dyra_plan_t p, int enable);
 
+/* Wait limit of one pipeline wait of a stage, in nanoseconds (0 restores the
+ * default of 2 s). Every wait inside the tensor-core kernels gives up after
+ * its limit: the kernel then raises DYRA_STATUS_WAIT_TIMEOUT, lets the copies
+ * and MMAs it already issued finish, frees its tensor memory and returns, so
+ * the context stays usable and the next forward is correct. A short limit
+ * makes a wait run out on purpose, to test that path. Only stage 1 (gram), a
+ * kernel whose every CTA drains its own copies, takes a limit; other stages
+ * return DYRA_ERR_UNSUPPORTED. The output of a forward whose wait ran out is
+ * not meaningful. */
+int dyra_debug_set_wait_limit(dyra_plan_t p, int stage, uint64_t ns);
+
 /* Milliseconds of each of the 5 stages of the last forward (synchronises on
  * its final event). Returns DYRA_ERR_INVALID_ARG if timing was not enabled. */
 int dyra_debug_stage_times(dyra_plan_t p, float *ms5);

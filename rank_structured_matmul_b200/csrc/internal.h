@@ -86,6 +86,10 @@ struct Bf16Forward {
   // T to about 16 bits
   bool split_t = false;
   void* Tplo = nullptr;  // (B*k) x d_in
+  // Diagnostic: limit of one pipeline wait of the Gram stage in ns (0: the
+  // default sm100::kWaitLimitNs). A short limit makes a wait run out, which
+  // the stage reports as DYRA_STATUS_WAIT_TIMEOUT before returning.
+  unsigned long long gram_wait_ns = 0;
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)

@@ -890,6 +890,7 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   c.trigger_after_wait = 0;
   c.b_parts = 1;
   c.b_part_desc = 0;
+  c.wait_ns = sm100::kWaitLimitNs;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -1196,6 +1197,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
                          static_cast<size_t>(128) * p.kpad * 4)
         return -3;
       if (a.trace) p.c.trace = a.trace + 1 * kTraceCtas * kTraceSlots;
+      if (a.gram_wait_ns) p.c.wait_ns = a.gram_wait_ns;
       if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S)) return -1;
     }
     mark(2);

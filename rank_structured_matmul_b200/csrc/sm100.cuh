@@ -97,18 +97,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 struct WaitCtx {
   volatile int* abort;  // shared memory
   int* status;          // global memory
+  unsigned long long limit_ns;  // how long one wait may take (kWaitLimitNs unless shortened)
 };
 
 // Wait for phase `parity` of `bar`. Returns false if the CTA is aborting or
-// the wait ran past kWaitLimitNs (then the abort word and the status word
-// are raised).
+// the wait ran past w.limit_ns (then the abort word and the status word are
+// raised).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > w.limit_ns) {
       *w.abort = 1;
       atomicOr(w.status, kStatusTimeout);
       return false;

@@ -81,6 +81,9 @@ struct GemmCommon {
   // the smem descriptor step from one part to the next
   uint32_t b_parts;
   uint64_t b_part_desc;
+  // limit of one pipeline wait in ns (sm100::kWaitLimitNs; a diagnostic may
+  // shorten it to make a wait run out). Drains keep kWaitLimitNs.
+  unsigned long long wait_ns;
 };
 
 // Issues one stage's ks MMAs (K = 16 each) back to back. The tensor pipe idles
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (c.trigger_after_wait) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
-  WaitCtx w{abort_flag, c.status};
+  WaitCtx w{abort_flag, c.status, c.wait_ns};
   // producer state kept for the drain after the closing barrier
   uint32_t last_phase[kMaxStages];
   uint32_t issued = 0;

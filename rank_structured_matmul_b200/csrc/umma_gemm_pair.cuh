@@ -93,7 +93,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (c.trigger_after_wait) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
-  WaitCtx w{abort_flag, c.status};
+  WaitCtx w{abort_flag, c.status, c.wait_ns};
   // producer state kept for the drain after the closing barrier
   uint32_t last_phase[kMaxStages];
   uint32_t issued = 0;

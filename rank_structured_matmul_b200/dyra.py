@@ -56,6 +56,7 @@ SIGNATURES = {
     "dyra_debug_set_stage_timing": (_i, [_vp, _i]),
     "dyra_debug_stage_times": (_i, [_vp, ctypes.POINTER(ctypes.c_float)]),
     "dyra_debug_set_trace": (_i, [_vp, _i]),
+    "dyra_debug_set_wait_limit": (_i, [_vp, _i, ctypes.c_uint64]),
     "dyra_debug_trace_bytes": (ctypes.c_size_t, []),
     "dyra_debug_trace_copy": (_i, [_vp, _vp, ctypes.c_size_t]),
 }
@@ -211,6 +212,11 @@ def dyra_debug_gram_split(plan: int, B: int, T: int):
 def dyra_debug_set_stage_timing(plan: int, enable: bool) -> None:
     _check(lib().dyra_debug_set_stage_timing(plan, int(bool(enable))),
            "dyra_debug_set_stage_timing")
+
+
+def dyra_debug_set_wait_limit(plan: int, stage: int, ns: int) -> None:
+    """Wait limit of one pipeline wait of `stage` in ns (0: the default)."""
+    _check(lib().dyra_debug_set_wait_limit(plan, int(stage), int(ns)), "dyra_debug_set_wait_limit")
 
 
 def dyra_debug_stage_times(plan: int):

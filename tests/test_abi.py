@@ -117,10 +117,12 @@ def _declared_signatures():
 def _kind(c_param):
     """The ctypes class a C parameter declaration needs."""
     t = re.sub(r"\b[A-Za-z_][A-Za-z_0-9]*$", "", c_param).strip()  # drop the parameter name
-    if "*" in t or t.endswith("_t") and t not in ("int64_t", "size_t", "dyra_dtype_t"):
+    if "*" in t or t.endswith("_t") and t not in ("int64_t", "uint64_t", "size_t", "dyra_dtype_t"):
         return "ptr"
-    return {"int": "int", "dyra_dtype_t": "int", "int64_t": "int64", "float": "float",
-            "size_t": "size"}[t]
+    # uint64_t and size_t are the same 64-bit unsigned type on LP64 Linux
+    # (ctypes.c_uint64 is ctypes.c_size_t there)
+    return {"int": "int", "dyra_dtype_t": "int", "int64_t": "int64", "uint64_t": "size",
+            "float": "float", "size_t": "size"}[t]
 
 
 def test_binding_signatures_match_the_header():
