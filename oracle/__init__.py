@@ -10,6 +10,7 @@ oracle.monarch holds the Monarch static part (DyRA App. B) and DyRA on top of it
 from .dyra_oracle import (  # noqa: F401
     Factors,
     als_half_steps,
+    als_updates,
     als_inference,
     dense,
     error_report,

@@ -234,18 +234,37 @@ def als_half_steps(Xb: np.ndarray, W_res: np.ndarray, R0: np.ndarray, lam: float
     return pairs
 
 
-def als_inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, W_res: np.ndarray,
-                  R0: np.ndarray, lam: float, B: int, T: int, t: float) -> np.ndarray:
-    """DyRA with t ALS iterations per instance ([DyRA] Sec. 3.3, Fig. 9 right).
+def als_updates(t: float, schedule: str = "pairs") -> int:
+    """How many ALS updates (half-steps) t iterations run.
 
-    One iteration is a left and a right update (Alg. 1 is t = 1); a half
-    iteration ends on a left update, so t = 1.5 runs L, R, L and t = 2 runs
-    L, R, L, R. The output of instance b is (X_b V) U^T + L R with the last
-    pair. t = 0 is the weight-only layer.
+    "pairs": an iteration is a left and a right update, as Alg. 1 runs for
+    t = 1, and a half iteration ends on a left update; t = 1.5 runs L, R, L.
+    "printed": Sec. 3.3 spells t = 1.5 as the five updates L, R, L, R, L. It
+    gives no other half-integer sequence, so here a half-integer t runs
+    ceil(t) pairs and then one more left update; integer t agree with "pairs".
     """
     steps = int(round(2 * t))
     if steps != 2 * t or steps < 0:
         raise ValueError("t must be a non-negative multiple of 0.5")
+    if schedule == "pairs" or steps % 2 == 0:
+        return steps
+    if schedule == "printed":
+        return steps + 2
+    raise ValueError("unknown schedule %r" % schedule)
+
+
+def als_inference(X: np.ndarray, U: np.ndarray, V: np.ndarray, W_res: np.ndarray,
+                  R0: np.ndarray, lam: float, B: int, T: int, t: float,
+                  schedule: str = "pairs") -> np.ndarray:
+    """DyRA with t ALS iterations per instance ([DyRA] Sec. 3.3, Fig. 9 right).
+
+    One iteration is a left and a right update (Alg. 1 is t = 1); a half
+    iteration ends on a left update, so t = 1.5 runs L, R, L and t = 2 runs
+    L, R, L, R. With schedule="printed", t = 1.5 runs the sequence the text
+    prints, L, R, L, R, L (see als_updates). The output of instance b is
+    (X_b V) U^T + L R with the last pair. t = 0 is the weight-only layer.
+    """
+    steps = als_updates(t, schedule)
     X = np.asarray(X, dtype=np.float64)
     if X.shape[0] != B * T:
         raise ValueError("X has %d rows, expected B*T = %d" % (X.shape[0], B * T))

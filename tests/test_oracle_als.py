@@ -363,3 +363,45 @@ def test_planted_als_mistakes_are_caught(monkeypatch, target, mutant):
         except (AssertionError, np.linalg.LinAlgError, ValueError):
             failures += 1
     assert failures > 0, "no pin catches the planted mistake %s" % mutant.__name__
+
+
+# ------------------------------------------- the printed t = 1.5 sequence ----
+
+def test_printed_schedule_counts():
+    """Sec. 3.3 prints t = 1.5 as L, R, L, R, L: five updates starting and
+    ending with a left update. Integer t are the same under both schedules."""
+    assert orc.als_updates(1.5, "printed") == 5
+    assert orc.als_updates(1.5, "pairs") == 3
+    for t in (0, 1, 2, 3):
+        assert orc.als_updates(t, "printed") == orc.als_updates(t, "pairs") == 2 * t
+    with pytest.raises(ValueError):
+        orc.als_updates(1.25)
+    with pytest.raises(ValueError):
+        orc.als_updates(1.5, "other")
+
+
+def test_printed_t15_is_two_pairs_then_a_left_update():
+    """Under the printed schedule, t = 1.5 is t = 2 followed by one more left
+    update: the right factor is t = 2's, and the left factor is the ridge
+    minimiser against it (zero gradient), so the fit is never worse than t = 2's."""
+    rng = np.random.default_rng(11)
+    T, d_in, d_out, k, lam = 40, 12, 10, 3, 1e-3
+    Xb = rng.standard_normal((T, d_in))
+    W_res = rng.standard_normal((d_out, d_in))
+    R0 = np.linalg.qr(rng.standard_normal((d_out, k)))[0].T
+    E = Xb @ W_res.T
+    pairs = orc.als_half_steps(Xb, W_res, R0, lam, 5)
+    L5, R5 = pairs[-1]
+    L4, R4 = pairs[3]
+    np.testing.assert_array_equal(R5, R4)
+    grad = (L5 @ R5 - E) @ R5.T + lam * L5
+    assert np.abs(grad).max() < 1e-9 * max(1.0, np.abs(E).max())
+    obj = lambda L, R: np.sum((E - L @ R) ** 2) + lam * (np.sum(L ** 2) + np.sum(R ** 2))
+    assert obj(L5, R5) <= obj(L4, R4) + 1e-12
+    U = rng.standard_normal((d_out, 2))
+    V = rng.standard_normal((d_in, 2))
+    Y = orc.als_inference(Xb, U, V, W_res, R0, lam, 1, T, 1.5, schedule="printed")
+    np.testing.assert_allclose(Y, (Xb @ V) @ U.T + L5 @ R5, rtol=1e-12, atol=1e-12)
+    Y2 = orc.als_inference(Xb, U, V, W_res, R0, lam, 1, T, 2.0, schedule="printed")
+    np.testing.assert_allclose(Y2, orc.als_inference(Xb, U, V, W_res, R0, lam, 1, T, 2.0),
+                               rtol=0, atol=0)
