@@ -147,12 +147,41 @@ int dyra_set_linear(dyra_plan_t p, const void *bias, float alpha, dyra_stream_t 
  * L_b = X_b (R_b W_res)^T (R_b R_b^T + lambda I)^-1, so it costs one more pass
  * over X. Default 2.
  *   half_steps : 2 .. 64, else DYRA_ERR_INVALID_ARG.
- * Only the CUDA-core kernels (fp32 plans, or bf16 plans under
- * DYRA_KERNELS=simt) run more than two; the tensor-core kernels return
- * DYRA_ERR_UNSUPPORTED, as does dyra_forward_batched_noalloc, for any other
- * count. Takes effect at the next forward.
+ * Every kernel set runs any count. With more than two the bf16 tensor-core
+ * forward forms each R update explicitly (the Gram sums kept in fp32 and the
+ * small system solved from the left, then the rank-k GEMM) and each further
+ * L update as X_b (R_b W_res)^T solved against R_b R_b^T + lambda I, one
+ * stage after another without the compensated correction; the workspace then
+ * holds B*k*(d_in + k) floats for the Gram sums. dyra_forward_batched_noalloc
+ * returns DYRA_ERR_UNSUPPORTED for any count but 2. Takes effect at the next
+ * forward.
  */
 int dyra_set_als_steps(dyra_plan_t p, int half_steps);
+
+/* Solvers of the per-instance k x k system of the correction. */
+enum {
+  DYRA_SOLVER_LDL = 0,           /* blocked LDL^T factorisation (the default) */
+  DYRA_SOLVER_NEWTON_SCHULZ = 1  /* Newton-Schulz iteration for the inverse */
+};
+
+/*
+ * Solver of the small ridge system (L_b^T L_b + lambda I) of the correction
+ * ([DyRA] Sec. 2.4: a Cholesky solve for small correction ranks, a
+ * Newton-Schulz iterative solver for larger ones).
+ *   solver    : DYRA_SOLVER_LDL, or DYRA_SOLVER_NEWTON_SCHULZ: from
+ *               X_0 = I / ||G||_inf the iteration X <- X (2 I - G X) runs until
+ *               the largest entry of I - G X is below 1e-6, stops shrinking
+ *               near fp32 rounding, or max_iters steps have run; an instance
+ *               whose residual is not below 1e-2 then gets no correction and
+ *               raises DYRA_STATUS_NONPOSITIVE_PIVOT.
+ *   max_iters : 1 .. 200 (the iteration's limit; ignored by DYRA_SOLVER_LDL).
+ * Newton-Schulz runs in fp32 on the CUDA cores, one block per instance, and
+ * needs a bf16 tensor-core plan with 1 <= k <= 64 (else DYRA_ERR_UNSUPPORTED);
+ * it is used by the one-step forward (dyra_set_als_steps(p, 2)). Errors:
+ * DYRA_ERR_INVALID_ARG for a NULL plan or a value out of range. Takes effect at
+ * the next forward.
+ */
+int dyra_set_solver(dyra_plan_t p, int solver, int max_iters);
 
 /*
  * dyra_forward_batched on HOST buffers: X (B*T x d_in) and Y (B*T x d_out) in

@@ -62,9 +62,12 @@ struct dyra_plan {
   void* Ctlo = nullptr;  // bf16, compensated correction: d_out x (B*k)
   void* Tplo = nullptr;  // bf16, compensated correction: (B*k) x d_in
   size_t cap_Z = 0, cap_L = 0, cap_TG = 0, cap_Tp = 0, cap_Ct = 0, cap_MD = 0;
-  // ALS updates per forward (dyra_set_als_steps; CUDA-core plans beyond 2) and
-  // the buffers the further L updates use
+  // ALS updates per forward (dyra_set_als_steps) and the buffers the further
+  // L updates of the CUDA-core kernels use
   int als_half_steps = 2;
+  // solver of the small systems (dyra_set_solver)
+  int solver = DYRA_SOLVER_LDL;
+  int ns_iters = 40;
   void* Lt = nullptr;    // (B*k) x T
   void* P2 = nullptr;    // (B*k) x d_in
   float* TG2 = nullptr;  // B x k x (T + k)
@@ -169,7 +172,8 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T);
 
 // Whether a tensor-core forward of B x T rows uses the compensated correction.
 bool use_hilo(const dyra_plan* p, int64_t B, int64_t T) {
-  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->monarch || p->hilo_mode == 0)
+  if (p->k == 0 || p->dtype != DYRA_BF16 || p->force_simt || p->monarch || p->hilo_mode == 0 ||
+      p->als_half_steps != 2)
     return false;
   return p->hilo_mode == 1 || (B == 1 && T <= 2048);
 }
@@ -222,7 +226,9 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
     if (k > 0) {
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
       void* tg = p->TG;
-      rc = grow(tg, p->cap_TG, static_cast<size_t>(B) * k * k * sizeof(float));
+      // more ALS iterations keep L_b^T X_b and L_b^T L_b together in fp32
+      const size_t tg_cols = p->als_half_steps > 2 ? static_cast<size_t>(p->d_in) + k : k;
+      rc = grow(tg, p->cap_TG, static_cast<size_t>(B) * k * tg_cols * sizeof(float));
       p->TG = static_cast<float*>(tg);
       if (rc) return rc;
       if ((rc = grow(p->Tp, p->cap_Tp, static_cast<size_t>(B) * k * p->d_in * es))) return rc;
@@ -366,6 +372,9 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.stage_events = p->stage_timing ? p->stage_ev : nullptr;
     a.trace = p->trace;
     a.gram_wait_ns = p->gram_wait_ns;
+    a.half_steps = p->als_half_steps;
+    a.solver = p->solver;
+    a.ns_iters = p->ns_iters;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     a.bias = p->has_bias ? p->bias : nullptr;
@@ -662,10 +671,21 @@ int dyra_set_linear(dyra_plan_t p, const void* bias, float alpha, dyra_stream_t 
   return DYRA_OK;
 }
 
+int dyra_set_solver(dyra_plan_t p, int solver, int max_iters) {
+  if (p == nullptr || (solver != DYRA_SOLVER_LDL && solver != DYRA_SOLVER_NEWTON_SCHULZ) ||
+      max_iters < 1 || max_iters > 200)
+    return DYRA_ERR_INVALID_ARG;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
+  if (solver == DYRA_SOLVER_NEWTON_SCHULZ && (!umma || p->k == 0 || p->k > 64))
+    return DYRA_ERR_UNSUPPORTED;
+  p->solver = solver;
+  p->ns_iters = max_iters;
+  drop_graphs(p);  // captured forwards hold the old solver
+  return DYRA_OK;
+}
+
 int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
   if (p == nullptr || half_steps < 2 || half_steps > 64) return DYRA_ERR_INVALID_ARG;
-  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
-  if (umma && half_steps != 2) return DYRA_ERR_UNSUPPORTED;
   p->als_half_steps = half_steps;
   drop_graphs(p);  // captured forwards hold the old count
   return DYRA_OK;
@@ -1158,6 +1178,8 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
     a.bias = p->has_bias ? p->bias : nullptr;
     a.alpha = p->alpha;
+    a.solver = p->solver;
+    a.ns_iters = p->ns_iters;
     rc = dyra::launch_bf16_forward(a, p->dev, s);
   } else if (p->dtype == DYRA_BF16) {
     dyra::SimtForward<__nv_bfloat16> a;

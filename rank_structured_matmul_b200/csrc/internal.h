@@ -90,6 +90,14 @@ struct Bf16Forward {
   // default sm100::kWaitLimitNs). A short limit makes a wait run out, which
   // the stage reports as DYRA_STATUS_WAIT_TIMEOUT before returning.
   unsigned long long gram_wait_ns = 0;
+  // Solver of the small systems: 0 the blocked LDL^T factorisation, 1 the
+  // Newton-Schulz iteration (at most ns_iters steps; k <= 64)
+  int solver = 0;
+  int ns_iters = 40;
+  // ALS updates ([DyRA] Sec. 3.3): 2 is Alg. 1; more run the explicit
+  // alternating chain (launch_bf16_als). TG then needs B x k x (d_in + k)
+  // floats.
+  int half_steps = 2;
 };
 
 constexpr int kTraceCtas = 256;  // trace rows per stage (grids are at most this wide)
@@ -154,18 +162,26 @@ template <typename T>
 int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo& dev, cudaStream_t s);
 
 // Solve (L^T L + lambda I) T' = T for every instance from the Gram partials
-// (the CUDA-core path): every solve block factors G_b itself.
+// (the CUDA-core path, and the right updates of further ALS iterations on the
+// tensor-core path): every solve block factors G_b itself; alpha scales T'.
 template <typename TOut>
 int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
-                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace = nullptr);
+                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace = nullptr,
+                 float alpha = 1.f);
 
 // Floats per instance of the factor records for correction rank k (0 when
 // k > 64: the solve then factors G_b itself).
 int factor_record_floats(int k);
 
+// Newton-Schulz inverse of G_b + lambda I per instance (k <= 64), published
+// as factor records behind the instance flags for launch_ltilde's mode 2.
+int launch_ns_inverse(const float* G, int64_t B, int k, float lambda, int max_iters, float* MD,
+                      int* flags, int* status, cudaStream_t s);
+
 // L~ = L G^-1 per instance, over L (bf16 plans; kernels_simt.cu). mode 0: every
 // block factors G_b; 1: the instance's first block factors it and publishes a
-// record (MD, flags). G: B x k x k fp32 (G_b without the ridge).
+// record (MD, flags); 2: every block reads the records another kernel
+// published (k <= 64). G: B x k x k fp32 (G_b without the ridge).
 // defer_wait (with pdl): the grid launched just before waited for the one
 // that wrote G and L before letting this one start; this grid then waits
 // for it only before its blocks exit.

@@ -56,7 +56,7 @@ constexpr int kSolveThreads = 128;
 template <typename TOut>
 __global__ void __launch_bounds__(kSolveThreads)
     solve_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
-                 TOut* __restrict__ Tp, int* status) {
+                 TOut* __restrict__ Tp, int* status, float alpha) {
   extern __shared__ float sm[];
   const int ldg = k + 1;
   float* G = sm;                     // k x (k+1): lower triangle becomes R
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kSolveThreads)
     const bool zero = bad != 0;
     for (int i = 0; i < k; ++i)
       Tp[(static_cast<size_t>(b) * k + i) * d_in + col] =
-          from_f<TOut>(zero ? 0.f : Ycol[i * kSolveThreads + tid]);
+          from_f<TOut>(zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid]);
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kSolveThreads)
 // the other splits are added afterwards.
 constexpr int kSolveThreads2 = 256;
 constexpr int kSolveCols = 128;  // columns of T_b per CTA
-enum SolveMode { kSolveSelf = 0, kSolveShared = 1 };
+enum SolveMode { kSolveSelf = 0, kSolveShared = 1, kSolveGiven = 2 };
 
 template <int KMAX>
 struct SolveSmem {
@@ -162,7 +162,7 @@ template <typename TOut, int KMAX>
 __global__ void __launch_bounds__(kSolveThreads2)
     solve_ldl_kernel(const float* __restrict__ TG, int S, int B, int k, int d_in, float lambda,
                      TOut* __restrict__ Tp, int* status,
-                     unsigned long long* trace) {
+                     unsigned long long* trace, float alpha) {
   using Sm = SolveSmem<KMAX>;
   constexpr int LDG = LdlBlockScratch<KMAX>::LD;
   extern __shared__ __align__(16) unsigned char smem_bytes[];
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kSolveThreads2)
     TOut* dst = Tp + (static_cast<size_t>(b) * k + i) * d_in + col;
 #pragma unroll
     for (int v = 0; v < 4; ++v)
-      if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : acc[u][v]);
+      if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : alpha * acc[u][v]);
   }
   if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
@@ -330,7 +330,9 @@ __global__ void __launch_bounds__(kSolveThreads2)
 // once (fp32) and the block's rows are multiplied by it in a register-tiled
 // product (G_b is symmetric, so a row times G_b^-1 is G_b^-1 times the row).
 // Who factors: every CTA (kSolveSelf), or the instance's first CTA, which
-// publishes G_b^-1 and a failure flag for the others (kSolveShared).
+// publishes G_b^-1 and a failure flag for the others (kSolveShared), or no
+// CTA: another kernel (the Newton-Schulz iteration) published the records
+// (kSolveGiven).
 // defer_wait: the grid launched just before this one (the GEMM for Q) has
 // already waited for the Gram stage before letting this grid start, so this
 // grid reads G and L at once and waits for that grid only before it exits
@@ -383,9 +385,9 @@ __global__ void __maxnreg__(152)
   __nv_bfloat16* const Vs = KMAX <= 32 ? sm.Vs : reinterpret_cast<__nv_bfloat16*>(sm.ldl.Gs);
   const int b = blockIdx.x, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const bool factors = MODE == kSolveSelf || blockIdx.y == 0;
-  float* rec = MODE == kSolveShared ? MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>()
-                                    : nullptr;
+  const bool factors = MODE == kSolveSelf || (MODE == kSolveShared && blockIdx.y == 0);
+  float* rec = MODE != kSolveSelf ? MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>()
+                                  : nullptr;
   unsigned long long* const tr =
       trace ? trace + (blockIdx.y * gridDim.x + blockIdx.x) % kTraceCtas * kTraceSlots : nullptr;
   if (tr && tid == 0) tr[0] = sm100::globaltimer_ns();
@@ -579,6 +581,139 @@ __global__ void __maxnreg__(152)
   if (tr && tid == 0) tr[8] = sm100::globaltimer_ns();
 }
 
+// Newton-Schulz inverse of G_b + lambda I, one CTA per instance ([DyRA]
+// Sec. 2.4 names a Newton-Schulz iterative solver for larger correction ranks
+// in place of the sequential Cholesky solve). From X_0 = I / ||G||_inf, whose
+// spectrum lies in (0, 1], the iteration X <- X (2 I - G X) squares the
+// residual I - G X at every step; it stops when the largest entry of the
+// residual is below 1e-6, when it stops shrinking near the fp32 rounding
+// floor, or after max_iters steps. The result is published as the solve's
+// factor record of the instance (G_b^-1 row-major with stride KMAX, then a
+// failure flag) behind its ready flag, which the kSolveGiven solve reads. A
+// residual that is not finite, or is not below 1e-2 at the end, flags the
+// instance: its correction becomes zero and DYRA_STATUS_NONPOSITIVE_PIVOT is
+// raised.
+constexpr int kNsThreads = 256;
+template <int KMAX>
+__host__ __device__ constexpr int ns_ld() {
+  return KMAX + 4;  // row stride of the kernel's three KMAX x KMAX tiles
+}
+template <int KMAX>
+constexpr size_t ns_smem_bytes() {
+  return 3 * sizeof(float) * KMAX * ns_ld<KMAX>();
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kNsThreads)
+    ns_inverse_kernel(const float* __restrict__ G, int k, float lambda, int max_iters, float* MD,
+                      int* flags, int* status) {
+  constexpr int LD = ns_ld<KMAX>();
+  constexpr int TPR = KMAX / 16;  // each thread owns a TPR x TPR block of the product
+  extern __shared__ __align__(16) float ns_smem[];
+  float* const Gs = ns_smem;          // G + lambda I, zero beyond k
+  float* const Xs = Gs + KMAX * LD;   // the iterate X
+  float* const Ps = Xs + KMAX * LD;   // G X
+  __shared__ float red[kNsThreads / 32];
+  __shared__ float resid;
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int ti = tid / 16, tj = tid % 16;  // thread block row / column
+  sm100::pdl_launch_dependents();
+  const float* Gb = G + static_cast<size_t>(b) * k * k;
+  for (int e = tid; e < KMAX * KMAX; e += kNsThreads) {
+    const int i = e / KMAX, q = e % KMAX;
+    Gs[i * LD + q] = i < k && q < k ? __ldcg(Gb + i * k + q) + (i == q ? lambda : 0.f) : 0.f;
+  }
+  __syncthreads();
+  // ||G||_inf: the largest absolute row sum
+  float rs = 0.f;
+  if (tid < k)
+    for (int q = 0; q < k; ++q) rs += fabsf(Gs[tid * LD + q]);
+  for (int o = 16; o > 0; o >>= 1) rs = fmaxf(rs, __shfl_xor_sync(0xffffffffu, rs, o));
+  if ((tid & 31) == 0) red[tid >> 5] = rs;
+  __syncthreads();
+  float gnorm = 0.f;
+  for (int w = 0; w < kNsThreads / 32; ++w) gnorm = fmaxf(gnorm, red[w]);
+  const float x0 = gnorm > 0.f && isfinite(gnorm) ? 1.f / gnorm : 0.f;
+  for (int e = tid; e < KMAX * KMAX; e += kNsThreads) {
+    const int i = e / KMAX, q = e % KMAX;
+    Xs[i * LD + q] = i == q && i < k ? x0 : 0.f;
+  }
+  __syncthreads();
+  // C = A B for the thread's block (rows TPR*ti.., columns TPR*tj..)
+  auto block_product = [&](const float* A, const float* Bm, float (&c)[TPR][TPR]) {
+#pragma unroll
+    for (int u = 0; u < TPR; ++u)
+#pragma unroll
+      for (int v = 0; v < TPR; ++v) c[u][v] = 0.f;
+    for (int q = 0; q < k; ++q) {
+      float a[TPR], bv[TPR];
+#pragma unroll
+      for (int u = 0; u < TPR; ++u) a[u] = A[(TPR * ti + u) * LD + q];
+#pragma unroll
+      for (int v = 0; v < TPR; ++v) bv[v] = Bm[q * LD + TPR * tj + v];
+#pragma unroll
+      for (int u = 0; u < TPR; ++u)
+#pragma unroll
+        for (int v = 0; v < TPR; ++v) c[u][v] = fmaf(a[u], bv[v], c[u][v]);
+    }
+  };
+  float prev = 3.4e38f, r = 3.4e38f;
+  for (int it = 0; it < max_iters; ++it) {
+    float c[TPR][TPR];
+    block_product(Gs, Xs, c);  // P = G X
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < TPR; ++u)
+#pragma unroll
+      for (int v = 0; v < TPR; ++v) {
+        const int i = TPR * ti + u, q = TPR * tj + v;
+        Ps[i * LD + q] = c[u][v];
+        if (i < k && q < k) {
+          const float d = (i == q ? 1.f : 0.f) - c[u][v];
+          mx = isfinite(d) ? fmaxf(mx, fabsf(d)) : 3.4e38f;
+        }
+      }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    if (tid == 0) {
+      float m = 0.f;
+      for (int w = 0; w < kNsThreads / 32; ++w) m = fmaxf(m, red[w]);
+      resid = m;
+    }
+    __syncthreads();
+    r = resid;
+    if (r < 1e-6f || (r < 1e-2f && r > 0.5f * prev)) break;
+    prev = r;
+    block_product(Xs, Ps, c);  // X P
+    __syncthreads();           // every read of X done
+#pragma unroll
+    for (int u = 0; u < TPR; ++u)
+#pragma unroll
+      for (int v = 0; v < TPR; ++v) {
+        const int i = TPR * ti + u, q = TPR * tj + v;
+        Xs[i * LD + q] = 2.f * Xs[i * LD + q] - c[u][v];
+      }
+    __syncthreads();
+  }
+  const bool bad = !(r < 1e-2f);
+  float* rec = MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
+  for (int e = tid; e < KMAX * KMAX; e += kNsThreads) {
+    const int i = e / KMAX, q = e % KMAX;
+    rec[e] = Xs[i * LD + q];
+  }
+  if (tid == 0) rec[KMAX * KMAX] = bad ? 1.f : 0.f;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    sm100::st_release_gpu(flags + b, 1);
+    if (bad) atomicOr(status, sm100::kStatusPivot);
+  }
+  // the grid before this one (the GEMM for Q) is complete before this one
+  // is, so the stages after the solve may rely on both
+  sm100::pdl_wait();
+}
+
 // General variant of the same (any k <= 128): every CTA factors G_b itself
 // (Cholesky G_b = R R^T in shared memory) and solves R R^T w = l for 128 rows
 // of L_b, one per thread.
@@ -735,7 +870,8 @@ __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P,
 
 template <typename TOut, int KMAX>
 int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, int splits, int64_t B, int k,
-                     int d_in, float lambda, TOut* Tp, int* status, unsigned long long* trace) {
+                     int d_in, float lambda, TOut* Tp, int* status, unsigned long long* trace,
+                     float alpha) {
   auto kfn = solve_ldl_kernel<TOut, KMAX>;
   static KernelSetup setup;
   const int d = setup_device();
@@ -753,14 +889,14 @@ int launch_solve_ldl(cudaLaunchConfig_t& cfg, const float* TG, int splits, int64
   cfg.blockDim = dim3(kSolveThreads2);
   cfg.dynamicSmemBytes = sizeof(SolveSmem<KMAX>);
   return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
-                            status, trace) == cudaSuccess
+                            status, trace, alpha) == cudaSuccess
              ? 0
              : -1;
 }
 
 template <typename TOut>
 int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float lambda, TOut* Tp,
-                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace) {
+                 int* status, cudaStream_t s, bool pdl, unsigned long long* trace, float alpha) {
   if (B == 0 || k == 0) return 0;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -770,9 +906,11 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
   cfg.numAttrs = pdl ? 1 : 0;
   cfg.stream = s;
   if (k <= 32)
-    return launch_solve_ldl<TOut, 32>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace);
+    return launch_solve_ldl<TOut, 32>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace,
+                                      alpha);
   if (k <= 64)
-    return launch_solve_ldl<TOut, 64>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace);
+    return launch_solve_ldl<TOut, 64>(cfg, TG, splits, B, k, d_in, lambda, Tp, status, trace,
+                                      alpha);
   const size_t smem = (static_cast<size_t>(k) * (k + 1) + static_cast<size_t>(k) * kSolveThreads) *
                       sizeof(float);
   auto kfn = solve_kernel<TOut>;
@@ -789,7 +927,7 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
   cfg.blockDim = dim3(kSolveThreads);
   cfg.dynamicSmemBytes = smem;
   return cudaLaunchKernelEx(&cfg, kfn, TG, splits, static_cast<int>(B), k, d_in, lambda, Tp,
-                            status) == cudaSuccess
+                            status, alpha) == cudaSuccess
              ? 0
              : -1;
 }
@@ -834,13 +972,35 @@ int launch_ltilde_fast(cudaLaunchConfig_t& cfg, const float* G, __nv_bfloat16* L
              : -1;
 }
 
+int launch_ns_inverse(const float* G, int64_t B, int k, float lambda, int max_iters, float* MD,
+                      int* flags, int* status, cudaStream_t s) {
+  if (B == 0 || k == 0) return 0;
+  if (k > 64 || MD == nullptr || flags == nullptr || B > 2147483647) return -1;
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (setup.smem[d].load() == 0) {
+    if (cudaFuncSetAttribute(ns_inverse_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(ns_smem_bytes<64>())) != cudaSuccess)
+      return -1;
+    setup.smem[d].store(static_cast<uint32_t>(ns_smem_bytes<64>()));
+  }
+  if (k <= 32)
+    ns_inverse_kernel<32><<<static_cast<unsigned>(B), kNsThreads, ns_smem_bytes<32>(), s>>>(
+        G, k, lambda, max_iters, MD, flags, status);
+  else
+    ns_inverse_kernel<64><<<static_cast<unsigned>(B), kNsThreads, ns_smem_bytes<64>(), s>>>(
+        G, k, lambda, max_iters, MD, flags, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int mode, int64_t B,
                   int64_t T, int k, float lambda, float alpha, int* status, cudaStream_t s, bool pdl,
                   bool defer_wait, unsigned long long* trace) {
   const int dw = pdl && defer_wait ? 1 : 0;
   if (B == 0 || T == 0 || k == 0) return 0;
   if (k % 8 != 0) return -1;  // bf16 plans: 16-byte rows of L
-  if (mode == kSolveShared && (MD == nullptr || flags == nullptr)) return -1;
+  if (mode != kSolveSelf && (MD == nullptr || flags == nullptr || k > 64)) return -1;
   if ((T + ltilde_rows_per_block(k) - 1) / ltilde_rows_per_block(k) > 65535 || B > 2147483647)
     return -1;
   auto* Lb = static_cast<__nv_bfloat16*>(L);
@@ -856,12 +1016,18 @@ int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int
     return mode == kSolveShared
                ? launch_ltilde_fast<32, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                       alpha, status, dw, trace)
+           : mode == kSolveGiven
+               ? launch_ltilde_fast<32, kSolveGiven>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                     alpha, status, dw, trace)
                : launch_ltilde_fast<32, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                     alpha, status, dw, trace);
   if (k <= 64)
     return mode == kSolveShared
                ? launch_ltilde_fast<64, kSolveShared>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                       alpha, status, dw, trace)
+           : mode == kSolveGiven
+               ? launch_ltilde_fast<64, kSolveGiven>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
+                                                     alpha, status, dw, trace)
                : launch_ltilde_fast<64, kSolveSelf>(cfg, G, Lb, Lo, MD, flags, B, T, k, lambda,
                                                     alpha, status, dw, trace);
   const size_t smem = ltilde_smem_bytes(k);
@@ -886,10 +1052,10 @@ int launch_ltilde(const float* G, void* L, void* Llo, float* MD, int* flags, int
 }
 
 template int launch_solve<float>(const float*, int, int64_t, int, int, float, float*, int*,
-                                 cudaStream_t, bool, unsigned long long*);
+                                 cudaStream_t, bool, unsigned long long*, float);
 template int launch_solve<__nv_bfloat16>(const float*, int, int64_t, int, int, float,
                                          __nv_bfloat16*, int*, cudaStream_t, bool,
-                                         unsigned long long*);
+                                         unsigned long long*, float);
 
 template <typename T>
 int launch_pack_vp(const T* V, const T* P, T* VPt, int d_in, int r, int k, cudaStream_t s) {
@@ -940,7 +1106,8 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
       if (gemm(k, k, Tr, Lp, lq, lm, lb, Lp, lm, lq, lb, a.TG + a.d_in, J, 1,
                static_cast<int64_t>(k) * J, Bn, 0, s))
         return -1;
-      if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr))
+      if (launch_solve<T>(a.TG, 1, a.B, k, a.d_in, a.lambda, a.Tp, a.status, s, false, nullptr,
+                          1.f))
         return -1;
       // R = T' W_res^T  (B*k x d_out)
       if (gemm(Bn * k, a.d_out, a.d_in, a.Tp, a.d_in, 1, 0, a.W_res, 1, a.d_in, 0, a.Cm, a.d_out,
@@ -963,7 +1130,8 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
                static_cast<int64_t>(k) * J, Bn, 0, s))
         return -1;
       // L_b^T = (R_b R_b^T + lambda I)^-1 (X_b P2_b^T)^T  -> Lt[b*k + i][t]
-      if (launch_solve<T>(a.TG2, 1, a.B, k, Tr, a.lambda, a.Lt, a.status, s, false, nullptr))
+      if (launch_solve<T>(a.TG2, 1, a.B, k, Tr, a.lambda, a.Lt, a.status, s, false, nullptr,
+                          1.f))
         return -1;
       Lp = a.Lt;
       lm = 1;

@@ -383,9 +383,16 @@ struct GramPolicy {
     CUtensorMap tmLb;  // (k, T, B),    box (w, 64, 1),  w*2-byte swizzle (B role)
     int d_in, k, kpad, w, nbox_b, T, B, S, Ts, mtx, mt_total;
     uint32_t b_layout;
+    // 1: the X view holds one instance that every instance b reads (its third
+    // coordinate is 0 for all b), e.g. W_res for the L update of more ALS
+    // iterations, where "T" counts d_out rows
+    int x_inst_fixed;
     __nv_bfloat16* Tb;  // (B*k) x d_in
     __nv_bfloat16* Tlo;  // (B*k) x d_in: the bf16 rounding errors of Tb, or nullptr
     float* G;           // B x k x k
+    // when set, T and G go here instead, in fp32, as B x k x (d_in + k):
+    // row i of instance b holds (L_b^T X_b)[i][0..d_in) then (L_b^T L_b)[i][0..k)
+    float* TGf;
   };
   struct Tile {
     int mt, b, s, t0, t1;
@@ -422,8 +429,9 @@ struct GramPolicy {
     const int row = t.t0 + it * 64;
     if (t.mt < p.mtx) {
       const int j0 = t.mt * 128;
-      tma_load_3d(sa, &p.tmX, bar, j0, row, t.b);
-      tma_load_3d(sa + 8192u, &p.tmX, bar, j0 + 64, row, t.b);
+      const int bx = p.x_inst_fixed ? 0 : t.b;
+      tma_load_3d(sa, &p.tmX, bar, j0, row, bx);
+      tma_load_3d(sa + 8192u, &p.tmX, bar, j0 + 64, row, bx);
     } else {
       const int i0 = (t.mt - p.mtx) * 128;
       tma_load_3d(sa, &p.tmLa, bar, i0, row, t.b);
@@ -447,6 +455,23 @@ struct GramPolicy {
   template <int n>
   static __device__ __forceinline__ void store_row(const Params& p, const Tile& t, int row, int i0,
                                                    const float (&v)[n]) {
+    if (p.TGf != nullptr) {
+      const int J = p.d_in + p.k;
+      float* inst = p.TGf + static_cast<size_t>(t.b) * p.k * J;
+      int col;  // column of instance b's k x J block that this thread's row feeds
+      if (t.mt < p.mtx) {
+        col = t.mt * 128 + row;
+        if (col >= p.d_in) return;
+      } else {
+        const int i2 = (t.mt - p.mtx) * 128 + row;
+        if (i2 >= p.k) return;
+        col = p.d_in + i2;
+      }
+#pragma unroll
+      for (int u = 0; u < n; ++u)
+        if (i0 + u < p.k) inst[static_cast<size_t>(i0 + u) * J + col] = v[u];
+      return;
+    }
     if (t.mt < p.mtx) {
       const int j = t.mt * 128 + row;
       if (j >= p.d_in) return;
@@ -716,6 +741,84 @@ struct OutPolicy {
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
   static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx& e) { store_drain(e); }
+};
+
+// ============================================================= x . rw^T ====
+// The left update of a further ALS iteration ([DyRA] Eq. 4) needs, per
+// instance b, P2_b = X_b (R_b W_res)^T (T x k). Tile: 128 rows of X (through
+// the (d_in, T, B) view, so each instance segment of a tile that straddles
+// instances is masked by the copy's out-of-bounds fill, as in the output
+// stage) times the k x d_in block of R W_res of that instance (K-major B
+// operand, rows b*k ..), K = d_in per segment. The accumulator's first k
+// columns leave as bf16 rows of P2 (N x k) through 16-byte stores.
+struct XRwPolicy {
+  struct Params {
+    GemmCommon c;
+    CUtensorMap tmX;   // (d_in, T, B), box (64, 128, 1)
+    CUtensorMap tmRW;  // (d_in, B*k),  box (64, kpad)
+    __nv_bfloat16* P2;  // N x k
+    int N, d_in, k, kpad, T, B, nkd;
+  };
+  struct Tile {
+    int m0, b_lo, nseg;
+  };
+  static constexpr uint32_t kEpiSmemBytes = 0;
+
+  static __device__ __forceinline__ void prefetch(const Params& p) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmRW);
+  }
+  static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
+    t.m0 = tile * 128;
+    t.b_lo = t.m0 / p.T;
+    const int b_hi = min(p.B - 1, (t.m0 + 127) / p.T);
+    t.nseg = b_hi - t.b_lo + 1;
+  }
+  static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
+    return t.nseg * p.nkd;
+  }
+  static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
+                                              uint32_t sb, uint32_t bar) {
+    const int seg = it / p.nkd;
+    const int ch = it - seg * p.nkd;
+    const int b = t.b_lo + seg;
+    tma_load_3d(sa, &p.tmX, bar, ch * 64, t.m0 - b * p.T, b);
+    tma_load_2d(sb, &p.tmRW, bar, ch * 64, b * p.k);
+  }
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
+    const int ch = it % p.nkd;
+    return min(4, ceil_div_dev(p.d_in - ch * 64, 16));
+  }
+  static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
+    return kmajor_desc(a, ks);
+  }
+  static __device__ __forceinline__ uint64_t bdesc(const Params&, uint32_t b, int ks) {
+    return kmajor_desc(b, ks);
+  }
+  static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
+                                                  EpiCtx& e) {
+    const int row = t.m0 + e.row;
+    for (int cc = 0; cc < p.kpad; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + cc, v);
+      tmem_ld_wait();
+      if (row >= p.N) continue;
+      __nv_bfloat16* dst = p.P2 + static_cast<size_t>(row) * p.k + cc;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        if (cc + 8 * c8 >= p.k) break;  // k is a multiple of 8
+        uint4 q;
+        q.x = pack_bf16x2(f32(v[8 * c8 + 0]), f32(v[8 * c8 + 1]));
+        q.y = pack_bf16x2(f32(v[8 * c8 + 2]), f32(v[8 * c8 + 3]));
+        q.z = pack_bf16x2(f32(v[8 * c8 + 4]), f32(v[8 * c8 + 5]));
+        q.w = pack_bf16x2(f32(v[8 * c8 + 6]), f32(v[8 * c8 + 7]));
+        *reinterpret_cast<uint4*>(dst + 8 * c8) = q;
+      }
+    }
+  }
+  static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
+  static __device__ __forceinline__ void finish(const Params&, int, uint32_t, unsigned long long*) {}
+  static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
 };
 
 // ============================================================ proj, pairs ====
@@ -1084,195 +1187,449 @@ void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits
   *splits = static_cast<int>((blocks + per - 1) / per);
 }
 
+namespace {
+
+// One Gram stage (GramPolicy) over a pair of 3-D row views: X (d_in, rows,
+// instances of X) and L (k, rows, B), strides in bytes. The one-step forward
+// runs it over (X_b, L_b); the L update of further ALS iterations over
+// (W_res, R_b^T), with rows = d_out.
+struct GramStage {
+  const void* X;
+  uint64_t xd[3], xs[2];
+  int x_inst_fixed;
+  const void* L;
+  uint64_t ld[3], ls[2];
+  int d_in, k, rows, B, S, Ts;
+  __nv_bfloat16* Tb;
+  __nv_bfloat16* Tlo;
+  float* G;
+  float* TGf;
+  unsigned long long* trace;
+  unsigned long long wait_ns;
+};
+
+int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cudaStream_t s,
+                      bool pdl) {
+  GramPolicy::Params p;
+  p.d_in = g.d_in;
+  p.k = g.k;
+  p.kpad = g.k <= 32 ? 32 : ceil_div(g.k, 64) * 64;
+  p.w = std::min(p.kpad, 64);
+  p.nbox_b = p.kpad / p.w;
+  p.T = g.rows;
+  p.B = g.B;
+  p.S = g.S;
+  p.Ts = g.Ts;
+  p.mtx = ceil_div(g.d_in, 128);
+  p.mt_total = p.mtx + ceil_div(g.k, 128);
+  p.x_inst_fixed = g.x_inst_fixed;
+  p.Tb = g.Tb;
+  p.Tlo = g.Tlo;
+  p.G = g.G;
+  p.TGf = g.TGf;
+  p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
+  uint32_t bx[3] = {64, 64, 1};
+  if (!encode_tmap_bf16(&p.tmX, g.X, 3, g.xd, g.xs, bx, 128)) return -2;
+  if (!encode_tmap_bf16(&p.tmLa, g.L, 3, g.ld, g.ls, bx, 128)) return -2;
+  uint32_t bl[3] = {static_cast<uint32_t>(p.w), 64, 1};
+  if (!encode_tmap_bf16(&p.tmLb, g.L, 3, g.ld, g.ls, bl, p.w * 2)) return -2;
+  const int tiles = p.mt_total * p.B * p.S;
+  const uint32_t smem =
+      setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
+                               p.kpad, true, true, status, dev);
+  if (!smem) return -3;
+  // split rows keep a 128 x kpad fp32 partial in the operand stages
+  if (p.S > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
+                     static_cast<size_t>(128) * p.kpad * 4)
+    return -3;
+  p.c.trace = g.trace;
+  if (g.wait_ns) p.c.wait_ns = g.wait_ns;
+  return launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S) ? -1 : 0;
+}
+
+// The Gram stage of the layer: L_b^T [X_b | L_b] per instance, L = a.L.
+GramStage layer_gram(const Bf16Forward& a) {
+  GramStage g = {};
+  g.X = a.X;
+  g.xd[0] = static_cast<uint64_t>(a.d_in);
+  g.xd[1] = static_cast<uint64_t>(a.T);
+  g.xd[2] = static_cast<uint64_t>(a.B);
+  g.xs[0] = static_cast<uint64_t>(a.d_in) * 2;
+  g.xs[1] = static_cast<uint64_t>(a.d_in) * 2 * static_cast<uint64_t>(a.T);
+  g.L = a.L;
+  g.ld[0] = static_cast<uint64_t>(a.k);
+  g.ld[1] = static_cast<uint64_t>(a.T);
+  g.ld[2] = static_cast<uint64_t>(a.B);
+  g.ls[0] = static_cast<uint64_t>(a.k) * 2;
+  g.ls[1] = static_cast<uint64_t>(a.k) * 2 * static_cast<uint64_t>(a.T);
+  g.d_in = a.d_in;
+  g.k = a.k;
+  g.rows = static_cast<int>(a.T);
+  g.B = static_cast<int>(a.B);
+  g.S = a.splits;
+  g.Ts = a.split_rows;
+  return g;
+}
+
+// The rank-k factor GEMM C^T = W_res Tb^T (d_out x B*k) from the K-major
+// (B*k) x d_in operand Tb (with its low part Tlo when split_t), optionally
+// also storing the low parts of C^T (Ctlo, hilo).
+struct RFactorStage {
+  const void* Tb;
+  const void* Tlo;
+  void* Ct;
+  void* Ctlo;
+  bool split_t, hilo;
+  int smem_cap;
+  unsigned long long* trace;
+};
+
+int launch_rfactor_stage(const RFactorStage& r, const Bf16Forward& a, const DeviceInfo& dev,
+                         cudaStream_t s, bool pdl) {
+  RFactorPolicy::Params p;
+  const int Bk = static_cast<int>(a.B) * a.k;
+  p.d_in = a.d_in;
+  p.d_out = a.d_out;
+  p.Bk = Bk;
+  p.bn = std::min(256, (pick_bn(Bk) + 63) / 64 * 64);  // whole 64-column store boxes
+  p.n_tiles_n = ceil_div(Bk, p.bn);
+  uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.d_out)};
+  uint64_t sw[1] = {static_cast<uint64_t>(a.d_in) * 2};
+  uint32_t bw[2] = {64, 128};
+  if (!encode_tmap_bf16(&p.tmW, a.W_res, 2, dw, sw, bw, 128)) return -2;
+  // Pairs halve each SM's share of T' per k-step; they need enough pair
+  // tiles to keep the SMs busy and an even column tile.
+  const bool rf_pairs = a.use_pairs && p.bn % 32 == 0 && p.bn >= 64 &&
+                        ceil_div(a.d_out, 256) * p.n_tiles_n >= dev.sm_count / 4;
+  uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
+  uint32_t bt[2] = {64, static_cast<uint32_t>(rf_pairs ? p.bn / 2 : p.bn)};
+  if (!encode_tmap_bf16(&p.tmT, r.Tb, 2, dt, sw, bt, 128)) return -2;
+  p.split_t = r.split_t ? 1 : 0;
+  if (r.split_t) {
+    if (!encode_tmap_bf16(&p.tmTlo, r.Tlo, 2, dt, sw, bt, 128)) return -2;
+  } else {
+    p.tmTlo = p.tmT;
+  }
+  const uint32_t parts = r.split_t ? 2u : 1u;  // B operands per stage
+  uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
+  uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
+  uint32_t bc[2] = {64, 128};
+  if (!encode_tmap_bf16(&p.tmC, r.Ct, 2, dc, sc, bc, 128)) return -2;
+  p.hilo = r.hilo ? 1 : 0;
+  if (r.hilo) {
+    if (!encode_tmap_bf16(&p.tmClo, r.Ctlo, 2, dc, sc, bc, 128)) return -2;
+  } else {
+    p.tmClo = p.tmC;
+  }
+  if (rf_pairs) {
+    const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
+    const uint32_t part_bytes = static_cast<uint32_t>(p.bn / 2) * 128u;
+    const uint32_t smem =
+        setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
+                                        false, a.status, dev, r.smem_cap);
+    if (!smem) return -3;
+    p.c.b_parts = parts;
+    p.c.b_part_desc = part_bytes >> 4;
+    p.c.trigger_after_wait = 1;
+    p.c.idesc = idesc_bf16(256, p.bn, false, false);
+    p.c.trace = r.trace;
+    return launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+  }
+  const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
+  const uint32_t part_bytes = static_cast<uint32_t>(p.bn) * 128u;
+  const uint32_t smem =
+      setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false, false,
+                                  a.status, dev, r.smem_cap);
+  if (!smem) return -3;
+  p.c.b_parts = parts;
+  p.c.b_part_desc = part_bytes >> 4;
+  p.c.trigger_after_wait = 1;
+  p.c.trace = r.trace;
+  return launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+}
+
+// The output stage Y = Z U^T (+ bias) + sum_b mask_b(L) C_b with the
+// correction's left factor L (N x k) and right factor C^T (d_out x B*k)
+// (k = 0: the static part alone), with their low parts when hilo.
+int launch_out_stage(const void* L, const void* Llo, const void* Ct, const void* Ctlo, bool hilo,
+                     int k, const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+  const int64_t N = a.B * a.T;
+  OutPolicy::Params p;
+  p.N = static_cast<int>(N);
+  p.r = a.r;
+  p.k = k;
+  p.T = static_cast<int>(a.T);
+  p.B = static_cast<int>(a.B);
+  p.bn = a.d_out % 256 == 0 ? 256 : (a.d_out % 128 == 0 ? 128 : 64);
+  if (a.d_out < p.bn) p.bn = 64;
+  p.n_tiles_n = ceil_div(a.d_out, p.bn);
+  p.nkz = ceil_div(a.r, 64);
+  p.nkl = k > 0 ? ceil_div(k, 64) : 0;
+  p.bias = static_cast<const __nv_bfloat16*>(a.bias);
+  p.d_out = a.d_out;
+
+  uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
+  uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+  uint32_t bz[2] = {64, 128};
+  if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bz, 128)) return -2;
+  uint64_t du[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(a.d_out)};
+  const bool use_pairs = a.use_pairs && p.bn >= 128;
+  const uint32_t bbox = static_cast<uint32_t>(use_pairs ? p.bn / 2 : p.bn);
+  uint32_t bu[2] = {64, bbox};
+  if (!encode_tmap_bf16(&p.tmU, a.U, 2, du, sz, bu, 128)) return -2;
+  if (k > 0) {
+    uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
+                      static_cast<uint64_t>(a.B)};
+    uint64_t sl[2] = {static_cast<uint64_t>(k) * 2,
+                      static_cast<uint64_t>(k) * 2 * static_cast<uint64_t>(a.T)};
+    uint32_t bl[3] = {64, 128, 1};
+    if (!encode_tmap_bf16(&p.tmL, L, 3, dl, sl, bl, 128)) return -2;
+    const int64_t Bk = a.B * k;
+    uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
+    uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
+    uint32_t bc[2] = {64, bbox};
+    if (!encode_tmap_bf16(&p.tmC, Ct, 2, dc, sc, bc, 128)) return -2;
+    if (hilo) {
+      if (!encode_tmap_bf16(&p.tmLlo, Llo, 3, dl, sl, bl, 128)) return -2;
+      if (!encode_tmap_bf16(&p.tmClo, Ctlo, 2, dc, sc, bc, 128)) return -2;
+    } else {
+      p.tmLlo = p.tmL;
+      p.tmClo = p.tmC;
+    }
+  } else {
+    p.tmL = p.tmZ;
+    p.tmC = p.tmU;
+    p.tmLlo = p.tmZ;
+    p.tmClo = p.tmU;
+  }
+  p.hilo = k > 0 && hilo ? 1 : 0;
+  uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
+  uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
+  uint32_t by[2] = {64, 128};
+  if (!encode_tmap_bf16(&p.tmY, a.Y, 2, dy, sy, by, 128)) return -2;
+  unsigned long long* tr = a.trace ? a.trace + 4 * kTraceCtas * kTraceSlots : nullptr;
+  if (use_pairs) {
+    const int tiles = ceil_div(N, 256) * p.n_tiles_n;
+    const uint32_t smem = setup_common<OutPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
+                                                      p.bn, false, false, a.status, dev);
+    if (!smem) return -3;
+    p.c.idesc = idesc_bf16(256, p.bn, false, false);
+    p.c.trace = tr;
+    return launch_gemm_pair<OutPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+  }
+  const int tiles = ceil_div(N, 128) * p.n_tiles_n;
+  const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
+                                                false, a.status, dev);
+  if (!smem) return -3;
+  p.c.trace = tr;
+  return launch_gemm<OutPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+}
+
+// P2_b = X_b (RW_b)^T over P2 (N x k), RW: (B*k) x d_in (XRwPolicy).
+int launch_xrw_stage(const void* RW, void* P2, const Bf16Forward& a, const DeviceInfo& dev,
+                     cudaStream_t s, bool pdl) {
+  const int64_t N = a.B * a.T;
+  XRwPolicy::Params p;
+  p.N = static_cast<int>(N);
+  p.d_in = a.d_in;
+  p.k = a.k;
+  p.kpad = ceil_div(a.k, 16) * 16;
+  p.T = static_cast<int>(a.T);
+  p.B = static_cast<int>(a.B);
+  p.nkd = ceil_div(a.d_in, 64);
+  p.P2 = static_cast<__nv_bfloat16*>(P2);
+  uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
+                    static_cast<uint64_t>(a.B)};
+  uint64_t sx[2] = {static_cast<uint64_t>(a.d_in) * 2,
+                    static_cast<uint64_t>(a.d_in) * 2 * static_cast<uint64_t>(a.T)};
+  uint32_t bx[3] = {64, 128, 1};
+  if (!encode_tmap_bf16(&p.tmX, a.X, 3, dx, sx, bx, 128)) return -2;
+  uint64_t dr[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.B * a.k)};
+  uint64_t sr[1] = {static_cast<uint64_t>(a.d_in) * 2};
+  uint32_t br[2] = {64, static_cast<uint32_t>(p.kpad)};
+  if (!encode_tmap_bf16(&p.tmRW, RW, 2, dr, sr, br, 128)) return -2;
+  const int tiles = static_cast<int>(ceil_div(N, static_cast<int64_t>(128)));
+  const uint32_t smem = setup_common<XRwPolicy>(p.c, tiles, 128 * 128,
+                                                static_cast<uint32_t>(p.kpad) * 128, p.kpad,
+                                                false, false, a.status, dev);
+  if (!smem) return -3;
+  return launch_gemm<XRwPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+}
+
+int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* counters,
+                      const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+  const int64_t N = a.B * a.T;
+  const int rk = a.r + a.k;  // VPt rows always hold [V | P]
+  ProjPolicy::Params p;
+  const ProjShape ps =
+      proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count, a.proj_pair_min_tiles);
+  p.N = static_cast<int>(N);
+  p.d_in = a.d_in;
+  p.r = a.r;
+  p.k = k_eff;
+  p.tma_store = ps.tma_store;
+  p.bn = ps.bn;
+  p.n_tiles_n = ps.n_tiles_n;
+  p.Z = static_cast<__nv_bfloat16*>(a.Z);
+  p.L = static_cast<__nv_bfloat16*>(a.L);
+  const bool records = p.k > 0 && MD && counters && factor_record_floats(p.k) > 0;
+  p.cnt = records ? counters : nullptr;
+  p.ncnt = static_cast<int>(a.B);
+  p.ksplit = ps.ksplit;
+  p.kper = ps.kper;
+  uint64_t dx[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(N)};
+  uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
+  uint32_t bx[2] = {64, 128};
+  if (!encode_tmap_bf16(&p.tmX, a.X, 2, dx, sx, bx, 128)) return -2;
+  uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(rk)};
+  uint32_t bw[2] = {64, static_cast<uint32_t>(ps.pairs ? p.bn / 2 : p.bn)};
+  if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
+  uint32_t bs[2] = {64, 128};
+  uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
+  uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+  if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bs, 128)) return -2;
+  if (p.k > 0) {
+    uint64_t dl[2] = {static_cast<uint64_t>(p.k), static_cast<uint64_t>(N)};
+    uint64_t sl[1] = {static_cast<uint64_t>(p.k) * 2};
+    if (!encode_tmap_bf16(&p.tmL, a.L, 2, dl, sl, bs, 128)) return -2;
+  } else {
+    p.tmL = p.tmZ;
+  }
+  unsigned long long* tr = a.trace ? a.trace + 0 * kTraceCtas * kTraceSlots : nullptr;
+  if (ps.pairs) {
+    const uint32_t smem = setup_common<ProjPairPolicy>(p.c, ps.tiles, 128 * 128,
+                                                       (p.bn / 2) * 128, p.bn, false, false,
+                                                       a.status, dev);
+    if (!smem) return -3;
+    p.c.idesc = idesc_bf16(256, p.bn, false, false);
+    p.c.trace = tr;
+    return launch_gemm_pair<ProjPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+  }
+  const uint32_t smem = setup_common<ProjPolicy>(p.c, ps.tiles * p.ksplit, 128 * 128,
+                                                 p.bn * 128, p.bn, false, false, a.status, dev);
+  if (!smem) return -3;
+  // split-K keeps a 128 x bn fp32 partial in the operand stages
+  if (p.ksplit > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
+                          static_cast<size_t>(128) * p.bn * 4)
+    return -3;
+  p.c.trace = tr;
+  return launch_gemm<ProjPolicy>(p, smem, dev, s, pdl, p.ksplit) ? -1 : 0;
+}
+
+// half_steps >= 3 alternating updates ([DyRA] Sec. 2.2, Eq. 4-5 with the
+// ridge of footnote 2; Sec. 3.3 compares 1, 1.5 and 2 iterations), from
+// Alg. 1's first left factor L = X P. Each right update is formed
+// explicitly, R_b = (L_b^T L_b + lambda I)^-1 (L_b^T X_b) W_res^T: the Gram
+// stage writes L_b^T X_b and L_b^T L_b in fp32, the solve applies the
+// inverse from the left (T'_b, bf16) and the rank-k GEMM gives R^T = W_res
+// T'^T. Each further left update is L_b = X_b (R_b W_res)^T (R_b R_b^T +
+// lambda I)^-1: the Gram stage over (W_res, R_b^T), whose rows are the d_out
+// output features, gives R_b W_res and R_b R_b^T, the X (R W_res)^T GEMM
+// writes P2 over L, and the solve turns it into L in place. The output stage
+// adds L_b R_b of the last pair; the correction weight alpha scales the last
+// update. Stages follow one another in stream order.
+int launch_bf16_als(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s) {
+  const bool pdl = false;
+  const int k = a.k;
+  auto mark = [&](int i) {
+    if (a.stage_events) cudaEventRecord(a.stage_events[i], s);
+  };
+  mark(0);
+  if (launch_proj_stage(a, k, nullptr, nullptr, dev, s, pdl)) return -1;
+  mark(1);
+  int splits2 = 1, rows2 = 64;
+  gram_split(a.d_out, a.B, a.d_in, k, dev.sm_count, &splits2, &rows2);
+  for (int h = 2; h <= a.half_steps; ++h) {
+    const float w = h == a.half_steps ? a.alpha : 1.f;
+    if (h % 2 == 0) {  // right update from the current L (over a.L)
+      GramStage g = layer_gram(a);
+      g.TGf = a.TG;
+      if (launch_gram_stage(g, a.status, dev, s, pdl)) return -1;
+      if (launch_solve<__nv_bfloat16>(a.TG, 1, a.B, k, a.d_in, a.lambda,
+                                      static_cast<__nv_bfloat16*>(a.Tp), a.status, s, pdl,
+                                      nullptr, w))
+        return -1;
+      RFactorStage r = {a.Tp, nullptr, a.Ct, nullptr, false, false, 0, nullptr};
+      if (launch_rfactor_stage(r, a, dev, s, pdl)) return -1;
+    } else {  // left update from the current R (R^T over a.Ct)
+      GramStage g = {};
+      g.X = a.W_res;
+      g.xd[0] = static_cast<uint64_t>(a.d_in);
+      g.xd[1] = static_cast<uint64_t>(a.d_out);
+      g.xd[2] = 1;
+      g.xs[0] = static_cast<uint64_t>(a.d_in) * 2;
+      g.xs[1] = static_cast<uint64_t>(a.d_in) * 2 * static_cast<uint64_t>(a.d_out);
+      g.x_inst_fixed = 1;
+      g.L = a.Ct;  // R_b^T: element (j, b*k + i) of the d_out x B*k matrix
+      g.ld[0] = static_cast<uint64_t>(k);
+      g.ld[1] = static_cast<uint64_t>(a.d_out);
+      g.ld[2] = static_cast<uint64_t>(a.B);
+      g.ls[0] = static_cast<uint64_t>(a.B) * k * 2;
+      g.ls[1] = static_cast<uint64_t>(k) * 2;
+      g.d_in = a.d_in;
+      g.k = k;
+      g.rows = a.d_out;
+      g.B = static_cast<int>(a.B);
+      g.S = splits2;
+      g.Ts = rows2;
+      g.Tb = static_cast<__nv_bfloat16*>(a.Tp);  // R_b W_res
+      g.G = a.TG;                                // R_b R_b^T
+      if (launch_gram_stage(g, a.status, dev, s, pdl)) return -1;
+      if (launch_xrw_stage(a.Tp, a.L, a, dev, s, pdl)) return -1;
+      if (launch_ltilde(a.TG, a.L, nullptr, nullptr, nullptr, 0, a.B, a.T, k, a.lambda, w,
+                        a.status, s, pdl, /*defer_wait=*/false, nullptr))
+        return -1;
+    }
+  }
+  mark(2);
+  mark(3);
+  mark(4);
+  if (launch_out_stage(a.L, nullptr, a.Ct, nullptr, false, k, a, dev, s, pdl)) return -1;
+  mark(5);
+  return 0;
+}
+
+}  // namespace
+
 int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s) {
   const int64_t N = a.B * a.T;
   if (N == 0) return 0;
   const int k = a.weight_only ? 0 : a.k;
-  const int rk = a.r + a.k;  // VPt rows always hold [V | P]
+  if (k > 0 && a.half_steps > 2) return launch_bf16_als(a, dev, s);
   const bool pdl = true;
   auto mark = [&](int i) {
     if (a.stage_events) cudaEventRecord(a.stage_events[i], s);
   };
   mark(0);
-
-  // ---------------------------------------------------------------- proj
-  {
-    ProjPolicy::Params p;
-    const int k_eff = a.weight_only ? 0 : a.k;
-    const ProjShape ps =
-        proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count, a.proj_pair_min_tiles);
-    p.N = static_cast<int>(N);
-    p.d_in = a.d_in;
-    p.r = a.r;
-    p.k = k_eff;
-    p.tma_store = ps.tma_store;
-    p.bn = ps.bn;
-    p.n_tiles_n = ps.n_tiles_n;
-    p.Z = static_cast<__nv_bfloat16*>(a.Z);
-    p.L = static_cast<__nv_bfloat16*>(a.L);
-    const bool records = p.k > 0 && a.MD && a.counters && factor_record_floats(p.k) > 0;
-    p.cnt = records ? a.counters : nullptr;
-    p.ncnt = static_cast<int>(a.B);
-    p.ksplit = ps.ksplit;
-    p.kper = ps.kper;
-    uint64_t dx[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(N)};
-    uint64_t sx[1] = {static_cast<uint64_t>(a.d_in) * 2};
-    uint32_t bx[2] = {64, 128};
-    if (!encode_tmap_bf16(&p.tmX, a.X, 2, dx, sx, bx, 128)) return -2;
-    uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(rk)};
-    uint32_t bw[2] = {64, static_cast<uint32_t>(ps.pairs ? p.bn / 2 : p.bn)};
-    if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
-    uint32_t bs[2] = {64, 128};
-    uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
-    uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
-    if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bs, 128)) return -2;
-    if (p.k > 0) {
-      uint64_t dl[2] = {static_cast<uint64_t>(p.k), static_cast<uint64_t>(N)};
-      uint64_t sl[1] = {static_cast<uint64_t>(p.k) * 2};
-      if (!encode_tmap_bf16(&p.tmL, a.L, 2, dl, sl, bs, 128)) return -2;
-    } else {
-      p.tmL = p.tmZ;
-    }
-    if (ps.pairs) {
-      const uint32_t smem = setup_common<ProjPairPolicy>(p.c, ps.tiles, 128 * 128,
-                                                         (p.bn / 2) * 128, p.bn, false, false,
-                                                         a.status, dev);
-      if (!smem) return -3;
-      p.c.idesc = idesc_bf16(256, p.bn, false, false);
-      if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
-      if (launch_gemm_pair<ProjPairPolicy>(p, smem, dev, s, pdl)) return -1;
-    } else {
-      const uint32_t smem = setup_common<ProjPolicy>(p.c, ps.tiles * p.ksplit, 128 * 128,
-                                                     p.bn * 128, p.bn, false, false, a.status, dev);
-      if (!smem) return -3;
-      // split-K keeps a 128 x bn fp32 partial in the operand stages
-      if (p.ksplit > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
-                              static_cast<size_t>(128) * p.bn * 4)
-        return -3;
-      if (a.trace) p.c.trace = a.trace + 0 * kTraceCtas * kTraceSlots;
-      if (launch_gemm<ProjPolicy>(p, smem, dev, s, pdl, p.ksplit)) return -1;
-    }
-  }
+  if (launch_proj_stage(a, k, a.MD, a.counters, dev, s, pdl)) return -1;
   mark(1);
 
   if (k > 0) {
-    // -------------------------------------------------------------- gram
-    {
-      GramPolicy::Params p;
-      p.d_in = a.d_in;
-      p.k = a.k;
-      p.kpad = a.k <= 32 ? 32 : ceil_div(a.k, 64) * 64;
-      p.w = std::min(p.kpad, 64);
-      p.nbox_b = p.kpad / p.w;
-      p.T = static_cast<int>(a.T);
-      p.B = static_cast<int>(a.B);
-      p.S = a.splits;
-      p.Ts = a.split_rows;
-      p.mtx = ceil_div(a.d_in, 128);
-      p.mt_total = p.mtx + ceil_div(a.k, 128);
-      p.Tb = static_cast<__nv_bfloat16*>(a.Tp);
-      p.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
-      p.G = a.TG;
-      p.b_layout = p.w == 64 ? kLayoutSw128 : kLayoutSw64;  // w is 32 or 64
-      uint64_t dx[3] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.T),
-                        static_cast<uint64_t>(a.B)};
-      uint64_t sx[2] = {static_cast<uint64_t>(a.d_in) * 2,
-                        static_cast<uint64_t>(a.d_in) * 2 * static_cast<uint64_t>(a.T)};
-      uint32_t bx[3] = {64, 64, 1};
-      if (!encode_tmap_bf16(&p.tmX, a.X, 3, dx, sx, bx, 128)) return -2;
-      uint64_t dl[3] = {static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.T),
-                        static_cast<uint64_t>(a.B)};
-      uint64_t sl[2] = {static_cast<uint64_t>(a.k) * 2,
-                        static_cast<uint64_t>(a.k) * 2 * static_cast<uint64_t>(a.T)};
-      if (!encode_tmap_bf16(&p.tmLa, a.L, 3, dl, sl, bx, 128)) return -2;
-      uint32_t bl[3] = {static_cast<uint32_t>(p.w), 64, 1};
-      if (!encode_tmap_bf16(&p.tmLb, a.L, 3, dl, sl, bl, p.w * 2)) return -2;
-      const int tiles = p.mt_total * p.B * p.S;
-      const uint32_t smem =
-          setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
-                                   p.kpad, true, true, a.status, dev);
-      if (!smem) return -3;
-      // split rows keep a 128 x kpad fp32 partial in the operand stages
-      if (p.S > 1 && static_cast<size_t>(p.c.stages) * (p.c.a_stage_bytes + p.c.b_stage_bytes) <
-                         static_cast<size_t>(128) * p.kpad * 4)
-        return -3;
-      if (a.trace) p.c.trace = a.trace + 1 * kTraceCtas * kTraceSlots;
-      if (a.gram_wait_ns) p.c.wait_ns = a.gram_wait_ns;
-      if (launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S)) return -1;
-    }
+    GramStage g = layer_gram(a);
+    g.Tb = static_cast<__nv_bfloat16*>(a.Tp);
+    g.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
+    g.G = a.TG;
+    g.trace = a.trace ? a.trace + 1 * kTraceCtas * kTraceSlots : nullptr;
+    g.wait_ns = a.gram_wait_ns;
+    if (launch_gram_stage(g, a.status, dev, s, pdl)) return -1;
     mark(2);
-    // ----------------------------------------------------------- rfactor
     // Q = T W_res^T needs the Gram stage's T only. The solve is launched
     // after it and runs beside it: this grid lets the solve start once its
     // own wait for the Gram stage is over, and its shared memory leaves room
     // on every SM for one solve block.
-    const int rf_smem_cap =
+    RFactorStage r;
+    r.Tb = a.Tp;
+    r.Tlo = a.Tplo;
+    r.Ct = a.Ct;
+    r.Ctlo = a.Ctlo;
+    r.split_t = a.split_t;
+    r.hilo = a.hilo;
+    r.smem_cap =
         dev.smem_per_sm > 0 && a.k <= 64
             ? dev.smem_per_sm - 2 * dev.smem_reserved - static_cast<int>(ltilde_smem_bytes(a.k))
             : 0;
-    {
-      RFactorPolicy::Params p;
-      const int Bk = static_cast<int>(a.B) * a.k;
-      p.d_in = a.d_in;
-      p.d_out = a.d_out;
-      p.Bk = Bk;
-      p.bn = std::min(256, (pick_bn(Bk) + 63) / 64 * 64);  // whole 64-column store boxes
-      p.n_tiles_n = ceil_div(Bk, p.bn);
-      uint64_t dw[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(a.d_out)};
-      uint64_t sw[1] = {static_cast<uint64_t>(a.d_in) * 2};
-      uint32_t bw[2] = {64, 128};
-      if (!encode_tmap_bf16(&p.tmW, a.W_res, 2, dw, sw, bw, 128)) return -2;
-      // Pairs halve each SM's share of T' per k-step; they need enough pair
-      // tiles to keep the SMs busy and an even column tile.
-      const bool rf_pairs = a.use_pairs && p.bn % 32 == 0 && p.bn >= 64 &&
-                            ceil_div(a.d_out, 256) * p.n_tiles_n >= dev.sm_count / 4;
-      uint64_t dt[2] = {static_cast<uint64_t>(a.d_in), static_cast<uint64_t>(Bk)};
-      uint32_t bt[2] = {64, static_cast<uint32_t>(rf_pairs ? p.bn / 2 : p.bn)};
-      if (!encode_tmap_bf16(&p.tmT, a.Tp, 2, dt, sw, bt, 128)) return -2;
-      p.split_t = a.split_t ? 1 : 0;
-      if (a.split_t) {
-        if (!encode_tmap_bf16(&p.tmTlo, a.Tplo, 2, dt, sw, bt, 128)) return -2;
-      } else {
-        p.tmTlo = p.tmT;
-      }
-      const uint32_t parts = a.split_t ? 2u : 1u;  // B operands per stage
-      uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
-      uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
-      uint32_t bc[2] = {64, 128};
-      if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
-      p.hilo = a.hilo ? 1 : 0;
-      if (a.hilo) {
-        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
-      } else {
-        p.tmClo = p.tmC;
-      }
-      if (rf_pairs) {
-        const int tiles = ceil_div(a.d_out, 256) * p.n_tiles_n;
-        const uint32_t part_bytes = static_cast<uint32_t>(p.bn / 2) * 128u;
-        const uint32_t smem =
-            setup_common<RFactorPairPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
-                                            false, a.status, dev, rf_smem_cap);
-        if (!smem) return -3;
-        p.c.b_parts = parts;
-        p.c.b_part_desc = part_bytes >> 4;
-        p.c.trigger_after_wait = 1;
-        p.c.idesc = idesc_bf16(256, p.bn, false, false);
-        if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
-        if (launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl)) return -1;
-      } else {
-        const int tiles = ceil_div(a.d_out, 128) * p.n_tiles_n;
-        const uint32_t part_bytes = static_cast<uint32_t>(p.bn) * 128u;
-        const uint32_t smem =
-            setup_common<RFactorPolicy>(p.c, tiles, 128 * 128, parts * part_bytes, p.bn, false,
-                                        false, a.status, dev, rf_smem_cap);
-        if (!smem) return -3;
-        p.c.b_parts = parts;
-        p.c.b_part_desc = part_bytes >> 4;
-        p.c.trigger_after_wait = 1;
-        if (a.trace) p.c.trace = a.trace + 3 * kTraceCtas * kTraceSlots;
-        if (launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl)) return -1;
-      }
-    }
+    r.trace = a.trace ? a.trace + 3 * kTraceCtas * kTraceSlots : nullptr;
+    if (launch_rfactor_stage(r, a, dev, s, pdl)) return -1;
     mark(3);
     // ------------------------------------------------------------- solve
     // L~ = L G^-1 over L, beside the GEMM for Q: it reads what the Gram
@@ -1287,6 +1644,15 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
                  ? 1
                  : 0;
     if (!records) mode = 0;
+    if (a.solver == 1) {
+      // Newton-Schulz: one kernel inverts every G_b + lambda I and publishes
+      // the records (it starts once the GEMM for Q is complete); every solve
+      // block then reads its instance's record
+      if (!records) return -1;
+      if (launch_ns_inverse(a.TG, a.B, a.k, a.lambda, a.ns_iters, a.MD, a.counters, a.status, s))
+        return -1;
+      mode = 2;
+    }
     if (launch_ltilde(a.TG, a.L, a.hilo ? a.Llo : nullptr, a.MD, a.counters, mode, a.B, a.T, a.k,
                       a.lambda, a.alpha, a.status, s, pdl, /*defer_wait=*/true,
                       a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
@@ -1296,79 +1662,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
     mark(3);
   }
   mark(4);
-
-  // ------------------------------------------------------------------ out
-  {
-    OutPolicy::Params p;
-    p.N = static_cast<int>(N);
-    p.r = a.r;
-    p.k = k;
-    p.T = static_cast<int>(a.T);
-    p.B = static_cast<int>(a.B);
-    p.bn = a.d_out % 256 == 0 ? 256 : (a.d_out % 128 == 0 ? 128 : 64);
-    if (a.d_out < p.bn) p.bn = 64;
-    p.n_tiles_n = ceil_div(a.d_out, p.bn);
-    p.nkz = ceil_div(a.r, 64);
-    p.nkl = k > 0 ? ceil_div(k, 64) : 0;
-    p.bias = static_cast<const __nv_bfloat16*>(a.bias);
-    p.d_out = a.d_out;
-
-    uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
-    uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
-    uint32_t bz[2] = {64, 128};
-    if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bz, 128)) return -2;
-    uint64_t du[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(a.d_out)};
-    const bool use_pairs = a.use_pairs && p.bn >= 128;
-    const uint32_t bbox = static_cast<uint32_t>(use_pairs ? p.bn / 2 : p.bn);
-    uint32_t bu[2] = {64, bbox};
-    if (!encode_tmap_bf16(&p.tmU, a.U, 2, du, sz, bu, 128)) return -2;
-    if (k > 0) {
-      uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
-                        static_cast<uint64_t>(a.B)};
-      uint64_t sl[2] = {static_cast<uint64_t>(k) * 2,
-                        static_cast<uint64_t>(k) * 2 * static_cast<uint64_t>(a.T)};
-      uint32_t bl[3] = {64, 128, 1};
-      if (!encode_tmap_bf16(&p.tmL, a.L, 3, dl, sl, bl, 128)) return -2;
-      const int64_t Bk = a.B * k;
-      uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
-      uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
-      uint32_t bc[2] = {64, bbox};
-      if (!encode_tmap_bf16(&p.tmC, a.Ct, 2, dc, sc, bc, 128)) return -2;
-      if (a.hilo) {
-        if (!encode_tmap_bf16(&p.tmLlo, a.Llo, 3, dl, sl, bl, 128)) return -2;
-        if (!encode_tmap_bf16(&p.tmClo, a.Ctlo, 2, dc, sc, bc, 128)) return -2;
-      } else {
-        p.tmLlo = p.tmL;
-        p.tmClo = p.tmC;
-      }
-    } else {
-      p.tmL = p.tmZ;
-      p.tmC = p.tmU;
-      p.tmLlo = p.tmZ;
-      p.tmClo = p.tmU;
-    }
-    p.hilo = k > 0 && a.hilo ? 1 : 0;
-    uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
-    uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
-    uint32_t by[2] = {64, 128};
-    if (!encode_tmap_bf16(&p.tmY, a.Y, 2, dy, sy, by, 128)) return -2;
-    if (use_pairs) {
-      const int tiles = ceil_div(N, 256) * p.n_tiles_n;
-      const uint32_t smem = setup_common<OutPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
-                                                        p.bn, false, false, a.status, dev);
-      if (!smem) return -3;
-      p.c.idesc = idesc_bf16(256, p.bn, false, false);
-      if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
-      if (launch_gemm_pair<OutPairPolicy>(p, smem, dev, s, pdl)) return -1;
-    } else {
-      const int tiles = ceil_div(N, 128) * p.n_tiles_n;
-      const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn,
-                                                    false, false, a.status, dev);
-      if (!smem) return -3;
-      if (a.trace) p.c.trace = a.trace + 4 * kTraceCtas * kTraceSlots;
-      if (launch_gemm<OutPolicy>(p, smem, dev, s, pdl)) return -1;
-    }
-  }
+  if (launch_out_stage(a.L, a.Llo, a.Ct, a.Ctlo, a.hilo, k, a, dev, s, pdl)) return -1;
   mark(5);
   return 0;
 }

@@ -38,6 +38,7 @@ SIGNATURES = {
     "dyra_load_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_set_linear": (_i, [_vp, _vp, _f, _vp]),
     "dyra_set_als_steps": (_i, [_vp, _i]),
+    "dyra_set_solver": (_i, [_vp, _i, _i]),
     "dyra_forward_batched_host": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_plan_create_monarch": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "dyra_load_monarch": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
@@ -134,6 +135,14 @@ def dyra_load_factors(plan: int, U, V, P, W_res, lam: float, stream=None) -> Non
 def dyra_set_linear(plan: int, bias, alpha: float = 1.0, stream=None) -> None:
     _check(lib().dyra_set_linear(plan, _ptr(bias), float(alpha), _stream(stream)),
            "dyra_set_linear")
+
+
+DYRA_SOLVER_LDL = 0
+DYRA_SOLVER_NEWTON_SCHULZ = 1
+
+
+def dyra_set_solver(plan: int, solver: int, max_iters: int = 40) -> None:
+    _check(lib().dyra_set_solver(plan, int(solver), int(max_iters)), "dyra_set_solver")
 
 
 def dyra_set_als_steps(plan: int, half_steps: int) -> None:

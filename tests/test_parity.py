@@ -190,6 +190,8 @@ LINEAR = [
     ("linear_k72", 256, 512, 64, 72, 2, 300, "bf16", 0.5, True),        # the general solve
     ("linear_weight_only", 256, 512, 64, 0, 3, 201, "bf16", 1.0, True),
     ("linear_f32", 96, 80, 12, 8, 3, 50, "f32", 0.5, True),
+    ("linear_vit_fc1", 1024, 4096, 256, 32, 32, 201, "bf16", 0.7, True),  # the ViT-L fc1 shape
+    ("linear_compensated", 512, 1024, 64, 64, 1, 300, "bf16", 0.7, True),  # one instance: hi/lo parts
 ]
 
 
@@ -228,28 +230,79 @@ def test_bias_and_alpha(case):
     layer.close()
 
 
+NEWTON_SCHULZ = [
+    # name, d_in, d_out, r, k, B, T
+    ("ns_instances", 256, 512, 64, 32, 3, 201),       # straddling tiles, k = 32
+    ("ns_k64_one", 512, 1024, 64, 64, 1, 700),        # one instance: compensated correction
+    ("ns_k40", 200, 328, 40, 40, 2, 150),             # k not a multiple of 16
+    ("ns_vit_fc1", 1024, 4096, 256, 32, 32, 201),     # the ViT-L fc1 shape
+]
+
+
+@pytest.mark.parametrize("case", NEWTON_SCHULZ, ids=[c[0] for c in NEWTON_SCHULZ])
+def test_newton_schulz_solver(case):
+    """The Newton-Schulz solver of the small ridge systems (DyRA Sec. 2.4)
+    meets the oracle's exact solve, and agrees with the LDL^T solver's layer."""
+    name, d_in, d_out, r, k, B, T = case
+    s = LayerSpec(name, d_in, d_out, r, k, B, T, "bf16", 0.7, "lognormal", seed=6)
+    f = prepared(s)
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    Y_ldl = layer.forward(X, B=B, T=T).clone()
+    dyra.dyra_set_solver(layer.plan, dyra.DYRA_SOLVER_NEWTON_SCHULZ, 40)
+    Y = layer.forward(X, B=B, T=T)
+    assert layer.status() == 0
+    check(s, Y, f)
+    d = oracle.rel_fro(Y.double().cpu().numpy(), Y_ldl.double().cpu().numpy())
+    assert d <= 1e-2, "%s: Newton-Schulz vs LDL %.3e" % (name, d)
+    dyra.dyra_set_solver(layer.plan, dyra.DYRA_SOLVER_LDL, 40)
+    assert torch.equal(layer.forward(X, B=B, T=T), Y_ldl)
+    layer.close()
+
+
+def test_newton_schulz_solver_limits():
+    s, f = _small(k=72)
+    layer = make_layer(s, f)
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_set_solver(layer.plan, dyra.DYRA_SOLVER_NEWTON_SCHULZ, 40)
+    assert e.value.code == dyra.DYRA_ERR_UNSUPPORTED
+    for bad in ((2, 40), (1, 0), (1, 201)):
+        with pytest.raises(dyra.DyraError) as e:
+            dyra.dyra_set_solver(layer.plan, *bad)
+        assert e.value.code == dyra.DYRA_ERR_INVALID_ARG
+    layer.close()
+
+
 ALS = [
-    # name, d_in, d_out, r, k, B, T, dtype, t
-    ("als_f32_t1.5", 96, 80, 12, 8, 3, 50, "f32", 1.5),
-    ("als_f32_t2", 96, 80, 12, 8, 3, 50, "f32", 2.0),
-    ("als_f32_t3_k40", 128, 96, 16, 40, 2, 60, "f32", 3.0),
-    ("als_bf16_simt_t2", 256, 512, 64, 32, 3, 201, "bf16", 2.0),
+    # name, d_in, d_out, r, k, B, T, dtype, t, kernels
+    ("als_f32_t1.5", 96, 80, 12, 8, 3, 50, "f32", 1.5, "simt"),
+    ("als_f32_t2", 96, 80, 12, 8, 3, 50, "f32", 2.0, "simt"),
+    ("als_f32_t3_k40", 128, 96, 16, 40, 2, 60, "f32", 3.0, "simt"),
+    ("als_bf16_simt_t2", 256, 512, 64, 32, 3, 201, "bf16", 2.0, "simt"),
+    # the tensor-core chain: instances straddling 128-row tiles, a ragged tail
+    ("als_bf16_t1.5", 256, 512, 64, 32, 3, 201, "bf16", 1.5, "umma"),
+    ("als_bf16_t2", 256, 512, 64, 32, 3, 201, "bf16", 2.0, "umma"),
+    ("als_bf16_t3", 256, 512, 64, 32, 3, 201, "bf16", 3.0, "umma"),
+    ("als_bf16_t2.5_k40", 200, 328, 40, 40, 2, 150, "bf16", 2.5, "umma"),  # k, d_in, d_out odd
+    ("als_bf16_t1.5_k64_one", 512, 1024, 64, 64, 1, 700, "bf16", 1.5, "umma"),  # row splits
+    ("als_bf16_t2_k72", 256, 512, 64, 72, 2, 300, "bf16", 2.0, "umma"),  # the general solve
+    ("als_vit_fc1_t1.5", 1024, 4096, 256, 32, 32, 201, "bf16", 1.5, "umma"),  # the ViT-L fc1 shape
 ]
 
 
 @pytest.mark.parametrize("case", ALS, ids=[c[0] for c in ALS])
 def test_als_iterations(case):
     """t alternating least-squares iterations (DyRA Sec. 2.2, Sec. 3.3) on the
-    CUDA-core kernels, against the oracle's ALS from the same start; t = 1
-    again afterwards gives the one-step layer."""
-    name, d_in, d_out, r, k, B, T, dtype, t = case
+    CUDA-core or the tensor-core kernels, against the oracle's ALS from the
+    same start; t = 1 again afterwards gives the one-step layer."""
+    name, d_in, d_out, r, k, B, T, dtype, t, kernels = case
     s = LayerSpec(name, d_in, d_out, r, k, B, T, dtype, 0.7, "outlier", n_outlier=4,
                   outlier_scale=10.0, seed=2)
     w = generate(s)
     fo = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, r, k, s.lam)
     f = {n: oracle.round_to(a, dtype) for n, a in
          (("X", w.X), ("U", fo.U), ("V", fo.V), ("P", fo.P), ("W_res", fo.W_res))}
-    layer = make_layer(s, f, kernels="simt")
+    layer = make_layer(s, f, kernels=kernels)
     X = to_dev(f["X"], dtype)
     layer.set_als_iterations(t)
     Y = layer.forward(X, B=B, T=T)
@@ -262,12 +315,42 @@ def test_als_iterations(case):
     layer.close()
 
 
-def test_als_iterations_need_the_cuda_core_kernels():
+def test_als_iterations_on_the_tensor_cores_keep_the_one_step_path():
+    """Switching a tensor-core plan to t = 2 and back gives the one-step output
+    bit for bit, and the allocation-free entry refuses t > 1."""
     s, f = _small()
     layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    Y1 = layer.forward(X, B=s.B, T=s.T).clone()
+    layer.set_als_iterations(2)
+    Y2 = layer.forward(X, B=s.B, T=s.T).clone()
+    assert layer.status() == 0 and not torch.equal(Y1, Y2)
+    Yn = torch.empty_like(Y2)
+    with pytest.raises(dyra.DyraError) as e:
+        dyra.dyra_forward_batched_noalloc(layer.plan, X, Yn, s.B, s.T)
+    assert e.value.code == dyra.DYRA_ERR_UNSUPPORTED
     layer.set_als_iterations(1)
-    with pytest.raises(dyra.DyraError):
-        layer.set_als_iterations(2)
+    assert torch.equal(layer.forward(X, B=s.B, T=s.T), Y1)
+    layer.close()
+
+
+def test_als_printed_t15_schedule_on_the_tensor_cores():
+    """The update sequence the text prints for t = 1.5 (L, R, L, R, L: five
+    updates) runs as half_steps = 5 and matches the oracle's printed schedule."""
+    s = LayerSpec("als_printed", 256, 512, 64, 32, 3, 201, "bf16", 0.7, "outlier", n_outlier=4,
+                  outlier_scale=10.0, seed=2)
+    w = generate(s)
+    fo = oracle.offline_prepare_from_svd(w.left, w.sigma, w.right, s.r, s.k, s.lam)
+    f = {n: oracle.round_to(a, "bf16") for n, a in
+         (("X", w.X), ("U", fo.U), ("V", fo.V), ("P", fo.P), ("W_res", fo.W_res))}
+    layer = make_layer(s, f)
+    X = to_dev(f["X"], "bf16")
+    dyra.dyra_set_als_steps(layer.plan, oracle.als_updates(1.5, "printed"))
+    Y = layer.forward(X, B=s.B, T=s.T)
+    assert layer.status() == 0
+    Yo = oracle.als_inference(f["X"], f["U"], f["V"], f["W_res"], fo.R0, s.lam, s.B, s.T, 1.5,
+                              schedule="printed")
+    assert oracle.rel_fro(Y.double().cpu().numpy(), Yo) <= TOL["bf16"]
     layer.close()
 
 
