@@ -65,8 +65,11 @@ enum {
 enum {
   DYRA_STATUS_NONPOSITIVE_PIVOT = 1, /* Cholesky of L^T L + lambda I met a pivot <= 0 or NaN;
                                         that instance's correction was set to zero */
-  DYRA_STATUS_WAIT_TIMEOUT = 2       /* a kernel's pipeline wait exceeded its time limit and the
+  DYRA_STATUS_WAIT_TIMEOUT = 2,      /* a kernel's pipeline wait exceeded its time limit and the
                                         kernel returned early; outputs are undefined */
+  DYRA_STATUS_BOUNDS = 4             /* bounds-checked build (libdyra_debug.so, compiled with
+                                        DYRA_DEBUG) only: a kernel computed a global index outside
+                                        its buffer and skipped that access; outputs are undefined */
 };
 
 /*

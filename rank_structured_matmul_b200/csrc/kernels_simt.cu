@@ -125,8 +125,10 @@ __global__ void __launch_bounds__(kSolveThreads)
     }
     const bool zero = bad != 0;
     for (int i = 0; i < k; ++i)
-      Tp[(static_cast<size_t>(b) * k + i) * d_in + col] =
-          from_f<TOut>(zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid]);
+      if (sm100::in_bounds(status, (static_cast<size_t>(b) * k + i) * d_in + col, 1,
+                           static_cast<size_t>(B) * k * d_in))
+        Tp[(static_cast<size_t>(b) * k + i) * d_in + col] =
+            from_f<TOut>(zero ? 0.f : alpha * Ycol[i * kSolveThreads + tid]);
   }
   if (tid == 0 && blockIdx.y == 0 && bad) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
@@ -310,7 +312,9 @@ __global__ void __launch_bounds__(kSolveThreads2)
     TOut* dst = Tp + (static_cast<size_t>(b) * k + i) * d_in + col;
 #pragma unroll
     for (int v = 0; v < 4; ++v)
-      if (col + v < d_in) dst[v] = from_f<TOut>(zero ? 0.f : alpha * acc[u][v]);
+      if (col + v < d_in &&
+          sm100::in_bounds(status, (dst - Tp) + v, 1, static_cast<size_t>(B) * k * d_in))
+        dst[v] = from_f<TOut>(zero ? 0.f : alpha * acc[u][v]);
   }
   if (tid == 0 && blockIdx.y == 0 && zero) atomicOr(status, sm100::kStatusPivot);
   __syncthreads();
@@ -404,7 +408,9 @@ __global__ void __maxnreg__(152)
     constexpr int C8 = KMAX / 8;
     for (int e = tid; e < ROWS * C8; e += kLtThreads) {
       const int rr = e / C8, c8 = e % C8;
-      const bool valid = rr < nrows && 8 * c8 < k;
+      const bool valid = rr < nrows && 8 * c8 < k &&
+                         sm100::in_bounds(status, (rows - L) + static_cast<size_t>(rr) * k + 8 * c8,
+                                          8, static_cast<size_t>(gridDim.x) * T * k);
       const __nv_bfloat16* src = valid ? rows + static_cast<size_t>(rr) * k + 8 * c8 : rows;
       __nv_bfloat16* dst = Vs + rr * VS + 8 * c8;
       if (async)
@@ -553,6 +559,7 @@ __global__ void __maxnreg__(152)
       const int rl = p0 + RT * rg + rr;
       if (rl >= nrows || 4 * cg >= k) continue;
       __nv_bfloat16* dst = rows + static_cast<size_t>(rl) * k + 4 * cg;
+      if (!sm100::in_bounds(status, dst - L, 4, static_cast<size_t>(gridDim.x) * T * k)) continue;
       // a failed factorisation writes zeros (not alpha times a non-finite value)
       const __nv_bfloat162 lo = __floats2bfloat162_rn(zero ? 0.f : alpha * acc[rr][0],
                                                       zero ? 0.f : alpha * acc[rr][1]);
@@ -698,9 +705,10 @@ __global__ void __launch_bounds__(kNsThreads)
   }
   const bool bad = !(r < 1e-2f);
   float* rec = MD + static_cast<size_t>(b) * ldl_record_floats<KMAX>();
+  const size_t rec_extent = static_cast<size_t>(gridDim.x) * ldl_record_floats<KMAX>();
   for (int e = tid; e < KMAX * KMAX; e += kNsThreads) {
     const int i = e / KMAX, q = e % KMAX;
-    rec[e] = Xs[i * LD + q];
+    if (sm100::in_bounds(status, (rec - MD) + e, 1, rec_extent)) rec[e] = Xs[i * LD + q];
   }
   if (tid == 0) rec[KMAX * KMAX] = bad ? 1.f : 0.f;
   __syncthreads();
@@ -758,7 +766,8 @@ __global__ void __launch_bounds__(kSolveThreads)
     __syncthreads();
   }
   const int t = blockIdx.y * kSolveThreads + tid;
-  if (t < T) {
+  if (t < T && sm100::in_bounds(status, (static_cast<size_t>(b) * T + t) * k, k,
+                                static_cast<size_t>(gridDim.x) * T * k)) {
     __nv_bfloat16* row = L + (static_cast<size_t>(b) * T + t) * k;
     for (int i = 0; i < k; ++i) Ycol[i * kSolveThreads + tid] = __bfloat162float(row[i]);
     for (int i = 0; i < k; ++i) {  // R y = l

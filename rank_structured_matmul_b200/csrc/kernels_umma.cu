@@ -273,10 +273,12 @@ struct ProjPolicy {
         for (int g = 0; g < 4; ++g) {
           const int col = t.n0 + cc + 8 * g;
           if (col < rk) {
-            void* dst = col < p.r
-                            ? static_cast<void*>(p.Z + static_cast<size_t>(grow) * p.r + col)
-                            : static_cast<void*>(p.L + static_cast<size_t>(grow) * p.k + (col - p.r));
-            store8_bf16(dst, v, g);
+            const bool z = col < p.r;
+            const size_t at = z ? static_cast<size_t>(grow) * p.r + col
+                                : static_cast<size_t>(grow) * p.k + (col - p.r);
+            if (!in_bounds(p.c.status, at, 8, static_cast<size_t>(p.N) * (z ? p.r : p.k)))
+              continue;
+            store8_bf16(z ? static_cast<void*>(p.Z + at) : static_cast<void*>(p.L + at), v, g);
           }
         }
       }
@@ -351,8 +353,11 @@ struct ProjPolicy {
         const int c4 = static_cast<int>(off[u]) / 128, row = static_cast<int>(off[u]) - c4 * 128;
         const int grow = t.m0 + row, col = t.n0 + 4 * c4;
         if (grow >= p.N || col >= rk) continue;
-        __nv_bfloat16* dst = col < p.r ? p.Z + static_cast<size_t>(grow) * p.r + col
-                                       : p.L + static_cast<size_t>(grow) * p.k + (col - p.r);
+        const bool z = col < p.r;
+        const size_t at = z ? static_cast<size_t>(grow) * p.r + col
+                            : static_cast<size_t>(grow) * p.k + (col - p.r);
+        if (!in_bounds(p.c.status, at, 4, static_cast<size_t>(p.N) * (z ? p.r : p.k))) continue;
+        __nv_bfloat16* dst = (z ? p.Z : p.L) + at;
         uint2 w;
         w.x = pack_bf16x2(acc[u].x, acc[u].y);
         w.y = pack_bf16x2(acc[u].z, acc[u].w);
@@ -467,9 +472,13 @@ struct GramPolicy {
         if (i2 >= p.k) return;
         col = p.d_in + i2;
       }
+      const size_t extent = static_cast<size_t>(p.B) * p.k * J;
 #pragma unroll
       for (int u = 0; u < n; ++u)
-        if (i0 + u < p.k) inst[static_cast<size_t>(i0 + u) * J + col] = v[u];
+        if (i0 + u < p.k &&
+            in_bounds(p.c.status, (inst - p.TGf) + static_cast<size_t>(i0 + u) * J + col, 1,
+                      extent))
+          inst[static_cast<size_t>(i0 + u) * J + col] = v[u];
       return;
     }
     if (t.mt < p.mtx) {
@@ -477,9 +486,11 @@ struct GramPolicy {
       if (j >= p.d_in) return;
       const size_t off = static_cast<size_t>(t.b) * p.k * p.d_in + j;
       __nv_bfloat16* dst = p.Tb + off;
+      const size_t extent = static_cast<size_t>(p.B) * p.k * p.d_in;
 #pragma unroll
       for (int u = 0; u < n; ++u)
-        if (i0 + u < p.k) {
+        if (i0 + u < p.k &&
+            in_bounds(p.c.status, off + static_cast<size_t>(i0 + u) * p.d_in, 1, extent)) {
           const __nv_bfloat16 h = __float2bfloat16_rn(v[u]);
           dst[static_cast<size_t>(i0 + u) * p.d_in] = h;
           if (p.Tlo != nullptr)
@@ -490,9 +501,12 @@ struct GramPolicy {
       const int i2 = (t.mt - p.mtx) * 128 + row;
       if (i2 >= p.k) return;
       float* dst = p.G + static_cast<size_t>(t.b) * p.k * p.k + i2;
+      const size_t extent = static_cast<size_t>(p.B) * p.k * p.k;
 #pragma unroll
       for (int u = 0; u < n; ++u)
-        if (i0 + u < p.k) dst[static_cast<size_t>(i0 + u) * p.k] = v[u];
+        if (i0 + u < p.k &&
+            in_bounds(p.c.status, (dst - p.G) + static_cast<size_t>(i0 + u) * p.k, 1, extent))
+          dst[static_cast<size_t>(i0 + u) * p.k] = v[u];
     }
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
@@ -807,6 +821,8 @@ struct XRwPolicy {
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
         if (cc + 8 * c8 >= p.k) break;  // k is a multiple of 8
+        if (!in_bounds(p.c.status, (dst - p.P2) + 8 * c8, 8, static_cast<size_t>(p.N) * p.k))
+          break;
         uint4 q;
         q.x = pack_bf16x2(f32(v[8 * c8 + 0]), f32(v[8 * c8 + 1]));
         q.y = pack_bf16x2(f32(v[8 * c8 + 2]), f32(v[8 * c8 + 3]));

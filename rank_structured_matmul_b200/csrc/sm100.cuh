@@ -18,6 +18,25 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 constexpr int kStatusPivot = 1;    // DYRA_STATUS_NONPOSITIVE_PIVOT
 constexpr int kStatusTimeout = 2;  // DYRA_STATUS_WAIT_TIMEOUT
+constexpr int kStatusBounds = 4;   // DYRA_STATUS_BOUNDS (DYRA_DEBUG build only)
+
+// Bounds check of the DYRA_DEBUG build: elements [i, i + n) of a buffer of
+// `extent` elements. In that build an access outside the buffer is skipped
+// and raises kStatusBounds in the status word; the release build compiles the
+// check away (the kernels' own guards keep their accesses in bounds).
+__device__ __forceinline__ bool in_bounds(int* status, size_t i, size_t n, size_t extent) {
+#ifdef DYRA_DEBUG
+  if (i + n <= extent) return true;
+  atomicOr(status, kStatusBounds);
+  return false;
+#else
+  (void)status;
+  (void)i;
+  (void)n;
+  (void)extent;
+  return true;
+#endif
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

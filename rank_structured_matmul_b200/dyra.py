@@ -3,7 +3,9 @@
 Argument marshalling only: tensors become device pointers, the current torch
 stream becomes the cudaStream_t, and negative return codes become DyraError.
 Every step of the layer runs in libdyra.so's CUDA kernels; there is no
-fallback. If the library is not built, loading it raises.
+fallback. If the library is not built, loading it raises. With
+DYRA_DEBUG_LIB=1 in the environment the bounds-checked build libdyra_debug.so
+is loaded instead (python -m rank_structured_matmul_b200.build --debug).
 """
 
 from __future__ import annotations
@@ -14,6 +16,7 @@ from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdyra.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libdyra_debug.so")
 
 DYRA_F32 = 0
 DYRA_BF16 = 1
@@ -30,6 +33,7 @@ DYRA_ERR_DEVICE = -8
 
 DYRA_STATUS_NONPOSITIVE_PIVOT = 1
 DYRA_STATUS_WAIT_TIMEOUT = 2
+DYRA_STATUS_BOUNDS = 4
 
 # name -> (restype, argtypes), mirroring include/dyra.h
 _vp, _i, _i64, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
@@ -79,10 +83,12 @@ def lib() -> ctypes.CDLL:
     """Load libdyra.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libdyra.so is not built: run `python -m "
-                               "rank_structured_matmul_b200.build`")
-        handle = ctypes.CDLL(LIB_PATH)
+        debug = os.environ.get("DYRA_DEBUG_LIB") == "1"
+        path = DEBUG_LIB_PATH if debug else LIB_PATH
+        if not os.path.exists(path):
+            raise RuntimeError("%s is not built: run `python -m rank_structured_matmul_b200.build%s`"
+                               % (os.path.basename(path), " --debug" if debug else ""))
+        handle = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(handle, name)
             fn.restype = res

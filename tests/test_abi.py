@@ -32,6 +32,17 @@ def test_library_exports_every_declared_symbol():
     assert set(dyra.SIGNATURES) <= names
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checked build (compiled with DYRA_DEBUG) has the same ABI."""
+    import ctypes
+    if not os.path.exists(dyra.DEBUG_LIB_PATH):
+        from rank_structured_matmul_b200.build import build
+        build(debug=True)
+    lib = ctypes.CDLL(dyra.DEBUG_LIB_PATH)
+    for n in sorted(declared_functions()):
+        assert hasattr(lib, n), "libdyra_debug.so does not export %s" % n
+
+
 def test_error_strings():
     for code in range(0, -9, -1):
         s = dyra.error_string(code)
