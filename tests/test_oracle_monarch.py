@@ -143,10 +143,75 @@ def check_dyra_never_worse_than_weight_only():
                                rtol=0, atol=1e-12)
 
 
+# ------------------------------------------- rectangular blocks (reading) ----
+
+RECT = ((3, 4, 2, 5), (2, 3, 4, 2), (1, 4, 3, 2))  # b1, b2, b1', b2'
+
+
+def rect_blocks(b1, b2, b1o, b2o, seed):
+    rng = np.random.default_rng(seed)
+    return ([rng.standard_normal((b1, b1o)) for _ in range(b2)],
+            [rng.standard_normal((b2, b2o)) for _ in range(b1o)])
+
+
+def check_rect_entry_formula():
+    """Entry (m1*b2 + j2, j1*b2' + i2) of P1 L P2^T R is L_j2[m1, j1] R_j1[j2, i2]
+    for rectangular blocks, element by element (a c1 x c2 matrix)."""
+    for b1, b2, b1o, b2o in RECT:
+        Lb, Rb = rect_blocks(b1, b2, b1o, b2o, seed=b1 + 10 * b2 + 100 * b1o)
+        W = mon.monarch_matrix(Lb, Rb)
+        assert W.shape == (b1 * b2, b1o * b2o)
+        for m1 in range(b1):
+            for j2 in range(b2):
+                for j1 in range(b1o):
+                    for i2 in range(b2o):
+                        want = Lb[j2][m1, j1] * Rb[j1][j2, i2]
+                        assert abs(W[m1 * b2 + j2, j1 * b2o + i2] - want) <= 1e-12
+
+
+def check_rect_recovery_and_blockwise_eckart_young():
+    """A rectangular Monarch matrix is its own projection; for any matrix the
+    projection error is the sum over the b1 x b2' blocks of ||S||^2 - s1(S)^2,
+    with s1 by power iteration."""
+    rng = np.random.default_rng(8)
+    for b1, b2, b1o, b2o in RECT:
+        M = mon.monarch_matrix(*rect_blocks(b1, b2, b1o, b2o, seed=3))
+        np.testing.assert_allclose(mon.monarch_matrix(*mon.monarch_project(M, b1, b2, b1o, b2o)), M,
+                                   rtol=0, atol=1e-10 * max(1.0, np.abs(M).max()))
+        W = rng.standard_normal((b1 * b2, b1o * b2o))
+        err = np.sum((W - mon.monarch_matrix(*mon.monarch_project(W, b1, b2, b1o, b2o))) ** 2)
+        want = 0.0
+        for j1 in range(b1o):
+            for j2 in range(b2):
+                S = np.array([[W[m1 * b2 + j2, j1 * b2o + i2] for i2 in range(b2o)]
+                              for m1 in range(b1)])
+                want += np.sum(S ** 2) - top_singular_value(S, iters=2000) ** 2
+        assert err == pytest.approx(want, rel=1e-8, abs=1e-10)
+
+
+def check_rect_dyra_invariants():
+    """DyRA on a rectangular Monarch part (d_in = b1 b2, d_out = b1' b2'):
+    k = 0 is the Monarch product, and no instance is worse than weight-only."""
+    b1, b2, b1o, b2o = 3, 4, 2, 5
+    s = LayerSpec("monr", b1 * b2, b1o * b2o, 1, 3, 2, 9, "f32", 0.5, "lognormal", seed=4)
+    w = generate(s)
+    f0 = mon.offline_prepare_monarch(w.weight(), b1, b2, 0, s.lam, b1o=b1o, b2o=b2o)
+    Y0 = mon.monarch_inference(w.X, f0, s.lam, s.B, s.T)
+    np.testing.assert_allclose(Y0, w.X @ mon.monarch_matrix(f0.Lb, f0.Rb), rtol=0, atol=1e-12)
+    f = mon.offline_prepare_monarch(w.weight(), b1, b2, 3, s.lam, b1o=b1o, b2o=b2o)
+    Y = mon.monarch_inference(w.X, f, s.lam, s.B, s.T)
+    Yd = w.X @ w.weight().T
+    Ywo = w.X @ f.What.T
+    for b in range(s.B):
+        rows = slice(b * s.T, (b + 1) * s.T)
+        assert np.linalg.norm(Yd[rows] - Y[rows]) <= np.linalg.norm(Yd[rows] - Ywo[rows]) * (1 + 1e-12)
+
+
 PINS = [check_entry_formula, check_shuffle_is_a_permutation, check_recovers_monarch_matrices,
         check_degenerate_block_counts_are_exact, check_blockwise_eckart_young, check_locally_optimal,
         check_dyra_k0_is_the_monarch_product, check_dyra_full_residual_is_exact,
-        check_dyra_never_worse_than_weight_only]
+        check_dyra_never_worse_than_weight_only, check_rect_entry_formula,
+        check_rect_recovery_and_blockwise_eckart_young, check_rect_dyra_invariants]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda p: p.__name__)
@@ -154,9 +219,19 @@ def test_monarch_pin(pin):
     pin()
 
 
-def test_rejects_non_square():
+def test_rejects_a_shape_that_does_not_match_the_blocks():
     with pytest.raises(ValueError):
         mon.monarch_project(np.zeros((12, 8)), 3, 4)
+    with pytest.raises(ValueError):
+        mon.monarch_project(np.zeros((12, 12)), 3, 4, 2, 5)
+
+
+def test_rect_parameter_count():
+    """b2 blocks of b1 x b1' and b1' blocks of b2 x b2'."""
+    W = np.random.default_rng(0).standard_normal((12, 10))
+    Lb, Rb = mon.monarch_project(W, 3, 4, 2, 5)
+    assert len(Lb) == 4 and all(L.shape == (3, 2) for L in Lb)
+    assert len(Rb) == 2 and all(R.shape == (4, 5) for R in Rb)
 
 
 def test_parameter_count():
@@ -176,20 +251,22 @@ def _identity_shuffle(b1, b2):
     return np.eye(b1 * b2)
 
 
-def _contiguous_rows(Wp, b1, b2):
+def _contiguous_rows(Wp, b1, b2, b1o=None, b2o=None):
     """Takes rows j2*b1 .. j2*b1 + b1 - 1 instead of the strided ones."""
-    Lb = [np.zeros((b1, b1)) for _ in range(b2)]
-    Rb = [np.zeros((b2, b2)) for _ in range(b1)]
-    for j1 in range(b1):
+    b1o = b1 if b1o is None else b1o
+    b2o = b2 if b2o is None else b2o
+    Lb = [np.zeros((b1, b1o)) for _ in range(b2)]
+    Rb = [np.zeros((b2, b2o)) for _ in range(b1o)]
+    for j1 in range(b1o):
         for j2 in range(b2):
-            u, s, vt = np.linalg.svd(Wp[j2 * b1:(j2 + 1) * b1, j1 * b2:(j1 + 1) * b2])
+            u, s, vt = np.linalg.svd(Wp[j2 * b1:(j2 + 1) * b1, j1 * b2o:(j1 + 1) * b2o])
             Lb[j2][:, j1] = np.sqrt(s[0]) * u[:, 0]
             Rb[j1][j2, :] = np.sqrt(s[0]) * vt[0]
     return Lb, Rb
 
 
-def _sigma_twice(Wp, b1, b2):
-    Lb, Rb = _PROJECT(Wp, b1, b2)
+def _sigma_twice(Wp, b1, b2, b1o=None, b2o=None):
+    Lb, Rb = _PROJECT(Wp, b1, b2, b1o, b2o)
     return [L * 1.0 for L in Lb], [R * 2.0 for R in Rb]
 
 
