@@ -89,25 +89,43 @@ int dyra_plan_create(dyra_plan_t *out, int d_in, int d_out, int r, int k, dyra_d
 /*
  * A plan whose static part is a Monarch matrix ([DyRA] App. B) instead of the
  * rank-r factorisation, for a square layer of n = b1 * b2 features (the pages
- * define Monarch for square weights). The correction (rank k, 0 <= k <= n,
- * k <= 128) is unchanged. In the paper's layout (Y = X W) the static product
- * is X W_hat with W_hat = P L P^T R: y[j1*b2 + i2] = sum over m1, j2 of
- * x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2], with P the perfect shuffle. These
- * plans run on the CUDA-core kernels (fp32, or bf16 with bf16 intermediates);
- * dyra_forward_batched_noalloc returns DYRA_ERR_UNSUPPORTED for them.
- * Errors as dyra_plan_create; DYRA_ERR_INVALID_ARG also when n != b1 * b2.
+ * define Monarch for square weights): dyra_plan_create_monarch_rect with
+ * b1' = b1 and b2' = b2. Errors as there; DYRA_ERR_INVALID_ARG also when
+ * n != b1 * b2.
  */
 int dyra_plan_create_monarch(dyra_plan_t *out, int n, int b1, int b2, int k, dyra_dtype_t dtype);
 
 /*
+ * A Monarch plan for a rectangular layer, d_in = b1 * b2 and d_out = b1o * b2o
+ * (the pages define Monarch for square weights only and also use it on
+ * rectangular MLP layers; this is the library's reading of that). In the
+ * paper's layout (Y = X W, W of shape d_in x d_out) the static product is
+ * X W_hat with W_hat = P1 L P2^T R, L = diag(L_1 .. L_b2) of b1 x b1o blocks,
+ * R = diag(R_1 .. R_b1o) of b2 x b2o blocks and P1, P2 the perfect shuffles of
+ * the b1 x b2 and b1o x b2 grids:
+ *   y[j1*b2o + i2] = sum over m1, j2 of x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2].
+ * The correction (rank k, 0 <= k <= min(d_in, d_out), k <= 128) is unchanged.
+ * bf16 plans run on the tensor cores (two block-diagonal GEMMs of the output
+ * stage's kernel, each behind a shuffle of its input's columns, the second
+ * taking the correction), fp32 plans on the CUDA cores. d_in, d_out and
+ * b2 * b1o are at most 49152. Errors as dyra_plan_create; DYRA_ERR_ALIGNMENT
+ * for bf16 unless d_in, d_out, k, b1 and b2 are multiples of 8.
+ * dyra_forward_batched_noalloc returns DYRA_ERR_UNSUPPORTED for these plans,
+ * and on the tensor cores dyra_set_als_steps accepts only 2.
+ */
+int dyra_plan_create_monarch_rect(dyra_plan_t *out, int b1, int b2, int b1o, int b2o, int k,
+                                  dyra_dtype_t dtype);
+
+/*
  * Load a Monarch plan's factors (the counterpart of dyra_load_factors):
- *   Lblocks : b2 blocks of b1 x b1, row-major, one after the other (L_j2[m1][j1])
- *   Rblocks : b1 blocks of b2 x b2, row-major, one after the other (R_j1[j2][i2])
+ *   Lblocks : b2 blocks of b1 x b1o, row-major, one after the other (L_j2[m1][j1])
+ *   Rblocks : b1o blocks of b2 x b2o, row-major, one after the other (R_j1[j2][i2])
+ *             (b1o = b1 and b2o = b2 for dyra_plan_create_monarch)
  *   P, W_res, lambda : as in dyra_load_factors, with W_res = W - W_hat^T in this
- *                      library's n x n (d_out x d_in) layout
+ *                      library's d_out x d_in layout
  * Device pointers in the plan dtype, copied on `stream`. DYRA_ERR_INVALID_ARG
- * for a plan not made by dyra_plan_create_monarch (and dyra_load_factors
- * rejects Monarch plans).
+ * for a plan not made by dyra_plan_create_monarch(_rect) (and
+ * dyra_load_factors rejects Monarch plans).
  */
 int dyra_load_monarch(dyra_plan_t p, const void *Lblocks, const void *Rblocks, const void *P,
                       const void *W_res, float lambda, dyra_stream_t stream);

@@ -22,7 +22,7 @@ struct dyra_plan {
   // Monarch static part ([DyRA] App. B) in place of U V^T: n = d_in = d_out =
   // b1 * b2, b2 blocks of b1 x b1 (Lblk) and b1 blocks of b2 x b2 (Rblk); r = 0
   bool monarch = false;
-  int mb1 = 0, mb2 = 0;
+  int mb1 = 0, mb2 = 0, mb1o = 0, mb2o = 0;  // d_in = mb1 mb2, d_out = mb1o mb2o
   void* Lblk = nullptr;
   void* Rblk = nullptr;
   void* Mtmp = nullptr;  // workspace: N x n, the product's intermediate
@@ -216,13 +216,19 @@ int ensure_workspace_impl(dyra_plan* p, int64_t B, int64_t T) {
   const size_t es = elem_size(p->dtype);
   const int k = p->k;
   int rc;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
+  const size_t nmid = p->monarch ? static_cast<size_t>(p->mb2) * p->mb1o : 0;
   if (p->monarch) {
+    // the intermediate X L-product; on the tensor cores also the shuffled X
+    // before it and the shuffled product after it (Z then holds the product)
     void* mt = p->Mtmp;
-    if ((rc = grow(mt, p->cap_Mtmp, static_cast<size_t>(N) * p->d_in * es))) return rc;
+    const size_t cols = umma ? std::max(static_cast<size_t>(p->d_in), nmid) : nmid;
+    if ((rc = grow(mt, p->cap_Mtmp, static_cast<size_t>(N) * cols * es))) return rc;
     p->Mtmp = mt;
   }
-  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
-    if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * p->r * es))) return rc;
+  if (umma) {
+    const size_t zcols = p->monarch ? nmid : static_cast<size_t>(p->r);
+    if ((rc = grow(p->Z, p->cap_Z, static_cast<size_t>(N) * zcols * es))) return rc;
     if (k > 0) {
       if ((rc = grow(p->L, p->cap_L, static_cast<size_t>(N) * k * es))) return rc;
       void* tg = p->TG;
@@ -343,7 +349,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
   int rc = ensure_workspace(p, B, T);
   if (rc) return rc;
 
-  if (p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch) {
+  if (p->dtype == DYRA_BF16 && !p->force_simt) {
     dyra::Bf16Forward a;
     a.d_in = p->d_in;
     a.d_out = p->d_out;
@@ -384,6 +390,16 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.Ctlo = a.hilo ? p->Ctlo : nullptr;
     a.split_t = a.hilo;
     a.Tplo = a.hilo ? p->Tplo : nullptr;
+    if (p->monarch) {
+      a.Lt = p->Lblk;
+      a.Rt = p->Rblk;
+      a.mb1 = p->mb1;
+      a.mb2 = p->mb2;
+      a.mb1o = p->mb1o;
+      a.mb2o = p->mb2o;
+      a.Xs = p->Mtmp;
+      a.Ms = p->Z;
+    }
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, a.stage_events || a.trace, s,
                             [&](cudaStream_t st) { return dyra::launch_bf16_forward(a, p->dev, st); });
     p->stage_recorded = p->stage_timing && rc == 0;
@@ -418,6 +434,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
       a.Rblk = static_cast<const __nv_bfloat16*>(p->Rblk);
       a.mb1 = p->mb1;
       a.mb2 = p->mb2;
+      a.mb1o = p->mb1o;
+      a.mb2o = p->mb2o;
       a.Mtmp = static_cast<__nv_bfloat16*>(p->Mtmp);
     }
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
@@ -453,6 +471,8 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
       a.Rblk = static_cast<const float*>(p->Rblk);
       a.mb1 = p->mb1;
       a.mb2 = p->mb2;
+      a.mb1o = p->mb1o;
+      a.mb2o = p->mb2o;
       a.Mtmp = static_cast<float*>(p->Mtmp);
     }
     rc = launch_maybe_graph(p, X, Y, B, T, a.weight_only, false, s,
@@ -543,18 +563,33 @@ int dyra_plan_create(dyra_plan_t* out, int d_in, int d_out, int r, int k, dyra_d
   return plan_create_impl(out, d_in, d_out, r, k, dtype);
 }
 
-int dyra_plan_create_monarch(dyra_plan_t* out, int n, int b1, int b2, int k, dyra_dtype_t dtype) {
+int dyra_plan_create_monarch_rect(dyra_plan_t* out, int b1, int b2, int b1o, int b2o, int k,
+                                  dyra_dtype_t dtype) {
   if (out == nullptr) return DYRA_ERR_INVALID_ARG;
   if (dtype != DYRA_F32 && dtype != DYRA_BF16) return DYRA_ERR_INVALID_ARG;
-  if (b1 < 1 || b2 < 1 || n != b1 * b2 || k < 0 || k > 128 || k > n) return DYRA_ERR_INVALID_ARG;
-  if (dtype == DYRA_BF16 && (n % 8 || k % 8)) return DYRA_ERR_ALIGNMENT;
-  const int rc = plan_create_impl(out, n, n, 0, k, dtype);
+  if (b1 < 1 || b2 < 1 || b1o < 1 || b2o < 1 || k < 0 || k > 128) return DYRA_ERR_INVALID_ARG;
+  const int64_t d_in = static_cast<int64_t>(b1) * b2, d_out = static_cast<int64_t>(b1o) * b2o;
+  const int64_t nmid = static_cast<int64_t>(b2) * b1o;
+  if (d_in > 49152 || d_out > 49152 || nmid > 49152 || k > std::min(d_in, d_out))
+    return DYRA_ERR_INVALID_ARG;
+  // bf16: 16-byte rows, and (tensor cores) 16-byte block offsets within rows
+  if (dtype == DYRA_BF16 && (d_in % 8 || d_out % 8 || k % 8 || b1 % 8 || b2 % 8))
+    return DYRA_ERR_ALIGNMENT;
+  const int rc = plan_create_impl(out, static_cast<int>(d_in), static_cast<int>(d_out), 0, k,
+                                  dtype);
   if (rc == DYRA_OK) {
     (*out)->monarch = true;
     (*out)->mb1 = b1;
     (*out)->mb2 = b2;
+    (*out)->mb1o = b1o;
+    (*out)->mb2o = b2o;
   }
   return rc;
+}
+
+int dyra_plan_create_monarch(dyra_plan_t* out, int n, int b1, int b2, int k, dyra_dtype_t dtype) {
+  if (out == nullptr || b1 < 1 || b2 < 1 || n != b1 * b2) return DYRA_ERR_INVALID_ARG;
+  return dyra_plan_create_monarch_rect(out, b1, b2, b1, b2, k, dtype);
 }
 
 static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
@@ -675,7 +710,7 @@ int dyra_set_solver(dyra_plan_t p, int solver, int max_iters) {
   if (p == nullptr || (solver != DYRA_SOLVER_LDL && solver != DYRA_SOLVER_NEWTON_SCHULZ) ||
       max_iters < 1 || max_iters > 200)
     return DYRA_ERR_INVALID_ARG;
-  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt && !p->monarch;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
   if (solver == DYRA_SOLVER_NEWTON_SCHULZ && (!umma || p->k == 0 || p->k > 64))
     return DYRA_ERR_UNSUPPORTED;
   p->solver = solver;
@@ -686,6 +721,9 @@ int dyra_set_solver(dyra_plan_t p, int solver, int max_iters) {
 
 int dyra_set_als_steps(dyra_plan_t p, int half_steps) {
   if (p == nullptr || half_steps < 2 || half_steps > 64) return DYRA_ERR_INVALID_ARG;
+  // the Monarch static part runs one ALS step on the tensor cores
+  if (p->monarch && p->dtype == DYRA_BF16 && !p->force_simt && half_steps != 2)
+    return DYRA_ERR_UNSUPPORTED;
   p->als_half_steps = half_steps;
   drop_graphs(p);  // captured forwards hold the old count
   return DYRA_OK;
@@ -772,19 +810,29 @@ int dyra_load_monarch(dyra_plan_t p, const void* Lblocks, const void* Rblocks, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t es = elem_size(p->dtype);
   const size_t n = static_cast<size_t>(p->d_in);
-  const size_t lb = static_cast<size_t>(p->mb2) * p->mb1 * p->mb1 * es;
-  const size_t rb = static_cast<size_t>(p->mb1) * p->mb2 * p->mb2 * es;
+  const size_t lb = static_cast<size_t>(p->mb2) * p->mb1 * p->mb1o * es;
+  const size_t rb = static_cast<size_t>(p->mb1o) * p->mb2 * p->mb2o * es;
   const size_t vpt = static_cast<size_t>(p->k) * n * es;
-  const size_t wb = p->k > 0 ? n * n * es : 0;
+  const size_t wb = p->k > 0 ? n * static_cast<size_t>(p->d_out) * es : 0;
+  const bool umma = p->dtype == DYRA_BF16 && !p->force_simt;
   int rc;
   if (!p->Lblk && (rc = dev_alloc(&p->Lblk, lb))) return rc;
   if (!p->Rblk && (rc = dev_alloc(&p->Rblk, rb))) return rc;
   if (vpt && !p->VPt && (rc = dev_alloc(&p->VPt, vpt))) return rc;
   if (wb && !p->W_res && (rc = dev_alloc(&p->W_res, wb))) return rc;
   p->factor_bytes = lb + rb + vpt + wb;
-  if (cudaMemcpyAsync(p->Lblk, Lblocks, lb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(p->Rblk, Rblocks, rb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
-      (wb && cudaMemcpyAsync(p->W_res, W_res, wb, cudaMemcpyDeviceToDevice, s) != cudaSuccess))
+  if (umma) {
+    // the tensor cores take each block transposed (K-major): L_j2^T and R_j1^T
+    if (dyra::launch_grid_transpose(Lblocks, p->Lblk, p->mb2, p->mb1, p->mb1o, p->dev.sm_count,
+                                    s) ||
+        dyra::launch_grid_transpose(Rblocks, p->Rblk, p->mb1o, p->mb2, p->mb2o, p->dev.sm_count,
+                                    s))
+      return DYRA_ERR_CUDA;
+  } else if (cudaMemcpyAsync(p->Lblk, Lblocks, lb, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+             cudaMemcpyAsync(p->Rblk, Rblocks, rb, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+    return DYRA_ERR_CUDA;
+  }
+  if (wb && cudaMemcpyAsync(p->W_res, W_res, wb, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return DYRA_ERR_CUDA;
   if (vpt) {  // P^T (k x n): the projection's B operand, as [V | P]^T with r = 0
     if (p->dtype == DYRA_BF16)

@@ -94,6 +94,15 @@ struct Bf16Forward {
   // Newton-Schulz iteration (at most ns_iters steps; k <= 64)
   int solver = 0;
   int ns_iters = 40;
+  // Monarch static part ([DyRA] App. B) in place of Z U^T (r = 0; VPt holds
+  // P^T only): Lt holds b2 blocks of b1' x b1 (L_j2 transposed, K-major), Rt
+  // b1' blocks of b2' x b2 (R_j1 transposed); Xs is N x d_in and Ms N x b2 b1'
+  // of workspace (both also carry the intermediate products).
+  const void* Lt = nullptr;
+  const void* Rt = nullptr;
+  int mb1 = 0, mb2 = 0, mb1o = 0, mb2o = 0;
+  void* Xs = nullptr;
+  void* Ms = nullptr;
   // ALS updates ([DyRA] Sec. 3.3): 2 is Alg. 1; more run the explicit
   // alternating chain (launch_bf16_als). TG then needs B x k x (d_in + k)
   // floats.
@@ -150,11 +159,11 @@ struct SimtForward {
   T* P2 = nullptr;       // (B*k) x d_in: R_b W_res, the L update's projector before its solve
   float* TG2 = nullptr;  // B x k x (Trows + k): [ (X_b P2_b^T)^T | R_b R_b^T ]
   // Monarch static part ([DyRA] App. B), r = 0: y = x W_hat in the paper's
-  // layout, W_hat = P L P^T R with Lblk b2 blocks of mb1 x mb1 and Rblk mb1
-  // blocks of mb2 x mb2 (row-major, contiguous); Mtmp is N x n
+  // layout, W_hat = P1 L P2^T R with Lblk mb2 blocks of mb1 x mb1o and Rblk
+  // mb1o blocks of mb2 x mb2o (row-major, contiguous); Mtmp is N x mb2 mb1o
   const T* Lblk = nullptr;
   const T* Rblk = nullptr;
-  int mb1 = 0, mb2 = 0;
+  int mb1 = 0, mb2 = 0, mb1o = 0, mb2o = 0;
   T* Mtmp = nullptr;
 };
 
@@ -172,6 +181,11 @@ int launch_solve(const float* TG, int splits, int64_t B, int k, int d_in, float 
 // Floats per instance of the factor records for correction rank k (0 when
 // k > 64: the solve then factors G_b itself).
 int factor_record_floats(int k);
+
+// out[row][q * P + p] = in[row][p * Q + q] for `rows` rows of P * Q bf16
+// values (P * Q a multiple of 8, at most 49152): the Monarch shuffle.
+int launch_grid_transpose(const void* in, void* out, int64_t rows, int P, int Q, int sm_count,
+                          cudaStream_t s);
 
 // Newton-Schulz inverse of G_b + lambda I per instance (k <= 64), published
 // as factor records behind the instance flags for launch_ltilde's mode 2.

@@ -863,6 +863,42 @@ int gemm(int M, int N, int K, const TA* A, int64_t am, int64_t ak, int64_t ab, c
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
+// out[row][q * P + p] = in[row][p * Q + q] for every row (p < P, q < Q): each
+// row, read as a row-major P x Q grid, is written back transposed. This is the
+// perfect shuffle of the Monarch factorisation ([DyRA] App. B), and the block
+// transpose of its factors. A block stages one row in shared memory at a time
+// (16-byte loads); the stores are 16-byte when P is a multiple of 8.
+constexpr int kShuffleThreads = 256;
+
+__global__ void __launch_bounds__(kShuffleThreads)
+    grid_transpose_kernel(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                          int64_t rows, int P, int Q) {
+  extern __shared__ __align__(16) __nv_bfloat16 row_s[];
+  const int n = P * Q;  // a multiple of 8
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const __nv_bfloat16* src = in + row * n;
+    __nv_bfloat16* dst = out + row * n;
+    for (int e = 8 * threadIdx.x; e < n; e += 8 * kShuffleThreads)
+      *reinterpret_cast<uint4*>(row_s + e) = __ldg(reinterpret_cast<const uint4*>(src + e));
+    __syncthreads();
+    if (P % 8 == 0) {
+      for (int o = 8 * threadIdx.x; o < n; o += 8 * kShuffleThreads) {
+        const int q = o / P, p = o - q * P;  // outputs o .. o + 7 share q
+        __align__(16) __nv_bfloat16 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = row_s[(p + u) * Q + q];
+        *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(v);
+      }
+    } else {
+      for (int o = threadIdx.x; o < n; o += kShuffleThreads) {
+        const int q = o / P, p = o - q * P;
+        dst[o] = row_s[p * Q + q];
+      }
+    }
+    __syncthreads();
+  }
+}
+
 template <typename T>
 __global__ void pack_vp_kernel(const T* __restrict__ V, const T* __restrict__ P, T* __restrict__ VPt,
                                int d_in, int r, int k) {
@@ -1066,6 +1102,27 @@ template int launch_solve<__nv_bfloat16>(const float*, int, int64_t, int, int, f
                                          __nv_bfloat16*, int*, cudaStream_t, bool,
                                          unsigned long long*, float);
 
+int launch_grid_transpose(const void* in, void* out, int64_t rows, int P, int Q, int sm_count,
+                          cudaStream_t s) {
+  if (rows == 0) return 0;
+  const int64_t n = static_cast<int64_t>(P) * Q;
+  if (P < 1 || Q < 1 || n % 8 != 0 || n > 49152) return -1;
+  const size_t smem = static_cast<size_t>(n) * sizeof(__nv_bfloat16);
+  static KernelSetup setup;
+  const int d = setup_device();
+  if (d < 0) return -1;
+  if (smem > 48 * 1024 && smem > setup.smem[d].load()) {
+    if (cudaFuncSetAttribute(grid_transpose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return -1;
+    setup.smem[d].store(static_cast<uint32_t>(smem));
+  }
+  const int64_t blocks = std::min<int64_t>(rows, static_cast<int64_t>(std::max(sm_count, 1)) * 8);
+  grid_transpose_kernel<<<static_cast<unsigned>(blocks), kShuffleThreads, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, P, Q);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 template <typename T>
 int launch_pack_vp(const T* V, const T* P, T* VPt, int d_in, int r, int k, cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(r + k) * d_in;
@@ -1149,14 +1206,15 @@ int launch_simt_forward(const SimtForward<T>& a, const DeviceInfo&, cudaStream_t
     }
   }
   if (a.Lblk != nullptr) {
-    // Monarch static part: y[j1*b2 + i2] = sum_{m1, j2} x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2],
-    // as two strided batched products through Mtmp[row][j2*b1 + j1]
-    const int n = a.d_in, b1 = a.mb1, b2 = a.mb2;
-    if (gemm(static_cast<int>(N), b1, b1, a.X, n, b2, 1, a.Lblk, b1, 1,
-             static_cast<int64_t>(b1) * b1, a.Mtmp, n, 1, b1, b2, 0, s))
+    // Monarch static part: y[j1*b2' + i2] = sum_{m1, j2} x[m1*b2 + j2] L_j2[m1][j1] R_j1[j2][i2],
+    // as two strided batched products through Mtmp[row][j2*b1' + j1]
+    const int b1 = a.mb1, b2 = a.mb2, b1o = a.mb1o, b2o = a.mb2o;
+    const int nmid = b2 * b1o;
+    if (gemm(static_cast<int>(N), b1o, b1, a.X, a.d_in, b2, 1, a.Lblk, b1o, 1,
+             static_cast<int64_t>(b1) * b1o, a.Mtmp, nmid, 1, b1o, b2, 0, s))
       return -1;
-    if (gemm(static_cast<int>(N), b2, b2, a.Mtmp, n, b1, 1, a.Rblk, b2, 1,
-             static_cast<int64_t>(b2) * b2, a.Y, n, 1, b2, b1, 0, s, 1.f, a.bias, b2))
+    if (gemm(static_cast<int>(N), b2o, b2, a.Mtmp, nmid, b1o, 1, a.Rblk, b2o, 1,
+             static_cast<int64_t>(b2) * b2o, a.Y, a.d_out, 1, b2o, b1o, 0, s, 1.f, a.bias, b2o))
       return -1;
   } else if (gemm(static_cast<int>(N), a.d_out, a.r, a.ZL, rk, 1, 0, a.U, 1, a.r, 0, a.Y, a.d_out,
                   1, 0, 1, 0, s, 1.f, a.bias)) {  // Y = Z U^T (+ b)

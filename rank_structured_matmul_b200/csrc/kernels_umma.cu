@@ -658,7 +658,32 @@ struct OutPolicy {
     const __nv_bfloat16* bias;  // d_out, added in the epilogue, or nullptr
     int d_out;
     int hilo;  // correction as hi L~ . hi Q + hi L~ . lo Q + lo L~ . hi Q
+    // Block-diagonal static part (zb_w > 0; a Monarch factor, [DyRA] App. B):
+    // output columns come in zb_n blocks of zb_w, and block c is the product
+    // of Z's columns c*zb_k .. + zb_k with block c of U, read through the 3-D
+    // view tmU (zb_k, zb_w, zb_n), box (64, rows, 1), whose out-of-bounds fill
+    // zeroes the tile's rows outside the block. nkz is then the K-steps of one
+    // block. zb_w == 0: the dense Z U^T (K = r).
+    int zb_w, zb_k, zb_n;
   };
+  // The static part's blocks that the tile's columns n0 .. n0 + bn - 1 touch.
+  static __device__ __forceinline__ void static_blocks(const Params& p, int n0, int& lo,
+                                                       int& nseg) {
+    if (p.zb_w > 0) {
+      lo = n0 / p.zb_w;
+      nseg = min(p.zb_n - 1, (n0 + p.bn - 1) / p.zb_w) - lo + 1;
+    } else {
+      lo = 0;
+      nseg = 1;
+    }
+  }
+  static __device__ __forceinline__ int static_iters(const Params& p, int z_nseg) {
+    return p.zb_w > 0 ? z_nseg * p.nkz : p.nkz;
+  }
+  static __device__ __forceinline__ int static_ksteps(const Params& p, int it) {
+    if (p.zb_w > 0) return min(4, ceil_div_dev(p.zb_k - (it % p.nkz) * 64, 16));
+    return min(4, ceil_div_dev(p.r - it * 64, 16));
+  }
   // K-step j of the correction: instance segment, sub-product (0 hi.hi,
   // 1 hi.lo, 2 lo.hi) and 64-wide chunk of k.
   static __device__ __forceinline__ void correction_step(const Params& p, int j, int& seg,
@@ -670,7 +695,7 @@ struct OutPolicy {
     ch = jj - sub * p.nkl;
   }
   struct Tile {
-    int m0, n0, b_lo, nseg;
+    int m0, n0, b_lo, nseg, z_lo, z_nseg;
   };
   static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
@@ -698,26 +723,35 @@ struct OutPolicy {
       t.b_lo = 0;
       t.nseg = 0;
     }
+    static_blocks(p, t.n0, t.z_lo, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return static_iters(p, t.z_nseg) + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
-    if (it < p.nkz) {
-      tma_load_2d(sa, &p.tmZ, bar, it * 64, t.m0);
-      tma_load_2d(sb, &p.tmU, bar, it * 64, t.n0);
+    const int ns = static_iters(p, t.z_nseg);
+    if (it < ns) {
+      if (p.zb_w > 0) {
+        const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
+        tma_load_2d(sa, &p.tmZ, bar, blk * p.zb_k + kk * 64, t.m0);
+        tma_load_3d(sb, &p.tmU, bar, kk * 64, t.n0 - blk * p.zb_w, blk);
+      } else {
+        tma_load_2d(sa, &p.tmZ, bar, it * 64, t.m0);
+        tma_load_2d(sb, &p.tmU, bar, it * 64, t.n0);
+      }
     } else {
       int seg, sub, ch;
-      correction_step(p, it - p.nkz, seg, sub, ch);
+      correction_step(p, it - ns, seg, sub, ch);
       const int b = t.b_lo + seg;
       tma_load_3d(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
       tma_load_2d(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, t.n0);
     }
   }
-  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
-    if (it < p.nkz) return min(4, ceil_div_dev(p.r - it * 64, 16));
-    const int ch = (it - p.nkz) % p.nkl;
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
+    const int ns = static_iters(p, t.z_nseg);
+    if (it < ns) return static_ksteps(p, it);
+    const int ch = (it - ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
@@ -926,7 +960,7 @@ struct ProjPairPolicy {
 struct OutPairPolicy {
   using Params = OutPolicy::Params;  // tmU / tmC boxes are (64, bn/2) here
   struct Tile {
-    int m0, n0, b_lo, nseg;
+    int m0, n0, b_lo, nseg, z_lo, z_nseg;
   };
   static constexpr uint32_t kEpiSmemBytes = OutPolicy::kEpiSmemBytes;
 
@@ -942,28 +976,37 @@ struct OutPairPolicy {
       t.b_lo = 0;
       t.nseg = 0;
     }
+    OutPolicy::static_blocks(p, t.n0, t.z_lo, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return p.nkz + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return OutPolicy::static_iters(p, t.z_nseg) + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
     const int ma = t.m0 + 128 * static_cast<int>(rank);
     const int nb = t.n0 + (p.bn / 2) * static_cast<int>(rank);
-    if (it < p.nkz) {
-      tma_load_2d_pair(sa, &p.tmZ, bar, it * 64, ma);
-      tma_load_2d_pair(sb, &p.tmU, bar, it * 64, nb);
+    const int ns = OutPolicy::static_iters(p, t.z_nseg);
+    if (it < ns) {
+      if (p.zb_w > 0) {
+        const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
+        tma_load_2d_pair(sa, &p.tmZ, bar, blk * p.zb_k + kk * 64, ma);
+        tma_load_3d_pair(sb, &p.tmU, bar, kk * 64, nb - blk * p.zb_w, blk);
+      } else {
+        tma_load_2d_pair(sa, &p.tmZ, bar, it * 64, ma);
+        tma_load_2d_pair(sb, &p.tmU, bar, it * 64, nb);
+      }
     } else {
       int seg, sub, ch;
-      OutPolicy::correction_step(p, it - p.nkz, seg, sub, ch);
+      OutPolicy::correction_step(p, it - ns, seg, sub, ch);
       const int b = t.b_lo + seg;
       tma_load_3d_pair(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, ma - b * p.T, b);
       tma_load_2d_pair(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, nb);
     }
   }
-  static __device__ __forceinline__ int ksteps(const Params& p, const Tile&, int it) {
-    if (it < p.nkz) return min(4, ceil_div_dev(p.r - it * 64, 16));
-    const int ch = (it - p.nkz) % p.nkl;
+  static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
+    const int ns = OutPolicy::static_iters(p, t.z_nseg);
+    if (it < ns) return OutPolicy::static_ksteps(p, it);
+    const int ch = (it - ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
@@ -979,6 +1022,8 @@ struct OutPairPolicy {
     h.n0 = t.n0;
     h.b_lo = t.b_lo;
     h.nseg = t.nseg;
+    h.z_lo = t.z_lo;
+    h.z_nseg = t.z_nseg;
     OutPolicy::epilogue(p, h, tacc, e);
   }
   static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
@@ -1364,35 +1409,59 @@ int launch_rfactor_stage(const RFactorStage& r, const Bf16Forward& a, const Devi
   return launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
 }
 
-// The output stage Y = Z U^T (+ bias) + sum_b mask_b(L) C_b with the
+// The static part of an output stage: Z (N x zcols) times U^T, dense (U is
+// d_out x zcols) or block-diagonal (zb_w > 0: U holds zb_n blocks of zb_w
+// rows x zb_k columns, K-major, and output block c takes Z's columns
+// c*zb_k .. + zb_k: a Monarch factor).
+struct OutStatic {
+  const void* Z;
+  int zcols;
+  const void* U;
+  int zb_w, zb_k, zb_n;
+};
+
+// The output stage Y = (static part) (+ bias) + sum_b mask_b(L) C_b with the
 // correction's left factor L (N x k) and right factor C^T (d_out x B*k)
 // (k = 0: the static part alone), with their low parts when hilo.
-int launch_out_stage(const void* L, const void* Llo, const void* Ct, const void* Ctlo, bool hilo,
-                     int k, const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const void* Ct,
+                     const void* Ctlo, bool hilo, int k, int d_out, void* Y, const void* bias,
+                     const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
   const int64_t N = a.B * a.T;
   OutPolicy::Params p;
   p.N = static_cast<int>(N);
-  p.r = a.r;
+  p.r = st.zcols;
   p.k = k;
   p.T = static_cast<int>(a.T);
   p.B = static_cast<int>(a.B);
-  p.bn = a.d_out % 256 == 0 ? 256 : (a.d_out % 128 == 0 ? 128 : 64);
-  if (a.d_out < p.bn) p.bn = 64;
-  p.n_tiles_n = ceil_div(a.d_out, p.bn);
-  p.nkz = ceil_div(a.r, 64);
+  p.bn = d_out % 256 == 0 ? 256 : (d_out % 128 == 0 ? 128 : 64);
+  if (d_out < p.bn) p.bn = 64;
+  p.n_tiles_n = ceil_div(d_out, p.bn);
+  p.zb_w = st.zb_w;
+  p.zb_k = st.zb_k;
+  p.zb_n = st.zb_n;
+  p.nkz = st.zb_w > 0 ? ceil_div(st.zb_k, 64) : ceil_div(st.zcols, 64);
   p.nkl = k > 0 ? ceil_div(k, 64) : 0;
-  p.bias = static_cast<const __nv_bfloat16*>(a.bias);
-  p.d_out = a.d_out;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.d_out = d_out;
 
-  uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
-  uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+  uint64_t dz[2] = {static_cast<uint64_t>(st.zcols), static_cast<uint64_t>(N)};
+  uint64_t sz[1] = {static_cast<uint64_t>(st.zcols) * 2};
   uint32_t bz[2] = {64, 128};
-  if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bz, 128)) return -2;
-  uint64_t du[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(a.d_out)};
+  if (!encode_tmap_bf16(&p.tmZ, st.Z, 2, dz, sz, bz, 128)) return -2;
   const bool use_pairs = a.use_pairs && p.bn >= 128;
   const uint32_t bbox = static_cast<uint32_t>(use_pairs ? p.bn / 2 : p.bn);
-  uint32_t bu[2] = {64, bbox};
-  if (!encode_tmap_bf16(&p.tmU, a.U, 2, du, sz, bu, 128)) return -2;
+  if (st.zb_w > 0) {
+    uint64_t du[3] = {static_cast<uint64_t>(st.zb_k), static_cast<uint64_t>(st.zb_w),
+                      static_cast<uint64_t>(st.zb_n)};
+    uint64_t su[2] = {static_cast<uint64_t>(st.zb_k) * 2,
+                      static_cast<uint64_t>(st.zb_k) * 2 * static_cast<uint64_t>(st.zb_w)};
+    uint32_t bu[3] = {64, bbox, 1};
+    if (!encode_tmap_bf16(&p.tmU, st.U, 3, du, su, bu, 128)) return -2;
+  } else {
+    uint64_t du[2] = {static_cast<uint64_t>(st.zcols), static_cast<uint64_t>(d_out)};
+    uint32_t bu[2] = {64, bbox};
+    if (!encode_tmap_bf16(&p.tmU, st.U, 2, du, sz, bu, 128)) return -2;
+  }
   if (k > 0) {
     uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
                       static_cast<uint64_t>(a.B)};
@@ -1401,7 +1470,7 @@ int launch_out_stage(const void* L, const void* Llo, const void* Ct, const void*
     uint32_t bl[3] = {64, 128, 1};
     if (!encode_tmap_bf16(&p.tmL, L, 3, dl, sl, bl, 128)) return -2;
     const int64_t Bk = a.B * k;
-    uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(a.d_out)};
+    uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(d_out)};
     uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
     uint32_t bc[2] = {64, bbox};
     if (!encode_tmap_bf16(&p.tmC, Ct, 2, dc, sc, bc, 128)) return -2;
@@ -1419,10 +1488,10 @@ int launch_out_stage(const void* L, const void* Llo, const void* Ct, const void*
     p.tmClo = p.tmU;
   }
   p.hilo = k > 0 && hilo ? 1 : 0;
-  uint64_t dy[2] = {static_cast<uint64_t>(a.d_out), static_cast<uint64_t>(N)};
-  uint64_t sy[1] = {static_cast<uint64_t>(a.d_out) * 2};
+  uint64_t dy[2] = {static_cast<uint64_t>(d_out), static_cast<uint64_t>(N)};
+  uint64_t sy[1] = {static_cast<uint64_t>(d_out) * 2};
   uint32_t by[2] = {64, 128};
-  if (!encode_tmap_bf16(&p.tmY, a.Y, 2, dy, sy, by, 128)) return -2;
+  if (!encode_tmap_bf16(&p.tmY, Y, 2, dy, sy, by, 128)) return -2;
   unsigned long long* tr = a.trace ? a.trace + 4 * kTraceCtas * kTraceSlots : nullptr;
   if (use_pairs) {
     const int tiles = ceil_div(N, 256) * p.n_tiles_n;
@@ -1501,9 +1570,11 @@ int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* cou
   uint32_t bw[2] = {64, static_cast<uint32_t>(ps.pairs ? p.bn / 2 : p.bn)};
   if (!encode_tmap_bf16(&p.tmW, a.VPt, 2, dw, sx, bw, 128)) return -2;
   uint32_t bs[2] = {64, 128};
-  uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
-  uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
-  if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bs, 128)) return -2;
+  if (a.r > 0) {
+    uint64_t dz[2] = {static_cast<uint64_t>(a.r), static_cast<uint64_t>(N)};
+    uint64_t sz[1] = {static_cast<uint64_t>(a.r) * 2};
+    if (!encode_tmap_bf16(&p.tmZ, a.Z, 2, dz, sz, bs, 128)) return -2;
+  }
   if (p.k > 0) {
     uint64_t dl[2] = {static_cast<uint64_t>(p.k), static_cast<uint64_t>(N)};
     uint64_t sl[1] = {static_cast<uint64_t>(p.k) * 2};
@@ -1511,6 +1582,7 @@ int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* cou
   } else {
     p.tmL = p.tmZ;
   }
+  if (a.r == 0) p.tmZ = p.tmL;  // no static columns (the projection of a Monarch plan)
   unsigned long long* tr = a.trace ? a.trace + 0 * kTraceCtas * kTraceSlots : nullptr;
   if (ps.pairs) {
     const uint32_t smem = setup_common<ProjPairPolicy>(p.c, ps.tiles, 128 * 128,
@@ -1600,8 +1672,117 @@ int launch_bf16_als(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s)
   mark(2);
   mark(3);
   mark(4);
-  if (launch_out_stage(a.L, nullptr, a.Ct, nullptr, false, k, a, dev, s, pdl)) return -1;
+  const OutStatic st = {a.Z, a.r, a.U, 0, 0, 0};
+  if (launch_out_stage(st, a.L, nullptr, a.Ct, nullptr, false, k, a.d_out, a.Y, a.bias, a, dev, s,
+                       pdl))
+    return -1;
   mark(5);
+  return 0;
+}
+
+}  // namespace
+
+namespace {
+
+void mark_stage(const Bf16Forward& a, int i, cudaStream_t s) {
+  if (a.stage_events) cudaEventRecord(a.stage_events[i], s);
+}
+
+// The correction of the one-step layer after the projection: the Gram stage,
+// the rank-k factor GEMM Q = T W_res^T and, beside it, the solve L~ = L G^-1
+// over L (programmatic dependent launches throughout).
+int launch_correction(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+  GramStage g = layer_gram(a);
+  g.Tb = static_cast<__nv_bfloat16*>(a.Tp);
+  g.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
+  g.G = a.TG;
+  g.trace = a.trace ? a.trace + 1 * kTraceCtas * kTraceSlots : nullptr;
+  g.wait_ns = a.gram_wait_ns;
+  if (launch_gram_stage(g, a.status, dev, s, pdl)) return -1;
+  mark_stage(a, 2, s);
+  // Q = T W_res^T needs the Gram stage's T only. The solve is launched
+  // after it and runs beside it: this grid lets the solve start once its
+  // own wait for the Gram stage is over, and its shared memory leaves room
+  // on every SM for one solve block.
+  RFactorStage r;
+  r.Tb = a.Tp;
+  r.Tlo = a.Tplo;
+  r.Ct = a.Ct;
+  r.Ctlo = a.Ctlo;
+  r.split_t = a.split_t;
+  r.hilo = a.hilo;
+  r.smem_cap =
+      dev.smem_per_sm > 0 && a.k <= 64
+          ? dev.smem_per_sm - 2 * dev.smem_reserved - static_cast<int>(ltilde_smem_bytes(a.k))
+          : 0;
+  r.trace = a.trace ? a.trace + 3 * kTraceCtas * kTraceSlots : nullptr;
+  if (launch_rfactor_stage(r, a, dev, s, pdl)) return -1;
+  mark_stage(a, 3, s);
+  // ------------------------------------------------------------- solve
+  // L~ = L G^-1 over L, beside the GEMM for Q: it reads what the Gram
+  // stage wrote and waits for the GEMM only before its blocks exit, so that
+  // the output stage can rely on both. Every block factors its G_b while
+  // that fits the SMs; beyond, the instance's first block factors it for
+  // the others.
+  const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
+  int mode = a.factor_mode;
+  if (mode < 0)
+    mode = a.B * ceil_div(a.T, static_cast<int64_t>(ltilde_rows_per_block(a.k))) > dev.sm_count
+               ? 1
+               : 0;
+  if (!records) mode = 0;
+  if (a.solver == 1) {
+    // Newton-Schulz: one kernel inverts every G_b + lambda I and publishes
+    // the records (it starts once the GEMM for Q is complete); every solve
+    // block then reads its instance's record
+    if (!records) return -1;
+    if (launch_ns_inverse(a.TG, a.B, a.k, a.lambda, a.ns_iters, a.MD, a.counters, a.status, s))
+      return -1;
+    mode = 2;
+  }
+  return launch_ltilde(a.TG, a.L, a.hilo ? a.Llo : nullptr, a.MD, a.counters, mode, a.B, a.T,
+                       a.k, a.lambda, a.alpha, a.status, s, pdl, /*defer_wait=*/true,
+                       a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr)
+             ? -1
+             : 0;
+}
+
+// Monarch static part ([DyRA] App. B, square or rectangular blocks) under
+// the same correction. The static product is two block-diagonal GEMMs on
+// the output stage's kernel, each behind a shuffle of its input's columns
+// (b1 b2 = d_in, b1' b2' = d_out, b2 b1' intermediate columns):
+//   Xs[row][j2 b1 + m1]  = X[row][m1 b2 + j2]                      (shuffle)
+//   M[row][j2 b1' + j1]  = sum_m1 Xs[row][j2 b1 + m1] L_j2[m1][j1]  (b2 blocks)
+//   Ms[row][j1 b2 + j2]  = M[row][j2 b1' + j1]                      (shuffle)
+//   Y[row][j1 b2' + i2]  = sum_j2 Ms[row][j1 b2 + j2] R_j1[j2][i2]  (b1' blocks)
+//                          + bias + the correction's L~ Q segments
+// The first three run in stream order; the correction chain follows with
+// programmatic dependent launches, and the last GEMM takes its segments.
+int launch_bf16_monarch(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s) {
+  const int64_t N = a.B * a.T;
+  const int k = a.weight_only ? 0 : a.k;
+  const int nmid = a.mb2 * a.mb1o;
+  mark_stage(a, 0, s);
+  if (launch_grid_transpose(a.X, a.Xs, N, a.mb1, a.mb2, dev.sm_count, s)) return -1;
+  const OutStatic st1 = {a.Xs, a.d_in, a.Lt, a.mb1o, a.mb1, a.mb2};
+  if (launch_out_stage(st1, nullptr, nullptr, nullptr, nullptr, false, 0, nmid, a.Ms, nullptr, a,
+                       dev, s, false))
+    return -1;
+  if (launch_grid_transpose(a.Ms, a.Xs, N, a.mb2, a.mb1o, dev.sm_count, s)) return -1;
+  mark_stage(a, 1, s);
+  if (k > 0) {
+    if (launch_proj_stage(a, k, a.MD, a.counters, dev, s, true)) return -1;
+    if (launch_correction(a, dev, s, true)) return -1;
+  } else {
+    mark_stage(a, 2, s);
+    mark_stage(a, 3, s);
+  }
+  mark_stage(a, 4, s);
+  const OutStatic st2 = {a.Xs, nmid, a.Rt, a.mb2o, a.mb2, a.mb1o};
+  if (launch_out_stage(st2, a.L, nullptr, a.Ct, nullptr, false, k, a.d_out, a.Y, a.bias, a, dev,
+                       s, true))
+    return -1;
+  mark_stage(a, 5, s);
   return 0;
 }
 
@@ -1610,76 +1791,25 @@ int launch_bf16_als(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s)
 int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s) {
   const int64_t N = a.B * a.T;
   if (N == 0) return 0;
+  if (a.Lt != nullptr) return launch_bf16_monarch(a, dev, s);
   const int k = a.weight_only ? 0 : a.k;
   if (k > 0 && a.half_steps > 2) return launch_bf16_als(a, dev, s);
   const bool pdl = true;
-  auto mark = [&](int i) {
-    if (a.stage_events) cudaEventRecord(a.stage_events[i], s);
-  };
-  mark(0);
+  mark_stage(a, 0, s);
   if (launch_proj_stage(a, k, a.MD, a.counters, dev, s, pdl)) return -1;
-  mark(1);
-
+  mark_stage(a, 1, s);
   if (k > 0) {
-    GramStage g = layer_gram(a);
-    g.Tb = static_cast<__nv_bfloat16*>(a.Tp);
-    g.Tlo = a.split_t ? static_cast<__nv_bfloat16*>(a.Tplo) : nullptr;
-    g.G = a.TG;
-    g.trace = a.trace ? a.trace + 1 * kTraceCtas * kTraceSlots : nullptr;
-    g.wait_ns = a.gram_wait_ns;
-    if (launch_gram_stage(g, a.status, dev, s, pdl)) return -1;
-    mark(2);
-    // Q = T W_res^T needs the Gram stage's T only. The solve is launched
-    // after it and runs beside it: this grid lets the solve start once its
-    // own wait for the Gram stage is over, and its shared memory leaves room
-    // on every SM for one solve block.
-    RFactorStage r;
-    r.Tb = a.Tp;
-    r.Tlo = a.Tplo;
-    r.Ct = a.Ct;
-    r.Ctlo = a.Ctlo;
-    r.split_t = a.split_t;
-    r.hilo = a.hilo;
-    r.smem_cap =
-        dev.smem_per_sm > 0 && a.k <= 64
-            ? dev.smem_per_sm - 2 * dev.smem_reserved - static_cast<int>(ltilde_smem_bytes(a.k))
-            : 0;
-    r.trace = a.trace ? a.trace + 3 * kTraceCtas * kTraceSlots : nullptr;
-    if (launch_rfactor_stage(r, a, dev, s, pdl)) return -1;
-    mark(3);
-    // ------------------------------------------------------------- solve
-    // L~ = L G^-1 over L, beside the GEMM for Q: it reads what the Gram
-    // stage wrote and waits for the GEMM only before its blocks exit, so that
-    // the output stage can rely on both. Every block factors its G_b while
-    // that fits the SMs; beyond, the instance's first block factors it for
-    // the others.
-    const bool records = a.MD && a.counters && factor_record_floats(a.k) > 0;
-    int mode = a.factor_mode;
-    if (mode < 0)
-      mode = a.B * ceil_div(a.T, static_cast<int64_t>(ltilde_rows_per_block(a.k))) > dev.sm_count
-                 ? 1
-                 : 0;
-    if (!records) mode = 0;
-    if (a.solver == 1) {
-      // Newton-Schulz: one kernel inverts every G_b + lambda I and publishes
-      // the records (it starts once the GEMM for Q is complete); every solve
-      // block then reads its instance's record
-      if (!records) return -1;
-      if (launch_ns_inverse(a.TG, a.B, a.k, a.lambda, a.ns_iters, a.MD, a.counters, a.status, s))
-        return -1;
-      mode = 2;
-    }
-    if (launch_ltilde(a.TG, a.L, a.hilo ? a.Llo : nullptr, a.MD, a.counters, mode, a.B, a.T, a.k,
-                      a.lambda, a.alpha, a.status, s, pdl, /*defer_wait=*/true,
-                      a.trace ? a.trace + 2 * kTraceCtas * kTraceSlots : nullptr))
-      return -1;
+    if (launch_correction(a, dev, s, pdl)) return -1;
   } else {
-    mark(2);
-    mark(3);
+    mark_stage(a, 2, s);
+    mark_stage(a, 3, s);
   }
-  mark(4);
-  if (launch_out_stage(a.L, a.Llo, a.Ct, a.Ctlo, a.hilo, k, a, dev, s, pdl)) return -1;
-  mark(5);
+  mark_stage(a, 4, s);
+  const OutStatic st = {a.Z, a.r, a.U, 0, 0, 0};
+  if (launch_out_stage(st, a.L, a.Llo, a.Ct, a.Ctlo, a.hilo, k, a.d_out, a.Y, a.bias, a, dev, s,
+                       pdl))
+    return -1;
+  mark_stage(a, 5, s);
   return 0;
 }
 

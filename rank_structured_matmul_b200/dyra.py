@@ -45,6 +45,7 @@ SIGNATURES = {
     "dyra_set_solver": (_i, [_vp, _i, _i]),
     "dyra_forward_batched_host": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
     "dyra_plan_create_monarch": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "dyra_plan_create_monarch_rect": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i, _i]),
     "dyra_load_monarch": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "dyra_forward": (_i, [_vp, _vp, _vp, _i64, _vp]),
     "dyra_forward_batched": (_i, [_vp, _vp, _vp, _i64, _i64, _vp]),
@@ -165,6 +166,14 @@ def dyra_plan_create_monarch(n: int, b1: int, b2: int, k: int, dtype: int) -> in
     h = ctypes.c_void_p()
     _check(lib().dyra_plan_create_monarch(ctypes.byref(h), n, b1, b2, k, dtype),
            "dyra_plan_create_monarch")
+    return h.value
+
+
+def dyra_plan_create_monarch_rect(b1: int, b2: int, b1o: int, b2o: int, k: int,
+                                  dtype: int) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().dyra_plan_create_monarch_rect(ctypes.byref(h), b1, b2, b1o, b2o, k, dtype),
+           "dyra_plan_create_monarch_rect")
     return h.value
 
 
@@ -363,19 +372,26 @@ class DyraLinear:
 
 class DyraMonarchLinear(DyraLinear):
     """A DyRA layer whose static part is a Monarch matrix (DyRA App. B) of
-    n = b1 * b2 features; load() takes the blocks instead of U and V."""
+    d_in = b1 * b2 input and d_out = b1o * b2o output features (square unless
+    b1o, b2o are given); load() takes the blocks instead of U and V."""
 
-    def __init__(self, n: int, b1: int, b2: int, k: int, dtype: str = "bf16"):
+    def __init__(self, n: int, b1: int, b2: int, k: int, dtype: str = "bf16",
+                 b1o: Optional[int] = None, b2o: Optional[int] = None):
         import torch
-        self.d_in = self.d_out = n
-        self.r, self.k, self.b1, self.b2 = 0, k, b1, b2
+        b1o = b1 if b1o is None else b1o
+        b2o = b2 if b2o is None else b2o
+        if n != b1 * b2:
+            raise ValueError("n must be b1 * b2")
+        self.d_in, self.d_out = n, b1o * b2o
+        self.r, self.k, self.b1, self.b2, self.b1o, self.b2o = 0, k, b1, b2, b1o, b2o
         self.dtype = dtype
         self.torch_dtype = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
-        self.plan = dyra_plan_create_monarch(n, b1, b2, k,
-                                             DYRA_BF16 if dtype == "bf16" else DYRA_F32)
+        self.plan = dyra_plan_create_monarch_rect(b1, b2, b1o, b2o, k,
+                                                  DYRA_BF16 if dtype == "bf16" else DYRA_F32)
 
     def load(self, Lblocks, Rblocks, P, W_res, lam: float, stream=None) -> None:
-        """Lblocks: (b2, b1, b1), Rblocks: (b1, b2, b2), P: (n, k), W_res: (n, n)."""
+        """Lblocks: (b2, b1, b1o), Rblocks: (b1o, b2, b2o), P: (d_in, k),
+        W_res: (d_out, d_in)."""
         import torch
         Lb, Rb, P, W_res = (self._dev(t) for t in (Lblocks, Rblocks, P, W_res))
         dyra_load_monarch(self.plan, Lb, Rb, P if self.k else None, W_res if self.k else None,

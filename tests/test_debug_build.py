@@ -34,9 +34,8 @@ SUBSET = " or ".join([
 
 def test_parity_subset_passes_under_the_bounds_checked_library():
     from rank_structured_matmul_b200 import dyra
-    if not os.path.exists(dyra.DEBUG_LIB_PATH):
-        from rank_structured_matmul_b200.build import build
-        build(debug=True)
+    from rank_structured_matmul_b200.build import build
+    build(debug=True)  # incremental: rebuilt only when a source is newer
     env = dict(os.environ, DYRA_DEBUG_LIB="1")
     out = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_parity.py"),
                           "-m", "gpu", "-q", "-x", "-p", "no:cacheprovider", "-k", SUBSET],

@@ -412,37 +412,78 @@ def test_compensated_correction(case):
 
 
 MONARCH = [
-    # name, b1, b2, k, B, T, dtype
-    ("monarch_f32", 8, 12, 8, 3, 50, "f32"),
-    ("monarch_f32_k0", 6, 6, 0, 2, 40, "f32"),
-    ("monarch_bf16", 16, 16, 32, 3, 201, "bf16"),
+    # name, b1, b2, b1', b2', k, B, T, dtype, kernels
+    ("monarch_f32", 8, 12, 8, 12, 8, 3, 50, "f32", "simt"),
+    ("monarch_f32_k0", 6, 6, 6, 6, 0, 2, 40, "f32", "simt"),
+    ("monarch_f32_rect", 6, 8, 4, 10, 8, 2, 45, "f32", "simt"),
+    ("monarch_bf16_simt", 16, 16, 16, 16, 32, 3, 201, "bf16", "simt"),
+    # the tensor cores: instances straddling tiles, blocks narrower than a tile
+    ("monarch_bf16", 16, 16, 16, 16, 32, 3, 201, "bf16", "umma"),
+    ("monarch_bf16_k0", 16, 16, 16, 16, 0, 2, 150, "bf16", "umma"),
+    ("monarch_bf16_rect", 16, 16, 8, 64, 32, 3, 201, "bf16", "umma"),
+    ("monarch_bf16_narrow", 32, 32, 64, 16, 32, 2, 130, "bf16", "umma"),
+    ("monarch_bf16_k64_one", 16, 32, 32, 16, 64, 1, 700, "bf16", "umma"),
+    ("monarch_vit_block_proj", 32, 32, 32, 32, 32, 64, 201, "bf16", "umma"),
 ]
 
 
-@pytest.mark.parametrize("case", MONARCH, ids=[c[0] for c in MONARCH])
-def test_monarch_static_part(case):
-    """A Monarch static part (DyRA App. B) under the same correction, on the
-    CUDA-core kernels, against the oracle's Monarch layer."""
+def _monarch_layer(case, seed=8):
     from oracle import monarch as mon
-    name, b1, b2, k, B, T, dtype = case
-    n = b1 * b2
-    s = LayerSpec(name, n, n, 1, k, B, T, dtype, 0.7, "lognormal", seed=8)
+    name, b1, b2, b1o, b2o, k, B, T, dtype, kernels = case
+    d_in, d_out = b1 * b2, b1o * b2o
+    s = LayerSpec(name, d_in, d_out, 1, k, B, T, dtype, 0.7, "lognormal", seed=seed)
     w = generate(s)
-    fo = mon.offline_prepare_monarch(w.weight(), b1, b2, k, s.lam)
+    fo = mon.offline_prepare_monarch(w.weight(), b1, b2, k, s.lam, b1o=b1o, b2o=b2o)
     rd = lambda a: oracle.round_to(a, dtype)
     Lb = rd(np.stack(fo.Lb))
     Rb = rd(np.stack(fo.Rb))
     P, W_res, X = rd(fo.P), rd(fo.W_res), rd(w.X)
-    layer = dyra.DyraMonarchLinear(n, b1, b2, k, dtype)
+    os.environ["DYRA_KERNELS"] = kernels
+    try:
+        layer = dyra.DyraMonarchLinear(d_in, b1, b2, k, dtype, b1o=b1o, b2o=b2o)
+    finally:
+        os.environ.pop("DYRA_KERNELS", None)
     layer.load(to_dev(Lb, dtype), to_dev(Rb, dtype), to_dev(P, dtype) if k else None,
                to_dev(W_res, dtype) if k else None, s.lam)
-    Y = layer.forward(to_dev(X, dtype), B=B, T=T)
-    assert layer.status() == 0
     fr = mon.MonarchFactors(list(Lb), list(Rb), mon.monarch_matrix(list(Lb), list(Rb)).T, P, W_res,
                             fo.R0)
-    Yo = mon.monarch_inference(X, fr, s.lam, B, T)
+    return s, layer, X, fr
+
+
+@pytest.mark.parametrize("case", MONARCH, ids=[c[0] for c in MONARCH])
+def test_monarch_static_part(case):
+    """A Monarch static part (DyRA App. B; square, or rectangular blocks as read
+    for rectangular layers) under the same correction, on the tensor cores
+    (bf16) or the CUDA cores, against the oracle's Monarch layer."""
+    from oracle import monarch as mon
+    s, layer, X, fr = _monarch_layer(case)
+    dtype = s.dtype
+    Y = layer.forward(to_dev(X, dtype), B=s.B, T=s.T)
+    assert layer.status() == 0
+    Yo = mon.monarch_inference(X, fr, s.lam, s.B, s.T)
     err = oracle.rel_fro(Y.double().cpu().numpy(), Yo)
-    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (name, err)
+    assert err <= TOL[dtype], "%s: rel Frobenius %.3e" % (s.name, err)
+    layer.close()
+
+
+def test_monarch_bias_alpha_and_newton_schulz():
+    """The full linear layer (bias, alpha) and the Newton-Schulz solver on a
+    tensor-core Monarch plan, against the oracle."""
+    from oracle import monarch as mon
+    case = ("monarch_linear", 16, 16, 8, 64, 32, 3, 201, "bf16", "umma")
+    s, layer, X, fr = _monarch_layer(case, seed=9)
+    bias = oracle.round_to(np.random.default_rng(2).standard_normal(s.d_out) * 0.3, "bf16")
+    layer.set_linear(to_dev(bias, "bf16"), 0.6)
+    dyra.dyra_set_solver(layer.plan, dyra.DYRA_SOLVER_NEWTON_SCHULZ, 40)
+    Y = layer.forward(to_dev(X, "bf16"), B=s.B, T=s.T)
+    assert layer.status() == 0
+    Ys = X @ fr.What.T
+    Yc = mon.monarch_inference(X, fr, s.lam, s.B, s.T) - Ys
+    Yo = Ys + bias + 0.6 * Yc
+    assert oracle.rel_fro(Y.double().cpu().numpy(), Yo) <= TOL["bf16"]
+    with pytest.raises(dyra.DyraError) as e:
+        layer.set_als_iterations(2)
+    assert e.value.code == dyra.DYRA_ERR_UNSUPPORTED
     layer.close()
 
 
