@@ -484,6 +484,89 @@ def per_config(names, dev, pk, steps, warmup, headline_entry=None):
     return entries, clk
 
 
+def extras(dev, steps, warmup):
+    """The NEXT rows, timed and checked like the workloads: the ViT-L fc1 layer
+    with a bias and a correction weight ([DyRA] Sec. 2.4), with t = 1.5 and 2
+    ALS iterations (Sec. 3.3), with the Newton-Schulz solver (Sec. 2.4), and a
+    Monarch static part (App. B) on the ViT-L block proj shape, each beside the
+    plain layer's time and checked against the oracle on whole instances."""
+    import torch
+    import oracle
+    from oracle import monarch as mon
+    from rank_structured_matmul_b200 import dyra, prep
+    from synth import generate, spec
+    timer = Timer(dev)
+    out = {}
+    s = spec("vit_fc1")
+    run = LayerRun(s, dev)
+    n_inst = 5
+    rows = n_inst * s.T
+    fo, (Xr, Ur, Vr, Pr, Wr) = oracle_inputs(s, run.w)
+    Xs = Xr[:rows]
+    base_us = timer(run.step, steps, warmup) * 1e3
+
+    def check(Yo):
+        return oracle.rel_fro(run.Y[:rows].double().cpu().numpy(), Yo)
+
+    bias = oracle.round_to(np.random.default_rng(11).standard_normal(s.d_out) * 0.3, "bf16")
+    run.layer.set_linear(torch.from_numpy(bias), 0.7)
+    us = timer(run.step, steps, warmup) * 1e3
+    out["vit_fc1_bias_alpha"] = {
+        "us": us, "plain_us": base_us, "overhead": us / base_us - 1.0,
+        "rel_fro_vs_oracle": check(oracle.inference(Xs, Ur, Vr, Pr, Wr, s.lam, n_inst, s.T,
+                                                    bias=bias, alpha=0.7)),
+        "device_status": run.layer.status()}
+    run.layer.set_linear(None, 1.0)
+    for t in (1.5, 2.0):
+        run.layer.set_als_iterations(t)
+        us = timer(run.step, steps, warmup) * 1e3
+        out["vit_fc1_t%g" % t] = {
+            "us": us, "plain_us": base_us, "launches": {1.5: 9, 2.0: 13}[t],
+            "rel_fro_vs_oracle": check(oracle.als_inference(Xs, Ur, Vr, Wr, fo.R0, s.lam, n_inst,
+                                                            s.T, t)),
+            "device_status": run.layer.status()}
+    run.layer.set_als_iterations(1)
+    dyra.dyra_set_solver(run.layer.plan, dyra.DYRA_SOLVER_NEWTON_SCHULZ, 40)
+    us = timer(run.step, steps, warmup) * 1e3
+    out["vit_fc1_newton_schulz"] = {
+        "us": us, "plain_us": base_us,
+        "rel_fro_vs_oracle": check(oracle.inference(Xs, Ur, Vr, Pr, Wr, s.lam, n_inst, s.T)),
+        "device_status": run.layer.status()}
+    run.close()
+
+    # Monarch static part, b1 = b2 = 32, on the ViT-L block proj shape
+    sm = spec("vit_block_proj")
+    w = generate(sm)
+    b = 32
+    f = prep.prepare_monarch(w.weight(), b, b, sm.k, sm.lam)
+    td = torch.bfloat16
+    layer = dyra.DyraMonarchLinear(sm.d_in, b, b, sm.k, "bf16")
+    layer.load(f.Lblocks, f.Rblocks, f.P, f.W_res, sm.lam)
+    X = torch.from_numpy(w.X).to(dev, td)
+    Y = torch.empty(sm.N, sm.d_out, device=dev, dtype=td)
+    mstep = lambda: layer.forward(X, B=sm.B, T=sm.T, Y=Y)
+    us = timer(mstep, steps, warmup) * 1e3
+    Wd = torch.from_numpy(w.weight()).to(dev, td)
+    Yd = torch.empty_like(Y)
+    dense_us = timer(lambda: torch.matmul(X, Wd.t(), out=Yd), steps, 3) * 1e3
+    rd = lambda a: oracle.round_to(np.asarray(a), "bf16")
+    Lb, Rb = rd(f.Lblocks.numpy()), rd(f.Rblocks.numpy())
+    fr = mon.MonarchFactors(list(Lb), list(Rb), mon.monarch_matrix(list(Lb), list(Rb)).T,
+                            rd(f.P.numpy()), rd(f.W_res.numpy()), None)
+    Xm = rd(w.X[:rows])
+    Yo = mon.monarch_inference(Xm, fr, sm.lam, n_inst, sm.T)
+    Ydense = oracle.dense(Xm, w.weight())
+    out["vit_block_proj_monarch"] = {
+        "us": us, "cublas_dense_us": dense_us, "speedup_vs_cublas_dense": dense_us / us,
+        "blocks": [b, b], "k": sm.k,
+        "rel_fro_vs_oracle": oracle.rel_fro(Y[:rows].double().cpu().numpy(), Yo),
+        "oracle_err_weight_only": oracle.rel_fro(Xm @ fr.What.T, Ydense),
+        "oracle_err_dyra": oracle.rel_fro(Yo, Ydense),
+        "device_status": layer.status()}
+    layer.close()
+    return out
+
+
 def dataclass_prefix(w, s):
     """The N-row prefix of a larger draw of the same layer."""
     import dataclasses
@@ -649,6 +732,7 @@ def run_dyra(args):
         line["per_config"] = entries
         line["per_config_clocks"] = clk_pc
         line["per_config_steps"] = args.per_config_steps
+        line["extras"] = extras(dev, args.per_config_steps, 5)
     for r in runs:
         r.close()
     if rank == 0:

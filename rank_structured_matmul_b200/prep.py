@@ -66,3 +66,42 @@ def prepare_from_svd(left, sigma, right, r: int, k: int, lam: float, R0=None) ->
         return LayerFactors(U, V, torch.zeros(right.shape[0], 0, dtype=torch.float64), W_res)
     R0 = left[:, r:r + k].T if R0 is None else _start(R0, k)
     return LayerFactors(U, V, _p_from_r0(W_res, R0, lam), W_res)
+
+
+class MonarchLayerFactors(NamedTuple):
+    Lblocks: torch.Tensor  # b2 x b1 x b1o: L_j2[m1][j1]
+    Rblocks: torch.Tensor  # b1o x b2 x b2o: R_j1[j2][i2]
+    P: torch.Tensor        # d_in x k
+    W_res: torch.Tensor    # d_out x d_in
+
+
+def prepare_monarch(W, b1: int, b2: int, k: int, lam: float, b1o=None, b2o=None,
+                    R0=None) -> MonarchLayerFactors:
+    """Offline preparation with a Monarch static part ("DyRA: Dynamic Residual
+    Approximation for Efficient Matrix Multiplication in DNNs", App. B, and
+    Alg. 1 Offline) for W of shape d_out x d_in, d_in = b1 b2, d_out = b1o b2o
+    (b1o = b1, b2o = b2 unless given). In the paper's layout W^T, entry
+    (m1 b2 + j2, j1 b2o + i2) of the Monarch matrix is L_j2[m1][j1] R_j1[j2][i2],
+    so each block of rows m1 b2 + j2 (m1 < b1) and columns j1 b2o + i2 is rank
+    one: its best rank-1 approximation sqrt(s) u . sqrt(s) v^T gives column j1
+    of L_j2 and row j2 of R_j1. W_res = W - W_hat^T, R0 the top-k output-side
+    singular vectors of W_res unless given, and the projector P of Eq. 7."""
+    b1o = b1 if b1o is None else b1o
+    b2o = b2 if b2o is None else b2o
+    W = torch.as_tensor(W, dtype=torch.float64).cpu()
+    if W.shape != (b1o * b2o, b1 * b2):
+        raise ValueError("W must be %d x %d" % (b1o * b2o, b1 * b2))
+    # blocks[j2][j1] = the b1 x b2o block of rows m1 b2 + j2, columns j1 b2o + i2
+    blocks = W.T.reshape(b1, b2, b1o, b2o).permute(1, 2, 0, 3)
+    u, s, vh = torch.linalg.svd(blocks)
+    root = s[..., 0].sqrt()
+    Lb = (u[..., :, 0] * root[..., None]).permute(0, 2, 1).contiguous()   # [j2][m1][j1]
+    Rb = (vh[..., 0, :] * root[..., None]).permute(1, 0, 2).contiguous()  # [j1][j2][i2]
+    What_p = torch.einsum("bmj,jbi->mbji", Lb, Rb).reshape(b1 * b2, b1o * b2o)
+    W_res = W - What_p.T
+    if k == 0:
+        return MonarchLayerFactors(Lb, Rb, torch.zeros(W.shape[1], 0, dtype=torch.float64), W_res)
+    if R0 is None:
+        R0 = torch.linalg.svd(W_res, full_matrices=False)[0][:, :k].T
+    return MonarchLayerFactors(Lb, Rb, _p_from_r0(W_res, _start(R0, k), lam), W_res)
+

@@ -39,3 +39,21 @@ def test_k0_shapes():
     w = _layer()
     a = prep.prepare_from_svd(w.left, w.sigma, w.right, 6, 0, 0.0)
     assert a.P.shape == (40, 0)
+
+
+def test_monarch_preparation_matches_the_oracle():
+    """The host Monarch preparation (torch) and the oracle's (NumPy), written
+    independently, give the same static matrix and residual, square and
+    rectangular (signs of the block factors may differ; their products may not)."""
+    import numpy as np
+    from oracle import monarch as mon
+    rng = np.random.default_rng(3)
+    for b1, b2, b1o, b2o in ((4, 3, 4, 3), (4, 3, 2, 5)):
+        W = rng.standard_normal((b1o * b2o, b1 * b2))
+        f = prep.prepare_monarch(W, b1, b2, 2, 1e-3, b1o, b2o)
+        fo = mon.offline_prepare_monarch(W, b1, b2, 2, 1e-3, b1o=b1o, b2o=b2o)
+        np.testing.assert_allclose(f.W_res.numpy(), fo.W_res, rtol=0, atol=1e-12)
+        What = mon.monarch_matrix(list(f.Lblocks.numpy()), list(f.Rblocks.numpy())).T
+        np.testing.assert_allclose(What, fo.What, rtol=0, atol=1e-12)
+        Pn = f.P.numpy()
+        np.testing.assert_allclose(np.abs(Pn), np.abs(fo.P), rtol=0, atol=1e-10)
