@@ -63,8 +63,9 @@ constexpr uint32_t kStoreBoxBytes = 128u * 128u;  // 128 rows x 64 bf16
 constexpr uint32_t kStoreBoxes = 2;
 
 // With LO set, the box receives the low part of each value instead,
-// bf16(v - bf16(v)): the two boxes together carry v to about 16 bits.
-template <bool LO = false>
+// bf16(v - bf16(v)): the two boxes together carry v to about 16 bits. BIAS
+// compiles the bias add in (the callers without one keep the plain loop).
+template <bool LO = false, bool BIAS = false>
 __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const void* tmap, int x,
                                                int y, EpiCtx& e,
                                                const __nv_bfloat16* bias = nullptr,
@@ -80,7 +81,7 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
   named_bar_sync(1, 128);
   uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
   tmem_ld_wait();
-  if (bias != nullptr) {
+  if constexpr (BIAS) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -126,51 +127,6 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
   }
 }
 
-// The second half of store_box_bf16 for a box whose accumulator values the
-// caller already holds (loaded and waited for): lets the caller load the next
-// box from TMEM while this one is converted and stored.
-__device__ __forceinline__ void store_loaded_box_bf16(const uint32_t (&vv)[2][32], const void* tmap,
-                                                      int x, int y, EpiCtx& e,
-                                                      const __nv_bfloat16* bias = nullptr,
-                                                      int ncols = 0) {
-  const uint32_t buf = e.counter % kStoreBoxes;
-  ++e.counter;
-  if (e.tid == 0) tma_store_wait_read<kStoreBoxes - 1>();
-  named_bar_sync(1, 128);
-  uint8_t* sbuf = e.smem + buf * kStoreBoxBytes;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      const int chunk = half * 4 + ch;
-      const uint32_t off =
-          static_cast<uint32_t>(e.row) * 128u + static_cast<uint32_t>((chunk ^ (e.row & 7)) * 16);
-      float b[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
-      if (bias != nullptr && c < ncols) {
-        const uint4 bq = __ldg(reinterpret_cast<const uint4*>(bias + c));
-        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          b[2 * jj] = __uint_as_float(w[jj] << 16);
-          b[2 * jj + 1] = __uint_as_float(w[jj] & 0xffff0000u);
-        }
-      }
-      uint4 q;
-      q.x = pack_bf16x2(f32(vv[half][8 * ch + 0]) + b[0], f32(vv[half][8 * ch + 1]) + b[1]);
-      q.y = pack_bf16x2(f32(vv[half][8 * ch + 2]) + b[2], f32(vv[half][8 * ch + 3]) + b[3]);
-      q.z = pack_bf16x2(f32(vv[half][8 * ch + 4]) + b[4], f32(vv[half][8 * ch + 5]) + b[5]);
-      q.w = pack_bf16x2(f32(vv[half][8 * ch + 6]) + b[6], f32(vv[half][8 * ch + 7]) + b[7]);
-      *reinterpret_cast<uint4*>(sbuf + off) = q;
-    }
-  }
-  fence_async_shared();
-  named_bar_sync(1, 128);
-  if (e.tid == 0) {
-    tma_store_2d(tmap, e.smem_u32 + buf * kStoreBoxBytes, x, y);
-    tma_store_commit();
-  }
-}
 
 __device__ __forceinline__ void store_drain(EpiCtx& e) {
   if (e.tid == 0) tma_store_wait_all();
@@ -380,7 +336,11 @@ struct ProjPolicy {
 // its fp32 partial tile in its own operand stages and, after a cluster
 // barrier, sums one slice of rows over all S partials through distributed
 // shared memory (split-K, as in the projection).
-struct GramPolicy {
+// kAls: the options the L update of further ALS iterations needs (an X view
+// shared by every instance, and T and G in fp32 as B x k x (d_in + k)); the
+// one-step layer's Gram stage is compiled without them.
+template <bool kAls>
+struct GramPolicyT {
   struct Params {
     GemmCommon c;
     CUtensorMap tmX;   // (d_in, T, B), box (64, 64, 1), 128B swizzle
@@ -434,7 +394,7 @@ struct GramPolicy {
     const int row = t.t0 + it * 64;
     if (t.mt < p.mtx) {
       const int j0 = t.mt * 128;
-      const int bx = p.x_inst_fixed ? 0 : t.b;
+      const int bx = kAls && p.x_inst_fixed ? 0 : t.b;
       tma_load_3d(sa, &p.tmX, bar, j0, row, bx);
       tma_load_3d(sa + 8192u, &p.tmX, bar, j0 + 64, row, bx);
     } else {
@@ -460,7 +420,7 @@ struct GramPolicy {
   template <int n>
   static __device__ __forceinline__ void store_row(const Params& p, const Tile& t, int row, int i0,
                                                    const float (&v)[n]) {
-    if (p.TGf != nullptr) {
+    if (kAls && p.TGf != nullptr) {
       const int J = p.d_in + p.k;
       float* inst = p.TGf + static_cast<size_t>(t.b) * p.k * J;
       int col;  // column of instance b's k x J block that this thread's row feeds
@@ -575,11 +535,18 @@ struct GramPolicy {
   }
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
 };
+using GramPolicy = GramPolicyT<false>;
+using GramAlsPolicy = GramPolicyT<true>;
+
 
 // ================================================================ rfactor ====
 // C^T = W_res . T'^T (d_out x B*k): A = W_res (K-major), B = T' (K-major).
 // W_res is streamed from HBM once per n-tile column of C^T.
 struct RFactorPolicy {
+  // The solve's blocks (152 registers) run beside this GEMM's on the same SMs:
+  // a register partition then holds two warps of each (2*152*32 + 2*104*32 =
+  // 16384 registers), so the GEMM is held to 104.
+  static constexpr int kMaxRegs = 104;
   struct Params {
     GemmCommon c;
     CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
@@ -695,7 +662,7 @@ struct OutPolicy {
     ch = jj - sub * p.nkl;
   }
   struct Tile {
-    int m0, n0, b_lo, nseg, z_lo, z_nseg;
+    int m0, n0, b_lo, nseg, z_lo, z_nseg, ns;  // ns: the static part's K-steps
   };
   static constexpr uint32_t kEpiSmemBytes = kStoreBoxes * kStoreBoxBytes;
 
@@ -724,13 +691,14 @@ struct OutPolicy {
       t.nseg = 0;
     }
     static_blocks(p, t.n0, t.z_lo, t.z_nseg);
+    t.ns = static_iters(p, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return static_iters(p, t.z_nseg) + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
-    const int ns = static_iters(p, t.z_nseg);
+    const int ns = t.ns;
     if (it < ns) {
       if (p.zb_w > 0) {
         const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
@@ -749,9 +717,8 @@ struct OutPolicy {
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
-    const int ns = static_iters(p, t.z_nseg);
-    if (it < ns) return static_ksteps(p, it);
-    const int ch = (it - ns) % p.nkl;
+    if (it < t.ns) return static_ksteps(p, it);
+    const int ch = (it - t.ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
@@ -762,28 +729,13 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    // The next box's TMEM loads are in flight while this box is converted and
-    // stored (tcgen05.wait::ld waits for every earlier load of the thread, so
-    // each wait comes after the previous box is written out).
-    const int nb = p.bn / 64;
-    uint32_t va[2][32], vb[2][32];
-    tmem_ld_32x32b_x32(tacc, va[0]);
-    tmem_ld_32x32b_x32(tacc + 32, va[1]);
-    tmem_ld_wait();
-    for (int bx = 0; bx < nb; bx += 2) {
-      if (bx + 1 < nb) {
-        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64, vb[0]);
-        tmem_ld_32x32b_x32(tacc + (bx + 1) * 64 + 32, vb[1]);
-      }
-      store_loaded_box_bf16(va, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias, p.d_out);
-      if (bx + 1 >= nb) break;
-      tmem_ld_wait();
-      if (bx + 2 < nb) {
-        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64, va[0]);
-        tmem_ld_32x32b_x32(tacc + (bx + 2) * 64 + 32, va[1]);
-      }
-      store_loaded_box_bf16(vb, &p.tmY, t.n0 + (bx + 1) * 64, t.m0, e, p.bias, p.d_out);
-      tmem_ld_wait();
+    if (p.bias != nullptr) {
+      for (int bx = 0; bx < p.bn / 64; ++bx)
+        store_box_bf16<false, true>(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias,
+                                    p.d_out);
+    } else {
+      for (int bx = 0; bx < p.bn / 64; ++bx)
+        store_box_bf16(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e);
     }
   }
   static __device__ __forceinline__ bool cluster_finish(const Params&) { return false; }
@@ -876,6 +828,7 @@ struct XRwPolicy {
 // of W_res and rows n0 + (bn/2) r of T' and stores its 128 rows of C^T.
 struct RFactorPairPolicy {
   using Params = RFactorPolicy::Params;  // tmT box is (64, bn/2) here
+  static constexpr int kMaxRegs = RFactorPolicy::kMaxRegs;
   using Tile = RFactorPolicy::Tile;
   static constexpr uint32_t kEpiSmemBytes = RFactorPolicy::kEpiSmemBytes;
   static __device__ __forceinline__ void prefetch(const Params& p) { RFactorPolicy::prefetch(p); }
@@ -960,7 +913,7 @@ struct ProjPairPolicy {
 struct OutPairPolicy {
   using Params = OutPolicy::Params;  // tmU / tmC boxes are (64, bn/2) here
   struct Tile {
-    int m0, n0, b_lo, nseg, z_lo, z_nseg;
+    int m0, n0, b_lo, nseg, z_lo, z_nseg, ns;
   };
   static constexpr uint32_t kEpiSmemBytes = OutPolicy::kEpiSmemBytes;
 
@@ -977,15 +930,16 @@ struct OutPairPolicy {
       t.nseg = 0;
     }
     OutPolicy::static_blocks(p, t.n0, t.z_lo, t.z_nseg);
+    t.ns = OutPolicy::static_iters(p, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return OutPolicy::static_iters(p, t.z_nseg) + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
     const int ma = t.m0 + 128 * static_cast<int>(rank);
     const int nb = t.n0 + (p.bn / 2) * static_cast<int>(rank);
-    const int ns = OutPolicy::static_iters(p, t.z_nseg);
+    const int ns = t.ns;
     if (it < ns) {
       if (p.zb_w > 0) {
         const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
@@ -1004,9 +958,8 @@ struct OutPairPolicy {
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
-    const int ns = OutPolicy::static_iters(p, t.z_nseg);
-    if (it < ns) return OutPolicy::static_ksteps(p, it);
-    const int ch = (it - ns) % p.nkl;
+    if (it < t.ns) return OutPolicy::static_ksteps(p, it);
+    const int ch = (it - t.ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
@@ -1024,6 +977,7 @@ struct OutPairPolicy {
     h.nseg = t.nseg;
     h.z_lo = t.z_lo;
     h.z_nseg = t.z_nseg;
+    h.ns = t.ns;
     OutPolicy::epilogue(p, h, tacc, e);
   }
   static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
@@ -1269,9 +1223,10 @@ struct GramStage {
   unsigned long long wait_ns;
 };
 
-int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cudaStream_t s,
-                      bool pdl) {
-  GramPolicy::Params p;
+template <class Pol>
+int launch_gram_stage_as(const GramStage& g, int* status, const DeviceInfo& dev, cudaStream_t s,
+                         bool pdl) {
+  typename Pol::Params p;
   p.d_in = g.d_in;
   p.k = g.k;
   p.kpad = g.k <= 32 ? 32 : ceil_div(g.k, 64) * 64;
@@ -1296,7 +1251,7 @@ int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cu
   if (!encode_tmap_bf16(&p.tmLb, g.L, 3, g.ld, g.ls, bl, p.w * 2)) return -2;
   const int tiles = p.mt_total * p.B * p.S;
   const uint32_t smem =
-      setup_common<GramPolicy>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
+      setup_common<Pol>(p.c, tiles, 128 * 128, static_cast<uint32_t>(p.kpad) * 128,
                                p.kpad, true, true, status, dev);
   if (!smem) return -3;
   // split rows keep a 128 x kpad fp32 partial in the operand stages
@@ -1305,7 +1260,14 @@ int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cu
     return -3;
   p.c.trace = g.trace;
   if (g.wait_ns) p.c.wait_ns = g.wait_ns;
-  return launch_gemm<GramPolicy>(p, smem, dev, s, pdl, p.S) ? -1 : 0;
+  return launch_gemm<Pol>(p, smem, dev, s, pdl, p.S) ? -1 : 0;
+}
+
+int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cudaStream_t s,
+                      bool pdl) {
+  return g.TGf != nullptr || g.x_inst_fixed
+             ? launch_gram_stage_as<GramAlsPolicy>(g, status, dev, s, pdl)
+             : launch_gram_stage_as<GramPolicy>(g, status, dev, s, pdl);
 }
 
 // The Gram stage of the layer: L_b^T [X_b | L_b] per instance, L = a.L.

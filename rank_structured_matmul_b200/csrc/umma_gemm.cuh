@@ -27,6 +27,8 @@
 //   static constexpr uint32_t kEpiSmemBytes;
 #pragma once
 
+#include <type_traits>
+
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -135,8 +137,20 @@ __host__ __device__ inline uint32_t gemm_smem_bytes(int stages, uint32_t a_bytes
   return 1024u + static_cast<uint32_t>(stages) * (a_bytes + b_bytes) + epi_bytes + 256u;
 }
 
+// Register cap of a policy's kernel: Pol::kMaxRegs if it declares one (a
+// GEMM that must share its SMs with another kernel's blocks), else the
+// hardware limit.
+template <class Pol, class = void>
+struct MaxRegs {
+  static constexpr int value = 255;
+};
 template <class Pol>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+struct MaxRegs<Pol, std::void_t<decltype(Pol::kMaxRegs)>> {
+  static constexpr int value = Pol::kMaxRegs;
+};
+
+template <class Pol>
+__global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::value)
     umma_gemm_kernel(const __grid_constant__ typename Pol::Params p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];

@@ -27,6 +27,7 @@ namespace dyra {
 
 template <class Pol>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    __maxnreg__(MaxRegs<Pol>::value)
     umma_gemm_pair_kernel(const __grid_constant__ typename Pol::Params p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
