@@ -476,6 +476,8 @@ def per_config(names, dev, pk, steps, warmup, headline_entry=None):
                 tl = timer(r.step, steps, 3)
                 tdl = timer(r.dense_step, steps, 3)
                 e["layers"][r.s.name] = {"us": tl * 1e3, "cublas_dense_us": tdl * 1e3}
+        else:
+            e["static_matched"] = static_entry(runs[0], timer, steps)
         for r in runs:
             r.free_dense()
             r.close()
@@ -564,6 +566,28 @@ def extras(dev, steps, warmup):
         "oracle_err_dyra": oracle.rel_fro(Yo, Ydense),
         "device_status": layer.status()}
     layer.close()
+    return out
+
+
+def static_entry(run, timer, steps):
+    """The FLOPs-matched static layer of one workload ([DyRA] App. E.4; NEXT
+    f1): rank, time, and the oracle's error of it and of DyRA against the
+    dense product on the parity rows."""
+    import torch
+    import oracle
+    from rank_structured_matmul_b200 import dyra
+    s, w = run.s, run.w
+    rs = static_matched_rank(s)
+    st = dyra.DyraLinear(s.d_in, s.d_out, rs, 0, s.dtype)
+    st.load(torch.as_tensor(np.ascontiguousarray(w.left[:, :rs] * w.sigma[:rs])),
+            torch.as_tensor(np.ascontiguousarray(w.right[:, :rs])), None, None, s.lam)
+    Ys = torch.empty_like(run.Y)
+    us = timer(lambda: st.forward(run.X, B=s.B, T=s.T, Y=Ys), steps, 3) * 1e3
+    errs = static_errors([(run, rs, st, Ys)])
+    out = {"rank": rs, "r_plus_k": s.r + s.k, "us": us, "device_status": st.status(),
+           "oracle_err_vs_dense": errs["oracle_err_vs_dense"][0],
+           "rel_fro_vs_oracle": errs["rel_fro_vs_oracle"]}
+    st.close()
     return out
 
 

@@ -184,9 +184,19 @@ struct ProjPolicy {
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
-    const int kg = t.ks * p.kper + it;
-    tma_load_2d(sa, &p.tmX, bar, kg * 64, t.m0);
-    tma_load_2d(sb, &p.tmW, bar, kg * 64, t.n0);
+    load_early(p, t, it, sa, sb, bar);
+    load_late(p, t, it, sa, sb, bar);
+  }
+  // [V | P]^T is a loaded weight, ready before any grid of the forward runs;
+  // X may be the output of the grid just before this one.
+  static constexpr bool kEarly = true;
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t, uint32_t sb, uint32_t bar) {
+    tma_load_2d(sb, &p.tmW, bar, (t.ks * p.kper + it) * 64, t.n0);
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t sa, uint32_t, uint32_t bar) {
+    tma_load_2d(sa, &p.tmX, bar, (t.ks * p.kper + it) * 64, t.m0);
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
     return min(4, ceil_div_dev(p.d_in - (t.ks * p.kper + it) * 64, 16));
@@ -579,7 +589,17 @@ struct RFactorPolicy {
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
+    load_early(p, t, it, sa, sb, bar);
+    load_late(p, t, it, sa, sb, bar);
+  }
+  // W_res is a loaded weight; T comes from the Gram stage, the grid before.
+  static constexpr bool kEarly = true;
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t sa, uint32_t, uint32_t bar) {
     tma_load_2d(sa, &p.tmW, bar, it * 64, t.m0);
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t, uint32_t sb, uint32_t bar) {
     tma_load_2d(sb, &p.tmT, bar, it * 64, t.n0);
     if (p.split_t) tma_load_2d(sb + static_cast<uint32_t>(p.bn) * 128u, &p.tmTlo, bar, it * 64, t.n0);
   }
@@ -695,6 +715,20 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
     return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+  }
+  // With Params::early (set only where the grid chain guarantees it: the
+  // rank-k GEMM before the solve triggers its dependents only after its own
+  // wait, so Z of the projection is complete before this grid launches) the
+  // static stages (Z and U) are loaded before the dependency wait and their
+  // MMAs may run before it ends; the correction's operands come after it.
+  static constexpr bool kEarly = true;
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t sa, uint32_t sb, uint32_t bar) {
+    if (it < t.ns) load(p, t, it, sa, sb, bar);
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t sa, uint32_t sb, uint32_t bar) {
+    if (it >= t.ns) load(p, t, it, sa, sb, bar);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar) {
@@ -841,7 +875,18 @@ struct RFactorPairPolicy {
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
+    load_early(p, t, it, sa, sb, bar, rank);
+    load_late(p, t, it, sa, sb, bar, rank);
+  }
+  static constexpr bool kEarly = true;  // as RFactorPolicy: W_res early, T late
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t sa, uint32_t, uint32_t bar,
+                                                    uint32_t rank) {
     tma_load_2d_pair(sa, &p.tmW, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t, uint32_t sb, uint32_t bar,
+                                                   uint32_t rank) {
     tma_load_2d_pair(sb, &p.tmT, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
     if (p.split_t)
       tma_load_2d_pair(sb + static_cast<uint32_t>(p.bn / 2) * 128u, &p.tmTlo, bar, it * 64,
@@ -884,8 +929,19 @@ struct ProjPairPolicy {
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
-    tma_load_2d_pair(sa, &p.tmX, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
+    load_early(p, t, it, sa, sb, bar, rank);
+    load_late(p, t, it, sa, sb, bar, rank);
+  }
+  static constexpr bool kEarly = true;  // as ProjPolicy: [V | P]^T early, X late
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t, uint32_t sb, uint32_t bar,
+                                                    uint32_t rank) {
     tma_load_2d_pair(sb, &p.tmW, bar, it * 64, t.n0 + (p.bn / 2) * static_cast<int>(rank));
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t sa, uint32_t, uint32_t bar,
+                                                   uint32_t rank) {
+    tma_load_2d_pair(sa, &p.tmX, bar, it * 64, t.m0 + 128 * static_cast<int>(rank));
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
     return ProjPolicy::ksteps(p, t, it);
@@ -934,6 +990,17 @@ struct OutPairPolicy {
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
     return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+  }
+  static constexpr bool kEarly = true;  // as OutPolicy: static stages early
+  static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
+                                                    uint32_t sa, uint32_t sb, uint32_t bar,
+                                                    uint32_t rank) {
+    if (it < t.ns) load(p, t, it, sa, sb, bar, rank);
+  }
+  static __device__ __forceinline__ void load_late(const Params& p, const Tile& t, int it,
+                                                   uint32_t sa, uint32_t sb, uint32_t bar,
+                                                   uint32_t rank) {
+    if (it >= t.ns) load(p, t, it, sa, sb, bar, rank);
   }
   static __device__ __forceinline__ void load(const Params& p, const Tile& t, int it, uint32_t sa,
                                               uint32_t sb, uint32_t bar, uint32_t rank) {
@@ -1009,6 +1076,7 @@ uint32_t setup_common(GemmCommon& c, int num_tiles, uint32_t a_bytes, uint32_t b
   c.b_parts = 1;
   c.b_part_desc = 0;
   c.wait_ns = sm100::kWaitLimitNs;
+  c.early = 0;
   c.a_stage_bytes = a_bytes;
   c.b_stage_bytes = b_bytes;
   c.acc_cols = static_cast<uint32_t>((mma_n + 31) / 32 * 32);
@@ -1354,6 +1422,7 @@ int launch_rfactor_stage(const RFactorStage& r, const Bf16Forward& a, const Devi
     p.c.b_parts = parts;
     p.c.b_part_desc = part_bytes >> 4;
     p.c.trigger_after_wait = 1;
+    p.c.early = pdl ? 1 : 0;  // W_res before the wait
     p.c.idesc = idesc_bf16(256, p.bn, false, false);
     p.c.trace = r.trace;
     return launch_gemm_pair<RFactorPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
@@ -1367,6 +1436,7 @@ int launch_rfactor_stage(const RFactorStage& r, const Bf16Forward& a, const Devi
   p.c.b_parts = parts;
   p.c.b_part_desc = part_bytes >> 4;
   p.c.trigger_after_wait = 1;
+  p.c.early = pdl ? 1 : 0;  // W_res before the wait
   p.c.trace = r.trace;
   return launch_gemm<RFactorPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
 }
@@ -1385,9 +1455,13 @@ struct OutStatic {
 // The output stage Y = (static part) (+ bias) + sum_b mask_b(L) C_b with the
 // correction's left factor L (N x k) and right factor C^T (d_out x B*k)
 // (k = 0: the static part alone), with their low parts when hilo.
+// early_static: the static operands are complete when this grid launches (it
+// follows the correction chain, or a grid that does not trigger early), so
+// they may be loaded before the dependency wait.
 int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const void* Ct,
                      const void* Ctlo, bool hilo, int k, int d_out, void* Y, const void* bias,
-                     const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl) {
+                     const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl,
+                     bool early_static = false) {
   const int64_t N = a.B * a.T;
   OutPolicy::Params p;
   p.N = static_cast<int>(N);
@@ -1462,6 +1536,7 @@ int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const 
     if (!smem) return -3;
     p.c.idesc = idesc_bf16(256, p.bn, false, false);
     p.c.trace = tr;
+    p.c.early = pdl && early_static ? 1 : 0;
     return launch_gemm_pair<OutPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
   }
   const int tiles = ceil_div(N, 128) * p.n_tiles_n;
@@ -1469,6 +1544,7 @@ int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const 
                                                 false, a.status, dev);
   if (!smem) return -3;
   p.c.trace = tr;
+  p.c.early = pdl && early_static ? 1 : 0;
   return launch_gemm<OutPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
 }
 
@@ -1553,6 +1629,7 @@ int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* cou
     if (!smem) return -3;
     p.c.idesc = idesc_bf16(256, p.bn, false, false);
     p.c.trace = tr;
+    p.c.early = pdl ? 1 : 0;  // [V | P]^T before the wait
     return launch_gemm_pair<ProjPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
   }
   const uint32_t smem = setup_common<ProjPolicy>(p.c, ps.tiles * p.ksplit, 128 * 128,
@@ -1563,6 +1640,7 @@ int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* cou
                           static_cast<size_t>(128) * p.bn * 4)
     return -3;
   p.c.trace = tr;
+  p.c.early = pdl ? 1 : 0;  // [V | P]^T before the wait
   return launch_gemm<ProjPolicy>(p, smem, dev, s, pdl, p.ksplit) ? -1 : 0;
 }
 
@@ -1742,7 +1820,7 @@ int launch_bf16_monarch(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   mark_stage(a, 4, s);
   const OutStatic st2 = {a.Xs, nmid, a.Rt, a.mb2o, a.mb2, a.mb1o};
   if (launch_out_stage(st2, a.L, nullptr, a.Ct, nullptr, false, k, a.d_out, a.Y, a.bias, a, dev,
-                       s, true))
+                       s, true, /*early_static=*/true))
     return -1;
   mark_stage(a, 5, s);
   return 0;
@@ -1769,7 +1847,7 @@ int launch_bf16_forward(const Bf16Forward& a, const DeviceInfo& dev, cudaStream_
   mark_stage(a, 4, s);
   const OutStatic st = {a.Z, a.r, a.U, 0, 0, 0};
   if (launch_out_stage(st, a.L, a.Llo, a.Ct, a.Ctlo, a.hilo, k, a.d_out, a.Y, a.bias, a, dev, s,
-                       pdl))
+                       pdl, /*early_static=*/k > 0))
     return -1;
   mark_stage(a, 5, s);
   return 0;

@@ -86,6 +86,11 @@ struct GemmCommon {
   // limit of one pipeline wait in ns (sm100::kWaitLimitNs; a diagnostic may
   // shorten it to make a wait run out). Drains keep kWaitLimitNs.
   unsigned long long wait_ns;
+  // 1: the producer issues the operands of the first tile's first stages that
+  // do not depend on earlier grids (Pol::load_early) before the dependency
+  // wait, and the rest (Pol::load_late) after it; only the producer and the
+  // epilogue wait. Policies opt in with kEarly.
+  int early;
 };
 
 // Issues one stage's ks MMAs (K = 16 each) back to back. The tensor pipe idles
@@ -149,6 +154,17 @@ struct MaxRegs<Pol, std::void_t<decltype(Pol::kMaxRegs)>> {
   static constexpr int value = Pol::kMaxRegs;
 };
 
+// Whether a policy can split its first stages' copies around the dependency
+// wait (Pol::kEarly, with load_early / load_late).
+template <class Pol, class = void>
+struct HasEarly {
+  static constexpr bool value = false;
+};
+template <class Pol>
+struct HasEarly<Pol, std::void_t<decltype(Pol::kEarly)>> {
+  static constexpr bool value = Pol::kEarly;
+};
+
 template <class Pol>
 __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::value)
     umma_gemm_kernel(const __grid_constant__ typename Pol::Params p) {
@@ -208,9 +224,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
   // Every CTA of this grid is resident (grid <= SMs), so the next kernel in
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
+  // early: the producer waits after its first copies, the epilogue before
+  // its first output, and the MMA warp (shared memory and TMEM only) never.
+  const bool early = HasEarly<Pol>::value && c.early && !c.defer_wait;
   if (!c.trigger_after_wait) pdl_launch_dependents();
-  if (!c.defer_wait) pdl_wait();
-  if (c.trigger_after_wait) pdl_launch_dependents();
+  if (!c.defer_wait && !early) pdl_wait();
+  if (c.trigger_after_wait && !early) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status, c.wait_ns};
@@ -223,11 +242,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int pre = 0;  // stages of the first tile issued around the dependency wait
+      if constexpr (HasEarly<Pol>::value) {
+        if (early) {
+          typename Pol::Tile t0;
+          if (blockIdx.x < c.num_tiles) {
+            Pol::decode(p, blockIdx.x, t0);
+            pre = min(S, Pol::kiters(p, t0));
+          }
+          for (int it = 0; it < pre; ++it) {  // fresh slots: nothing to wait for
+            mbar_arrive_expect_tx(full_bar(it), c.a_stage_bytes + c.b_stage_bytes);
+            Pol::load_early(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
+                            full_bar(it));
+          }
+          pdl_wait();
+          if (c.trigger_after_wait) pdl_launch_dependents();
+          for (int it = 0; it < pre; ++it) {
+            Pol::load_late(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
+                           full_bar(it));
+            issued |= 1u << it;
+            last_phase[it] = 0;
+          }
+          stage = pre % S;
+          phase = pre == S ? 1u : 0u;
+        }
+      }
       for (int tile = blockIdx.x; ok && tile < c.num_tiles; tile += gridDim.x) {
         typename Pol::Tile t;
         Pol::decode(p, tile, t);
         const int nk = Pol::kiters(p, t);
-        for (int it = 0; it < nk; ++it) {
+        for (int it = tile == static_cast<int>(blockIdx.x) ? pre : 0; it < nk; ++it) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, w)) {
             ok = false;
             break;
@@ -304,6 +348,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
       if (tr) tr[kTrMmaDone] = globaltimer_ns();
     }
   } else {
+    if (early) pdl_wait();
     EpiCtx e;
     e.quad = warp & 3;
     e.lane = lane;

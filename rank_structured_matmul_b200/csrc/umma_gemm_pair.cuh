@@ -89,9 +89,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // Every CTA of this grid is resident (grid <= SMs), so the next kernel in
   // the stream may be launched now: its CTAs take SMs as ours leave and wait
   // in pdl_wait() for our results. This hides launch and set-up latency.
+  // early: as in the single-CTA skeleton (the producer waits after its first
+  // copies, the epilogue before its first output, the MMA warp never)
+  const bool early = HasEarly<Pol>::value && c.early && !c.defer_wait;
   if (!c.trigger_after_wait) pdl_launch_dependents();
-  if (!c.defer_wait) pdl_wait();
-  if (c.trigger_after_wait) pdl_launch_dependents();
+  if (!c.defer_wait && !early) pdl_wait();
+  if (c.trigger_after_wait && !early) pdl_launch_dependents();
   if (tr && threadIdx.x == 0) tr[kTrDepsReady] = globaltimer_ns();
 
   WaitCtx w{abort_flag, c.status, c.wait_ns};
@@ -104,11 +107,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      int pre = 0;  // stages of the first tile issued around the dependency wait
+      if constexpr (HasEarly<Pol>::value) {
+        if (early) {
+          typename Pol::Tile t0;
+          if (pair < c.num_tiles) {
+            Pol::decode(p, pair, t0);
+            pre = min(S, Pol::kiters(p, t0));
+          }
+          for (int it = 0; it < pre; ++it) {  // fresh slots: nothing to wait for
+            if (leader)
+              mbar_arrive_expect_tx(full_bar(it), 2u * (c.a_stage_bytes + c.b_stage_bytes));
+            Pol::load_early(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
+                            full_bar(it), rank);
+          }
+          pdl_wait();
+          if (c.trigger_after_wait) pdl_launch_dependents();
+          for (int it = 0; it < pre; ++it) {
+            Pol::load_late(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
+                           full_bar(it), rank);
+            issued |= 1u << it;
+            last_phase[it] = 0;
+          }
+          stage = pre % S;
+          phase = pre == S ? 1u : 0u;
+        }
+      }
       for (int tile = pair; ok && tile < c.num_tiles; tile += npairs) {
         typename Pol::Tile t;
         Pol::decode(p, tile, t);
         const int nk = Pol::kiters(p, t);
-        for (int it = 0; it < nk; ++it) {
+        for (int it = tile == pair ? pre : 0; it < nk; ++it) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, w)) {
             ok = false;
             break;
@@ -185,6 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (tr) tr[kTrMmaDone] = globaltimer_ns();
     }
   } else {
+    if (early) pdl_wait();
     EpiCtx e;
     e.quad = warp & 3;
     e.lane = lane;
