@@ -33,6 +33,7 @@ struct dyra_plan {
   bool force_simt = false;  // DYRA_KERNELS=simt: CUDA-core kernels for bf16 too (debugging)
   bool use_pairs = true;    // DYRA_PAIR=0: single-CTA output stage (comparison)
   int proj_pair_min_tiles = 0;  // DYRA_PROJ_PAIR_MIN=n: projection pairs from n pair tiles
+  int proj_bn = 0;              // DYRA_PROJ_BN=128|192|256: projection column tile
   // Where G_b is factored (bf16, k <= 64): by every solve block
   // (DYRA_FACTOR=self), once per instance by the first solve block, which
   // publishes it (DYRA_FACTOR=shared), or by size (unset: every block while
@@ -383,6 +384,7 @@ int run_forward(dyra_plan* p, const void* X, void* Y, int64_t B, int64_t T, bool
     a.ns_iters = p->ns_iters;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.proj_bn = p->proj_bn;
     a.bias = p->has_bias ? p->bias : nullptr;
     a.alpha = p->alpha;
     a.hilo = correct && use_hilo(p, B, T);
@@ -624,6 +626,9 @@ static int plan_create_impl(dyra_plan_t* out, int d_in, int d_out, int r, int k,
   p->use_pairs = !(pv != nullptr && pv[0] == '0');
   const char* ppv = std::getenv("DYRA_PROJ_PAIR_MIN");
   p->proj_pair_min_tiles = ppv ? std::atoi(ppv) : 0;
+  const char* pbv = std::getenv("DYRA_PROJ_BN");
+  p->proj_bn = pbv ? std::atoi(pbv) : 0;
+  if (p->proj_bn != 128 && p->proj_bn != 192 && p->proj_bn != 256) p->proj_bn = 0;
   const char* fv = std::getenv("DYRA_FACTOR");
   p->factor_mode = fv == nullptr                     ? -1
                    : std::strcmp(fv, "self") == 0   ? 0
@@ -1224,6 +1229,7 @@ extern "C" int dyra_forward_batched_noalloc(dyra_plan_t p, const void* X, void* 
     a.trace = nullptr;
     a.use_pairs = p->use_pairs;
     a.proj_pair_min_tiles = p->proj_pair_min_tiles;
+    a.proj_bn = p->proj_bn;
     a.bias = p->has_bias ? p->bias : nullptr;
     a.alpha = p->alpha;
     a.solver = p->solver;

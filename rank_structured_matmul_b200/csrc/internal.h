@@ -73,6 +73,7 @@ struct Bf16Forward {
   unsigned long long* trace;  // optional: 5 stages x kTraceCtas x kTraceSlots timestamps
   bool use_pairs;             // run the output stage on CTA pairs
   int proj_pair_min_tiles;    // see proj_shape (0: default)
+  int proj_bn = 0;            // projection column tile 128, 192 or 256 (0: proj_shape's choice)
   const void* bias = nullptr;  // d_out bf16 values added to Y, or nullptr
   float alpha = 1.f;           // weight of the correction (the solve scales L~ by it)
   // Compensated correction: L~ and Q^T are also stored as their bf16 rounding
@@ -127,9 +128,10 @@ struct ProjShape {
   bool pairs;
 };
 // pair_min_tiles: pair tiles needed before the projection runs on CTA pairs
-// (0: a quarter of the SM count).
+// (0: a quarter of the SM count); force_bn: 128, 192 or 256 fixes the column
+// tile (0: chosen by the cost model).
 ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count,
-                     int pair_min_tiles = 0);
+                     int pair_min_tiles = 0, int force_bn = 0);
 
 // ------------------------------------------------------- SIMT (fp32) ----
 

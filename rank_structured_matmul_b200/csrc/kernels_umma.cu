@@ -348,8 +348,9 @@ struct ProjPolicy {
 // shared memory (split-K, as in the projection).
 // kAls: the options the L update of further ALS iterations needs (an X view
 // shared by every instance, and T and G in fp32 as B x k x (d_in + k)); the
-// one-step layer's Gram stage is compiled without them.
-template <bool kAls>
+// one-step layer's Gram stage is compiled without them. kLo: T is also stored
+// as its bf16 rounding errors (Tlo, the split T of the compensated correction).
+template <bool kAls, bool kLo>
 struct GramPolicyT {
   struct Params {
     GemmCommon c;
@@ -363,7 +364,7 @@ struct GramPolicyT {
     // iterations, where "T" counts d_out rows
     int x_inst_fixed;
     __nv_bfloat16* Tb;  // (B*k) x d_in
-    __nv_bfloat16* Tlo;  // (B*k) x d_in: the bf16 rounding errors of Tb, or nullptr
+    __nv_bfloat16* Tlo;  // (B*k) x d_in: the bf16 rounding errors of Tb (kLo)
     float* G;           // B x k x k
     // when set, T and G go here instead, in fp32, as B x k x (d_in + k):
     // row i of instance b holds (L_b^T X_b)[i][0..d_in) then (L_b^T L_b)[i][0..k)
@@ -463,7 +464,7 @@ struct GramPolicyT {
             in_bounds(p.c.status, off + static_cast<size_t>(i0 + u) * p.d_in, 1, extent)) {
           const __nv_bfloat16 h = __float2bfloat16_rn(v[u]);
           dst[static_cast<size_t>(i0 + u) * p.d_in] = h;
-          if (p.Tlo != nullptr)
+          if (kLo)
             p.Tlo[off + static_cast<size_t>(i0 + u) * p.d_in] =
                 __float2bfloat16_rn(v[u] - __bfloat162float(h));
         }
@@ -545,8 +546,9 @@ struct GramPolicyT {
   }
   static __device__ __forceinline__ void epilogue_drain(const Params&, EpiCtx&) {}
 };
-using GramPolicy = GramPolicyT<false>;
-using GramAlsPolicy = GramPolicyT<true>;
+using GramPolicy = GramPolicyT<false, false>;
+using GramLoPolicy = GramPolicyT<false, true>;
+using GramAlsPolicy = GramPolicyT<true, false>;
 
 
 // ================================================================ rfactor ====
@@ -557,6 +559,7 @@ struct RFactorPolicy {
   // a register partition then holds two warps of each (2*152*32 + 2*104*32 =
   // 16384 registers), so the GEMM is held to 104.
   static constexpr int kMaxRegs = 104;
+  static constexpr bool kBParts = true;  // split T: hi and lo parts per stage
   struct Params {
     GemmCommon c;
     CUtensorMap tmW;  // (d_in, d_out), box (64, 128)
@@ -632,8 +635,7 @@ struct RFactorPolicy {
 // The bf16 result goes out through swizzled shared-memory boxes and TMA
 // stores; two boxes rotate, so one store drains while the next box is
 // written (more boxes would cost a pipeline stage).
-struct OutPolicy {
-  struct Params {
+struct OutParams {
     GemmCommon c;
     CUtensorMap tmZ;  // (r, N),        box (64, 128)
     CUtensorMap tmU;  // (r, d_out),    box (64, bn)
@@ -652,11 +654,18 @@ struct OutPolicy {
     // zeroes the tile's rows outside the block. nkz is then the K-steps of one
     // block. zb_w == 0: the dense Z U^T (K = r).
     int zb_w, zb_k, zb_n;
-  };
+};
+
+// kExt compiles in the options beyond the one-step layer: the compensated
+// correction (hilo), the block-diagonal static part (zb_w > 0) and the bias.
+// The plain layer runs OutPolicyT<false>, which ignores those fields.
+template <bool kExt>
+struct OutPolicyT {
+  using Params = OutParams;
   // The static part's blocks that the tile's columns n0 .. n0 + bn - 1 touch.
   static __device__ __forceinline__ void static_blocks(const Params& p, int n0, int& lo,
                                                        int& nseg) {
-    if (p.zb_w > 0) {
+    if (kExt && p.zb_w > 0) {
       lo = n0 / p.zb_w;
       nseg = min(p.zb_n - 1, (n0 + p.bn - 1) / p.zb_w) - lo + 1;
     } else {
@@ -665,17 +674,17 @@ struct OutPolicy {
     }
   }
   static __device__ __forceinline__ int static_iters(const Params& p, int z_nseg) {
-    return p.zb_w > 0 ? z_nseg * p.nkz : p.nkz;
+    return kExt && p.zb_w > 0 ? z_nseg * p.nkz : p.nkz;
   }
   static __device__ __forceinline__ int static_ksteps(const Params& p, int it) {
-    if (p.zb_w > 0) return min(4, ceil_div_dev(p.zb_k - (it % p.nkz) * 64, 16));
+    if (kExt && p.zb_w > 0) return min(4, ceil_div_dev(p.zb_k - (it % p.nkz) * 64, 16));
     return min(4, ceil_div_dev(p.r - it * 64, 16));
   }
   // K-step j of the correction: instance segment, sub-product (0 hi.hi,
   // 1 hi.lo, 2 lo.hi) and 64-wide chunk of k.
   static __device__ __forceinline__ void correction_step(const Params& p, int j, int& seg,
                                                          int& sub, int& ch) {
-    const int per = p.nkl * (p.hilo ? 3 : 1);
+    const int per = p.nkl * (kExt && p.hilo ? 3 : 1);
     seg = j / per;
     const int jj = j - seg * per;
     sub = jj / p.nkl;
@@ -692,7 +701,7 @@ struct OutPolicy {
     if (p.nkl > 0) {
       tma_prefetch_desc(&p.tmL);
       tma_prefetch_desc(&p.tmC);
-      if (p.hilo) {
+      if (kExt && p.hilo) {
         tma_prefetch_desc(&p.tmLlo);
         tma_prefetch_desc(&p.tmClo);
       }
@@ -714,7 +723,7 @@ struct OutPolicy {
     t.ns = static_iters(p, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return t.ns + t.nseg * p.nkl * (kExt && p.hilo ? 3 : 1);
   }
   // With Params::early (set only where the grid chain guarantees it: the
   // rank-k GEMM before the solve triggers its dependents only after its own
@@ -734,7 +743,7 @@ struct OutPolicy {
                                               uint32_t sb, uint32_t bar) {
     const int ns = t.ns;
     if (it < ns) {
-      if (p.zb_w > 0) {
+      if (kExt && p.zb_w > 0) {
         const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
         tma_load_2d(sa, &p.tmZ, bar, blk * p.zb_k + kk * 64, t.m0);
         tma_load_3d(sb, &p.tmU, bar, kk * 64, t.n0 - blk * p.zb_w, blk);
@@ -746,8 +755,8 @@ struct OutPolicy {
       int seg, sub, ch;
       correction_step(p, it - ns, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
-      tma_load_2d(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, t.n0);
+      tma_load_3d(sa, kExt && sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, t.m0 - b * p.T, b);
+      tma_load_2d(sb, kExt && sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, t.n0);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
@@ -763,7 +772,7 @@ struct OutPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    if (p.bias != nullptr) {
+    if (kExt && p.bias != nullptr) {
       for (int bx = 0; bx < p.bn / 64; ++bx)
         store_box_bf16<false, true>(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias,
                                     p.d_out);
@@ -863,6 +872,7 @@ struct XRwPolicy {
 struct RFactorPairPolicy {
   using Params = RFactorPolicy::Params;  // tmT box is (64, bn/2) here
   static constexpr int kMaxRegs = RFactorPolicy::kMaxRegs;
+  static constexpr bool kBParts = RFactorPolicy::kBParts;
   using Tile = RFactorPolicy::Tile;
   static constexpr uint32_t kEpiSmemBytes = RFactorPolicy::kEpiSmemBytes;
   static __device__ __forceinline__ void prefetch(const Params& p) { RFactorPolicy::prefetch(p); }
@@ -965,15 +975,17 @@ struct ProjPairPolicy {
 // =============================================================== out, pairs ====
 // The output stage on CTA pairs: tile 256 x bn, CTA r of the pair owns rows
 // m0 + 128 r .. +127 of A and of Y, and rows n0 + (bn/2) r .. + bn/2 - 1 of
-// the B operand ([U ; C_b]); the epilogue is OutPolicy's for its 128 rows.
-struct OutPairPolicy {
-  using Params = OutPolicy::Params;  // tmU / tmC boxes are (64, bn/2) here
+// the B operand ([U ; C_b]); the epilogue is OutPolicyT's for its 128 rows.
+template <bool kExt>
+struct OutPairPolicyT {
+  using Single = OutPolicyT<kExt>;
+  using Params = OutParams;  // tmU / tmC boxes are (64, bn/2) here
   struct Tile {
     int m0, n0, b_lo, nseg, z_lo, z_nseg, ns;
   };
-  static constexpr uint32_t kEpiSmemBytes = OutPolicy::kEpiSmemBytes;
+  static constexpr uint32_t kEpiSmemBytes = Single::kEpiSmemBytes;
 
-  static __device__ __forceinline__ void prefetch(const Params& p) { OutPolicy::prefetch(p); }
+  static __device__ __forceinline__ void prefetch(const Params& p) { Single::prefetch(p); }
   static __device__ __forceinline__ void decode(const Params& p, int tile, Tile& t) {
     t.m0 = (tile / p.n_tiles_n) * 256;
     t.n0 = (tile % p.n_tiles_n) * p.bn;
@@ -985,13 +997,13 @@ struct OutPairPolicy {
       t.b_lo = 0;
       t.nseg = 0;
     }
-    OutPolicy::static_blocks(p, t.n0, t.z_lo, t.z_nseg);
-    t.ns = OutPolicy::static_iters(p, t.z_nseg);
+    Single::static_blocks(p, t.n0, t.z_lo, t.z_nseg);
+    t.ns = Single::static_iters(p, t.z_nseg);
   }
   static __device__ __forceinline__ int kiters(const Params& p, const Tile& t) {
-    return t.ns + t.nseg * p.nkl * (p.hilo ? 3 : 1);
+    return t.ns + t.nseg * p.nkl * (kExt && p.hilo ? 3 : 1);
   }
-  static constexpr bool kEarly = true;  // as OutPolicy: static stages early
+  static constexpr bool kEarly = true;  // as OutPolicyT: static stages early
   static __device__ __forceinline__ void load_early(const Params& p, const Tile& t, int it,
                                                     uint32_t sa, uint32_t sb, uint32_t bar,
                                                     uint32_t rank) {
@@ -1008,7 +1020,7 @@ struct OutPairPolicy {
     const int nb = t.n0 + (p.bn / 2) * static_cast<int>(rank);
     const int ns = t.ns;
     if (it < ns) {
-      if (p.zb_w > 0) {
+      if (kExt && p.zb_w > 0) {
         const int seg = it / p.nkz, kk = it - seg * p.nkz, blk = t.z_lo + seg;
         tma_load_2d_pair(sa, &p.tmZ, bar, blk * p.zb_k + kk * 64, ma);
         tma_load_3d_pair(sb, &p.tmU, bar, kk * 64, nb - blk * p.zb_w, blk);
@@ -1018,14 +1030,14 @@ struct OutPairPolicy {
       }
     } else {
       int seg, sub, ch;
-      OutPolicy::correction_step(p, it - ns, seg, sub, ch);
+      Single::correction_step(p, it - ns, seg, sub, ch);
       const int b = t.b_lo + seg;
-      tma_load_3d_pair(sa, sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, ma - b * p.T, b);
-      tma_load_2d_pair(sb, sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, nb);
+      tma_load_3d_pair(sa, kExt && sub == 2 ? &p.tmLlo : &p.tmL, bar, ch * 64, ma - b * p.T, b);
+      tma_load_2d_pair(sb, kExt && sub == 1 ? &p.tmClo : &p.tmC, bar, b * p.k + ch * 64, nb);
     }
   }
   static __device__ __forceinline__ int ksteps(const Params& p, const Tile& t, int it) {
-    if (it < t.ns) return OutPolicy::static_ksteps(p, it);
+    if (it < t.ns) return Single::static_ksteps(p, it);
     const int ch = (it - t.ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
@@ -1037,7 +1049,7 @@ struct OutPairPolicy {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    OutPolicy::Tile h;
+    typename Single::Tile h;
     h.m0 = t.m0 + 128 * e.rank;
     h.n0 = t.n0;
     h.b_lo = t.b_lo;
@@ -1045,10 +1057,10 @@ struct OutPairPolicy {
     h.z_lo = t.z_lo;
     h.z_nseg = t.z_nseg;
     h.ns = t.ns;
-    OutPolicy::epilogue(p, h, tacc, e);
+    Single::epilogue(p, h, tacc, e);
   }
   static __device__ __forceinline__ void epilogue_drain(const Params& p, EpiCtx& e) {
-    OutPolicy::epilogue_drain(p, e);
+    Single::epilogue_drain(p, e);
   }
 };
 
@@ -1191,7 +1203,7 @@ int pick_bn(int n) {
 }  // namespace
 
 ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int sm_count,
-                     int pair_min_tiles) {
+                     int pair_min_tiles, int force_bn) {
   ProjShape ps;
   const int n_cols = r + k_eff;
   ps.tma_store = (r % 64 == 0 && k_eff <= 64) ? 1 : 0;
@@ -1202,6 +1214,7 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
   const int pair_min = pair_min_tiles > 0 ? pair_min_tiles : sm_count / 4;
   int64_t best = -1;
   for (int bn : {192, 256, 128}) {
+    if (force_bn > 0 && bn != force_bn) continue;
     const int nt = ceil_div(n_cols, bn);
     for (int pairs = 1; pairs >= 0; --pairs) {
       if (pairs && !use_pairs) continue;
@@ -1333,9 +1346,12 @@ int launch_gram_stage_as(const GramStage& g, int* status, const DeviceInfo& dev,
 
 int launch_gram_stage(const GramStage& g, int* status, const DeviceInfo& dev, cudaStream_t s,
                       bool pdl) {
-  return g.TGf != nullptr || g.x_inst_fixed
-             ? launch_gram_stage_as<GramAlsPolicy>(g, status, dev, s, pdl)
-             : launch_gram_stage_as<GramPolicy>(g, status, dev, s, pdl);
+  if (g.TGf != nullptr || g.x_inst_fixed) {
+    if (g.Tlo != nullptr) return -3;  // no split T in the fp32 layout
+    return launch_gram_stage_as<GramAlsPolicy>(g, status, dev, s, pdl);
+  }
+  return g.Tlo != nullptr ? launch_gram_stage_as<GramLoPolicy>(g, status, dev, s, pdl)
+                          : launch_gram_stage_as<GramPolicy>(g, status, dev, s, pdl);
 }
 
 // The Gram stage of the layer: L_b^T [X_b | L_b] per instance, L = a.L.
@@ -1458,12 +1474,37 @@ struct OutStatic {
 // early_static: the static operands are complete when this grid launches (it
 // follows the correction chain, or a grid that does not trigger early), so
 // they may be loaded before the dependency wait.
+template <bool kExt>
+int launch_out_as(OutParams& p, bool use_pairs, const Bf16Forward& a, const DeviceInfo& dev,
+                  cudaStream_t s, bool pdl, bool early_static) {
+  unsigned long long* tr = a.trace ? a.trace + 4 * kTraceCtas * kTraceSlots : nullptr;
+  if (use_pairs) {
+    using Pol = OutPairPolicyT<kExt>;
+    const int tiles = ceil_div(p.N, 256) * p.n_tiles_n;
+    const uint32_t smem = setup_common<Pol>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
+                                            false, a.status, dev);
+    if (!smem) return -3;
+    p.c.idesc = idesc_bf16(256, p.bn, false, false);
+    p.c.trace = tr;
+    p.c.early = pdl && early_static ? 1 : 0;
+    return launch_gemm_pair<Pol>(p, smem, dev, s, pdl) ? -1 : 0;
+  }
+  using Pol = OutPolicyT<kExt>;
+  const int tiles = ceil_div(p.N, 128) * p.n_tiles_n;
+  const uint32_t smem =
+      setup_common<Pol>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false, a.status, dev);
+  if (!smem) return -3;
+  p.c.trace = tr;
+  p.c.early = pdl && early_static ? 1 : 0;
+  return launch_gemm<Pol>(p, smem, dev, s, pdl) ? -1 : 0;
+}
+
 int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const void* Ct,
                      const void* Ctlo, bool hilo, int k, int d_out, void* Y, const void* bias,
                      const Bf16Forward& a, const DeviceInfo& dev, cudaStream_t s, bool pdl,
                      bool early_static = false) {
   const int64_t N = a.B * a.T;
-  OutPolicy::Params p;
+  OutParams p;
   p.N = static_cast<int>(N);
   p.r = st.zcols;
   p.k = k;
@@ -1528,24 +1569,10 @@ int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const 
   uint64_t sy[1] = {static_cast<uint64_t>(d_out) * 2};
   uint32_t by[2] = {64, 128};
   if (!encode_tmap_bf16(&p.tmY, Y, 2, dy, sy, by, 128)) return -2;
-  unsigned long long* tr = a.trace ? a.trace + 4 * kTraceCtas * kTraceSlots : nullptr;
-  if (use_pairs) {
-    const int tiles = ceil_div(N, 256) * p.n_tiles_n;
-    const uint32_t smem = setup_common<OutPairPolicy>(p.c, tiles, 128 * 128, (p.bn / 2) * 128,
-                                                      p.bn, false, false, a.status, dev);
-    if (!smem) return -3;
-    p.c.idesc = idesc_bf16(256, p.bn, false, false);
-    p.c.trace = tr;
-    p.c.early = pdl && early_static ? 1 : 0;
-    return launch_gemm_pair<OutPairPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
-  }
-  const int tiles = ceil_div(N, 128) * p.n_tiles_n;
-  const uint32_t smem = setup_common<OutPolicy>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false,
-                                                false, a.status, dev);
-  if (!smem) return -3;
-  p.c.trace = tr;
-  p.c.early = pdl && early_static ? 1 : 0;
-  return launch_gemm<OutPolicy>(p, smem, dev, s, pdl) ? -1 : 0;
+  // the plain one-step layer takes the kernel compiled without the options
+  const bool ext = p.hilo || p.zb_w > 0 || p.bias != nullptr;
+  return ext ? launch_out_as<true>(p, use_pairs, a, dev, s, pdl, early_static)
+             : launch_out_as<false>(p, use_pairs, a, dev, s, pdl, early_static);
 }
 
 // P2_b = X_b (RW_b)^T over P2 (N x k), RW: (B*k) x d_in (XRwPolicy).
@@ -1585,7 +1612,8 @@ int launch_proj_stage(const Bf16Forward& a, int k_eff, const float* MD, int* cou
   const int rk = a.r + a.k;  // VPt rows always hold [V | P]
   ProjPolicy::Params p;
   const ProjShape ps =
-      proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count, a.proj_pair_min_tiles);
+      proj_shape(N, a.d_in, a.r, k_eff, a.use_pairs, dev.sm_count, a.proj_pair_min_tiles,
+                 a.proj_bn);
   p.N = static_cast<int>(N);
   p.d_in = a.d_in;
   p.r = a.r;

@@ -165,6 +165,17 @@ struct HasEarly<Pol, std::void_t<decltype(Pol::kEarly)>> {
   static constexpr bool value = Pol::kEarly;
 };
 
+// Whether a policy may run with more than one B operand per stage
+// (Pol::kBParts; GemmCommon::b_parts is 1 for the others).
+template <class Pol, class = void>
+struct HasBParts {
+  static constexpr bool value = false;
+};
+template <class Pol>
+struct HasBParts<Pol, std::void_t<decltype(Pol::kBParts)>> {
+  static constexpr bool value = Pol::kBParts;
+};
+
 template <class Pol>
 __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::value)
     umma_gemm_kernel(const __grid_constant__ typename Pol::Params p) {
@@ -323,8 +334,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
           if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
           issue_stage<false>(d, a0, da, b0, db, idesc, ks, it == 0);
-          for (uint32_t part = 1; part < c.b_parts; ++part)
-            issue_stage<false>(d, a0, da, b0 + part * c.b_part_desc, db, idesc, ks, false);
+          if constexpr (HasBParts<Pol>::value)
+            for (uint32_t part = 1; part < c.b_parts; ++part)
+              issue_stage<false>(d, a0, da, b0 + part * c.b_part_desc, db, idesc, ks, false);
           mma_commit(empty_bar(stage));
           a += c.a_stage_bytes;
           b += c.b_stage_bytes;

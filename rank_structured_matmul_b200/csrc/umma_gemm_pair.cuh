@@ -190,8 +190,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (tr && local == 0 && it == 0) tr[kTrFirstData] = globaltimer_ns();
           tc_fence_after();
           issue_stage<true>(d, a0, da, b0, db, idesc, ks, it == 0);
-          for (uint32_t part = 1; part < c.b_parts; ++part)
-            issue_stage<true>(d, a0, da, b0 + part * c.b_part_desc, db, idesc, ks, false);
+          if constexpr (HasBParts<Pol>::value)
+            for (uint32_t part = 1; part < c.b_parts; ++part)
+              issue_stage<true>(d, a0, da, b0 + part * c.b_part_desc, db, idesc, ks, false);
           mma_commit_pair(empty_bar(stage));
           a += c.a_stage_bytes;
           b += c.b_stage_bytes;
