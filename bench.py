@@ -45,10 +45,10 @@ UNIT = "TFLOP/s (dense-equivalent)"
 HEADLINE = "llama_up_8192"
 BLOCK = ("vit_block_qkv", "vit_block_proj", "vit_block_fc1", "vit_block_fc2")
 STAGE_KERNELS = {"proj": "ProjPolicy (CTA pairs, or split-K clusters at skinny N)",
-                 "gram": "umma_gemm_kernel<GramPolicy>",
+                 "gram": "umma_gemm_kernel<GramPolicyT<false, false>>",
                  "solve": "ltilde_kernel (L~ = L G^-1, beside the rank-k factor GEMM)",
                  "rfactor": "RFactorPolicy (Q = T W_res^T; CTA pairs when there are enough tiles)",
-                 "out": "umma_gemm_pair_kernel<OutPairPolicy>"}
+                 "out": "umma_gemm_pair_kernel<OutPairPolicyT<false>>"}
 FLUSH_BYTES = 256 << 20
 L2_NOTE = "GPU arm: 256 MiB written before every step, outside the step events"
 DATA = ("synthetic (seeded; shapes and statistics of the workload, random-orthogonal weights "
@@ -182,13 +182,14 @@ def parity_rows(s, max_rows: int = 1024):
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every millisecond while the
-    timed region runs (read-only NVML queries; nvidia-smi as a fallback)."""
+    """SM clock and clock-event reasons sampled back to back while the timed
+    region runs (two read-only NVML queries per sample, the maximum clock read
+    once; nvidia-smi as a fallback)."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4}
 
-    def __init__(self, cuda_index: int, period_s: float = 0.001):
+    def __init__(self, cuda_index: int, period_s: float = 0.0):
         self.cuda_index = cuda_index
         self.period = period_s
         self.rows = []
@@ -196,6 +197,7 @@ class ClockSampler:
         self.stop_flag = False
         self.handle = None
         self.nvml = None
+        self.max_mhz = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -222,7 +224,9 @@ class ClockSampler:
     def _sample(self):
         n, h = self.nvml, self.handle
         sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
-        mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+        if self.max_mhz is None:
+            self.max_mhz = float(n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM))
+        mx = self.max_mhz
         try:
             bits = n.nvmlDeviceGetCurrentClocksEventReasons(h)
         except Exception:
@@ -235,7 +239,8 @@ class ClockSampler:
                 self._sample()
             except Exception:
                 return
-            time.sleep(self.period)
+            if self.period > 0:
+                time.sleep(self.period)
 
     def start(self):
         if self.handle is None:
@@ -260,7 +265,9 @@ class ClockSampler:
                          if any(r[2] & bit for r in rows))
         return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": rows[0][1],
                 "sm_mhz_min": float(min(r[0] for r in rows)), "reasons": reasons,
-                "samples": len(rows), "source": "nvml, every %g ms" % (self.period * 1e3)}
+                "samples": len(rows),
+                "source": "nvml, every %g ms" % (self.period * 1e3) if self.period > 0
+                else "nvml, back to back"}
 
     def _smi_once(self):
         fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
@@ -369,6 +376,12 @@ class Timer:
         return float(np.mean([a.elapsed_time(b) for a, b in ev]))
 
 
+def dense_time(timer, fn, steps):
+    """cuBLAS dense time of a step: the lower mean of two timed loops (the
+    baseline's occasional slow loop would otherwise flatter the comparison)."""
+    return min(timer(fn, steps, 3), timer(fn, steps, 0))
+
+
 def stage_times(runs, timer, n_steps):
     """Mean per-stage device time of each layer (events between the stage
     launches, a separate loop with stage timing switched on), in ms."""
@@ -457,7 +470,7 @@ def per_config(names, dev, pk, steps, warmup, headline_entry=None):
         seq = lambda: [r.step() for r in runs]
         dense = lambda: [r.dense_step() for r in runs]
         t = timer(seq, steps, warmup)
-        td = timer(dense, steps, 3)
+        td = dense_time(timer, dense, steps)
         flops = sum(2.0 * r.s.N * r.s.d_in * r.s.d_out for r in runs)
         roof_us = sum(layer_roofline_us(r.s, pk) for r in runs)
         e = {"us": t * 1e3, "cublas_dense_us": td * 1e3, "speedup_vs_cublas_dense": td / t,
@@ -474,7 +487,7 @@ def per_config(names, dev, pk, steps, warmup, headline_entry=None):
             e["layers"] = {}
             for r in runs:
                 tl = timer(r.step, steps, 3)
-                tdl = timer(r.dense_step, steps, 3)
+                tdl = dense_time(timer, r.dense_step, steps)
                 e["layers"][r.s.name] = {"us": tl * 1e3, "cublas_dense_us": tdl * 1e3}
         else:
             e["static_matched"] = static_entry(runs[0], timer, steps)
@@ -653,7 +666,7 @@ def run_dyra(args):
         return
 
     # ---- cuBLAS dense X W^T of the same shapes, timed the same way
-    dense_ms = max_over_ranks(timer(lambda: [r.dense_step() for r in runs], args.steps, 3),
+    dense_ms = max_over_ranks(dense_time(timer, lambda: [r.dense_step() for r in runs], args.steps),
                               world, dev)
     for r in runs:
         r.free_dense()
