@@ -48,7 +48,7 @@ STAGE_KERNELS = {"proj": "ProjPolicy (CTA pairs, or split-K clusters at skinny N
                  "gram": "umma_gemm_kernel<GramPolicyT<false, false>>",
                  "solve": "ltilde_kernel (L~ = L G^-1, beside the rank-k factor GEMM)",
                  "rfactor": "RFactorPolicy (Q = T W_res^T; CTA pairs when there are enough tiles)",
-                 "out": "umma_gemm_pair_kernel<OutPairPolicyT<false>>"}
+                 "out": "umma_gemm_pair_kernel<OutPairPolicyT<false, false>>"}
 FLUSH_BYTES = 256 << 20
 L2_NOTE = "GPU arm: 256 MiB written before every step, outside the step events"
 DATA = ("synthetic (seeded; shapes and statistics of the workload, random-orthogonal weights "
@@ -182,14 +182,14 @@ def parity_rows(s, max_rows: int = 1024):
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled back to back while the timed
+    """SM clock and clock-event reasons sampled every 0.2 ms while the timed
     region runs (two read-only NVML queries per sample, the maximum clock read
     once; nvidia-smi as a fallback)."""
 
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4}
 
-    def __init__(self, cuda_index: int, period_s: float = 0.0):
+    def __init__(self, cuda_index: int, period_s: float = 0.0002):
         self.cuda_index = cuda_index
         self.period = period_s
         self.rows = []
@@ -563,7 +563,7 @@ def extras(dev, steps, warmup):
     us = timer(mstep, steps, warmup) * 1e3
     Wd = torch.from_numpy(w.weight()).to(dev, td)
     Yd = torch.empty_like(Y)
-    dense_us = timer(lambda: torch.matmul(X, Wd.t(), out=Yd), steps, 3) * 1e3
+    dense_us = dense_time(timer, lambda: torch.matmul(X, Wd.t(), out=Yd), steps) * 1e3
     rd = lambda a: oracle.round_to(np.asarray(a), "bf16")
     Lb, Rb = rd(f.Lblocks.numpy()), rd(f.Rblocks.numpy())
     fr = mon.MonarchFactors(list(Lb), list(Rb), mon.monarch_matrix(list(Lb), list(Rb)).T,

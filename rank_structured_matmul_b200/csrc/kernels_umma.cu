@@ -72,6 +72,17 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
                                                int ncols = 0) {
   const uint32_t buf = e.counter % kStoreBoxes;
   ++e.counter;
+  // the box's 64 bias values (8 columns per load, all inside or all beyond
+  // ncols) are loaded first, so that their latency passes during the TMEM
+  // loads and the wait for the store buffer
+  uint4 bq[BIAS ? 8 : 1];
+  if constexpr (BIAS) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = x + j * 8;
+      bq[j] = c < ncols ? __ldg(reinterpret_cast<const uint4*>(bias + c)) : make_uint4(0, 0, 0, 0);
+    }
+  }
   // both TMEM loads in flight before one wait, and during the wait for the
   // store buffer
   uint32_t vv[2][32];
@@ -86,10 +97,8 @@ __device__ __forceinline__ void store_box_bf16(uint32_t tacc, int col0, const vo
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        const int c = x + half * 32 + ch * 8;  // 8 columns, all inside or all beyond ncols
-        const uint4 bq = c < ncols ? __ldg(reinterpret_cast<const uint4*>(bias + c))
-                                   : make_uint4(0, 0, 0, 0);
-        const uint32_t w[4] = {bq.x, bq.y, bq.z, bq.w};
+        const uint4& b8 = bq[half * 4 + ch];
+        const uint32_t w[4] = {b8.x, b8.y, b8.z, b8.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t& v0 = vv[half][8 * ch + 2 * j];
@@ -656,10 +665,10 @@ struct OutParams {
     int zb_w, zb_k, zb_n;
 };
 
-// kExt compiles in the options beyond the one-step layer: the compensated
-// correction (hilo), the block-diagonal static part (zb_w > 0) and the bias.
-// The plain layer runs OutPolicyT<false>, which ignores those fields.
-template <bool kExt>
+// kExt compiles in the compensated correction (hilo) and the block-diagonal
+// static part (zb_w > 0), kBias the bias. The plain layer runs
+// OutPolicyT<false, false>, which ignores those fields.
+template <bool kExt, bool kBias>
 struct OutPolicyT {
   using Params = OutParams;
   // The static part's blocks that the tile's columns n0 .. n0 + bn - 1 touch.
@@ -772,7 +781,7 @@ struct OutPolicyT {
   }
   static __device__ __forceinline__ void epilogue(const Params& p, const Tile& t, uint32_t tacc,
                                                   EpiCtx& e) {
-    if (kExt && p.bias != nullptr) {
+    if (kBias && p.bias != nullptr) {
       for (int bx = 0; bx < p.bn / 64; ++bx)
         store_box_bf16<false, true>(tacc, bx * 64, &p.tmY, t.n0 + bx * 64, t.m0, e, p.bias,
                                     p.d_out);
@@ -976,9 +985,9 @@ struct ProjPairPolicy {
 // The output stage on CTA pairs: tile 256 x bn, CTA r of the pair owns rows
 // m0 + 128 r .. +127 of A and of Y, and rows n0 + (bn/2) r .. + bn/2 - 1 of
 // the B operand ([U ; C_b]); the epilogue is OutPolicyT's for its 128 rows.
-template <bool kExt>
+template <bool kExt, bool kBias>
 struct OutPairPolicyT {
-  using Single = OutPolicyT<kExt>;
+  using Single = OutPolicyT<kExt, kBias>;
   using Params = OutParams;  // tmU / tmC boxes are (64, bn/2) here
   struct Tile {
     int m0, n0, b_lo, nseg, z_lo, z_nseg, ns;
@@ -1474,12 +1483,12 @@ struct OutStatic {
 // early_static: the static operands are complete when this grid launches (it
 // follows the correction chain, or a grid that does not trigger early), so
 // they may be loaded before the dependency wait.
-template <bool kExt>
+template <bool kExt, bool kBias>
 int launch_out_as(OutParams& p, bool use_pairs, const Bf16Forward& a, const DeviceInfo& dev,
                   cudaStream_t s, bool pdl, bool early_static) {
   unsigned long long* tr = a.trace ? a.trace + 4 * kTraceCtas * kTraceSlots : nullptr;
   if (use_pairs) {
-    using Pol = OutPairPolicyT<kExt>;
+    using Pol = OutPairPolicyT<kExt, kBias>;
     const int tiles = ceil_div(p.N, 256) * p.n_tiles_n;
     const uint32_t smem = setup_common<Pol>(p.c, tiles, 128 * 128, (p.bn / 2) * 128, p.bn, false,
                                             false, a.status, dev);
@@ -1489,7 +1498,7 @@ int launch_out_as(OutParams& p, bool use_pairs, const Bf16Forward& a, const Devi
     p.c.early = pdl && early_static ? 1 : 0;
     return launch_gemm_pair<Pol>(p, smem, dev, s, pdl) ? -1 : 0;
   }
-  using Pol = OutPolicyT<kExt>;
+  using Pol = OutPolicyT<kExt, kBias>;
   const int tiles = ceil_div(p.N, 128) * p.n_tiles_n;
   const uint32_t smem =
       setup_common<Pol>(p.c, tiles, 128 * 128, p.bn * 128, p.bn, false, false, a.status, dev);
@@ -1569,10 +1578,13 @@ int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const 
   uint64_t sy[1] = {static_cast<uint64_t>(d_out) * 2};
   uint32_t by[2] = {64, 128};
   if (!encode_tmap_bf16(&p.tmY, Y, 2, dy, sy, by, 128)) return -2;
-  // the plain one-step layer takes the kernel compiled without the options
-  const bool ext = p.hilo || p.zb_w > 0 || p.bias != nullptr;
-  return ext ? launch_out_as<true>(p, use_pairs, a, dev, s, pdl, early_static)
-             : launch_out_as<false>(p, use_pairs, a, dev, s, pdl, early_static);
+  // each layer takes the kernel compiled with only the options it uses
+  const bool ext = p.hilo || p.zb_w > 0;
+  if (p.bias != nullptr)
+    return ext ? launch_out_as<true, true>(p, use_pairs, a, dev, s, pdl, early_static)
+               : launch_out_as<false, true>(p, use_pairs, a, dev, s, pdl, early_static);
+  return ext ? launch_out_as<true, false>(p, use_pairs, a, dev, s, pdl, early_static)
+             : launch_out_as<false, false>(p, use_pairs, a, dev, s, pdl, early_static);
 }
 
 // P2_b = X_b (RW_b)^T over P2 (N x k), RW: (B*k) x d_in (XRwPolicy).
