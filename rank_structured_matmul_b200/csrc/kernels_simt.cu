@@ -794,9 +794,11 @@ __global__ void __launch_bounds__(kSolveThreads)
 
 // C[b][m][n] (+)= alpha sum_q A[b][m][q] * Bm[b][q][n] (+ bias[n]) with
 // arbitrary element strides.
+// kGK: the k step. Long K takes 64 (64 x 64 elements of each operand in
+// flight per step, a quarter of the dependent load round trips of 16); short
+// K takes 16, which wastes less work on the zero-filled tail.
 constexpr int kGT = 64;   // tile
-constexpr int kGK = 16;   // k step
-template <typename TA, typename TB, typename TC>
+template <typename TA, typename TB, typename TC, int kGK>
 __global__ void __launch_bounds__(256)
     simt_gemm_kernel(int M, int N, int K, const TA* __restrict__ A, int64_t am, int64_t ak,
                      int64_t ab, const TB* __restrict__ Bm, int64_t bk, int64_t bn, int64_t bb,
@@ -810,14 +812,30 @@ __global__ void __launch_bounds__(256)
   A += batch * ab;
   Bm += batch * bb;
   C += batch * cb;
+  // consecutive threads walk the operand's unit-stride dimension (coalesced)
+  const bool a_k_fast = ak == 1, b_k_fast = bk == 1 && bn != 1;
   float acc[4][4] = {};
+  constexpr int kPer = kGK * kGT / 256;  // elements of each operand per thread and step
   for (int q0 = 0; q0 < K; q0 += kGK) {
-    for (int idx = threadIdx.x; idx < kGK * kGT; idx += 256) {
-      const int qq = idx / kGT, mm = idx % kGT;
-      const int gm = m0 + mm, gq = q0 + qq;
-      As[qq][mm] = (gm < M && gq < K) ? to_f<TA>(A[gm * am + gq * ak]) : 0.f;
-      const int gn = n0 + mm;
-      Bs[qq][mm] = (gn < N && gq < K) ? to_f<TB>(Bm[gq * bk + gn * bn]) : 0.f;
+    // every load of the step in flight before the first store to shared memory
+    float va[kPer], vb[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int idx = threadIdx.x + 256 * j;
+      const int qa = a_k_fast ? idx % kGK : idx / kGT, ma = a_k_fast ? idx / kGK : idx % kGT;
+      const int gm = m0 + ma, gqa = q0 + qa;
+      va[j] = (gm < M && gqa < K) ? to_f<TA>(A[gm * am + gqa * ak]) : 0.f;
+      const int qb = b_k_fast ? idx % kGK : idx / kGT, nb = b_k_fast ? idx / kGK : idx % kGT;
+      const int gn = n0 + nb, gqb = q0 + qb;
+      vb[j] = (gn < N && gqb < K) ? to_f<TB>(Bm[gqb * bk + gn * bn]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int idx = threadIdx.x + 256 * j;
+      const int qa = a_k_fast ? idx % kGK : idx / kGT, ma = a_k_fast ? idx / kGK : idx % kGT;
+      const int qb = b_k_fast ? idx % kGK : idx / kGT, nb = b_k_fast ? idx / kGK : idx % kGT;
+      As[qa][ma] = va[j];
+      Bs[qb][nb] = vb[j];
     }
     __syncthreads();
 #pragma unroll
@@ -858,8 +876,14 @@ int gemm(int M, int N, int K, const TA* A, int64_t am, int64_t ak, int64_t ab, c
          const TC* bias = nullptr, int64_t bias_b = 0) {
   if (M <= 0 || N <= 0 || batches <= 0) return 0;
   dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, batches);
-  simt_gemm_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb, C,
-                                                    cm, cn, cb, accumulate, alpha, bias, bias_b);
+  if (K >= 128)
+    simt_gemm_kernel<TA, TB, TC, 64><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb,
+                                                          C, cm, cn, cb, accumulate, alpha, bias,
+                                                          bias_b);
+  else
+    simt_gemm_kernel<TA, TB, TC, 16><<<grid, 256, 0, s>>>(M, N, K, A, am, ak, ab, Bm, bk, bn, bb,
+                                                          C, cm, cn, cb, accumulate, alpha, bias,
+                                                          bias_b);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

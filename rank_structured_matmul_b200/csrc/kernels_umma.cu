@@ -247,7 +247,7 @@ struct ProjPolicy {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int col = t.n0 + cc + 8 * g;
-          if (col < rk) {
+          if (col < rk && cc + 8 * g < p.bn) {  // the last 32 columns may pass the tile
             const bool z = col < p.r;
             const size_t at = z ? static_cast<size_t>(grow) * p.r + col
                                 : static_cast<size_t>(grow) * p.k + (col - p.r);
@@ -663,6 +663,10 @@ struct OutParams {
     // zeroes the tile's rows outside the block. nkz is then the K-steps of one
     // block. zb_w == 0: the dense Z U^T (K = r).
     int zb_w, zb_k, zb_n;
+    // 1 (k <= 32): the correction's boxes are 32 columns wide (64-byte
+    // swizzle), half the bytes of a 64-wide box, of which k <= 32 columns
+    // would be used; its stages then hold 64-byte rows
+    int narrow;
 };
 
 // kExt compiles in the compensated correction (hilo) and the block-diagonal
@@ -772,6 +776,25 @@ struct OutPolicyT {
     if (it < t.ns) return static_ksteps(p, it);
     const int ch = (it - t.ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
+  }
+  // narrow correction stages: half the bytes, K-major rows of 64 bytes
+  // (8-row atoms 512 bytes apart); the k-th group of 16 columns is 32 bytes
+  // further into each row, as in the 128-byte layout
+  static constexpr bool kStageLayouts = true;
+  static __device__ __forceinline__ bool narrow_stage(const Params& p, const Tile& t, int it) {
+    return p.narrow && it >= t.ns;
+  }
+  static __device__ __forceinline__ uint32_t stage_tx(const Params& p, const Tile& t, int it) {
+    const uint32_t full = p.c.a_stage_bytes + p.c.b_stage_bytes;
+    return narrow_stage(p, t, it) ? full / 2 : full;
+  }
+  static __device__ __forceinline__ uint64_t stage_adesc(const Params& p, const Tile& t, int it,
+                                                         uint32_t a) {
+    return narrow_stage(p, t, it) ? smem_desc(a, 16u, 512u, kLayoutSw64) : kmajor_desc(a, 0);
+  }
+  static __device__ __forceinline__ uint64_t stage_bdesc(const Params& p, const Tile& t, int it,
+                                                         uint32_t b) {
+    return narrow_stage(p, t, it) ? smem_desc(b, 16u, 512u, kLayoutSw64) : kmajor_desc(b, 0);
   }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
     return kmajor_desc(a, ks);
@@ -1050,6 +1073,19 @@ struct OutPairPolicyT {
     const int ch = (it - t.ns) % p.nkl;
     return min(4, ceil_div_dev(p.k - ch * 64, 16));
   }
+  static constexpr bool kStageLayouts = true;  // as Single: narrow correction stages
+  static __device__ __forceinline__ uint32_t stage_tx(const Params& p, const Tile& t, int it) {
+    const uint32_t full = p.c.a_stage_bytes + p.c.b_stage_bytes;
+    return p.narrow && it >= t.ns ? full / 2 : full;
+  }
+  static __device__ __forceinline__ uint64_t stage_adesc(const Params& p, const Tile& t, int it,
+                                                         uint32_t a) {
+    return p.narrow && it >= t.ns ? smem_desc(a, 16u, 512u, kLayoutSw64) : kmajor_desc(a, 0);
+  }
+  static __device__ __forceinline__ uint64_t stage_bdesc(const Params& p, const Tile& t, int it,
+                                                         uint32_t b) {
+    return p.narrow && it >= t.ns ? smem_desc(b, 16u, 512u, kLayoutSw64) : kmajor_desc(b, 0);
+  }
   static __device__ __forceinline__ uint64_t adesc(const Params&, uint32_t a, int ks) {
     return kmajor_desc(a, ks);
   }
@@ -1219,11 +1255,17 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
   // Column tile and CTA pairs: the stage is bound by the bytes each CTA
   // streams per k-step (128 rows of X, plus bn / 2 rows of [V | P]^T on a
   // pair or bn rows alone) times the rounds of tiles per SM. Pick the
-  // cheapest of bn = 128, 192, 256 (whole 64-column store boxes).
+  // cheapest of bn = 128, 192, 256 (whole 64-column store boxes) and the
+  // width that splits the columns evenly over the fewest tiles (a multiple
+  // of 16; e.g. 2 x 144 for 288 columns instead of 2 x 192), whose stores
+  // then go out as 16-byte row pieces.
   const int pair_min = pair_min_tiles > 0 ? pair_min_tiles : sm_count / 4;
+  const int exact =
+      std::min(256, ceil_div(ceil_div(n_cols, std::max(1, ceil_div(n_cols, 256))), 16) * 16);
   int64_t best = -1;
-  for (int bn : {192, 256, 128}) {
+  for (int bn : {192, 256, 128, exact}) {
     if (force_bn > 0 && bn != force_bn) continue;
+    if (bn == exact && force_bn != exact && (exact % 64 == 0 || exact < 16)) continue;
     const int nt = ceil_div(n_cols, bn);
     for (int pairs = 1; pairs >= 0; --pairs) {
       if (pairs && !use_pairs) continue;
@@ -1240,6 +1282,7 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
       }
     }
   }
+  if (ps.bn % 64 != 0) ps.tma_store = 0;
   ps.ksplit = 1;
   const int kit = ceil_div(d_in, 64);
   ps.kper = kit;
@@ -1247,10 +1290,11 @@ ProjShape proj_shape(int64_t N, int d_in, int r, int k_eff, bool use_pairs, int 
     // Split-K: narrower column tiles first (more tiles, and half the fp32
     // partial each CTA sums over the cluster), then up to 8 splits per tile
     // (portable cluster size).
-    if (ps.bn > 128) {
+    if (ps.bn > 128 || ps.bn % 32 != 0) {  // whole 32-column TMEM loads into the partial
       ps.bn = 128;
       ps.n_tiles_n = ceil_div(n_cols, ps.bn);
       ps.tiles = static_cast<int>(ceil_div(N, 128)) * ps.n_tiles_n;
+      ps.tma_store = (r % 64 == 0 && k_eff <= 64) ? 1 : 0;
     }
     const int want = std::min(sm_count / ps.tiles, std::min(kit / 4, 8));
     if (want > 1) {
@@ -1548,21 +1592,24 @@ int launch_out_stage(const OutStatic& st, const void* L, const void* Llo, const 
     uint32_t bu[2] = {64, bbox};
     if (!encode_tmap_bf16(&p.tmU, st.U, 2, du, sz, bu, 128)) return -2;
   }
+  p.narrow = k > 0 && k <= 32 ? 1 : 0;
   if (k > 0) {
     uint64_t dl[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(a.T),
                       static_cast<uint64_t>(a.B)};
     uint64_t sl[2] = {static_cast<uint64_t>(k) * 2,
                       static_cast<uint64_t>(k) * 2 * static_cast<uint64_t>(a.T)};
-    uint32_t bl[3] = {64, 128, 1};
-    if (!encode_tmap_bf16(&p.tmL, L, 3, dl, sl, bl, 128)) return -2;
+    const uint32_t kw = p.narrow ? 32u : 64u;  // box columns of the correction
+    const int sw = p.narrow ? 64 : 128;
+    uint32_t bl[3] = {kw, 128, 1};
+    if (!encode_tmap_bf16(&p.tmL, L, 3, dl, sl, bl, sw)) return -2;
     const int64_t Bk = a.B * k;
     uint64_t dc[2] = {static_cast<uint64_t>(Bk), static_cast<uint64_t>(d_out)};
     uint64_t sc[1] = {static_cast<uint64_t>(Bk) * 2};
-    uint32_t bc[2] = {64, bbox};
-    if (!encode_tmap_bf16(&p.tmC, Ct, 2, dc, sc, bc, 128)) return -2;
+    uint32_t bc[2] = {kw, bbox};
+    if (!encode_tmap_bf16(&p.tmC, Ct, 2, dc, sc, bc, sw)) return -2;
     if (hilo) {
-      if (!encode_tmap_bf16(&p.tmLlo, Llo, 3, dl, sl, bl, 128)) return -2;
-      if (!encode_tmap_bf16(&p.tmClo, Ctlo, 2, dc, sc, bc, 128)) return -2;
+      if (!encode_tmap_bf16(&p.tmLlo, Llo, 3, dl, sl, bl, sw)) return -2;
+      if (!encode_tmap_bf16(&p.tmClo, Ctlo, 2, dc, sc, bc, sw)) return -2;
     } else {
       p.tmLlo = p.tmL;
       p.tmClo = p.tmC;

@@ -176,6 +176,42 @@ struct HasBParts<Pol, std::void_t<decltype(Pol::kBParts)>> {
   static constexpr bool value = Pol::kBParts;
 };
 
+// Stages of different layouts (Pol::kStageLayouts): the policy gives each
+// stage's byte count and its first shared memory descriptors; otherwise every
+// stage holds a_stage_bytes + b_stage_bytes in the policy's one layout.
+template <class Pol, class = void>
+struct HasStageLayouts {
+  static constexpr bool value = false;
+};
+template <class Pol>
+struct HasStageLayouts<Pol, std::void_t<decltype(Pol::kStageLayouts)>> {
+  static constexpr bool value = Pol::kStageLayouts;
+};
+template <class Pol>
+__device__ __forceinline__ uint32_t stage_tx(const typename Pol::Params& p,
+                                             const typename Pol::Tile& t, int it) {
+  if constexpr (HasStageLayouts<Pol>::value)
+    return Pol::stage_tx(p, t, it);
+  else
+    return p.c.a_stage_bytes + p.c.b_stage_bytes;
+}
+template <class Pol>
+__device__ __forceinline__ uint64_t stage_adesc(const typename Pol::Params& p,
+                                                const typename Pol::Tile& t, int it, uint32_t a) {
+  if constexpr (HasStageLayouts<Pol>::value)
+    return Pol::stage_adesc(p, t, it, a);
+  else
+    return Pol::adesc(p, a, 0);
+}
+template <class Pol>
+__device__ __forceinline__ uint64_t stage_bdesc(const typename Pol::Params& p,
+                                                const typename Pol::Tile& t, int it, uint32_t b) {
+  if constexpr (HasStageLayouts<Pol>::value)
+    return Pol::stage_bdesc(p, t, it, b);
+  else
+    return Pol::bdesc(p, b, 0);
+}
+
 template <class Pol>
 __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::value)
     umma_gemm_kernel(const __grid_constant__ typename Pol::Params p) {
@@ -262,7 +298,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
             pre = min(S, Pol::kiters(p, t0));
           }
           for (int it = 0; it < pre; ++it) {  // fresh slots: nothing to wait for
-            mbar_arrive_expect_tx(full_bar(it), c.a_stage_bytes + c.b_stage_bytes);
+            mbar_arrive_expect_tx(full_bar(it), stage_tx<Pol>(p, t0, it));
             Pol::load_early(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
                             full_bar(it));
           }
@@ -287,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), c.a_stage_bytes + c.b_stage_bytes);
+          mbar_arrive_expect_tx(full_bar(stage), stage_tx<Pol>(p, t, it));
           Pol::load(p, t, it, sA + stage * c.a_stage_bytes, sB + stage * c.b_stage_bytes,
                     full_bar(stage));
           if (tr) {
@@ -326,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) __maxnreg__(MaxRegs<Pol>::val
         for (int it = 0; it < nk; ++it) {
           // what the stage's MMAs need besides its data, before the wait
           const int ks = Pol::ksteps(p, t, it);
-          const uint64_t a0 = Pol::adesc(p, a, 0), b0 = Pol::bdesc(p, b, 0);
+          const uint64_t a0 = stage_adesc<Pol>(p, t, it, a), b0 = stage_bdesc<Pol>(p, t, it, b);
           if (!mbar_wait(full_bar(stage), phase, w)) {
             ok = false;
             break;

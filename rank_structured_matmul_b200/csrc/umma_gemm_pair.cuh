@@ -117,7 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           for (int it = 0; it < pre; ++it) {  // fresh slots: nothing to wait for
             if (leader)
-              mbar_arrive_expect_tx(full_bar(it), 2u * (c.a_stage_bytes + c.b_stage_bytes));
+              mbar_arrive_expect_tx(full_bar(it), 2u * stage_tx<Pol>(p, t0, it));
             Pol::load_early(p, t0, it, sA + it * c.a_stage_bytes, sB + it * c.b_stage_bytes,
                             full_bar(it), rank);
           }
@@ -143,7 +143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           if (leader)
-            mbar_arrive_expect_tx(full_bar(stage), 2u * (c.a_stage_bytes + c.b_stage_bytes));
+            mbar_arrive_expect_tx(full_bar(stage), 2u * stage_tx<Pol>(p, t, it));
           Pol::load(p, t, it, sA + stage * c.a_stage_bytes, sB + stage * c.b_stage_bytes,
                     full_bar(stage), rank);
           if (tr) {
@@ -182,7 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int it = 0; it < nk; ++it) {
           // what the stage's MMAs need besides its data, before the wait
           const int ks = Pol::ksteps(p, t, it);
-          const uint64_t a0 = Pol::adesc(p, a, 0), b0 = Pol::bdesc(p, b, 0);
+          const uint64_t a0 = stage_adesc<Pol>(p, t, it, a), b0 = stage_bdesc<Pol>(p, t, it, b);
           if (!mbar_wait(full_bar(stage), phase, w)) {
             ok = false;
             break;
