@@ -42,6 +42,30 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int ks) {
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
 
+// Split-K reductions over distributed shared memory: float4 items off[u] of
+// the partials of cluster ranks ks .. ks + NJ - 1, all loads in flight at once.
+template <int NJ>
+__device__ __forceinline__ void load_partials(float4 (&v)[4][4], uint32_t stage_u32, int ks,
+                                              const uint32_t (&off)[4]) {
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const uint32_t base = mapa_shared(stage_u32, static_cast<uint32_t>(ks + j));
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[j][u] = ld_shared_cluster_v4(base + 16u * off[u]);
+  }
+}
+// Loads the min(4, S - ks) partials from rank ks on (each partial read once:
+// the reads are bound by the bandwidth of distributed shared memory).
+__device__ __forceinline__ void load_partials_from(float4 (&v)[4][4], uint32_t stage_u32, int ks,
+                                                   int S, const uint32_t (&off)[4]) {
+  switch (min(4, S - ks)) {
+    case 4: load_partials<4>(v, stage_u32, ks, off); break;
+    case 3: load_partials<3>(v, stage_u32, ks, off); break;
+    case 2: load_partials<2>(v, stage_u32, ks, off); break;
+    default: load_partials<1>(v, stage_u32, ks, off); break;
+  }
+}
+
 // Write eight fp32 accumulator values as one 16-byte bf16 vector.
 __device__ __forceinline__ void store8_bf16(void* dst, const uint32_t (&v)[32], int g) {
   st_global_v4(dst, pack_bf16x2(f32(v[8 * g + 0]), f32(v[8 * g + 1])),
@@ -305,12 +329,7 @@ struct ProjPolicy {
       for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int ks = 0; ks < p.ksplit; ks += 4) {
         float4 v[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t base = mapa_shared(stage_u32, static_cast<uint32_t>(min(ks + j, p.ksplit - 1)));
-#pragma unroll
-          for (int u = 0; u < 4; ++u) v[j][u] = ld_shared_cluster_v4(base + 16u * off[u]);
-        }
+        load_partials_from(v, stage_u32, ks, p.ksplit, off);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (ks + j < p.ksplit)
@@ -529,27 +548,44 @@ struct GramPolicyT {
     const int rs = (128 + p.S - 1) / p.S;
     const int row0 = ks_me * rs, nrows = min(128, row0 + rs) - row0;
     const int nitems = nrows > 0 ? nrows * c4n : 0;
-    for (int it = tid; it < nitems; it += 128) {
-      const int c4 = it / nrows, row = row0 + (it - c4 * nrows);
-      const uint32_t off = 16u * static_cast<uint32_t>(c4 * 128 + row);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int ks = 0; ks < p.S; ks += 4) {
-        float4 v[4];
+    // four items per thread and pass, the loads of all four from up to four
+    // partials in flight together (one round trip of distributed shared
+    // memory per pass instead of one per item), summed in split order
+    for (int i0 = tid; i0 < nitems; i0 += 4 * 128) {
+      uint32_t off[4];
+      bool valid[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          v[j] = ld_shared_cluster_v4(
-              mapa_shared(stage_u32, static_cast<uint32_t>(min(ks + j, p.S - 1))) + off);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (ks + j < p.S) {
-            acc.x += v[j].x;
-            acc.y += v[j].y;
-            acc.z += v[j].z;
-            acc.w += v[j].w;
-          }
+      for (int u = 0; u < 4; ++u) {
+        const int it = i0 + u * 128;
+        valid[u] = it < nitems;
+        const int c4 = valid[u] ? it / nrows : 0;
+        const int row = valid[u] ? row0 + (it - c4 * nrows) : row0;
+        off[u] = static_cast<uint32_t>(c4 * 128 + row);
       }
-      const float f[4] = {acc.x, acc.y, acc.z, acc.w};
-      store_row(p, t, row, 4 * c4, f);
+      float4 acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int ks = 0; ks < p.S; ks += 4) {
+        float4 v[4][4];
+        load_partials_from(v, stage_u32, ks, p.S, off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (ks + j < p.S)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              acc[u].x += v[j][u].x;
+              acc[u].y += v[j][u].y;
+              acc[u].z += v[j][u].z;
+              acc[u].w += v[j][u].w;
+            }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (!valid[u]) continue;
+        const int c4 = static_cast<int>(off[u]) / 128, row = static_cast<int>(off[u]) - c4 * 128;
+        const float f[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
+        store_row(p, t, row, 4 * c4, f);
+      }
     }
     if (tr && tid == 0) tr[kTrSplitReduced] = globaltimer_ns();
   }
@@ -1313,8 +1349,10 @@ int factor_record_floats(int k) {
 void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits,
                 int* split_rows) {
   // Split each instance's rows (whole 64-row blocks) to balance the tiles
-  // over the SMs: minimise (rounds of tiles per SM) x (blocks per tile),
-  // with a small charge per split for the fp32 partial sums it adds.
+  // over the SMs. A tile costs about 2 us of pipeline fill and epilogue plus
+  // 0.3 us per pipelined 64-row block, and a split tile 3 us more for the
+  // reduction of the partials over distributed shared memory (per-CTA
+  // timelines of the Gram stage); rounds of tiles per SM multiply it.
   const int64_t blocks = (T + 63) / 64;
   const int64_t mtiles = (d_in + 127) / 128 + (k + 127) / 128;
   const int64_t per_split_tiles = std::max<int64_t>(1, B * mtiles);
@@ -1325,7 +1363,8 @@ void gram_split(int64_t T, int64_t B, int d_in, int k, int sm_count, int* splits
     const int64_t used = (blocks + per - 1) / per;  // splits actually made
     if (used != sp) continue;
     const int64_t rounds = (per_split_tiles * sp + sm_count - 1) / sm_count;
-    const double cost = static_cast<double>(rounds * per) * (1.0 + 0.05 * static_cast<double>(sp));
+    const double tile_us = 2.0 + 0.3 * static_cast<double>(per) + (sp > 1 ? 3.0 : 0.0);
+    const double cost = static_cast<double>(rounds) * tile_us;
     if (sp == 1 || cost < best) {
       best = cost;
       best_s = sp;
