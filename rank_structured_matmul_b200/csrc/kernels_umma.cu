@@ -309,10 +309,15 @@ struct ProjPolicy {
     const int ks_me = static_cast<int>(cluster_ctarank());
     Tile t;
     decode(p, static_cast<int>(blockIdx.x), t);
-    const int rk = p.r + p.k, c4n = p.bn / 4;
+    // this CTA's slice of the tile's rows, cut at the last row of X, and the
+    // tile's columns inside [Z | L]: the rest is never stored, and the reads
+    // of the partials are bound by the bandwidth of distributed shared memory
+    const int rk = p.r + p.k;
+    const int c4n = min(p.bn / 4, max(0, (rk - t.n0 + 3) / 4));
     const int rs = (128 + p.ksplit - 1) / p.ksplit;
-    const int row0 = ks_me * rs, nrows = min(128, row0 + rs) - row0;
-    const int nitems = nrows > 0 ? nrows * c4n : 0;
+    const int row0 = ks_me * rs;
+    const int nrows = max(0, min(min(128, row0 + rs), p.N - t.m0) - row0);
+    const int nitems = nrows * c4n;
     for (int i0 = tid; i0 < nitems; i0 += 4 * 128) {
       uint32_t off[4];
       bool valid[4];
